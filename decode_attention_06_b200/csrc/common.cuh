@@ -1,0 +1,113 @@
+// common.cuh -- shared device helpers of libgqla: fixed layer widths, the
+// split-KV work plan, and the device error record.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gqla.h"
+
+namespace gqla {
+
+constexpr int kLatent = 512;             // r_kv
+constexpr int kRope = 64;                // d_R
+constexpr int kNope = 128;               // d_nope
+constexpr int kDv = 128;                 // d_v
+constexpr int kQk = kNope + kRope;       // 192: GQA-path key width
+constexpr int kRow = kLatent + kRope;    // 576: latent cache row
+constexpr int kKv = kNope + kDv;         // 256: one group's expanded row [K_nope | V]
+constexpr int kPage = 64;                // tokens per page
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Device error record at the start of the workspace: first error wins.
+struct DeviceError {
+    int code;
+    int info;
+};
+
+__device__ __forceinline__ void report_error(void *ws, int code, int info) {
+    if (!ws) return;
+    DeviceError *e = reinterpret_cast<DeviceError *>(ws);
+    if (atomicCAS(&e->code, 0, code) == 0) atomicExch(&e->info, info);
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV plan.
+//
+// The pages of the batch are concatenated sequence after sequence (sequence b
+// owns global pages [P_b, P_b + n_b), n_b = ceil(L_b / 64)) and cut into
+// `num_splits` chunks of ceil(T / num_splits) pages, T = sum_b n_b.  Chunk c
+// meets sequence b in at most one contiguous page range, its "piece", whose
+// partial result goes to slot b + c.  Distinct pieces get distinct slots
+// (a later chunk can only meet later sequences), so batch + num_splits slots
+// always suffice.  Every CTA and the combine derive the same plan from the
+// device-resident lengths; nothing is precomputed on the host.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ int pages_of(int len) { return len > 0 ? (len + kPage - 1) / kPage : 0; }
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+
+// One full warp: total pages T of the batch.
+__device__ __forceinline__ int warp_total_pages(const int32_t *seqlens, int batch) {
+    int acc = 0;
+    for (int b = threadIdx.x & 31; b < batch; b += 32) acc += pages_of(seqlens[b]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc;
+}
+
+// One full warp: the first sequence b whose page range ends after global page
+// `pos` (skipping empty sequences), and its first global page P_b.  Returns
+// b = batch if none.
+__device__ __forceinline__ void warp_find_sequence(const int32_t *seqlens, int batch, int pos,
+                                                   int *b_out, int *start_out) {
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    for (int b0 = 0; b0 < batch; b0 += 32) {
+        int b = b0 + lane;
+        int n = b < batch ? pages_of(seqlens[b]) : 0;
+        int incl = warp_incl_scan(n);
+        bool hit = b < batch && n > 0 && base + incl > pos;
+        unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+            int src = __ffs(m) - 1;
+            int excl = __shfl_sync(0xffffffffu, incl - n, src);
+            *b_out = b0 + src;
+            *start_out = base + excl;
+            return;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    *b_out = batch;
+    *start_out = base;
+}
+
+// One full warp: first global page P_b of sequence b.
+__device__ __forceinline__ int warp_sequence_start(const int32_t *seqlens, int b) {
+    int acc = 0;
+    for (int i = threadIdx.x & 31; i < b; i += 32) acc += pages_of(seqlens[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc;
+}
+
+__device__ __forceinline__ int chunk_pages(int total_pages, int num_splits) {
+    return (total_pages + num_splits - 1) / num_splits;
+}
+
+// Host-side argument checks shared by the entry points.
+inline bool dims_supported(const gqla_dims *d) {
+    return d->d_latent == kLatent && d->d_rope == kRope && d->d_nope == kNope && d->d_v == kDv;
+}
+
+}  // namespace gqla

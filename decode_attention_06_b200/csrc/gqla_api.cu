@@ -1,0 +1,199 @@
+// gqla_api.cu -- the extern "C" entry points of libgqla (declared in
+// include/gqla.h): argument validation, then launches on the caller's stream.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace gqla {
+cudaError_t launch_expand(const void *latent, int64_t num_slots, const void *w_uk,
+                          const void *w_uv, void *kv, void *k_rope, int num_groups,
+                          cudaStream_t stream);
+cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_groups,
+                                const void *w_uk, void *qa, cudaStream_t stream);
+cudaError_t launch_decode_gqa_simt(const void *q, int s_q, int heads, int num_groups,
+                                   const void *kv, const void *k_rope, int64_t num_slots,
+                                   const gqla_kv_index *idx, int num_splits, float scale,
+                                   float *o_part, float *lse_part, void *ws, cudaStream_t stream);
+cudaError_t launch_decode_absorb_simt(const void *qa, int s_q, int heads, const void *cache,
+                                      const gqla_kv_index *idx, int num_splits, float scale,
+                                      float *o_part, float *lse_part, void *ws,
+                                      cudaStream_t stream);
+cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int d_in,
+                           const float *o_part, const float *lse_part, const void *w_uv,
+                           void *out, float *lse_out, int heads, int num_groups,
+                           cudaStream_t stream);
+}  // namespace gqla
+
+using namespace gqla;
+
+namespace {
+
+constexpr size_t kWorkspaceBytes = 256;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const gqla_dims *d, int s_q) {
+    if (!d) return GQLA_ERR_INVALID_ARG;
+    if (d->num_heads <= 0 || d->num_groups <= 0 || d->num_heads % d->num_groups)
+        return GQLA_ERR_INVALID_ARG;
+    if (!(d->softmax_scale > 0.0f) || !isfinite(d->softmax_scale)) return GQLA_ERR_INVALID_ARG;
+    if (!dims_supported(d)) return GQLA_ERR_UNSUPPORTED;
+    const int G = d->num_heads / d->num_groups;
+    if (s_q < 1 || s_q > 2) return s_q < 1 ? GQLA_ERR_INVALID_ARG : GQLA_ERR_UNSUPPORTED;
+    if (G % 4 != 0 || G * s_q > 32) return GQLA_ERR_UNSUPPORTED;
+    return GQLA_OK;
+}
+
+int check_index(const gqla_kv_index *kv) {
+    if (!kv || !kv->page_table || !kv->seqlens) return GQLA_ERR_INVALID_ARG;
+    if (kv->batch <= 0 || kv->max_pages_per_seq <= 0 || kv->num_pages <= 0)
+        return GQLA_ERR_INVALID_ARG;
+    if (kv->batch > 65535) return GQLA_ERR_UNSUPPORTED;
+    if (kv->page_size != kPage) return GQLA_ERR_UNSUPPORTED;
+    return GQLA_OK;
+}
+
+int check_workspace(const void *ws, size_t bytes) {
+    if (!ws || bytes < kWorkspaceBytes || !aligned16(ws)) return GQLA_ERR_WORKSPACE;
+    return GQLA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int gqla_version(void) { return 1; }
+
+const char *gqla_status_string(int status) {
+    switch (status) {
+        case GQLA_OK: return "ok";
+        case GQLA_ERR_INVALID_ARG: return "invalid argument";
+        case GQLA_ERR_UNSUPPORTED: return "unsupported shape";
+        case GQLA_ERR_WORKSPACE: return "workspace missing or too small";
+        case GQLA_ERR_CUDA: return "CUDA error";
+        case GQLA_ERR_DEVICE: return "device-side check failed";
+        case GQLA_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+size_t gqla_workspace_bytes(void) { return kWorkspaceBytes; }
+
+int gqla_partial_slots(int batch, int num_splits) {
+    if (batch <= 0 || num_splits <= 0) return GQLA_ERR_INVALID_ARG;
+    return batch + num_splits;
+}
+
+int gqla_num_splits_hint(int path) {
+    if (path != 0 && path != 1) return GQLA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQLA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GQLA_ERR_CUDA;
+    return sms;
+}
+
+int gqla_read_device_error(const void *workspace, int *info, gqla_stream_t stream) {
+    if (!workspace) return GQLA_ERR_INVALID_ARG;
+    DeviceError e{0, 0};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&e, workspace, sizeof e, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GQLA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GQLA_ERR_CUDA;
+    if (info) *info = e.info;
+    return e.code;
+}
+
+int gqla_clear_device_error(void *workspace, gqla_stream_t stream) {
+    if (!workspace) return GQLA_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(workspace, 0, sizeof(DeviceError),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_expand_cache(const gqla_dims *dims, const void *latent, int64_t num_slots,
+                      const void *w_uk, const void *w_uv, void *kv_expanded, void *k_rope,
+                      gqla_stream_t stream) {
+    int st = check_dims(dims, 1);
+    if (st == GQLA_ERR_UNSUPPORTED && dims && dims_supported(dims)) st = GQLA_OK;  // head split irrelevant here
+    if (st != GQLA_OK) return st;
+    if (num_slots < 0) return GQLA_ERR_INVALID_ARG;
+    if (!latent || !w_uk || !w_uv || !kv_expanded || !k_rope) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(latent) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(kv_expanded) ||
+        !aligned16(k_rope))
+        return GQLA_ERR_INVALID_ARG;
+    if (num_slots > ((int64_t)1 << 31) - 1) return GQLA_ERR_UNSUPPORTED;
+    return cuda_status(launch_expand(latent, num_slots, w_uk, w_uv, kv_expanded, k_rope,
+                                     dims->num_groups, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_absorb_query(const gqla_dims *dims, const void *q, int batch, int s_q,
+                      const void *w_uk, void *q_absorbed, gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if (batch <= 0 || !q || !w_uk || !q_absorbed) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(w_uk) || !aligned16(q_absorbed)) return GQLA_ERR_INVALID_ARG;
+    const int rows = batch * s_q * dims->num_heads;
+    return cuda_status(launch_absorb_query(q, rows, dims->num_heads, dims->num_groups, w_uk,
+                                           q_absorbed, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
+                       const void *latent_cache, const gqla_kv_index *kv, int num_splits,
+                       float *o_part, float *lse_part, void *workspace, size_t workspace_bytes,
+                       gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if ((st = check_index(kv)) != GQLA_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes)) != GQLA_OK) return st;
+    if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
+    if (!q_absorbed || !latent_cache || !o_part || !lse_part) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(q_absorbed) || !aligned16(latent_cache) || !aligned16(o_part))
+        return GQLA_ERR_INVALID_ARG;
+    if ((s_q * dims->num_heads) % 16) return GQLA_ERR_UNSUPPORTED;
+    return cuda_status(launch_decode_absorb_simt(q_absorbed, s_q, dims->num_heads, latent_cache, kv,
+                                                 num_splits, dims->softmax_scale, o_part, lse_part,
+                                                 workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
+                    const void *k_rope, int64_t num_slots, const gqla_kv_index *kv,
+                    int num_splits, float *o_part, float *lse_part, void *workspace,
+                    size_t workspace_bytes, gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if ((st = check_index(kv)) != GQLA_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes)) != GQLA_OK) return st;
+    if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
+    if (!q || !kv_expanded || !k_rope || !o_part || !lse_part) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv_expanded) || !aligned16(k_rope) || !aligned16(o_part))
+        return GQLA_ERR_INVALID_ARG;
+    if (num_slots != (int64_t)kv->num_pages * kv->page_size) return GQLA_ERR_INVALID_ARG;
+    return cuda_status(launch_decode_gqa_simt(q, s_q, dims->num_heads, dims->num_groups,
+                                              kv_expanded, k_rope, num_slots, kv, num_splits,
+                                              dims->softmax_scale, o_part, lse_part, workspace,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
+                 int d_in, const float *o_part, const float *lse_part, const void *w_uv,
+                 void *out, float *lse_out, gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if ((st = check_index(kv)) != GQLA_OK) return st;
+    if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
+    if (!o_part || !lse_part || !out) return GQLA_ERR_INVALID_ARG;
+    if (d_in == kLatent) {
+        if (!w_uv) return GQLA_ERR_INVALID_ARG;
+    } else if (d_in == kDv) {
+        if (w_uv) return GQLA_ERR_INVALID_ARG;
+    } else {
+        return GQLA_ERR_INVALID_ARG;
+    }
+    return cuda_status(launch_combine(kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out,
+                                      lse_out, dims->num_heads, dims->num_groups,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

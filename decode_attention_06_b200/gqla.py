@@ -1,0 +1,255 @@
+"""Python binding of libgqla (include/gqla.h): argument marshalling only.
+
+Every function here checks tensor placement/dtype/shape, passes raw device
+pointers and the current CUDA stream to the C ABI, and raises on a non-zero
+status.  All arithmetic happens in the CUDA kernels of libgqla.so; there is no
+fallback: if the library is missing, importing this module fails.
+
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqla.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"libgqla.so not found at {_LIB_PATH}; build it with "
+        "`python -m decode_attention_06_b200.build_lib` (needs nvcc)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+D_LATENT, D_ROPE, D_NOPE, D_V = 512, 64, 128, 128
+D_QK, D_ROW = D_NOPE + D_ROPE, D_LATENT + D_ROPE
+PAGE_SIZE = 64
+
+STATUS = {0: "GQLA_OK", -1: "GQLA_ERR_INVALID_ARG", -2: "GQLA_ERR_UNSUPPORTED",
+          -3: "GQLA_ERR_WORKSPACE", -4: "GQLA_ERR_CUDA", -5: "GQLA_ERR_DEVICE",
+          -6: "GQLA_ERR_TIMEOUT"}
+
+
+class GqlaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {status} ({STATUS.get(status, '?')})")
+
+
+class gqla_dims(ctypes.Structure):
+    _fields_ = [("num_heads", ctypes.c_int), ("num_groups", ctypes.c_int),
+                ("d_latent", ctypes.c_int), ("d_rope", ctypes.c_int),
+                ("d_nope", ctypes.c_int), ("d_v", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float)]
+
+
+class gqla_kv_index(ctypes.Structure):
+    _fields_ = [("page_table", ctypes.c_void_p), ("seqlens", ctypes.c_void_p),
+                ("batch", ctypes.c_int), ("max_pages_per_seq", ctypes.c_int),
+                ("page_size", ctypes.c_int), ("num_pages", ctypes.c_int)]
+
+
+_P, _I, _I64, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_DP, _KP = ctypes.POINTER(gqla_dims), ctypes.POINTER(gqla_kv_index)
+_SIGS = {
+    "gqla_expand_cache": [_DP, _P, _I64, _P, _P, _P, _P, _P],
+    "gqla_absorb_query": [_DP, _P, _I, _I, _P, _P, _P],
+    "gqla_decode_absorb": [_DP, _P, _I, _P, _KP, _I, _P, _P, _P, _SZ, _P],
+    "gqla_decode_gqa": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _SZ, _P],
+    "gqla_combine": [_DP, _KP, _I, _I, _I, _P, _P, _P, _P, _P, _P],
+    "gqla_partial_slots": [_I, _I],
+    "gqla_workspace_bytes": [],
+    "gqla_num_splits_hint": [_I],
+    "gqla_read_device_error": [_P, ctypes.POINTER(ctypes.c_int), _P],
+    "gqla_clear_device_error": [_P, _P],
+    "gqla_status_string": [_I],
+    "gqla_version": [],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _I
+_lib.gqla_workspace_bytes.restype = _SZ
+_lib.gqla_status_string.restype = ctypes.c_char_p
+
+EXPORTED = tuple(_SIGS)
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise GqlaError(fn, st)
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def make_dims(num_heads: int, num_groups: int = 8, softmax_scale: Optional[float] = None):
+    return gqla_dims(num_heads, num_groups, D_LATENT, D_ROPE, D_NOPE, D_V,
+                     1.0 / math.sqrt(D_NOPE + D_ROPE) if softmax_scale is None else softmax_scale)
+
+
+def make_kv_index(page_table: torch.Tensor, seqlens: torch.Tensor, num_pages: int,
+                  page_size: int = PAGE_SIZE):
+    pt = _dev(page_table, "page_table", torch.int32)
+    sl = _dev(seqlens, "seqlens", torch.int32)
+    if page_table.dim() != 2 or seqlens.shape != (page_table.shape[0],):
+        raise ValueError("page_table must be [batch][max_pages] and seqlens [batch]")
+    idx = gqla_kv_index(pt, sl, page_table.shape[0], page_table.shape[1], page_size, num_pages)
+    idx._keep = (page_table, seqlens)  # keep the tensors alive with the struct
+    return idx
+
+
+# ------------------------------------------------------------------ the five calls
+
+def gqla_expand_cache(dims, latent, w_uk, w_uv, kv_expanded, k_rope, stream=None):
+    n = latent.numel() // D_ROW
+    g = dims.num_groups
+    _check("gqla_expand_cache", _lib.gqla_expand_cache(
+        ctypes.byref(dims), _dev(latent, "latent", torch.bfloat16), n,
+        _dev(w_uk, "w_uk", torch.bfloat16, (g, D_LATENT, D_NOPE)),
+        _dev(w_uv, "w_uv", torch.bfloat16, (g, D_LATENT, D_V)),
+        _dev(kv_expanded, "kv_expanded", torch.bfloat16, (g, n, D_NOPE + D_V)),
+        _dev(k_rope, "k_rope", torch.bfloat16, (n, D_ROPE)), _stream(stream)))
+
+
+def gqla_absorb_query(dims, q, w_uk, q_absorbed, stream=None):
+    B, s_q, h, _ = q.shape
+    _check("gqla_absorb_query", _lib.gqla_absorb_query(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16, (B, s_q, dims.num_heads, D_QK)), B, s_q,
+        _dev(w_uk, "w_uk", torch.bfloat16, (dims.num_groups, D_LATENT, D_NOPE)),
+        _dev(q_absorbed, "q_absorbed", torch.bfloat16, (B, s_q, h, D_ROW)), _stream(stream)))
+
+
+def gqla_decode_absorb(dims, q_absorbed, latent_cache, kv, num_splits, o_part, lse_part,
+                       workspace, stream=None):
+    B, s_q, h, _ = q_absorbed.shape
+    slots = gqla_partial_slots(kv.batch, num_splits)
+    _check("gqla_decode_absorb", _lib.gqla_decode_absorb(
+        ctypes.byref(dims), _dev(q_absorbed, "q_absorbed", torch.bfloat16, (kv.batch, s_q, dims.num_heads, D_ROW)),
+        s_q, _dev(latent_cache, "latent_cache", torch.bfloat16, (kv.num_pages, kv.page_size, D_ROW)),
+        ctypes.byref(kv), num_splits,
+        _dev(o_part, "o_part", torch.float32, (slots, s_q, h, D_LATENT)),
+        _dev(lse_part, "lse_part", torch.float32, (slots, s_q, h)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gqla_decode_gqa(dims, q, kv_expanded, k_rope, kv, num_splits, o_part, lse_part, workspace,
+                    stream=None):
+    B, s_q, h, _ = q.shape
+    n = kv.num_pages * kv.page_size
+    slots = gqla_partial_slots(kv.batch, num_splits)
+    _check("gqla_decode_gqa", _lib.gqla_decode_gqa(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16, (kv.batch, s_q, dims.num_heads, D_QK)), s_q,
+        _dev(kv_expanded, "kv_expanded", torch.bfloat16, (dims.num_groups, n, D_NOPE + D_V)),
+        _dev(k_rope, "k_rope", torch.bfloat16, (n, D_ROPE)), n, ctypes.byref(kv), num_splits,
+        _dev(o_part, "o_part", torch.float32, (slots, s_q, h, D_V)),
+        _dev(lse_part, "lse_part", torch.float32, (slots, s_q, h)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gqla_combine(dims, kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out, lse_out=None,
+                 stream=None):
+    slots = gqla_partial_slots(kv.batch, num_splits)
+    h = dims.num_heads
+    _check("gqla_combine", _lib.gqla_combine(
+        ctypes.byref(dims), ctypes.byref(kv), s_q, num_splits, d_in,
+        _dev(o_part, "o_part", torch.float32, (slots, s_q, h, d_in)),
+        _dev(lse_part, "lse_part", torch.float32, (slots, s_q, h)),
+        None if w_uv is None else _dev(w_uv, "w_uv", torch.bfloat16, (dims.num_groups, D_LATENT, D_V)),
+        _dev(out, "out", torch.bfloat16, (kv.batch, s_q, h, D_V)),
+        None if lse_out is None else _dev(lse_out, "lse_out", torch.float32, (kv.batch, s_q, h)),
+        _stream(stream)))
+
+
+# ------------------------------------------------------------------ helpers
+
+def gqla_partial_slots(batch: int, num_splits: int) -> int:
+    n = _lib.gqla_partial_slots(batch, num_splits)
+    if n < 0:
+        raise GqlaError("gqla_partial_slots", n)
+    return n
+
+
+def gqla_workspace_bytes() -> int:
+    return int(_lib.gqla_workspace_bytes())
+
+
+def gqla_num_splits_hint(path: str) -> int:
+    n = _lib.gqla_num_splits_hint({"absorb": 0, "gqa": 1}[path])
+    if n < 0:
+        raise GqlaError("gqla_num_splits_hint", n)
+    return n
+
+
+def gqla_read_device_error(workspace: torch.Tensor, stream=None):
+    info = ctypes.c_int(0)
+    st = _lib.gqla_read_device_error(_dev(workspace, "workspace"), ctypes.byref(info), _stream(stream))
+    return st, info.value
+
+
+def gqla_clear_device_error(workspace: torch.Tensor, stream=None):
+    _check("gqla_clear_device_error", _lib.gqla_clear_device_error(_dev(workspace, "workspace"), _stream(stream)))
+
+
+def gqla_status_string(status: int) -> str:
+    return _lib.gqla_status_string(status).decode()
+
+
+def gqla_version() -> int:
+    return _lib.gqla_version()
+
+
+def new_workspace(device=None) -> torch.Tensor:
+    """A zeroed workspace of gqla_workspace_bytes() bytes."""
+    return torch.zeros(gqla_workspace_bytes(), dtype=torch.uint8, device=device or "cuda")
+
+
+class DecodeBuffers:
+    """Device buffers for one decode step (allocated once, reused every step)."""
+
+    def __init__(self, dims, batch: int, s_q: int, num_splits: int, path: str, device="cuda"):
+        h = dims.num_heads
+        slots = gqla_partial_slots(batch, num_splits)
+        d_in = D_LATENT if path == "absorb" else D_V
+        self.path, self.s_q, self.num_splits, self.d_in = path, s_q, num_splits, d_in
+        self.q_absorbed = (torch.empty(batch, s_q, h, D_ROW, dtype=torch.bfloat16, device=device)
+                           if path == "absorb" else None)
+        self.o_part = torch.empty(slots, s_q, h, d_in, dtype=torch.float32, device=device)
+        self.lse_part = torch.empty(slots, s_q, h, dtype=torch.float32, device=device)
+        self.out = torch.empty(batch, s_q, h, D_V, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(batch, s_q, h, dtype=torch.float32, device=device)
+        self.workspace = new_workspace(device)
+
+
+def decode_step(dims, bufs: DecodeBuffers, q, w_uk, w_uv, kv, latent_cache=None,
+                kv_expanded=None, k_rope=None, stream=None):
+    """One decode step through the C ABI: absorb path = absorb_query ->
+    decode_absorb -> combine(W_UV); GQA path = decode_gqa -> combine."""
+    if bufs.path == "absorb":
+        gqla_absorb_query(dims, q, w_uk, bufs.q_absorbed, stream)
+        gqla_decode_absorb(dims, bufs.q_absorbed, latent_cache, kv, bufs.num_splits, bufs.o_part,
+                           bufs.lse_part, bufs.workspace, stream)
+        gqla_combine(dims, kv, bufs.s_q, bufs.num_splits, D_LATENT, bufs.o_part, bufs.lse_part,
+                     w_uv, bufs.out, bufs.lse, stream)
+    else:
+        gqla_decode_gqa(dims, q, kv_expanded, k_rope, kv, bufs.num_splits, bufs.o_part,
+                        bufs.lse_part, bufs.workspace, stream)
+        gqla_combine(dims, kv, bufs.s_q, bufs.num_splits, D_V, bufs.o_part, bufs.lse_part,
+                     None, bufs.out, bufs.lse, stream)
+    return bufs.out, bufs.lse

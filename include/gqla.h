@@ -1,0 +1,189 @@
+/*
+ * gqla.h -- C ABI of libgqla: GQLA (Group-Query Latent Attention) decode
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * GQLA indexes the latent up-projections W_UK and W_UV by g groups instead of
+ * by the h_q query heads, so one set of weights exposes two algebraically
+ * equivalent decoding paths (GQLA, paperlayer.ai summary of arXiv:2605.15250v3,
+ * sec. 2 "Algebraically equivalent decoding paths" and sec. 3 "Two equivalent
+ * decoding paths"; gist.science technical summary, sec. 2 "Architektur"):
+ *
+ *   MQA-absorb path  gqla_absorb_query -> gqla_decode_absorb -> gqla_combine
+ *       W_UK is folded into the query, every head attends over the 576-element
+ *       latent row [c (512) | k^R (64)], the value is the 512-d latent itself,
+ *       and W_UV is applied after the split combine.
+ *   GQA path         gqla_expand_cache (once) -> gqla_decode_gqa -> gqla_combine
+ *       the cache is expanded once per group into K_nope = c W_UK_g and
+ *       V = c W_UV_g (128 each) beside the shared RoPE key; h_q/g query heads
+ *       share each group (pwwt.cn article, sec. 3 and sec. 5: 16 heads per group).
+ *
+ * Conventions for every call:
+ *  - All tensor arguments are DEVICE pointers owned by the caller, dense,
+ *    row-major, 16-byte aligned.  Nothing is allocated, freed or copied to
+ *    the host, and no call synchronises: work is enqueued on `stream`
+ *    (NULL = the legacy default stream) and the call returns.
+ *  - bf16 means IEEE bfloat16 (2 bytes).  "h" is dims->num_heads, "g" is
+ *    dims->num_groups, G = h/g heads per group; head hd belongs to group hd/G.
+ *  - Token t of sequence b lives at pool slot page_table[b][t/page_size] *
+ *    page_size + t % page_size.  The s_q query tokens of a step are already
+ *    the last s_q cached tokens: query s sees tokens t <= seqlen - s_q + s.
+ *  - Return value: GQLA_OK, or a negative gqla_status.  Argument errors are
+ *    detected before anything is launched.  Errors found on the device (a
+ *    page index outside the pool, a sequence longer than its page-table row,
+ *    a bounded wait that ran out) never trap: the kernel skips the bad work,
+ *    records the first error in the workspace, and gqla_read_device_error()
+ *    returns it.
+ *  - Calls on the same workspace must not overlap on the GPU.
+ *
+ * Supported shapes: d_latent 512, d_rope 64, d_nope 128, d_v 128, page_size
+ * 64, s_q in {1, 2}, h % g == 0 with (h/g) * s_q <= 32, batch <= 65535.
+ * Anything else returns GQLA_ERR_UNSUPPORTED.
+ */
+#ifndef GQLA_H_
+#define GQLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *gqla_stream_t;
+
+typedef enum {
+    GQLA_OK = 0,
+    GQLA_ERR_INVALID_ARG = -1,  /* null pointer, negative size, inconsistent dims */
+    GQLA_ERR_UNSUPPORTED = -2,  /* valid but not one of the supported shapes      */
+    GQLA_ERR_WORKSPACE = -3,    /* workspace missing or smaller than required    */
+    GQLA_ERR_CUDA = -4,         /* a CUDA runtime/driver call or launch failed   */
+    GQLA_ERR_DEVICE = -5,       /* device-side check failed (bad page index ...) */
+    GQLA_ERR_TIMEOUT = -6       /* a bounded device-side wait ran out            */
+} gqla_status;
+
+/* Layer dimensions.  softmax_scale is applied to q.k before the softmax; the
+ * pages do not state it, the MLA convention 1/sqrt(d_nope + d_rope) =
+ * 1/sqrt(192) is the expected value. */
+typedef struct {
+    int num_heads;       /* h_q: e.g. 128 (DeepSeek-V3 shape) or 32 (LLaMA-3-8B) */
+    int num_groups;      /* g: 8                                                   */
+    int d_latent;        /* r_kv: 512                                              */
+    int d_rope;          /* d_R: 64                                                */
+    int d_nope;          /* per-head no-RoPE key width: 128                        */
+    int d_v;             /* per-head value width: 128                              */
+    float softmax_scale; /* 1/sqrt(d_nope + d_rope)                                */
+} gqla_dims;
+
+/* Paged KV index shared by both decode paths and the combine. */
+typedef struct {
+    const int32_t *page_table; /* device int32 [batch][max_pages_per_seq]           */
+    const int32_t *seqlens;    /* device int32 [batch], cached tokens incl. the s_q new ones */
+    int batch;                 /* number of sequences, 1..65535                      */
+    int max_pages_per_seq;     /* row length of page_table                           */
+    int page_size;             /* tokens per page: 64                                */
+    int num_pages;             /* pages in the pool; a page index outside [0, num_pages) is a device error */
+} gqla_kv_index;
+
+/*
+ * One-shot cache expansion for the GQA path (deploy-time, not per step:
+ * pwwt.cn article, sec. 3; paperlayer.ai sec. 3 "Two equivalent decoding
+ * paths", the one-shot cache expansion).
+ *   latent       bf16 [num_slots][576]   rows [c | k^R]
+ *   w_uk, w_uv   bf16 [g][512][128]
+ *   kv_expanded  bf16 [g][num_slots][256] out: [c W_UK_g | c W_UV_g]
+ *   k_rope       bf16 [num_slots][64]    out: k^R copied
+ * Rounding contract: each output is accumulated in fp32 from +0.0 by one
+ * fused multiply-add per latent index 0..511 in ascending order, then
+ * rounded once to bf16 (nearest, ties to even).  Results are therefore
+ * bit-reproducible by any implementation of that order.
+ */
+int gqla_expand_cache(const gqla_dims *dims, const void *latent, int64_t num_slots,
+                      const void *w_uk, const void *w_uv, void *kv_expanded, void *k_rope,
+                      gqla_stream_t stream);
+
+/*
+ * Query absorption ("folds W_UK into Q": paperlayer.ai sec. 2).
+ *   q           bf16 [batch][s_q][h][192]  (0..127 q^C, 128..191 q^R, RoPE applied)
+ *   w_uk        bf16 [g][512][128]
+ *   q_absorbed  bf16 [batch][s_q][h][576]  out: [W_UK_{g(h)} q^C ; q^R], fp32 accumulation
+ */
+int gqla_absorb_query(const gqla_dims *dims, const void *q, int batch, int s_q,
+                      const void *w_uk, void *q_absorbed, gqla_stream_t stream);
+
+/*
+ * Split-KV partial attention, MQA-absorb path: every head scores its absorbed
+ * query against the latent row and accumulates the 512-d latent.
+ *   q_absorbed    bf16 [batch][s_q][h][576]
+ *   latent_cache  bf16 [num_pages][page_size][576]
+ *   kv            page table / lengths (kv->batch is the batch)
+ *   num_splits    C >= 1: the batch's pages, concatenated sequence after
+ *                 sequence, are cut into C equal chunks, one per CTA; a chunk
+ *                 that meets sequence b yields one partial in slot (b + chunk).
+ *   o_part  fp32 [gqla_partial_slots(batch, C)][s_q][h][512]  out, normalised per partial
+ *   lse_part fp32 [gqla_partial_slots(batch, C)][s_q][h]      out, natural-log LSE of the
+ *                 scaled scores (-inf for an empty partial); unused slots are not written
+ *   workspace  >= gqla_workspace_bytes() bytes of device memory, zeroed once
+ *              before first use (holds the device error record)
+ */
+int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
+                       const void *latent_cache, const gqla_kv_index *kv, int num_splits,
+                       float *o_part, float *lse_part, void *workspace, size_t workspace_bytes,
+                       gqla_stream_t stream);
+
+/*
+ * Split-KV partial attention, GQA path: the G*s_q query rows of each group
+ * score [K_nope_g | k^R] (192) and accumulate V_g (128).
+ *   q            bf16 [batch][s_q][h][192]
+ *   kv_expanded  bf16 [g][num_slots][256], k_rope bf16 [num_slots][64]
+ *                (as written by gqla_expand_cache; num_slots = num_pages * page_size)
+ *   o_part  fp32 [gqla_partial_slots(batch, C)][s_q][h][128], lse_part as above.
+ */
+int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
+                    const void *k_rope, int64_t num_slots, const gqla_kv_index *kv,
+                    int num_splits, float *o_part, float *lse_part, void *workspace,
+                    size_t workspace_bytes, gqla_stream_t stream);
+
+/*
+ * Log-sum-exp merge of the partials of each sequence, then (absorb path,
+ * d_in == 512) the per-group up-projection out = o~ W_UV_{g(h)} ("folds W_UV
+ * into O": paperlayer.ai sec. 2).
+ *   o_part / lse_part as written by a decode call with the same kv and num_splits
+ *   d_in      512 (absorb partials; w_uv required) or 128 (GQA partials; w_uv NULL)
+ *   out       bf16 [batch][s_q][h][128]
+ *   lse_out   fp32 [batch][s_q][h] or NULL
+ * A row with no visible token gets out = 0 and lse = -inf.
+ */
+int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
+                 int d_in, const float *o_part, const float *lse_part, const void *w_uv,
+                 void *out, float *lse_out, gqla_stream_t stream);
+
+/* Number of partial slots the decode calls address: batch + num_splits. */
+int gqla_partial_slots(int batch, int num_splits);
+
+/* Workspace bytes the decode calls need. */
+size_t gqla_workspace_bytes(void);
+
+/* A split count that fills the current device (SM count x resident CTAs of the
+ * path's decode kernel); path 0 = absorb, 1 = GQA.  Returns < 0 on error. */
+int gqla_num_splits_hint(int path);
+
+/* Reads (synchronising `stream`) and returns the first device-side error
+ * recorded in `workspace` (GQLA_OK if none); `info`, if not NULL, receives
+ * a code-specific detail (e.g. the sequence index).  Does not clear it. */
+int gqla_read_device_error(const void *workspace, int *info, gqla_stream_t stream);
+
+/* Clears the device error record (asynchronously, on `stream`). */
+int gqla_clear_device_error(void *workspace, gqla_stream_t stream);
+
+/* Static description of a status code. */
+const char *gqla_status_string(int status);
+
+/* Library ABI version: 1. */
+int gqla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQLA_H_ */

@@ -120,16 +120,14 @@ int gqla_oracle_decode(int batch, int s_q, int num_heads, int num_groups, int pa
         const double *wv = w_uv + (int64_t)gi * LAT * DV;
         for (int64_t t = 0; t < L; ++t) {
             const double *c = token_row(cache, page_table, max_pages, page_size, b, t);
-            for (int d = 0; d < NOPE; ++d) {
-                double k = 0.0, v = 0.0;
-                for (int r = 0; r < LAT; ++r) {
-                    k += c[r] * wk[r * NOPE + d];
-                    v += c[r] * wv[r * DV + d];
+            double *k = K + t * QK, *v = V + t * DV;
+            for (int d = 0; d < NOPE; ++d) k[d] = v[d] = 0.0;
+            for (int r = 0; r < LAT; ++r)      /* each sum still runs over r = 0..511 in order */
+                for (int d = 0; d < NOPE; ++d) {
+                    k[d] += c[r] * wk[r * NOPE + d];
+                    v[d] += c[r] * wv[r * DV + d];
                 }
-                K[t * QK + d] = k;
-                V[t * DV + d] = v;
-            }
-            for (int j = 0; j < ROPE; ++j) K[t * QK + NOPE + j] = c[LAT + j];
+            for (int j = 0; j < ROPE; ++j) k[NOPE + j] = c[LAT + j];
         }
         for (int s = 0; s < s_q; ++s) {
             int64_t visible = L - s_q + s + 1;

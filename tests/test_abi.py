@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+entry point include/gqla.h declares, and rejects bad arguments before any
+launch (no CUDA call is reached by these cases)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from decode_attention_06_b200 import build_lib
+    build_lib.build()
+    return ctypes.CDLL(build_lib.LIB)
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gqla_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_calls():
+    names = _declared()
+    for n in ["gqla_expand_cache", "gqla_absorb_query", "gqla_decode_absorb",
+              "gqla_decode_gqa", "gqla_combine"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_exposes_every_declared_symbol(lib):
+    from decode_attention_06_b200 import gqla
+    assert sorted(gqla.EXPORTED) == _declared()
+    for n in _declared():
+        assert callable(getattr(gqla, n))
+
+
+def test_pure_host_helpers(lib):
+    lib.gqla_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.gqla_version() == 1
+    assert lib.gqla_workspace_bytes() >= 8
+    assert lib.gqla_partial_slots(3, 5) == 8
+    assert lib.gqla_partial_slots(0, 5) == -1
+    lib.gqla_status_string.restype = ctypes.c_char_p
+    assert lib.gqla_status_string(0) == b"ok"
+    assert lib.gqla_status_string(-6).startswith(b"device-side wait")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("num_heads", ctypes.c_int), ("num_groups", ctypes.c_int),
+                ("d_latent", ctypes.c_int), ("d_rope", ctypes.c_int),
+                ("d_nope", ctypes.c_int), ("d_v", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float)]
+
+
+class KvIndex(ctypes.Structure):
+    _fields_ = [("page_table", ctypes.c_void_p), ("seqlens", ctypes.c_void_p),
+                ("batch", ctypes.c_int), ("max_pages_per_seq", ctypes.c_int),
+                ("page_size", ctypes.c_int), ("num_pages", ctypes.c_int)]
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every case fails validation first
+
+
+def _dims(h=128, g=8, lat=512, scale=0.072):
+    return Dims(h, g, lat, 64, 128, 128, scale)
+
+
+def _kv(batch=2, page_size=64):
+    return KvIndex(FAKE, FAKE, batch, 4, page_size, 16)
+
+
+@pytest.mark.parametrize("case,expected", [
+    ("null_dims", -1), ("bad_heads", -1), ("latent_256", -2), ("s_q_3", -2), ("s_q_0", -1),
+    ("page_32", -2), ("no_workspace", -3), ("small_workspace", -3), ("zero_splits", -1),
+    ("null_q", -1), ("misaligned_q", -1), ("slots_mismatch", -1), ("batch_0", -1),
+    ("bad_scale", -1),
+])
+def test_decode_gqa_rejects_bad_arguments(lib, case, expected):
+    d, kv = _dims(), _kv()
+    s_q, splits, ws, wsb, q, slots = 1, 4, FAKE, 256, FAKE, 16 * 64
+    if case == "null_dims":
+        dp = None
+    else:
+        if case == "bad_heads": d.num_heads = 100
+        if case == "latent_256": d.d_latent = 256
+        if case == "bad_scale": d.softmax_scale = float("nan")
+        dp = ctypes.byref(d)
+    if case == "s_q_3": s_q = 3
+    if case == "s_q_0": s_q = 0
+    if case == "page_32": kv.page_size = 32
+    if case == "no_workspace": ws = None
+    if case == "small_workspace": wsb = 4
+    if case == "zero_splits": splits = 0
+    if case == "null_q": q = None
+    if case == "misaligned_q": q = ctypes.c_void_p((1 << 20) + 2)
+    if case == "slots_mismatch": slots = 17
+    if case == "batch_0": kv.batch = 0
+    st = lib.gqla_decode_gqa(dp, q, s_q, FAKE, FAKE, ctypes.c_int64(slots), ctypes.byref(kv),
+                             splits, FAKE, FAKE, ws, ctypes.c_size_t(wsb), None)
+    assert st == expected
+
+
+def test_other_calls_reject_bad_arguments(lib):
+    d, kv = _dims(), _kv()
+    assert lib.gqla_expand_cache(ctypes.byref(d), None, ctypes.c_int64(64), FAKE, FAKE, FAKE, FAKE, None) == -1
+    assert lib.gqla_expand_cache(ctypes.byref(d), FAKE, ctypes.c_int64(-1), FAKE, FAKE, FAKE, FAKE, None) == -1
+    assert lib.gqla_absorb_query(ctypes.byref(d), FAKE, 0, 1, FAKE, FAKE, None) == -1
+    assert lib.gqla_absorb_query(ctypes.byref(d), FAKE, 2, 5, FAKE, FAKE, None) == -2
+    assert lib.gqla_decode_absorb(ctypes.byref(d), FAKE, 1, FAKE, ctypes.byref(kv), 4, FAKE, FAKE,
+                                  None, ctypes.c_size_t(0), None) == -3
+    # absorb combine needs W_UV, the GQA combine must not get one; d_in must be 512 or 128
+    assert lib.gqla_combine(ctypes.byref(d), ctypes.byref(kv), 1, 4, 512, FAKE, FAKE, None, FAKE, None, None) == -1
+    assert lib.gqla_combine(ctypes.byref(d), ctypes.byref(kv), 1, 4, 128, FAKE, FAKE, FAKE, FAKE, None, None) == -1
+    assert lib.gqla_combine(ctypes.byref(d), ctypes.byref(kv), 1, 4, 256, FAKE, FAKE, None, FAKE, None, None) == -1
+    assert lib.gqla_read_device_error(None, None, None) == -1
+    assert lib.gqla_num_splits_hint(7) == -1

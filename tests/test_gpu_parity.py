@@ -1,0 +1,150 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Both paths, every workload shape, ragged tails, empty splits and sequences,
+random page tables; full-size workloads on sampled (sequence, group) units.
+Tolerance: max-abs <= 2e-2 and rel-Frobenius <= 1e-2 (bf16 inputs, fp32
+accumulation); the cache expansion is compared bit for bit.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from decode_attention_06_b200 import synth
+from tests.helpers import compare, compare_lse, oracle_ref, run_decode, sub_case, to_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+
+
+# ------------------------------------------------------------------ expansion and absorption
+
+@pytest.mark.parametrize("n_pages,extra", [(3, 0), (5, 17)])
+def test_expand_cache_bit_exact(n_pages, extra):
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(32, 8, [64 * n_pages], 1, seed=100 + n_pages)
+    lat = case["latent"].reshape(-1, 576)
+    if extra:  # a slot count that is not a multiple of the 128-slot tile
+        lat = torch.cat([lat, lat[:extra] * 0.5]).contiguous()
+    n = lat.shape[0]
+    dims = gqla.make_dims(32, 8)
+    kv = torch.empty(8, n, 256, dtype=torch.bfloat16, device="cuda")
+    kr = torch.empty(n, 64, dtype=torch.bfloat16, device="cuda")
+    gqla.gqla_expand_cache(dims, lat.cuda(), case["w_uk"].cuda(), case["w_uv"].cuda(), kv, kr)
+    torch.cuda.synchronize()
+    ref_kv, ref_kr = oracle.expand_f32seq_bits(lat, case["w_uk"], case["w_uv"])
+    got_kv = kv.cpu().view(torch.int16).numpy().view(np.uint16)
+    got_kr = kr.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert (got_kv == ref_kv).all(), f"{(got_kv != ref_kv).sum()} expanded values differ"
+    assert (got_kr == ref_kr).all()
+
+
+@pytest.mark.parametrize("h,B,s_q", [(32, 3, 1), (128, 5, 2), (128, 9, 1)])
+def test_absorb_query_matches_oracle(h, B, s_q):
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(h, 8, [1] * B, s_q, seed=110 + h + B)
+    dims = gqla.make_dims(h, 8)
+    qa = torch.empty(B, s_q, h, 576, dtype=torch.bfloat16, device="cuda")
+    gqla.gqla_absorb_query(dims, case["q"].cuda(), case["w_uk"].cuda(), qa)
+    torch.cuda.synchronize()
+    ref = oracle.absorb_query(case["q"], case["w_uk"], 8)
+    got = qa.float().cpu().numpy()
+    # fp32 accumulation then one bf16 rounding: |err| <= 2^-8 |x| + tiny
+    assert (np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5).all()
+    np.testing.assert_array_equal(got[..., 512:], ref[..., 512:])
+
+
+# ------------------------------------------------------------------ decode parity, small shapes
+
+SMALL = [
+    # id, h, seqlens, s_q, paged, num_splits
+    ("llama_l256", 32, [256], 1, False, None),
+    ("llama_l256_3splits", 32, [256], 1, False, 3),
+    ("h128_ragged_paged", 128, [1000, 64, 1, 777], 1, True, 7),
+    ("h128_mtp_paged", 128, [513, 130], 2, True, 5),
+    ("h32_mtp_ragged", 32, [2000, 3, 70], 2, False, 16),
+    ("more_splits_than_pages", 32, [64, 65], 1, False, 9),
+    ("one_split", 128, [300, 200], 2, True, 1),
+    ("zero_length_sequence", 32, [0, 65, 0], 1, False, 4),
+    ("mtp_single_token", 32, [1, 2], 2, False, 2),
+]
+
+
+@pytest.mark.parametrize("path", ["gqa", "absorb"])
+@pytest.mark.parametrize("cid,h,seqlens,s_q,paged,splits", SMALL, ids=[c[0] for c in SMALL])
+def test_decode_parity_small(path, cid, h, seqlens, s_q, paged, splits):
+    case = synth.make_case(h, 8, seqlens, s_q, paged=paged, seed=zlib.crc32(cid.encode()) % 1000,
+                           spare_pages=2)
+    out, lse, ws, _ = run_decode(to_gpu(case), path, splits)
+    ref, ref_lse = oracle_ref(case)
+    compare(out, ref, what=f"{path}/{cid}")
+    compare_lse(lse, ref_lse, what=f"{path}/{cid}")
+    from decode_attention_06_b200 import gqla
+    assert gqla.gqla_read_device_error(ws)[0] == 0
+
+
+def test_paths_agree():
+    case = synth.make_case(128, 8, [700, 129], 2, paged=True, seed=120)
+    g = to_gpu(case)
+    a, la, _, _ = run_decode(g, "absorb", 6)
+    b, lb, _, _ = run_decode(g, "gqa", 6)
+    compare(a, b.float().cpu().numpy().astype(np.float64), what="absorb vs gqa")
+
+
+def test_bad_page_index_is_reported_not_faulted():
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(32, 8, [200, 100], 1, seed=121)
+    case["page_table"] = case["page_table"].clone()
+    case["page_table"][1, 0] = case["num_pages"] + 5  # outside the pool
+    for path in ("gqa", "absorb"):
+        _, _, ws, _ = run_decode(to_gpu(case), path, 4)
+        st, info = gqla.gqla_read_device_error(ws)
+        assert st == -5 and info == 1
+        gqla.gqla_clear_device_error(ws)
+        assert gqla.gqla_read_device_error(ws)[0] == 0
+
+
+def test_sequence_longer_than_page_row_is_reported():
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(32, 8, [128, 64], 1, seed=122)
+    case["seqlens"] = torch.tensor([128, 64 * 9], dtype=torch.int32)  # row has 2 pages only
+    _, _, ws, _ = run_decode(to_gpu(case), "gqa", 2)
+    assert gqla.gqla_read_device_error(ws) == (-5, 1)
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+
+FULL = [(name, s) for name, w in synth.WORKLOADS.items() for s in w.s_q]
+
+
+@pytest.mark.parametrize("path", ["gqa", "absorb"])
+@pytest.mark.parametrize("name,s_q", FULL, ids=[f"{n}-sq{s}" for n, s in FULL])
+def test_decode_parity_full_size_sampled(path, name, s_q):
+    w = synth.WORKLOADS[name]
+    case = synth.make_workload(name, s_q=s_q, device="cuda")
+    out, lse, ws, _ = run_decode(case, path)
+    B = w.batch
+    rng = np.random.default_rng(w.seed)
+    picks = sorted(set([0, B - 1] + rng.integers(0, B, size=2).tolist()))[:3]
+    if w.lengths[0] == "uniform" and w.lengths[2] > 16384:
+        picks = picks[:1]
+    sub = sub_case(case, picks)
+    groups = [0, w.num_groups - 1]
+    units = [(i, gi) for i in range(len(picks)) for gi in groups]
+    ref, ref_lse = oracle_ref(sub, units=units)
+    G = w.num_heads // w.num_groups
+    mask = np.zeros(ref.shape[:3], dtype=bool)
+    for i, gi in units:
+        mask[i, :, gi * G:(gi + 1) * G] = True
+    got = out[torch.tensor(picks, device="cuda")]
+    compare(got, ref, mask=mask, what=f"{path}/{name}/sq{s_q}")
+    compare_lse(lse[torch.tensor(picks, device="cuda")], ref_lse, mask=mask)
+    from decode_attention_06_b200 import gqla
+    assert gqla.gqla_read_device_error(ws)[0] == 0
