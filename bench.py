@@ -1,0 +1,498 @@
+"""Benchmark of the GQLA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one decode step of the batch through the whole hot path: the
+MQA-absorb path (gqla_absorb_query -> gqla_decode_absorb -> gqla_combine with
+W_UV) and the GQA path (gqla_decode_gqa -> gqla_combine) over the same batch.
+The one-shot cache expansion (gqla_expand_cache) is a deploy-time conversion,
+not part of a step; it is timed once and reported under "expand".
+
+value   = decode tokens per second of the whole job: N ranks x batch x s_q
+          tokens per step / (device time per step, max over ranks); each rank
+          decodes its own batch (independent sequences, no collective on the
+          data path: weak scaling).
+e2e     = the same through the C ABI with host buffers: each step copies the
+          queries, page table and lengths from pinned host memory and reads
+          both paths' outputs back, inside the timed region.
+Timing  = CUDA events on the launching stream around every call and step,
+          L2 flushed (a 256 MiB write) before every timed step, outside the
+          step's events; W >= 3 untimed warm-up steps first.
+roofline: the dominant kernel's algorithmic bytes (or FLOPs) per launch over
+          its mean event-timed duration, against MEASURED_PEAKS.json.
+cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload
+          (rank 0, N = 1 only).  --impl reference times the oracle alone.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+DEFAULT_WORKLOAD = "dsv3_h128_b32_l4096"
+METRIC = "decode-attn tokens/s & µs/step per path; % of B200 HBM / tensor roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+# Kernel source files whose ncu counters are stored in profiles/traffic.json;
+# a stored figure is used only while the source hash still matches.
+KERNEL_SOURCES = {
+    "decode_gqa": ["decode_attention_06_b200/csrc/decode_simt.cu"],
+    "decode_absorb": ["decode_attention_06_b200/csrc/decode_simt.cu"],
+}
+
+
+# ------------------------------------------------------------------ helpers
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _src_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _stored_traffic(kernel, workload):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p) or kernel not in KERNEL_SOURCES:
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_hash") != _src_hash(KERNEL_SOURCES[kernel]):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index, period_s=0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._dev = device_index
+        self._thread = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self._dev)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: report no samples rather than guessing
+            self._nvml = None
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons - {"gpu_idle"})}
+
+
+# ------------------------------------------------------------------ workload accounting
+
+def accounting(w, case, s_q, num_splits):
+    """Algorithmic bytes / FLOPs per launch (what the kernel must move / compute)."""
+    seqlens = case["seqlens"].cpu().tolist()
+    B, h, g = len(seqlens), w.num_heads, w.num_groups
+    tokens = sum(seqlens)
+    # visible (query, token) pairs: query s of a length-L sequence sees L - s_q + s + 1 tokens
+    pairs = sum(max(0, L - s_q + s + 1) for L in seqlens for s in range(s_q))
+    pages = [math.ceil(L / 64) for L in seqlens]
+    T = sum(pages)
+    k = math.ceil(T / num_splits) if T else 1
+    pieces, start = 0, 0
+    for n in pages:
+        if n:
+            pieces += (start + n - 1) // k - start // k + 1
+        start += n
+    rows = B * s_q * h
+    acc = {
+        "decode_absorb": {
+            "bytes": tokens * 1152 + rows * 576 * 2 + pieces * s_q * h * (512 + 1) * 4,
+            "flops": 2.0 * h * pairs * (576 + 512),
+        },
+        "decode_gqa": {
+            "bytes": tokens * 4224 + rows * 192 * 2 + pieces * s_q * h * (128 + 1) * 4,
+            "flops": 2.0 * h * pairs * (192 + 128),
+        },
+        "absorb_query": {"bytes": rows * (192 + 576) * 2 + g * 512 * 128 * 2,
+                         "flops": 2.0 * rows * 512 * 128},
+        "combine_absorb": {"bytes": pieces * s_q * h * 513 * 4 + rows * 128 * 2 + g * 512 * 128 * 2,
+                           "flops": 2.0 * rows * 512 * 128},
+        "combine_gqa": {"bytes": pieces * s_q * h * 129 * 4 + rows * 128 * 2, "flops": 0.0},
+        "expand": {"bytes": case["num_pages"] * 64 * (1152 + 4224) + 2 * g * 512 * 128 * 2,
+                   "flops": 2.0 * case["num_pages"] * 64 * 512 * 256 * g},
+    }
+    return acc, {"tokens": tokens, "pairs": pairs, "pieces": pieces}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def _gather(case, batch_ids):
+    """CPU copy of the chosen sequences with their pages only (for the oracle)."""
+    ps = case["page_size"]
+    pt = case["page_table"].cpu()
+    sl = case["seqlens"].cpu()
+    pages, rows = [], []
+    for b in batch_ids:
+        n = max(1, math.ceil(int(sl[b]) / ps))
+        rows.append(list(range(len(pages), len(pages) + n)))
+        pages.extend(pt[b, :n].tolist())
+    dev = case["latent"].device
+    latent = case["latent"][torch.tensor(pages, device=dev)].cpu()
+    new_pt = torch.zeros(len(batch_ids), max(len(r) for r in rows), dtype=torch.int32)
+    for i, r in enumerate(rows):
+        new_pt[i, :len(r)] = torch.tensor(r, dtype=torch.int32)
+    q = case["q"][torch.tensor(batch_ids, device=case["q"].device)].cpu()
+    return q, latent, new_pt, sl[batch_ids].clone()
+
+
+def cpu_oracle_rate(case, w, s_q, budget_s=10.0, unit_groups=None):
+    """Run the oracle on successive sequences (all groups, or `unit_groups` of
+    them) until budget_s has elapsed; return (tokens/s, cores, description)."""
+    import oracle
+    cores = oracle.num_threads()
+    B = case["seqlens"].numel()
+    per_call = max(1, cores // (unit_groups or w.num_groups))
+    done_seqs, elapsed, b = 0, 0.0, 0
+    while b < B and (elapsed < budget_s or done_seqs == 0):
+        ids = list(range(b, min(B, b + per_call)))
+        q, lat, pt, sl = _gather(case, ids)
+        units = None
+        if unit_groups:
+            units = [(i, gi) for i in range(len(ids)) for gi in range(unit_groups)]
+        t0 = time.perf_counter()
+        oracle.decode(q, lat, pt, sl, case["w_uk"].cpu(), case["w_uv"].cpu(), w.num_groups,
+                      units=units)
+        elapsed += time.perf_counter() - t0
+        done_seqs += len(ids)
+        b += len(ids)
+    frac = (unit_groups or w.num_groups) / w.num_groups
+    rate = done_seqs * s_q * frac / elapsed
+    what = (f"{done_seqs} of {B} sequences"
+            + (f", {unit_groups} of {w.num_groups} groups" if unit_groups else ", all groups")
+            + f", {elapsed:.1f} s fp64 oracle")
+    return rate, cores, what
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+def run_ours(args, rank, world, local_rank):
+    from decode_attention_06_b200 import gqla, synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    s_q = args.s_q or w.s_q[0]
+    case = synth.make_case(w.num_heads, w.num_groups, w.seqlens(), s_q, paged=w.paged,
+                           seed=w.seed + 1000 * rank, device=str(dev))
+    h, g = w.num_heads, w.num_groups
+    B = case["seqlens"].numel()
+    dims = gqla.make_dims(h, g)
+    kv = gqla.make_kv_index(case["page_table"], case["seqlens"], case["num_pages"])
+    n_slots = case["num_pages"] * case["page_size"]
+    splits = {"absorb": args.splits or gqla.gqla_num_splits_hint("absorb"),
+              "gqa": args.splits or gqla.gqla_num_splits_hint("gqa")}
+    kvx = torch.empty(g, n_slots, 256, dtype=torch.bfloat16, device=dev)
+    kr = torch.empty(n_slots, 64, dtype=torch.bfloat16, device=dev)
+    ba = gqla.DecodeBuffers(dims, B, s_q, splits["absorb"], "absorb", device=dev)
+    bg = gqla.DecodeBuffers(dims, B, s_q, splits["gqa"], "gqa", device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # one-shot expansion, timed on its own
+    gqla.gqla_expand_cache(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.fill_(1.0)
+    e0.record()
+    gqla.gqla_expand_cache(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
+    e1.record()
+    torch.cuda.synchronize()
+    expand_ms = e0.elapsed_time(e1)
+
+    names = ["absorb_query", "decode_absorb", "combine_absorb", "decode_gqa", "combine_gqa"]
+    calls = [
+        lambda: gqla.gqla_absorb_query(dims, case["q"], case["w_uk"], ba.q_absorbed),
+        lambda: gqla.gqla_decode_absorb(dims, ba.q_absorbed, case["latent"], kv, ba.num_splits,
+                                        ba.o_part, ba.lse_part, ba.workspace),
+        lambda: gqla.gqla_combine(dims, kv, s_q, ba.num_splits, 512, ba.o_part, ba.lse_part,
+                                  case["w_uv"], ba.out, ba.lse),
+        lambda: gqla.gqla_decode_gqa(dims, case["q"], kvx, kr, kv, bg.num_splits, bg.o_part,
+                                     bg.lse_part, bg.workspace),
+        lambda: gqla.gqla_combine(dims, kv, s_q, bg.num_splits, 128, bg.o_part, bg.lse_part,
+                                  None, bg.out, bg.lse),
+    ]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+          for _ in range(args.steps)]
+
+    def step(events=None):
+        for i, c in enumerate(calls):
+            if events is not None:
+                events[i].record(stream)
+            c()
+        if events is not None:
+            events[-1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for k in range(args.steps):
+            flush.fill_(1.0)  # evict the caches from L2 (outside the step's events)
+            step(ev[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    per_call = [[ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)]
+                for i in range(len(calls))]
+    step_ms = [ev[k][0].elapsed_time(ev[k][-1]) for k in range(args.steps)]
+    ms_step = sum(step_ms) / args.steps
+    st_a, _ = gqla.gqla_read_device_error(ba.workspace)
+    st_g, _ = gqla.gqla_read_device_error(bg.workspace)
+    if st_a or st_g:
+        raise RuntimeError(f"device-side error during the bench: {st_a} {st_g}")
+
+    # ---- e2e: host buffers through the C ABI, copies inside the timed region
+    q_h = case["q"].cpu().pin_memory()
+    pt_h = case["page_table"].cpu().pin_memory()
+    sl_h = case["seqlens"].cpu().pin_memory()
+    outa_h = torch.empty(ba.out.shape, dtype=torch.bfloat16).pin_memory()
+    outg_h = torch.empty(bg.out.shape, dtype=torch.bfloat16).pin_memory()
+    q_d, pt_d, sl_d = case["q"], case["page_table"], case["seqlens"]
+    h2d = q_h.numel() * 2 + pt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = outa_h.numel() * 2 + outg_h.numel() * 2
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for k in range(args.steps + args.warmup):
+        flush.fill_(1.0)
+        if k >= args.warmup:
+            e2e_ev[k - args.warmup][0].record(stream)
+        q_d.copy_(q_h, non_blocking=True)
+        pt_d.copy_(pt_h, non_blocking=True)
+        sl_d.copy_(sl_h, non_blocking=True)
+        step()
+        outa_h.copy_(ba.out, non_blocking=True)
+        outg_h.copy_(bg.out, non_blocking=True)
+        if k >= args.warmup:
+            e2e_ev[k - args.warmup][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+
+    # ---- max over ranks
+    t = torch.tensor([ms_step, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_step, e2e_ms = float(t[0]), float(t[1])
+    tokens_step = B * s_q
+    value = world * tokens_step / (ms_step * 1e-3)
+    e2e_value = world * tokens_step / (e2e_ms * 1e-3)
+
+    acc, counts = accounting(w, case, s_q, splits["gqa"])
+    acc_a, _ = accounting(w, case, s_q, splits["absorb"])
+    acc["decode_absorb"] = acc_a["decode_absorb"]
+    acc["combine_absorb"] = acc_a["combine_absorb"]
+    mean = {n: sum(v) / len(v) for n, v in zip(names, per_call)}
+    peaks, peak_kind = _peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])
+
+    def roof(name):
+        sec = mean[name] * 1e-3
+        gbs = acc[name]["bytes"] / sec / 1e9
+        tfs = acc[name]["flops"] / sec / 1e12
+        return {"us": mean[name] * 1e3, "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak,
+                "tflops": tfs, "tensor_frac": tfs / tc_peak}
+
+    per_kernel = {n: roof(n) for n in names}
+    share = {n: mean[n] / sum(mean.values()) for n in names}
+    dominant = max(names, key=lambda n: mean[n])
+    dk = per_kernel[dominant]
+    t_mem = acc[dominant]["bytes"] / (hbm_peak * 1e9)
+    t_cmp = acc[dominant]["flops"] / (tc_peak * 1e12)
+    if t_cmp > t_mem:
+        roofline = {"bound": "tensor", "achieved": dk["tflops"], "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": dk["tensor_frac"]}
+    else:
+        roofline = {"bound": "hbm", "achieved": dk["hbm_gbs"], "peak": hbm_peak,
+                    "unit": "GB/s", "frac": dk["hbm_frac"]}
+    roofline.update({"kernel": dominant, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)"
+                     if peak_kind == "measured" else "fallback",
+                     "algorithmic_bytes_per_launch": acc[dominant]["bytes"],
+                     "algorithmic_flops_per_launch": acc[dominant]["flops"],
+                     "traffic": _stored_traffic(dominant, args.workload)})
+
+    def path_info(kernels, dec):
+        us = sum(mean[k] for k in kernels) * 1e3
+        t_m = acc[dec]["bytes"] / (hbm_peak * 1e9)
+        t_c = acc[dec]["flops"] / (tc_peak * 1e12)
+        bound = "tensor" if t_c > t_m else "hbm"
+        frac = (t_c if bound == "tensor" else t_m) / (mean[dec] * 1e-3)
+        return {"us_per_step": us, "tokens_per_s": world * tokens_step / (us * 1e-6),
+                "decode_kernel": dec, "decode_us": mean[dec] * 1e3, "binding": bound,
+                "binding_roofline_frac": frac, "hbm_frac": per_kernel[dec]["hbm_frac"],
+                "tensor_frac": per_kernel[dec]["tensor_frac"]}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 cache/queries, N(0,1/512) bf16 W_UK/W_UV)",
+        "config": {"workload": args.workload, "num_heads": h, "num_groups": g, "batch": B,
+                   "context": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths[1:]),
+                   "s_q": s_q, "paged": w.paged, "paths": ["absorb", "gqa"],
+                   "tokens_per_step": tokens_step, "num_splits": splits,
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world} (independent batches per GPU)"},
+        "roofline": roofline,
+        "per_path": {"absorb": path_info(["absorb_query", "decode_absorb", "combine_absorb"],
+                                         "decode_absorb"),
+                     "gqa": path_info(["decode_gqa", "combine_gqa"], "decode_gqa")},
+        "per_kernel": {n: dict(per_kernel[n], share=share[n]) for n in names},
+        "expand": {"ms": expand_ms, "slots": n_slots,
+                   "tflops": acc["expand"]["flops"] / (expand_ms * 1e-3) / 1e12},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": len(calls) * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, what = cpu_oracle_rate(case, w, s_q, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
+                                  "kind": "oracle", "sample": what}
+    return result
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step decodes one (sequence, group)
+    unit of the workload on the host cores."""
+    from decode_attention_06_b200 import synth
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    s_q = args.s_q or w.s_q[0]
+    case = synth.make_case(w.num_heads, w.num_groups, w.seqlens(), s_q, paged=w.paged,
+                           seed=w.seed)
+    B = case["seqlens"].numel()
+    times = []
+    for k in range(args.warmup + args.steps):
+        b = k % B
+        q, lat, pt, sl = _gather(case, [b])
+        t0 = time.perf_counter()
+        oracle.decode(q, lat, pt, sl, case["w_uk"], case["w_uv"], w.num_groups,
+                      units=[(0, k % w.num_groups)])
+        if k >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    tokens = s_q / w.num_groups  # one group of one sequence = 1/g of its s_q tokens
+    value = tokens / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same generator and workload as the GPU arm)",
+        "config": {"workload": args.workload, "num_heads": w.num_heads,
+                   "num_groups": w.num_groups, "batch": B, "s_q": s_q,
+                   "paths": ["un-absorbed definition"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": "one (sequence, group) unit per step: all heads of one "
+                                   "group of one sequence, fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--s-q", dest="s_q", type=int, default=None)
+    ap.add_argument("--splits", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
