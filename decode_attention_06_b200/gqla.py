@@ -59,6 +59,7 @@ _SIGS = {
     "gqla_decode_absorb": [_DP, _P, _I, _P, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_combine": [_DP, _KP, _I, _I, _I, _P, _P, _P, _P, _P, _P],
+    "gqla_decode_gqa_noalloc": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _P],
     "gqla_partial_slots": [_I, _I],
     "gqla_workspace_bytes": [],
     "gqla_num_splits_hint": [_I],
@@ -174,6 +175,21 @@ def gqla_combine(dims, kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out, l
         None if w_uv is None else _dev(w_uv, "w_uv", torch.bfloat16, (dims.num_groups, D_LATENT, D_V)),
         _dev(out, "out", torch.bfloat16, (kv.batch, s_q, h, D_V)),
         None if lse_out is None else _dev(lse_out, "lse_out", torch.float32, (kv.batch, s_q, h)),
+        _stream(stream)))
+
+
+def gqla_decode_gqa_noalloc(dims, q, kv_expanded, k_rope, kv, num_splits, out, lse_out=None,
+                            device_error=None, stream=None):
+    """GQA decode step with library-owned static scratch (no o_part/lse_part/workspace)."""
+    B, s_q, h, _ = q.shape
+    n = kv.num_pages * kv.page_size
+    _check("gqla_decode_gqa_noalloc", _lib.gqla_decode_gqa_noalloc(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16, (kv.batch, s_q, dims.num_heads, D_QK)), s_q,
+        _dev(kv_expanded, "kv_expanded", torch.bfloat16, (dims.num_groups, n, D_NOPE + D_V)),
+        _dev(k_rope, "k_rope", torch.bfloat16, (n, D_ROPE)), n, ctypes.byref(kv), num_splits,
+        _dev(out, "out", torch.bfloat16, (kv.batch, s_q, h, D_V)),
+        None if lse_out is None else _dev(lse_out, "lse_out", torch.float32, (kv.batch, s_q, h)),
+        None if device_error is None else _dev(device_error, "device_error", torch.int32, (2,)),
         _stream(stream)))
 
 

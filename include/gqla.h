@@ -158,6 +158,41 @@ int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int nu
                  int d_in, const float *o_part, const float *lse_part, const void *w_uv,
                  void *out, float *lse_out, gqla_stream_t stream);
 
+/*
+ * GQA-path decode step that allocates nothing: gqla_decode_gqa followed by
+ * gqla_combine, with the split partials, their LSEs and the device error
+ * record kept in a file-scope device array owned by the library.  The pages
+ * have no counterpart of this call: it exists for callers that cannot
+ * allocate device memory -- code under an allocator that forbids cudaMalloc
+ * once serving has started, plugins that are handed only their input and
+ * output buffers, or threads that must not call into an allocator on the
+ * decode path -- and so cannot supply o_part / lse_part / workspace.
+ *
+ *   Inputs and outputs are those of gqla_decode_gqa and gqla_combine (GQA
+ *   partials, d_in = 128): q, kv_expanded, k_rope, num_slots, kv, num_splits
+ *   as there; out bf16 [batch][s_q][h][128], lse_out fp32 [batch][s_q][h] or
+ *   NULL; device_error: NULL, or a device int32[2] that receives {status,
+ *   info} of the device-side checks of this call (what gqla_read_device_error
+ *   would return for an ordinary workspace).
+ *   Limit: the partials of (batch + num_splits) * s_q * h rows, 516 bytes
+ *   each (rounded up), plus 256 bytes must fit in GQLA_NOALLOC_SCRATCH_BYTES
+ *   (32 MiB); larger requests return GQLA_ERR_WORKSPACE before any launch.
+ *   Every GPU that loads libgqla reserves this array until the process exits.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   with cudaGetSymbolAddress (with that device current); make that first
+ *   call before any stream capture.  Nothing is allocated or freed, by this
+ *   call or by any library it uses.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents (the error record is cleared at the start of each call).
+ *   Calls that overlap on the GPU -- on different streams, or from different
+ *   threads -- race on it and give undefined results; serialise them.
+ */
+#define GQLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+int gqla_decode_gqa_noalloc(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
+                            const void *k_rope, int64_t num_slots, const gqla_kv_index *kv,
+                            int num_splits, void *out, float *lse_out, int32_t *device_error,
+                            gqla_stream_t stream);
+
 /* Number of partial slots the decode calls address: batch + num_splits. */
 int gqla_partial_slots(int batch, int num_splits);
 
