@@ -1,7 +1,6 @@
-// decode_simt.cu -- split-KV partial attention on the FP32 pipes, both paths.
+// decode_simt.cu -- split-KV partial attention of the MQA-absorb path on the FP32 pipes.
 //
-// One CTA per (chunk of the split plan, group) for the GQA path and per
-// (chunk, 16 query rows) for the absorb path.  Each page of 64 tokens is
+// One CTA per (chunk of the split plan, 16 query rows).  Each page of 64 tokens is
 // staged in shared memory, scores and the online softmax run in fp32 (base-2
 // exponent with log2(e) folded into the scale), and the partial output is
 // written normalised with its natural-log LSE.  This is the plain CUDA-core
@@ -13,160 +12,7 @@ namespace gqla {
 
 namespace {
 
-constexpr int MAXR = 32;  // query rows per CTA (G * s_q for the GQA path)
-
 __device__ __forceinline__ float bf(const __nv_bfloat16 &x) { return __bfloat162float(x); }
-
-// ---------------------------------------------------------------------------
-// GQA path.  grid (num_splits, g), 256 threads.
-// Shared: q [R][192] fp32, K [64][193] fp32, V [64][128] fp32, P [R][64] fp32.
-// Row i of the CTA is query token s = i / G, head gi*G + i % G.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) decode_gqa_simt_kernel(
-    const __nv_bfloat16 *__restrict__ q, int s_q, int heads, int G,
-    const __nv_bfloat16 *__restrict__ kv, const __nv_bfloat16 *__restrict__ k_rope,
-    int64_t num_slots, const int32_t *__restrict__ page_table,
-    const int32_t *__restrict__ seqlens, int batch, int max_pages, int num_pages,
-    int num_splits, float scale_log2, float *__restrict__ o_part, float *__restrict__ lse_part,
-    void *ws) {
-    extern __shared__ __align__(16) float smem[];
-    float *qs = smem;                       // [MAXR][192]
-    float *Ks = qs + MAXR * kQk;            // [64][193]
-    float *Vs = Ks + kPage * (kQk + 1);     // [64][128]
-    float *Ps = Vs + kPage * kDv;           // [MAXR][64]
-    __shared__ float s_m[MAXR], s_l[MAXR], s_alpha[MAXR];
-    __shared__ int s_plan[4];
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int c = blockIdx.x, gi = blockIdx.y;
-    const int R = G * s_q;
-
-    if (warp == 0) {
-        int total = warp_total_pages(seqlens, batch);
-        int k = chunk_pages(total, num_splits);
-        int r0 = c * k, r1 = min(total, r0 + k);
-        int b = batch, start = 0;
-        if (r0 < r1) warp_find_sequence(seqlens, batch, r0, &b, &start);
-        if (lane == 0) { s_plan[0] = r0; s_plan[1] = r1; s_plan[2] = b; s_plan[3] = start; }
-    }
-    __syncthreads();
-    const int r0 = s_plan[0], r1 = s_plan[1];
-    int b = s_plan[2], P = s_plan[3];
-    const __nv_bfloat16 *kvg = kv + (size_t)gi * num_slots * kKv;
-
-    for (; b < batch && P < r1; ++b) {
-        const int L = seqlens[b];
-        const int n = pages_of(L);
-        if (n == 0) continue;
-        const int p_begin = max(r0, P) - P, p_end = min(r1, P + n) - P;
-        P += n;
-        if (L > max_pages * kPage) {
-            if (tid == 0) report_error(ws, GQLA_ERR_DEVICE, b);
-            continue;
-        }
-        __syncthreads();
-        for (int i = tid; i < R * kQk; i += 256) {
-            int row = i / kQk, d = i % kQk;
-            int s = row / G, h = gi * G + row % G;
-            qs[i] = bf(q[(((int64_t)b * s_q + s) * heads + h) * kQk + d]);
-        }
-        if (tid < R) { s_m[tid] = -INFINITY; s_l[tid] = 0.0f; }
-        float o[MAXR / 2];
-#pragma unroll
-        for (int i = 0; i < MAXR / 2; ++i) o[i] = 0.0f;
-        const int dv = tid & 127, half = tid >> 7;
-
-        for (int p = p_begin; p < p_end; ++p) {
-            const int page = page_table[(int64_t)b * max_pages + p];
-            const bool bad = page < 0 || page >= num_pages;
-            if (bad && tid == 0) report_error(ws, GQLA_ERR_DEVICE, b);
-            __syncthreads();
-            if (!bad) {
-                for (int i = tid; i < kPage * (kKv / 8); i += 256) {  // K_nope | V rows
-                    int t = i / (kKv / 8), part = i % (kKv / 8);
-                    int64_t slot = (int64_t)page * kPage + t;
-                    uint4 v = *reinterpret_cast<const uint4 *>(kvg + slot * kKv + part * 8);
-                    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&v);
-                    for (int j = 0; j < 8; ++j) {
-                        int col = part * 8 + j;
-                        if (col < kNope) Ks[t * (kQk + 1) + col] = bf(e[j]);
-                        else Vs[t * kDv + col - kNope] = bf(e[j]);
-                    }
-                }
-                for (int i = tid; i < kPage * (kRope / 8); i += 256) {
-                    int t = i / (kRope / 8), part = i % (kRope / 8);
-                    int64_t slot = (int64_t)page * kPage + t;
-                    uint4 v = *reinterpret_cast<const uint4 *>(k_rope + slot * kRope + part * 8);
-                    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&v);
-                    for (int j = 0; j < 8; ++j) Ks[t * (kQk + 1) + kNope + part * 8 + j] = bf(e[j]);
-                }
-            }
-            __syncthreads();
-            // scores (log2 domain), masked -> -inf
-            for (int i = tid; i < R * kPage; i += 256) {
-                int row = i / kPage, t = i % kPage;
-                int s = row / G;
-                int tok = p * kPage + t;
-                float v = -INFINITY;
-                if (!bad && tok <= L - s_q + s) {
-                    float acc = 0.0f;
-                    const float *qr = qs + row * kQk;
-                    const float *kr = Ks + t * (kQk + 1);
-                    for (int d = 0; d < kQk; ++d) acc = fmaf(qr[d], kr[d], acc);
-                    v = acc * scale_log2;
-                }
-                Ps[row * kPage + t] = v;
-            }
-            __syncthreads();
-            // online softmax statistics, one warp per row
-            for (int row = warp; row < R; row += 8) {
-                float a = Ps[row * kPage + lane], bb = Ps[row * kPage + lane + 32];
-                float mx = fmaxf(a, bb);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                float m_old = s_m[row];
-                float m_new = fmaxf(m_old, mx);
-                float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_old - m_new);
-                float pa = (a == -INFINITY) ? 0.0f : exp2f(a - m_new);
-                float pb = (bb == -INFINITY) ? 0.0f : exp2f(bb - m_new);
-                Ps[row * kPage + lane] = pa;
-                Ps[row * kPage + lane + 32] = pb;
-                float sum = pa + pb;
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-                if (lane == 0) {
-                    s_m[row] = m_new;
-                    s_l[row] = s_l[row] * alpha + sum;
-                    s_alpha[row] = alpha;
-                }
-            }
-            __syncthreads();
-            const int t_end = bad ? 0 : min(kPage, L - p * kPage);  // pool rows past L are never read
-#pragma unroll
-            for (int i = 0; i < MAXR / 2; ++i) {
-                int row = half * (MAXR / 2) + i;
-                if (row >= R) break;
-                float acc = o[i] * s_alpha[row];
-                const float *pr = Ps + row * kPage;
-                for (int t = 0; t < t_end; ++t) acc = fmaf(pr[t], Vs[t * kDv + dv], acc);
-                o[i] = acc;
-            }
-        }
-        __syncthreads();
-        const int slot = b + c;
-#pragma unroll
-        for (int i = 0; i < MAXR / 2; ++i) {
-            int row = half * (MAXR / 2) + i;
-            if (row >= R) break;
-            int s = row / G, h = gi * G + row % G;
-            float l = s_l[row];
-            int64_t idx = ((int64_t)slot * s_q + s) * heads + h;
-            o_part[idx * kDv + dv] = l > 0.0f ? o[i] / l : 0.0f;
-            if (dv == 0)
-                lse_part[idx] = l > 0.0f ? (s_m[row] + __log2f(l)) * 0.6931471805599453f : -INFINITY;
-        }
-    }
-}
 
 // ---------------------------------------------------------------------------
 // MQA-absorb path.  grid (num_splits, s_q*h/16), 256 threads, 16 rows per CTA.
@@ -303,22 +149,6 @@ __global__ void __launch_bounds__(256) decode_absorb_simt_kernel(
 }
 
 }  // namespace
-
-cudaError_t launch_decode_gqa_simt(const void *q, int s_q, int heads, int num_groups,
-                                   const void *kv, const void *k_rope, int64_t num_slots,
-                                   const gqla_kv_index *idx, int num_splits, float scale,
-                                   float *o_part, float *lse_part, void *ws, cudaStream_t stream) {
-    const int G = heads / num_groups;
-    size_t smem = sizeof(float) * (MAXR * kQk + kPage * (kQk + 1) + kPage * kDv + MAXR * kPage);
-    cudaFuncSetAttribute(decode_gqa_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    dim3 grid(num_splits, num_groups);
-    decode_gqa_simt_kernel<<<grid, 256, smem, stream>>>(
-        static_cast<const __nv_bfloat16 *>(q), s_q, heads, G, static_cast<const __nv_bfloat16 *>(kv),
-        static_cast<const __nv_bfloat16 *>(k_rope), num_slots, idx->page_table, idx->seqlens,
-        idx->batch, idx->max_pages_per_seq, idx->num_pages, num_splits, scale * kLog2e, o_part,
-        lse_part, ws);
-    return cudaGetLastError();
-}
 
 cudaError_t launch_decode_absorb_simt(const void *qa, int s_q, int heads, const void *cache,
                                       const gqla_kv_index *idx, int num_splits, float scale,

@@ -10,10 +10,10 @@ cudaError_t launch_expand(const void *latent, int64_t num_slots, const void *w_u
                           cudaStream_t stream);
 cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_groups,
                                 const void *w_uk, void *qa, cudaStream_t stream);
-cudaError_t launch_decode_gqa_simt(const void *q, int s_q, int heads, int num_groups,
-                                   const void *kv, const void *k_rope, int64_t num_slots,
-                                   const gqla_kv_index *idx, int num_splits, float scale,
-                                   float *o_part, float *lse_part, void *ws, cudaStream_t stream);
+cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups, const void *kv,
+                              const void *k_rope, int64_t num_slots, const gqla_kv_index *idx,
+                              int num_splits, float scale, float *o_part, float *lse_part,
+                              void *ws, cudaStream_t stream);
 cudaError_t launch_decode_absorb_simt(const void *qa, int s_q, int heads, const void *cache,
                                       const gqla_kv_index *idx, int num_splits, float scale,
                                       float *o_part, float *lse_part, void *ws,
@@ -170,10 +170,11 @@ int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *k
     if (!aligned16(q) || !aligned16(kv_expanded) || !aligned16(k_rope) || !aligned16(o_part))
         return GQLA_ERR_INVALID_ARG;
     if (num_slots != (int64_t)kv->num_pages * kv->page_size) return GQLA_ERR_INVALID_ARG;
-    return cuda_status(launch_decode_gqa_simt(q, s_q, dims->num_heads, dims->num_groups,
-                                              kv_expanded, k_rope, num_slots, kv, num_splits,
-                                              dims->softmax_scale, o_part, lse_part, workspace,
-                                              reinterpret_cast<cudaStream_t>(stream)));
+    if (dims->num_groups != 8) return GQLA_ERR_UNSUPPORTED;
+    return cuda_status(launch_decode_gqa(q, s_q, dims->num_heads, dims->num_groups, kv_expanded,
+                                         k_rope, num_slots, kv, num_splits, dims->softmax_scale,
+                                         o_part, lse_part, workspace,
+                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
