@@ -6,25 +6,32 @@
 //
 // The path is HBM-bound (about 19 FLOP per cache byte at s_q = 1), so the
 // design goal is to stream the 4224 bytes per token exactly once at full
-// bandwidth and hide everything else behind it:
+// bandwidth and hide everything else behind it.
 //
-//  * One CTA per chunk of the split plan (grid = SM count), 192 threads:
-//      warp 0      TMA producer: per page, the shared RoPE keys (8 KB), then
-//                  per group K_nope_g and V_g (4 boxes of 64 x 64 bf16,
-//                  32 KB) into a 3-4 stage ring (128B-swizzled);
-//      warp 1      TMEM owner and single-thread tcgen05.mma issuer;
-//      warps 2-5   softmax, rescaling and the epilogue.
-//  * The query rows of a group (G*s_q <= 32) are far below the 64/128-row
-//    MMA minimum, so the products are transposed ("swap-AB"): the 64 tokens
-//    of a page are the M dimension and the group's query rows the N
-//    dimension.
-//      S^T[64 tok][NQ]   = [K_nope_g | k^R] (64 x 192, K-major) x q_g^T
-//      O^T_g[128 dv][NQ] += V_g^T (MN-major) x P^T (MN-major, bf16)
-//    O^T of all 8 groups stays resident in TMEM for the whole piece.
-//  * Online softmax in the base-2 domain with lazy rescaling: the running
-//    maximum of a column moves only when a tile exceeds it by more than
-//    2^8, so O^T in TMEM is rescaled rarely.  Column maxima and sums over
-//    the 64 tokens are warp butterflies plus a 4-warp exchange.
+//  * Work unit = (128 tokens = two consecutive pages of one sequence, group).
+//    The query rows of a group (G*s_q <= 32) are far below the MMA's minimum
+//    M, so the products are transposed ("swap-AB"): the 128 tokens are the M
+//    dimension and the group's query rows the N dimension (NQ = 16 or 32,
+//    zero-padded):
+//      S^T[128 tok][NQ]    = [K_nope_g | k^R] (128 x 192, K-major) x q_g^T
+//      O^T_g[128 dv][NQ]  += V_g^T (MN-major) x P^T (MN-major, bf16)
+//    With M = 128 every TMEM lane, and so every softmax thread, owns one
+//    token.  O^T of all 8 groups stays resident in TMEM for a whole piece.
+//  * One CTA per chunk of the split plan (grid = SM count), 320 threads:
+//      warp 0      TMA producer over three rings: q_g + K_nope_g (freed as
+//                  soon as S^T is done), V_g (freed after O^T += ...), and
+//                  per page pair the shared RoPE keys; each ring refills as
+//                  soon as a slot frees, so loads run well ahead;
+//      warp 1      TMEM owner; one thread issues the score MMAs;
+//      warps 2-9   two softmax warpgroups (groups 0,2,4,6 and 1,3,5,7): each
+//                  runs its online softmax, issues its own PV MMAs (one
+//                  elected thread) and writes its epilogue.
+//  * Online softmax in the base-2 domain with lazy rescaling: P is formed
+//    against the running column maxima straight away, and one barrier-with-
+//    OR over the warpgroup both publishes P and asks whether any score rose
+//    more than 2^8 above its maximum.  Only then (and on a piece's first
+//    tile) are the tile's column maxima reduced across warps, O^T in TMEM
+//    rescaled and P recomputed.
 //  * Every wait is bounded; a wait that runs out records GQLA_ERR_TIMEOUT
 //    and the CTA drains and exits instead of hanging.
 #include <cudaTypedefs.h>
@@ -38,35 +45,38 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;        // warp 0 TMA, warp 1 score MMA, warps 2-9: two softmax warpgroups
+constexpr int kTok = 128;            // tokens per unit (two pages)
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kKvBox = 64 * 64 * 2;  // one 64-token x 64-column bf16 box
+constexpr int kBox = 64 * 64 * 2;    // one 64-row x 64-column bf16 TMA box (8 KB)
 
 template <int NQ>
 struct GqaSmem {
-    static constexpr int kStages = NQ == 16 ? 4 : 3;
-    static constexpr int kStageBytes = 4 * kKvBox;       // K lo | K hi | V lo | V hi
-    static constexpr int kKrBytes = kKvBox;              // 64 tokens x 64 RoPE dims
-    static constexpr int kQBlock = 8 * NQ * 128;         // 64 q dims x (8 groups x NQ rows)
-    static constexpr int kPBytes = 64 * NQ * 2;          // P^T [64 tokens][NQ] bf16
-    static constexpr int oStage = 0;
-    static constexpr int oKr = oStage + kStages * kStageBytes;
-    static constexpr int oQ = oKr + 2 * kKrBytes;
-    static constexpr int oP = oQ + 3 * kQBlock;
-    static constexpr int oRed = oP + 2 * ((kPBytes + 1023) / 1024) * 1024;  // float [NQ][4]
-    static constexpr int oMrun = oRed + NQ * 4 * 4;                        // float [2][8][NQ]
-    static constexpr int oLw = oMrun + 2 * 8 * NQ * 4;                     // float [4][8][NQ]
-    static constexpr int oBar = oLw + 4 * 8 * NQ * 4;
-    // barriers: full[S], empty[S], kr_full[2], kr_empty[2], s_full[2], s_free[2],
-    //           p_full[2], p_free[2], q_full, o_done, drain
-    static constexpr int kNumBars = 2 * kStages + 15;
+    static constexpr int kKSlots = NQ == 16 ? 3 : 2;
+    static constexpr int kVSlots = 2;
+    static constexpr int kQBytes = 3 * NQ * 128;        // q_g: 3 column blocks x NQ rows x 128 B
+    static constexpr int kKBytes = 4 * kBox;            // K lo | K hi, 128 rows each
+    static constexpr int kKSlotBytes = kKBytes + ((kQBytes + 1023) / 1024) * 1024;
+    static constexpr int kVBytes = 4 * kBox;            // V lo | V hi, 128 rows each
+    static constexpr int kKrBytes = 2 * kBox;           // 128 rows x 64 RoPE dims
+    static constexpr int kPBytes = kTok * NQ * 2;       // P^T [128 tokens][NQ] bf16
+    static constexpr int oK = 0;
+    static constexpr int oV = oK + kKSlots * kKSlotBytes;
+    static constexpr int oKr = oV + kVSlots * kVBytes;
+    static constexpr int oP = oKr + 2 * kKrBytes;            // one P^T buffer per warpgroup
+    static constexpr int oRed = oP + 2 * kPBytes;            // float [2 wg][NQ][4 warps]
+    static constexpr int oMrun = oRed + 2 * NQ * 4 * 4;      // float [8 groups][NQ]
+    static constexpr int oLred = oMrun + 8 * NQ * 4;         // float [8 groups][NQ][4 warps]
+    static constexpr int oBar = oLred + 8 * NQ * 4 * 4;
+    // k_full/k_empty[KS], v_full/v_empty[VS], kr_full/kr_empty[2], s_full/s_free[4],
+    // p_free[2], o_done[2], drain
+    static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 4 + 8 + 4 + 1;
     static constexpr int oMisc = oBar + kNumBars * 8;  // tmem base, abort flag, plan[4]
     static constexpr int kBytes = oMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
 struct GqaParams {
-    const __nv_bfloat16 *q;
     const int32_t *page_table;
     const int32_t *seqlens;
     float *o_part;
@@ -97,6 +107,59 @@ __device__ __forceinline__ bool next_piece(const GqaParams &p, PieceIter &it, in
     return false;
 }
 
+// The two pages of a unit and how many of their rows are real tokens.
+struct PagePair {
+    int page0, page1;  // -1: missing (past the piece) or outside the pool
+    int rows0, rows1;  // valid token rows in each page
+    bool bad;          // a page index outside the pool was met
+};
+
+__device__ __forceinline__ PagePair load_pair(const GqaParams &p, int b, int L, int pg, int pe) {
+    const int32_t *row = p.page_table + (int64_t)b * p.max_pages;
+    PagePair pp;
+    const int a0 = row[pg];
+    const int a1 = pg + 1 < pe ? row[pg + 1] : 0;
+    const bool bad0 = a0 < 0 || a0 >= p.num_pages;
+    const bool bad1 = pg + 1 < pe && (a1 < 0 || a1 >= p.num_pages);
+    pp.bad = bad0 || bad1;
+    pp.page0 = bad0 ? -1 : a0;
+    pp.page1 = (pg + 1 < pe && !bad1) ? a1 : -1;
+    pp.rows0 = bad0 ? 0 : min(kPage, L - pg * kPage);
+    pp.rows1 = pp.page1 >= 0 ? min(kPage, L - (pg + 1) * kPage) : 0;
+    return pp;
+}
+
+// Walks the units (sequence, page pair, group) of a chunk in pipeline order.
+struct UnitCursor {
+    PieceIter it;
+    int b, L, pg, pe, gi;
+    PagePair pp;
+    bool valid;
+    __device__ __forceinline__ bool next_valid_piece(const GqaParams &p) {
+        int pb;
+        bool too_long;
+        while (next_piece(p, it, b, L, pb, pe, too_long)) {
+            if (too_long) continue;
+            pg = pb;
+            gi = 0;
+            pp = load_pair(p, b, L, pg, pe);
+            return true;
+        }
+        return false;
+    }
+    __device__ __forceinline__ void start(const GqaParams &p, const PieceIter &it0) {
+        it = it0;
+        valid = next_valid_piece(p);
+    }
+    __device__ __forceinline__ void advance(const GqaParams &p) {
+        if (++gi < 8) return;
+        gi = 0;
+        pg += 2;
+        if (pg < pe) { pp = load_pair(p, b, L, pg, pe); return; }
+        valid = next_valid_piece(p);
+    }
+};
+
 // Butterfly over the lanes of each NQ-lane group: each lane starts with NQ
 // column values and ends holding column (lane % NQ) reduced over the group.
 template <int NQ, bool MAX>
@@ -115,44 +178,106 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[NQ], int lane) {
     return v[0];
 }
 
-__device__ __forceinline__ void named_bar_sync() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+// Column reduction over all 32 lanes; lane n (and n + 16 when NQ = 16) ends with column n.
+template <int NQ, bool MAX>
+__device__ __forceinline__ float column_reduce32(float (&v)[NQ], int lane) {
+    float r = transpose_reduce<NQ, MAX>(v, lane);
+    if constexpr (NQ == 16) {
+        const float o = __shfl_xor_sync(0xffffffffu, r, 16);
+        r = MAX ? fmaxf(r, o) : r + o;
+    }
+    return r;
+}
+
+// Barrier over the 128 threads of one softmax warpgroup (ids 1 and 2).
+__device__ __forceinline__ void wg_bar(int wg) {
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
+}
+
+// Same barrier, returning whether the predicate was true in any of the 128 threads.
+__device__ __forceinline__ bool wg_bar_any(int wg, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(1 + wg)
+        : "memory");
+    return r != 0;
+}
+
+// Score of column n in log2 units, or -inf where the token is masked: not a
+// real token, or (s_q = 2) the newest token hidden from the first query token,
+// whose columns are n < G.
+__device__ __forceinline__ float score_of(uint32_t raw, int n, bool tok_ok, bool hide_low, int G,
+                                          float scale_log2) {
+    return (tok_ok && !(hide_low && n < G)) ? __uint_as_float(raw) * scale_log2 : -INFINITY;
+}
+
+// P = 2^(score - m) in bf16 into this thread's P^T row (MN-major, 32B/64B-swizzled);
+// ps receives the rounded probabilities.
+template <int NQ>
+__device__ __forceinline__ void write_p(const uint32_t (&sv)[NQ], const float (&mu)[NQ],
+                                        float (&ps)[NQ], bool tok_ok, bool hide_low, int G,
+                                        float scale_log2, uint8_t *pbuf, int tok) {
+#pragma unroll
+    for (int n = 0; n < NQ; n += 8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            const float x0 = score_of(sv[n + e], n + e, tok_ok, hide_low, G, scale_log2);
+            const float x1 = score_of(sv[n + e + 1], n + e + 1, tok_ok, hide_low, G, scale_log2);
+            const float m0 = mu[n + e] == -INFINITY ? 0.0f : mu[n + e];
+            const float m1 = mu[n + e + 1] == -INFINITY ? 0.0f : mu[n + e + 1];
+            const float p0 = x0 == -INFINITY ? 0.0f : exp2f(x0 - m0);
+            const float p1 = x1 == -INFINITY ? 0.0f : exp2f(x1 - m1);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            w[e / 2] = *reinterpret_cast<uint32_t *>(&h2);
+            const float2 back = __bfloat1622float2(h2);
+            ps[n + e] = back.x;
+            ps[n + e + 1] = back.y;
+        }
+        *reinterpret_cast<uint4 *>(pbuf + swz(tok * NQ * 2 + n * 2, NQ * 2)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
 }
 
 template <int NQ>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap kv_map,
-                         const __grid_constant__ CUtensorMap kr_map, const GqaParams p) {
+                         const __grid_constant__ CUtensorMap kr_map,
+                         const __grid_constant__ CUtensorMap q_map, const GqaParams p) {
     using SM = GqaSmem<NQ>;
-    constexpr int S = SM::kStages;
+    constexpr int KS = SM::kKSlots, VS = SM::kVSlots;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::oBar);
-    uint64_t *full = bars, *empty = bars + S;
-    uint64_t *kr_full = bars + 2 * S, *kr_empty = kr_full + 2;
-    uint64_t *s_full = kr_empty + 2, *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2, *p_free = p_full + 2;
-    uint64_t *q_full = p_free + 2, *o_done = q_full + 1, *drain = o_done + 1;
+    uint64_t *k_full = bars, *k_empty = bars + KS;
+    uint64_t *v_full = bars + 2 * KS, *v_empty = v_full + VS;
+    uint64_t *kr_full = v_empty + VS, *kr_empty = kr_full + 2;
+    uint64_t *s_full = kr_empty + 2, *s_free = s_full + 4;
+    uint64_t *p_free = s_free + 4, *o_done = p_free + 2;
+    uint64_t *drain = o_done + 2;
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(smem + SM::oMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::oMisc + 4);
     int *plan = reinterpret_cast<int *>(smem + SM::oMisc + 8);
-    float *red = reinterpret_cast<float *>(smem + SM::oRed);
-    float *mrun = reinterpret_cast<float *>(smem + SM::oMrun);
-    float *lw = reinterpret_cast<float *>(smem + SM::oLw);
+    GQLA_PROF_DECL;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
+    const int real_cols = p.G * p.s_q;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < KS; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+        for (int i = 0; i < VS; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&kr_full[i], 1); mbar_init(&kr_empty[i], 1);
-            mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128);
-            mbar_init(&p_full[i], 128); mbar_init(&p_free[i], 1);
+            mbar_init(&p_free[i], 1); mbar_init(&o_done[i], 1);
         }
-        mbar_init(q_full, 128);
-        mbar_init(o_done, 1);
+        for (int i = 0; i < 4; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128); }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -170,126 +295,173 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
         tc_fence_before();
     }
+    if (real_cols < NQ) {  // q rows past G*s_q are never written by TMA: zero them once
+        const int pad = NQ - real_cols;
+        for (int i = threadIdx.x; i < KS * 3 * pad * 8; i += kThreads) {
+            const int slot = i / (3 * pad * 8), rem = i % (3 * pad * 8);
+            const int blk = rem / (pad * 8), rr = rem % (pad * 8);
+            *reinterpret_cast<uint4 *>(smem + SM::oK + slot * SM::kKSlotBytes + SM::kKBytes +
+                                       blk * NQ * 128 + (real_cols + rr / 8) * 128 + (rr % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_smem;
-    const uint32_t t_s = tmem;            // S^T buffers: columns [0, 2 NQ), M = 64 layout
-    const uint32_t t_o = tmem + 2 * NQ;   // O^T_g: columns [2 NQ + g NQ, ...), all 128 lanes
-    PieceIter it0{plan[2], plan[3], plan[0], plan[1]};
+    const uint32_t t_s = tmem;            // S^T buffers: 4 x NQ columns, one token per lane
+    const uint32_t t_o = tmem + 4 * NQ;   // O^T_g: NQ columns per group, one dv per lane
+    const PieceIter it0{plan[2], plan[3], plan[0], plan[1]};
 
-    const uint32_t sm_stage = smem_u32(smem + SM::oStage);
+    const uint32_t sm_k = smem_u32(smem + SM::oK);
+    const uint32_t sm_v = smem_u32(smem + SM::oV);
     const uint32_t sm_kr = smem_u32(smem + SM::oKr);
-    const uint32_t sm_q = smem_u32(smem + SM::oQ);
     const uint32_t sm_p = smem_u32(smem + SM::oP);
-    constexpr int kPStride = ((SM::kPBytes + 1023) / 1024) * 1024;
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             prefetch_tensormap(&kv_map);
             prefetch_tensormap(&kr_map);
-            PieceIter it = it0;
-            int b, L, pb, pe;
-            bool too_long;
-            uint32_t j = 0, pc = 0;
-            while (next_piece(p, it, b, L, pb, pe, too_long)) {
-                if (too_long) { report_error(p.ws, GQLA_ERR_DEVICE, b); continue; }
-                for (int pg = pb; pg < pe; ++pg, ++pc) {
-                    const int page = p.page_table[(int64_t)b * p.max_pages + pg];
-                    const bool bad = page < 0 || page >= p.num_pages;
-                    if (bad) report_error(p.ws, GQLA_ERR_DEVICE, b);
-                    const int kb = pc & 1;
-                    if (!mbar_wait(&kr_empty[kb], ((pc >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                    if (!bad && !*abort_flag) {
-                        mbar_arrive_expect_tx(&kr_full[kb], SM::kKrBytes);
-                        tma_load_2d(smem + SM::oKr + kb * SM::kKrBytes, &kr_map, &kr_full[kb], 0, page * kPage);
-                    } else {
-                        mbar_arrive(&kr_full[kb]);
-                    }
-                    for (int gi = 0; gi < 8; ++gi, ++j) {
-                        const int st = j % S;
-                        if (!mbar_wait(&empty[st], ((j / S) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                        uint8_t *dst = smem + SM::oStage + st * SM::kStageBytes;
-                        if (!bad && !*abort_flag) {
-                            mbar_arrive_expect_tx(&full[st], SM::kStageBytes);
-#pragma unroll
-                            for (int box = 0; box < 4; ++box)
-                                tma_load_3d(dst + box * kKvBox, &kv_map, &full[st], box * 64, page * kPage, gi);
-                        } else {
-                            mbar_arrive(&full[st]);
+            prefetch_tensormap(&q_map);
+            {
+                PieceIter it = it0;
+                int b, L, pb, pe;
+                bool too_long;
+                while (next_piece(p, it, b, L, pb, pe, too_long))
+                    if (too_long) report_error(p.ws, GQLA_ERR_DEVICE, b);
+            }
+            const uint32_t q_bytes = 3u * 128u * (uint32_t)real_cols;
+            UnitCursor kc, vc;
+            kc.start(p, it0);
+            vc.start(p, it0);
+            uint32_t kpos = 0, vpos = 0, pc = 0;
+            // Issue whichever load has a free slot: q_g + K_g as far ahead as their ring
+            // allows (with the pair's RoPE keys before its first group), V_g never ahead of K_g.
+            long long idle_since = clock64();
+            while (kc.valid || vc.valid) {
+                bool progressed = false;
+                if (kc.valid && !*abort_flag) {
+                    const int ks = kpos % KS, kb = pc & 1;
+                    const bool need_kr = kc.gi == 0;
+                    if ((!need_kr || mbar_test_wait(&kr_empty[kb], ((pc >> 1) & 1) ^ 1)) &&
+                        mbar_test_wait(&k_empty[ks], ((kpos / KS) & 1) ^ 1)) {
+                        const PagePair &pp = kc.pp;
+                        const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                        if (need_kr) {
+                            if (pp.bad) report_error(p.ws, GQLA_ERR_DEVICE, kc.b);
+                            uint8_t *dst = smem + SM::oKr + kb * SM::kKrBytes;
+                            if (np) {
+                                mbar_arrive_expect_tx(&kr_full[kb], np * kBox);
+                                if (pp.page0 >= 0) tma_load_2d(dst, &kr_map, &kr_full[kb], 0, pp.page0 * kPage);
+                                if (pp.page1 >= 0)
+                                    tma_load_2d(dst + kBox, &kr_map, &kr_full[kb], 0, pp.page1 * kPage);
+                            } else {
+                                mbar_arrive(&kr_full[kb]);
+                            }
+                            ++pc;
                         }
+                        uint8_t *dst = smem + SM::oK + ks * SM::kKSlotBytes;
+                        mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
+#pragma unroll
+                        for (int cb = 0; cb < 3; ++cb)  // q_g rows (s, hg) of this sequence
+                            tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
+                                        kc.gi * p.G, kc.b * p.s_q);
+#pragma unroll
+                        for (int cb = 0; cb < 2; ++cb) {  // K_nope lo / hi: page 0 rows, then page 1 rows
+                            if (pp.page0 >= 0)
+                                tma_load_3d(dst + cb * 2 * kBox, &kv_map, &k_full[ks], cb * 64,
+                                            pp.page0 * kPage, kc.gi);
+                            if (pp.page1 >= 0)
+                                tma_load_3d(dst + cb * 2 * kBox + kBox, &kv_map, &k_full[ks], cb * 64,
+                                            pp.page1 * kPage, kc.gi);
+                        }
+                        kc.advance(p);
+                        ++kpos;
+                        progressed = true;
                     }
+                }
+                if (vc.valid && vpos < kpos && !*abort_flag) {
+                    const int vs = vpos % VS;
+                    if (mbar_test_wait(&v_empty[vs], ((vpos / VS) & 1) ^ 1)) {
+                        const PagePair &pp = vc.pp;
+                        const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                        uint8_t *dst = smem + SM::oV + vs * SM::kVBytes;
+                        if (np) {
+                            mbar_arrive_expect_tx(&v_full[vs], np * 2 * kBox);
+#pragma unroll
+                            for (int cb = 0; cb < 2; ++cb) {
+                                if (pp.page0 >= 0)
+                                    tma_load_3d(dst + cb * 2 * kBox, &kv_map, &v_full[vs], 128 + cb * 64,
+                                                pp.page0 * kPage, vc.gi);
+                                if (pp.page1 >= 0)
+                                    tma_load_3d(dst + cb * 2 * kBox + kBox, &kv_map, &v_full[vs],
+                                                128 + cb * 64, pp.page1 * kPage, vc.gi);
+                            }
+                        } else {
+                            mbar_arrive(&v_full[vs]);
+                        }
+                        vc.advance(p);
+                        ++vpos;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    idle_since = clock64();
+                } else if (!*abort_flag && clock64() - idle_since <= kWaitCycles) {
+                    __nanosleep(20);
+                } else {
+                    *abort_flag = 1;  // give up: the consumers stop waiting on us as well
+                    break;
                 }
             }
             // never leave with copies in flight: wait (bounded) for the last loads issued
-            for (uint32_t u = (j > (uint32_t)S ? j - S : 0); u < j; ++u) {
-                int dummy = 0;
-                mbar_wait(&full[u % S], (u / S) & 1, reinterpret_cast<volatile int *>(&dummy));
-            }
+            int dummy = 0;
+            volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
+            for (uint32_t u = (kpos > (uint32_t)KS ? kpos - KS : 0); u < kpos; ++u)
+                mbar_wait(&k_full[u % KS], (u / KS) & 1, no_abort);
+            for (uint32_t u = (vpos > (uint32_t)VS ? vpos - VS : 0); u < vpos; ++u)
+                mbar_wait(&v_full[u % VS], (u / VS) & 1, no_abort);
+            for (uint32_t u = (pc > 2u ? pc - 2 : 0); u < pc; ++u)
+                mbar_wait(&kr_full[u & 1], (u >> 1) & 1, no_abort);
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
+        // ---------------------------------------------------------------- score MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16(64, NQ, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16(128, NQ, 1, 1);
-            constexpr uint32_t p_sw = NQ == 16 ? kSw32 : kSw64;
-            constexpr uint32_t p_sbo = NQ == 16 ? 256 : 512;
+            constexpr uint32_t idesc_s = idesc_bf16(kTok, NQ, 0, 0);
             PieceIter it = it0;
             int b, L, pb, pe;
             bool too_long;
-            uint32_t j = 0, pc = 0, k = 0;
-            auto issue_pv = [&](uint32_t u, bool first) {
-                const int buf = u & 1;
-                if (!mbar_wait(&p_full[buf], (u >> 1) & 1, abort_flag)) *abort_flag = 1;
-                tc_fence_after();
-                const int gi = u % 8;
-                const uint32_t v_lo = sm_stage + (u % S) * SM::kStageBytes + 2 * kKvBox;
-                const uint32_t pbuf = sm_p + buf * kPStride;
-                if (!*abort_flag) {
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        uint64_t ad = smem_desc(v_lo + ks * 2048, kKvBox, 1024, kSw128);
-                        uint64_t bd = smem_desc(pbuf + ks * 16 * NQ * 2, SM::kPBytes, p_sbo, p_sw);
-                        mma_bf16(t_o + gi * NQ, ad, bd, idesc_pv, (first && ks == 0) ? 0u : 1u);
-                    }
-                }
-                mma_commit(&p_free[buf]);
-                mma_commit(&empty[u % S]);
-            };
+            uint32_t u = 0, pc = 0;
             while (next_piece(p, it, b, L, pb, pe, too_long)) {
                 if (too_long) continue;
-                if (!mbar_wait(q_full, k & 1, abort_flag)) *abort_flag = 1;
-                tc_fence_after();
-                const uint32_t j0 = j;
-                for (int pg = pb; pg < pe; ++pg, ++pc) {
+                for (int pg = pb; pg < pe; pg += 2, ++pc) {
                     const int kb = pc & 1;
-                    if (!mbar_wait(&kr_full[kb], (pc >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(2, &kr_full[kb], (pc >> 1) & 1, abort_flag)) *abort_flag = 1;
                     const uint32_t kr = sm_kr + kb * SM::kKrBytes;
-                    for (int gi = 0; gi < 8; ++gi, ++j) {
-                        const int st = j % S, buf = j & 1;
-                        if (!mbar_wait(&full[st], (j / S) & 1, abort_flag)) *abort_flag = 1;
-                        if (!mbar_wait(&s_free[buf], ((j >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    for (int gi = 0; gi < 8; ++gi, ++u) {
+                        // S^T(u) = [K_nope_g | k^R] q_g^T into S buffer u & 3
+                        const int ks_ = u % KS, sb = u & 3;
+                        if (!GQLA_WAIT(3, &k_full[ks_], (u / KS) & 1, abort_flag)) *abort_flag = 1;
+                        if (!GQLA_WAIT(4, &s_free[sb], ((u >> 2) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                         tc_fence_after();
-                        const uint32_t kst = sm_stage + st * SM::kStageBytes;
-                        const uint32_t qg = sm_q + gi * NQ * 128;
+                        const uint32_t kst = sm_k + ks_ * SM::kKSlotBytes;
+                        const uint32_t qg = kst + SM::kKBytes;
                         if (!*abort_flag) {
 #pragma unroll
                             for (int ks = 0; ks < 12; ++ks) {
-                                const uint32_t a = ks < 8 ? kst + (ks >> 2) * kKvBox + (ks & 3) * 32
+                                const uint32_t a = ks < 8 ? kst + (ks >> 2) * 2 * kBox + (ks & 3) * 32
                                                           : kr + (ks - 8) * 32;
-                                const uint32_t bq = qg + (ks >> 2) * SM::kQBlock + (ks & 3) * 32;
-                                mma_bf16(t_s + buf * NQ, smem_desc(a, 16, 1024, kSw128),
+                                const uint32_t bq = qg + (ks >> 2) * NQ * 128 + (ks & 3) * 32;
+                                mma_bf16(t_s + sb * NQ, smem_desc(a, 16, 1024, kSw128),
                                          smem_desc(bq, 16, 1024, kSw128), idesc_s, ks > 0 ? 1u : 0u);
                             }
                         }
-                        mma_commit(&s_full[buf]);
+                        mma_commit(&s_full[sb]);
+                        mma_commit(&k_empty[ks_]);
                         if (gi == 7) mma_commit(&kr_empty[kb]);
-                        if (j > j0) issue_pv(j - 1, (j - 1 - j0) < 8);
                     }
                 }
-                issue_pv(j - 1, (j - 1 - j0) < 8);
-                mma_commit(o_done);
-                ++k;
             }
             // drain: nothing may still be running when TMEM is freed
             mma_commit(drain);
@@ -297,206 +469,221 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(drain, 0, reinterpret_cast<volatile int *>(&dummy));
         }
     } else {
-        // ---------------------------------------------------------------- softmax + epilogue
-        const int quad = warp & 3;         // TMEM lane quadrant of this warp
-        const int wq = warp - 2;           // 0..3 among the softmax warps
-        const int stid = threadIdx.x - 64; // 0..127
-        const bool has_tok = lane < 16;
-        const int tok_in_tile = 16 * quad + lane;
-        const int dv = 32 * quad + lane;
+        // ---------------------------------------------------------------- softmax, PV, epilogue
+        // Warpgroup wg owns the groups gi = wg, wg + 2, wg + 4, wg + 6 (units of
+        // one parity), so the two warpgroups never share a group.
+        constexpr uint32_t idesc_pv = idesc_bf16(128, NQ, 1, 1);
+        constexpr uint32_t p_sw = NQ == 16 ? kSw32 : kSw64;
+        constexpr uint32_t p_sbo = NQ == 16 ? 256 : 512;
+        const int wg = (warp - 2) >> 2;        // 0 or 1
+        const int wq = (warp - 2) & 3;         // warp within the warpgroup
+        const int quad = warp & 3;             // TMEM lane quadrant of this warp
+        const int wtid = (threadIdx.x - 64) & 127;
+        const int tok = 32 * quad + lane;      // this thread's token row in a unit (and dv row of O^T)
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        const int real_cols = p.G * p.s_q;
-        uint8_t *qsm = smem + SM::oQ;
+        float *red = reinterpret_cast<float *>(smem + SM::oRed) + wg * NQ * 4;
+        float *mrun = reinterpret_cast<float *>(smem + SM::oMrun);
+        float *lred = reinterpret_cast<float *>(smem + SM::oLred);
+        uint8_t *pbuf = smem + SM::oP + wg * SM::kPBytes;
+        const uint32_t pa = sm_p + wg * SM::kPBytes;
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
         uint32_t j = 0, k = 0;
         while (next_piece(p, it, b, L, pb, pe, too_long)) {
             if (too_long) continue;
-            // ---- q rows of all groups, 128B-swizzled K-major (rows gi*NQ + n), zero padding rows
-            for (int i = stid; i < 8 * NQ * 24; i += 128) {
-                const int R = i / 24, ch = i % 24;
-                const int gi = R / NQ, n = R % NQ;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (n < real_cols) {
-                    const int s = n / p.G, hg = n % p.G;
-                    v = *reinterpret_cast<const uint4 *>(
-                        p.q + (((int64_t)b * p.s_q + s) * p.heads + gi * p.G + hg) * kQk + ch * 8);
-                }
-                *reinterpret_cast<uint4 *>(qsm + (ch >> 3) * SM::kQBlock + swz(R * 128 + (ch & 7) * 16, 128)) = v;
-            }
-            for (int i = lane; i < 8 * NQ; i += 32) lw[(wq * 8) * NQ + i] = 0.0f;
-            fence_proxy_async_smem();
-            mbar_arrive(q_full);
-
-            const int np = pe - pb;
-            for (int ip = 0; ip < np; ++ip) {
-                const int pg = pb + ip;
-                const int page = p.page_table[(int64_t)b * p.max_pages + pg];
-                const bool bad = page < 0 || page >= p.num_pages;
-                const int n_valid = bad ? 0 : min(kPage, L - pg * kPage);
-                const int tok = pg * kPage + tok_in_tile;
-                const bool tok_ok = has_tok && tok_in_tile < n_valid;
-                const float *mold_row = mrun + ((ip & 1) ^ 1) * 8 * NQ;
-                float *mnew_row = mrun + (ip & 1) * 8 * NQ;
-                for (int gi = 0; gi < 8; ++gi, ++j) {
-                    const int buf = j & 1;
-                    // scores of this warp's 16 tokens
-                    if (!mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag)) *abort_flag = 1;
+            const int npairs = (pe - pb + 1) >> 1;
+            for (int ip = 0; ip < npairs; ++ip) {
+                const int pg = pb + 2 * ip;
+                const PagePair pp = load_pair(p, b, L, pg, pe);
+                const bool tok_ok = tok < 64 ? tok < pp.rows0 : tok - 64 < pp.rows1;
+                const bool partial = pp.rows0 < 64 || pp.rows1 < 64;
+                // query s sees token t iff t <= L - s_q + s; columns are n = s*G + hg, so with
+                // s_q <= 2 only the last token can be hidden, and only from columns n < G
+                const bool hide_low = pg * kPage + tok - (L - p.s_q) > 0;
+#pragma unroll 1
+                for (int gl = 0; gl < 4; ++gl) {
+                    const int gi = 2 * gl + wg;
+                    const uint32_t jj = j + ip * 8 + gi;
+                    // lane n (< NQ) keeps the column-n sum over this warp's tokens in shared memory
+                    float *lw = lred + (gi * NQ + (lane & (NQ - 1))) * 4 + wq;
+                    const int sb = jj & 3;
+                    GQLA_SPAN_BEGIN(t_unit);
+                    if (!GQLA_WAIT(6, &s_full[sb], (jj >> 2) & 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
                     uint32_t sv[NQ];
-                    tmem_ld16(t_s + lane_off + buf * NQ, sv);
-                    if constexpr (NQ == 32) tmem_ld16(t_s + lane_off + buf * NQ + 16, sv + 16);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(&s_free[buf]);
-                    // query s sees token t iff t <= L - s_q + s; columns are n = s*G + hg,
-                    // so with s_q <= 2 only the last token can be hidden, from columns n < G
-                    float x[NQ];
-                    const int s_min = tok - (L - p.s_q);
-#pragma unroll
-                    for (int n = 0; n < NQ; ++n) {
-                        const bool vis = tok_ok && (s_min <= 0 || n >= p.G);
-                        x[n] = vis ? __uint_as_float(sv[n]) * p.scale_log2 : -INFINITY;
-                    }
-                    // column maxima over the 64 tokens
-                    {
-                        float t[NQ];
-#pragma unroll
-                        for (int n = 0; n < NQ; ++n) t[n] = x[n];
-                        const float m = transpose_reduce<NQ, true>(t, lane);
-                        if (lane < NQ) red[lane * 4 + wq] = m;
-                    }
-                    named_bar_sync();
-                    float mu[NQ], alpha[NQ];
-                    bool need = false;
+                    GQLA_SPAN_BEGIN(t_ld);
+                    tmem_ld16(t_s + lane_off + sb * NQ, sv);
+                    if constexpr (NQ == 32) tmem_ld16(t_s + lane_off + sb * NQ + 16, sv + 16);
+                    float mu[NQ];
 #pragma unroll
                     for (int n = 0; n < NQ; n += 4) {
-                        float4 m_old4 = ip ? *reinterpret_cast<const float4 *>(mold_row + gi * NQ + n)
-                                           : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-                        const float mo[4] = {m_old4.x, m_old4.y, m_old4.z, m_old4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float4 r4 = *reinterpret_cast<const float4 *>(red + (n + e) * 4);
-                            const float mt = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
-                            const float mn = (mt > mo[e] + kRescaleLog2) ? mt : mo[e];
-                            mu[n + e] = mn;
-                            alpha[n + e] = (mn == mo[e]) ? 1.0f : exp2f(mo[e] - mn);
-                            need |= (ip > 0) && (mn != mo[e]);
-                        }
+                        const float4 m4 = *reinterpret_cast<const float4 *>(mrun + gi * NQ + n);
+                        mu[n] = m4.x; mu[n + 1] = m4.y; mu[n + 2] = m4.z; mu[n + 3] = m4.w;
                     }
-                    if (stid == 0) {
+                    tmem_wait_ld();
+                    GQLA_SPAN_END(11, t_ld);
+                    tc_fence_before();
+                    mbar_arrive(&s_free[sb]);
+                    bool exceed = ip == 0;
 #pragma unroll
-                        for (int n = 0; n < NQ; n += 4)
-                            *reinterpret_cast<float4 *>(mnew_row + gi * NQ + n) =
-                                make_float4(mu[n], mu[n + 1], mu[n + 2], mu[n + 3]);
-                    }
-                    // P^T buffer and O^T_g are free once PV(j - 2) has completed
-                    if (!mbar_wait(&p_free[buf], ((j >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    for (int n = 0; n < NQ; ++n)
+                        exceed |= score_of(sv[n], n, tok_ok, hide_low, p.G, p.scale_log2) > mu[n] + kRescaleLog2;
+                    // the P^T buffer (and O^T_g) are free once this warpgroup's previous PV completed
+                    if (!GQLA_WAIT(7, &p_free[wg], ((jj >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
-                    if (need) {  // uniform across the four warps
-                        const uint32_t to = t_o + gi * NQ + lane_off;
-#pragma unroll
-                        for (int h16 = 0; h16 < NQ; h16 += 16) {
-                            uint32_t r[16];
-                            tmem_ld16(to + h16, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha[h16 + e]);
-                            tmem_st16(to + h16, r);
-                        }
-                        tmem_wait_st();
-                    }
-                    // probabilities (bf16) into P^T, this warp's 16 token rows
                     float ps[NQ];
-                    {
-                        uint8_t *pbuf = smem + SM::oP + buf * kPStride;
-#pragma unroll
-                        for (int n = 0; n < NQ; n += 8) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                const float m0 = mu[n + e] == -INFINITY ? 0.0f : mu[n + e];
-                                const float m1 = mu[n + e + 1] == -INFINITY ? 0.0f : mu[n + e + 1];
-                                const float p0 = x[n + e] == -INFINITY ? 0.0f : exp2f(x[n + e] - m0);
-                                const float p1 = x[n + e + 1] == -INFINITY ? 0.0f : exp2f(x[n + e + 1] - m1);
-                                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                                w[e / 2] = *reinterpret_cast<uint32_t *>(&h2);
-                                const float2 back = __bfloat1622float2(h2);
-                                ps[n + e] = back.x;
-                                ps[n + e + 1] = back.y;
-                            }
-                            if (has_tok)
-                                *reinterpret_cast<uint4 *>(pbuf + swz(tok_in_tile * NQ * 2 + n * 2, NQ * 2)) =
-                                    make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    }
-                    // V rows of tokens past the sequence end (pool rows never written, maybe NaN) -> 0
-                    if (n_valid < kPage) {
-                        const int st = j % S;
-                        if (!mbar_wait(&full[st], (j / S) & 1, abort_flag)) *abort_flag = 1;
-                        uint8_t *vbase = smem + SM::oStage + st * SM::kStageBytes + 2 * kKvBox;
-                        for (int i = stid; i < 2 * (kPage - n_valid) * 8; i += 128) {
-                            const int half = i / ((kPage - n_valid) * 8);
-                            const int rem = i % ((kPage - n_valid) * 8);
-                            const int row = n_valid + rem / 8, ch = rem % 8;
-                            *reinterpret_cast<uint4 *>(vbase + half * kKvBox + row * 128 + ch * 16) =
+                    GQLA_SPAN_BEGIN(t_wp);
+                    if (ip > 0)  // optimistic: P against the running maxima
+                        write_p<NQ>(sv, mu, ps, tok_ok, hide_low, p.G, p.scale_log2, pbuf, tok);
+                    GQLA_SPAN_END(12, t_wp);
+                    const int vs = jj % VS;
+                    if (partial) {  // V rows that are not tokens (never written, maybe NaN) -> 0
+                        if (!GQLA_WAIT(8, &v_full[vs], (jj / VS) & 1, abort_flag)) *abort_flag = 1;
+                        uint8_t *vbase = smem + SM::oV + vs * SM::kVBytes;
+                        const int n0 = 64 - pp.rows0, n1 = 64 - pp.rows1;
+                        for (int i = wtid; i < 2 * (n0 + n1) * 8; i += 128) {
+                            const int cb = i / ((n0 + n1) * 8), rem = i % ((n0 + n1) * 8);
+                            const int r = rem / 8;
+                            const int row = r < n0 ? pp.rows0 + r : 64 + pp.rows1 + (r - n0);
+                            *reinterpret_cast<uint4 *>(vbase + cb * 2 * kBox + row * 128 + (rem % 8) * 16) =
                                 make_uint4(0, 0, 0, 0);
                         }
                     }
+                    GQLA_SPAN_BEGIN(t_fence);
                     fence_proxy_async_smem();
                     tc_fence_before();
-                    mbar_arrive(&p_full[buf]);
-                    // column sums of the rounded probabilities, per warp (lane n holds column n)
-                    {
-                        const float l = transpose_reduce<NQ, false>(ps, lane);
-                        if (lane < NQ) {
-                            float *slot = lw + (wq * 8 + gi) * NQ + lane;
-                            const float mo = ip ? mold_row[gi * NQ + lane] : -INFINITY;
+                    GQLA_SPAN_END(15, t_fence);
+                    GQLA_SPAN_BEGIN(t_vote);
+                    const bool slow = wg_bar_any(wg, exceed);
+                    GQLA_SPAN_END(9, t_vote);
+                    if (slow) {  // uniform over the warpgroup: new column maxima for this tile
+                        GQLA_SPAN_BEGIN(t_slow);
+                        {
+                            float t[NQ];
+#pragma unroll
+                            for (int n = 0; n < NQ; ++n) t[n] = score_of(sv[n], n, tok_ok, hide_low, p.G, p.scale_log2);
+                            const float m = column_reduce32<NQ, true>(t, lane);
+                            if (lane < NQ) red[lane * 4 + wq] = m;
+                        }
+                        wg_bar(wg);
+                        bool need = false;
+#pragma unroll
+                        for (int n = 0; n < NQ; ++n) {
+                            const float4 r4 = *reinterpret_cast<const float4 *>(red + n * 4);
+                            const float mt = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
+                            const float mn = ip == 0 ? mt : ((mt > mu[n] + kRescaleLog2) ? mt : mu[n]);
+                            need |= ip > 0 && mn != mu[n];
+                            mu[n] = mn;
+                        }
+                        tc_fence_after();
+                        if (need) {  // O^T_g columns *= 2^(m_old - m_new)
+                            const uint32_t to = t_o + gi * NQ + lane_off;
+#pragma unroll
+                            for (int h16 = 0; h16 < NQ; h16 += 16) {
+                                uint32_t r[16];
+                                tmem_ld16(to + h16, r);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) {
+                                    const float mold = mrun[gi * NQ + h16 + e];
+                                    const float a = mold == mu[h16 + e] ? 1.0f : exp2f(mold - mu[h16 + e]);
+                                    r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
+                                }
+                                tmem_st16(to + h16, r);
+                            }
+                            tmem_wait_st();
+                        }
+                        if (lane < NQ) {  // this lane's own column partial follows the same rescale
                             const float4 r4 = *reinterpret_cast<const float4 *>(red + lane * 4);
                             const float mt = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
-                            const float mn = (mt > mo + kRescaleLog2) ? mt : mo;
-                            const float a = (mn == mo || ip == 0) ? 1.0f : exp2f(mo - mn);
-                            *slot = (ip ? *slot * a : 0.0f) + l;
+                            const float mold = mrun[gi * NQ + lane];
+                            const float mn = ip == 0 ? mt : ((mt > mold + kRescaleLog2) ? mt : mold);
+                            *lw = ip == 0 ? 0.0f : (mn == mold ? *lw : *lw * exp2f(mold - mn));
                         }
+                        write_p<NQ>(sv, mu, ps, tok_ok, hide_low, p.G, p.scale_log2, pbuf, tok);
+                        fence_proxy_async_smem();
+                        tc_fence_before();
+                        wg_bar(wg);  // P^T complete; everyone has read mrun / red
+                        if (wtid == 0) {
+#pragma unroll
+                            for (int n = 0; n < NQ; n += 4)
+                                *reinterpret_cast<float4 *>(mrun + gi * NQ + n) =
+                                    make_float4(mu[n], mu[n + 1], mu[n + 2], mu[n + 3]);
+                        }
+                        GQLA_SPAN_END(17, t_slow);
                     }
-                    named_bar_sync();  // red[] is rewritten by the next unit
+                    if (wtid == 0) {  // O^T_g (+)= V_g^T P^T
+                        if (!GQLA_WAIT(13, &v_full[vs], (jj / VS) & 1, abort_flag)) *abort_flag = 1;
+                        tc_fence_after();
+                        const uint32_t v_lo = sm_v + vs * SM::kVBytes;
+                        if (!*abort_flag) {
+#pragma unroll
+                            for (int ks = 0; ks < kTok / 16; ++ks) {
+                                uint64_t ad = smem_desc(v_lo + ks * 2048, 2 * kBox, 1024, kSw128);
+                                uint64_t bd = smem_desc(pa + ks * 16 * NQ * 2, SM::kPBytes, p_sbo, p_sw);
+                                mma_bf16(t_o + gi * NQ, ad, bd, idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
+                            }
+                        }
+                        mma_commit(&p_free[wg]);
+                        mma_commit(&v_empty[vs]);
+                    }
+                    // column sums of the rounded probabilities over this warp's tokens
+                    GQLA_SPAN_BEGIN(t_sum);
+                    {
+                        const float l = column_reduce32<NQ, false>(ps, lane);
+                        if (lane < NQ) *lw += l;
+                    }
+                    GQLA_SPAN_END(16, t_sum);
+                    GQLA_SPAN_END(10, t_unit);
                 }
             }
+            j += npairs * 8;
+            GQLA_SPAN_BEGIN(t_epi);
             // ---- epilogue: normalise O^T and write the partials of slot b + c
-            if (!mbar_wait(o_done, k & 1, abort_flag)) *abort_flag = 1;
+            if (wtid == 0) mma_commit(&o_done[wg]);
+            if (!GQLA_WAIT(14, &o_done[wg], k & 1, abort_flag)) *abort_flag = 1;
             tc_fence_after();
-            named_bar_sync();
-            const float *mfin = mrun + ((np - 1) & 1) * 8 * NQ;
+            wg_bar(wg);
             const int slot = b + c;
-            for (int gi = 0; gi < 8; ++gi) {
+            const int dv = tok;
+#pragma unroll 1
+            for (int gl = 0; gl < 4; ++gl) {
+                const int gi = 2 * gl + wg;
                 uint32_t r[NQ];
+                GQLA_SPAN_BEGIN(t_eld);
                 tmem_ld16(t_o + gi * NQ + lane_off, r);
                 if constexpr (NQ == 32) tmem_ld16(t_o + gi * NQ + lane_off + 16, r + 16);
                 tmem_wait_ld();
+                GQLA_SPAN_END(18, t_eld);
+                GQLA_SPAN_BEGIN(t_est);
 #pragma unroll
                 for (int n = 0; n < NQ; ++n) {
                     if (n >= real_cols) break;
-                    const float l = lw[(0 * 8 + gi) * NQ + n] + lw[(1 * 8 + gi) * NQ + n] +
-                                    lw[(2 * 8 + gi) * NQ + n] + lw[(3 * 8 + gi) * NQ + n];
-                    const int s = n / p.G, hg = n % p.G;
+                    const float4 l4 = *reinterpret_cast<const float4 *>(lred + (gi * NQ + n) * 4);
+                    const float l = (l4.x + l4.y) + (l4.z + l4.w);
+                    const int s = n / p.G, hg = n - s * p.G;
                     const int64_t row = ((int64_t)slot * p.s_q + s) * p.heads + gi * p.G + hg;
                     p.o_part[row * kDv + dv] = l > 0.0f ? __uint_as_float(r[n]) / l : 0.0f;
-                    if (stid == 0) {
-                        const float m = mfin[gi * NQ + n];
+                    if (wtid == n) {
+                        const float m = mrun[gi * NQ + n];
                         p.lse_part[row] = (l > 0.0f && m != -INFINITY)
                                               ? (m + __log2f(l)) * 0.6931471805599453f
                                               : -INFINITY;
                     }
                 }
+                GQLA_SPAN_END(19, t_est);
             }
             tc_fence_before();
-            named_bar_sync();
+            GQLA_SPAN_BEGIN(t_ebar);
+            wg_bar(wg);  // lred / mrun are reused by the next piece
+            GQLA_SPAN_END(20, t_ebar);
+            GQLA_SPAN_END(21, t_epi);
             ++k;
         }
     }
 
+    GQLA_PROF_FLUSH;
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) report_error(p.ws, GQLA_ERR_TIMEOUT, c);
     if (warp == 1) {
@@ -535,13 +722,13 @@ bool make_map(CUtensorMap *map, const void *base, int rank, const cuuint64_t *di
 }
 
 template <int NQ>
-cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const GqaParams &p,
-                      cudaStream_t stream) {
+cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const CUtensorMap &qm,
+                      const GqaParams &p, cudaStream_t stream) {
     const int bytes = GqaSmem<NQ>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(decode_gqa_tc_kernel<NQ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    decode_gqa_tc_kernel<NQ><<<p.num_splits, kThreads, bytes, stream>>>(kvm, krm, p);
+    decode_gqa_tc_kernel<NQ><<<p.num_splits, kThreads, bytes, stream>>>(kvm, krm, qm, p);
     return cudaGetLastError();
 }
 
@@ -552,7 +739,8 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
                               int num_splits, float scale, float *o_part, float *lse_part,
                               void *ws, cudaStream_t stream) {
     if (num_groups != 8) return cudaErrorInvalidValue;
-    CUtensorMap kvm, krm;
+    const int G = heads / num_groups;
+    CUtensorMap kvm, krm, qm;
     {
         cuuint64_t dims[3] = {256, (cuuint64_t)num_slots, 8};
         cuuint64_t strides[2] = {256 * 2, (cuuint64_t)num_slots * 256 * 2};
@@ -565,8 +753,13 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
         cuuint32_t box[2] = {64, 64};
         if (!make_map(&krm, k_rope, 2, dims, strides, box)) return cudaErrorInvalidValue;
     }
+    {  // q [batch * s_q][heads][192]: a box is the G heads of one group for all s_q tokens
+        cuuint64_t dims[3] = {(cuuint64_t)kQk, (cuuint64_t)heads, (cuuint64_t)idx->batch * s_q};
+        cuuint64_t strides[2] = {(cuuint64_t)kQk * 2, (cuuint64_t)heads * kQk * 2};
+        cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)s_q};
+        if (!make_map(&qm, q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
     GqaParams p;
-    p.q = static_cast<const __nv_bfloat16 *>(q);
     p.page_table = idx->page_table;
     p.seqlens = idx->seqlens;
     p.o_part = o_part;
@@ -578,9 +771,10 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
     p.num_splits = num_splits;
     p.s_q = s_q;
     p.heads = heads;
-    p.G = heads / num_groups;
+    p.G = G;
     p.scale_log2 = scale * kLog2e;
-    return p.G * s_q <= 16 ? launch_nq<16>(kvm, krm, p, stream) : launch_nq<32>(kvm, krm, p, stream);
+    return G * s_q <= 16 ? launch_nq<16>(kvm, krm, qm, p, stream)
+                         : launch_nq<32>(kvm, krm, qm, p, stream);
 }
 
 }  // namespace gqla

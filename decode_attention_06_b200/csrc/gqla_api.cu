@@ -58,13 +58,21 @@ int check_workspace(const void *ws, size_t bytes) {
     return GQLA_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return GQLA_OK;
+    g_last_cuda_error = e;
+    return GQLA_ERR_CUDA;
+}
 
 }  // namespace
 
 extern "C" {
 
 int gqla_version(void) { return 1; }
+
+const char *gqla_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char *gqla_status_string(int status) {
     switch (status) {

@@ -46,6 +46,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // About two seconds at B200 clocks: a wait that takes longer is a bug, and
 // the kernel gives up instead of hanging the GPU.
 constexpr long long kWaitCycles = 4000000000LL;
@@ -61,6 +74,54 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (clock64() - t0 > kWaitCycles) return false;
     }
 }
+
+// Wait-site profiling hook: compiled to the plain bounded wait unless the
+// translation unit defines GQLA_WAIT_PROFILE (a diagnostic build), in which
+// case each thread accumulates the cycles spent per numbered site in
+// registers and lane 0 of every warp adds them to a global table at exit.
+#ifdef GQLA_WAIT_PROFILE
+__device__ unsigned long long g_wait_cycles[32];
+__device__ unsigned long long g_wait_count[32];
+// per-warp accumulators in shared memory (lane 0 of each warp writes its own row)
+#define GQLA_PROF_DECL                                                       \
+    __shared__ unsigned long long gqla_prof_c_[16][24];                     \
+    __shared__ unsigned int gqla_prof_n_[16][24];                           \
+    if ((threadIdx.x & 31) == 0)                                            \
+        for (int i_ = 0; i_ < 24; ++i_)                                     \
+            gqla_prof_c_[threadIdx.x >> 5][i_] = 0, gqla_prof_n_[threadIdx.x >> 5][i_] = 0
+#define GQLA_PROF_ADD(site, dt)                                              \
+    do {                                                                     \
+        if ((threadIdx.x & 31) == 0) {                                       \
+            gqla_prof_c_[threadIdx.x >> 5][site] += (dt);                    \
+            gqla_prof_n_[threadIdx.x >> 5][site] += 1;                       \
+        }                                                                    \
+    } while (0)
+#define GQLA_WAIT(site, bar, parity, abort)                                  \
+    ({                                                                       \
+        const long long t0_ = clock64();                                     \
+        const bool ok_ = ::gqla::sm100::mbar_wait(bar, parity, abort);       \
+        GQLA_PROF_ADD(site, clock64() - t0_);                                \
+        ok_;                                                                 \
+    })
+#define GQLA_SPAN_BEGIN(v) const long long v = clock64()
+#define GQLA_SPAN_END(site, v) GQLA_PROF_ADD(site, clock64() - v)
+#define GQLA_PROF_FLUSH                                                                     \
+    do {                                                                                    \
+        if ((threadIdx.x & 31) == 0)                                                        \
+            for (int i_ = 0; i_ < 24; ++i_)                                                 \
+                if (gqla_prof_n_[threadIdx.x >> 5][i_]) {                                   \
+                    atomicAdd(&::gqla::sm100::g_wait_cycles[i_], gqla_prof_c_[threadIdx.x >> 5][i_]); \
+                    atomicAdd(&::gqla::sm100::g_wait_count[i_],                             \
+                              (unsigned long long)gqla_prof_n_[threadIdx.x >> 5][i_]);      \
+                }                                                                           \
+    } while (0)
+#else
+#define GQLA_PROF_DECL (void)0
+#define GQLA_WAIT(site, bar, parity, abort) ::gqla::sm100::mbar_wait(bar, parity, abort)
+#define GQLA_SPAN_BEGIN(v) (void)0
+#define GQLA_SPAN_END(site, v) (void)0
+#define GQLA_PROF_FLUSH (void)0
+#endif
 
 // ------------------------------------------------------------------ TMA
 

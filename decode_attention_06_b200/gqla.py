@@ -35,7 +35,10 @@ STATUS = {0: "GQLA_OK", -1: "GQLA_ERR_INVALID_ARG", -2: "GQLA_ERR_UNSUPPORTED",
 class GqlaError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} returned {status} ({STATUS.get(status, '?')})")
+        extra = ""
+        if status == -4:
+            extra = ": " + _lib.gqla_last_cuda_error().decode()
+        super().__init__(f"{fn} returned {status} ({STATUS.get(status, '?')}){extra}")
 
 
 class gqla_dims(ctypes.Structure):
@@ -66,6 +69,7 @@ _SIGS = {
     "gqla_read_device_error": [_P, ctypes.POINTER(ctypes.c_int), _P],
     "gqla_clear_device_error": [_P, _P],
     "gqla_status_string": [_I],
+    "gqla_last_cuda_error": [],
     "gqla_version": [],
 }
 for _name, _args in _SIGS.items():
@@ -74,6 +78,7 @@ for _name, _args in _SIGS.items():
     _f.restype = _I
 _lib.gqla_workspace_bytes.restype = _SZ
 _lib.gqla_status_string.restype = ctypes.c_char_p
+_lib.gqla_last_cuda_error.restype = ctypes.c_char_p
 
 EXPORTED = tuple(_SIGS)
 
@@ -225,6 +230,10 @@ def gqla_clear_device_error(workspace: torch.Tensor, stream=None):
 
 def gqla_status_string(status: int) -> str:
     return _lib.gqla_status_string(status).decode()
+
+
+def gqla_last_cuda_error() -> str:
+    return _lib.gqla_last_cuda_error().decode()
 
 
 def gqla_version() -> int:

@@ -214,6 +214,10 @@ int gqla_clear_device_error(void *workspace, gqla_stream_t stream);
 /* Static description of a status code. */
 const char *gqla_status_string(int status);
 
+/* Description of the CUDA error behind the last GQLA_ERR_CUDA returned on the
+ * calling thread ("no error" if none). */
+const char *gqla_last_cuda_error(void);
+
 /* Library ABI version: 1. */
 int gqla_version(void);
 
