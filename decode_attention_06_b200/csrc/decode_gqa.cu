@@ -45,7 +45,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;        // warp 0 TMA, warp 1 score MMA, warps 2-9: two softmax warpgroups
+constexpr int kThreads = 352;        // warp 0 TMA, warp 1 score MMA, warps 2-9 softmax, warp 10 PV MMA
 constexpr int kTok = 128;            // tokens per unit (two pages)
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kBox = 64 * 64 * 2;    // one 64-row x 64-column bf16 TMA box (8 KB)
@@ -69,9 +69,10 @@ struct GqaSmem {
     static constexpr int oLred = oMrun + 8 * NQ * 4;         // float [8 groups][NQ][4 warps]
     static constexpr int oBar = oLred + 8 * NQ * 4 * 4;
     // k_full/k_empty[KS], v_full/v_empty[VS], kr_full/kr_empty[2], s_full/s_free[4],
-    // p_free[2], o_done[2], drain
-    static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 4 + 8 + 4 + 1;
-    static constexpr int oMisc = oBar + kNumBars * 8;  // tmem base, abort flag, plan[4]
+    // p_full/p_free[2], o_done[2], drain x2
+    static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 4 + 8 + 6 + 2;
+    static constexpr int oEpi = oBar + kNumBars * 8;   // float inv_l[2 wg][NQ], lse[2 wg][NQ]
+    static constexpr int oMisc = oEpi + 4 * NQ * 4;  // tmem base, abort flag, plan[4]
     static constexpr int kBytes = oMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
@@ -259,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *v_full = bars + 2 * KS, *v_empty = v_full + VS;
     uint64_t *kr_full = v_empty + VS, *kr_empty = kr_full + 2;
     uint64_t *s_full = kr_empty + 2, *s_free = s_full + 4;
-    uint64_t *p_free = s_free + 4, *o_done = p_free + 2;
-    uint64_t *drain = o_done + 2;
+    uint64_t *p_full = s_free + 4, *p_free = p_full + 2, *o_done = p_free + 2;
+    uint64_t *drain = o_done + 2;  // [0] score issuer, [1] PV issuer
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(smem + SM::oMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::oMisc + 4);
     int *plan = reinterpret_cast<int *>(smem + SM::oMisc + 8);
@@ -275,10 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < VS; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&kr_full[i], 1); mbar_init(&kr_empty[i], 1);
-            mbar_init(&p_free[i], 1); mbar_init(&o_done[i], 1);
+            mbar_init(&p_full[i], 128); mbar_init(&p_free[i], 1); mbar_init(&o_done[i], 1);
+            mbar_init(&drain[i], 1);
         }
         for (int i = 0; i < 4; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128); }
-        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -464,17 +465,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // drain: nothing may still be running when TMEM is freed
-            mma_commit(drain);
+            mma_commit(&drain[0]);
             int dummy = 0;
-            mbar_wait(drain, 0, reinterpret_cast<volatile int *>(&dummy));
+            mbar_wait(&drain[0], 0, reinterpret_cast<volatile int *>(&dummy));
+        }
+    } else if (warp == 10) {
+        // ---------------------------------------------------------------- PV MMA issuer
+        // O^T_g(u) (+)= V_g^T P^T(u), in unit order, as soon as the owning warpgroup
+        // has published P^T(u) and V_g(u) has landed; no softmax warp waits for V.
+        if (lane == 0) {
+            constexpr uint32_t idesc_pv = idesc_bf16(128, NQ, 1, 1);
+            constexpr uint32_t p_sw = NQ == 16 ? kSw32 : kSw64;
+            constexpr uint32_t p_sbo = NQ == 16 ? 256 : 512;
+            PieceIter it = it0;
+            int b, L, pb, pe;
+            bool too_long;
+            uint32_t u = 0;
+            while (next_piece(p, it, b, L, pb, pe, too_long)) {
+                if (too_long) continue;
+                const int npairs = (pe - pb + 1) >> 1;
+                for (int ip = 0; ip < npairs; ++ip) {
+                    for (int gi = 0; gi < 8; ++gi, ++u) {
+                        const int w = gi & 1, vs = u % VS;
+                        if (!GQLA_WAIT(5, &p_full[w], (u >> 1) & 1, abort_flag)) *abort_flag = 1;
+                        if (!GQLA_WAIT(13, &v_full[vs], (u / VS) & 1, abort_flag)) *abort_flag = 1;
+                        tc_fence_after();
+                        const uint32_t v_lo = sm_v + vs * SM::kVBytes;
+                        const uint32_t pa = sm_p + w * SM::kPBytes;
+                        if (!*abort_flag) {
+#pragma unroll
+                            for (int ks = 0; ks < kTok / 16; ++ks) {
+                                uint64_t ad = smem_desc(v_lo + ks * 2048, 2 * kBox, 1024, kSw128);
+                                uint64_t bd = smem_desc(pa + ks * 16 * NQ * 2, SM::kPBytes, p_sbo, p_sw);
+                                mma_bf16(t_o + gi * NQ, ad, bd, idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
+                            }
+                        }
+                        mma_commit(&p_free[w]);
+                        mma_commit(&v_empty[vs]);
+                    }
+                }
+                mma_commit(&o_done[0]);
+                mma_commit(&o_done[1]);
+            }
+            mma_commit(&drain[1]);
+            int dummy = 0;
+            mbar_wait(&drain[1], 0, reinterpret_cast<volatile int *>(&dummy));
         }
     } else {
         // ---------------------------------------------------------------- softmax, PV, epilogue
         // Warpgroup wg owns the groups gi = wg, wg + 2, wg + 4, wg + 6 (units of
         // one parity), so the two warpgroups never share a group.
-        constexpr uint32_t idesc_pv = idesc_bf16(128, NQ, 1, 1);
-        constexpr uint32_t p_sw = NQ == 16 ? kSw32 : kSw64;
-        constexpr uint32_t p_sbo = NQ == 16 ? 256 : 512;
         const int wg = (warp - 2) >> 2;        // 0 or 1
         const int wq = (warp - 2) & 3;         // warp within the warpgroup
         const int quad = warp & 3;             // TMEM lane quadrant of this warp
@@ -485,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float *mrun = reinterpret_cast<float *>(smem + SM::oMrun);
         float *lred = reinterpret_cast<float *>(smem + SM::oLred);
         uint8_t *pbuf = smem + SM::oP + wg * SM::kPBytes;
-        const uint32_t pa = sm_p + wg * SM::kPBytes;
+        float *inv_l = reinterpret_cast<float *>(smem + SM::oEpi) + wg * 2 * NQ;  // [NQ] 1/l, [NQ] lse
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
@@ -613,21 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         GQLA_SPAN_END(17, t_slow);
                     }
-                    if (wtid == 0) {  // O^T_g (+)= V_g^T P^T
-                        if (!GQLA_WAIT(13, &v_full[vs], (jj / VS) & 1, abort_flag)) *abort_flag = 1;
-                        tc_fence_after();
-                        const uint32_t v_lo = sm_v + vs * SM::kVBytes;
-                        if (!*abort_flag) {
-#pragma unroll
-                            for (int ks = 0; ks < kTok / 16; ++ks) {
-                                uint64_t ad = smem_desc(v_lo + ks * 2048, 2 * kBox, 1024, kSw128);
-                                uint64_t bd = smem_desc(pa + ks * 16 * NQ * 2, SM::kPBytes, p_sbo, p_sw);
-                                mma_bf16(t_o + gi * NQ, ad, bd, idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
-                            }
-                        }
-                        mma_commit(&p_free[wg]);
-                        mma_commit(&v_empty[vs]);
-                    }
+                    mbar_arrive(&p_full[wg]);
                     // column sums of the rounded probabilities over this warp's tokens
                     GQLA_SPAN_BEGIN(t_sum);
                     {
@@ -641,38 +667,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             j += npairs * 8;
             GQLA_SPAN_BEGIN(t_epi);
             // ---- epilogue: normalise O^T and write the partials of slot b + c
-            if (wtid == 0) mma_commit(&o_done[wg]);
             if (!GQLA_WAIT(14, &o_done[wg], k & 1, abort_flag)) *abort_flag = 1;
             tc_fence_after();
-            wg_bar(wg);
+            wg_bar(wg);  // all column partials of this warpgroup are in lred
             const int slot = b + c;
             const int dv = tok;
+            // rows of the partial for columns n = s*G + hg: ((slot*s_q + s)*h + gi*G + hg)
+            const int64_t row_s0 = (int64_t)slot * p.s_q * p.heads;
 #pragma unroll 1
             for (int gl = 0; gl < 4; ++gl) {
                 const int gi = 2 * gl + wg;
+                if (wtid < NQ) {  // per column: 1 / l and the natural-log LSE
+                    const float4 l4 = *reinterpret_cast<const float4 *>(lred + (gi * NQ + wtid) * 4);
+                    const float l = (l4.x + l4.y) + (l4.z + l4.w);
+                    const float m = mrun[gi * NQ + wtid];
+                    const bool ok = l > 0.0f && m != -INFINITY;
+                    inv_l[wtid] = ok ? 1.0f / l : 0.0f;
+                    inv_l[NQ + wtid] = ok ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+                    if (wtid < real_cols) {
+                        const int s = wtid / p.G, hg = wtid - s * p.G;
+                        p.lse_part[row_s0 + (int64_t)s * p.heads + gi * p.G + hg] = inv_l[NQ + wtid];
+                    }
+                }
                 uint32_t r[NQ];
                 GQLA_SPAN_BEGIN(t_eld);
                 tmem_ld16(t_o + gi * NQ + lane_off, r);
                 if constexpr (NQ == 32) tmem_ld16(t_o + gi * NQ + lane_off + 16, r + 16);
                 tmem_wait_ld();
                 GQLA_SPAN_END(18, t_eld);
+                wg_bar(wg);  // inv_l ready
                 GQLA_SPAN_BEGIN(t_est);
+                float *dst = p.o_part + (row_s0 + gi * p.G) * kDv + dv;
+                int s = 0, hg = 0;
 #pragma unroll
                 for (int n = 0; n < NQ; ++n) {
-                    if (n >= real_cols) break;
-                    const float4 l4 = *reinterpret_cast<const float4 *>(lred + (gi * NQ + n) * 4);
-                    const float l = (l4.x + l4.y) + (l4.z + l4.w);
-                    const int s = n / p.G, hg = n - s * p.G;
-                    const int64_t row = ((int64_t)slot * p.s_q + s) * p.heads + gi * p.G + hg;
-                    p.o_part[row * kDv + dv] = l > 0.0f ? __uint_as_float(r[n]) / l : 0.0f;
-                    if (wtid == n) {
-                        const float m = mrun[gi * NQ + n];
-                        p.lse_part[row] = (l > 0.0f && m != -INFINITY)
-                                              ? (m + __log2f(l)) * 0.6931471805599453f
-                                              : -INFINITY;
-                    }
+                    if (n < real_cols)
+                        dst[((int64_t)s * p.heads + hg) * kDv] = __uint_as_float(r[n]) * inv_l[n];
+                    if (++hg == p.G) { hg = 0; ++s; }
                 }
                 GQLA_SPAN_END(19, t_est);
+                wg_bar(wg);  // inv_l is rewritten for the next group
             }
             tc_fence_before();
             GQLA_SPAN_BEGIN(t_ebar);

@@ -84,8 +84,8 @@ __device__ unsigned long long g_wait_cycles[32];
 __device__ unsigned long long g_wait_count[32];
 // per-warp accumulators in shared memory (lane 0 of each warp writes its own row)
 #define GQLA_PROF_DECL                                                       \
-    __shared__ unsigned long long gqla_prof_c_[16][24];                     \
-    __shared__ unsigned int gqla_prof_n_[16][24];                           \
+    __shared__ unsigned long long gqla_prof_c_[11][24];                     \
+    __shared__ unsigned int gqla_prof_n_[11][24];                           \
     if ((threadIdx.x & 31) == 0)                                            \
         for (int i_ = 0; i_ < 24; ++i_)                                     \
             gqla_prof_c_[threadIdx.x >> 5][i_] = 0, gqla_prof_n_[threadIdx.x >> 5][i_] = 0
