@@ -49,8 +49,10 @@ L2_FLUSH_BYTES = 256 << 20
 # Kernel source files whose ncu counters are stored in profiles/traffic.json;
 # a stored figure is used only while the source hash still matches.
 KERNEL_SOURCES = {
-    "decode_gqa": ["decode_attention_06_b200/csrc/decode_simt.cu"],
-    "decode_absorb": ["decode_attention_06_b200/csrc/decode_simt.cu"],
+    "decode_gqa": ["decode_attention_06_b200/csrc/decode_gqa.cu",
+                   "decode_attention_06_b200/csrc/sm100.cuh"],
+    "decode_absorb": ["decode_attention_06_b200/csrc/decode_absorb.cu",
+                      "decode_attention_06_b200/csrc/sm100.cuh"],
 }
 
 
@@ -241,8 +243,8 @@ def run_ours(args, rank, world, local_rank):
     dims = gqla.make_dims(h, g)
     kv = gqla.make_kv_index(case["page_table"], case["seqlens"], case["num_pages"])
     n_slots = case["num_pages"] * case["page_size"]
-    splits = {"absorb": args.splits or gqla.gqla_num_splits_hint("absorb"),
-              "gqa": args.splits or gqla.gqla_num_splits_hint("gqa")}
+    splits = {"absorb": args.splits or gqla.gqla_num_splits_hint("absorb", h, s_q),
+              "gqa": args.splits or gqla.gqla_num_splits_hint("gqa", h, s_q)}
     kvx = torch.empty(g, n_slots, 256, dtype=torch.bfloat16, device=dev)
     kr = torch.empty(n_slots, 64, dtype=torch.bfloat16, device=dev)
     ba = gqla.DecodeBuffers(dims, B, s_q, splits["absorb"], "absorb", device=dev)

@@ -1,0 +1,549 @@
+// decode_absorb.cu -- split-KV partial attention of the MQA-absorb path on the
+// tcgen05 tensor cores (GQLA, paperlayer.ai summary, sec. 2 and sec. 3: W_UK is
+// folded into the query and every head attends directly over the latent row
+// [c (512) | k^R (64)]; the value is the 512-d latent itself).
+//
+// Per (sequence, block of up to 128 query rows) the products are
+//   S = q~ C^T   (M = 128 rows, K = 576, N = tokens)
+//   O += P C_lat (M = 128 rows, K = tokens, N = 512)
+// The fp32 O alone (128 x 512) fills a whole SM's tensor memory, so the work
+// is split over a 2-CTA cluster by latent column: CTA r owns the columns
+// [256r, 256r + 256) of the latent and [32r, 32r + 32) of the RoPE key.  Each
+// CTA streams only its 288 columns of every cache row (the pair reads each
+// byte of the cache exactly once), computes a partial score tile over them,
+// and the two partials are exchanged through distributed shared memory in
+// fp16; both CTAs then add the same two rounded partials, so their P and
+// softmax statistics are bit-identical and each accumulates its own 256
+// columns of O.
+//
+//  * Tile = 64 tokens (one page).  Roles, 352 threads per CTA:
+//      warp 0      TMA producer: the q~ columns of the row block (once per
+//                  piece) and a 3-slot ring of cache tiles (4 latent boxes
+//                  128B-swizzled + 1 RoPE box 64B-swizzled, 36 KB);
+//      warp 1      TMEM owner, issues S = q~ C^T into a double-buffered S;
+//      warps 2-9   online softmax, two warps per TMEM lane quadrant, each
+//                  taking 32 of the tile's 64 tokens: partial-score exchange
+//                  with the peer CTA, row maxima (lazy rescaling of O rows
+//                  when a maximum rises by more than 2^8), P written to TMEM;
+//      warp 10     issues O += P C (A operand read from TMEM) in tile order.
+//  * Every wait is bounded and reports GQLA_ERR_TIMEOUT instead of hanging;
+//    both CTAs of a cluster always execute the same sequence of steps.
+#include <cudaTypedefs.h>
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace gqla {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 352;
+constexpr int kRows = 128;           // MMA M: query rows of one row block (zero-padded)
+constexpr int kT = 64;               // tokens per tile
+constexpr int kRing = 3;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct AbsorbSmem {
+    static constexpr int kQLat = 4 * kRows * 128;        // q~ latent columns, 4 x [128 rows][64]
+    static constexpr int kQRope = kRows * 64;            // q~ RoPE columns [128 rows][32]
+    static constexpr int kLatBox = kT * 128;             // [64 tokens][64 cols]
+    static constexpr int kSlot = 4 * kLatBox + kT * 64;  // 4 latent boxes + RoPE [64 tokens][32]
+    static constexpr int kX = kRows * kT * 2;            // fp16 partial scores [128 rows][64]
+    static constexpr int oQ = 0;
+    static constexpr int oRing = oQ + kQLat + kQRope;
+    static constexpr int oX = oRing + kRing * kSlot;
+    static constexpr int oRm = oX + 2 * kX;              // float [2 halves][128 rows]
+    static constexpr int oL = oRm + 2 * kRows * 4;       // float [2 halves][128 rows]
+    static constexpr int oBar = oL + 2 * kRows * 4;
+    // ring_full/empty[3], q_full, q_empty, s_full/s_free[2], p_full/p_free[2],
+    // x_full/x_empty[2], o_done, drain[2]
+    static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 4 + 1 + 2;
+    static constexpr int oMisc = oBar + kNumBars * 8;    // tmem base, abort, plan[4]
+    static constexpr int kBytes = oMisc + 32;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+struct AbsorbParams {
+    const int32_t *page_table;
+    const int32_t *seqlens;
+    float *o_part;
+    float *lse_part;
+    void *ws;
+    int batch, max_pages, num_pages, num_splits, s_q, heads;
+    int rows_total;   // s_q * heads: query rows of one sequence
+    int row_blocks;   // ceil(rows_total / 128)
+    float scale_log2;
+};
+
+struct PieceIter {
+    int b, P, r0, r1;
+};
+
+__device__ __forceinline__ bool next_piece(const AbsorbParams &p, PieceIter &it, int &b, int &L,
+                                           int &pb, int &pe, bool &too_long) {
+    while (it.b < p.batch && it.P < it.r1) {
+        b = it.b++;
+        L = p.seqlens[b];
+        const int n = pages_of(L);
+        if (n == 0) continue;
+        pb = max(it.r0, it.P) - it.P;
+        pe = min(it.r1, it.P + n) - it.P;
+        it.P += n;
+        too_long = L > p.max_pages * kPage;
+        return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void pair_bar(int quad) {  // the two softmax warps of one lane quadrant
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+}
+
+__device__ __forceinline__ void softmax_bar() {  // all eight softmax warps
+    asm volatile("bar.sync 5, 256;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    decode_absorb_tc_kernel(const __grid_constant__ CUtensorMap lat_map,
+                            const __grid_constant__ CUtensorMap rope_map,
+                            const __grid_constant__ CUtensorMap qlat_map,
+                            const __grid_constant__ CUtensorMap qrope_map, const AbsorbParams p) {
+    using SM = AbsorbSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::oBar);
+    uint64_t *ring_full = bars, *ring_empty = bars + kRing;
+    uint64_t *q_full = bars + 2 * kRing, *q_empty = q_full + 1;
+    uint64_t *s_full = q_empty + 1, *s_free = s_full + 2;
+    uint64_t *p_full = s_free + 2, *p_free = p_full + 2;
+    uint64_t *x_full = p_free + 2, *x_empty = x_full + 2;
+    uint64_t *o_done = x_empty + 2, *drain = o_done + 1;
+    uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(smem + SM::oMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::oMisc + 4);
+    int *plan = reinterpret_cast<int *>(smem + SM::oMisc + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const uint32_t peer = rank ^ 1u;
+    const int cluster = blockIdx.x >> 1;
+    const int c = cluster / p.row_blocks;   // chunk of the split plan
+    const int rb = cluster % p.row_blocks;  // row block within the sequence's s_q * h rows
+    const int rows_here = min(kRows, p.rows_total - rb * kRows);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kRing; ++i) { mbar_init(&ring_full[i], 1); mbar_init(&ring_empty[i], 1); }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 256);
+            mbar_init(&p_full[i], 256); mbar_init(&p_free[i], 1);
+            mbar_init(&x_full[i], 256); mbar_init(&x_empty[i], 256);
+            mbar_init(&drain[i], 1);
+        }
+        mbar_init(o_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        int total = warp_total_pages(p.seqlens, p.batch);
+        int k = chunk_pages(total, p.num_splits);
+        int r0 = c * k, r1 = min(total, r0 + k);
+        int b = p.batch, start = 0;
+        if (r0 < r1) warp_find_sequence(p.seqlens, p.batch, r0, &b, &start);
+        if (lane == 0) { plan[0] = r0; plan[1] = r1; plan[2] = b; plan[3] = start; }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base_smem, 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    cluster_sync();  // the peer's barriers are initialised before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_smem;
+    const uint32_t t_o = tmem;            // O: columns [0, 256), this CTA's latent half
+    const uint32_t t_s = tmem + 256;      // S: 2 x 64 columns
+    const uint32_t t_p = tmem + 384;      // P (bf16 pairs): 2 x 32 columns
+    const PieceIter it0{plan[2], plan[3], plan[0], plan[1]};
+    const uint32_t sm_q = smem_u32(smem + SM::oQ);
+    const uint32_t sm_ring = smem_u32(smem + SM::oRing);
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&lat_map);
+            prefetch_tensormap(&rope_map);
+            prefetch_tensormap(&qlat_map);
+            prefetch_tensormap(&qrope_map);
+            PieceIter it = it0;
+            int b, L, pb, pe;
+            bool too_long;
+            uint32_t t = 0, k = 0;
+            while (next_piece(p, it, b, L, pb, pe, too_long)) {
+                if (too_long) {
+                    if (rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
+                    continue;
+                }
+                // q~ columns of this row block (the previous piece's scores must be done)
+                if (!mbar_wait(q_empty, (k & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                if (!*abort_flag) {
+                    const int row0 = b * p.rows_total + rb * kRows;
+                    mbar_arrive_expect_tx(q_full, SM::kQLat + SM::kQRope);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        tma_load_2d(smem + SM::oQ + i * kRows * 128, &qlat_map, q_full,
+                                    256 * rank + 64 * i, row0);
+                    tma_load_2d(smem + SM::oQ + SM::kQLat, &qrope_map, q_full, 512 + 32 * rank, row0);
+                } else {
+                    mbar_arrive(q_full);
+                }
+                const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
+                for (int pg = pb; pg < pe; ++pg, ++t) {
+                    const int page = prow[pg];
+                    const bool bad = page < 0 || page >= p.num_pages;
+                    if (bad && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
+                    const int slot = t % kRing;
+                    if (!mbar_wait(&ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    uint8_t *dst = smem + SM::oRing + slot * SM::kSlot;
+                    if (!bad && !*abort_flag) {
+                        mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            tma_load_2d(dst + i * SM::kLatBox, &lat_map, &ring_full[slot],
+                                        256 * rank + 64 * i, page * kPage);
+                        tma_load_2d(dst + 4 * SM::kLatBox, &rope_map, &ring_full[slot], 512 + 32 * rank,
+                                    page * kPage);
+                    } else {
+                        mbar_arrive(&ring_full[slot]);
+                    }
+                }
+                ++k;
+            }
+            int dummy = 0;
+            volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
+            for (uint32_t u = (t > (uint32_t)kRing ? t - kRing : 0); u < t; ++u)
+                mbar_wait(&ring_full[u % kRing], (u / kRing) & 1, no_abort);
+            if (k) mbar_wait(q_full, (k - 1) & 1, no_abort);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- score MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(kRows, kT, 0, 0);
+            PieceIter it = it0;
+            int b, L, pb, pe;
+            bool too_long;
+            uint32_t t = 0, k = 0;
+            while (next_piece(p, it, b, L, pb, pe, too_long)) {
+                if (too_long) continue;
+                if (!mbar_wait(q_full, k & 1, abort_flag)) *abort_flag = 1;
+                for (int pg = pb; pg < pe; ++pg, ++t) {
+                    const int slot = t % kRing, sb = t & 1;
+                    if (!mbar_wait(&ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
+                    if (!mbar_wait(&s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    tc_fence_after();
+                    const uint32_t tile = sm_ring + slot * SM::kSlot;
+                    if (!*abort_flag) {
+#pragma unroll
+                        for (int ks = 0; ks < 16; ++ks) {  // latent: 4 swizzle atoms x 4 steps of 16
+                            const uint64_t ad = smem_desc(sm_q + (ks >> 2) * kRows * 128 + (ks & 3) * 32, 16, 1024, kSw128);
+                            const uint64_t bd = smem_desc(tile + (ks >> 2) * SM::kLatBox + (ks & 3) * 32, 16, 1024, kSw128);
+                            mma_bf16(t_s + sb * kT, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                        }
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {  // RoPE: 32 columns, 64B-swizzled rows
+                            const uint64_t ad = smem_desc(sm_q + SM::kQLat + ks * 32, 16, 512, kSw64);
+                            const uint64_t bd = smem_desc(tile + 4 * SM::kLatBox + ks * 32, 16, 512, kSw64);
+                            mma_bf16(t_s + sb * kT, ad, bd, idesc_s, 1u);
+                        }
+                    }
+                    mma_commit(&s_full[sb]);
+                }
+                mma_commit(q_empty);  // q~ may be replaced once these scores are done
+                ++k;
+            }
+            mma_commit(&drain[0]);
+            int dummy = 0;
+            mbar_wait(&drain[0], 0, reinterpret_cast<volatile int *>(&dummy));
+        }
+    } else if (warp == 10) {
+        // ---------------------------------------------------------------- PV MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_pv = idesc_bf16(kRows, 256, 0, 1);
+            PieceIter it = it0;
+            int b, L, pb, pe;
+            bool too_long;
+            uint32_t t = 0;
+            while (next_piece(p, it, b, L, pb, pe, too_long)) {
+                if (too_long) continue;
+                for (int pg = pb; pg < pe; ++pg, ++t) {
+                    const int slot = t % kRing, sb = t & 1;
+                    if (!mbar_wait(&p_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    tc_fence_after();
+                    const uint32_t tile = sm_ring + slot * SM::kSlot;
+                    if (!*abort_flag) {
+#pragma unroll
+                        for (int ks = 0; ks < kT / 16; ++ks) {
+                            // B = C_lat[tokens][256 cols of this CTA]: MN-major, 4 atoms of 64 columns
+                            const uint64_t bd = smem_desc(tile + ks * 2048, SM::kLatBox, 1024, kSw128);
+                            mma_bf16_ts(t_o, t_p + sb * 32 + ks * 8, bd, idesc_pv,
+                                        (pg == pb && ks == 0) ? 0u : 1u);
+                        }
+                    }
+                    mma_commit(&p_free[sb]);
+                    mma_commit(&ring_empty[slot]);
+                }
+                mma_commit(o_done);
+            }
+            mma_commit(&drain[1]);
+            int dummy = 0;
+            mbar_wait(&drain[1], 0, reinterpret_cast<volatile int *>(&dummy));
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax + epilogue
+        const int quad = warp & 3;               // TMEM lane quadrant
+        const int hf = (warp - 2) >> 2;          // which 32 tokens of the tile
+        const int row = 32 * quad + lane;        // query row of the row block (= TMEM lane)
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
+        const int grow = rb * kRows + row;       // row within the sequence's s_q * h rows
+        const int s_of_row = grow < p.rows_total ? grow / p.heads : p.s_q - 1;
+        float *rm = reinterpret_cast<float *>(smem + SM::oRm);
+        float *lsm = reinterpret_cast<float *>(smem + SM::oL);
+        uint8_t *xbuf = smem + SM::oX;
+        const uint32_t x_local = smem_u32(xbuf);
+        const uint32_t x_remote = map_peer(x_local, peer);
+        const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
+        const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
+        PieceIter it = it0;
+        int b, L, pb, pe;
+        bool too_long;
+        uint32_t t = 0, k = 0;
+        while (next_piece(p, it, b, L, pb, pe, too_long)) {
+            if (too_long) continue;
+            float m_run = -INFINITY, l_run = 0.0f;  // this row, this warp's half of every tile
+            const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
+            // query s of this row sees tokens t <= L - s_q + s
+            const int last_visible = L - p.s_q + s_of_row;
+            for (int pg = pb; pg < pe; ++pg, ++t) {
+                const int sb = t & 1, slot = t % kRing;
+                const int page = prow[pg];
+                const bool bad = page < 0 || page >= p.num_pages;
+                const int n_valid = bad ? 0 : min(kT, L - pg * kPage);
+                // ---- own partial scores (this warp's 32 tokens) -> fp16 -> peer
+                if (!mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
+                tc_fence_after();
+                uint32_t sv[32];
+                tmem_ld32(t_s + lane_off + sb * kT + hf * 32, sv);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&s_free[sb]);
+                uint32_t h2[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    __half2 v = __floats2half2_rn(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+                    h2[i] = *reinterpret_cast<uint32_t *>(&v);
+                }
+                if (!mbar_wait_cluster(&x_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                const uint32_t xoff = sb * SM::kX + row * (kT * 2) + hf * 64;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    st_cluster_v4(x_remote + xoff + 16 * i,
+                                  make_uint4(h2[4 * i], h2[4 * i + 1], h2[4 * i + 2], h2[4 * i + 3]));
+                mbar_arrive_remote(xfull_remote + sb * 8);
+                // ---- full scores = own + peer (the same rounded partials in both CTAs)
+                if (!mbar_wait_cluster(&x_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
+                float x[32];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 pv = *reinterpret_cast<const uint4 *>(xbuf + xoff + 16 * i);
+                    const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&h2[4 * i + e]));
+                        const float2 bq = __half22float2(*reinterpret_cast<const __half2 *>(&pw[e]));
+                        const int j = 8 * i + 2 * e;
+                        const int tk = pg * kPage + hf * 32 + j;
+                        x[j] = (hf * 32 + j < n_valid && tk <= last_visible) ? (a.x + bq.x) * p.scale_log2 : -INFINITY;
+                        x[j + 1] = (hf * 32 + j + 1 < n_valid && tk + 1 <= last_visible)
+                                       ? (a.y + bq.y) * p.scale_log2 : -INFINITY;
+                    }
+                }
+                mbar_arrive_remote(xempty_remote + sb * 8);
+                // ---- row maximum over the 64 tokens (pair exchange)
+                float mx = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, x[j]);
+                rm[hf * kRows + row] = mx;
+                pair_bar(quad);
+                const float mt = fmaxf(mx, rm[(hf ^ 1) * kRows + row]);
+                pair_bar(quad);  // rm is rewritten by the next tile
+                const bool first = pg == pb;
+                float m_new = m_run;
+                if (first || mt > m_run + kRescaleLog2) m_new = mt;
+                const bool need = !first && m_new != m_run;
+                const float alpha = need ? exp2f(m_run - m_new) : 1.0f;
+                // P buffer sb is free once PV(t - 2) completed
+                if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, need)) {
+                    // O rows are rescaled only after PV(t - 1) has completed
+                    if (t > 0 && !first)
+                        if (!mbar_wait(&p_free[sb ^ 1], ((t - 1) >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c16 = 0; c16 < 128; c16 += 16) {  // this warp's 128 of the 256 O columns
+                        uint32_t r[16];
+                        const uint32_t ta = t_o + lane_off + hf * 128 + c16;
+                        tmem_ld16(ta, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        tmem_st16(ta, r);
+                    }
+                    tmem_wait_st();
+                }
+                l_run = first ? 0.0f : l_run * alpha;
+                m_run = m_new;
+                // ---- P = 2^(x - m) in bf16 into TMEM (this warp's 16 columns = 32 tokens)
+                const float mu = m_run == -INFINITY ? 0.0f : m_run;
+                uint32_t pw[16];
+                float lsum = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float p0 = x[2 * i] == -INFINITY ? 0.0f : exp2f(x[2 * i] - mu);
+                    const float p1 = x[2 * i + 1] == -INFINITY ? 0.0f : exp2f(x[2 * i + 1] - mu);
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+                    pw[i] = *reinterpret_cast<uint32_t *>(&hb);
+                    const float2 back = __bfloat1622float2(hb);
+                    lsum += back.x + back.y;
+                }
+                l_run += lsum;
+                tmem_st16(t_p + lane_off + sb * 32 + hf * 16, pw);
+                // latent rows that are not tokens (never written, maybe NaN) -> 0
+                if (n_valid < kT) {
+                    if (!mbar_wait(&ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
+                    uint8_t *tile = smem + SM::oRing + slot * SM::kSlot;
+                    const int nz = kT - n_valid;
+                    for (int i = (warp - 2) * 32 + lane; i < 4 * nz * 8; i += 256) {
+                        const int box = i / (nz * 8), rem = i % (nz * 8);
+                        *reinterpret_cast<uint4 *>(tile + box * SM::kLatBox + (n_valid + rem / 8) * 128 +
+                                                   (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&p_full[sb]);
+            }
+            // ---- epilogue: O / l for this CTA's 256 columns (this warp: 128), LSE by rank 0
+            if (!mbar_wait(o_done, k & 1, abort_flag)) *abort_flag = 1;
+            tc_fence_after();
+            lsm[hf * kRows + row] = l_run;
+            pair_bar(quad);
+            const float l = l_run + lsm[(hf ^ 1) * kRows + row];
+            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+            const int slot_out = b + c;
+            const bool live = row < rows_here;
+            const int s = grow / p.heads, hd = grow - s * p.heads;
+            const int64_t orow = ((int64_t)slot_out * p.s_q + s) * p.heads + hd;
+            float *dst = p.o_part + orow * kLatent + 256 * rank + hf * 128;
+#pragma unroll 1
+            for (int c16 = 0; c16 < 128; c16 += 16) {  // loads by the whole warp, stores by live rows
+                uint32_t r[16];
+                tmem_ld16(t_o + lane_off + hf * 128 + c16, r);
+                tmem_wait_ld();
+                if (live) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4 *>(dst + c16 + e) =
+                            make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
+                                        __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+                }
+            }
+            if (live && rank == 0 && hf == 0)
+                p.lse_part[orow] = (l > 0.0f && m_run != -INFINITY)
+                                       ? (m_run + __log2f(l)) * 0.6931471805599453f
+                                       : -INFINITY;
+            tc_fence_before();
+            softmax_bar();  // O may be overwritten by the next piece's first PV
+            ++k;
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) report_error(p.ws, GQLA_ERR_TIMEOUT, c);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    cluster_sync();  // no remote access may target a CTA that has exited
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2D bf16 map over [rows][576] with a box of `box_cols` x `box_rows`.
+bool make_map_2d(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_cols,
+                 uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kRow, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kRow * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
+                                 const gqla_kv_index *idx, int num_splits, float scale,
+                                 float *o_part, float *lse_part, void *ws, cudaStream_t stream) {
+    CUtensorMap lat, rope, qlat, qrope;
+    const uint64_t slots = (uint64_t)idx->num_pages * kPage;
+    const uint64_t qrows = (uint64_t)idx->batch * s_q * heads;
+    if (!make_map_2d(&lat, cache, slots, 64, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&rope, cache, slots, 32, kT, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_2d(&qlat, qa, qrows, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&qrope, qa, qrows, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    AbsorbParams p;
+    p.page_table = idx->page_table;
+    p.seqlens = idx->seqlens;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.ws = ws;
+    p.batch = idx->batch;
+    p.max_pages = idx->max_pages_per_seq;
+    p.num_pages = idx->num_pages;
+    p.num_splits = num_splits;
+    p.s_q = s_q;
+    p.heads = heads;
+    p.rows_total = s_q * heads;
+    p.row_blocks = (p.rows_total + kRows - 1) / kRows;
+    p.scale_log2 = scale * kLog2e;
+    cudaError_t e = cudaFuncSetAttribute(decode_absorb_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, AbsorbSmem::kAlloc);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)num_splits * p.row_blocks * 2;
+    decode_absorb_tc_kernel<<<grid, kThreads, AbsorbSmem::kAlloc, stream>>>(lat, rope, qlat, qrope, p);
+    return cudaGetLastError();
+}
+
+}  // namespace gqla

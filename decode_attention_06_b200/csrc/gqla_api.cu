@@ -14,10 +14,9 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
                               const void *k_rope, int64_t num_slots, const gqla_kv_index *idx,
                               int num_splits, float scale, float *o_part, float *lse_part,
                               void *ws, cudaStream_t stream);
-cudaError_t launch_decode_absorb_simt(const void *qa, int s_q, int heads, const void *cache,
-                                      const gqla_kv_index *idx, int num_splits, float scale,
-                                      float *o_part, float *lse_part, void *ws,
-                                      cudaStream_t stream);
+cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
+                                 const gqla_kv_index *idx, int num_splits, float scale,
+                                 float *o_part, float *lse_part, void *ws, cudaStream_t stream);
 cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int d_in,
                            const float *o_part, const float *lse_part, const void *w_uv,
                            void *out, float *lse_out, int heads, int num_groups,
@@ -94,13 +93,15 @@ int gqla_partial_slots(int batch, int num_splits) {
     return batch + num_splits;
 }
 
-int gqla_num_splits_hint(int path) {
-    if (path != 0 && path != 1) return GQLA_ERR_INVALID_ARG;
+int gqla_num_splits_hint(int path, int num_heads, int s_q) {
+    if ((path != 0 && path != 1) || num_heads <= 0 || s_q <= 0) return GQLA_ERR_INVALID_ARG;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GQLA_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GQLA_ERR_CUDA;
-    return sms;
+    if (path == 1) return sms;
+    const int row_blocks = (s_q * num_heads + 127) / 128;
+    return sms / (2 * row_blocks) > 0 ? sms / (2 * row_blocks) : 1;
 }
 
 int gqla_read_device_error(const void *workspace, int *info, gqla_stream_t stream) {
@@ -159,10 +160,12 @@ int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
     if (!q_absorbed || !latent_cache || !o_part || !lse_part) return GQLA_ERR_INVALID_ARG;
     if (!aligned16(q_absorbed) || !aligned16(latent_cache) || !aligned16(o_part))
         return GQLA_ERR_INVALID_ARG;
-    if ((s_q * dims->num_heads) % 16) return GQLA_ERR_UNSUPPORTED;
-    return cuda_status(launch_decode_absorb_simt(q_absorbed, s_q, dims->num_heads, latent_cache, kv,
-                                                 num_splits, dims->softmax_scale, o_part, lse_part,
-                                                 workspace, reinterpret_cast<cudaStream_t>(stream)));
+    if ((s_q * dims->num_heads) % 32) return GQLA_ERR_UNSUPPORTED;
+    if ((int64_t)num_splits * ((s_q * dims->num_heads + 127) / 128) * 2 > 65535 * 2)
+        return GQLA_ERR_UNSUPPORTED;
+    return cuda_status(launch_decode_absorb(q_absorbed, s_q, dims->num_heads, latent_cache, kv,
+                                            num_splits, dims->softmax_scale, o_part, lse_part,
+                                            workspace, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,

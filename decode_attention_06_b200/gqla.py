@@ -65,7 +65,7 @@ _SIGS = {
     "gqla_decode_gqa_noalloc": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _P],
     "gqla_partial_slots": [_I, _I],
     "gqla_workspace_bytes": [],
-    "gqla_num_splits_hint": [_I],
+    "gqla_num_splits_hint": [_I, _I, _I],
     "gqla_read_device_error": [_P, ctypes.POINTER(ctypes.c_int), _P],
     "gqla_clear_device_error": [_P, _P],
     "gqla_status_string": [_I],
@@ -211,8 +211,8 @@ def gqla_workspace_bytes() -> int:
     return int(_lib.gqla_workspace_bytes())
 
 
-def gqla_num_splits_hint(path: str) -> int:
-    n = _lib.gqla_num_splits_hint({"absorb": 0, "gqa": 1}[path])
+def gqla_num_splits_hint(path: str, num_heads: int, s_q: int) -> int:
+    n = _lib.gqla_num_splits_hint({"absorb": 0, "gqa": 1}[path], num_heads, s_q)
     if n < 0:
         raise GqlaError("gqla_num_splits_hint", n)
     return n

@@ -199,9 +199,11 @@ int gqla_partial_slots(int batch, int num_splits);
 /* Workspace bytes the decode calls need. */
 size_t gqla_workspace_bytes(void);
 
-/* A split count that fills the current device (SM count x resident CTAs of the
- * path's decode kernel); path 0 = absorb, 1 = GQA.  Returns < 0 on error. */
-int gqla_num_splits_hint(int path);
+/* A split count that fills the current device with one wave: the GQA decode
+ * runs one CTA per split, the absorb decode a 2-CTA cluster per split and per
+ * 128 query rows of a sequence (s_q * num_heads rows).  path 0 = absorb,
+ * 1 = GQA.  Returns < 0 on error. */
+int gqla_num_splits_hint(int path, int num_heads, int s_q);
 
 /* Reads (synchronising `stream`) and returns the first device-side error
  * recorded in `workspace` (GQLA_OK if none); `info`, if not NULL, receives

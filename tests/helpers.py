@@ -26,7 +26,7 @@ def run_decode(gcase, path, num_splits=None, stream=None):
     kv = gqla.make_kv_index(gcase["page_table"], gcase["seqlens"], gcase["num_pages"])
     B = gcase["seqlens"].numel()
     if num_splits is None:
-        num_splits = gqla.gqla_num_splits_hint(path)
+        num_splits = gqla.gqla_num_splits_hint(path, h, s_q)
     bufs = gqla.DecodeBuffers(dims, B, s_q, num_splits, path)
     extras = {}
     if path == "gqa":

@@ -122,4 +122,5 @@ def test_other_calls_reject_bad_arguments(lib):
     assert lib.gqla_combine(ctypes.byref(d), ctypes.byref(kv), 1, 4, 128, FAKE, FAKE, FAKE, FAKE, None, None) == -1
     assert lib.gqla_combine(ctypes.byref(d), ctypes.byref(kv), 1, 4, 256, FAKE, FAKE, None, FAKE, None, None) == -1
     assert lib.gqla_read_device_error(None, None, None) == -1
-    assert lib.gqla_num_splits_hint(7) == -1
+    assert lib.gqla_num_splits_hint(7, 128, 1) == -1
+    assert lib.gqla_num_splits_hint(0, 0, 1) == -1
