@@ -16,15 +16,19 @@
 // softmax statistics are bit-identical and each accumulates its own 256
 // columns of O.
 //
-//  * Tile = 64 tokens (one page).  Roles, 352 threads per CTA:
+//  * Tile = 32 tokens (half a page).  Roles, 352 threads per CTA:
 //      warp 0      TMA producer: the q~ columns of the row block (once per
-//                  piece) and a 3-slot ring of cache tiles (4 latent boxes
-//                  128B-swizzled + 1 RoPE box 64B-swizzled, 36 KB);
+//                  piece) and a 5-slot ring of cache tiles (4 latent boxes
+//                  128B-swizzled + 1 RoPE box 64B-swizzled, 18 KB);
 //      warp 1      TMEM owner, issues S = q~ C^T into a double-buffered S;
 //      warps 2-9   online softmax, two warps per TMEM lane quadrant, each
-//                  taking 32 of the tile's 64 tokens: partial-score exchange
-//                  with the peer CTA, row maxima (lazy rescaling of O rows
-//                  when a maximum rises by more than 2^8), P written to TMEM;
+//                  taking 16 of the tile's 32 tokens: partial-score exchange
+//                  with the peer CTA (each warp stages its 2 KB locally and
+//                  sends it with one asynchronous bulk copy that completes
+//                  on the peer's mbarrier), row maxima (lazy rescaling of O rows
+//                  when a maximum rises by more than 2^8), P written to TMEM.
+//                  The loop is software-pipelined: tile i + 1's partial is
+//                  sent before tile i is finished, hiding the exchange;
 //      warp 10     issues O += P C (A operand read from TMEM) in tile order.
 //  * Every wait is bounded and reports GQLA_ERR_TIMEOUT instead of hanging;
 //    both CTAs of a cluster always execute the same sequence of steps.
@@ -43,21 +47,23 @@ using namespace sm100;
 
 constexpr int kThreads = 352;
 constexpr int kRows = 128;           // MMA M: query rows of one row block (zero-padded)
-constexpr int kT = 64;               // tokens per tile
-constexpr int kRing = 3;
+constexpr int kT = 32;               // tokens per tile (half a page)
+constexpr int kRing = 5;
 constexpr float kRescaleLog2 = 8.0f;
 
 struct AbsorbSmem {
     static constexpr int kQLat = 4 * kRows * 128;        // q~ latent columns, 4 x [128 rows][64]
     static constexpr int kQRope = kRows * 64;            // q~ RoPE columns [128 rows][32]
-    static constexpr int kLatBox = kT * 128;             // [64 tokens][64 cols]
-    static constexpr int kSlot = 4 * kLatBox + kT * 64;  // 4 latent boxes + RoPE [64 tokens][32]
-    static constexpr int kX = kRows * kT * 2;            // fp16 partial scores [128 rows][64]
+    static constexpr int kLatBox = kT * 128;             // [32 tokens][64 cols]
+    static constexpr int kSlot = 4 * kLatBox + kT * 64;  // 4 latent boxes + RoPE [32 tokens][32]
+    static constexpr int kX = kRows * kT * 2;            // fp16 partial scores, [8 warps][32 rows][16]
+    static constexpr int kXw = kX / 8;                   // one warp's block
     static constexpr int oQ = 0;
     static constexpr int oRing = oQ + kQLat + kQRope;
-    static constexpr int oX = oRing + kRing * kSlot;
-    static constexpr int oRm = oX + 2 * kX;              // float [2 halves][128 rows]
-    static constexpr int oL = oRm + 2 * kRows * 4;       // float [2 halves][128 rows]
+    static constexpr int oX = oRing + kRing * kSlot;     // the peer's partials (2 buffers)
+    static constexpr int oStg = oX + 2 * kX;             // this CTA's partials, sent from here (2 buffers)
+    static constexpr int oRm = oStg + 2 * kX;            // float [2 tiles][2 halves][128 rows]
+    static constexpr int oL = oRm + 4 * kRows * 4;       // float [2 halves][128 rows]
     static constexpr int oBar = oL + 2 * kRows * 4;
     // ring_full/empty[3], q_full, q_empty, s_full/s_free[2], p_full/p_free[2],
     // x_full/x_empty[2], o_done, drain[2]
@@ -126,6 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(smem + SM::oMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::oMisc + 4);
     int *plan = reinterpret_cast<int *>(smem + SM::oMisc + 8);
+    GQLA_PROF_DECL;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -142,7 +149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 256);
             mbar_init(&p_full[i], 256); mbar_init(&p_free[i], 1);
-            mbar_init(&x_full[i], 256); mbar_init(&x_empty[i], 256);
+            mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 8);
             mbar_init(&drain[i], 1);
         }
         mbar_init(o_done, 1);
@@ -167,8 +174,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_base_smem;
     const uint32_t t_o = tmem;            // O: columns [0, 256), this CTA's latent half
-    const uint32_t t_s = tmem + 256;      // S: 2 x 64 columns
-    const uint32_t t_p = tmem + 384;      // P (bf16 pairs): 2 x 32 columns
+    const uint32_t t_s = tmem + 256;      // S: 2 x kT columns
+    const uint32_t t_p = tmem + 256 + 2 * kT;  // P (bf16 pairs): 2 x kT/2 columns
     const PieceIter it0{plan[2], plan[3], plan[0], plan[1]};
     const uint32_t sm_q = smem_u32(smem + SM::oQ);
     const uint32_t sm_ring = smem_u32(smem + SM::oRing);
@@ -190,7 +197,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     continue;
                 }
                 // q~ columns of this row block (the previous piece's scores must be done)
-                if (!mbar_wait(q_empty, (k & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                if (!GQLA_WAIT(1, q_empty, (k & 1) ^ 1, abort_flag)) *abort_flag = 1;
                 if (!*abort_flag) {
                     const int row0 = b * p.rows_total + rb * kRows;
                     mbar_arrive_expect_tx(q_full, SM::kQLat + SM::kQRope);
@@ -203,21 +210,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     mbar_arrive(q_full);
                 }
                 const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
-                for (int pg = pb; pg < pe; ++pg, ++t) {
-                    const int page = prow[pg];
+                for (int i = 0; i < 2 * (pe - pb); ++i, ++t) {
+                    const int page = prow[pb + i / 2];
                     const bool bad = page < 0 || page >= p.num_pages;
-                    if (bad && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
+                    if (bad && (i & 1) == 0 && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
                     const int slot = t % kRing;
-                    if (!mbar_wait(&ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(0, &ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                     uint8_t *dst = smem + SM::oRing + slot * SM::kSlot;
                     if (!bad && !*abort_flag) {
                         mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            tma_load_2d(dst + i * SM::kLatBox, &lat_map, &ring_full[slot],
-                                        256 * rank + 64 * i, page * kPage);
+                        for (int bx = 0; bx < 4; ++bx)
+                            tma_load_2d(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
+                                        256 * rank + 64 * bx, page * kPage + (i & 1) * kT);
                         tma_load_2d(dst + 4 * SM::kLatBox, &rope_map, &ring_full[slot], 512 + 32 * rank,
-                                    page * kPage);
+                                    page * kPage + (i & 1) * kT);
                     } else {
                         mbar_arrive(&ring_full[slot]);
                     }
@@ -240,11 +247,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t t = 0, k = 0;
             while (next_piece(p, it, b, L, pb, pe, too_long)) {
                 if (too_long) continue;
-                if (!mbar_wait(q_full, k & 1, abort_flag)) *abort_flag = 1;
-                for (int pg = pb; pg < pe; ++pg, ++t) {
+                if (!GQLA_WAIT(2, q_full, k & 1, abort_flag)) *abort_flag = 1;
+                for (int i = 0; i < 2 * (pe - pb); ++i, ++t) {
                     const int slot = t % kRing, sb = t & 1;
-                    if (!mbar_wait(&ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
-                    if (!mbar_wait(&s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(3, &ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(4, &s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
                     const uint32_t tile = sm_ring + slot * SM::kSlot;
                     if (!*abort_flag) {
@@ -280,9 +287,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t t = 0;
             while (next_piece(p, it, b, L, pb, pe, too_long)) {
                 if (too_long) continue;
-                for (int pg = pb; pg < pe; ++pg, ++t) {
+                for (int i = 0; i < 2 * (pe - pb); ++i, ++t) {
                     const int slot = t % kRing, sb = t & 1;
-                    if (!mbar_wait(&p_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(5, &p_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
                     const uint32_t tile = sm_ring + slot * SM::kSlot;
                     if (!*abort_flag) {
@@ -290,8 +297,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         for (int ks = 0; ks < kT / 16; ++ks) {
                             // B = C_lat[tokens][256 cols of this CTA]: MN-major, 4 atoms of 64 columns
                             const uint64_t bd = smem_desc(tile + ks * 2048, SM::kLatBox, 1024, kSw128);
-                            mma_bf16_ts(t_o, t_p + sb * 32 + ks * 8, bd, idesc_pv,
-                                        (pg == pb && ks == 0) ? 0u : 1u);
+                            mma_bf16_ts(t_o, t_p + sb * (kT / 2) + ks * 8, bd, idesc_pv,
+                                        (i == 0 && ks == 0) ? 0u : 1u);
                         }
                     }
                     mma_commit(&p_free[sb]);
@@ -313,9 +320,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int s_of_row = grow < p.rows_total ? grow / p.heads : p.s_q - 1;
         float *rm = reinterpret_cast<float *>(smem + SM::oRm);
         float *lsm = reinterpret_cast<float *>(smem + SM::oL);
+        const int w8 = warp - 2;                 // softmax warp index: its 2 KB block of a buffer
         uint8_t *xbuf = smem + SM::oX;
-        const uint32_t x_local = smem_u32(xbuf);
-        const uint32_t x_remote = map_peer(x_local, peer);
+        uint8_t *stg = smem + SM::oStg;
+        const uint32_t x_remote = map_peer(smem_u32(xbuf), peer);
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
         const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
         PieceIter it = it0;
@@ -328,71 +336,105 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             // query s of this row sees tokens t <= L - s_q + s
             const int last_visible = L - p.s_q + s_of_row;
-            for (int pg = pb; pg < pe; ++pg, ++t) {
-                const int sb = t & 1, slot = t % kRing;
-                const int page = prow[pg];
-                const bool bad = page < 0 || page >= p.num_pages;
-                const int n_valid = bad ? 0 : min(kT, L - pg * kPage);
-                // ---- own partial scores (this warp's 32 tokens) -> fp16 -> peer
-                if (!mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
+            const uint32_t t0 = t;
+            const int nt = 2 * (pe - pb);
+            // stage A of tile i: this warp's partial scores -> fp16 -> staged -> sent to the peer
+            auto stage_a = [&](int i, uint32_t (&h2)[8]) {
+                const uint32_t tt = t0 + i;
+                const int sb = tt & 1;
+                if (!GQLA_WAIT(6, &s_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
                 tc_fence_after();
-                uint32_t sv[32];
-                tmem_ld32(t_s + lane_off + sb * kT + hf * 32, sv);
+                uint32_t sv[16];
+                GQLA_SPAN_BEGIN(a1);
+                tmem_ld16(t_s + lane_off + sb * kT + hf * 16, sv);
                 tmem_wait_ld();
+                GQLA_SPAN_END(17, a1);
                 tc_fence_before();
                 mbar_arrive(&s_free[sb]);
-                uint32_t h2[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    __half2 v = __floats2half2_rn(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
-                    h2[i] = *reinterpret_cast<uint32_t *>(&v);
+                for (int j = 0; j < 8; ++j) {
+                    __half2 v = __floats2half2_rn(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
+                    h2[j] = *reinterpret_cast<uint32_t *>(&v);
                 }
-                if (!mbar_wait_cluster(&x_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                const uint32_t xoff = sb * SM::kX + row * (kT * 2) + hf * 64;
+                if (w8 == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kX);
+                // our staging buffer sb is free once the peer has consumed tile tt - 2
+                if (!GQLA_WAITC(7, &x_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                const uint32_t xoff = sb * SM::kX + w8 * SM::kXw + lane * 32;
+                GQLA_SPAN_BEGIN(a2);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    st_cluster_v4(x_remote + xoff + 16 * i,
-                                  make_uint4(h2[4 * i], h2[4 * i + 1], h2[4 * i + 2], h2[4 * i + 3]));
-                mbar_arrive_remote(xfull_remote + sb * 8);
+                for (int j = 0; j < 2; ++j)
+                    *reinterpret_cast<uint4 *>(stg + xoff + 16 * j) =
+                        make_uint4(h2[4 * j], h2[4 * j + 1], h2[4 * j + 2], h2[4 * j + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                GQLA_SPAN_END(18, a2);
+                GQLA_SPAN_BEGIN(a3);
+                if (lane == 0)
+                    bulk_copy_to_peer(x_remote + sb * SM::kX + w8 * SM::kXw, stg + sb * SM::kX + w8 * SM::kXw,
+                                      SM::kXw, xfull_remote + sb * 8);
+                __syncwarp();
+                GQLA_SPAN_END(19, a3);
+            };
+            uint32_t hc[8];
+            stage_a(0, hc);
+            for (int i = 0; i < nt; ++i) {
+                // the next tile's exchange is in flight while this one is finished
+                uint32_t hn[8];
+                if (i + 1 < nt) stage_a(i + 1, hn);
+                const uint32_t tt = t0 + i;
+                const int pg = pb + i / 2;
+                const int tok0 = pg * kPage + (i & 1) * kT;  // first token of this tile
+                const int sb = tt & 1, slot = tt % kRing;
+                const int page = prow[pg];
+                const bool bad = page < 0 || page >= p.num_pages;
+                const int n_valid = bad ? 0 : max(0, min(kT, L - tok0));
+                GQLA_SPAN_BEGIN(t_tile);
                 // ---- full scores = own + peer (the same rounded partials in both CTAs)
-                if (!mbar_wait_cluster(&x_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
-                float x[32];
+                if (!GQLA_WAITC(8, &x_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
+                const uint32_t xoff = sb * SM::kX + w8 * SM::kXw + lane * 32;
+                float x[16];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 pv = *reinterpret_cast<const uint4 *>(xbuf + xoff + 16 * i);
+                for (int j4 = 0; j4 < 2; ++j4) {
+                    const uint4 pv = *reinterpret_cast<const uint4 *>(xbuf + xoff + 16 * j4);
                     const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&h2[4 * i + e]));
+                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&hc[4 * j4 + e]));
                         const float2 bq = __half22float2(*reinterpret_cast<const __half2 *>(&pw[e]));
-                        const int j = 8 * i + 2 * e;
-                        const int tk = pg * kPage + hf * 32 + j;
-                        x[j] = (hf * 32 + j < n_valid && tk <= last_visible) ? (a.x + bq.x) * p.scale_log2 : -INFINITY;
-                        x[j + 1] = (hf * 32 + j + 1 < n_valid && tk + 1 <= last_visible)
+                        const int j = 8 * j4 + 2 * e;
+                        const int tk = tok0 + hf * 16 + j;
+                        x[j] = (hf * 16 + j < n_valid && tk <= last_visible) ? (a.x + bq.x) * p.scale_log2 : -INFINITY;
+                        x[j + 1] = (hf * 16 + j + 1 < n_valid && tk + 1 <= last_visible)
                                        ? (a.y + bq.y) * p.scale_log2 : -INFINITY;
                     }
                 }
-                mbar_arrive_remote(xempty_remote + sb * 8);
+                GQLA_SPAN_BEGIN(b1);
+                fence_proxy_async_smem();  // our reads of X[sb] precede the peer's next copy into it
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote + sb * 8);
+                __syncwarp();
+                GQLA_SPAN_END(20, b1);
+                GQLA_SPAN_BEGIN(b2);
                 // ---- row maximum over the 64 tokens (pair exchange)
                 float mx = -INFINITY;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, x[j]);
-                rm[hf * kRows + row] = mx;
+                for (int j = 0; j < 16; ++j) mx = fmaxf(mx, x[j]);
+                rm[(tt & 1) * 2 * kRows + hf * kRows + row] = mx;
                 pair_bar(quad);
-                const float mt = fmaxf(mx, rm[(hf ^ 1) * kRows + row]);
-                pair_bar(quad);  // rm is rewritten by the next tile
-                const bool first = pg == pb;
+                const float mt = fmaxf(mx, rm[(tt & 1) * 2 * kRows + (hf ^ 1) * kRows + row]);
+                GQLA_SPAN_END(21, b2);
+                const bool first = i == 0;
                 float m_new = m_run;
                 if (first || mt > m_run + kRescaleLog2) m_new = mt;
                 const bool need = !first && m_new != m_run;
                 const float alpha = need ? exp2f(m_run - m_new) : 1.0f;
-                // P buffer sb is free once PV(t - 2) completed
-                if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                // P buffer sb is free once PV(tt - 2) completed
+                if (!GQLA_WAIT(9, &p_free[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, need)) {
-                    // O rows are rescaled only after PV(t - 1) has completed
-                    if (t > 0 && !first)
-                        if (!mbar_wait(&p_free[sb ^ 1], ((t - 1) >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    // O rows are rescaled only after PV(tt - 1) has completed
+                    if (!first)
+                        if (!mbar_wait(&p_free[sb ^ 1], ((tt - 1) >> 1) & 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
 #pragma unroll 1
                     for (int c16 = 0; c16 < 128; c16 += 16) {  // this warp's 128 of the 256 O columns
@@ -408,28 +450,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 l_run = first ? 0.0f : l_run * alpha;
                 m_run = m_new;
-                // ---- P = 2^(x - m) in bf16 into TMEM (this warp's 16 columns = 32 tokens)
+                // ---- P = 2^(x - m) in bf16 into TMEM (this warp's 8 columns = 16 tokens)
+                GQLA_SPAN_BEGIN(b3);
                 const float mu = m_run == -INFINITY ? 0.0f : m_run;
-                uint32_t pw[16];
+                uint32_t pw[8];
                 float lsum = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = x[2 * i] == -INFINITY ? 0.0f : exp2f(x[2 * i] - mu);
-                    const float p1 = x[2 * i + 1] == -INFINITY ? 0.0f : exp2f(x[2 * i + 1] - mu);
+                for (int j = 0; j < 8; ++j) {
+                    const float p0 = x[2 * j] == -INFINITY ? 0.0f : fast_exp2(x[2 * j] - mu);
+                    const float p1 = x[2 * j + 1] == -INFINITY ? 0.0f : fast_exp2(x[2 * j + 1] - mu);
                     __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-                    pw[i] = *reinterpret_cast<uint32_t *>(&hb);
+                    pw[j] = *reinterpret_cast<uint32_t *>(&hb);
                     const float2 back = __bfloat1622float2(hb);
                     lsum += back.x + back.y;
                 }
                 l_run += lsum;
-                tmem_st16(t_p + lane_off + sb * 32 + hf * 16, pw);
+                GQLA_SPAN_END(22, b3);
+                GQLA_SPAN_BEGIN(b4);
+                tmem_st8(t_p + lane_off + sb * (kT / 2) + hf * 8, pw);
                 // latent rows that are not tokens (never written, maybe NaN) -> 0
                 if (n_valid < kT) {
-                    if (!mbar_wait(&ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
+                    if (!mbar_wait(&ring_full[slot], (tt / kRing) & 1, abort_flag)) *abort_flag = 1;
                     uint8_t *tile = smem + SM::oRing + slot * SM::kSlot;
                     const int nz = kT - n_valid;
-                    for (int i = (warp - 2) * 32 + lane; i < 4 * nz * 8; i += 256) {
-                        const int box = i / (nz * 8), rem = i % (nz * 8);
+                    for (int z = w8 * 32 + lane; z < 4 * nz * 8; z += 256) {
+                        const int box = z / (nz * 8), rem = z % (nz * 8);
                         *reinterpret_cast<uint4 *>(tile + box * SM::kLatBox + (n_valid + rem / 8) * 128 +
                                                    (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
                     }
@@ -438,9 +483,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[sb]);
+                GQLA_SPAN_END(23, b4);
+                GQLA_SPAN_END(10, t_tile);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) hc[j] = hn[j];
             }
+            t = t0 + nt;
             // ---- epilogue: O / l for this CTA's 256 columns (this warp: 128), LSE by rank 0
-            if (!mbar_wait(o_done, k & 1, abort_flag)) *abort_flag = 1;
+            GQLA_SPAN_BEGIN(t_epi);
+            if (!GQLA_WAIT(15, o_done, k & 1, abort_flag)) *abort_flag = 1;
             tc_fence_after();
             lsm[hf * kRows + row] = l_run;
             pair_bar(quad);
@@ -470,10 +521,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                        : -INFINITY;
             tc_fence_before();
             softmax_bar();  // O may be overwritten by the next piece's first PV
+            GQLA_SPAN_END(16, t_epi);
             ++k;
         }
     }
 
+    GQLA_PROF_FLUSH;
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) report_error(p.ws, GQLA_ERR_TIMEOUT, c);
     if (warp == 1) {

@@ -232,8 +232,8 @@ __device__ __forceinline__ void write_p(const uint32_t (&sv)[NQ], const float (&
             const float x1 = score_of(sv[n + e + 1], n + e + 1, tok_ok, hide_low, G, scale_log2);
             const float m0 = mu[n + e] == -INFINITY ? 0.0f : mu[n + e];
             const float m1 = mu[n + e + 1] == -INFINITY ? 0.0f : mu[n + e + 1];
-            const float p0 = x0 == -INFINITY ? 0.0f : exp2f(x0 - m0);
-            const float p1 = x1 == -INFINITY ? 0.0f : exp2f(x1 - m1);
+            const float p0 = x0 == -INFINITY ? 0.0f : fast_exp2(x0 - m0);
+            const float p1 = x1 == -INFINITY ? 0.0f : fast_exp2(x1 - m1);
             __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             w[e / 2] = *reinterpret_cast<uint32_t *>(&h2);
             const float2 back = __bfloat1622float2(h2);

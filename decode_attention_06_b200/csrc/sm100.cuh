@@ -103,6 +103,13 @@ __device__ unsigned long long g_wait_count[32];
         GQLA_PROF_ADD(site, clock64() - t0_);                                \
         ok_;                                                                 \
     })
+#define GQLA_WAITC(site, bar, parity, abort)                                 \
+    ({                                                                       \
+        const long long t0_ = clock64();                                     \
+        const bool ok_ = ::gqla::sm100::mbar_wait_cluster(bar, parity, abort); \
+        GQLA_PROF_ADD(site, clock64() - t0_);                                \
+        ok_;                                                                 \
+    })
 #define GQLA_SPAN_BEGIN(v) const long long v = clock64()
 #define GQLA_SPAN_END(site, v) GQLA_PROF_ADD(site, clock64() - v)
 #define GQLA_PROF_FLUSH                                                                     \
@@ -118,6 +125,7 @@ __device__ unsigned long long g_wait_count[32];
 #else
 #define GQLA_PROF_DECL (void)0
 #define GQLA_WAIT(site, bar, parity, abort) ::gqla::sm100::mbar_wait(bar, parity, abort)
+#define GQLA_WAITC(site, bar, parity, abort) ::gqla::sm100::mbar_wait_cluster(bar, parity, abort)
 #define GQLA_SPAN_BEGIN(v) (void)0
 #define GQLA_SPAN_END(site, v) (void)0
 #define GQLA_PROF_FLUSH (void)0
@@ -296,10 +304,43 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
     }
 }
 
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into a
+// peer CTA's shared memory; completes `bytes` of transaction count on the
+// peer's mbarrier.  Asynchronous: the issuing thread does not wait.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const void *src,
+                                                  uint32_t bytes, uint32_t mbar_cluster) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst_cluster),
+        "r"(smem_u32(src)), "r"(bytes), "r"(mbar_cluster)
+        : "memory");
+}
+
+// Arrive on a peer CTA's mbarrier without ordering this thread's memory accesses.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
 // All threads of all CTAs of the cluster (aligned: every thread executes it).
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
+// 2^x with the hardware approximation (a single MUFU.EX2; flushes subnormal
+// results to zero, which is harmless for softmax weights that are rounded to
+// bf16 afterwards).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // ------------------------------------------------------------------ descriptors
