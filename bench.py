@@ -15,9 +15,11 @@ value   = decode tokens per second of the whole job: N ranks x batch x s_q
 e2e     = the same through the C ABI with host buffers: each step copies the
           queries, page table and lengths from pinned host memory and reads
           both paths' outputs back, inside the timed region.
-Timing  = CUDA events on the launching stream around every call and step,
-          L2 flushed (a 256 MiB write) before every timed step, outside the
-          step's events; W >= 3 untimed warm-up steps first.
+Timing  = the step is captured once into a CUDA graph with an event record
+          before and after every call; each timed step replays the graph and
+          reads those events (device time, no host launch overhead).  L2 is
+          flushed (a 256 MiB write) before every step, outside its events;
+          W >= 3 untimed eager and W graph warm-up steps come first.
 roofline: the dominant kernel's algorithmic bytes (or FLOPs) per launch over
           its mean event-timed duration, against MEASURED_PEAKS.json.
 cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload
@@ -274,35 +276,47 @@ def run_ours(args, rank, world, local_rank):
         lambda: gqla.gqla_combine(dims, kv, s_q, bg.num_splits, 128, bg.o_part, bg.lse_part,
                                   None, bg.out, bg.lse),
     ]
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
-          for _ in range(args.steps)]
-
     def step(events=None):
         for i, c in enumerate(calls):
             if events is not None:
-                events[i].record(stream)
+                events[i].record()
             c()
         if events is not None:
-            events[-1].record(stream)
+            events[-1].record()
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
         step()
     torch.cuda.synchronize()
+
+    # The step is captured once into a CUDA graph (the five launches replay
+    # without host launch overhead); event records inside the graph time each
+    # call on the device at every replay.
+    gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(gev)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        graph.replay()
+    torch.cuda.synchronize()
+
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    per_call = [[] for _ in calls]
+    step_ms = []
     with ClockSampler(local_rank) as clocks:
         for k in range(args.steps):
             flush.fill_(1.0)  # evict the caches from L2 (outside the step's events)
-            step(ev[k])
-        torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            for i in range(len(calls)):
+                per_call[i].append(gev[i].elapsed_time(gev[i + 1]))
+            step_ms.append(gev[0].elapsed_time(gev[-1]))
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    per_call = [[ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)]
-                for i in range(len(calls))]
-    step_ms = [ev[k][0].elapsed_time(ev[k][-1]) for k in range(args.steps)]
     ms_step = sum(step_ms) / args.steps
     st_a, _ = gqla.gqla_read_device_error(ba.workspace)
     st_g, _ = gqla.gqla_read_device_error(bg.workspace)

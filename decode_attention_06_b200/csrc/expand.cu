@@ -1,6 +1,6 @@
-// expand.cu -- one-shot per-group cache expansion for the GQA path and the
-// query absorption for the MQA-absorb path (GQLA, paperlayer.ai summary,
-// sec. 3 "Two equivalent decoding paths"; pwwt.cn article, sec. 3).
+// expand.cu -- one-shot per-group cache expansion for the GQA path (GQLA,
+// paperlayer.ai summary, sec. 3 "Two equivalent decoding paths"; pwwt.cn
+// article, sec. 3).
 //
 // Expansion: kv[g][n][0:128] = c_n W_UK_g, kv[g][n][128:256] = c_n W_UV_g,
 // k_rope[n] = k^R_n.  The rounding order is part of the contract (fp32, one
@@ -120,97 +120,6 @@ __global__ void copy_rope_kernel(const __nv_bfloat16 *__restrict__ latent, int64
     *reinterpret_cast<uint4 *>(k_rope + slot * kRope + part * 8) = v;
 }
 
-// ---------------------------------------------------------------------------
-// Query absorption: qa[r][k] = sum_d W_UK_{g(r)}[k][d] q[r][d] (k < 512),
-// qa[r][512 + j] = q[r][128 + j].  Rows of one group share W_UK_g, so a block
-// takes 64 rows of one group and 128 of the 512 outputs.
-// grid: x = row tiles of one group, y = g * 4 column tiles.  256 threads.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) absorb_query_kernel(const __nv_bfloat16 *__restrict__ q,
-                                                           const __nv_bfloat16 *__restrict__ w_uk,
-                                                           __nv_bfloat16 *__restrict__ qa,
-                                                           int rows_per_group, int heads,
-                                                           int heads_per_group) {
-    constexpr int DC = 32;                             // d chunk
-    __shared__ __align__(16) float Qs[DC][64 + 4];     // [d][row]
-    __shared__ __align__(16) float Ws[DC][128 + 4];    // [d][k]
-    const int tid = threadIdx.x;
-    const int grp = blockIdx.y >> 2, ktile = blockIdx.y & 3;
-    const int j0 = blockIdx.x * 64;
-    const __nv_bfloat16 *W = w_uk + (size_t)grp * kLatent * kNope + (size_t)ktile * 128 * kNope;
-
-    auto row_of = [&](int j) -> int64_t {  // j-th row of this group -> global row
-        return (int64_t)(j / heads_per_group) * heads + grp * heads_per_group + j % heads_per_group;
-    };
-
-    const int tx = tid % 32, ty = tid / 32;  // rows ty*8..+8, cols tx*4..+4
-    float acc[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-
-    for (int dc = 0; dc < kNope; dc += DC) {
-        __syncthreads();
-        // q chunk: 64 rows x 32 d = 256 uint4; W chunk: 128 k x 32 d = 512 uint4
-        {
-            int r = tid / 4, d0 = (tid % 4) * 8;
-            float f[8];
-            if (j0 + r < rows_per_group) {
-                uint4 v = *reinterpret_cast<const uint4 *>(q + row_of(j0 + r) * kQk + dc + d0);
-                unpack8(v, f);
-            } else {
-#pragma unroll
-                for (int t = 0; t < 8; ++t) f[t] = 0.0f;
-            }
-#pragma unroll
-            for (int t = 0; t < 8; ++t) Qs[d0 + t][r] = f[t];
-        }
-        for (int i = tid; i < 128 * 4; i += 256) {
-            int k = i / 4, d0 = (i % 4) * 8;
-            float f[8];
-            uint4 v = *reinterpret_cast<const uint4 *>(W + (size_t)k * kNope + dc + d0);
-            unpack8(v, f);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) Ws[d0 + t][k] = f[t];
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int d = 0; d < DC; ++d) {
-            float4 a0 = *reinterpret_cast<const float4 *>(&Qs[d][ty * 8]);
-            float4 a1 = *reinterpret_cast<const float4 *>(&Qs[d][ty * 8 + 4]);
-            float4 b = *reinterpret_cast<const float4 *>(&Ws[d][tx * 4]);
-            float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            float bb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(a[i], bb[j], acc[i][j]);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int j = j0 + ty * 8 + i;
-        if (j >= rows_per_group) continue;
-        __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[i][0], acc[i][1]);
-        __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[i][2], acc[i][3]);
-        uint2 st;
-        st.x = *reinterpret_cast<uint32_t *>(&p0);
-        st.y = *reinterpret_cast<uint32_t *>(&p1);
-        *reinterpret_cast<uint2 *>(qa + row_of(j) * kRow + ktile * 128 + tx * 4) = st;
-    }
-    // RoPE part copied by the first column tile
-    if (ktile == 0) {
-        for (int i = tid; i < 64 * 8; i += 256) {
-            int r = i / 8, part = i % 8;
-            if (j0 + r >= rows_per_group) continue;
-            int64_t row = row_of(j0 + r);
-            uint4 v = *reinterpret_cast<const uint4 *>(q + row * kQk + kNope + part * 8);
-            *reinterpret_cast<uint4 *>(qa + row * kRow + kLatent + part * 8) = v;
-        }
-    }
-}
-
 }  // namespace
 
 cudaError_t launch_expand(const void *latent, int64_t num_slots, const void *w_uk,
@@ -227,18 +136,6 @@ cudaError_t launch_expand(const void *latent, int64_t num_slots, const void *w_u
     int64_t vec = num_slots * 8;
     copy_rope_kernel<<<(unsigned)((vec + 255) / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(latent), num_slots, static_cast<__nv_bfloat16 *>(k_rope));
-    return cudaGetLastError();
-}
-
-cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_groups,
-                                const void *w_uk, void *qa, cudaStream_t stream) {
-    const int G = heads / num_groups;
-    const int rows_per_group = rows / heads * G;
-    if (rows_per_group == 0) return cudaSuccess;
-    dim3 grid((rows_per_group + 63) / 64, num_groups * 4);
-    absorb_query_kernel<<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(w_uk),
-        static_cast<__nv_bfloat16 *>(qa), rows_per_group, heads, G);
     return cudaGetLastError();
 }
 

@@ -196,6 +196,8 @@ int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int nu
     if ((st = check_index(kv)) != GQLA_OK) return st;
     if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
     if (!o_part || !lse_part || !out) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(o_part) || !aligned16(out) || (w_uv && !aligned16(w_uv)))
+        return GQLA_ERR_INVALID_ARG;
     if (d_in == kLatent) {
         if (!w_uv) return GQLA_ERR_INVALID_ARG;
     } else if (d_in == kDv) {

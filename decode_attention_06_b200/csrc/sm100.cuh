@@ -273,6 +273,14 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
 // Arrive on an mbarrier of another CTA of the cluster, releasing this thread's
 // earlier shared::cluster stores to whoever acquires the phase.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {

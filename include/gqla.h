@@ -107,6 +107,9 @@ int gqla_expand_cache(const gqla_dims *dims, const void *latent, int64_t num_slo
  *   q           bf16 [batch][s_q][h][192]  (0..127 q^C, 128..191 q^R, RoPE applied)
  *   w_uk        bf16 [g][512][128]
  *   q_absorbed  bf16 [batch][s_q][h][576]  out: [W_UK_{g(h)} q^C ; q^R], fp32 accumulation
+ * All pointers 16-byte aligned.  Runs on the tensor cores; its device-side
+ * waits are bounded, and one that runs out (a fault elsewhere) leaves
+ * q_absorbed unwritten, since this call has no workspace to report into.
  */
 int gqla_absorb_query(const gqla_dims *dims, const void *q, int batch, int s_q,
                       const void *w_uk, void *q_absorbed, gqla_stream_t stream);
@@ -152,7 +155,11 @@ int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *k
  *   d_in      512 (absorb partials; w_uv required) or 128 (GQA partials; w_uv NULL)
  *   out       bf16 [batch][s_q][h][128]
  *   lse_out   fp32 [batch][s_q][h] or NULL
- * A row with no visible token gets out = 0 and lse = -inf.
+ * o_part, out and w_uv 16-byte aligned.  A row with no visible token gets
+ * out = 0 and lse = -inf.  For d_in == 512 the merged latent row is rounded
+ * to bf16 (the tensor-core operand type) before the product with W_UV, which
+ * accumulates in fp32.  Like gqla_absorb_query this call has no workspace: a
+ * bounded device-side wait that runs out leaves `out` unwritten.
  */
 int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
                  int d_in, const float *o_part, const float *lse_part, const void *w_uv,
