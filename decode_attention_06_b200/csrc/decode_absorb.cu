@@ -12,24 +12,31 @@
 // CTA streams only its 288 columns of every cache row (the pair reads each
 // byte of the cache exactly once), computes a partial score tile over them,
 // and the two partials are exchanged through distributed shared memory in
-// fp16; both CTAs then add the same two rounded partials, so their P and
-// softmax statistics are bit-identical and each accumulates its own 256
-// columns of O.
+// fp16; both CTAs add the same two rounded partials, so their P and softmax
+// statistics are bit-identical, and each accumulates its own 256 columns of O.
 //
-//  * Tile = 32 tokens (half a page).  Roles, 352 threads per CTA:
-//      warp 0      TMA producer: the q~ columns of the row block (once per
-//                  piece) and a 5-slot ring of cache tiles (4 latent boxes
-//                  128B-swizzled + 1 RoPE box 64B-swizzled, 18 KB);
-//      warp 1      TMEM owner, issues S = q~ C^T into a double-buffered S;
+//  * Tile = one 64-token page.  An MMA instruction costs at least ~45 cycles
+//    whatever its N, so the score tile is made 64 tokens wide.  Tensor memory
+//    holds O (256 columns), a double-buffered S (2 x 64) and the latent half
+//    of q~ (128 columns of bf16 pairs), so the score MMA reads q~ from TMEM;
+//    P goes through shared memory, beside a 4-slot ring of cache tiles.
+//    Roles, 352 threads:
+//      warp 0      TMA producer: the RoPE columns of q~ (once per piece) and
+//                  the ring (4 latent boxes 128B-swizzled + 1 RoPE box
+//                  64B-swizzled, 36 KB per 64-token tile);
+//      warp 1      TMEM owner, issues S = q~ C^T (latent part with A in TMEM);
 //      warps 2-9   online softmax, two warps per TMEM lane quadrant, each
-//                  taking 16 of the tile's 32 tokens: partial-score exchange
-//                  with the peer CTA (each warp stages its 2 KB locally and
-//                  sends it with one asynchronous bulk copy that completes
-//                  on the peer's mbarrier), row maxima (lazy rescaling of O rows
-//                  when a maximum rises by more than 2^8), P written to TMEM.
-//                  The loop is software-pipelined: tile i + 1's partial is
-//                  sent before tile i is finished, hiding the exchange;
-//      warp 10     issues O += P C (A operand read from TMEM) in tile order.
+//                  taking 32 of the tile's 64 tokens: the fp16 partial
+//                  scores go straight from registers into the peer CTA's
+//                  receive buffer with st.async (completing on the peer's
+//                  mbarrier), row maxima (lazy rescaling of O rows when a
+//                  maximum rises by more than 2^8), P written to shared
+//                  memory (bf16, 128B-swizzled, the PV MMA's A operand).  Tile
+//                  i + 1's partial is sent before tile i is finished when its
+//                  scores are already available;
+//      warp 10     issues O += P C in tile order.
+//  * Per piece the softmax warps first copy the latent half of q~ from global
+//    memory into TMEM, and end with O / l written from TMEM to the partials.
 //  * Every wait is bounded and reports GQLA_ERR_TIMEOUT instead of hanging;
 //    both CTAs of a cluster always execute the same sequence of steps.
 #include <cudaTypedefs.h>
@@ -38,6 +45,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tensor_map.cuh"
 
 namespace gqla {
 
@@ -47,35 +55,38 @@ using namespace sm100;
 
 constexpr int kThreads = 352;
 constexpr int kRows = 128;           // MMA M: query rows of one row block (zero-padded)
-constexpr int kT = 32;               // tokens per tile (half a page)
-constexpr int kRing = 5;
+constexpr int kT = 64;               // tokens per tile (one page)
+constexpr int kRing = 4;
 constexpr float kRescaleLog2 = 8.0f;
 
 struct AbsorbSmem {
-    static constexpr int kQLat = 4 * kRows * 128;        // q~ latent columns, 4 x [128 rows][64]
-    static constexpr int kQRope = kRows * 64;            // q~ RoPE columns [128 rows][32]
-    static constexpr int kLatBox = kT * 128;             // [32 tokens][64 cols]
-    static constexpr int kSlot = 4 * kLatBox + kT * 64;  // 4 latent boxes + RoPE [32 tokens][32]
-    static constexpr int kX = kRows * kT * 2;            // fp16 partial scores, [8 warps][32 rows][16]
-    static constexpr int kXw = kX / 8;                   // one warp's block
+    static constexpr int kQRope = kRows * 64;             // q~ RoPE columns [128 rows][32]
+    static constexpr int kLatBox = kT * 128;              // [64 tokens][64 cols]
+    static constexpr int kRopeBox = kT * 64;              // [64 tokens][32 cols]
+    static constexpr int kSlot = 4 * kLatBox + kRopeBox;  // 36 KB
+    static constexpr int kX = kRows * kT * 2;             // fp16 partial scores, [8 warps][32 rows][32]
+    static constexpr int kXw = kX / 8;                    // one warp's block
+    static constexpr int kP = kRows * kT * 2;             // P, [128 rows][64 tokens] bf16, 128B-swizzled
     static constexpr int oQ = 0;
-    static constexpr int oRing = oQ + kQLat + kQRope;
-    static constexpr int oX = oRing + kRing * kSlot;     // the peer's partials (2 buffers)
-    static constexpr int oStg = oX + 2 * kX;             // this CTA's partials, sent from here (2 buffers)
-    static constexpr int oRm = oStg + 2 * kX;            // float [2 tiles][2 halves][128 rows]
-    static constexpr int oL = oRm + 4 * kRows * 4;       // float [2 halves][128 rows]
+    static constexpr int oP = oQ + kQRope;                // 2 buffers
+    static constexpr int oRing = oP + 2 * kP;
+    static constexpr int oX = oRing + kRing * kSlot;      // the peer's partials (2 buffers)
+    static constexpr int oRm = oX + 2 * kX;               // float [2 tiles][2 halves][128 rows]
+    static constexpr int oL = oRm + 4 * kRows * 4;        // float [2 halves][128 rows]
     static constexpr int oBar = oL + 2 * kRows * 4;
     // ring_full/empty[3], q_full, q_empty, s_full/s_free[2], p_full/p_free[2],
     // x_full/x_empty[2], o_done, drain[2]
     static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 4 + 1 + 2;
-    static constexpr int oMisc = oBar + kNumBars * 8;    // tmem base, abort, plan[4]
+    static constexpr int oMisc = oBar + kNumBars * 8;     // tmem base, abort, plan[4]
     static constexpr int kBytes = oMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;
 };
+static_assert(AbsorbSmem::kAlloc <= 227 * 1024, "shared memory");
 
 struct AbsorbParams {
     const int32_t *page_table;
     const int32_t *seqlens;
+    const __nv_bfloat16 *qa;
     float *o_part;
     float *lse_part;
     void *ws;
@@ -109,14 +120,9 @@ __device__ __forceinline__ void pair_bar(int quad) {  // the two softmax warps o
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
 }
 
-__device__ __forceinline__ void softmax_bar() {  // all eight softmax warps
-    asm volatile("bar.sync 5, 256;" ::: "memory");
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_absorb_tc_kernel(const __grid_constant__ CUtensorMap lat_map,
                             const __grid_constant__ CUtensorMap rope_map,
-                            const __grid_constant__ CUtensorMap qlat_map,
                             const __grid_constant__ CUtensorMap qrope_map, const AbsorbParams p) {
     using SM = AbsorbSmem;
     extern __shared__ uint8_t smem_raw[];
@@ -144,8 +150,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i) { mbar_init(&ring_full[i], 1); mbar_init(&ring_empty[i], 1); }
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
+        mbar_init(q_full, 1 + 8);  // RoPE TMA + the 8 softmax warps' TMEM copies
+        mbar_init(q_empty, 8);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 256);
             mbar_init(&p_full[i], 256); mbar_init(&p_free[i], 1);
@@ -173,64 +179,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // the peer's barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem = *tmem_base_smem;
-    const uint32_t t_o = tmem;            // O: columns [0, 256), this CTA's latent half
-    const uint32_t t_s = tmem + 256;      // S: 2 x kT columns
-    const uint32_t t_p = tmem + 256 + 2 * kT;  // P (bf16 pairs): 2 x kT/2 columns
+    const uint32_t t_o = tmem;             // O: columns [0, 256), this CTA's latent half
+    const uint32_t t_s = tmem + 256;       // S: 2 x kT columns
+    const uint32_t t_q = tmem + 384;       // q~ latent half (bf16 pairs): 128 columns
     const PieceIter it0{plan[2], plan[3], plan[0], plan[1]};
     const uint32_t sm_q = smem_u32(smem + SM::oQ);
     const uint32_t sm_ring = smem_u32(smem + SM::oRing);
+    const uint32_t sm_p = smem_u32(smem + SM::oP);
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
+        // Lane 0 issues; the whole warp fetches the page indices 32 at a time so
+        // that no page-table load sits between two tiles.
         if (lane == 0) {
             prefetch_tensormap(&lat_map);
             prefetch_tensormap(&rope_map);
-            prefetch_tensormap(&qlat_map);
             prefetch_tensormap(&qrope_map);
-            PieceIter it = it0;
-            int b, L, pb, pe;
-            bool too_long;
-            uint32_t t = 0, k = 0;
-            while (next_piece(p, it, b, L, pb, pe, too_long)) {
-                if (too_long) {
-                    if (rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
-                    continue;
-                }
-                // q~ columns of this row block (the previous piece's scores must be done)
+        }
+        PieceIter it = it0;
+        int b, L, pb, pe;
+        bool too_long;
+        uint32_t t = 0, k = 0;
+        while (next_piece(p, it, b, L, pb, pe, too_long)) {
+            if (too_long) {
+                if (lane == 0 && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
+                continue;
+            }
+            // RoPE columns of q~ for this row block (the previous piece's scores are done)
+            if (lane == 0) {
                 if (!GQLA_WAIT(1, q_empty, (k & 1) ^ 1, abort_flag)) *abort_flag = 1;
                 if (!*abort_flag) {
                     const int row0 = b * p.rows_total + rb * kRows;
-                    mbar_arrive_expect_tx(q_full, SM::kQLat + SM::kQRope);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        tma_load_2d(smem + SM::oQ + i * kRows * 128, &qlat_map, q_full,
-                                    256 * rank + 64 * i, row0);
-                    tma_load_2d(smem + SM::oQ + SM::kQLat, &qrope_map, q_full, 512 + 32 * rank, row0);
+                    mbar_arrive_expect_tx(q_full, SM::kQRope);
+                    tma_load_2d(smem + SM::oQ, &qrope_map, q_full, 512 + 32 * rank, row0);
                 } else {
                     mbar_arrive(q_full);
                 }
-                const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
-                for (int i = 0; i < 2 * (pe - pb); ++i, ++t) {
-                    const int page = prow[pb + i / 2];
-                    const bool bad = page < 0 || page >= p.num_pages;
-                    if (bad && (i & 1) == 0 && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
-                    const int slot = t % kRing;
-                    if (!GQLA_WAIT(0, &ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                    uint8_t *dst = smem + SM::oRing + slot * SM::kSlot;
-                    if (!bad && !*abort_flag) {
-                        mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
+            }
+            const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
+            for (int i0 = pb; i0 < pe; i0 += 32) {
+                const int n = min(32, pe - i0);
+                const int my_page = lane < n ? prow[i0 + lane] : 0;
+                for (int j = 0; j < n; ++j, ++t) {
+                    const int page = __shfl_sync(0xffffffffu, my_page, j);
+                    if (lane == 0) {
+                        const bool bad = page < 0 || page >= p.num_pages;
+                        if (bad && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
+                        const int slot = t % kRing;
+                        if (!GQLA_WAIT(0, &ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                        uint8_t *dst = smem + SM::oRing + slot * SM::kSlot;
+                        if (!bad && !*abort_flag) {
+                            mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
 #pragma unroll
-                        for (int bx = 0; bx < 4; ++bx)
-                            tma_load_2d(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
-                                        256 * rank + 64 * bx, page * kPage + (i & 1) * kT);
-                        tma_load_2d(dst + 4 * SM::kLatBox, &rope_map, &ring_full[slot], 512 + 32 * rank,
-                                    page * kPage + (i & 1) * kT);
-                    } else {
-                        mbar_arrive(&ring_full[slot]);
+                            for (int bx = 0; bx < 4; ++bx)
+                                tma_load_2d(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
+                                            256 * rank + 64 * bx, page * kPage);
+                            tma_load_2d(dst + 4 * SM::kLatBox, &rope_map, &ring_full[slot], 512 + 32 * rank,
+                                        page * kPage);
+                        } else {
+                            mbar_arrive(&ring_full[slot]);
+                        }
                     }
                 }
-                ++k;
             }
+            ++k;
+        }
+        if (lane == 0) {
+            // no TMA may still be writing when the CTA exits
             int dummy = 0;
             volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
             for (uint32_t u = (t > (uint32_t)kRing ? t - kRing : 0); u < t; ++u)
@@ -248,7 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             while (next_piece(p, it, b, L, pb, pe, too_long)) {
                 if (too_long) continue;
                 if (!GQLA_WAIT(2, q_full, k & 1, abort_flag)) *abort_flag = 1;
-                for (int i = 0; i < 2 * (pe - pb); ++i, ++t) {
+                for (int i = 0; i < pe - pb; ++i, ++t) {
                     const int slot = t % kRing, sb = t & 1;
                     if (!GQLA_WAIT(3, &ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
                     if (!GQLA_WAIT(4, &s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
@@ -256,21 +271,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t tile = sm_ring + slot * SM::kSlot;
                     if (!*abort_flag) {
 #pragma unroll
-                        for (int ks = 0; ks < 16; ++ks) {  // latent: 4 swizzle atoms x 4 steps of 16
-                            const uint64_t ad = smem_desc(sm_q + (ks >> 2) * kRows * 128 + (ks & 3) * 32, 16, 1024, kSw128);
+                        for (int ks = 0; ks < 16; ++ks) {  // latent: A = q~ in TMEM, 16 dims = 8 columns
                             const uint64_t bd = smem_desc(tile + (ks >> 2) * SM::kLatBox + (ks & 3) * 32, 16, 1024, kSw128);
-                            mma_bf16(t_s + sb * kT, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                            mma_bf16_ts(t_s + sb * kT, t_q + ks * 8, bd, idesc_s, ks > 0 ? 1u : 0u);
                         }
 #pragma unroll
                         for (int ks = 0; ks < 2; ++ks) {  // RoPE: 32 columns, 64B-swizzled rows
-                            const uint64_t ad = smem_desc(sm_q + SM::kQLat + ks * 32, 16, 512, kSw64);
+                            const uint64_t ad = smem_desc(sm_q + ks * 32, 16, 512, kSw64);
                             const uint64_t bd = smem_desc(tile + 4 * SM::kLatBox + ks * 32, 16, 512, kSw64);
                             mma_bf16(t_s + sb * kT, ad, bd, idesc_s, 1u);
                         }
                     }
                     mma_commit(&s_full[sb]);
                 }
-                mma_commit(q_empty);  // q~ may be replaced once these scores are done
                 ++k;
             }
             mma_commit(&drain[0]);
@@ -287,7 +300,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t t = 0;
             while (next_piece(p, it, b, L, pb, pe, too_long)) {
                 if (too_long) continue;
-                for (int i = 0; i < 2 * (pe - pb); ++i, ++t) {
+                for (int i = 0; i < pe - pb; ++i, ++t) {
                     const int slot = t % kRing, sb = t & 1;
                     if (!GQLA_WAIT(5, &p_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
@@ -297,8 +310,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         for (int ks = 0; ks < kT / 16; ++ks) {
                             // B = C_lat[tokens][256 cols of this CTA]: MN-major, 4 atoms of 64 columns
                             const uint64_t bd = smem_desc(tile + ks * 2048, SM::kLatBox, 1024, kSw128);
-                            mma_bf16_ts(t_o, t_p + sb * (kT / 2) + ks * 8, bd, idesc_pv,
-                                        (i == 0 && ks == 0) ? 0u : 1u);
+                            // A = P[128 rows][64 tokens], K-major: 16 tokens = 32 bytes of a row
+                            const uint64_t ad = smem_desc(sm_p + sb * SM::kP + ks * 32, 16, 1024, kSw128);
+                            mma_bf16(t_o, ad, bd, idesc_pv, (i == 0 && ks == 0) ? 0u : 1u);
                         }
                     }
                     mma_commit(&p_free[sb]);
@@ -321,11 +335,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float *rm = reinterpret_cast<float *>(smem + SM::oRm);
         float *lsm = reinterpret_cast<float *>(smem + SM::oL);
         const int w8 = warp - 2;                 // softmax warp index: its 2 KB block of a buffer
-        uint8_t *xbuf = smem + SM::oX;
-        uint8_t *stg = smem + SM::oStg;
-        const uint32_t x_remote = map_peer(smem_u32(xbuf), peer);
+        const uint8_t *xbuf = smem + SM::oX;
+        const uint32_t x_remote = map_peer(smem_u32(smem + SM::oX), peer) + w8 * SM::kXw + lane * 64;
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
         const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
+        const __half2 scale2 = __float2half2_rn(p.scale_log2);
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
@@ -337,97 +351,126 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // query s of this row sees tokens t <= L - s_q + s
             const int last_visible = L - p.s_q + s_of_row;
             const uint32_t t0 = t;
-            const int nt = 2 * (pe - pb);
-            // stage A of tile i: this warp's partial scores -> fp16 -> staged -> sent to the peer
-            auto stage_a = [&](int i, uint32_t (&h2)[8]) {
+            const int nt = pe - pb;
+            // ---- this warp's quarter of q~'s latent half (its 32 rows x 128 columns) into TMEM;
+            // the previous piece's scores, the last readers of that TMEM, are complete
+            {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    p.qa + ((int64_t)b * p.rows_total + grow) * kRow + 256 * rank + hf * 128);
+                const bool live = row < rows_here;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 v = live ? src[4 * h + j] : make_uint4(0, 0, 0, 0);
+                        w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+                    }
+                    tmem_st16(t_q + lane_off + hf * 64 + 16 * h, w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_full);
+            }
+            // stage A of tile i: this warp's partial scores -> fp16 -> the peer's receive buffer
+            auto stage_a = [&](int i, uint32_t (&h2)[16]) {
                 const uint32_t tt = t0 + i;
                 const int sb = tt & 1;
                 if (!GQLA_WAIT(6, &s_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
                 tc_fence_after();
-                uint32_t sv[16];
-                GQLA_SPAN_BEGIN(a1);
-                tmem_ld16(t_s + lane_off + sb * kT + hf * 16, sv);
+                uint32_t sv[32];
+                tmem_ld32(t_s + lane_off + sb * kT + hf * 32, sv);
                 tmem_wait_ld();
-                GQLA_SPAN_END(17, a1);
                 tc_fence_before();
                 mbar_arrive(&s_free[sb]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 16; ++j) {
                     __half2 v = __floats2half2_rn(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
                     h2[j] = *reinterpret_cast<uint32_t *>(&v);
                 }
                 if (w8 == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kX);
-                // our staging buffer sb is free once the peer has consumed tile tt - 2
+                // the peer's receive buffer sb is free once it has read tile tt - 2
                 if (!GQLA_WAITC(7, &x_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                const uint32_t xoff = sb * SM::kX + w8 * SM::kXw + lane * 32;
-                GQLA_SPAN_BEGIN(a2);
 #pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    *reinterpret_cast<uint4 *>(stg + xoff + 16 * j) =
-                        make_uint4(h2[4 * j], h2[4 * j + 1], h2[4 * j + 2], h2[4 * j + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                GQLA_SPAN_END(18, a2);
-                GQLA_SPAN_BEGIN(a3);
-                if (lane == 0)
-                    bulk_copy_to_peer(x_remote + sb * SM::kX + w8 * SM::kXw, stg + sb * SM::kX + w8 * SM::kXw,
-                                      SM::kXw, xfull_remote + sb * 8);
-                __syncwarp();
-                GQLA_SPAN_END(19, a3);
+                for (int j = 0; j < 4; ++j)
+                    st_async_v4(x_remote + sb * SM::kX + 16 * j,
+                                make_uint4(h2[4 * j], h2[4 * j + 1], h2[4 * j + 2], h2[4 * j + 3]),
+                                xfull_remote + sb * 8);
             };
-            uint32_t hc[8];
+            uint32_t hc[16];
             stage_a(0, hc);
+            bool have_next = false;  // stage A of tile i + 1 already done
+            int page = prow[pb];
             for (int i = 0; i < nt; ++i) {
-                // the next tile's exchange is in flight while this one is finished
-                uint32_t hn[8];
-                if (i + 1 < nt) stage_a(i + 1, hn);
+                // Tile i + 1's exchange is started early only when its scores are
+                // already there: waiting for them here would tie the release of
+                // tile i (and of its ring slot) to the arrival of the next tile.
+                uint32_t hn[16];
+                const bool next_ready =
+                    i + 1 < nt && __shfl_sync(0xffffffffu,  // one decision per warp
+                                              (int)mbar_test_wait(&s_full[(t0 + i + 1) & 1], ((t0 + i + 1) >> 1) & 1), 0);
+                if (next_ready) {
+                    stage_a(i + 1, hn);
+                    have_next = true;
+                }
+                const int page_next = i + 1 < nt ? prow[pb + i + 1] : 0;  // in flight meanwhile
                 const uint32_t tt = t0 + i;
-                const int pg = pb + i / 2;
-                const int tok0 = pg * kPage + (i & 1) * kT;  // first token of this tile
+                const int pg = pb + i;
+                const int tok0 = pg * kPage;  // first token of this tile
                 const int sb = tt & 1, slot = tt % kRing;
-                const int page = prow[pg];
                 const bool bad = page < 0 || page >= p.num_pages;
                 const int n_valid = bad ? 0 : max(0, min(kT, L - tok0));
                 GQLA_SPAN_BEGIN(t_tile);
-                // ---- full scores = own + peer (the same rounded partials in both CTAs)
+                // ---- full raw scores = own + peer (the same rounded partials in both CTAs)
                 if (!GQLA_WAITC(8, &x_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
-                const uint32_t xoff = sb * SM::kX + w8 * SM::kXw + lane * 32;
-                float x[16];
+                __half2 x[16];
+                GQLA_SPAN_BEGIN(b1);
+                {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(xbuf + sb * SM::kX + w8 * SM::kXw + lane * 64);
 #pragma unroll
-                for (int j4 = 0; j4 < 2; ++j4) {
-                    const uint4 pv = *reinterpret_cast<const uint4 *>(xbuf + xoff + 16 * j4);
-                    const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+                    for (int j4 = 0; j4 < 4; ++j4) {
+                        const uint4 pv = src[j4];
+                        const uint32_t pw4[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&hc[4 * j4 + e]));
-                        const float2 bq = __half22float2(*reinterpret_cast<const __half2 *>(&pw[e]));
-                        const int j = 8 * j4 + 2 * e;
-                        const int tk = tok0 + hf * 16 + j;
-                        x[j] = (hf * 16 + j < n_valid && tk <= last_visible) ? (a.x + bq.x) * p.scale_log2 : -INFINITY;
-                        x[j + 1] = (hf * 16 + j + 1 < n_valid && tk + 1 <= last_visible)
-                                       ? (a.y + bq.y) * p.scale_log2 : -INFINITY;
+                        for (int e = 0; e < 4; ++e)
+                            x[4 * j4 + e] = __hadd2(*reinterpret_cast<const __half2 *>(&hc[4 * j4 + e]),
+                                                    *reinterpret_cast<const __half2 *>(&pw4[e]));
                     }
                 }
-                GQLA_SPAN_BEGIN(b1);
-                fence_proxy_async_smem();  // our reads of X[sb] precede the peer's next copy into it
+                // the peer may refill our receive buffer sb (the values above are consumed)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote + sb * 8);
-                __syncwarp();
                 GQLA_SPAN_END(20, b1);
                 GQLA_SPAN_BEGIN(b2);
-                // ---- row maximum over the 64 tokens (pair exchange)
-                float mx = -INFINITY;
+                // ---- mask tokens past the sequence or past this query's causal limit
+                const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + hf * 32);  // last visible index here
+                if (lim < 31) {
+                    const __half ninf = __ushort_as_half((unsigned short)0xFC00u);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) mx = fmaxf(mx, x[j]);
+                    for (int j = 0; j < 16; ++j) {
+                        if (2 * j > lim) x[j].x = ninf;
+                        if (2 * j + 1 > lim) x[j].y = ninf;
+                    }
+                }
+                // ---- row maximum over the 64 tokens (pair exchange)
+                __half2 hm8[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) hm8[j] = __hmax2(x[j], x[j + 8]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) hm8[j] = __hmax2(hm8[j], hm8[j + 4]);
+                const __half2 hm = __hmax2(__hmax2(hm8[0], hm8[2]), __hmax2(hm8[1], hm8[3]));
+                const float mx = fmaxf(__low2float(hm), __high2float(hm)) * p.scale_log2;  // log2 units
                 rm[(tt & 1) * 2 * kRows + hf * kRows + row] = mx;
                 pair_bar(quad);
                 const float mt = fmaxf(mx, rm[(tt & 1) * 2 * kRows + (hf ^ 1) * kRows + row]);
                 GQLA_SPAN_END(21, b2);
                 const bool first = i == 0;
                 float m_new = m_run;
-                if (first || mt > m_run + kRescaleLog2) m_new = mt;
+                // the running maximum is kept on the fp16 grid: P below subtracts it in fp16
+                if (first || mt > m_run + kRescaleLog2) m_new = __half2float(__float2half_rn(mt));
                 const bool need = !first && m_new != m_run;
-                const float alpha = need ? exp2f(m_run - m_new) : 1.0f;
+                const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;
                 // P buffer sb is free once PV(tt - 2) completed
                 if (!GQLA_WAIT(9, &p_free[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                 tc_fence_after();
@@ -450,24 +493,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 l_run = first ? 0.0f : l_run * alpha;
                 m_run = m_new;
-                // ---- P = 2^(x - m) in bf16 into TMEM (this warp's 8 columns = 16 tokens)
+                // ---- P = 2^(x scale - m), two tokens per fp16 ex2, in bf16 into shared
+                // memory (this warp's 32 tokens = bytes [64 hf, 64 hf + 64) of the row)
                 GQLA_SPAN_BEGIN(b3);
-                const float mu = m_run == -INFINITY ? 0.0f : m_run;
-                uint32_t pw[8];
+                const __half2 mneg2 = __float2half2_rn(m_run == -INFINITY ? 0.0f : -m_run);
+                uint32_t pw[16];
                 float lsum = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float p0 = x[2 * j] == -INFINITY ? 0.0f : fast_exp2(x[2 * j] - mu);
-                    const float p1 = x[2 * j + 1] == -INFINITY ? 0.0f : fast_exp2(x[2 * j + 1] - mu);
-                    __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+                for (int j = 0; j < 16; ++j) {
+                    const float2 pf = __half22float2(fast_exp2_h2(__hfma2(x[j], scale2, mneg2)));
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(pf.x, pf.y);
                     pw[j] = *reinterpret_cast<uint32_t *>(&hb);
-                    const float2 back = __bfloat1622float2(hb);
-                    lsum += back.x + back.y;
+                    lsum += pf.x + pf.y;
                 }
                 l_run += lsum;
                 GQLA_SPAN_END(22, b3);
                 GQLA_SPAN_BEGIN(b4);
-                tmem_st8(t_p + lane_off + sb * (kT / 2) + hf * 8, pw);
+                {
+                    uint8_t *prow_s = smem + SM::oP + sb * SM::kP + row * 128;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        *reinterpret_cast<uint4 *>(prow_s + (((hf * 4 + j) ^ (row & 7)) << 4)) =
+                            make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
+                }
                 // latent rows that are not tokens (never written, maybe NaN) -> 0
                 if (n_valid < kT) {
                     if (!mbar_wait(&ring_full[slot], (tt / kRing) & 1, abort_flag)) *abort_flag = 1;
@@ -478,17 +526,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint4 *>(tile + box * SM::kLatBox + (n_valid + rem / 8) * 128 +
                                                    (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
                     }
-                    fence_proxy_async_smem();
                 }
-                tmem_wait_st();
+                fence_proxy_async_smem();  // P (and any zeroed rows) -> the PV MMA
                 tc_fence_before();
                 mbar_arrive(&p_full[sb]);
                 GQLA_SPAN_END(23, b4);
                 GQLA_SPAN_END(10, t_tile);
+                if (i + 1 < nt && !have_next) stage_a(i + 1, hn);
+                have_next = false;
+                page = page_next;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) hc[j] = hn[j];
+                for (int j = 0; j < 16; ++j) hc[j] = hn[j];
             }
             t = t0 + nt;
+            // the last scores of the piece are read: the producer may load the next RoPE q~
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_empty);
             // ---- epilogue: O / l for this CTA's 256 columns (this warp: 128), LSE by rank 0
             GQLA_SPAN_BEGIN(t_epi);
             if (!GQLA_WAIT(15, o_done, k & 1, abort_flag)) *abort_flag = 1;
@@ -497,20 +550,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             pair_bar(quad);
             const float l = l_run + lsm[(hf ^ 1) * kRows + row];
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            const int slot_out = b + c;
             const bool live = row < rows_here;
-            const int s = grow / p.heads, hd = grow - s * p.heads;
-            const int64_t orow = ((int64_t)slot_out * p.s_q + s) * p.heads + hd;
+            const int64_t orow = (int64_t)(b + c) * p.rows_total + grow;  // slot b + c
             float *dst = p.o_part + orow * kLatent + 256 * rank + hf * 128;
 #pragma unroll 1
-            for (int c16 = 0; c16 < 128; c16 += 16) {  // loads by the whole warp, stores by live rows
-                uint32_t r[16];
-                tmem_ld16(t_o + lane_off + hf * 128 + c16, r);
+            for (int c32 = 0; c32 < 128; c32 += 32) {  // loads by the whole warp, stores by live rows
+                uint32_t r[32];
+                tmem_ld32(t_o + lane_off + hf * 128 + c32, r);
                 tmem_wait_ld();
                 if (live) {
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *reinterpret_cast<float4 *>(dst + c16 + e) =
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst + c32 + e) =
                             make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
                                         __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
                 }
@@ -520,7 +571,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                        ? (m_run + __log2f(l)) * 0.6931471805599453f
                                        : -INFINITY;
             tc_fence_before();
-            softmax_bar();  // O may be overwritten by the next piece's first PV
             GQLA_SPAN_END(16, t_epi);
             ++k;
         }
@@ -536,31 +586,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // no remote access may target a CTA that has exited
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 // 2D bf16 map over [rows][576] with a box of `box_cols` x `box_rows`.
-bool make_map_2d(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_cols,
-                 uint32_t box_rows, CUtensorMapSwizzle swizzle) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)kRow, rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kRow * 2};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+bool make_row_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_cols,
+                  uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    const uint64_t dims[2] = {(uint64_t)kRow, rows};
+    const uint64_t strides[1] = {(uint64_t)kRow * 2};
+    const uint32_t box[2] = {box_cols, box_rows};
+    return make_bf16_map(map, base, 2, dims, strides, box, swizzle);
 }
 
 }  // namespace
@@ -568,17 +600,17 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box
 cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
                                  const gqla_kv_index *idx, int num_splits, float scale,
                                  float *o_part, float *lse_part, void *ws, cudaStream_t stream) {
-    CUtensorMap lat, rope, qlat, qrope;
+    CUtensorMap lat, rope, qrope;
     const uint64_t slots = (uint64_t)idx->num_pages * kPage;
     const uint64_t qrows = (uint64_t)idx->batch * s_q * heads;
-    if (!make_map_2d(&lat, cache, slots, 64, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&rope, cache, slots, 32, kT, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_2d(&qlat, qa, qrows, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&qrope, qa, qrows, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_row_map(&lat, cache, slots, 64, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_row_map(&rope, cache, slots, 32, kT, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_row_map(&qrope, qa, qrows, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     AbsorbParams p;
     p.page_table = idx->page_table;
     p.seqlens = idx->seqlens;
+    p.qa = static_cast<const __nv_bfloat16 *>(qa);
     p.o_part = o_part;
     p.lse_part = lse_part;
     p.ws = ws;
@@ -595,7 +627,7 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, AbsorbSmem::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)num_splits * p.row_blocks * 2;
-    decode_absorb_tc_kernel<<<grid, kThreads, AbsorbSmem::kAlloc, stream>>>(lat, rope, qlat, qrope, p);
+    decode_absorb_tc_kernel<<<grid, kThreads, AbsorbSmem::kAlloc, stream>>>(lat, rope, qrope, p);
     return cudaGetLastError();
 }
 

@@ -23,12 +23,12 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// Tiled bf16 map of `rank` (2 or 3) dimensions: dims[0] is the contiguous
-// one, strides_bytes[i] is the byte stride of dims[i + 1].  Out-of-range
-// elements of a box read as zero.
-inline bool make_bf16_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
-                          const uint64_t *strides_bytes, const uint32_t *box,
-                          CUtensorMapSwizzle swizzle) {
+// Tiled map of `rank` (2 or 3) dimensions: dims[0] is the contiguous one,
+// strides_bytes[i] is the byte stride of dims[i + 1].  Out-of-range elements
+// of a box read as zero; a store drops them.
+inline bool make_map(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, int rank,
+                     const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                     CUtensorMapSwizzle swizzle) {
     auto fn = tensor_map_encoder();
     if (!fn || rank < 2 || rank > 3) return false;
     cuuint64_t d[3], s[2];
@@ -38,9 +38,16 @@ inline bool make_bf16_map(CUtensorMap *map, const void *base, int rank, const ui
         b[i] = box[i];
     }
     for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), d, s, b, e,
+    return fn(map, dtype, rank, const_cast<void *>(base), d, s, b, e,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool make_bf16_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                          const uint64_t *strides_bytes, const uint32_t *box,
+                          CUtensorMapSwizzle swizzle) {
+    return make_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box,
+                    swizzle);
 }
 
 }  // namespace gqla
