@@ -20,13 +20,13 @@
 //    holds O (256 columns), a double-buffered S (2 x 64) and the latent half
 //    of q~ (128 columns of bf16 pairs), so the score MMA reads q~ from TMEM;
 //    P goes through shared memory, beside a 4-slot ring of cache tiles.
-//    Roles, 352 threads:
+//    Roles, 19 warps:
 //      warp 0      TMA producer: the RoPE columns of q~ (once per piece) and
 //                  the ring (4 latent boxes 128B-swizzled + 1 RoPE box
 //                  64B-swizzled, 36 KB per 64-token tile);
 //      warp 1      TMEM owner, issues S = q~ C^T (latent part with A in TMEM);
-//      warps 2-9   online softmax, two warps per TMEM lane quadrant, each
-//                  taking 32 of the tile's 64 tokens: the fp16 partial
+//      warps 2-17  online softmax, four warps per TMEM lane quadrant, each
+//                  taking 16 of the tile's 64 tokens: the fp16 partial
 //                  scores go straight from registers into the peer CTA's
 //                  receive buffer with st.async (completing on the peer's
 //                  mbarrier), row maxima (lazy rescaling of O rows when a
@@ -34,7 +34,7 @@
 //                  memory (bf16, 128B-swizzled, the PV MMA's A operand).  Tile
 //                  i + 1's partial is sent before tile i is finished when its
 //                  scores are already available;
-//      warp 10     issues O += P C in tile order.
+//      warp 18     issues O += P C in tile order.
 //  * Per piece the softmax warps first copy the latent half of q~ from global
 //    memory into TMEM, and end with O / l written from TMEM to the partials.
 //  * Every wait is bounded and reports GQLA_ERR_TIMEOUT instead of hanging;
@@ -53,27 +53,32 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 352;
+constexpr int kSmWarps = 16;                // softmax warps: kParts per TMEM lane quadrant
+constexpr int kParts = kSmWarps / 4;
+constexpr int kThreads = 32 * (3 + kSmWarps);
+constexpr int kPvWarp = 2 + kSmWarps;       // warp issuing O += P C
 constexpr int kRows = 128;           // MMA M: query rows of one row block (zero-padded)
 constexpr int kT = 64;               // tokens per tile (one page)
 constexpr int kRing = 4;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kTokW = kT / kParts;          // tokens of a tile per softmax warp
+constexpr int kSmThreads = 32 * kSmWarps;
 
 struct AbsorbSmem {
     static constexpr int kQRope = kRows * 64;             // q~ RoPE columns [128 rows][32]
     static constexpr int kLatBox = kT * 128;              // [64 tokens][64 cols]
     static constexpr int kRopeBox = kT * 64;              // [64 tokens][32 cols]
     static constexpr int kSlot = 4 * kLatBox + kRopeBox;  // 36 KB
-    static constexpr int kX = kRows * kT * 2;             // fp16 partial scores, [8 warps][32 rows][32]
-    static constexpr int kXw = kX / 8;                    // one warp's block
+    static constexpr int kX = kRows * kT * 2;             // fp16 partial scores, [warps][32 rows][kTokW]
+    static constexpr int kXw = kX / kSmWarps;             // one warp's block
     static constexpr int kP = kRows * kT * 2;             // P, [128 rows][64 tokens] bf16, 128B-swizzled
     static constexpr int oQ = 0;
     static constexpr int oP = oQ + kQRope;                // 2 buffers
     static constexpr int oRing = oP + 2 * kP;
     static constexpr int oX = oRing + kRing * kSlot;      // the peer's partials (2 buffers)
-    static constexpr int oRm = oX + 2 * kX;               // float [2 tiles][2 halves][128 rows]
-    static constexpr int oL = oRm + 4 * kRows * 4;        // float [2 halves][128 rows]
-    static constexpr int oBar = oL + 2 * kRows * 4;
+    static constexpr int oRm = oX + 2 * kX;               // float [2 tiles][kParts][128 rows]
+    static constexpr int oL = oRm + 2 * kParts * kRows * 4;  // float [kParts][128 rows]
+    static constexpr int oBar = oL + kParts * kRows * 4;
     // ring_full/empty[3], q_full, q_empty, s_full/s_free[2], p_full/p_free[2],
     // x_full/x_empty[2], o_done, drain[2]
     static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 4 + 1 + 2;
@@ -116,8 +121,8 @@ __device__ __forceinline__ bool next_piece(const AbsorbParams &p, PieceIter &it,
     return false;
 }
 
-__device__ __forceinline__ void pair_bar(int quad) {  // the two softmax warps of one lane quadrant
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+__device__ __forceinline__ void quad_bar(int quad) {  // the softmax warps of one lane quadrant
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "n"(32 * kParts) : "memory");
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -150,12 +155,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i) { mbar_init(&ring_full[i], 1); mbar_init(&ring_empty[i], 1); }
-        mbar_init(q_full, 1 + 8);  // RoPE TMA + the 8 softmax warps' TMEM copies
-        mbar_init(q_empty, 8);
+        mbar_init(q_full, 1 + kSmWarps);  // RoPE TMA + the softmax warps' TMEM copies
+        mbar_init(q_empty, kSmWarps);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 256);
-            mbar_init(&p_full[i], 256); mbar_init(&p_free[i], 1);
-            mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 8);
+            mbar_init(&s_full[i], 1); mbar_init(&s_free[i], kSmThreads);
+            mbar_init(&p_full[i], kSmThreads); mbar_init(&p_free[i], 1);
+            mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], kSmWarps);
             mbar_init(&drain[i], 1);
         }
         mbar_init(o_done, 1);
@@ -290,7 +295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int dummy = 0;
             mbar_wait(&drain[0], 0, reinterpret_cast<volatile int *>(&dummy));
         }
-    } else if (warp == 10) {
+    } else if (warp == kPvWarp) {
         // ---------------------------------------------------------------- PV MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_pv = idesc_bf16(kRows, 256, 0, 1);
@@ -326,17 +331,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
+        constexpr int kPr = kTokW / 2;           // fp16 pairs of a warp's tokens
         const int quad = warp & 3;               // TMEM lane quadrant
-        const int hf = (warp - 2) >> 2;          // which 32 tokens of the tile
+        const int w = warp - 2;                  // softmax warp index: its block of a buffer
+        const int part = w >> 2;                 // which kTokW tokens of the tile
         const int row = 32 * quad + lane;        // query row of the row block (= TMEM lane)
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         const int grow = rb * kRows + row;       // row within the sequence's s_q * h rows
         const int s_of_row = grow < p.rows_total ? grow / p.heads : p.s_q - 1;
         float *rm = reinterpret_cast<float *>(smem + SM::oRm);
         float *lsm = reinterpret_cast<float *>(smem + SM::oL);
-        const int w8 = warp - 2;                 // softmax warp index: its 2 KB block of a buffer
         const uint8_t *xbuf = smem + SM::oX;
-        const uint32_t x_remote = map_peer(smem_u32(smem + SM::oX), peer) + w8 * SM::kXw + lane * 64;
+        const uint32_t x_remote =
+            map_peer(smem_u32(smem + SM::oX), peer) + w * SM::kXw + lane * (kTokW * 2);
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
         const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
         const __half2 scale2 = __float2half2_rn(p.scale_log2);
@@ -346,27 +353,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t t = 0, k = 0;
         while (next_piece(p, it, b, L, pb, pe, too_long)) {
             if (too_long) continue;
-            float m_run = -INFINITY, l_run = 0.0f;  // this row, this warp's half of every tile
+            float m_run = -INFINITY, l_run = 0.0f;  // this row, this warp's tokens of every tile
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             // query s of this row sees tokens t <= L - s_q + s
             const int last_visible = L - p.s_q + s_of_row;
             const uint32_t t0 = t;
             const int nt = pe - pb;
-            // ---- this warp's quarter of q~'s latent half (its 32 rows x 128 columns) into TMEM;
-            // the previous piece's scores, the last readers of that TMEM, are complete
+            // ---- this warp's share of q~'s latent half (its 32 rows x 256/kParts columns)
+            // into TMEM; the previous piece's scores, its last readers, are complete
             {
+                constexpr int kQc = 256 / kParts;  // bf16 columns per warp
                 const uint4 *src = reinterpret_cast<const uint4 *>(
-                    p.qa + ((int64_t)b * p.rows_total + grow) * kRow + 256 * rank + hf * 128);
+                    p.qa + ((int64_t)b * p.rows_total + grow) * kRow + 256 * rank + part * kQc);
                 const bool live = row < rows_here;
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    uint32_t w[16];
+                for (int h = 0; h < kQc / 32; ++h) {
+                    uint32_t wv[16];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint4 v = live ? src[4 * h + j] : make_uint4(0, 0, 0, 0);
-                        w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+                        wv[4 * j] = v.x; wv[4 * j + 1] = v.y; wv[4 * j + 2] = v.z; wv[4 * j + 3] = v.w;
                     }
-                    tmem_st16(t_q + lane_off + hf * 64 + 16 * h, w);
+                    tmem_st16(t_q + lane_off + part * (kQc / 2) + 16 * h, wv);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -374,31 +382,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(q_full);
             }
             // stage A of tile i: this warp's partial scores -> fp16 -> the peer's receive buffer
-            auto stage_a = [&](int i, uint32_t (&h2)[16]) {
+            auto stage_a = [&](int i, uint32_t (&h2)[kPr]) {
                 const uint32_t tt = t0 + i;
                 const int sb = tt & 1;
                 if (!GQLA_WAIT(6, &s_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
                 tc_fence_after();
-                uint32_t sv[32];
-                tmem_ld32(t_s + lane_off + sb * kT + hf * 32, sv);
+                uint32_t sv[kTokW];
+#pragma unroll
+                for (int c16 = 0; c16 < kTokW; c16 += 16)
+                    tmem_ld16(t_s + lane_off + sb * kT + part * kTokW + c16, sv + c16);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&s_free[sb]);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < kPr; ++j) {
                     __half2 v = __floats2half2_rn(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
                     h2[j] = *reinterpret_cast<uint32_t *>(&v);
                 }
-                if (w8 == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kX);
+                if (w == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kX);
                 // the peer's receive buffer sb is free once it has read tile tt - 2
                 if (!GQLA_WAITC(7, &x_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < kPr / 4; ++j)
                     st_async_v4(x_remote + sb * SM::kX + 16 * j,
                                 make_uint4(h2[4 * j], h2[4 * j + 1], h2[4 * j + 2], h2[4 * j + 3]),
                                 xfull_remote + sb * 8);
             };
-            uint32_t hc[16];
+            uint32_t hc[kPr];
             stage_a(0, hc);
             bool have_next = false;  // stage A of tile i + 1 already done
             int page = prow[pb];
@@ -406,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // Tile i + 1's exchange is started early only when its scores are
                 // already there: waiting for them here would tie the release of
                 // tile i (and of its ring slot) to the arrival of the next tile.
-                uint32_t hn[16];
+                uint32_t hn[kPr];
                 const bool next_ready =
                     i + 1 < nt && __shfl_sync(0xffffffffu,  // one decision per warp
                                               (int)mbar_test_wait(&s_full[(t0 + i + 1) & 1], ((t0 + i + 1) >> 1) & 1), 0);
@@ -424,12 +434,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 GQLA_SPAN_BEGIN(t_tile);
                 // ---- full raw scores = own + peer (the same rounded partials in both CTAs)
                 if (!GQLA_WAITC(8, &x_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
-                __half2 x[16];
+                __half2 x[kPr];
                 GQLA_SPAN_BEGIN(b1);
                 {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(xbuf + sb * SM::kX + w8 * SM::kXw + lane * 64);
+                    const uint4 *src =
+                        reinterpret_cast<const uint4 *>(xbuf + sb * SM::kX + w * SM::kXw + lane * (kTokW * 2));
 #pragma unroll
-                    for (int j4 = 0; j4 < 4; ++j4) {
+                    for (int j4 = 0; j4 < kPr / 4; ++j4) {
                         const uint4 pv = src[j4];
                         const uint32_t pw4[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
@@ -444,26 +455,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 GQLA_SPAN_END(20, b1);
                 GQLA_SPAN_BEGIN(b2);
                 // ---- mask tokens past the sequence or past this query's causal limit
-                const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + hf * 32);  // last visible index here
-                if (lim < 31) {
+                const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + part * kTokW);
+                if (lim < kTokW - 1) {
                     const __half ninf = __ushort_as_half((unsigned short)0xFC00u);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
+                    for (int j = 0; j < kPr; ++j) {
                         if (2 * j > lim) x[j].x = ninf;
                         if (2 * j + 1 > lim) x[j].y = ninf;
                     }
                 }
-                // ---- row maximum over the 64 tokens (pair exchange)
-                __half2 hm8[8];
+                // ---- row maximum over the 64 tokens (exchange among the quadrant's warps)
+                __half2 hm;
+                {
+                    __half2 tr[kPr];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) hm8[j] = __hmax2(x[j], x[j + 8]);
+                    for (int j = 0; j < kPr; ++j) tr[j] = x[j];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) hm8[j] = __hmax2(hm8[j], hm8[j + 4]);
-                const __half2 hm = __hmax2(__hmax2(hm8[0], hm8[2]), __hmax2(hm8[1], hm8[3]));
+                    for (int st = kPr / 2; st >= 1; st >>= 1)
+#pragma unroll
+                        for (int j = 0; j < st; ++j) tr[j] = __hmax2(tr[j], tr[j + st]);
+                    hm = tr[0];
+                }
                 const float mx = fmaxf(__low2float(hm), __high2float(hm)) * p.scale_log2;  // log2 units
-                rm[(tt & 1) * 2 * kRows + hf * kRows + row] = mx;
-                pair_bar(quad);
-                const float mt = fmaxf(mx, rm[(tt & 1) * 2 * kRows + (hf ^ 1) * kRows + row]);
+                rm[((tt & 1) * kParts + part) * kRows + row] = mx;
+                quad_bar(quad);
+                float mt = mx;
+#pragma unroll
+                for (int q = 0; q < kParts; ++q) mt = fmaxf(mt, rm[((tt & 1) * kParts + q) * kRows + row]);
                 GQLA_SPAN_END(21, b2);
                 const bool first = i == 0;
                 float m_new = m_run;
@@ -480,9 +498,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         if (!mbar_wait(&p_free[sb ^ 1], ((tt - 1) >> 1) & 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
 #pragma unroll 1
-                    for (int c16 = 0; c16 < 128; c16 += 16) {  // this warp's 128 of the 256 O columns
+                    for (int c16 = 0; c16 < 256 / kParts; c16 += 16) {  // this warp's share of the O columns
                         uint32_t r[16];
-                        const uint32_t ta = t_o + lane_off + hf * 128 + c16;
+                        const uint32_t ta = t_o + lane_off + part * (256 / kParts) + c16;
                         tmem_ld16(ta, r);
                         tmem_wait_ld();
 #pragma unroll
@@ -494,13 +512,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 l_run = first ? 0.0f : l_run * alpha;
                 m_run = m_new;
                 // ---- P = 2^(x scale - m), two tokens per fp16 ex2, in bf16 into shared
-                // memory (this warp's 32 tokens = bytes [64 hf, 64 hf + 64) of the row)
+                // memory (this warp's tokens = bytes [2 kTokW part, 2 kTokW (part + 1)) of the row)
                 GQLA_SPAN_BEGIN(b3);
                 const __half2 mneg2 = __float2half2_rn(m_run == -INFINITY ? 0.0f : -m_run);
-                uint32_t pw[16];
+                uint32_t pw[kPr];
                 float lsum = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < kPr; ++j) {
                     const float2 pf = __half22float2(fast_exp2_h2(__hfma2(x[j], scale2, mneg2)));
                     __nv_bfloat162 hb = __floats2bfloat162_rn(pf.x, pf.y);
                     pw[j] = *reinterpret_cast<uint32_t *>(&hb);
@@ -512,8 +530,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 {
                     uint8_t *prow_s = smem + SM::oP + sb * SM::kP + row * 128;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4 *>(prow_s + (((hf * 4 + j) ^ (row & 7)) << 4)) =
+                    for (int j = 0; j < kPr / 4; ++j)
+                        *reinterpret_cast<uint4 *>(prow_s + (((part * (kPr / 4) + j) ^ (row & 7)) << 4)) =
                             make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
                 }
                 // latent rows that are not tokens (never written, maybe NaN) -> 0
@@ -521,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (!mbar_wait(&ring_full[slot], (tt / kRing) & 1, abort_flag)) *abort_flag = 1;
                     uint8_t *tile = smem + SM::oRing + slot * SM::kSlot;
                     const int nz = kT - n_valid;
-                    for (int z = w8 * 32 + lane; z < 4 * nz * 8; z += 256) {
+                    for (int z = w * 32 + lane; z < 4 * nz * 8; z += kSmThreads) {
                         const int box = z / (nz * 8), rem = z % (nz * 8);
                         *reinterpret_cast<uint4 *>(tile + box * SM::kLatBox + (n_valid + rem / 8) * 128 +
                                                    (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
@@ -536,27 +554,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 have_next = false;
                 page = page_next;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) hc[j] = hn[j];
+                for (int j = 0; j < kPr; ++j) hc[j] = hn[j];
             }
             t = t0 + nt;
             // the last scores of the piece are read: the producer may load the next RoPE q~
             __syncwarp();
             if (lane == 0) mbar_arrive(q_empty);
-            // ---- epilogue: O / l for this CTA's 256 columns (this warp: 128), LSE by rank 0
+            // ---- epilogue: O / l for this CTA's 256 columns (this warp: 256 / kParts), LSE by rank 0
             GQLA_SPAN_BEGIN(t_epi);
             if (!GQLA_WAIT(15, o_done, k & 1, abort_flag)) *abort_flag = 1;
             tc_fence_after();
-            lsm[hf * kRows + row] = l_run;
-            pair_bar(quad);
-            const float l = l_run + lsm[(hf ^ 1) * kRows + row];
+            lsm[part * kRows + row] = l_run;
+            quad_bar(quad);
+            float l = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kParts; ++q) l += lsm[q * kRows + row];
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
             const bool live = row < rows_here;
             const int64_t orow = (int64_t)(b + c) * p.rows_total + grow;  // slot b + c
-            float *dst = p.o_part + orow * kLatent + 256 * rank + hf * 128;
+            float *dst = p.o_part + orow * kLatent + 256 * rank + part * (256 / kParts);
 #pragma unroll 1
-            for (int c32 = 0; c32 < 128; c32 += 32) {  // loads by the whole warp, stores by live rows
+            for (int c32 = 0; c32 < 256 / kParts; c32 += 32) {  // loads by the whole warp, stores by live rows
                 uint32_t r[32];
-                tmem_ld32(t_o + lane_off + hf * 128 + c32, r);
+                tmem_ld32(t_o + lane_off + part * (256 / kParts) + c32, r);
                 tmem_wait_ld();
                 if (live) {
 #pragma unroll
@@ -566,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                         __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
                 }
             }
-            if (live && rank == 0 && hf == 0)
+            if (live && rank == 0 && part == 0)
                 p.lse_part[orow] = (l > 0.0f && m_run != -INFINITY)
                                        ? (m_run + __log2f(l)) * 0.6931471805599453f
                                        : -INFINITY;

@@ -83,17 +83,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 #ifdef GQLA_WAIT_PROFILE
 __device__ unsigned long long g_wait_cycles[32];
 __device__ unsigned long long g_wait_count[32];
-// per-warp accumulators in shared memory (lane 0 of each warp writes its own row)
+// per-warp accumulators in shared memory (lane 0 of each warp writes its own
+// row; kernels of up to 20 warps)
 #define GQLA_PROF_DECL                                                       \
-    __shared__ unsigned long long gqla_prof_c_[11][24];                     \
-    __shared__ unsigned int gqla_prof_n_[11][24];                           \
+    __shared__ unsigned int gqla_prof_c_[20][24];                           \
+    __shared__ unsigned int gqla_prof_n_[20][24];                           \
     if ((threadIdx.x & 31) == 0)                                            \
         for (int i_ = 0; i_ < 24; ++i_)                                     \
             gqla_prof_c_[threadIdx.x >> 5][i_] = 0, gqla_prof_n_[threadIdx.x >> 5][i_] = 0
 #define GQLA_PROF_ADD(site, dt)                                              \
     do {                                                                     \
         if ((threadIdx.x & 31) == 0) {                                       \
-            gqla_prof_c_[threadIdx.x >> 5][site] += (dt);                    \
+            gqla_prof_c_[threadIdx.x >> 5][site] += (unsigned int)(dt);      \
             gqla_prof_n_[threadIdx.x >> 5][site] += 1;                       \
         }                                                                    \
     } while (0)
@@ -118,7 +119,8 @@ __device__ unsigned long long g_wait_count[32];
         if ((threadIdx.x & 31) == 0)                                                        \
             for (int i_ = 0; i_ < 24; ++i_)                                                 \
                 if (gqla_prof_n_[threadIdx.x >> 5][i_]) {                                   \
-                    atomicAdd(&::gqla::sm100::g_wait_cycles[i_], gqla_prof_c_[threadIdx.x >> 5][i_]); \
+                    atomicAdd(&::gqla::sm100::g_wait_cycles[i_],                            \
+                              (unsigned long long)gqla_prof_c_[threadIdx.x >> 5][i_]);      \
                     atomicAdd(&::gqla::sm100::g_wait_count[i_],                             \
                               (unsigned long long)gqla_prof_n_[threadIdx.x >> 5][i_]);      \
                 }                                                                           \
