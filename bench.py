@@ -472,6 +472,30 @@ def run_reference(args, rank, world):
     }
 
 
+def ncu_summary(csv_path):
+    """Per-kernel launch count, total and share of device time from an ncu
+    `--metrics gpu__time_duration.sum --csv` launch list (host-side only)."""
+    import collections
+    import csv
+    rows = [r for r in csv.reader(open(csv_path)) if len(r) > 5]
+    idx = {h: i for i, h in enumerate(rows[0])}
+    agg = collections.defaultdict(lambda: [0, 0.0])
+    for r in rows[1:]:
+        if r[idx["Metric Name"]] != "gpu__time_duration.sum":
+            continue
+        name = r[idx["Kernel Name"]].split("(")[0].replace("void ", "")
+        for junk in ("(anonymous namespace)::", "<unnamed>::", "unnamed>::"):
+            name = name.replace(junk, "")
+        scale = {"ns": 1e-3, "us": 1.0, "usecond": 1.0, "nsecond": 1e-3, "ms": 1e3,
+                 "msecond": 1e3}.get(r[idx["Metric Unit"]], 1.0)
+        agg[name[:80]][0] += 1
+        agg[name[:80]][1] += float(r[idx["Metric Value"]].replace(",", "")) * scale
+    total = sum(v[1] for v in agg.values())
+    print(f"{'launches':>8} {'total us':>11} {'share':>7}  kernel")
+    for k, (n, t) in sorted(agg.items(), key=lambda x: -x[1][1]):
+        print(f"{n:8d} {t:11.1f} {100 * t / total:6.1f}%  {k}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,7 +507,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ncu-summary", metavar="CSV", default=None,
+                    help="print the per-kernel summary of an ncu launch list and exit")
     args = ap.parse_args()
+    if args.ncu_summary:
+        ncu_summary(args.ncu_summary)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
