@@ -35,8 +35,9 @@
 //                  i + 1's partial is sent before tile i is finished when its
 //                  scores are already available;
 //      warp 18     issues O += P C in tile order.
-//  * Per piece the softmax warps first copy the latent half of q~ from global
-//    memory into TMEM, and end with O / l written from TMEM to the partials.
+//  * The softmax warps copy each piece's latent half of q~ from global memory
+//    into TMEM as soon as the previous piece's scores are done, and write
+//    O / l with TMA stores staged in the (then idle) P buffers.
 //  * Every wait is bounded and reports GQLA_ERR_TIMEOUT instead of hanging;
 //    both CTAs of a cluster always execute the same sequence of steps.
 #include <cudaTypedefs.h>
@@ -125,10 +126,15 @@ __device__ __forceinline__ void quad_bar(int quad) {  // the softmax warps of on
     asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "n"(32 * kParts) : "memory");
 }
 
+__device__ __forceinline__ void softmax_bar() {  // all softmax warps
+    asm volatile("bar.sync 5, %0;" ::"n"(kSmThreads) : "memory");
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_absorb_tc_kernel(const __grid_constant__ CUtensorMap lat_map,
                             const __grid_constant__ CUtensorMap rope_map,
-                            const __grid_constant__ CUtensorMap qrope_map, const AbsorbParams p) {
+                            const __grid_constant__ CUtensorMap qrope_map,
+                            const __grid_constant__ CUtensorMap o_map, const AbsorbParams p) {
     using SM = AbsorbSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -347,6 +353,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
         const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
         const __half2 scale2 = __float2half2_rn(p.scale_log2);
+        // ---- this warp's share of q~'s latent half (its 32 rows x 256/kParts columns)
+        // into TMEM; the previous piece's scores, its last readers, are complete
+        auto copy_q = [&](int bq) {
+            constexpr int kQc = 256 / kParts;  // bf16 columns per warp
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.qa + ((int64_t)bq * p.rows_total + grow) * kRow + 256 * rank + part * kQc);
+            const bool live = row < rows_here;
+#pragma unroll
+            for (int h = 0; h < kQc / 32; ++h) {
+                uint32_t wv[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = live ? src[4 * h + j] : make_uint4(0, 0, 0, 0);
+                    wv[4 * j] = v.x; wv[4 * j + 1] = v.y; wv[4 * j + 2] = v.z; wv[4 * j + 3] = v.w;
+                }
+                tmem_st16(t_q + lane_off + part * (kQc / 2) + 16 * h, wv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_full);
+        };
+        const bool quad_live = 32 * quad < rows_here;  // rows_here is a multiple of 32
+        uint8_t *stg = smem + SM::oP + w * 2048;       // epilogue staging: [32 rows][16 fp32]
+        bool q_loaded = false;                         // q~ of the coming piece already in TMEM
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
@@ -359,28 +390,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int last_visible = L - p.s_q + s_of_row;
             const uint32_t t0 = t;
             const int nt = pe - pb;
-            // ---- this warp's share of q~'s latent half (its 32 rows x 256/kParts columns)
-            // into TMEM; the previous piece's scores, its last readers, are complete
-            {
-                constexpr int kQc = 256 / kParts;  // bf16 columns per warp
-                const uint4 *src = reinterpret_cast<const uint4 *>(
-                    p.qa + ((int64_t)b * p.rows_total + grow) * kRow + 256 * rank + part * kQc);
-                const bool live = row < rows_here;
-#pragma unroll
-                for (int h = 0; h < kQc / 32; ++h) {
-                    uint32_t wv[16];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint4 v = live ? src[4 * h + j] : make_uint4(0, 0, 0, 0);
-                        wv[4 * j] = v.x; wv[4 * j + 1] = v.y; wv[4 * j + 2] = v.z; wv[4 * j + 3] = v.w;
-                    }
-                    tmem_st16(t_q + lane_off + part * (kQc / 2) + 16 * h, wv);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(q_full);
-            }
+            if (!q_loaded) copy_q(b);
+            q_loaded = false;
             // stage A of tile i: this warp's partial scores -> fp16 -> the peer's receive buffer
             auto stage_a = [&](int i, uint32_t (&h2)[kPr]) {
                 const uint32_t tt = t0 + i;
@@ -557,10 +568,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < kPr; ++j) hc[j] = hn[j];
             }
             t = t0 + nt;
-            // the last scores of the piece are read: the producer may load the next RoPE q~
+            // the last scores of the piece are read: the producer may load the next RoPE q~,
+            // and the next piece's q~ goes into TMEM now, so that its scores overlap this epilogue
             __syncwarp();
             if (lane == 0) mbar_arrive(q_empty);
-            // ---- epilogue: O / l for this CTA's 256 columns (this warp: 256 / kParts), LSE by rank 0
+            {
+                PieceIter nx = it;
+                int b2, L2, pb2, pe2;
+                bool tl2 = false, more;
+                do {
+                    more = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
+                } while (more && tl2);
+                if (more) {
+                    copy_q(b2);
+                    q_loaded = true;
+                }
+            }
+            // ---- epilogue: O / l for this CTA's 256 columns (this warp: 256 / kParts) through
+            // TMA stores staged in this warp's 2 KB of the P buffers (free once the piece's
+            // last PV is done), LSE by rank 0
             GQLA_SPAN_BEGIN(t_epi);
             if (!GQLA_WAIT(15, o_done, k & 1, abort_flag)) *abort_flag = 1;
             tc_fence_after();
@@ -572,20 +598,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
             const bool live = row < rows_here;
             const int64_t orow = (int64_t)(b + c) * p.rows_total + grow;  // slot b + c
-            float *dst = p.o_part + orow * kLatent + 256 * rank + part * (256 / kParts);
+            const int orow0 = (b + c) * p.rows_total + rb * kRows + 32 * quad;
 #pragma unroll 1
-            for (int c32 = 0; c32 < 256 / kParts; c32 += 32) {  // loads by the whole warp, stores by live rows
-                uint32_t r[32];
-                tmem_ld32(t_o + lane_off + part * (256 / kParts) + c32, r);
+            for (int j = 0; j < 256 / kParts / 16; ++j) {
+                if (j > 0) {
+                    if (lane == 0) bulk_wait_group_read<0>();  // the previous chunk's store has read stg
+                    __syncwarp();
+                }
+                uint32_t r[16];
+                tmem_ld16(t_o + lane_off + part * (256 / kParts) + 16 * j, r);
                 tmem_wait_ld();
-                if (live) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(dst + c32 + e) =
-                            make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
-                                        __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+                for (int q4 = 0; q4 < 4; ++q4)  // 64-byte swizzle: chunk ^= (row / 2) % 4
+                    *reinterpret_cast<float4 *>(stg + lane * 64 + ((q4 ^ ((lane >> 1) & 3)) << 4)) =
+                        make_float4(__uint_as_float(r[4 * q4]) * inv, __uint_as_float(r[4 * q4 + 1]) * inv,
+                                    __uint_as_float(r[4 * q4 + 2]) * inv, __uint_as_float(r[4 * q4 + 3]) * inv);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && quad_live && !*abort_flag) {
+                    tma_store_2d(&o_map, stg, 256 * (int)rank + part * (256 / kParts) + 16 * j, orow0);
+                    bulk_commit_group();
                 }
             }
+            if (lane == 0) bulk_wait_group_read<0>();
+            // every warp's staging (spread over all the P rows) is read before any P is rewritten
+            softmax_bar();
             if (live && rank == 0 && part == 0)
                 p.lse_part[orow] = (l > 0.0f && m_run != -INFINITY)
                                        ? (m_run + __log2f(l)) * 0.6931471805599453f
@@ -594,6 +631,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             GQLA_SPAN_END(16, t_epi);
             ++k;
         }
+        if (lane == 0) bulk_wait_group<0>();  // the partials are written before the CTA exits
     }
 
     GQLA_PROF_FLUSH;
@@ -620,13 +658,22 @@ bool make_row_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t bo
 cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
                                  const gqla_kv_index *idx, int num_splits, float scale,
                                  float *o_part, float *lse_part, void *ws, cudaStream_t stream) {
-    CUtensorMap lat, rope, qrope;
+    CUtensorMap lat, rope, qrope, omap;
     const uint64_t slots = (uint64_t)idx->num_pages * kPage;
     const uint64_t qrows = (uint64_t)idx->batch * s_q * heads;
     if (!make_row_map(&lat, cache, slots, 64, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_row_map(&rope, cache, slots, 32, kT, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_row_map(&qrope, qa, qrows, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
+    {
+        const uint64_t orows = (uint64_t)(idx->batch + num_splits) * s_q * heads;
+        const uint64_t dims[2] = {(uint64_t)kLatent, orows};
+        const uint64_t strides[1] = {(uint64_t)kLatent * 4};
+        const uint32_t box[2] = {16, 32};
+        if (!make_map(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, o_part, 2, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
+    }
     AbsorbParams p;
     p.page_table = idx->page_table;
     p.seqlens = idx->seqlens;
@@ -647,7 +694,7 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, AbsorbSmem::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)num_splits * p.row_blocks * 2;
-    decode_absorb_tc_kernel<<<grid, kThreads, AbsorbSmem::kAlloc, stream>>>(lat, rope, qrope, p);
+    decode_absorb_tc_kernel<<<grid, kThreads, AbsorbSmem::kAlloc, stream>>>(lat, rope, qrope, omap, p);
     return cudaGetLastError();
 }
 
