@@ -216,23 +216,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (lane == 0 && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
                 continue;
             }
-            // RoPE columns of q~ for this row block (the previous piece's scores are done)
-            if (lane == 0) {
-                if (!GQLA_WAIT(1, q_empty, (k & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                if (!*abort_flag) {
-                    const int row0 = b * p.rows_total + rb * kRows;
-                    mbar_arrive_expect_tx(q_full, SM::kQRope);
-                    tma_load_2d(smem + SM::oQ, &qrope_map, q_full, 512 + 32 * rank, row0);
-                } else {
-                    mbar_arrive(q_full);
+            // RoPE columns of q~ for this row block; they wait for the previous piece's
+            // scores, so up to kRing - 1 of this piece's tiles are issued first
+            const int rope_at = min(pe - pb, kRing - 1);
+            auto load_rope = [&]() {
+                if (lane == 0) {
+                    if (!GQLA_WAIT(1, q_empty, (k & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    if (!*abort_flag) {
+                        const int row0 = b * p.rows_total + rb * kRows;
+                        mbar_arrive_expect_tx(q_full, SM::kQRope);
+                        tma_load_2d(smem + SM::oQ, &qrope_map, q_full, 512 + 32 * rank, row0);
+                    } else {
+                        mbar_arrive(q_full);
+                    }
                 }
-            }
+            };
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             for (int i0 = pb; i0 < pe; i0 += 32) {
                 const int n = min(32, pe - i0);
                 const int my_page = lane < n ? prow[i0 + lane] : 0;
                 for (int j = 0; j < n; ++j, ++t) {
                     const int page = __shfl_sync(0xffffffffu, my_page, j);
+                    if (i0 - pb + j == rope_at) load_rope();
                     if (lane == 0) {
                         const bool bad = page < 0 || page >= p.num_pages;
                         if (bad && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
@@ -253,6 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            if (rope_at == pe - pb) load_rope();
             ++k;
         }
         if (lane == 0) {
@@ -352,7 +358,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             map_peer(smem_u32(smem + SM::oX), peer) + w * SM::kXw + lane * (kTokW * 2);
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
         const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
-        const __half2 scale2 = __float2half2_rn(p.scale_log2);
         // ---- this warp's share of q~'s latent half (its 32 rows x 256/kParts columns)
         // into TMEM; the previous piece's scores, its last readers, are complete
         auto copy_q = [&](int bq) {
@@ -496,8 +501,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 GQLA_SPAN_END(21, b2);
                 const bool first = i == 0;
                 float m_new = m_run;
-                // the running maximum is kept on the fp16 grid: P below subtracts it in fp16
-                if (first || mt > m_run + kRescaleLog2) m_new = __half2float(__float2half_rn(mt));
+                if (first || mt > m_run + kRescaleLog2) m_new = mt;
                 const bool need = !first && m_new != m_run;
                 const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;
                 // P buffer sb is free once PV(tt - 2) completed
@@ -522,18 +526,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 l_run = first ? 0.0f : l_run * alpha;
                 m_run = m_new;
-                // ---- P = 2^(x scale - m), two tokens per fp16 ex2, in bf16 into shared
-                // memory (this warp's tokens = bytes [2 kTokW part, 2 kTokW (part + 1)) of the row)
+                // ---- P = 2^(x scale - m) (fp32 ex2) in bf16 -- the top half of the fp32
+                // value, rounded towards zero; the row sum adds the same truncated values,
+                // so O / l stays unbiased -- into shared memory: bytes
+                // [2 kTokW part, 2 kTokW (part + 1)) of the row
                 GQLA_SPAN_BEGIN(b3);
-                const __half2 mneg2 = __float2half2_rn(m_run == -INFINITY ? 0.0f : -m_run);
+                const float mu = m_run == -INFINITY ? 0.0f : m_run;
                 uint32_t pw[kPr];
                 float lsum = 0.0f;
 #pragma unroll
                 for (int j = 0; j < kPr; ++j) {
-                    const float2 pf = __half22float2(fast_exp2_h2(__hfma2(x[j], scale2, mneg2)));
-                    __nv_bfloat162 hb = __floats2bfloat162_rn(pf.x, pf.y);
-                    pw[j] = *reinterpret_cast<uint32_t *>(&hb);
-                    lsum += pf.x + pf.y;
+                    const float2 xf = __half22float2(x[j]);
+                    const uint32_t p0 = __float_as_uint(fast_exp2(fmaf(xf.x, p.scale_log2, -mu)));
+                    const uint32_t p1 = __float_as_uint(fast_exp2(fmaf(xf.y, p.scale_log2, -mu)));
+                    pw[j] = __byte_perm(p0, p1, 0x7632);
+                    lsum += __uint_as_float(p0 & 0xFFFF0000u) + __uint_as_float(p1 & 0xFFFF0000u);
                 }
                 l_run += lsum;
                 GQLA_SPAN_END(22, b3);
