@@ -11,10 +11,10 @@
 //
 // Both kernels are bound by the read of the fp32 partials; they keep many
 // independent 16-byte loads in flight per thread.  The absorb path's
-// 512 -> 128 product runs on the tcgen05 tensor cores: a cluster of eight
-// CTAs splits the 512-long contraction, each merging an eighth of the latent
-// columns of its 128 rows, and the eight fp32 partial products are summed
-// through distributed shared memory.
+// 512 -> 128 product runs on the tcgen05 tensor cores: in a pair of CTAs each
+// merges half of the latent columns of a 64-row tile into bf16, one bulk copy
+// gathers both halves in the first CTA, and that CTA runs the whole K = 512
+// product.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -173,36 +173,34 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
 }
 
 // ---------------------------------------------------------------------------
-// MQA-absorb path (d_in = 512).  A cluster of 8 CTAs per tile of up to 128
-// rows of one group (bst pairs x G heads, as in the query absorption); CTA kq
-// of the cluster merges latent columns [64 kq, 64 kq + 64) of the tile's rows
-// and multiplies them by rows [64 kq, 64 kq + 64) of W_UV_g:
-//   Y_kq[128 x 128] = A_kq[128 x 64] * B_kq[64 x 128]   (tcgen05, fp32 in TMEM)
-// then CTA kq sums Y_0..Y_7 for rows [16 kq, 16 kq + 16) over DSMEM.
+// MQA-absorb path (d_in = 512).  A cluster of 2 CTAs per tile of up to 64 rows
+// of one group (bst pairs x G heads).  CTA kq merges latent columns
+// [256 kq, 256 kq + 256) of the tile's rows into bf16 (the MMA's A operand,
+// K-major, 128-byte swizzle); CTA 1 sends its half into CTA 0's shared memory
+// with one bulk copy, and CTA 0 runs the whole product
+//   out[64 x 128] = A[64 x 512] * W_UV_g[512 x 128]   (tcgen05 M = 64, fp32 in TMEM)
+// and writes the bf16 rows.
 // ---------------------------------------------------------------------------
-constexpr int kClCtas = 8;
-constexpr int kClCols = kLatent / kClCtas;  // 64 latent columns per CTA
 constexpr int kClThreads = 256;
-constexpr int kClMaxPairs = 32;  // bst <= 128 / 4
+constexpr int kClRows = 64;      // rows of a tile (MMA M)
+constexpr int kClMaxPairs = 32;  // bst <= 64 / 4 = 16
 constexpr int kClChunk = 32;     // partials whose weights are staged at a time
-constexpr int kYStride = 132;    // fp32 row pitch of the partial product (bank spread)
 
 struct ClSmem {
-    static constexpr int oA = 0;                       // [128 rows][64] bf16, SW128 K-major
-    static constexpr int oB = 16384;                   // 2 N blocks x [64 k][64 n] bf16, SW128
-    static constexpr int oW = 32768;                   // [32 partials][128 rows] fp32 weights
-    static constexpr int oY = 0;                       // [128][132] fp32, after the MMA
-    static constexpr int oRowM = 69632;                // [128] fp32 max lse
-    static constexpr int oRowInv = oRowM + 512;        // [128] fp32 1 / denominator
-    static constexpr int oPlan = oRowInv + 512;        // c0[32], c1[32], max partials
+    static constexpr int kAHalf = kClRows * 256 * 2;       // one CTA's 4 K blocks of A
+    static constexpr int oA = 0;                           // 8 K blocks x [64 rows][64] bf16
+    static constexpr int oB = 2 * kAHalf;                  // W_UV_g: 2 N blocks x [512 k][64 n] bf16
+    static constexpr int oStage = 0;                       // epilogue [64 rows][128] bf16, over A
+    static constexpr int oW = oB + 512 * 128 * 2;          // [32 partials][64 rows] fp32 weights
+    static constexpr int oRowInv = oW + kClChunk * kClRows * 4;
+    static constexpr int oPlan = oRowInv + kClRows * 4;    // c0[32], c1[32], max partials
     static constexpr int oBar = oPlan + 2 * kClMaxPairs * 4 + 16;
-    static constexpr int kBytes = oBar + 32;
+    static constexpr int kBytes = oBar + 40;
     static constexpr int kAlloc = kBytes + 1024;
 };
-static_assert(ClSmem::oW + 128 * kClChunk * 4 <= ClSmem::oRowM, "weights overlap");
-static_assert(ClSmem::oY + 128 * kYStride * 4 <= ClSmem::oRowM, "Y overlaps the row data");
+static_assert(ClSmem::kAlloc <= 227 * 1024, "shared memory");
 
-__global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads, 2)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     combine_latent_tc_kernel(const __grid_constant__ CUtensorMap wmap, CombineParams p, int bst) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -212,30 +210,36 @@ __global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads, 2)
     int *s_c0 = reinterpret_cast<int *>(smem + ClSmem::oPlan);
     int *s_c1 = s_c0 + kClMaxPairs;
     int *s_maxp = s_c1 + kClMaxPairs;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ClSmem::oBar);
-    uint64_t *done = full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 2);
+    uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + ClSmem::oBar);
+    uint64_t *b_full = a_full + 1;
+    uint64_t *done = a_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(a_full + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int kq = (int)cluster_rank();
+    const bool leader = kq == 0;
     const int tile = blockIdx.y, grp = blockIdx.z;
     const int bs0 = tile * bst;
     const int rows_in_tile = p.G * bst;
     const int64_t part_stride = (int64_t)p.s_q * p.heads;
 
     if (tid == 0) {
-        prefetch_tensormap(&wmap);
-        mbar_init(full, 1);
+        mbar_init(a_full, 1);
+        mbar_init(b_full, 1);
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_barrier_init();
-        mbar_arrive_expect_tx(full, 2 * kClCols * 128);
-        for (int nb = 0; nb < 2; ++nb)
-            tma_load_2d(smem + ClSmem::oB + nb * kClCols * 128, &wmap, full, nb * 64,
-                        grp * kLatent + kq * kClCols);
+        if (leader) {
+            prefetch_tensormap(&wmap);
+            mbar_arrive_expect_tx(b_full, 512 * 128 * 2);
+            for (int nb = 0; nb < 2; ++nb)
+                for (int kh = 0; kh < 2; ++kh)
+                    tma_load_2d(smem + ClSmem::oB + nb * 65536 + kh * 32768, &wmap, b_full, nb * 64,
+                                grp * kLatent + kh * 256);
+        }
     }
-    if (warp == 1) {
+    if (warp == 1 && leader) {
         tmem_alloc(tmem_slot, 128);
         tmem_relinquish();
     }
@@ -248,16 +252,15 @@ __global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads, 2)
         }
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised before any remote transfer
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
 
-    // ---- threads 0..127: one row each -- max LSE, then weights per chunk
+    // ---- threads 0..63: one row each -- max LSE, then weights per chunk
     float den = 0.0f, Mr = -INFINITY;
     const float *lse_row = p.lse_part;
     int np_r = 0;
     bool live_r = false;
-    if (tid < 128) {
+    if (tid < kClRows) {
         const int j = tid / p.G;
         live_r = tid < rows_in_tile && bs0 + j < p.bs_total;
         if (live_r) {
@@ -276,30 +279,29 @@ __global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads, 2)
         }
     }
 
-    // ---- merge: warp w owns rows 16w .. 16w+15 as 8 row pairs; lanes 0-15
-    // take the first row of a pair, 16-31 the second, 4 columns each.
-    const int sub = lane >> 4, c4 = (lane & 15) * 4;
-    float4 acc[8];
+    // ---- merge: warp w owns rows 8w .. 8w+7; lane j covers columns 4j and 128 + 4j of
+    // this CTA's 256 latent columns
+    float4 acc[8][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
     const float *src[8];
-    int npq[8];
+    int npr[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int r = 16 * warp + 2 * i;  // even row: both rows of the pair share the pair (bs)
+        const int r = 8 * warp + i;
         const int j = r / p.G;
         const bool live = r < rows_in_tile && bs0 + j < p.bs_total;
-        npq[i] = live ? s_c1[j] - s_c0[j] : 0;
+        npr[i] = live ? s_c1[j] - s_c0[j] : 0;
         const int bs = bs0 + j, b = bs / p.s_q, s = bs % p.s_q;
         src[i] = p.o_part +
-                 (((int64_t)(b + (live ? s_c0[j] : 0)) * p.s_q + s) * p.heads + grp * p.G + r % p.G + sub) *
+                 (((int64_t)(b + (live ? s_c0[j] : 0)) * p.s_q + s) * p.heads + grp * p.G + r % p.G) *
                      kLatent +
-                 kq * kClCols + c4;
+                 kq * 256 + lane * 4;
     }
     const int maxp = *s_maxp;
     for (int cb = 0; cb < maxp; cb += kClChunk) {
         __syncthreads();  // the previous chunk's weights are consumed
-        if (tid < 128) {
+        if (tid < kClRows) {
             float l[kClChunk];
 #pragma unroll
             for (int k = 0; k < kClChunk; ++k)
@@ -308,63 +310,87 @@ __global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads, 2)
             for (int k = 0; k < kClChunk; ++k) {
                 const float w = l[k] == -INFINITY ? 0.0f : __expf(l[k] - Mr);
                 den += w;
-                sW[k * 128 + tid] = w;  // [partial][row]: conflict-free
+                sW[k * kClRows + tid] = w;  // [partial][row]: conflict-free
             }
         }
         __syncthreads();
         const int n = min(kClChunk, maxp - cb);
-        for (int j0 = 0; j0 < n; j0 += 2) {
-            float4 v[2][8];
+#pragma unroll 1
+        for (int jj = 0; jj < n; ++jj) {
+            float4 v[8][2];
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj)
+            for (int i = 0; i < 8; ++i) {
+                const bool on = cb + jj < npr[i];
+                const float *q = src[i] + (int64_t)(cb + jj) * part_stride * kLatent;
+                v[i][0] = on ? ldg4(q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[i][1] = on ? ldg4(q + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    v[jj][i] = cb + j0 + jj < npq[i]
-                                   ? ldg4(src[i] + (int64_t)(cb + j0 + jj) * part_stride * kLatent)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < 8; ++i) {
+                const float wj = sW[jj * kClRows + 8 * warp + i];
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float wj = j0 + jj < n ? sW[(j0 + jj) * 128 + 16 * warp + 2 * i + sub] : 0.0f;
-                    acc[i].x = fmaf(wj, v[jj][i].x, acc[i].x);
-                    acc[i].y = fmaf(wj, v[jj][i].y, acc[i].y);
-                    acc[i].z = fmaf(wj, v[jj][i].z, acc[i].z);
-                    acc[i].w = fmaf(wj, v[jj][i].w, acc[i].w);
+                for (int h = 0; h < 2; ++h) {
+                    acc[i][h].x = fmaf(wj, v[i][h].x, acc[i][h].x);
+                    acc[i][h].y = fmaf(wj, v[i][h].y, acc[i][h].y);
+                    acc[i][h].z = fmaf(wj, v[i][h].z, acc[i][h].z);
+                    acc[i][h].w = fmaf(wj, v[i][h].w, acc[i][h].w);
                 }
+            }
         }
     }
-    if (tid < 128) {
+    if (tid < kClRows) {
         sInv[tid] = den > 0.0f ? 1.0f / den : 0.0f;
-        if (kq == 0 && p.lse_out && live_r)
+        if (leader && p.lse_out && live_r)
             p.lse_out[(int64_t)(bs0 + tid / p.G) * p.heads + grp * p.G + tid % p.G] =
                 den > 0.0f ? Mr + __logf(den) : -INFINITY;
     }
     __syncthreads();
 
-    // ---- merged rows -> A (bf16, K-major, 128-byte swizzle)
+    // ---- merged rows -> this CTA's four K blocks of A (bf16, K-major, 128-byte swizzle),
+    // at the same place they take in the leader's A
     {
         const int chunk = (lane & 15) >> 1, half8 = (lane & 1) * 8;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int r = 16 * warp + 2 * i + sub;
+            const int r = 8 * warp + i;
             const float inv = sInv[r];
-            *reinterpret_cast<uint2 *>(smem + ClSmem::oA + r * 128 + ((chunk ^ (r & 7)) << 4) + half8) =
-                pack_bf16x4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int kb = kq * 4 + 2 * h + (lane >> 4);
+                *reinterpret_cast<uint2 *>(smem + ClSmem::oA + kb * (kClRows * 128) + r * 128 +
+                                           ((chunk ^ (r & 7)) << 4) + half8) =
+                    pack_bf16x4(acc[i][h].x * inv, acc[i][h].y * inv, acc[i][h].z * inv,
+                                acc[i][h].w * inv);
+            }
         }
     }
     fence_proxy_async_smem();
     __syncthreads();
 
+    if (!leader) {
+        // ---- send this half of A to the leader; its mbarrier counts the bytes
+        if (tid == 0)
+            bulk_copy_to_peer(map_peer(smem_u32(smem + ClSmem::oA + ClSmem::kAHalf), 0),
+                              smem + ClSmem::oA + ClSmem::kAHalf, ClSmem::kAHalf,
+                              map_peer(smem_u32(a_full), 0));
+        cluster_sync();  // the leader has received the half: this CTA's memory may go
+        return;
+    }
+
+    // ---- leader: the other half of A and W_UV_g in place -> 32 MMAs (M = 64, K = 512)
+    const uint32_t tmem = *tmem_slot;
     if (tid == 0) {
-        if (mbar_wait(full, 0, abort_flag)) {
+        mbar_arrive_expect_tx(a_full, ClSmem::kAHalf);
+        const bool ok = mbar_wait_cluster(a_full, 0, abort_flag) && mbar_wait(b_full, 0, abort_flag);
+        if (ok) {
             tc_fence_after();
-            constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+            constexpr uint32_t idesc = idesc_bf16(kClRows, 128, 0, 1);
             const uint32_t a0 = smem_u32(smem + ClSmem::oA), b0 = smem_u32(smem + ClSmem::oB);
 #pragma unroll
-            for (int kk = 0; kk < kClCols / 16; ++kk) {
-                const uint64_t ad = smem_desc(a0 + kk * 32, 16, 1024, kSw128);
-                const uint64_t bd = smem_desc(b0 + kk * 2048, kClCols * 128, 1024, kSw128);
+            for (int kk = 0; kk < kLatent / 16; ++kk) {
+                const uint64_t ad =
+                    smem_desc(a0 + (kk >> 2) * (kClRows * 128) + (kk & 3) * 32, 16, 1024, kSw128);
+                const uint64_t bd = smem_desc(b0 + kk * 2048, 65536, 1024, kSw128);
                 mma_bf16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
             }
             mma_commit(done);
@@ -374,61 +400,42 @@ __global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads, 2)
     }
     const bool ok = mbar_wait(done, 0, abort_flag);
     tc_fence_after();
-
-    // ---- partial product -> Y (fp32) in this CTA's shared memory
+    // ---- epilogue: TMEM (M = 64: row m in lane (m % 16) + 32 (m / 16)) -> bf16 rows in
+    // shared memory (over A: the MMAs are done) -> coalesced 256-byte row stores
     if (ok) {
-        const int r = 32 * (warp & 3) + lane;
-        const int cbase = (warp >> 2) * 64;
-        float *y = reinterpret_cast<float *>(smem + ClSmem::oY) + r * kYStride + cbase;
+        const int q = warp & 3, cbase = (warp >> 2) * 64;
+        const int r = 16 * q + lane;  // valid for lanes 0..15
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             uint32_t v[32];
-            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cbase + 32 * h, v);
+            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + cbase + 32 * h, v);
             tmem_wait_ld();
+            if (lane < 16) {
+                uint8_t *dst = smem + ClSmem::oStage + r * 256 + (cbase + 32 * h) * 2;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                reinterpret_cast<float4 *>(y + 32 * h)[i] =
-                    make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                for (int e = 0; e < 4; ++e) {
+                    const uint2 lo = pack_bf16x4(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1]),
+                                                 __uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3]));
+                    const uint2 hi = pack_bf16x4(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5]),
+                                                 __uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7]));
+                    reinterpret_cast<uint4 *>(dst)[e] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (ok && !*abort_flag) {
+        for (int i = tid; i < kClRows * 16; i += kClThreads) {
+            const int r = i >> 4, part16 = i & 15;
+            const int j = r / p.G;
+            if (r >= rows_in_tile || bs0 + j >= p.bs_total) continue;
+            const int64_t orow = (int64_t)(bs0 + j) * p.heads + grp * p.G + r % p.G;
+            reinterpret_cast<uint4 *>(p.out + orow * kDv)[part16] =
+                reinterpret_cast<const uint4 *>(smem + ClSmem::oStage + r * 256)[part16];
         }
     }
     tc_fence_before();
-    cluster_sync();  // all partial products written
-
-    // ---- rows [16 kq, 16 kq + 16): sum the partial products, store bf16
-    {
-        const int r = 16 * kq + (tid >> 4);
-        const int col = (tid & 15) * 8;
-        const int j = r / p.G;
-        const bool live = r < rows_in_tile && bs0 + j < p.bs_total;
-        const uint32_t local = smem_u32(smem + ClSmem::oY) + (uint32_t)(r * kYStride + col) * 4;
-        float4 v[2 * kClCtas];  // all remote loads issued before the first use
-#pragma unroll
-        for (int src_rank = 0; src_rank < kClCtas; ++src_rank) {
-            const uint32_t a = map_peer(local, (uint32_t)src_rank);
-            v[2 * src_rank] = ld_cluster_f4(a);
-            v[2 * src_rank + 1] = ld_cluster_f4(a + 16);
-        }
-        float sum[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
-#pragma unroll
-        for (int src_rank = 0; src_rank < kClCtas; ++src_rank)
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                sum[4 * i] += v[2 * src_rank + i].x;
-                sum[4 * i + 1] += v[2 * src_rank + i].y;
-                sum[4 * i + 2] += v[2 * src_rank + i].z;
-                sum[4 * i + 3] += v[2 * src_rank + i].w;
-            }
-        if (live && !*abort_flag) {
-            const uint2 lo = pack_bf16x4(sum[0], sum[1], sum[2], sum[3]);
-            const uint2 hi = pack_bf16x4(sum[4], sum[5], sum[6], sum[7]);
-            *reinterpret_cast<uint4 *>(p.out + ((int64_t)(bs0 + j) * p.heads + grp * p.G + r % p.G) * kDv +
-                                       col) = make_uint4(lo.x, lo.y, hi.x, hi.y);
-        }
-    }
-    cluster_sync();  // no CTA leaves while a peer may still read its partial product
+    cluster_sync();  // pairs with the sender's: its copy has landed
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 128);
@@ -449,17 +456,17 @@ cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int
                            32 * kQuadsPerBlock, 0, stream>>>(p);
         return cudaGetLastError();
     }
-    const int bst = 128 / p.G;
+    const int bst = kClRows / p.G;
     CUtensorMap wmap;
     const uint64_t dims[2] = {(uint64_t)kDv, (uint64_t)num_groups * kLatent};
     const uint64_t strides[1] = {(uint64_t)kDv * 2};
-    const uint32_t box[2] = {64, (uint32_t)kClCols};
+    const uint32_t box[2] = {64, 256};
     if (!make_bf16_map(&wmap, w_uv, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(combine_latent_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, ClSmem::kAlloc);
     if (e != cudaSuccess) return e;
-    dim3 grid(kClCtas, (unsigned)((p.bs_total + bst - 1) / bst), (unsigned)num_groups);
+    dim3 grid(2, (unsigned)((p.bs_total + bst - 1) / bst), (unsigned)num_groups);
     combine_latent_tc_kernel<<<grid, kClThreads, ClSmem::kAlloc, stream>>>(wmap, p, bst);
     return cudaGetLastError();
 }
