@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
 //   out[64 x 128] = A[64 x 512] * W_UV_g[512 x 128]   (tcgen05 M = 64, fp32 in TMEM)
 // and writes the bf16 rows.
 // ---------------------------------------------------------------------------
-constexpr int kClThreads = 256;
+constexpr int kClThreads = 512;
 constexpr int kClRows = 64;      // rows of a tile (MMA M)
 constexpr int kClMaxPairs = 32;  // bst <= 64 / 4 = 16
 constexpr int kClChunk = 32;     // partials whose weights are staged at a time
@@ -279,16 +279,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         }
     }
 
-    // ---- merge: warp w owns rows 8w .. 8w+7; lane j covers columns 4j and 128 + 4j of
-    // this CTA's 256 latent columns
-    float4 acc[8][2];
+    // ---- merge: warp w owns rows 4w .. 4w+3; lane j covers columns 4j and 128 + 4j of
+    // this CTA's 256 latent columns; two partials are read per step
+    constexpr int kRw = kClRows / (kClThreads / 32);  // rows per warp
+    float4 acc[kRw][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float *src[8];
-    int npr[8];
+    for (int i = 0; i < kRw; ++i) acc[i][0] = acc[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *src[kRw];
+    int npr[kRw];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = 8 * warp + i;
+    for (int i = 0; i < kRw; ++i) {
+        const int r = kRw * warp + i;
         const int j = r / p.G;
         const bool live = r < rows_in_tile && bs0 + j < p.bs_total;
         npr[i] = live ? s_c1[j] - s_c0[j] : 0;
@@ -316,26 +317,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         __syncthreads();
         const int n = min(kClChunk, maxp - cb);
 #pragma unroll 1
-        for (int jj = 0; jj < n; ++jj) {
-            float4 v[8][2];
+        for (int j0 = 0; j0 < n; j0 += 2) {
+            float4 v[2][kRw][2];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const bool on = cb + jj < npr[i];
-                const float *q = src[i] + (int64_t)(cb + jj) * part_stride * kLatent;
-                v[i][0] = on ? ldg4(q) : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[i][1] = on ? ldg4(q + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float wj = sW[jj * kClRows + 8 * warp + i];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    acc[i][h].x = fmaf(wj, v[i][h].x, acc[i][h].x);
-                    acc[i][h].y = fmaf(wj, v[i][h].y, acc[i][h].y);
-                    acc[i][h].z = fmaf(wj, v[i][h].z, acc[i][h].z);
-                    acc[i][h].w = fmaf(wj, v[i][h].w, acc[i][h].w);
+                for (int i = 0; i < kRw; ++i) {
+                    const bool on = cb + j0 + u < npr[i];
+                    const float *q = src[i] + (int64_t)(cb + j0 + u) * part_stride * kLatent;
+                    v[u][i][0] = on ? ldg4(q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[u][i][1] = on ? ldg4(q + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int i = 0; i < kRw; ++i) {
+                    const float wj = j0 + u < n ? sW[(j0 + u) * kClRows + kRw * warp + i] : 0.0f;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        acc[i][h].x = fmaf(wj, v[u][i][h].x, acc[i][h].x);
+                        acc[i][h].y = fmaf(wj, v[u][i][h].y, acc[i][h].y);
+                        acc[i][h].z = fmaf(wj, v[u][i][h].z, acc[i][h].z);
+                        acc[i][h].w = fmaf(wj, v[u][i][h].w, acc[i][h].w);
+                    }
+                }
         }
     }
     if (tid < kClRows) {
@@ -351,8 +356,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     {
         const int chunk = (lane & 15) >> 1, half8 = (lane & 1) * 8;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = 8 * warp + i;
+        for (int i = 0; i < kRw; ++i) {
+            const int r = kRw * warp + i;
             const float inv = sInv[r];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -403,10 +408,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     // ---- epilogue: TMEM (M = 64: row m in lane (m % 16) + 32 (m / 16)) -> bf16 rows in
     // shared memory (over A: the MMAs are done) -> coalesced 256-byte row stores
     if (ok) {
-        const int q = warp & 3, cbase = (warp >> 2) * 64;
+        constexpr int kCw = 128 / (kClThreads / 128);  // columns per warp
+        const int q = warp & 3, cbase = (warp >> 2) * kCw;
         const int r = 16 * q + lane;  // valid for lanes 0..15
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kCw / 32; ++h) {
             uint32_t v[32];
             tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + cbase + 32 * h, v);
             tmem_wait_ld();
