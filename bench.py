@@ -14,12 +14,14 @@ value   = decode tokens per second of the whole job: N ranks x batch x s_q
           data path: weak scaling).
 e2e     = the same through the C ABI with host buffers: each step copies the
           queries, page table and lengths from pinned host memory and reads
-          both paths' outputs back, inside the timed region.
-Timing  = the step is captured once into a CUDA graph with an event record
-          before and after every call; each timed step replays the graph and
-          reads those events (device time, no host launch overhead).  L2 is
-          flushed (a 256 MiB write) before every step, outside its events;
-          W >= 3 untimed eager and W graph warm-up steps come first.
+          both paths' outputs back into pinned memory, inside the timed region
+          (the copies and the five calls replayed as one CUDA graph).
+Timing  = the step is captured into a CUDA graph; each timed step replays it
+          between two CUDA events on the stream (device time, no host launch
+          overhead).  The per-call breakdown comes from a second graph with an
+          event record around every call.  L2 is flushed (a 256 MiB write)
+          before every step, outside its events; W >= 3 untimed eager and W
+          graph warm-up steps come first.
 roofline: the dominant kernel's algorithmic bytes (or FLOPs) per launch over
           its mean event-timed duration, against MEASURED_PEAKS.json.
 cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload
@@ -289,35 +291,47 @@ def run_ours(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
 
-    # The step is captured once into a CUDA graph (the five launches replay
-    # without host launch overhead); event records inside the graph time each
-    # call on the device at every replay.
-    gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+    # The step is captured into a CUDA graph twice: as is (the five launches
+    # replay without host overhead, each kernel's set-up overlapping the
+    # previous kernel's tail) for the step time, and with an event record
+    # around every call for the per-call breakdown.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
+        step()
+    gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev):
         step(gev)
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        graph.replay()
+    for g_ in (graph, graph_ev):
+        for _ in range(args.warmup):
+            flush.fill_(1.0)
+            g_.replay()
     torch.cuda.synchronize()
 
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    per_call = [[] for _ in calls]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     step_ms = []
     with ClockSampler(local_rank) as clocks:
         for k in range(args.steps):
             flush.fill_(1.0)  # evict the caches from L2 (outside the step's events)
+            e0.record(stream)
             graph.replay()
+            e1.record(stream)
             torch.cuda.synchronize()
-            for i in range(len(calls)):
-                per_call[i].append(gev[i].elapsed_time(gev[i + 1]))
-            step_ms.append(gev[0].elapsed_time(gev[-1]))
+            step_ms.append(e0.elapsed_time(e1))
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     ms_step = sum(step_ms) / args.steps
+    per_call = [[] for _ in calls]
+    for k in range(args.steps):
+        flush.fill_(1.0)
+        graph_ev.replay()
+        torch.cuda.synchronize()
+        for i in range(len(calls)):
+            per_call[i].append(gev[i].elapsed_time(gev[i + 1]))
     st_a, _ = gqla.gqla_read_device_error(ba.workspace)
     st_g, _ = gqla.gqla_read_device_error(bg.workspace)
     if st_a or st_g:
@@ -332,22 +346,34 @@ def run_ours(args, rank, world, local_rank):
     q_d, pt_d, sl_d = case["q"], case["page_table"], case["seqlens"]
     h2d = q_h.numel() * 2 + pt_h.numel() * 4 + sl_h.numel() * 4
     d2h = outa_h.numel() * 2 + outg_h.numel() * 2
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    for k in range(args.steps + args.warmup):
-        flush.fill_(1.0)
-        if k >= args.warmup:
-            e2e_ev[k - args.warmup][0].record(stream)
+    def e2e_step():
         q_d.copy_(q_h, non_blocking=True)
         pt_d.copy_(pt_h, non_blocking=True)
         sl_d.copy_(sl_h, non_blocking=True)
         step()
         outa_h.copy_(ba.out, non_blocking=True)
         outg_h.copy_(bg.out, non_blocking=True)
-        if k >= args.warmup:
-            e2e_ev[k - args.warmup][1].record(stream)
+
+    for _ in range(args.warmup):  # eager warm-up, then the same step as one graph
+        e2e_step()
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+    graph_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_e2e):
+        e2e_step()
+    for _ in range(args.warmup):
+        graph_e2e.replay()
+    torch.cuda.synchronize()
+    e2e_times = []
+    for k in range(args.steps):
+        flush.fill_(1.0)
+        e0.record(stream)
+        graph_e2e.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_times.append(e0.elapsed_time(e1))
+    e2e_ms = sum(e2e_times) / args.steps
+    if not torch.equal(outa_h, ba.out.cpu()) or not torch.equal(outg_h, bg.out.cpu()):
+        raise RuntimeError("end-to-end outputs differ from the device results")
 
     # ---- max over ranks
     t = torch.tensor([ms_step, e2e_ms], dtype=torch.float64, device=dev)

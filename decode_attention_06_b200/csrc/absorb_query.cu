@@ -68,16 +68,20 @@ __global__ void __launch_bounds__(kAqThreads, 2)
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    griddep_wait();  // the previous kernel's results are visible from here on
+    griddep_launch_dependents();
+    if (threadIdx.x == 0) {
         const uint32_t a_bytes = (uint32_t)rows_in_tile * 128;
         mbar_arrive_expect_tx(full, 2 * a_bytes + 2 * kAqB);
         for (int kb = 0; kb < 2; ++kb) {
             tma_load_3d(sA + kb * kAqA, &qmap, full, kb * 64, grp * p.G, bs0);
             tma_load_2d(sB + kb * kAqB, &wmap, full, kb * 64, grp * kLatent + half * 256);
         }
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -186,8 +190,7 @@ cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_grou
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kAqSmem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((bs_total + bst - 1) / bst), (unsigned)num_groups, 2);
-    absorb_query_tc_kernel<<<grid, kAqThreads, kAqSmem, stream>>>(qmap, wmap, p);
-    return cudaGetLastError();
+    return launch_dependent(absorb_query_tc_kernel, grid, dim3(kAqThreads), kAqSmem, stream, qmap, wmap, p);
 }
 
 }  // namespace gqla

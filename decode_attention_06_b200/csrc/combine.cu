@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
     const int q_first = blockIdx.x * kQuadsPerBlock;
     const int bs_lo = q_first / quads_per_pair;
     const int n_pairs = (q_first + kQuadsPerBlock - 1) / quads_per_pair - bs_lo + 1;
+    griddep_wait();  // the previous kernel's results are visible from here on
+    griddep_launch_dependents();
     if (warp == 0) plan_pairs(p, bs_lo, n_pairs, s_c0, s_c1);
     __syncthreads();
 
@@ -230,6 +232,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_barrier_init();
+    }
+    griddep_wait();  // the previous kernel's results are visible from here on
+    griddep_launch_dependents();
+    if (tid == 0) {
         if (leader) {
             prefetch_tensormap(&wmap);
             mbar_arrive_expect_tx(b_full, 512 * 128 * 2);
@@ -458,9 +464,9 @@ cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int
                     kv->batch, num_splits, s_q, heads, heads / num_groups, kv->batch * s_q};
     if (d_in == kDv) {
         const int64_t quads = (int64_t)p.bs_total * (heads / 4);
-        combine_v_kernel<<<(unsigned)((quads + kQuadsPerBlock - 1) / kQuadsPerBlock),
-                           32 * kQuadsPerBlock, 0, stream>>>(p);
-        return cudaGetLastError();
+        return launch_dependent(combine_v_kernel,
+                                dim3((unsigned)((quads + kQuadsPerBlock - 1) / kQuadsPerBlock)),
+                                dim3(32 * kQuadsPerBlock), 0, stream, p);
     }
     const int bst = kClRows / p.G;
     CUtensorMap wmap;
@@ -473,8 +479,8 @@ cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, ClSmem::kAlloc);
     if (e != cudaSuccess) return e;
     dim3 grid(2, (unsigned)((p.bs_total + bst - 1) / bst), (unsigned)num_groups);
-    combine_latent_tc_kernel<<<grid, kClThreads, ClSmem::kAlloc, stream>>>(wmap, p, bst);
-    return cudaGetLastError();
+    return launch_dependent(combine_latent_tc_kernel, grid, dim3(kClThreads), ClSmem::kAlloc, stream,
+                            wmap, p, bst);
 }
 
 }  // namespace gqla

@@ -105,6 +105,25 @@ __device__ __forceinline__ int chunk_pages(int total_pages, int num_splits) {
     return (total_pages + num_splits - 1) / num_splits;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream finishes, and waits for it with
+// griddepcontrol.wait before touching global memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // Host-side argument checks shared by the entry points.
 inline bool dims_supported(const gqla_dims *d) {
     return d->d_latent == kLatent && d->d_rope == kRope && d->d_nope == kNope && d->d_v == kDv;

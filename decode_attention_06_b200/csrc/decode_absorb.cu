@@ -173,6 +173,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
+    griddep_wait();  // the previous kernel's results are visible from here on
+    griddep_launch_dependents();
     if (warp == 0) {
         int total = warp_total_pages(p.seqlens, p.batch);
         int k = chunk_pages(total, p.num_splits);
@@ -701,8 +703,8 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, AbsorbSmem::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)num_splits * p.row_blocks * 2;
-    decode_absorb_tc_kernel<<<grid, kThreads, AbsorbSmem::kAlloc, stream>>>(lat, rope, qrope, omap, p);
-    return cudaGetLastError();
+    return launch_dependent(decode_absorb_tc_kernel, dim3(grid), dim3(kThreads), AbsorbSmem::kAlloc,
+                            stream, lat, rope, qrope, omap, p);
 }
 
 }  // namespace gqla

@@ -283,6 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
+    griddep_wait();  // the previous kernel's results are visible from here on
+    griddep_launch_dependents();
     if (warp == 0) {
         int total = warp_total_pages(p.seqlens, p.batch);
         int k = chunk_pages(total, p.num_splits);
@@ -762,8 +764,8 @@ cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const CUte
     cudaError_t e = cudaFuncSetAttribute(decode_gqa_tc_kernel<NQ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    decode_gqa_tc_kernel<NQ><<<p.num_splits, kThreads, bytes, stream>>>(kvm, krm, qm, p);
-    return cudaGetLastError();
+    return launch_dependent(decode_gqa_tc_kernel<NQ>, dim3(p.num_splits), dim3(kThreads), bytes, stream,
+                            kvm, krm, qm, p);
 }
 
 }  // namespace

@@ -134,6 +134,22 @@ __device__ unsigned long long g_wait_count[32];
 #define GQLA_PROF_FLUSH (void)0
 #endif
 
+// ------------------------------------------------------------------ dependent launch
+
+// Wait until the grids this one depends on (the previous kernel in the stream,
+// when it was launched with programmatic serialization) have completed and
+// their writes are visible.  A no-op otherwise.  Every global access of a
+// kernel comes after it.
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel in the stream to start its set-up (its own accesses of
+// global memory still wait for this grid to complete).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x,
