@@ -7,11 +7,11 @@
 //
 // Rows of one group share W_UK_g, so a CTA owns a tile of up to 128 rows of
 // one group -- `bst` consecutive (sequence, query token) pairs x the group's
-// G heads -- and one half (256 columns) of the latent output:
-//   D[128 x 256] = A[128 x 128] * B[128 x 256],  A = q^C rows (K-major),
-//   B^T = W_UK_g[half] as stored ([latent][d_nope], K-major).
+// G heads -- and one quarter (128 columns) of the latent output:
+//   D[128 x 128] = A[128 x 128] * B[128 x 128],  A = q^C rows (K-major),
+//   B^T = W_UK_g[quarter] as stored ([latent][d_nope], K-major).
 // Both operands arrive by TMA in the 128-byte swizzled layout; one thread
-// issues 8 MMAs of K = 16 into a 256-column TMEM accumulator; the four warps
+// issues 8 MMAs of K = 16 into a 128-column TMEM accumulator; the four warps
 // convert their 32 rows to bf16 into shared memory and write the tile out
 // row by row, each row one contiguous 512-byte segment.
 #include <cuda.h>
@@ -28,9 +28,10 @@ using namespace sm100;
 
 constexpr int kAqThreads = 128;
 constexpr int kAqA = 128 * 128;        // one K block of A: 128 rows x 64 dims (bytes)
-constexpr int kAqB = 256 * 128;        // one K block of B: 256 latent rows x 64 dims
+constexpr int kAqN = 128;              // latent columns per CTA
+constexpr int kAqB = kAqN * 128;       // one K block of B: 128 latent rows x 64 dims
 constexpr int kAqBar = 2 * kAqA + 2 * kAqB;
-constexpr int kAqStage = 512 + 16;     // staging row pitch (bytes): 256 bf16 + bank skew
+constexpr int kAqStage = 2 * kAqN + 16;  // staging row pitch (bytes): 128 bf16 + bank skew
 static_assert(128 * kAqStage <= kAqBar, "staging tile overlaps the barriers");
 constexpr int kAqSmem = kAqBar + 64 + 1024;  // + alignment slack
 
@@ -57,7 +58,7 @@ __global__ void __launch_bounds__(kAqThreads, 2)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(full + 3);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x, grp = blockIdx.y, half = blockIdx.z;
+    const int tile = blockIdx.x, grp = blockIdx.y, quarter = blockIdx.z;
     const int bs0 = tile * p.bst;
     const int rows_in_tile = p.G * p.bst;
 
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(kAqThreads, 2)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, kAqN);
         tmem_relinquish();
     }
     griddep_wait();  // the previous kernel's results are visible from here on
@@ -80,7 +81,7 @@ __global__ void __launch_bounds__(kAqThreads, 2)
         mbar_arrive_expect_tx(full, 2 * a_bytes + 2 * kAqB);
         for (int kb = 0; kb < 2; ++kb) {
             tma_load_3d(sA + kb * kAqA, &qmap, full, kb * 64, grp * p.G, bs0);
-            tma_load_2d(sB + kb * kAqB, &wmap, full, kb * 64, grp * kLatent + half * 256);
+            tma_load_2d(sB + kb * kAqB, &wmap, full, kb * 64, grp * kLatent + quarter * kAqN);
         }
     }
     tc_fence_before();
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(kAqThreads, 2)
     if (threadIdx.x == 0) {
         if (mbar_wait(full, 0, abort_flag)) {
             tc_fence_after();
-            constexpr uint32_t idesc = idesc_bf16(128, 256, 0, 0);
+            constexpr uint32_t idesc = idesc_bf16(128, kAqN, 0, 0);
             const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(kAqThreads, 2)
     if (ok) {
         const int r = warp * 32 + lane;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 0; c < kAqN; c += 32) {
             uint32_t v[32];
             tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, v);
             tmem_wait_ld();
@@ -134,15 +135,17 @@ __global__ void __launch_bounds__(kAqThreads, 2)
     }
     __syncthreads();
     if (ok) {
-        // rows_in_tile rows; warp w takes rows w, w+4, ...; lane l writes 16 bytes
-        for (int r = warp; r < rows_in_tile; r += 4) {
+        // rows_in_tile rows of 256 bytes; a warp writes two rows at a time, 16 bytes a lane
+        for (int r0 = 2 * warp; r0 < rows_in_tile; r0 += 8) {
+            const int r = r0 + (lane >> 4);
             const int bs = bs0 + r / p.G;
-            if (bs >= p.bs_total) break;
-            const int64_t row = (int64_t)bs * p.heads + grp * p.G + r % p.G;
-            reinterpret_cast<uint4 *>(p.qa + row * kRow + half * 256)[lane] =
-                *reinterpret_cast<const uint4 *>(stage + r * kAqStage + lane * 16);
+            if (r < rows_in_tile && bs < p.bs_total) {
+                const int64_t row = (int64_t)bs * p.heads + grp * p.G + r % p.G;
+                reinterpret_cast<uint4 *>(p.qa + row * kRow + quarter * kAqN)[lane & 15] =
+                    *reinterpret_cast<const uint4 *>(stage + r * kAqStage + (lane & 15) * 16);
+            }
         }
-        if (half == 0) {  // RoPE part: q[row][128:192] -> qa[row][512:576], 8 lanes per row
+        if (quarter == 0) {  // RoPE part: q[row][128:192] -> qa[row][512:576], 8 lanes per row
             for (int i = threadIdx.x; i < rows_in_tile * 8; i += kAqThreads) {
                 const int r = i >> 3, part = i & 7;
                 const int bs = bs0 + r / p.G;
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(kAqThreads, 2)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, kAqN);
     }
 }
 
@@ -180,7 +183,7 @@ cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_grou
     {
         const uint64_t dims[2] = {(uint64_t)kNope, (uint64_t)num_groups * kLatent};
         const uint64_t strides[1] = {(uint64_t)kNope * 2};
-        const uint32_t box[2] = {64, 256};
+        const uint32_t box[2] = {64, (uint32_t)kAqN};
         if (!make_bf16_map(&wmap, w_uk, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
@@ -189,7 +192,7 @@ cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_grou
     cudaError_t e = cudaFuncSetAttribute(absorb_query_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kAqSmem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((bs_total + bst - 1) / bst), (unsigned)num_groups, 2);
+    dim3 grid((unsigned)((bs_total + bst - 1) / bst), (unsigned)num_groups, kLatent / kAqN);
     return launch_dependent(absorb_query_tc_kernel, grid, dim3(kAqThreads), kAqSmem, stream, qmap, wmap, p);
 }
 

@@ -115,11 +115,8 @@ struct PagePair {
     bool bad;          // a page index outside the pool was met
 };
 
-__device__ __forceinline__ PagePair load_pair(const GqaParams &p, int b, int L, int pg, int pe) {
-    const int32_t *row = p.page_table + (int64_t)b * p.max_pages;
+__device__ __forceinline__ PagePair make_pair(const GqaParams &p, int L, int pg, int pe, int a0, int a1) {
     PagePair pp;
-    const int a0 = row[pg];
-    const int a1 = pg + 1 < pe ? row[pg + 1] : 0;
     const bool bad0 = a0 < 0 || a0 >= p.num_pages;
     const bool bad1 = pg + 1 < pe && (a1 < 0 || a1 >= p.num_pages);
     pp.bad = bad0 || bad1;
@@ -130,10 +127,18 @@ __device__ __forceinline__ PagePair load_pair(const GqaParams &p, int b, int L, 
     return pp;
 }
 
+__device__ __forceinline__ PagePair load_pair(const GqaParams &p, int b, int L, int pg, int pe) {
+    const int32_t *row = p.page_table + (int64_t)b * p.max_pages;
+    return make_pair(p, L, pg, pe, row[pg], pg + 1 < pe ? row[pg + 1] : 0);
+}
+
 // Walks the units (sequence, page pair, group) of a chunk in pipeline order.
+// The next pair's page indices are requested halfway through the current
+// pair, so the page table is never waited for inside a piece.
 struct UnitCursor {
     PieceIter it;
     int b, L, pg, pe, gi;
+    int n0, n1;  // page indices of the pair after this one (valid from gi == 4)
     PagePair pp;
     bool valid;
     __device__ __forceinline__ bool next_valid_piece(const GqaParams &p) {
@@ -153,10 +158,16 @@ struct UnitCursor {
         valid = next_valid_piece(p);
     }
     __device__ __forceinline__ void advance(const GqaParams &p) {
-        if (++gi < 8) return;
+        ++gi;
+        if (gi == 4 && pg + 2 < pe) {
+            const int32_t *row = p.page_table + (int64_t)b * p.max_pages;
+            n0 = row[pg + 2];
+            n1 = pg + 3 < pe ? row[pg + 3] : 0;
+        }
+        if (gi < 8) return;
         gi = 0;
         pg += 2;
-        if (pg < pe) { pp = load_pair(p, b, L, pg, pe); return; }
+        if (pg < pe) { pp = make_pair(p, L, pg, pe, n0, n1); return; }
         valid = next_valid_piece(p);
     }
 };
