@@ -19,8 +19,9 @@ e2e     = the same through the C ABI with host buffers: each step copies the
 Timing  = the step is captured into a CUDA graph; each timed step replays it
           between two CUDA events on the stream (device time, no host launch
           overhead).  The per-call breakdown comes from a second graph with an
-          event record around every call.  L2 is flushed (a 256 MiB write)
-          before every step, outside its events; W >= 3 untimed eager and W
+          event record around every call.  L2 is flushed (a 256 MiB write, then a
+          256 MiB read so no dirty line is left) before every step, outside
+          its events; W >= 3 untimed eager and W
           graph warm-up steps come first.
 roofline: the dominant kernel's algorithmic bytes (or FLOPs) per launch over
           its mean event-timed duration, against MEASURED_PEAKS.json.
@@ -254,12 +255,22 @@ def run_ours(args, rank, world, local_rank):
     ba = gqla.DecodeBuffers(dims, B, s_q, splits["absorb"], "absorb", device=dev)
     bg = gqla.DecodeBuffers(dims, B, s_q, splits["gqa"], "gqa", device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sum = torch.empty((), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        # Write a buffer larger than L2, then read another one: the write
+        # evicts every line of the step's data, and the read makes L2 write
+        # the dirty lines of the first buffer back before the step starts,
+        # so their write-back does not land in the next timed kernel.
+        flush.fill_(1.0)
+        torch.sum(flush_rd, dim=0, out=flush_sum)
 
     # one-shot expansion, timed on its own
     gqla.gqla_expand_cache(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    flush.fill_(1.0)
+    flush_l2()
     e0.record()
     gqla.gqla_expand_cache(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
     e1.record()
@@ -287,7 +298,7 @@ def run_ours(args, rank, world, local_rank):
             events[-1].record()
 
     for _ in range(args.warmup):
-        flush.fill_(1.0)
+        flush_l2()
         step()
     torch.cuda.synchronize()
 
@@ -304,7 +315,7 @@ def run_ours(args, rank, world, local_rank):
         step(gev)
     for g_ in (graph, graph_ev):
         for _ in range(args.warmup):
-            flush.fill_(1.0)
+            flush_l2()
             g_.replay()
     torch.cuda.synchronize()
 
@@ -315,7 +326,7 @@ def run_ours(args, rank, world, local_rank):
     step_ms = []
     with ClockSampler(local_rank) as clocks:
         for k in range(args.steps):
-            flush.fill_(1.0)  # evict the caches from L2 (outside the step's events)
+            flush_l2()  # evict the step's data from L2 (outside the step's events)
             e0.record(stream)
             graph.replay()
             e1.record(stream)
@@ -327,7 +338,7 @@ def run_ours(args, rank, world, local_rank):
     ms_step = sum(step_ms) / args.steps
     per_call = [[] for _ in calls]
     for k in range(args.steps):
-        flush.fill_(1.0)
+        flush_l2()
         graph_ev.replay()
         torch.cuda.synchronize()
         for i in range(len(calls)):
@@ -365,7 +376,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_times = []
     for k in range(args.steps):
-        flush.fill_(1.0)
+        flush_l2()
         e0.record(stream)
         graph_e2e.replay()
         e1.record(stream)
@@ -438,7 +449,7 @@ def run_ours(args, rank, world, local_rank):
                    "context": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths[1:]),
                    "s_q": s_q, "paged": w.paged, "paths": ["absorb", "gqa"],
                    "tokens_per_step": tokens_step, "num_splits": splits,
-                   "l2": "flushed (256 MiB write) before every timed step",
+                   "l2": "flushed (256 MiB write + 256 MiB read) before every timed step",
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "roofline": roofline,
         "per_path": {"absorb": path_info(["absorb_query", "decode_absorb", "combine_absorb"],

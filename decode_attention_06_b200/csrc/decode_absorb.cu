@@ -134,7 +134,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_absorb_tc_kernel(const __grid_constant__ CUtensorMap lat_map,
                             const __grid_constant__ CUtensorMap rope_map,
                             const __grid_constant__ CUtensorMap qrope_map,
-                            const __grid_constant__ CUtensorMap o_map, const AbsorbParams p) {
+                            const __grid_constant__ CUtensorMap o_map_wide,
+                            const __grid_constant__ CUtensorMap o_map_narrow, const AbsorbParams p) {
     using SM = AbsorbSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -175,13 +176,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     griddep_wait();  // the previous kernel's results are visible from here on
     griddep_launch_dependents();
+    // first page indices of the first piece, loaded by the producer warp while the
+    // CTA and the cluster synchronise (valid when pre_ok)
+    int pre_page = 0;
+    bool pre_ok = false;
     if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&lat_map);
+            prefetch_tensormap(&rope_map);
+            prefetch_tensormap(&qrope_map);
+        }
         int total = warp_total_pages(p.seqlens, p.batch);
         int k = chunk_pages(total, p.num_splits);
         int r0 = c * k, r1 = min(total, r0 + k);
         int b = p.batch, start = 0;
         if (r0 < r1) warp_find_sequence(p.seqlens, p.batch, r0, &b, &start);
         if (lane == 0) { plan[0] = r0; plan[1] = r1; plan[2] = b; plan[3] = start; }
+        if (b < p.batch) {
+            const int n = pages_of(p.seqlens[b]);  // > 0: the search skips empty sequences
+            if (n <= p.max_pages) {                 // not a sequence that is reported as too long
+                const int pb0 = r0 - start, pe0 = min(r1 - start, n);
+                pre_ok = true;
+                if (lane < min(32, pe0 - pb0)) pre_page = p.page_table[(int64_t)b * p.max_pages + pb0 + lane];
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_base_smem, 512);
@@ -204,11 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------------- TMA producer
         // Lane 0 issues; the whole warp fetches the page indices 32 at a time so
         // that no page-table load sits between two tiles.
-        if (lane == 0) {
-            prefetch_tensormap(&lat_map);
-            prefetch_tensormap(&rope_map);
-            prefetch_tensormap(&qrope_map);
-        }
+        const uint64_t stream_policy = l2_evict_first_policy();  // the cache is read once
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
@@ -236,7 +250,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             for (int i0 = pb; i0 < pe; i0 += 32) {
                 const int n = min(32, pe - i0);
-                const int my_page = lane < n ? prow[i0 + lane] : 0;
+                // (the first piece is the one the early load above was for)
+                const int my_page = pre_ok ? pre_page : (lane < n ? prow[i0 + lane] : 0);
+                pre_ok = false;
                 for (int j = 0; j < n; ++j, ++t) {
                     const int page = __shfl_sync(0xffffffffu, my_page, j);
                     if (i0 - pb + j == rope_at) load_rope();
@@ -250,10 +266,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
 #pragma unroll
                             for (int bx = 0; bx < 4; ++bx)
-                                tma_load_2d(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
-                                            256 * rank + 64 * bx, page * kPage);
-                            tma_load_2d(dst + 4 * SM::kLatBox, &rope_map, &ring_full[slot], 512 + 32 * rank,
-                                        page * kPage);
+                                tma_load_2d_hint(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
+                                                 256 * rank + 64 * bx, page * kPage, stream_policy);
+                            tma_load_2d_hint(dst + 4 * SM::kLatBox, &rope_map, &ring_full[slot], 512 + 32 * rank,
+                                             page * kPage, stream_policy);
                         } else {
                             mbar_arrive(&ring_full[slot]);
                         }
@@ -383,7 +399,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(q_full);
         };
         const bool quad_live = 32 * quad < rows_here;  // rows_here is a multiple of 32
-        uint8_t *stg = smem + SM::oP + w * 2048;       // epilogue staging: [32 rows][16 fp32]
         bool q_loaded = false;                         // q~ of the coming piece already in TMEM
         PieceIter it = it0;
         int b, L, pb, pe;
@@ -581,21 +596,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // and the next piece's q~ goes into TMEM now, so that its scores overlap this epilogue
             __syncwarp();
             if (lane == 0) mbar_arrive(q_empty);
+            bool more_pieces;
             {
                 PieceIter nx = it;
                 int b2, L2, pb2, pe2;
-                bool tl2 = false, more;
+                bool tl2 = false;
                 do {
-                    more = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
-                } while (more && tl2);
-                if (more) {
+                    more_pieces = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
+                } while (more_pieces && tl2);
+                if (more_pieces) {
                     copy_q(b2);
                     q_loaded = true;
                 }
             }
             // ---- epilogue: O / l for this CTA's 256 columns (this warp: 256 / kParts) through
-            // TMA stores staged in this warp's 2 KB of the P buffers (free once the piece's
-            // last PV is done), LSE by rank 0
+            // TMA stores staged in shared memory.  After the last piece the ring is free
+            // (every tile is consumed) and holds all of it: 8 KB per warp, two 128-byte-swizzled
+            // boxes, one store round.  Between pieces the ring holds the next piece's tiles, so
+            // each warp stages 2 KB at a time in the P buffers (free once the piece's last PV
+            // is done).  LSE by rank 0.
             GQLA_SPAN_BEGIN(t_epi);
             if (!GQLA_WAIT(15, o_done, k & 1, abort_flag)) *abort_flag = 1;
             tc_fence_after();
@@ -608,30 +627,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool live = row < rows_here;
             const int64_t orow = (int64_t)(b + c) * p.rows_total + grow;  // slot b + c
             const int orow0 = (b + c) * p.rows_total + rb * kRows + 32 * quad;
-#pragma unroll 1
-            for (int j = 0; j < 256 / kParts / 16; ++j) {
-                if (j > 0) {
-                    if (lane == 0) bulk_wait_group_read<0>();  // the previous chunk's store has read stg
-                    __syncwarp();
-                }
-                uint32_t r[16];
-                tmem_ld16(t_o + lane_off + part * (256 / kParts) + 16 * j, r);
-                tmem_wait_ld();
+            const int ocol0 = 256 * (int)rank + part * (256 / kParts);
+            if (!more_pieces) {
+                uint8_t *stg = smem + SM::oRing + w * 8192;  // [2 boxes][32 rows][128 B]
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)  // 64-byte swizzle: chunk ^= (row / 2) % 4
-                    *reinterpret_cast<float4 *>(stg + lane * 64 + ((q4 ^ ((lane >> 1) & 3)) << 4)) =
-                        make_float4(__uint_as_float(r[4 * q4]) * inv, __uint_as_float(r[4 * q4 + 1]) * inv,
-                                    __uint_as_float(r[4 * q4 + 2]) * inv, __uint_as_float(r[4 * q4 + 3]) * inv);
+                for (int j = 0; j < 256 / kParts / 16; ++j) {
+                    uint32_t r[16];
+                    tmem_ld16(t_o + lane_off + part * (256 / kParts) + 16 * j, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {  // 128-byte swizzle: chunk ^= row % 8
+                        const int chunk = (j & 1) * 4 + q4;
+                        *reinterpret_cast<float4 *>(stg + (j >> 1) * 4096 + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                            make_float4(__uint_as_float(r[4 * q4]) * inv, __uint_as_float(r[4 * q4 + 1]) * inv,
+                                        __uint_as_float(r[4 * q4 + 2]) * inv, __uint_as_float(r[4 * q4 + 3]) * inv);
+                    }
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && quad_live && !*abort_flag) {
-                    tma_store_2d(&o_map, stg, 256 * (int)rank + part * (256 / kParts) + 16 * j, orow0);
+                    tma_store_2d(&o_map_wide, stg, ocol0, orow0);
+                    tma_store_2d(&o_map_wide, stg + 4096, ocol0 + 32, orow0);
                     bulk_commit_group();
                 }
+            } else {
+                uint8_t *stg = smem + SM::oP + w * 2048;  // [32 rows][16 fp32], 64-byte swizzle
+#pragma unroll 1
+                for (int j = 0; j < 256 / kParts / 16; ++j) {
+                    if (j > 0) {
+                        if (lane == 0) bulk_wait_group_read<0>();  // the previous chunk's store has read stg
+                        __syncwarp();
+                    }
+                    uint32_t r[16];
+                    tmem_ld16(t_o + lane_off + part * (256 / kParts) + 16 * j, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)  // 64-byte swizzle: chunk ^= (row / 2) % 4
+                        *reinterpret_cast<float4 *>(stg + lane * 64 + ((q4 ^ ((lane >> 1) & 3)) << 4)) =
+                            make_float4(__uint_as_float(r[4 * q4]) * inv, __uint_as_float(r[4 * q4 + 1]) * inv,
+                                        __uint_as_float(r[4 * q4 + 2]) * inv, __uint_as_float(r[4 * q4 + 3]) * inv);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && quad_live && !*abort_flag) {
+                        tma_store_2d(&o_map_narrow, stg, ocol0 + 16 * j, orow0);
+                        bulk_commit_group();
+                    }
+                }
+                if (lane == 0) bulk_wait_group_read<0>();
+                // every warp's staging (spread over all the P rows) is read before any P is rewritten
+                softmax_bar();
             }
-            if (lane == 0) bulk_wait_group_read<0>();
-            // every warp's staging (spread over all the P rows) is read before any P is rewritten
-            softmax_bar();
             if (live && rank == 0 && part == 0)
                 p.lse_part[orow] = (l > 0.0f && m_run != -INFINITY)
                                        ? (m_run + __log2f(l)) * 0.6931471805599453f
@@ -667,7 +712,7 @@ bool make_row_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t bo
 cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
                                  const gqla_kv_index *idx, int num_splits, float scale,
                                  float *o_part, float *lse_part, void *ws, cudaStream_t stream) {
-    CUtensorMap lat, rope, qrope, omap;
+    CUtensorMap lat, rope, qrope, omap_w, omap_n;
     const uint64_t slots = (uint64_t)idx->num_pages * kPage;
     const uint64_t qrows = (uint64_t)idx->batch * s_q * heads;
     if (!make_row_map(&lat, cache, slots, 64, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -675,11 +720,15 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
         !make_row_map(&qrope, qa, qrows, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     {
+        // partials fp32 [B + C][s_q][h][512]: 32 x 32 boxes (128-byte rows) for the last
+        // piece's stores, 16 x 32 boxes for those between pieces
         const uint64_t orows = (uint64_t)(idx->batch + num_splits) * s_q * heads;
         const uint64_t dims[2] = {(uint64_t)kLatent, orows};
         const uint64_t strides[1] = {(uint64_t)kLatent * 4};
-        const uint32_t box[2] = {16, 32};
-        if (!make_map(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, o_part, 2, dims, strides, box,
+        const uint32_t box_w[2] = {32, 32}, box_n[2] = {16, 32};
+        if (!make_map(&omap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, o_part, 2, dims, strides, box_w,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&omap_n, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, o_part, 2, dims, strides, box_n,
                       CU_TENSOR_MAP_SWIZZLE_64B))
             return cudaErrorInvalidValue;
     }
@@ -704,7 +753,7 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)num_splits * p.row_blocks * 2;
     return launch_dependent(decode_absorb_tc_kernel, dim3(grid), dim3(kThreads), AbsorbSmem::kAlloc,
-                            stream, lat, rope, qrope, omap, p);
+                            stream, lat, rope, qrope, omap_w, omap_n, p);
 }
 
 }  // namespace gqla
