@@ -54,35 +54,42 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kSmWarps = 16;                // softmax warps: kParts per TMEM lane quadrant
-constexpr int kParts = kSmWarps / 4;
+constexpr int kXWarps = 8;                  // score warps: two per TMEM lane quadrant
+constexpr int kYWarps = 8;                  // softmax warps of the CTA's own rows
+constexpr int kSmWarps = kXWarps + kYWarps;
 constexpr int kThreads = 32 * (3 + kSmWarps);
 constexpr int kPvWarp = 2 + kSmWarps;       // warp issuing O += P C
 constexpr int kRows = 128;           // MMA M: query rows of one row block (zero-padded)
 constexpr int kT = 64;               // tokens per tile (one page)
 constexpr int kRing = 4;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kTokW = kT / kParts;          // tokens of a tile per softmax warp
-constexpr int kSmThreads = 32 * kSmWarps;
+constexpr int kXThreads = 32 * kXWarps;
+constexpr int kXTok = kT / 2;               // tokens of a tile per score warp
+constexpr int kXCols = 256 / 2;             // O columns per score warp
+constexpr int kOwn = kRows / 2;             // rows whose softmax a CTA of the pair computes
 
 struct AbsorbSmem {
     static constexpr int kQRope = kRows * 64;             // q~ RoPE columns [128 rows][32]
     static constexpr int kLatBox = kT * 128;              // [64 tokens][64 cols]
     static constexpr int kRopeBox = kT * 64;              // [64 tokens][32 cols]
     static constexpr int kSlot = 4 * kLatBox + kRopeBox;  // 36 KB
-    static constexpr int kX = kRows * kT * 2;             // fp16 partial scores, [warps][32 rows][kTokW]
-    static constexpr int kXw = kX / kSmWarps;             // one warp's block
+    // partial scores of this CTA's 64 rows: [2 sources][64 rows][64 tokens] fp16, the
+    // 16-byte chunks of a row XOR-swizzled by row % 8; the peer's half arrives by st.async
+    static constexpr int kX = 2 * kOwn * kT * 2;
+    static constexpr int kXRemote = kOwn * kT * 2;
     static constexpr int kP = kRows * kT * 2;             // P, [128 rows][64 tokens] bf16, 128B-swizzled
+    // the peer's 64 rows of P (bulk copies) and their O rescale factors (st.async)
+    static constexpr int kPRemote = kOwn * kT * 2 + kOwn * 4;
     static constexpr int oQ = 0;
     static constexpr int oP = oQ + kQRope;                // 2 buffers
     static constexpr int oRing = oP + 2 * kP;
-    static constexpr int oX = oRing + kRing * kSlot;      // the peer's partials (2 buffers)
-    static constexpr int oRm = oX + 2 * kX;               // float [2 tiles][kParts][128 rows]
-    static constexpr int oL = oRm + 2 * kParts * kRows * 4;  // float [kParts][128 rows]
-    static constexpr int oBar = oL + kParts * kRows * 4;
-    // ring_full/empty[3], q_full, q_empty, s_full/s_free[2], p_full/p_free[2],
-    // x_full/x_empty[2], o_done, drain[2]
-    static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 4 + 1 + 2;
+    static constexpr int oX = oRing + kRing * kSlot;      // 2 buffers
+    static constexpr int oAlpha = oX + 2 * kX;            // float [2 buffers][128 rows]
+    static constexpr int oL = oAlpha + 2 * kRows * 4;     // float [128 rows]: row sums of a piece
+    static constexpr int oBar = oL + kRows * 4;
+    // ring_full/empty[kRing], q_full, q_empty, s_full/s_free[2], x_full/x_empty[2],
+    // p_full/p_empty[2], o_ready[2], pv_done[2], l_full, o_done, drain[2]
+    static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 4 + 2 + 2 + 1 + 1 + 2;
     static constexpr int oMisc = oBar + kNumBars * 8;     // tmem base, abort, plan[4]
     static constexpr int kBytes = oMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;
@@ -122,20 +129,11 @@ __device__ __forceinline__ bool next_piece(const AbsorbParams &p, PieceIter &it,
     return false;
 }
 
-__device__ __forceinline__ void quad_bar(int quad) {  // the softmax warps of one lane quadrant
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "n"(32 * kParts) : "memory");
-}
-
-__device__ __forceinline__ void softmax_bar() {  // all softmax warps
-    asm volatile("bar.sync 5, %0;" ::"n"(kSmThreads) : "memory");
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_absorb_tc_kernel(const __grid_constant__ CUtensorMap lat_map,
                             const __grid_constant__ CUtensorMap rope_map,
                             const __grid_constant__ CUtensorMap qrope_map,
-                            const __grid_constant__ CUtensorMap o_map_wide,
-                            const __grid_constant__ CUtensorMap o_map_narrow, const AbsorbParams p) {
+                            const __grid_constant__ CUtensorMap o_map, const AbsorbParams p) {
     using SM = AbsorbSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -144,9 +142,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint64_t *ring_full = bars, *ring_empty = bars + kRing;
     uint64_t *q_full = bars + 2 * kRing, *q_empty = q_full + 1;
     uint64_t *s_full = q_empty + 1, *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2, *p_free = p_full + 2;
-    uint64_t *x_full = p_free + 2, *x_empty = x_full + 2;
-    uint64_t *o_done = x_empty + 2, *drain = o_done + 1;
+    uint64_t *x_full = s_free + 2, *x_empty = x_full + 2;
+    uint64_t *p_full = x_empty + 2, *p_empty = p_full + 2;
+    uint64_t *o_ready = p_empty + 2, *pv_done = o_ready + 2;
+    uint64_t *l_full = pv_done + 2, *o_done = l_full + 1, *drain = o_done + 1;
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(smem + SM::oMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::oMisc + 4);
     int *plan = reinterpret_cast<int *>(smem + SM::oMisc + 8);
@@ -162,14 +161,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i) { mbar_init(&ring_full[i], 1); mbar_init(&ring_empty[i], 1); }
-        mbar_init(q_full, 1 + kSmWarps);  // RoPE TMA + the softmax warps' TMEM copies
-        mbar_init(q_empty, kSmWarps);
+        mbar_init(q_full, 1 + kXWarps);  // RoPE TMA + the score warps' TMEM copies
+        mbar_init(q_empty, kXWarps);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1); mbar_init(&s_free[i], kSmThreads);
-            mbar_init(&p_full[i], kSmThreads); mbar_init(&p_free[i], 1);
-            mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], kSmWarps);
+            mbar_init(&s_full[i], 1); mbar_init(&s_free[i], kXThreads);
+            mbar_init(&x_full[i], 1 + kXWarps);      // expect_tx of the peer's half + local score warps
+            mbar_init(&x_empty[i], 2 * kYWarps);     // every softmax warp of both CTAs has read it
+            mbar_init(&p_full[i], 1 + kYWarps);      // expect_tx of the peer's rows + local softmax warps
+            mbar_init(&p_empty[i], 2);               // PV of both CTAs done with the buffer
+            mbar_init(&o_ready[i], kXWarps);
+            mbar_init(&pv_done[i], 1);
             mbar_init(&drain[i], 1);
         }
+        mbar_init(l_full, 1 + kYWarps);
         mbar_init(o_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -291,6 +295,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------------- score MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(kRows, kT, 0, 0);
+            // descriptors of ring slot 0 and of the RoPE q~; a single issuing thread pays
+            // for every instruction of a descriptor, so each MMA only adds an offset
+            const uint64_t lat_d0 = smem_desc(sm_ring, 16, 1024, kSw128);
+            const uint64_t rope_d0 = smem_desc(sm_ring + 4 * SM::kLatBox, 16, 512, kSw64);
+            const uint64_t q_d0 = smem_desc(sm_q, 16, 512, kSw64);
             PieceIter it = it0;
             int b, L, pb, pe;
             bool too_long;
@@ -303,19 +312,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (!GQLA_WAIT(3, &ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
                     if (!GQLA_WAIT(4, &s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
-                    const uint32_t tile = sm_ring + slot * SM::kSlot;
+                    const uint64_t lat_d = desc_advance(lat_d0, slot * SM::kSlot);
+                    const uint64_t rope_d = desc_advance(rope_d0, slot * SM::kSlot);
+                    const uint32_t t_sb = t_s + sb * kT;
                     if (!*abort_flag) {
 #pragma unroll
-                        for (int ks = 0; ks < 16; ++ks) {  // latent: A = q~ in TMEM, 16 dims = 8 columns
-                            const uint64_t bd = smem_desc(tile + (ks >> 2) * SM::kLatBox + (ks & 3) * 32, 16, 1024, kSw128);
-                            mma_bf16_ts(t_s + sb * kT, t_q + ks * 8, bd, idesc_s, ks > 0 ? 1u : 0u);
-                        }
+                        for (int ks = 0; ks < 16; ++ks)  // latent: A = q~ in TMEM, 16 dims = 8 columns
+                            mma_bf16_ts(t_sb, t_q + ks * 8, desc_advance(lat_d, (ks >> 2) * SM::kLatBox + (ks & 3) * 32),
+                                        idesc_s, ks > 0 ? 1u : 0u);
 #pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) {  // RoPE: 32 columns, 64B-swizzled rows
-                            const uint64_t ad = smem_desc(sm_q + ks * 32, 16, 512, kSw64);
-                            const uint64_t bd = smem_desc(tile + 4 * SM::kLatBox + ks * 32, 16, 512, kSw64);
-                            mma_bf16(t_s + sb * kT, ad, bd, idesc_s, 1u);
-                        }
+                        for (int ks = 0; ks < 2; ++ks)  // RoPE: 32 columns, 64B-swizzled rows
+                            mma_bf16(t_sb, desc_advance(q_d0, ks * 32), desc_advance(rope_d, ks * 32), idesc_s, 1u);
                     }
                     mma_commit(&s_full[sb]);
                 }
@@ -329,6 +336,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------------- PV MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_pv = idesc_bf16(kRows, 256, 0, 1);
+            const uint64_t v_d0 = smem_desc(sm_ring, SM::kLatBox, 1024, kSw128);
+            const uint64_t p_d0 = smem_desc(sm_p, 16, 1024, kSw128);
             PieceIter it = it0;
             int b, L, pb, pe;
             bool too_long;
@@ -337,20 +346,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (too_long) continue;
                 for (int i = 0; i < pe - pb; ++i, ++t) {
                     const int slot = t % kRing, sb = t & 1;
-                    if (!GQLA_WAIT(5, &p_full[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(5, &o_ready[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
-                    const uint32_t tile = sm_ring + slot * SM::kSlot;
+                    // B = C_lat[tokens][256 cols of this CTA]: MN-major, 4 atoms of 64 columns;
+                    // A = P[128 rows][64 tokens], K-major: 16 tokens = 32 bytes of a row
+                    const uint64_t v_d = desc_advance(v_d0, slot * SM::kSlot);
+                    const uint64_t p_d = desc_advance(p_d0, sb * SM::kP);
                     if (!*abort_flag) {
 #pragma unroll
-                        for (int ks = 0; ks < kT / 16; ++ks) {
-                            // B = C_lat[tokens][256 cols of this CTA]: MN-major, 4 atoms of 64 columns
-                            const uint64_t bd = smem_desc(tile + ks * 2048, SM::kLatBox, 1024, kSw128);
-                            // A = P[128 rows][64 tokens], K-major: 16 tokens = 32 bytes of a row
-                            const uint64_t ad = smem_desc(sm_p + sb * SM::kP + ks * 32, 16, 1024, kSw128);
-                            mma_bf16(t_o, ad, bd, idesc_pv, (i == 0 && ks == 0) ? 0u : 1u);
-                        }
+                        for (int ks = 0; ks < kT / 16; ++ks)
+                            mma_bf16(t_o, desc_advance(p_d, ks * 32), desc_advance(v_d, ks * 2048), idesc_pv,
+                                     (i == 0 && ks == 0) ? 0u : 1u);
                     }
-                    mma_commit(&p_free[sb]);
+                    mma_commit_multicast(&p_empty[sb], 0x3);  // P buffer sb of both CTAs is free
+                    mma_commit(&pv_done[sb]);
                     mma_commit(&ring_empty[slot]);
                 }
                 mma_commit(o_done);
@@ -359,180 +368,119 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int dummy = 0;
             mbar_wait(&drain[1], 0, reinterpret_cast<volatile int *>(&dummy));
         }
-    } else {
-        // ---------------------------------------------------------------- softmax + epilogue
-        constexpr int kPr = kTokW / 2;           // fp16 pairs of a warp's tokens
-        const int quad = warp & 3;               // TMEM lane quadrant
-        const int w = warp - 2;                  // softmax warp index: its block of a buffer
-        const int part = w >> 2;                 // which kTokW tokens of the tile
-        const int row = 32 * quad + lane;        // query row of the row block (= TMEM lane)
+    } else if (warp < 2 + kXWarps) {
+        // ---------------------------------------------------------------- score warps
+        // Stage A of tile j: scores -> fp16 -> the owner of each row (row r of the block
+        // belongs to rank (r / 16) % 2, so both CTAs use all four TMEM lane quadrants);
+        // stage C of tile j - 1: once P and the rescale factors of all 128 rows are in,
+        // O rows are rescaled where a row maximum rose and PV is released.  Also the q~
+        // copies into TMEM and the epilogue.  Two warps per lane quadrant: warp half
+        // `xpart` takes tokens [32 xpart, 32 xpart + 32) of a tile and O columns
+        // [128 xpart, 128 xpart + 128).
+        const int quad = warp & 3;
+        const int xw = warp - 2;
+        const int xpart = xw >> 2;
+        const int row = 32 * quad + lane;        // TMEM row
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         const int grow = rb * kRows + row;       // row within the sequence's s_q * h rows
-        const int s_of_row = grow < p.rows_total ? grow / p.heads : p.s_q - 1;
-        float *rm = reinterpret_cast<float *>(smem + SM::oRm);
-        float *lsm = reinterpret_cast<float *>(smem + SM::oL);
-        const uint8_t *xbuf = smem + SM::oX;
-        const uint32_t x_remote =
-            map_peer(smem_u32(smem + SM::oX), peer) + w * SM::kXw + lane * (kTokW * 2);
+        const uint32_t a_owner = (lane >> 4) & 1;
+        const int a_orow = 16 * quad + (lane & 15);  // this row's index among its owner's rows
+        const float *alph = reinterpret_cast<const float *>(smem + SM::oAlpha);
+        const float *lsm = reinterpret_cast<const float *>(smem + SM::oL);
+        const uint32_t x_remote = map_peer(smem_u32(smem + SM::oX), peer);
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
-        const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
-        // ---- this warp's share of q~'s latent half (its 32 rows x 256/kParts columns)
-        // into TMEM; the previous piece's scores, its last readers, are complete
+        const bool quad_live = 32 * quad < rows_here;  // rows_here is a multiple of 32
+        // this warp's share of q~'s latent half (32 rows x 128 columns) into TMEM; the
+        // previous piece's scores, its last readers, are complete
         auto copy_q = [&](int bq) {
-            constexpr int kQc = 256 / kParts;  // bf16 columns per warp
             const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.qa + ((int64_t)bq * p.rows_total + grow) * kRow + 256 * rank + part * kQc);
+                p.qa + ((int64_t)bq * p.rows_total + grow) * kRow + 256 * rank + kXCols * xpart);
             const bool live = row < rows_here;
 #pragma unroll
-            for (int h = 0; h < kQc / 32; ++h) {
+            for (int h = 0; h < kXCols / 32; ++h) {
                 uint32_t wv[16];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint4 v = live ? src[4 * h + j] : make_uint4(0, 0, 0, 0);
                     wv[4 * j] = v.x; wv[4 * j + 1] = v.y; wv[4 * j + 2] = v.z; wv[4 * j + 3] = v.w;
                 }
-                tmem_st16(t_q + lane_off + part * (kQc / 2) + 16 * h, wv);
+                tmem_st16(t_q + lane_off + (kXCols / 2) * xpart + 16 * h, wv);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(q_full);
         };
-        const bool quad_live = 32 * quad < rows_here;  // rows_here is a multiple of 32
-        bool q_loaded = false;                         // q~ of the coming piece already in TMEM
+        // the first two tiles' P buffers expect the peer's rows
+        if (xw == 0 && lane == 0) {
+            mbar_arrive_expect_tx(&p_full[0], SM::kPRemote);
+            mbar_arrive_expect_tx(&p_full[1], SM::kPRemote);
+        }
+        bool q_loaded = false;  // q~ of the coming piece already in TMEM
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
         uint32_t t = 0, k = 0;
         while (next_piece(p, it, b, L, pb, pe, too_long)) {
             if (too_long) continue;
-            float m_run = -INFINITY, l_run = 0.0f;  // this row, this warp's tokens of every tile
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
-            // query s of this row sees tokens t <= L - s_q + s
-            const int last_visible = L - p.s_q + s_of_row;
             const uint32_t t0 = t;
             const int nt = pe - pb;
             if (!q_loaded) copy_q(b);
             q_loaded = false;
-            // stage A of tile i: this warp's partial scores -> fp16 -> the peer's receive buffer
-            auto stage_a = [&](int i, uint32_t (&h2)[kPr]) {
+            auto stage_a = [&](int i) {
                 const uint32_t tt = t0 + i;
                 const int sb = tt & 1;
                 if (!GQLA_WAIT(6, &s_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
+                GQLA_SPAN_BEGIN(t_a);
                 tc_fence_after();
-                uint32_t sv[kTokW];
-#pragma unroll
-                for (int c16 = 0; c16 < kTokW; c16 += 16)
-                    tmem_ld16(t_s + lane_off + sb * kT + part * kTokW + c16, sv + c16);
+                uint32_t sv[kXTok];
+                tmem_ld16(t_s + lane_off + sb * kT + kXTok * xpart, sv);
+                tmem_ld16(t_s + lane_off + sb * kT + kXTok * xpart + 16, sv + 16);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&s_free[sb]);
+                uint32_t h2[kXTok / 2];
 #pragma unroll
-                for (int j = 0; j < kPr; ++j) {
+                for (int j = 0; j < kXTok / 2; ++j) {
                     __half2 v = __floats2half2_rn(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
                     h2[j] = *reinterpret_cast<uint32_t *>(&v);
                 }
-                if (w == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kX);
-                // the peer's receive buffer sb is free once it has read tile tt - 2
+                // receive buffers sb of both CTAs are free once tile tt - 2 has been read
                 if (!GQLA_WAITC(7, &x_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                if (xw == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kXRemote);
+                const uint32_t roff = sb * SM::kX + (rank * kOwn + a_orow) * (kT * 2);
 #pragma unroll
-                for (int j = 0; j < kPr / 4; ++j)
-                    st_async_v4(x_remote + sb * SM::kX + 16 * j,
-                                make_uint4(h2[4 * j], h2[4 * j + 1], h2[4 * j + 2], h2[4 * j + 3]),
-                                xfull_remote + sb * 8);
-            };
-            uint32_t hc[kPr];
-            stage_a(0, hc);
-            bool have_next = false;  // stage A of tile i + 1 already done
-            int page = prow[pb];
-            for (int i = 0; i < nt; ++i) {
-                // Tile i + 1's exchange is started early only when its scores are
-                // already there: waiting for them here would tie the release of
-                // tile i (and of its ring slot) to the arrival of the next tile.
-                uint32_t hn[kPr];
-                const bool next_ready =
-                    i + 1 < nt && __shfl_sync(0xffffffffu,  // one decision per warp
-                                              (int)mbar_test_wait(&s_full[(t0 + i + 1) & 1], ((t0 + i + 1) >> 1) & 1), 0);
-                if (next_ready) {
-                    stage_a(i + 1, hn);
-                    have_next = true;
+                for (int q = 0; q < 4; ++q) {  // 16-byte chunks 4 xpart + q of the row, swizzled
+                    const uint32_t coff = roff + ((((kXTok / 8) * xpart + q) ^ (a_orow & 7)) << 4);
+                    const uint4 v = make_uint4(h2[4 * q], h2[4 * q + 1], h2[4 * q + 2], h2[4 * q + 3]);
+                    if (a_owner == rank)
+                        *reinterpret_cast<uint4 *>(smem + SM::oX + coff) = v;
+                    else
+                        st_async_v4(x_remote + coff, v, xfull_remote + sb * 8);
                 }
-                const int page_next = i + 1 < nt ? prow[pb + i + 1] : 0;  // in flight meanwhile
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&x_full[sb]);  // this warp's local partials are in
+                GQLA_SPAN_END(13, t_a);
+            };
+            auto stage_c = [&](int i, int page) {
                 const uint32_t tt = t0 + i;
-                const int pg = pb + i;
-                const int tok0 = pg * kPage;  // first token of this tile
                 const int sb = tt & 1, slot = tt % kRing;
                 const bool bad = page < 0 || page >= p.num_pages;
-                const int n_valid = bad ? 0 : max(0, min(kT, L - tok0));
-                GQLA_SPAN_BEGIN(t_tile);
-                // ---- full raw scores = own + peer (the same rounded partials in both CTAs)
-                if (!GQLA_WAITC(8, &x_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
-                __half2 x[kPr];
-                GQLA_SPAN_BEGIN(b1);
-                {
-                    const uint4 *src =
-                        reinterpret_cast<const uint4 *>(xbuf + sb * SM::kX + w * SM::kXw + lane * (kTokW * 2));
-#pragma unroll
-                    for (int j4 = 0; j4 < kPr / 4; ++j4) {
-                        const uint4 pv = src[j4];
-                        const uint32_t pw4[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            x[4 * j4 + e] = __hadd2(*reinterpret_cast<const __half2 *>(&hc[4 * j4 + e]),
-                                                    *reinterpret_cast<const __half2 *>(&pw4[e]));
-                    }
-                }
-                // the peer may refill our receive buffer sb (the values above are consumed)
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote + sb * 8);
-                GQLA_SPAN_END(20, b1);
-                GQLA_SPAN_BEGIN(b2);
-                // ---- mask tokens past the sequence or past this query's causal limit
-                const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + part * kTokW);
-                if (lim < kTokW - 1) {
-                    const __half ninf = __ushort_as_half((unsigned short)0xFC00u);
-#pragma unroll
-                    for (int j = 0; j < kPr; ++j) {
-                        if (2 * j > lim) x[j].x = ninf;
-                        if (2 * j + 1 > lim) x[j].y = ninf;
-                    }
-                }
-                // ---- row maximum over the 64 tokens (exchange among the quadrant's warps)
-                __half2 hm;
-                {
-                    __half2 tr[kPr];
-#pragma unroll
-                    for (int j = 0; j < kPr; ++j) tr[j] = x[j];
-#pragma unroll
-                    for (int st = kPr / 2; st >= 1; st >>= 1)
-#pragma unroll
-                        for (int j = 0; j < st; ++j) tr[j] = __hmax2(tr[j], tr[j + st]);
-                    hm = tr[0];
-                }
-                const float mx = fmaxf(__low2float(hm), __high2float(hm)) * p.scale_log2;  // log2 units
-                rm[((tt & 1) * kParts + part) * kRows + row] = mx;
-                quad_bar(quad);
-                float mt = mx;
-#pragma unroll
-                for (int q = 0; q < kParts; ++q) mt = fmaxf(mt, rm[((tt & 1) * kParts + q) * kRows + row]);
-                GQLA_SPAN_END(21, b2);
-                const bool first = i == 0;
-                float m_new = m_run;
-                if (first || mt > m_run + kRescaleLog2) m_new = mt;
-                const bool need = !first && m_new != m_run;
-                const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;
-                // P buffer sb is free once PV(tt - 2) completed
-                if (!GQLA_WAIT(9, &p_free[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, need)) {
+                const int n_valid = bad ? 0 : max(0, min(kT, L - (pb + i) * kPage));
+                if (!GQLA_WAITC(11, &p_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
+                GQLA_SPAN_BEGIN(t_c);
+                if (xw == 0 && lane == 0) mbar_arrive_expect_tx(&p_full[sb], SM::kPRemote);  // tile tt + 2
+                const float alpha = alph[sb * kRows + row];
+                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
                     // O rows are rescaled only after PV(tt - 1) has completed
-                    if (!first)
-                        if (!mbar_wait(&p_free[sb ^ 1], ((tt - 1) >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    if (i > 0)
+                        if (!mbar_wait(&pv_done[(tt - 1) & 1], ((tt - 1) >> 1) & 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
 #pragma unroll 1
-                    for (int c16 = 0; c16 < 256 / kParts; c16 += 16) {  // this warp's share of the O columns
+                    for (int c16 = 0; c16 < kXCols; c16 += 16) {
                         uint32_t r[16];
-                        const uint32_t ta = t_o + lane_off + part * (256 / kParts) + c16;
+                        const uint32_t ta = t_o + lane_off + kXCols * xpart + c16;
                         tmem_ld16(ta, r);
                         tmem_wait_ld();
 #pragma unroll
@@ -541,61 +489,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     tmem_wait_st();
                 }
-                l_run = first ? 0.0f : l_run * alpha;
-                m_run = m_new;
-                // ---- P = 2^(x scale - m) (fp32 ex2) in bf16 -- the top half of the fp32
-                // value, rounded towards zero; the row sum adds the same truncated values,
-                // so O / l stays unbiased -- into shared memory: bytes
-                // [2 kTokW part, 2 kTokW (part + 1)) of the row
-                GQLA_SPAN_BEGIN(b3);
-                const float mu = m_run == -INFINITY ? 0.0f : m_run;
-                uint32_t pw[kPr];
-                float lsum = 0.0f;
-#pragma unroll
-                for (int j = 0; j < kPr; ++j) {
-                    const float2 xf = __half22float2(x[j]);
-                    const uint32_t p0 = __float_as_uint(fast_exp2(fmaf(xf.x, p.scale_log2, -mu)));
-                    const uint32_t p1 = __float_as_uint(fast_exp2(fmaf(xf.y, p.scale_log2, -mu)));
-                    pw[j] = __byte_perm(p0, p1, 0x7632);
-                    lsum += __uint_as_float(p0 & 0xFFFF0000u) + __uint_as_float(p1 & 0xFFFF0000u);
-                }
-                l_run += lsum;
-                GQLA_SPAN_END(22, b3);
-                GQLA_SPAN_BEGIN(b4);
-                {
-                    uint8_t *prow_s = smem + SM::oP + sb * SM::kP + row * 128;
-#pragma unroll
-                    for (int j = 0; j < kPr / 4; ++j)
-                        *reinterpret_cast<uint4 *>(prow_s + (((part * (kPr / 4) + j) ^ (row & 7)) << 4)) =
-                            make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
-                }
                 // latent rows that are not tokens (never written, maybe NaN) -> 0
                 if (n_valid < kT) {
                     if (!mbar_wait(&ring_full[slot], (tt / kRing) & 1, abort_flag)) *abort_flag = 1;
                     uint8_t *tile = smem + SM::oRing + slot * SM::kSlot;
                     const int nz = kT - n_valid;
-                    for (int z = w * 32 + lane; z < 4 * nz * 8; z += kSmThreads) {
+                    for (int z = xw * 32 + lane; z < 4 * nz * 8; z += kXThreads) {
                         const int box = z / (nz * 8), rem = z % (nz * 8);
                         *reinterpret_cast<uint4 *>(tile + box * SM::kLatBox + (n_valid + rem / 8) * 128 +
                                                    (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
                     }
+                    fence_proxy_async_smem();
                 }
-                fence_proxy_async_smem();  // P (and any zeroed rows) -> the PV MMA
                 tc_fence_before();
-                mbar_arrive(&p_full[sb]);
-                GQLA_SPAN_END(23, b4);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&o_ready[sb]);
+                GQLA_SPAN_END(18, t_c);
+            };
+            int page_prev = 0;
+            for (int j = 0; j <= nt; ++j) {
+                const int page_j = j < nt ? prow[pb + j] : 0;
+                GQLA_SPAN_BEGIN(t_tile);
+                if (j < nt) {
+                    stage_a(j);
+                    // the last scores of the piece are read: the producer may load the next RoPE q~
+                    if (j == nt - 1) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(q_empty);
+                    }
+                }
+                if (j >= 1) stage_c(j - 1, page_prev);
                 GQLA_SPAN_END(10, t_tile);
-                if (i + 1 < nt && !have_next) stage_a(i + 1, hn);
-                have_next = false;
-                page = page_next;
-#pragma unroll
-                for (int j = 0; j < kPr; ++j) hc[j] = hn[j];
+                page_prev = page_j;
             }
             t = t0 + nt;
-            // the last scores of the piece are read: the producer may load the next RoPE q~,
-            // and the next piece's q~ goes into TMEM now, so that its scores overlap this epilogue
-            __syncwarp();
-            if (lane == 0) mbar_arrive(q_empty);
+            // the next piece's q~ goes into TMEM now, so that its scores overlap this epilogue
             bool more_pieces;
             {
                 PieceIter nx = it;
@@ -609,85 +537,196 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     q_loaded = true;
                 }
             }
-            // ---- epilogue: O / l for this CTA's 256 columns (this warp: 256 / kParts) through
-            // TMA stores staged in shared memory.  After the last piece the ring is free
-            // (every tile is consumed) and holds all of it: 8 KB per warp, two 128-byte-swizzled
-            // boxes, one store round.  Between pieces the ring holds the next piece's tiles, so
-            // each warp stages 2 KB at a time in the P buffers (free once the piece's last PV
-            // is done).  LSE by rank 0.
+            // ---- epilogue: O / l for this warp's 32 rows x 128 columns through TMA stores of
+            // 32 x 32 fp32 boxes (128-byte swizzle) staged in shared memory.  After the last
+            // piece the ring is free (every tile is consumed) and holds all of it, one store
+            // round; between pieces the ring holds the next piece's tiles and each warp stages
+            // one box at a time in the P buffers (free once the piece's last PV is done; P of
+            // the next piece is written only after this warp's next scores).
             GQLA_SPAN_BEGIN(t_epi);
             if (!GQLA_WAIT(15, o_done, k & 1, abort_flag)) *abort_flag = 1;
+            if (!GQLA_WAIT(12, l_full, k & 1, abort_flag)) *abort_flag = 1;
             tc_fence_after();
-            lsm[part * kRows + row] = l_run;
-            quad_bar(quad);
-            float l = 0.0f;
-#pragma unroll
-            for (int q = 0; q < kParts; ++q) l += lsm[q * kRows + row];
+            const float l = lsm[row];
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            const bool live = row < rows_here;
-            const int64_t orow = (int64_t)(b + c) * p.rows_total + grow;  // slot b + c
             const int orow0 = (b + c) * p.rows_total + rb * kRows + 32 * quad;
-            const int ocol0 = 256 * (int)rank + part * (256 / kParts);
-            if (!more_pieces) {
-                uint8_t *stg = smem + SM::oRing + w * 8192;  // [2 boxes][32 rows][128 B]
+            const int ocol0 = 256 * (int)rank + kXCols * xpart;
+            const bool last = !more_pieces;
+            uint8_t *stg0 = last ? smem + SM::oRing + xw * (kXCols * 128) : smem + SM::oP + xw * 4096;
+#pragma unroll 1
+            for (int m = 0; m < kXCols / 32; ++m) {
+                uint8_t *stg = last ? stg0 + m * 4096 : stg0;
+                if (!last && m > 0) {
+                    if (lane == 0) bulk_wait_group_read<0>();  // the previous box's store has read stg
+                    __syncwarp();
+                }
 #pragma unroll
-                for (int j = 0; j < 256 / kParts / 16; ++j) {
+                for (int h = 0; h < 2; ++h) {
                     uint32_t r[16];
-                    tmem_ld16(t_o + lane_off + part * (256 / kParts) + 16 * j, r);
+                    tmem_ld16(t_o + lane_off + kXCols * xpart + 32 * m + 16 * h, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {  // 128-byte swizzle: chunk ^= row % 8
-                        const int chunk = (j & 1) * 4 + q4;
-                        *reinterpret_cast<float4 *>(stg + (j >> 1) * 4096 + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                    for (int q4 = 0; q4 < 4; ++q4)  // 128-byte swizzle: chunk ^= row % 8
+                        *reinterpret_cast<float4 *>(stg + lane * 128 + (((4 * h + q4) ^ (lane & 7)) << 4)) =
                             make_float4(__uint_as_float(r[4 * q4]) * inv, __uint_as_float(r[4 * q4 + 1]) * inv,
                                         __uint_as_float(r[4 * q4 + 2]) * inv, __uint_as_float(r[4 * q4 + 3]) * inv);
-                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && quad_live && !*abort_flag) {
-                    tma_store_2d(&o_map_wide, stg, ocol0, orow0);
-                    tma_store_2d(&o_map_wide, stg + 4096, ocol0 + 32, orow0);
+                    tma_store_2d(&o_map, stg, ocol0 + 32 * m, orow0);
                     bulk_commit_group();
                 }
-            } else {
-                uint8_t *stg = smem + SM::oP + w * 2048;  // [32 rows][16 fp32], 64-byte swizzle
-#pragma unroll 1
-                for (int j = 0; j < 256 / kParts / 16; ++j) {
-                    if (j > 0) {
-                        if (lane == 0) bulk_wait_group_read<0>();  // the previous chunk's store has read stg
-                        __syncwarp();
-                    }
-                    uint32_t r[16];
-                    tmem_ld16(t_o + lane_off + part * (256 / kParts) + 16 * j, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)  // 64-byte swizzle: chunk ^= (row / 2) % 4
-                        *reinterpret_cast<float4 *>(stg + lane * 64 + ((q4 ^ ((lane >> 1) & 3)) << 4)) =
-                            make_float4(__uint_as_float(r[4 * q4]) * inv, __uint_as_float(r[4 * q4 + 1]) * inv,
-                                        __uint_as_float(r[4 * q4 + 2]) * inv, __uint_as_float(r[4 * q4 + 3]) * inv);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && quad_live && !*abort_flag) {
-                        tma_store_2d(&o_map_narrow, stg, ocol0 + 16 * j, orow0);
-                        bulk_commit_group();
-                    }
-                }
-                if (lane == 0) bulk_wait_group_read<0>();
-                // every warp's staging (spread over all the P rows) is read before any P is rewritten
-                softmax_bar();
             }
-            if (live && rank == 0 && part == 0)
-                p.lse_part[orow] = (l > 0.0f && m_run != -INFINITY)
-                                       ? (m_run + __log2f(l)) * 0.6931471805599453f
-                                       : -INFINITY;
+            if (lane == 0) bulk_wait_group_read<0>();  // staging read before the next tiles' P
+            __syncwarp();
             tc_fence_before();
             GQLA_SPAN_END(16, t_epi);
             ++k;
         }
         if (lane == 0) bulk_wait_group<0>();  // the partials are written before the CTA exits
+    } else {
+        // ---------------------------------------------------------------- softmax warps
+        // Stage B of every tile for this CTA's 64 rows: both partial scores added, row
+        // maxima (lazy rescaling of O rows when a maximum rises by more than 2^8), P in
+        // bf16 written here and bulk-copied to the same rows of the peer's buffer, with
+        // each row's O rescale factor.  Four lanes per row, 16 tokens each.
+        const int yw = warp - 2 - kXWarps;
+        const int ob = 8 * yw + (lane >> 2);  // owned row index 0..63
+        const int brow = 32 * (ob >> 4) + 16 * (int)rank + (ob & 15);
+        const int bq4 = lane & 3;             // tokens [16 bq4, 16 bq4 + 16): chunks 2 bq4, 2 bq4 + 1
+        const int bgrow = rb * kRows + brow;
+        const int s_of_brow = bgrow < p.rows_total ? bgrow / p.heads : p.s_q - 1;
+        const bool blive = brow < rows_here;
+        float *alph = reinterpret_cast<float *>(smem + SM::oAlpha);
+        float *lsm = reinterpret_cast<float *>(smem + SM::oL);
+        const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
+        const uint32_t p_remote = map_peer(sm_p, peer);
+        const uint32_t pfull_remote = map_peer(smem_u32(p_full), peer);
+        const uint32_t alpha_remote = map_peer(smem_u32(alph), peer);
+        const uint32_t l_remote = map_peer(smem_u32(lsm), peer);
+        const uint32_t lfull_remote = map_peer(smem_u32(l_full), peer);
+        PieceIter it = it0;
+        int b, L, pb, pe;
+        bool too_long;
+        uint32_t t = 0;
+        while (next_piece(p, it, b, L, pb, pe, too_long)) {
+            if (too_long) continue;
+            float m_run = -INFINITY, l_run = 0.0f;  // the owned row (4 lanes' tokens)
+            const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
+            const int last_visible = L - p.s_q + s_of_brow;  // this row's query sees t <= this
+            const int nt = pe - pb;
+            int page = prow[pb];
+            for (int i = 0; i < nt; ++i, ++t) {
+                const int page_next = i + 1 < nt ? prow[pb + i + 1] : 0;  // in flight meanwhile
+                const uint32_t tt = t;
+                const int sb = tt & 1;
+                const int tok0 = (pb + i) * kPage;
+                const bool bad = page < 0 || page >= p.num_pages;
+                const int n_valid = bad ? 0 : max(0, min(kT, L - tok0));
+                GQLA_SPAN_BEGIN(t_b0);
+                if (!GQLA_WAITC(8, &x_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
+                GQLA_SPAN_BEGIN(t_b);
+                const uint8_t *xb = smem + SM::oX + sb * SM::kX;
+                uint4 u[2][2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t coff = ((2 * bq4 + h) ^ (ob & 7)) << 4;
+                    u[0][h] = *reinterpret_cast<const uint4 *>(xb + ob * (kT * 2) + coff);
+                    u[1][h] = *reinterpret_cast<const uint4 *>(xb + (kOwn + ob) * (kT * 2) + coff);
+                }
+                float x[16];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t a4[4] = {u[0][h].x, u[0][h].y, u[0][h].z, u[0][h].w};
+                    const uint32_t b4[4] = {u[1][h].x, u[1][h].y, u[1][h].z, u[1][h].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 fa = __half22float2(*reinterpret_cast<const __half2 *>(&a4[e]));
+                        const float2 fb = __half22float2(*reinterpret_cast<const __half2 *>(&b4[e]));
+                        x[8 * h + 2 * e] = fa.x + fb.x;
+                        x[8 * h + 2 * e + 1] = fa.y + fb.y;
+                    }
+                }
+                __syncwarp();
+                // both CTAs' buffers sb may be refilled once every softmax warp has read them
+                if (lane == 0) {
+                    mbar_arrive(&x_empty[sb]);
+                    mbar_arrive_remote_relaxed(xempty_remote + sb * 8);
+                }
+                // mask tokens past the sequence or past this query's causal limit
+                const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + 16 * bq4);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (e > lim) x[e] = -INFINITY;
+                float mx = x[0];
+#pragma unroll
+                for (int e = 1; e < 16; ++e) mx = fmaxf(mx, x[e]);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float mt = mx * p.scale_log2;  // log2 units
+                const bool first = i == 0;
+                float m_new = m_run;
+                if (first || mt > m_run + kRescaleLog2) m_new = mt;
+                const float alpha = (!first && m_new != m_run) ? fast_exp2(m_run - m_new) : 1.0f;
+                l_run = first ? 0.0f : l_run * alpha;
+                m_run = m_new;
+                // P = 2^(x scale - m) (fp32 ex2) in bf16 -- the top half of the fp32 value,
+                // rounded towards zero; the row sum adds the same truncated values
+                const float mu = m_run == -INFINITY ? 0.0f : m_run;
+                uint32_t pw[8];
+                float lsum = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t p0 = __float_as_uint(fast_exp2(fmaf(x[2 * e], p.scale_log2, -mu)));
+                    const uint32_t p1 = __float_as_uint(fast_exp2(fmaf(x[2 * e + 1], p.scale_log2, -mu)));
+                    pw[e] = __byte_perm(p0, p1, 0x7632);
+                    lsum += __uint_as_float(p0 & 0xFFFF0000u) + __uint_as_float(p1 & 0xFFFF0000u);
+                }
+                l_run += lsum;
+                GQLA_SPAN_END(14, t_b);
+                // P buffer sb of both CTAs is free once both PV(tt - 2) are done
+                if (!GQLA_WAIT(9, &p_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                GQLA_SPAN_BEGIN(t_b2);
+                uint8_t *prow_s = smem + SM::oP + sb * SM::kP + brow * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    *reinterpret_cast<uint4 *>(prow_s + (((2 * bq4 + h) ^ (brow & 7)) << 4)) =
+                        make_uint4(pw[4 * h], pw[4 * h + 1], pw[4 * h + 2], pw[4 * h + 3]);
+                if (bq4 == 0) {
+                    alph[sb * kRows + brow] = alpha;
+                    st_async_b32(alpha_remote + (sb * kRows + brow) * 4, __float_as_uint(alpha),
+                                 pfull_remote + sb * 8);
+                }
+                fence_proxy_async_smem();  // P -> the PV MMAs of both CTAs (async proxy)
+                __syncwarp();
+                if (lane == 0) {
+                    // this warp's 8 rows of P are 1 KB of contiguous rows: the same rows of the peer's buffer
+                    const uint32_t r0 = sb * SM::kP + brow * 128;
+                    bulk_copy_to_peer(p_remote + r0, smem + SM::oP + r0, 8 * 128, pfull_remote + sb * 8);
+                    mbar_arrive(&p_full[sb]);
+                }
+                GQLA_SPAN_END(17, t_b2);
+                GQLA_SPAN_END(19, t_b0);
+                page = page_next;
+            }
+            // ---- the owned rows' sums and LSE; the sums of all 128 rows are gathered in
+            // both CTAs' lsm for the score warps' epilogue
+            float l = l_run;
+            l += __shfl_xor_sync(0xffffffffu, l, 1);
+            l += __shfl_xor_sync(0xffffffffu, l, 2);
+            if (yw == 0 && lane == 0) mbar_arrive_expect_tx(l_full, kOwn * 4);
+            if (bq4 == 0) {
+                lsm[brow] = l;
+                st_async_b32(l_remote + brow * 4, __float_as_uint(l), lfull_remote);
+                if (blive)
+                    p.lse_part[(int64_t)(b + c) * p.rows_total + bgrow] =
+                        (l > 0.0f && m_run != -INFINITY) ? (m_run + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(l_full);
+        }
     }
-
     GQLA_PROF_FLUSH;
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) report_error(p.ws, GQLA_ERR_TIMEOUT, c);
@@ -712,7 +751,7 @@ bool make_row_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t bo
 cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
                                  const gqla_kv_index *idx, int num_splits, float scale,
                                  float *o_part, float *lse_part, void *ws, cudaStream_t stream) {
-    CUtensorMap lat, rope, qrope, omap_w, omap_n;
+    CUtensorMap lat, rope, qrope, omap;
     const uint64_t slots = (uint64_t)idx->num_pages * kPage;
     const uint64_t qrows = (uint64_t)idx->batch * s_q * heads;
     if (!make_row_map(&lat, cache, slots, 64, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -720,16 +759,13 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
         !make_row_map(&qrope, qa, qrows, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     {
-        // partials fp32 [B + C][s_q][h][512]: 32 x 32 boxes (128-byte rows) for the last
-        // piece's stores, 16 x 32 boxes for those between pieces
+        // partials fp32 [B + C][s_q][h][512], stored in 32 x 32 boxes (128-byte rows)
         const uint64_t orows = (uint64_t)(idx->batch + num_splits) * s_q * heads;
         const uint64_t dims[2] = {(uint64_t)kLatent, orows};
         const uint64_t strides[1] = {(uint64_t)kLatent * 4};
-        const uint32_t box_w[2] = {32, 32}, box_n[2] = {16, 32};
-        if (!make_map(&omap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, o_part, 2, dims, strides, box_w,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&omap_n, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, o_part, 2, dims, strides, box_n,
-                      CU_TENSOR_MAP_SWIZZLE_64B))
+        const uint32_t box[2] = {32, 32};
+        if (!make_map(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, o_part, 2, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
     AbsorbParams p;
@@ -753,7 +789,7 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)num_splits * p.row_blocks * 2;
     return launch_dependent(decode_absorb_tc_kernel, dim3(grid), dim3(kThreads), AbsorbSmem::kAlloc,
-                            stream, lat, rope, qrope, omap_w, omap_n, p);
+                            stream, lat, rope, qrope, omap, p);
 }
 
 }  // namespace gqla

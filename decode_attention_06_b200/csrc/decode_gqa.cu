@@ -459,16 +459,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!GQLA_WAIT(3, &k_full[ks_], (u / KS) & 1, abort_flag)) *abort_flag = 1;
                         if (!GQLA_WAIT(4, &s_free[sb], ((u >> 2) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                         tc_fence_after();
-                        const uint32_t kst = sm_k + ks_ * SM::kKSlotBytes;
-                        const uint32_t qg = kst + SM::kKBytes;
+                        // descriptors from the slot bases: each MMA only adds an offset
+                        const uint64_t k_d = smem_desc(sm_k + ks_ * SM::kKSlotBytes, 16, 1024, kSw128);
+                        const uint64_t q_d = desc_advance(k_d, SM::kKBytes);
+                        const uint64_t kr_d = smem_desc(kr, 16, 1024, kSw128);
                         if (!*abort_flag) {
 #pragma unroll
                             for (int ks = 0; ks < 12; ++ks) {
-                                const uint32_t a = ks < 8 ? kst + (ks >> 2) * 2 * kBox + (ks & 3) * 32
-                                                          : kr + (ks - 8) * 32;
-                                const uint32_t bq = qg + (ks >> 2) * NQ * 128 + (ks & 3) * 32;
-                                mma_bf16(t_s + sb * NQ, smem_desc(a, 16, 1024, kSw128),
-                                         smem_desc(bq, 16, 1024, kSw128), idesc_s, ks > 0 ? 1u : 0u);
+                                const uint64_t ad = ks < 8 ? desc_advance(k_d, (ks >> 2) * 2 * kBox + (ks & 3) * 32)
+                                                           : desc_advance(kr_d, (ks - 8) * 32);
+                                const uint64_t bd = desc_advance(q_d, (ks >> 2) * NQ * 128 + (ks & 3) * 32);
+                                mma_bf16(t_s + sb * NQ, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
                             }
                         }
                         mma_commit(&s_full[sb]);
@@ -490,6 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc_pv = idesc_bf16(128, NQ, 1, 1);
             constexpr uint32_t p_sw = NQ == 16 ? kSw32 : kSw64;
             constexpr uint32_t p_sbo = NQ == 16 ? 256 : 512;
+            const uint64_t v_d0 = smem_desc(sm_v, 2 * kBox, 1024, kSw128);
+            const uint64_t p_d0 = smem_desc(sm_p, SM::kPBytes, p_sbo, p_sw);
             PieceIter it = it0;
             int b, L, pb, pe;
             bool too_long;
@@ -503,15 +506,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!GQLA_WAIT(5, &p_full[w], (u >> 1) & 1, abort_flag)) *abort_flag = 1;
                         if (!GQLA_WAIT(13, &v_full[vs], (u / VS) & 1, abort_flag)) *abort_flag = 1;
                         tc_fence_after();
-                        const uint32_t v_lo = sm_v + vs * SM::kVBytes;
-                        const uint32_t pa = sm_p + w * SM::kPBytes;
+                        const uint64_t v_d = desc_advance(v_d0, vs * SM::kVBytes);
+                        const uint64_t p_d = desc_advance(p_d0, w * SM::kPBytes);
                         if (!*abort_flag) {
 #pragma unroll
-                            for (int ks = 0; ks < kTok / 16; ++ks) {
-                                uint64_t ad = smem_desc(v_lo + ks * 2048, 2 * kBox, 1024, kSw128);
-                                uint64_t bd = smem_desc(pa + ks * 16 * NQ * 2, SM::kPBytes, p_sbo, p_sw);
-                                mma_bf16(t_o + gi * NQ, ad, bd, idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
-                            }
+                            for (int ks = 0; ks < kTok / 16; ++ks)
+                                mma_bf16(t_o + gi * NQ, desc_advance(v_d, ks * 2048), desc_advance(p_d, ks * 16 * NQ * 2),
+                                         idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
                         }
                         mma_commit(&p_free[w]);
                         mma_commit(&v_empty[vs]);

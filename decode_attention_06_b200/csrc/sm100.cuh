@@ -268,6 +268,16 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
         : "memory");
 }
 
+// Commit arriving on the mbarrier at the same shared-memory offset in every CTA
+// of `cta_mask` (bit r: cluster rank r).
+__device__ __forceinline__ void mma_commit_multicast(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -396,6 +406,15 @@ __device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, uint4 v, uint3
         : "memory");
 }
 
+// Asynchronous 4-byte store into a peer CTA's shared memory; completes 4 bytes
+// of the transaction count of the peer's mbarrier.
+__device__ __forceinline__ void st_async_b32(uint32_t dst_cluster, uint32_t v, uint32_t mbar_cluster) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                     dst_cluster),
+                 "r"(v), "r"(mbar_cluster)
+                 : "memory");
+}
+
 // Arrive on a peer CTA's mbarrier without ordering this thread's memory accesses.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
@@ -445,6 +464,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     d |= static_cast<uint64_t>(1u) << 46;
     d |= static_cast<uint64_t>(swizzle & 7u) << 61;
     return d;
+}
+
+// The descriptor of the same layout `bytes` further on (the start address field,
+// bits 0-13, holds address / 16 and stays below 2^14 for every shared address).
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+    return desc + static_cast<uint64_t>(bytes >> 4);
 }
 
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M x N, operand majors
