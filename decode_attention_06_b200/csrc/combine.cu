@@ -115,10 +115,14 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
     const int64_t row0 = ((int64_t)(b + c0) * p.s_q + s) * p.heads + h0;
     const int64_t part_stride = (int64_t)p.s_q * p.heads;
 
-    float M[4];
+    // LSE of partial c = lane (the first 32), kept for the weights of the first block
+    float l0[4], M[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) M[i] = -INFINITY;
-    for (int c = lane; c < nparts; c += 32)
+    for (int i = 0; i < 4; ++i) {
+        l0[i] = lane < nparts ? __ldg(p.lse_part + row0 + lane * part_stride + i) : -INFINITY;
+        M[i] = l0[i];
+    }
+    for (int c = lane + 32; c < nparts; c += 32)
 #pragma unroll
         for (int i = 0; i < 4; ++i) M[i] = fmaxf(M[i], __ldg(p.lse_part + row0 + c * part_stride + i));
 #pragma unroll
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
         const int c = cb + lane;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float l = c < nparts ? __ldg(p.lse_part + row0 + c * part_stride + i) : -INFINITY;
+            const float l = cb == 0 ? l0[i] : c < nparts ? __ldg(p.lse_part + row0 + c * part_stride + i) : -INFINITY;
             w[i] = l == -INFINITY ? 0.0f : __expf(l - M[i]);
             den[i] += w[i];
         }
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
 constexpr int kClThreads = 512;
 constexpr int kClRows = 64;      // rows of a tile (MMA M)
 constexpr int kClMaxPairs = 32;  // bst <= 64 / 4 = 16
-constexpr int kClChunk = 32;     // partials whose weights are staged at a time
+constexpr int kClChunk = 16;     // partials whose weights are staged at a time
 
 struct ClSmem {
     static constexpr int kAHalf = kClRows * 256 * 2;       // one CTA's 4 K blocks of A
@@ -261,30 +265,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     cluster_sync();  // barriers of both CTAs initialised before any remote transfer
     tc_fence_after();
 
-    // ---- threads 0..63: one row each -- max LSE, then weights per chunk
-    float den = 0.0f, Mr = -INFINITY;
-    const float *lse_row = p.lse_part;
-    int np_r = 0;
-    bool live_r = false;
-    if (tid < kClRows) {
-        const int j = tid / p.G;
-        live_r = tid < rows_in_tile && bs0 + j < p.bs_total;
-        if (live_r) {
-            const int bs = bs0 + j, b = bs / p.s_q, s = bs % p.s_q;
-            np_r = s_c1[j] - s_c0[j];
-            lse_row = p.lse_part + ((int64_t)(b + s_c0[j]) * p.s_q + s) * p.heads + grp * p.G +
-                      tid % p.G;
-        }
-        for (int c = 0; c < np_r; c += 8) {
-            float l[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                l[k] = c + k < np_r ? __ldg(lse_row + (c + k) * part_stride) : -INFINITY;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) Mr = fmaxf(Mr, l[k]);
-        }
-    }
-
     // ---- merge: warp w owns rows 4w .. 4w+3; lane j covers columns 4j and 128 + 4j of
     // this CTA's 256 latent columns; two partials are read per step
     constexpr int kRw = kClRows / (kClThreads / 32);  // rows per warp
@@ -305,14 +285,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
                      kLatent +
                  kq * 256 + lane * 4;
     }
+    float4 v[2][kRw][2];
+    auto load2 = [&](int c) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int i = 0; i < kRw; ++i) {
+                const bool on = c + u < npr[i];
+                const float *q = src[i] + (int64_t)(c + u) * part_stride * kLatent;
+                v[u][i][0] = on ? ldg4(q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[u][i][1] = on ? ldg4(q + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+    };
+
+    // ---- threads 0..63: one row each -- max LSE and the weights of its partials
+    // (one pass while a row has at most kClChunk partials)
+    float den = 0.0f, Mr = -INFINITY;
+    const float *lse_row = p.lse_part;
+    int np_r = 0;
+    bool live_r = false;
     const int maxp = *s_maxp;
+    if (tid < kClRows) {
+        const int j = tid / p.G;
+        live_r = tid < rows_in_tile && bs0 + j < p.bs_total;
+        if (live_r) {
+            const int bs = bs0 + j, b = bs / p.s_q, s = bs % p.s_q;
+            np_r = s_c1[j] - s_c0[j];
+            lse_row = p.lse_part + ((int64_t)(b + s_c0[j]) * p.s_q + s) * p.heads + grp * p.G +
+                      tid % p.G;
+        }
+        if (maxp > kClChunk) {
+            for (int c = 0; c < np_r; c += 8) {
+                float l[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    l[k] = c + k < np_r ? __ldg(lse_row + (c + k) * part_stride) : -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) Mr = fmaxf(Mr, l[k]);
+            }
+        }
+    }
     for (int cb = 0; cb < maxp; cb += kClChunk) {
-        __syncthreads();  // the previous chunk's weights are consumed
+        if (cb > 0) __syncthreads();  // the previous chunk's weights are consumed
         if (tid < kClRows) {
             float l[kClChunk];
 #pragma unroll
             for (int k = 0; k < kClChunk; ++k)
                 l[k] = cb + k < np_r ? __ldg(lse_row + (cb + k) * part_stride) : -INFINITY;
+            if (maxp <= kClChunk) {
+#pragma unroll
+                for (int k = 0; k < kClChunk; ++k) Mr = fmaxf(Mr, l[k]);
+            }
 #pragma unroll
             for (int k = 0; k < kClChunk; ++k) {
                 const float w = l[k] == -INFINITY ? 0.0f : __expf(l[k] - Mr);
@@ -324,16 +347,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         const int n = min(kClChunk, maxp - cb);
 #pragma unroll 1
         for (int j0 = 0; j0 < n; j0 += 2) {
-            float4 v[2][kRw][2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int i = 0; i < kRw; ++i) {
-                    const bool on = cb + j0 + u < npr[i];
-                    const float *q = src[i] + (int64_t)(cb + j0 + u) * part_stride * kLatent;
-                    v[u][i][0] = on ? ldg4(q) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[u][i][1] = on ? ldg4(q + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
+            load2(cb + j0);
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -396,14 +410,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         if (ok) {
             tc_fence_after();
             constexpr uint32_t idesc = idesc_bf16(kClRows, 128, 0, 1);
-            const uint32_t a0 = smem_u32(smem + ClSmem::oA), b0 = smem_u32(smem + ClSmem::oB);
+            const uint64_t a_d = smem_desc(smem_u32(smem + ClSmem::oA), 16, 1024, kSw128);
+            const uint64_t b_d = smem_desc(smem_u32(smem + ClSmem::oB), 65536, 1024, kSw128);
 #pragma unroll
-            for (int kk = 0; kk < kLatent / 16; ++kk) {
-                const uint64_t ad =
-                    smem_desc(a0 + (kk >> 2) * (kClRows * 128) + (kk & 3) * 32, 16, 1024, kSw128);
-                const uint64_t bd = smem_desc(b0 + kk * 2048, 65536, 1024, kSw128);
-                mma_bf16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
-            }
+            for (int kk = 0; kk < kLatent / 16; ++kk)
+                mma_bf16(tmem, desc_advance(a_d, (kk >> 2) * (kClRows * 128) + (kk & 3) * 32),
+                         desc_advance(b_d, kk * 2048), idesc, kk > 0 ? 1u : 0u);
             mma_commit(done);
         } else {
             *abort_flag = 1;
