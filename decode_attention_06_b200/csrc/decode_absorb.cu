@@ -73,8 +73,11 @@ struct AbsorbSmem {
     static constexpr int kLatBox = kT * 128;              // [64 tokens][64 cols]
     static constexpr int kRopeBox = kT * 64;              // [64 tokens][32 cols]
     static constexpr int kSlot = 4 * kLatBox + kRopeBox;  // 36 KB
-    // partial scores of this CTA's 64 rows: [2 sources][64 rows][64 tokens] fp16, the
-    // 16-byte chunks of a row XOR-swizzled by row % 8; the peer's half arrives by st.async
+    // partial scores of this CTA's 64 rows, fp16, in 1 KB blocks
+    // [2 sources][2 token halves][4 lane quadrants][16 rows][32 tokens]: one block is what
+    // one score warp computes for the rows of one owner, so the peer's blocks arrive as
+    // whole bulk copies; 16-byte chunks of a block row XOR-swizzled by (row / 2) % 4
+    static constexpr int kXBlock = 16 * 64;
     static constexpr int kX = 2 * kOwn * kT * 2;
     static constexpr int kXRemote = kOwn * kT * 2;
     static constexpr int kP = kRows * kT * 2;             // P, [128 rows][64 tokens] bf16, 128B-swizzled
@@ -84,7 +87,8 @@ struct AbsorbSmem {
     static constexpr int oP = oQ + kQRope;                // 2 buffers
     static constexpr int oRing = oP + 2 * kP;
     static constexpr int oX = oRing + kRing * kSlot;      // 2 buffers
-    static constexpr int oAlpha = oX + 2 * kX;            // float [2 buffers][128 rows]
+    static constexpr int oXStage = oX + 2 * kX;           // [8 score warps] outgoing blocks
+    static constexpr int oAlpha = oXStage + kXWarps * kXBlock;  // float [2 buffers][128 rows]
     static constexpr int oL = oAlpha + 2 * kRows * 4;     // float [128 rows]: row sums of a piece
     static constexpr int oBar = oL + kRows * 4;
     // ring_full/empty[kRing], q_full, q_empty, s_full/s_free[2], x_full/x_empty[2],
@@ -449,17 +453,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // receive buffers sb of both CTAs are free once tile tt - 2 has been read
                 if (!GQLA_WAITC(7, &x_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                 if (xw == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kXRemote);
-                const uint32_t roff = sb * SM::kX + (rank * kOwn + a_orow) * (kT * 2);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {  // 16-byte chunks 4 xpart + q of the row, swizzled
-                    const uint32_t coff = roff + ((((kXTok / 8) * xpart + q) ^ (a_orow & 7)) << 4);
-                    const uint4 v = make_uint4(h2[4 * q], h2[4 * q + 1], h2[4 * q + 2], h2[4 * q + 3]);
-                    if (a_owner == rank)
-                        *reinterpret_cast<uint4 *>(smem + SM::oX + coff) = v;
-                    else
-                        st_async_v4(x_remote + coff, v, xfull_remote + sb * 8);
+                // this warp's block for each owner: rows 16 quad .. 16 quad + 15 of the owner,
+                // tokens 32 xpart .. 32 xpart + 31; the peer's block goes out by bulk copy
+                const uint32_t blk = (((rank * 2 + xpart) * 4 + quad) * SM::kXBlock);
+                uint8_t *dst = a_owner == rank ? smem + SM::oX + sb * SM::kX + blk : smem + SM::oXStage + xw * SM::kXBlock;
+                const int r16 = lane & 15;
+                if (tt > 0) {
+                    // the previous tile's outgoing block has been read by its bulk copy
+                    if (lane == 0) bulk_wait_group_read<0>();
+                    __syncwarp();
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(dst + r16 * 64 + ((q ^ ((r16 >> 1) & 3)) << 4)) =
+                        make_uint4(h2[4 * q], h2[4 * q + 1], h2[4 * q + 2], h2[4 * q + 3]);
+                fence_proxy_async_smem();  // the outgoing block -> the bulk copy (async proxy)
                 __syncwarp();
+                if (lane == 0) {
+                    bulk_copy_to_peer(x_remote + sb * SM::kX + blk, smem + SM::oXStage + xw * SM::kXBlock,
+                                      SM::kXBlock, xfull_remote + sb * 8);
+                    bulk_commit_group();
+                }
                 if (lane == 0) mbar_arrive(&x_full[sb]);  // this warp's local partials are in
                 GQLA_SPAN_END(13, t_a);
             };
@@ -627,13 +641,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 GQLA_SPAN_BEGIN(t_b0);
                 if (!GQLA_WAITC(8, &x_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
                 GQLA_SPAN_BEGIN(t_b);
-                const uint8_t *xb = smem + SM::oX + sb * SM::kX;
+                // this row's block from each source (token half bq4 / 2), chunks 2 (bq4 % 2), +1
+                const int bxp = bq4 >> 1, bq = ob >> 4, br = ob & 15;
                 uint4 u[2][2];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t coff = ((2 * bq4 + h) ^ (ob & 7)) << 4;
-                    u[0][h] = *reinterpret_cast<const uint4 *>(xb + ob * (kT * 2) + coff);
-                    u[1][h] = *reinterpret_cast<const uint4 *>(xb + (kOwn + ob) * (kT * 2) + coff);
+                for (int src2 = 0; src2 < 2; ++src2) {
+                    const uint8_t *blkp = smem + SM::oX + sb * SM::kX + (((src2 * 2 + bxp) * 4 + bq) * SM::kXBlock) + br * 64;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        u[src2][h] = *reinterpret_cast<const uint4 *>(blkp + (((2 * (bq4 & 1) + h) ^ ((br >> 1) & 3)) << 4));
                 }
                 // full scores = own partial + peer partial, added in fp16 (both rounded the same way)
                 __half2 x[8];
