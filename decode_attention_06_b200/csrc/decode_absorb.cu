@@ -396,17 +396,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const bool quad_live = 32 * quad < rows_here;  // rows_here is a multiple of 32
         // this warp's share of q~'s latent half (32 rows x 128 columns) into TMEM; the
         // previous piece's scores, its last readers, are complete
+        auto q_row = [&](int bq) {
+            return reinterpret_cast<const uint4 *>(p.qa + ((int64_t)bq * p.rows_total + grow) * kRow +
+                                                   256 * rank + kXCols * xpart);
+        };
         auto copy_q = [&](int bq) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.qa + ((int64_t)bq * p.rows_total + grow) * kRow + 256 * rank + kXCols * xpart);
+            const uint4 *src = q_row(bq);
             const bool live = row < rows_here;
+            uint4 v[kXCols / 8];  // the whole 256-byte share in one round trip
+#pragma unroll
+            for (int j = 0; j < kXCols / 8; ++j) v[j] = live ? src[j] : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int h = 0; h < kXCols / 32; ++h) {
                 uint32_t wv[16];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const uint4 v = live ? src[4 * h + j] : make_uint4(0, 0, 0, 0);
-                    wv[4 * j] = v.x; wv[4 * j + 1] = v.y; wv[4 * j + 2] = v.z; wv[4 * j + 3] = v.w;
+                    wv[4 * j] = v[4 * h + j].x; wv[4 * j + 1] = v[4 * h + j].y;
+                    wv[4 * j + 2] = v[4 * h + j].z; wv[4 * j + 3] = v[4 * h + j].w;
                 }
                 tmem_st16(t_q + lane_off + (kXCols / 2) * xpart + 16 * h, wv);
             }
@@ -432,6 +438,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int nt = pe - pb;
             if (!q_loaded) copy_q(b);
             q_loaded = false;
+            {
+                // the next piece's q~ share heads for L2 now; its copy into TMEM at the end of
+                // this piece then waits for L2, not for HBM
+                PieceIter nx = it;
+                int b2, L2, pb2, pe2;
+                bool tl2 = false, more;
+                do {
+                    more = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
+                } while (more && tl2);
+                if (more && row < rows_here) {
+                    const uint4 *nq = q_row(b2);
+                    prefetch_l2(nq);
+                    prefetch_l2(nq + 8);
+                }
+            }
             auto stage_a = [&](int i) {
                 const uint32_t tt = t0 + i;
                 const int sb = tt & 1;
