@@ -165,7 +165,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i) { mbar_init(&ring_full[i], 1); mbar_init(&ring_empty[i], 1); }
-        mbar_init(q_full, 1 + kXWarps);  // RoPE TMA + the score warps' TMEM copies
+        mbar_init(q_full, 1 + kYWarps);  // RoPE TMA + the softmax warps' TMEM copies
         mbar_init(q_empty, kXWarps);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1); mbar_init(&s_free[i], kXThreads);
@@ -386,47 +386,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int xpart = xw >> 2;
         const int row = 32 * quad + lane;        // TMEM row
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        const int grow = rb * kRows + row;       // row within the sequence's s_q * h rows
-        const uint32_t a_owner = (lane >> 4) & 1;
-        const int a_orow = 16 * quad + (lane & 15);  // this row's index among its owner's rows
+        const uint32_t a_owner = (lane >> 4) & 1;   // the owner of this row (stage A)
         const float *alph = reinterpret_cast<const float *>(smem + SM::oAlpha);
         const float *lsm = reinterpret_cast<const float *>(smem + SM::oL);
         const uint32_t x_remote = map_peer(smem_u32(smem + SM::oX), peer);
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
         const bool quad_live = 32 * quad < rows_here;  // rows_here is a multiple of 32
-        // this warp's share of q~'s latent half (32 rows x 128 columns) into TMEM; the
-        // previous piece's scores, its last readers, are complete
-        auto q_row = [&](int bq) {
-            return reinterpret_cast<const uint4 *>(p.qa + ((int64_t)bq * p.rows_total + grow) * kRow +
-                                                   256 * rank + kXCols * xpart);
-        };
-        auto copy_q = [&](int bq) {
-            const uint4 *src = q_row(bq);
-            const bool live = row < rows_here;
-            uint4 v[kXCols / 8];  // the whole 256-byte share in one round trip
-#pragma unroll
-            for (int j = 0; j < kXCols / 8; ++j) v[j] = live ? src[j] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int h = 0; h < kXCols / 32; ++h) {
-                uint32_t wv[16];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    wv[4 * j] = v[4 * h + j].x; wv[4 * j + 1] = v[4 * h + j].y;
-                    wv[4 * j + 2] = v[4 * h + j].z; wv[4 * j + 3] = v[4 * h + j].w;
-                }
-                tmem_st16(t_q + lane_off + (kXCols / 2) * xpart + 16 * h, wv);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(q_full);
-        };
         // the first two tiles' P buffers expect the peer's rows
         if (xw == 0 && lane == 0) {
             mbar_arrive_expect_tx(&p_full[0], SM::kPRemote);
             mbar_arrive_expect_tx(&p_full[1], SM::kPRemote);
         }
-        bool q_loaded = false;  // q~ of the coming piece already in TMEM
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
@@ -436,23 +406,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             const uint32_t t0 = t;
             const int nt = pe - pb;
-            if (!q_loaded) copy_q(b);
-            q_loaded = false;
-            {
-                // the next piece's q~ share heads for L2 now; its copy into TMEM at the end of
-                // this piece then waits for L2, not for HBM
-                PieceIter nx = it;
-                int b2, L2, pb2, pe2;
-                bool tl2 = false, more;
-                do {
-                    more = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
-                } while (more && tl2);
-                if (more && row < rows_here) {
-                    const uint4 *nq = q_row(b2);
-                    prefetch_l2(nq);
-                    prefetch_l2(nq + 8);
-                }
-            }
             auto stage_a = [&](int i) {
                 const uint32_t tt = t0 + i;
                 const int sb = tt & 1;
@@ -558,7 +511,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 page_prev = page_j;
             }
             t = t0 + nt;
-            // the next piece's q~ goes into TMEM now, so that its scores overlap this epilogue
+            // is another piece coming (its tiles then occupy the ring)?
             bool more_pieces;
             {
                 PieceIter nx = it;
@@ -567,10 +520,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 do {
                     more_pieces = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
                 } while (more_pieces && tl2);
-                if (more_pieces) {
-                    copy_q(b2);
-                    q_loaded = true;
-                }
             }
             // ---- epilogue: O / l for this warp's 32 rows x 128 columns through TMA stores of
             // 32 x 32 fp32 boxes (128-byte swizzle) staged in shared memory.  After the last
@@ -633,6 +582,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int bgrow = rb * kRows + brow;
         const int s_of_brow = bgrow < p.rows_total ? bgrow / p.heads : p.s_q - 1;
         const bool blive = brow < rows_here;
+        // the q~ copies into TMEM: like the score warps, two warps per lane quadrant, warp
+        // half `xpart` taking q~ columns [128 xpart, 128 xpart + 128) of the CTA's half
+        const int quad = warp & 3, xpart = yw >> 2;
+        const int row = 32 * quad + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
+        const int grow = rb * kRows + row;
+
         float *alph = reinterpret_cast<float *>(smem + SM::oAlpha);
         float *lsm = reinterpret_cast<float *>(smem + SM::oL);
         const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
@@ -641,12 +597,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t alpha_remote = map_peer(smem_u32(alph), peer);
         const uint32_t l_remote = map_peer(smem_u32(lsm), peer);
         const uint32_t lfull_remote = map_peer(smem_u32(l_full), peer);
+        // this warp's share of q~'s latent half (32 rows x 128 columns) into TMEM; the
+        // previous piece's scores, its last readers, are complete (every tile's partials
+        // are in, so every score MMA is done)
+        auto q_row = [&](int bq) {
+            return reinterpret_cast<const uint4 *>(p.qa + ((int64_t)bq * p.rows_total + grow) * kRow +
+                                                   256 * rank + kXCols * xpart);
+        };
+        auto copy_q = [&](int bq) {
+            const uint4 *src = q_row(bq);
+            const bool live = row < rows_here;
+            uint4 v[kXCols / 8];  // the whole 256-byte share in one round trip
+#pragma unroll
+            for (int j = 0; j < kXCols / 8; ++j) v[j] = live ? src[j] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int h = 0; h < kXCols / 32; ++h) {
+                uint32_t wv[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    wv[4 * j] = v[4 * h + j].x; wv[4 * j + 1] = v[4 * h + j].y;
+                    wv[4 * j + 2] = v[4 * h + j].z; wv[4 * j + 3] = v[4 * h + j].w;
+                }
+                tmem_st16(t_q + lane_off + (kXCols / 2) * xpart + 16 * h, wv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_full);
+        };
+        bool q_loaded = false;  // q~ of the coming piece already in TMEM
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
         uint32_t t = 0;
         while (next_piece(p, it, b, L, pb, pe, too_long)) {
             if (too_long) continue;
+            if (!q_loaded) copy_q(b);
+            q_loaded = false;
+            // the next piece's q~ share heads for L2 now; its copy into TMEM at the end of this
+            // piece then waits for L2, not for HBM
+            PieceIter nx = it;
+            int b2, L2, pb2, pe2;
+            bool tl2 = false, more;
+            do {
+                more = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
+            } while (more && tl2);
+            if (more && row < rows_here) {
+                const uint4 *nq = q_row(b2);
+                prefetch_l2(nq);
+                prefetch_l2(nq + 8);
+            }
             float m_run = -INFINITY, l_run = 0.0f;  // the owned row (4 lanes' tokens)
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             const int last_visible = L - p.s_q + s_of_brow;  // this row's query sees t <= this
@@ -766,6 +766,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(l_full);
+            // the next piece's q~ into TMEM, while the score warps write this piece's O
+            if (more) {
+                copy_q(b2);
+                q_loaded = true;
+            }
         }
     }
     GQLA_PROF_FLUSH;
