@@ -10,34 +10,40 @@
 // is split over a 2-CTA cluster by latent column: CTA r owns the columns
 // [256r, 256r + 256) of the latent and [32r, 32r + 32) of the RoPE key.  Each
 // CTA streams only its 288 columns of every cache row (the pair reads each
-// byte of the cache exactly once), computes a partial score tile over them,
-// and the two partials are exchanged through distributed shared memory in
-// fp16; both CTAs add the same two rounded partials, so their P and softmax
-// statistics are bit-identical, and each accumulates its own 256 columns of O.
+// byte of the cache exactly once) and computes a partial score tile over
+// them.  The softmax rows are split too: row i of the block belongs to rank
+// (i / 16) % 2.  Each CTA sends the peer the fp16 partials of the peer's rows,
+// adds the two partials of its own 64 rows, computes their P (bf16) and sends
+// those P rows, with each row's O rescale factor, back; both CTAs then hold P
+// for all 128 rows and each accumulates its own 256 columns of O.
 //
-//  * Tile = one 64-token page.  An MMA instruction costs at least ~45 cycles
-//    whatever its N, so the score tile is made 64 tokens wide.  Tensor memory
-//    holds O (256 columns), a double-buffered S (2 x 64) and the latent half
-//    of q~ (128 columns of bf16 pairs), so the score MMA reads q~ from TMEM;
-//    P goes through shared memory, beside a 4-slot ring of cache tiles.
-//    Roles, 19 warps:
-//      warp 0      TMA producer: the RoPE columns of q~ (once per piece) and
-//                  the ring (4 latent boxes 128B-swizzled + 1 RoPE box
-//                  64B-swizzled, 36 KB per 64-token tile);
-//      warp 1      TMEM owner, issues S = q~ C^T (latent part with A in TMEM);
-//      warps 2-17  online softmax, four warps per TMEM lane quadrant, each
-//                  taking 16 of the tile's 64 tokens: the fp16 partial
-//                  scores go straight from registers into the peer CTA's
-//                  receive buffer with st.async (completing on the peer's
-//                  mbarrier), row maxima (lazy rescaling of O rows when a
-//                  maximum rises by more than 2^8), P written to shared
-//                  memory (bf16, 128B-swizzled, the PV MMA's A operand).  Tile
-//                  i + 1's partial is sent before tile i is finished when its
-//                  scores are already available;
+//  * Tile = one 64-token page (an MMA instruction costs about the same at any
+//    N up to 64).  Tensor memory holds O (256 columns), a double-buffered S
+//    (2 x 64) and the latent half of q~ (128 columns of bf16 pairs: the score
+//    MMA reads q~ from TMEM); P goes through shared memory, beside a 4-slot
+//    ring of cache tiles.
+//  * Roles, 19 warps:
+//      warp 0      TMA producer: the RoPE columns of q~ (once per piece) and the
+//                  ring (4 latent boxes 128B-swizzled + 1 RoPE box 64B-swizzled,
+//                  36 KB per tile), cache tiles read with an L2 evict-first policy;
+//      warp 1      TMEM owner, issues S = q~ C^T;
+//      warps 2-9   score warps, two per TMEM lane quadrant, 32 tokens each.  Stage A
+//                  of tile j: scores -> fp16; the block of the CTA's own rows goes
+//                  into its receive buffer, the block of the peer's rows leaves as
+//                  one 1 KB bulk copy.  Stage C of tile j - 1: once P of all rows is
+//                  in, O rows whose maximum rose are rescaled and PV is released.
+//                  Also the epilogue;
+//      warps 10-17 softmax warps of the CTA's 64 rows (stage B), four lanes per
+//                  row: partials added, row maxima (lazy rescaling: a maximum has
+//                  to rise by more than 2^8), P = 2^(s - m) written to both CTAs'
+//                  P buffers (bulk copy of each warp's 8 rows); also the q~ copies
+//                  into TMEM, each piece's next q~ prefetched into L2;
 //      warp 18     issues O += P C in tile order.
-//  * The softmax warps copy each piece's latent half of q~ from global memory
-//    into TMEM as soon as the previous piece's scores are done, and write
-//    O / l with TMA stores staged in the (then idle) P buffers.
+//    The stages of consecutive tiles overlap: the score warps run A(j) while the
+//    softmax warps run B(j - 1).
+//  * The epilogue writes O / l with TMA stores of 32 x 32 fp32 boxes staged in
+//    shared memory: in the idle ring after the last piece, in the P buffers
+//    between pieces.
 //  * Every wait is bounded and reports GQLA_ERR_TIMEOUT instead of hanging;
 //    both CTAs of a cluster always execute the same sequence of steps.
 #include <cudaTypedefs.h>
