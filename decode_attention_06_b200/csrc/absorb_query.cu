@@ -1,5 +1,5 @@
 // absorb_query.cu -- query absorption for the MQA-absorb path on the tcgen05
-// tensor cores ("folds W_UK into Q": GQLA, paperlayer.ai summary, sec. 2;
+// tensor cores: W_UK folded into the query (GQLA, paperlayer.ai summary, sec. 2;
 // pwwt.cn article, sec. 3).
 //
 //   qa[r][0:512]   = W_UK_{g(r)} q_r^C      (q^C = the first 128 query dims)

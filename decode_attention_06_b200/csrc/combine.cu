@@ -1,6 +1,6 @@
 // combine.cu -- log-sum-exp merge of the split-KV partials, and for the
 // MQA-absorb path the per-group up-projection out = o~ W_UV_g applied after
-// the merge ("folds W_UV into O": GQLA, paperlayer.ai summary, sec. 2).
+// the merge: W_UV folded into the output (GQLA, paperlayer.ai summary, sec. 2).
 //
 // Each partial o_i is normalised by its own softmax sum and carries
 // lse_i = ln sum_t exp(s_t) over its tokens, so

@@ -103,7 +103,7 @@ int gqla_expand_cache(const gqla_dims *dims, const void *latent, int64_t num_slo
                       gqla_stream_t stream);
 
 /*
- * Query absorption ("folds W_UK into Q": paperlayer.ai sec. 2).
+ * Query absorption: W_UK folded into the query (paperlayer.ai summary, sec. 2).
  *   q           bf16 [batch][s_q][h][192]  (0..127 q^C, 128..191 q^R, RoPE applied)
  *   w_uk        bf16 [g][512][128]
  *   q_absorbed  bf16 [batch][s_q][h][576]  out: [W_UK_{g(h)} q^C ; q^R], fp32 accumulation
