@@ -678,16 +678,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int h = 0; h < 2; ++h)
                         u[src2][h] = *reinterpret_cast<const uint4 *>(blkp + (((2 * (bq4 & 1) + h) ^ ((br >> 1) & 3)) << 4));
                 }
-                // full scores = own partial + peer partial, added in fp16 (both rounded the same way)
-                __half2 x[8];
+                // full scores = the two fp16 partials added in fp32 (one fp16 rounding per
+                // partial; an fp16 sum would add a third)
+                float x[16];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t a4[4] = {u[0][h].x, u[0][h].y, u[0][h].z, u[0][h].w};
                     const uint32_t b4[4] = {u[1][h].x, u[1][h].y, u[1][h].z, u[1][h].w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        x[4 * h + e] = __hadd2(*reinterpret_cast<const __half2 *>(&a4[e]),
-                                               *reinterpret_cast<const __half2 *>(&b4[e]));
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 fa = __half22float2(*reinterpret_cast<const __half2 *>(&a4[e]));
+                        const float2 fb = __half22float2(*reinterpret_cast<const __half2 *>(&b4[e]));
+                        x[8 * h + 2 * e] = fa.x + fb.x;
+                        x[8 * h + 2 * e + 1] = fa.y + fb.y;
+                    }
                 }
                 __syncwarp();
                 // both CTAs' buffers sb may be refilled once every softmax warp has read them
@@ -697,17 +701,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 // mask tokens past the sequence or past this query's causal limit
                 const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + 16 * bq4);
-                if (lim < 15) {
-                    const __half ninf = __ushort_as_half((unsigned short)0xFC00u);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        if (2 * e > lim) x[e].x = ninf;
-                        if (2 * e + 1 > lim) x[e].y = ninf;
-                    }
-                }
-                __half2 hm = __hmax2(__hmax2(__hmax2(x[0], x[1]), __hmax2(x[2], x[3])),
-                                     __hmax2(__hmax2(x[4], x[5]), __hmax2(x[6], x[7])));
-                float mx = fmaxf(__low2float(hm), __high2float(hm));
+                for (int e = 0; e < 16; ++e)
+                    if (e > lim) x[e] = -INFINITY;
+                float mx = x[0];
+#pragma unroll
+                for (int e = 1; e < 16; ++e) mx = fmaxf(mx, x[e]);
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
                 const float mt = mx * p.scale_log2;  // log2 units
@@ -724,9 +723,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 float lsum = 0.0f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float2 xf = __half22float2(x[e]);
-                    const uint32_t p0 = __float_as_uint(fast_exp2(fmaf(xf.x, p.scale_log2, -mu)));
-                    const uint32_t p1 = __float_as_uint(fast_exp2(fmaf(xf.y, p.scale_log2, -mu)));
+                    const uint32_t p0 = __float_as_uint(fast_exp2(fmaf(x[2 * e], p.scale_log2, -mu)));
+                    const uint32_t p1 = __float_as_uint(fast_exp2(fmaf(x[2 * e + 1], p.scale_log2, -mu)));
                     pw[e] = __byte_perm(p0, p1, 0x7632);
                     lsum += __uint_as_float(p0 & 0xFFFF0000u) + __uint_as_float(p1 & 0xFFFF0000u);
                 }

@@ -98,3 +98,25 @@ def sub_case(case, batch_ids):
         "num_pages": len(pages), "num_groups": case["num_groups"],
         "num_heads": case["num_heads"], "s_q": case["s_q"],
     }
+
+
+def rising_scores_case(s_q, factor=5.0, seqlens=(256, 200)):
+    """A paged batch whose RoPE keys grow with the logical page (by `factor` per page),
+    so that row maxima rise from page to page and the kernels' lazy rescaling of O
+    (threshold 2^8) runs on every page.  V is the latent part, so it keeps its scale.
+    The sequences are short on purpose: a few rescales per row keep the raw scores
+    within the range where the absorb path's fp16 partial scores hold 1e-2 accuracy
+    (see the absorb kernel's note on score precision)."""
+    case = _synth().make_case(128, 8, list(seqlens), s_q, paged=True, seed=131)
+    lat = case["latent"].float()
+    for b, L in enumerate(case["seqlens"].tolist()):
+        for i in range((L + 63) // 64):
+            pg = int(case["page_table"][b, i])
+            lat[pg, :, 512:] *= 1.0 + factor * i
+    case["latent"] = lat.to(torch.bfloat16)
+    return case
+
+
+def _synth():
+    from decode_attention_06_b200 import synth
+    return synth

@@ -13,7 +13,8 @@ import torch
 
 import oracle
 from decode_attention_06_b200 import synth
-from tests.helpers import compare, compare_lse, oracle_ref, run_decode, sub_case, to_gpu
+from tests.helpers import (compare, compare_lse, oracle_ref, rising_scores_case, run_decode,
+                           sub_case, to_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -96,6 +97,18 @@ def test_paths_agree():
     a, la, _, _ = run_decode(g, "absorb", 6)
     b, lb, _, _ = run_decode(g, "gqa", 6)
     compare(a, b.float().cpu().numpy().astype(np.float64), what="absorb vs gqa")
+
+
+@pytest.mark.parametrize("path", ["gqa", "absorb"])
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_decode_parity_rising_scores(path, s_q):
+    case = rising_scores_case(s_q)
+    out, lse, ws, _ = run_decode(to_gpu(case), path, 3)
+    ref, ref_lse = oracle_ref(case)
+    compare(out, ref, what=f"{path}/rising_sq{s_q}")
+    compare_lse(lse, ref_lse, what=f"{path}/rising_sq{s_q}")
+    from decode_attention_06_b200 import gqla
+    assert gqla.gqla_read_device_error(ws)[0] == 0
 
 
 def test_bad_page_index_is_reported_not_faulted():

@@ -368,3 +368,20 @@ def test_expand_f32seq_close_to_exact_and_rounded_once():
 ])
 def test_bf16_round_nearest_even(x, bits):
     assert oracle.bf16_rne_bits(x) == bits
+
+
+def test_rising_scores_case_rescales():
+    from tests.helpers import rising_scores_case
+    # the construction does what the test below relies on: row maxima of the scaled
+    # scores rise by more than 2^8 (8 log2 units) between most consecutive pages
+    case = rising_scores_case(1)
+    qa = oracle.absorb_query(case["q"], case["w_uk"], 8)            # [B][1][h][576]
+    lat = case["latent"].float().numpy().astype(np.float64)
+    rises = []
+    for b, L in enumerate(case["seqlens"].tolist()):
+        rows = np.concatenate([lat[int(case["page_table"][b, i])] for i in range((L + 63) // 64)])[:L]
+        s = qa[b, 0] @ rows.T / math.sqrt(192.0) * math.log2(math.e)   # [h][L], log2 units
+        pm = np.stack([s[:, j:j + 64].max(axis=1) for j in range(0, L, 64)], axis=1)
+        rises.append(np.diff(pm, axis=1).ravel())
+    rises = np.concatenate(rises)
+    assert (rises > 8.0).mean() > 0.4
