@@ -128,6 +128,10 @@ int gqla_absorb_query(const gqla_dims *dims, const void *q, int batch, int s_q,
  *                 scaled scores (-inf for an empty partial); unused slots are not written
  *   workspace  >= gqla_workspace_bytes() bytes of device memory, zeroed once
  *              before first use (holds the device error record)
+ * Precision: the two halves of each score (288 latent and RoPE columns each,
+ * one per CTA of a pair) are exchanged as fp16 and added in fp32, so very
+ * large raw scores (halves beyond a few hundred) lose accuracy; the GQA path
+ * forms scores in fp32.
  */
 int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
                        const void *latent_cache, const gqla_kv_index *kv, int num_splits,
