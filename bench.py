@@ -427,13 +427,8 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("end-to-end outputs differ from the device results")
 
     # ---- max over ranks
-    t = torch.tensor([ms_step, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_step, e2e_ms = float(t[0]), float(t[1])
     tokens_step = B * s_q
-    value = world * tokens_step / (ms_step * 1e-3)
-    e2e_value = world * tokens_step / (e2e_ms * 1e-3)
+    ms_step, e2e_ms, value, e2e_value = aggregate_over_ranks(ms_step, e2e_ms, world, tokens_step, dev)
 
     acc, counts = accounting(w, case, s_q, splits["gqa"])
     acc_a, _ = accounting(w, case, s_q, splits["absorb"])
@@ -571,6 +566,18 @@ def ncu_summary(csv_path):
     print(f"{'launches':>8} {'total us':>11} {'share':>7}  kernel")
     for k, (n, t) in sorted(agg.items(), key=lambda x: -x[1][1]):
         print(f"{n:8d} {t:11.1f} {100 * t / total:6.1f}%  {k}")
+
+
+def aggregate_over_ranks(ms_step, e2e_ms, world, tokens_per_rank, device):
+    """Replicas: every rank decodes its own batch.  The job's step time is the
+    slowest rank's (max over ranks); its throughput counts every rank's tokens."""
+    t = torch.tensor([ms_step, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_step, e2e_ms = float(t[0]), float(t[1])
+    value = world * tokens_per_rank / (ms_step * 1e-3)
+    e2e_value = world * tokens_per_rank / (e2e_ms * 1e-3)
+    return ms_step, e2e_ms, value, e2e_value
 
 
 def main():
