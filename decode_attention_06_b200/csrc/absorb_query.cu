@@ -84,6 +84,22 @@ __global__ void __launch_bounds__(kAqThreads, 2)
             tma_load_2d(sB + kb * kAqB, &wmap, full, kb * 64, grp * kLatent + quarter * kAqN);
         }
     }
+    // RoPE part of the query (quarter 0 only): loaded now, while the tiles are in
+    // flight, and stored with the epilogue; 8 lanes per row, rows_in_tile * 8 <= 8 * kAqThreads
+    constexpr int kRopeIt = 128 * 8 / kAqThreads;
+    uint4 rope[kRopeIt];
+    if (quarter == 0) {
+#pragma unroll
+        for (int j = 0; j < kRopeIt; ++j) {
+            const int i = threadIdx.x + j * kAqThreads, r = i >> 3, part = i & 7;
+            const int bs = bs0 + r / p.G;
+            rope[j] = make_uint4(0, 0, 0, 0);
+            if (r < rows_in_tile && bs < p.bs_total) {
+                const int64_t row = (int64_t)bs * p.heads + grp * p.G + r % p.G;
+                rope[j] = reinterpret_cast<const uint4 *>(p.q + row * kQk + kNope)[part];
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -93,13 +109,13 @@ __global__ void __launch_bounds__(kAqThreads, 2)
         if (mbar_wait(full, 0, abort_flag)) {
             tc_fence_after();
             constexpr uint32_t idesc = idesc_bf16(128, kAqN, 0, 0);
-            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+            const uint64_t a_d = smem_desc(smem_u32(sA), 16, 1024, kSw128);
+            const uint64_t b_d = smem_desc(smem_u32(sB), 16, 1024, kSw128);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = (kk & 3) * 32;  // 16 dims = 32 bytes inside the swizzled row
-                const uint64_t ad = smem_desc(a0 + (kk >> 2) * kAqA + off, 16, 1024, kSw128);
-                const uint64_t bd = smem_desc(b0 + (kk >> 2) * kAqB + off, 16, 1024, kSw128);
-                mma_bf16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                mma_bf16(tmem, desc_advance(a_d, (kk >> 2) * kAqA + off), desc_advance(b_d, (kk >> 2) * kAqB + off),
+                         idesc, kk > 0 ? 1u : 0u);
             }
             mma_commit(done);
         } else {
@@ -145,14 +161,15 @@ __global__ void __launch_bounds__(kAqThreads, 2)
                     *reinterpret_cast<const uint4 *>(stage + r * kAqStage + (lane & 15) * 16);
             }
         }
-        if (quarter == 0) {  // RoPE part: q[row][128:192] -> qa[row][512:576], 8 lanes per row
-            for (int i = threadIdx.x; i < rows_in_tile * 8; i += kAqThreads) {
-                const int r = i >> 3, part = i & 7;
+        if (quarter == 0) {  // RoPE part: q[row][128:192] -> qa[row][512:576]
+#pragma unroll
+            for (int j = 0; j < kRopeIt; ++j) {
+                const int i = threadIdx.x + j * kAqThreads, r = i >> 3, part = i & 7;
                 const int bs = bs0 + r / p.G;
-                if (bs >= p.bs_total) break;
-                const int64_t row = (int64_t)bs * p.heads + grp * p.G + r % p.G;
-                reinterpret_cast<uint4 *>(p.qa + row * kRow + kLatent)[part] =
-                    reinterpret_cast<const uint4 *>(p.q + row * kQk + kNope)[part];
+                if (r < rows_in_tile && bs < p.bs_total) {
+                    const int64_t row = (int64_t)bs * p.heads + grp * p.G + r % p.G;
+                    reinterpret_cast<uint4 *>(p.qa + row * kRow + kLatent)[part] = rope[j];
+                }
             }
         }
     }
