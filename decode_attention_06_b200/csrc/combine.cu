@@ -405,21 +405,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     // ---- leader: the other half of A and W_UV_g in place -> 32 MMAs (M = 64, K = 512)
     const uint32_t tmem = *tmem_slot;
     if (tid == 0) {
+        // this CTA's half of K first (its A blocks are in place), the peer's half once it lands
         mbar_arrive_expect_tx(a_full, ClSmem::kAHalf);
-        const bool ok = mbar_wait_cluster(a_full, 0, abort_flag) && mbar_wait(b_full, 0, abort_flag);
+        constexpr uint32_t idesc = idesc_bf16(kClRows, 128, 0, 1);
+        const uint64_t a_d = smem_desc(smem_u32(smem + ClSmem::oA), 16, 1024, kSw128);
+        const uint64_t b_d = smem_desc(smem_u32(smem + ClSmem::oB), 65536, 1024, kSw128);
+        bool ok = mbar_wait(b_full, 0, abort_flag);
         if (ok) {
             tc_fence_after();
-            constexpr uint32_t idesc = idesc_bf16(kClRows, 128, 0, 1);
-            const uint64_t a_d = smem_desc(smem_u32(smem + ClSmem::oA), 16, 1024, kSw128);
-            const uint64_t b_d = smem_desc(smem_u32(smem + ClSmem::oB), 65536, 1024, kSw128);
 #pragma unroll
-            for (int kk = 0; kk < kLatent / 16; ++kk)
+            for (int kk = 0; kk < kLatent / 32; ++kk)
                 mma_bf16(tmem, desc_advance(a_d, (kk >> 2) * (kClRows * 128) + (kk & 3) * 32),
                          desc_advance(b_d, kk * 2048), idesc, kk > 0 ? 1u : 0u);
-            mma_commit(done);
+            ok = mbar_wait_cluster(a_full, 0, abort_flag);
+        }
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = kLatent / 32; kk < kLatent / 16; ++kk)
+                mma_bf16(tmem, desc_advance(a_d, (kk >> 2) * (kClRows * 128) + (kk & 3) * 32),
+                         desc_advance(b_d, kk * 2048), idesc, 1u);
         } else {
             *abort_flag = 1;
         }
+        mma_commit(done);
     }
     const bool ok = mbar_wait(done, 0, abort_flag);
     tc_fence_after();
