@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (too_long) report_error(p.ws, GQLA_ERR_DEVICE, b);
             }
             const uint32_t q_bytes = 3u * 128u * (uint32_t)real_cols;
+            const uint64_t stream_policy = l2_evict_first_policy();  // the cache is read once
             UnitCursor kc, vc;
             kc.start(p, it0);
             vc.start(p, it0);
@@ -367,9 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             uint8_t *dst = smem + SM::oKr + kb * SM::kKrBytes;
                             if (np) {
                                 mbar_arrive_expect_tx(&kr_full[kb], np * kBox);
-                                if (pp.page0 >= 0) tma_load_2d(dst, &kr_map, &kr_full[kb], 0, pp.page0 * kPage);
+                                if (pp.page0 >= 0)
+                                    tma_load_2d_hint(dst, &kr_map, &kr_full[kb], 0, pp.page0 * kPage, stream_policy);
                                 if (pp.page1 >= 0)
-                                    tma_load_2d(dst + kBox, &kr_map, &kr_full[kb], 0, pp.page1 * kPage);
+                                    tma_load_2d_hint(dst + kBox, &kr_map, &kr_full[kb], 0, pp.page1 * kPage,
+                                                     stream_policy);
                             } else {
                                 mbar_arrive(&kr_full[kb]);
                             }
@@ -384,11 +387,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int cb = 0; cb < 2; ++cb) {  // K_nope lo / hi: page 0 rows, then page 1 rows
                             if (pp.page0 >= 0)
-                                tma_load_3d(dst + cb * 2 * kBox, &kv_map, &k_full[ks], cb * 64,
-                                            pp.page0 * kPage, kc.gi);
+                                tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &k_full[ks], cb * 64,
+                                                 pp.page0 * kPage, kc.gi, stream_policy);
                             if (pp.page1 >= 0)
-                                tma_load_3d(dst + cb * 2 * kBox + kBox, &kv_map, &k_full[ks], cb * 64,
-                                            pp.page1 * kPage, kc.gi);
+                                tma_load_3d_hint(dst + cb * 2 * kBox + kBox, &kv_map, &k_full[ks], cb * 64,
+                                                 pp.page1 * kPage, kc.gi, stream_policy);
                         }
                         kc.advance(p);
                         ++kpos;
@@ -406,11 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int cb = 0; cb < 2; ++cb) {
                                 if (pp.page0 >= 0)
-                                    tma_load_3d(dst + cb * 2 * kBox, &kv_map, &v_full[vs], 128 + cb * 64,
-                                                pp.page0 * kPage, vc.gi);
+                                    tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &v_full[vs], 128 + cb * 64,
+                                                     pp.page0 * kPage, vc.gi, stream_policy);
                                 if (pp.page1 >= 0)
-                                    tma_load_3d(dst + cb * 2 * kBox + kBox, &kv_map, &v_full[vs],
-                                                128 + cb * 64, pp.page1 * kPage, vc.gi);
+                                    tma_load_3d_hint(dst + cb * 2 * kBox + kBox, &kv_map, &v_full[vs],
+                                                     128 + cb * 64, pp.page1 * kPage, vc.gi, stream_policy);
                             }
                         } else {
                             mbar_arrive(&v_full[vs]);
