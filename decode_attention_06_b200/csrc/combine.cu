@@ -115,6 +115,16 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
     const int64_t row0 = ((int64_t)(b + c0) * p.s_q + s) * p.heads + h0;
     const int64_t part_stride = (int64_t)p.s_q * p.heads;
 
+    // the first eight partials do not depend on the weights: their loads go out with
+    // the LSE loads, so the common case (nparts <= 8) makes one round trip to memory
+    const float *base0 = p.o_part + row0 * kDv + lane * 4;
+    float4 v0[8][4];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            v0[jj][i] = jj < nparts ? ldg4(base0 + ((int64_t)jj * part_stride + i) * kDv)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
     // LSE of partial c = lane (the first 32), kept for the weights of the first block
     float l0[4], M[4];
 #pragma unroll
@@ -146,16 +156,30 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
         }
         const int n = min(32, nparts - cb);
         const float *base = p.o_part + (row0 + (int64_t)cb * part_stride) * kDv + lane * 4;
-        for (int j0 = 0; j0 < n; j0 += 8) {
-            float4 v[8][4];
+        int j0 = 0;
+        if (cb == 0) {  // the eight partials already in registers (zeros past nparts)
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float wj = __shfl_sync(0xffffffffu, w[i], jj);
+                    acc[i].x = fmaf(wj, v0[jj][i].x, acc[i].x);
+                    acc[i].y = fmaf(wj, v0[jj][i].y, acc[i].y);
+                    acc[i].z = fmaf(wj, v0[jj][i].z, acc[i].z);
+                    acc[i].w = fmaf(wj, v0[jj][i].w, acc[i].w);
+                }
+            j0 = 8;
+        }
+        for (; j0 < n; j0 += 4) {
+            float4 v[4][4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     v[jj][i] = j0 + jj < n ? ldg4(base + ((int64_t)(j0 + jj) * part_stride + i) * kDv)
                                            : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
+            for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float wj = __shfl_sync(0xffffffffu, w[i], (j0 + jj) & 31);
