@@ -167,13 +167,14 @@ def accounting(w, case, s_q, num_splits):
             pieces += (start + n - 1) // k - start // k + 1
         start += n
     rows = B * s_q * h
+    gqa_tok = (2 * g * 128 + 64) * 2  # expanded bytes per token: 4224 at g = 8, 2176 at g = 4
     acc = {
         "decode_absorb": {
             "bytes": tokens * 1152 + rows * 576 * 2 + pieces * s_q * h * (512 + 1) * 4,
             "flops": 2.0 * h * pairs * (576 + 512),
         },
         "decode_gqa": {
-            "bytes": tokens * 4224 + rows * 192 * 2 + pieces * s_q * h * (128 + 1) * 4,
+            "bytes": tokens * gqa_tok + rows * 192 * 2 + pieces * s_q * h * (128 + 1) * 4,
             "flops": 2.0 * h * pairs * (192 + 128),
         },
         "absorb_query": {"bytes": rows * (192 + 576) * 2 + g * 512 * 128 * 2,
@@ -181,7 +182,7 @@ def accounting(w, case, s_q, num_splits):
         "combine_absorb": {"bytes": pieces * s_q * h * 513 * 4 + rows * 128 * 2 + g * 512 * 128 * 2,
                            "flops": 2.0 * rows * 512 * 128},
         "combine_gqa": {"bytes": pieces * s_q * h * 129 * 4 + rows * 128 * 2, "flops": 0.0},
-        "expand": {"bytes": case["num_pages"] * 64 * (1152 + 4224) + 2 * g * 512 * 128 * 2,
+        "expand": {"bytes": case["num_pages"] * 64 * (1152 + gqa_tok) + 2 * g * 512 * 128 * 2,
                    "flops": 2.0 * case["num_pages"] * 64 * 512 * 256 * g},
     }
     return acc, {"tokens": tokens, "pairs": pairs, "pieces": pieces}

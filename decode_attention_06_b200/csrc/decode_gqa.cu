@@ -16,14 +16,14 @@
 //      S^T[128 tok][NQ]    = [K_nope_g | k^R] (128 x 192, K-major) x q_g^T
 //      O^T_g[128 dv][NQ]  += V_g^T (MN-major) x P^T (MN-major, bf16)
 //    With M = 128 every TMEM lane, and so every softmax thread, owns one
-//    token.  O^T of all 8 groups stays resident in TMEM for a whole piece.
+//    token.  O^T of all g (8 or 4) groups stays resident in TMEM for a whole piece.
 //  * One CTA per chunk of the split plan (grid = SM count), 320 threads:
 //      warp 0      TMA producer over three rings: q_g + K_nope_g (freed as
 //                  soon as S^T is done), V_g (freed after O^T += ...), and
 //                  per page pair the shared RoPE keys; each ring refills as
 //                  soon as a slot frees, so loads run well ahead;
 //      warp 1      TMEM owner; one thread issues the score MMAs;
-//      warps 2-9   two softmax warpgroups (groups 0,2,4,6 and 1,3,5,7): each
+//      warps 2-9   two softmax warpgroups (the even and the odd groups): each
 //                  runs its online softmax, issues its own PV MMAs (one
 //                  elected thread) and writes its epilogue.
 //  * Online softmax in the base-2 domain with lazy rescaling: P is formed
@@ -84,6 +84,7 @@ struct GqaParams {
     float *lse_part;
     void *ws;
     int batch, max_pages, num_pages, num_splits, s_q, heads, G;
+    int NG;  // KV groups g: 8, or 4 (the (g, s_q) = (4, 1) configuration's 2176-byte tokens)
     float scale_log2;
 };
 
@@ -138,7 +139,7 @@ __device__ __forceinline__ PagePair load_pair(const GqaParams &p, int b, int L, 
 struct UnitCursor {
     PieceIter it;
     int b, L, pg, pe, gi;
-    int n0, n1;  // page indices of the pair after this one (valid from gi == 4)
+    int n0, n1;  // page indices of the pair after this one (valid from gi == NG / 2)
     PagePair pp;
     bool valid;
     __device__ __forceinline__ bool next_valid_piece(const GqaParams &p) {
@@ -159,12 +160,12 @@ struct UnitCursor {
     }
     __device__ __forceinline__ void advance(const GqaParams &p) {
         ++gi;
-        if (gi == 4 && pg + 2 < pe) {
+        if (gi == p.NG / 2 && pg + 2 < pe) {
             const int32_t *row = p.page_table + (int64_t)b * p.max_pages;
             n0 = row[pg + 2];
             n1 = pg + 3 < pe ? row[pg + 3] : 0;
         }
-        if (gi < 8) return;
+        if (gi < p.NG) return;
         gi = 0;
         pg += 2;
         if (pg < pe) { pp = make_pair(p, L, pg, pe, n0, n1); return; }
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int kb = pc & 1;
                     if (!GQLA_WAIT(2, &kr_full[kb], (pc >> 1) & 1, abort_flag)) *abort_flag = 1;
                     const uint32_t kr = sm_kr + kb * SM::kKrBytes;
-                    for (int gi = 0; gi < 8; ++gi, ++u) {
+                    for (int gi = 0; gi < p.NG; ++gi, ++u) {
                         // S^T(u) = [K_nope_g | k^R] q_g^T into S buffer u & 3
                         const int ks_ = u % KS, sb = u & 3;
                         if (!GQLA_WAIT(3, &k_full[ks_], (u / KS) & 1, abort_flag)) *abort_flag = 1;
@@ -477,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         mma_commit(&s_full[sb]);
                         mma_commit(&k_empty[ks_]);
-                        if (gi == 7) mma_commit(&kr_empty[kb]);
+                        if (gi == p.NG - 1) mma_commit(&kr_empty[kb]);
                     }
                 }
             }
@@ -504,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (too_long) continue;
                 const int npairs = (pe - pb + 1) >> 1;
                 for (int ip = 0; ip < npairs; ++ip) {
-                    for (int gi = 0; gi < 8; ++gi, ++u) {
+                    for (int gi = 0; gi < p.NG; ++gi, ++u) {
                         const int w = gi & 1, vs = u % VS;
                         if (!GQLA_WAIT(5, &p_full[w], (u >> 1) & 1, abort_flag)) *abort_flag = 1;
                         if (!GQLA_WAIT(13, &v_full[vs], (u / VS) & 1, abort_flag)) *abort_flag = 1;
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- softmax, PV, epilogue
-        // Warpgroup wg owns the groups gi = wg, wg + 2, wg + 4, wg + 6 (units of
+        // Warpgroup wg owns the groups gi = wg, wg + 2, ... (units of
         // one parity), so the two warpgroups never share a group.
         const int wg = (warp - 2) >> 2;        // 0 or 1
         const int wq = (warp - 2) & 3;         // warp within the warpgroup
@@ -559,9 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // s_q <= 2 only the last token can be hidden, and only from columns n < G
                 const bool hide_low = pg * kPage + tok - (L - p.s_q) > 0;
 #pragma unroll 1
-                for (int gl = 0; gl < 4; ++gl) {
+                for (int gl = 0; gl < p.NG / 2; ++gl) {
                     const int gi = 2 * gl + wg;
-                    const uint32_t jj = j + ip * 8 + gi;
+                    const uint32_t jj = j + ip * p.NG + gi;
                     // lane n (< NQ) keeps the column-n sum over this warp's tokens in shared memory
                     float *lw = lred + (gi * NQ + (lane & (NQ - 1))) * 4 + wq;
                     const int sb = jj & 3;
@@ -681,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     GQLA_SPAN_END(10, t_unit);
                 }
             }
-            j += npairs * 8;
+            j += npairs * p.NG;
             GQLA_SPAN_BEGIN(t_epi);
             // ---- epilogue: normalise O^T and write the partials of slot b + c
             if (!GQLA_WAIT(14, &o_done[wg], k & 1, abort_flag)) *abort_flag = 1;
@@ -692,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // rows of the partial for columns n = s*G + hg: ((slot*s_q + s)*h + gi*G + hg)
             const int64_t row_s0 = (int64_t)slot * p.s_q * p.heads;
 #pragma unroll 1
-            for (int gl = 0; gl < 4; ++gl) {
+            for (int gl = 0; gl < p.NG / 2; ++gl) {
                 const int gi = 2 * gl + wg;
                 if (wtid < NQ) {  // per column: 1 / l and the natural-log LSE
                     const float4 l4 = *reinterpret_cast<const float4 *>(lred + (gi * NQ + wtid) * 4);
@@ -789,11 +790,11 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
                               const void *k_rope, int64_t num_slots, const gqla_kv_index *idx,
                               int num_splits, float scale, float *o_part, float *lse_part,
                               void *ws, cudaStream_t stream) {
-    if (num_groups != 8) return cudaErrorInvalidValue;
+    if (num_groups != 8 && num_groups != 4) return cudaErrorInvalidValue;
     const int G = heads / num_groups;
     CUtensorMap kvm, krm, qm;
     {
-        cuuint64_t dims[3] = {256, (cuuint64_t)num_slots, 8};
+        cuuint64_t dims[3] = {256, (cuuint64_t)num_slots, (cuuint64_t)num_groups};
         cuuint64_t strides[2] = {256 * 2, (cuuint64_t)num_slots * 256 * 2};
         cuuint32_t box[3] = {64, 64, 1};
         if (!make_map(&kvm, kv, 3, dims, strides, box)) return cudaErrorInvalidValue;
@@ -823,6 +824,7 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
     p.s_q = s_q;
     p.heads = heads;
     p.G = G;
+    p.NG = num_groups;
     p.scale_log2 = scale * kLog2e;
     return G * s_q <= 16 ? launch_nq<16>(kvm, krm, qm, p, stream)
                          : launch_nq<32>(kvm, krm, qm, p, stream);

@@ -181,7 +181,7 @@ int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *k
     if (!aligned16(q) || !aligned16(kv_expanded) || !aligned16(k_rope) || !aligned16(o_part))
         return GQLA_ERR_INVALID_ARG;
     if (num_slots != (int64_t)kv->num_pages * kv->page_size) return GQLA_ERR_INVALID_ARG;
-    if (dims->num_groups != 8) return GQLA_ERR_UNSUPPORTED;
+    if (dims->num_groups != 8 && dims->num_groups != 4) return GQLA_ERR_UNSUPPORTED;
     return cuda_status(launch_decode_gqa(q, s_q, dims->num_heads, dims->num_groups, kv_expanded,
                                          k_rope, num_slots, kv, num_splits, dims->softmax_scale,
                                          o_part, lse_part, workspace,

@@ -69,6 +69,9 @@ WORKLOADS = {
         # LLaMA-3-8B converted shape, large batch of mixed lengths, plus a full-cache expansion
         Workload("llama3_8b_h32_b128_l2k_8k", 32, 8, 128, ("uniform", 2048, 8192), (1, 2),
                  False, 4, expand=True),
+        # the (g, s_q) = (4, 1) conversion point: 128 heads over 4 groups, 2176 bytes per
+        # expanded token (beyond the five configurations above)
+        Workload("dsv3_h128_g4_b32_l4096", 128, 4, 32, ("fixed", 4096), (1,), False, 5),
     ]
 }
 

@@ -67,7 +67,8 @@ typedef enum {
  * 1/sqrt(192) is the expected value. */
 typedef struct {
     int num_heads;       /* h_q: e.g. 128 (DeepSeek-V3 shape) or 32 (LLaMA-3-8B) */
-    int num_groups;      /* g: 8                                                   */
+    int num_groups;      /* g: 8, or 4 (the (g, s_q) = (4, 1) point); G*s_q <= 32,
+                            G a multiple of 4                                      */
     int d_latent;        /* r_kv: 512                                              */
     int d_rope;          /* d_R: 64                                                */
     int d_nope;          /* per-head no-RoPE key width: 128                        */
@@ -145,6 +146,7 @@ int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
  *   kv_expanded  bf16 [g][num_slots][256], k_rope bf16 [num_slots][64]
  *                (as written by gqla_expand_cache; num_slots = num_pages * page_size)
  *   o_part  fp32 [gqla_partial_slots(batch, C)][s_q][h][128], lse_part as above.
+ * g must be 8 or 4 (GQLA_ERR_UNSUPPORTED otherwise).
  */
 int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
                     const void *k_rope, int64_t num_slots, const gqla_kv_index *kv,
@@ -153,8 +155,8 @@ int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *k
 
 /*
  * Log-sum-exp merge of the partials of each sequence, then (absorb path,
- * d_in == 512) the per-group up-projection out = o~ W_UV_{g(h)} ("folds W_UV
- * into O": paperlayer.ai sec. 2).
+ * d_in == 512) the per-group up-projection out = o~ W_UV_{g(h)}: W_UV folded into
+ * the output (paperlayer.ai summary, sec. 2).
  *   o_part / lse_part as written by a decode call with the same kv and num_splits
  *   d_in      512 (absorb partials; w_uv required) or 128 (GQA partials; w_uv NULL)
  *   out       bf16 [batch][s_q][h][128]

@@ -91,6 +91,25 @@ def test_decode_parity_small(path, cid, h, seqlens, s_q, paged, splits):
     assert gqla.gqla_read_device_error(ws)[0] == 0
 
 
+SMALL_G4 = [
+    # the (g, s_q) = (4, 1) conversion and its MTP / small-head neighbours: 4 KV groups
+    ("g4_h128_paged", 128, [1000, 70], 1, True, 5),
+    ("g4_h32_mtp_ragged", 32, [513, 64, 3], 2, False, 6),
+]
+
+
+@pytest.mark.parametrize("path", ["gqa", "absorb"])
+@pytest.mark.parametrize("cid,h,seqlens,s_q,paged,splits", SMALL_G4, ids=[c[0] for c in SMALL_G4])
+def test_decode_parity_four_groups(path, cid, h, seqlens, s_q, paged, splits):
+    case = synth.make_case(h, 4, seqlens, s_q, paged=paged, seed=zlib.crc32(cid.encode()) % 1000)
+    out, lse, ws, _ = run_decode(to_gpu(case), path, splits)
+    ref, ref_lse = oracle_ref(case)
+    compare(out, ref, what=f"{path}/{cid}")
+    compare_lse(lse, ref_lse, what=f"{path}/{cid}")
+    from decode_attention_06_b200 import gqla
+    assert gqla.gqla_read_device_error(ws)[0] == 0
+
+
 def test_paths_agree():
     case = synth.make_case(128, 8, [700, 129], 2, paged=True, seed=120)
     g = to_gpu(case)
