@@ -23,16 +23,17 @@
 //    MMA reads q~ from TMEM); P goes through shared memory, beside a 4-slot
 //    ring of cache tiles.
 //  * Roles, 19 warps:
-//      warp 0      TMA producer: the RoPE columns of q~ (once per piece) and the
-//                  ring (4 latent boxes 128B-swizzled + 1 RoPE box 64B-swizzled,
-//                  36 KB per tile), cache tiles read with an L2 evict-first policy;
+//      warp 0      TMA producer of the ring (4 latent boxes 128B-swizzled + 1 RoPE
+//                  box 64B-swizzled, 36 KB per tile), cache tiles read with an L2
+//                  evict-first policy;
 //      warp 1      TMEM owner, issues S = q~ C^T;
 //      warps 2-9   score warps, two per TMEM lane quadrant, 32 tokens each.  Stage A
 //                  of tile j: scores -> fp16; the block of the CTA's own rows goes
 //                  into its receive buffer, the block of the peer's rows leaves as
 //                  one 1 KB bulk copy.  Stage C of tile j - 1: once P of all rows is
 //                  in, O rows whose maximum rose are rescaled and PV is released.
-//                  Also the epilogue;
+//                  Also each piece's RoPE q~ (by TMA, as soon as the previous
+//                  piece's scores are complete) and the epilogue;
 //      warps 10-17 softmax warps of the CTA's 64 rows (stage B), four lanes per
 //                  row: partials added, row maxima (lazy rescaling: a maximum has
 //                  to rise by more than 2^8), P = 2^(s - m) written to both CTAs'
@@ -97,9 +98,9 @@ struct AbsorbSmem {
     static constexpr int oAlpha = oXStage + kXWarps * kXBlock;  // float [2 buffers][128 rows]
     static constexpr int oL = oAlpha + 2 * kRows * 4;     // float [128 rows]: row sums of a piece
     static constexpr int oBar = oL + kRows * 4;
-    // ring_full/empty[kRing], q_full, q_empty, s_full/s_free[2], x_full/x_empty[2],
+    // ring_full/empty[kRing], q_full, s_full/s_free[2], x_full/x_empty[2],
     // p_full/p_empty[2], o_ready[2], pv_done[2], l_full, o_done, drain[2]
-    static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 4 + 2 + 2 + 1 + 1 + 2;
+    static constexpr int kNumBars = 2 * kRing + 1 + 4 + 4 + 4 + 2 + 2 + 1 + 1 + 2;
     static constexpr int oMisc = oBar + kNumBars * 8;     // tmem base, abort, plan[4]
     static constexpr int kBytes = oMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;
@@ -139,6 +140,16 @@ __device__ __forceinline__ bool next_piece(const AbsorbParams &p, PieceIter &it,
     return false;
 }
 
+// Is a piece that is not skipped still to come after `it`?  (`b2` its sequence.)
+__device__ __forceinline__ bool another_piece(const AbsorbParams &p, PieceIter it, int &b2) {
+    int L2, pb2, pe2;
+    bool tl2 = false, more;
+    do {
+        more = next_piece(p, it, b2, L2, pb2, pe2, tl2);
+    } while (more && tl2);
+    return more;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_absorb_tc_kernel(const __grid_constant__ CUtensorMap lat_map,
                             const __grid_constant__ CUtensorMap rope_map,
@@ -150,8 +161,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::oBar);
     uint64_t *ring_full = bars, *ring_empty = bars + kRing;
-    uint64_t *q_full = bars + 2 * kRing, *q_empty = q_full + 1;
-    uint64_t *s_full = q_empty + 1, *s_free = s_full + 2;
+    uint64_t *q_full = bars + 2 * kRing;
+    uint64_t *s_full = q_full + 1, *s_free = s_full + 2;
     uint64_t *x_full = s_free + 2, *x_empty = x_full + 2;
     uint64_t *p_full = x_empty + 2, *p_empty = p_full + 2;
     uint64_t *o_ready = p_empty + 2, *pv_done = o_ready + 2;
@@ -172,7 +183,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i) { mbar_init(&ring_full[i], 1); mbar_init(&ring_empty[i], 1); }
         mbar_init(q_full, 1 + kYWarps);  // RoPE TMA + the softmax warps' TMEM copies
-        mbar_init(q_empty, kXWarps);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1); mbar_init(&s_free[i], kXThreads);
             mbar_init(&x_full[i], 1 + kXWarps);      // expect_tx of the peer's half + local score warps
@@ -246,21 +256,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (lane == 0 && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
                 continue;
             }
-            // RoPE columns of q~ for this row block; they wait for the previous piece's
-            // scores, so up to kRing - 1 of this piece's tiles are issued first
-            const int rope_at = min(pe - pb, kRing - 1);
-            auto load_rope = [&]() {
-                if (lane == 0) {
-                    if (!GQLA_WAIT(1, q_empty, (k & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                    if (!*abort_flag) {
-                        const int row0 = b * p.rows_total + rb * kRows;
-                        mbar_arrive_expect_tx(q_full, SM::kQRope);
-                        tma_load_2d(smem + SM::oQ, &qrope_map, q_full, 512 + 32 * rank, row0);
-                    } else {
-                        mbar_arrive(q_full);
-                    }
-                }
-            };
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             for (int i0 = pb; i0 < pe; i0 += 32) {
                 const int n = min(32, pe - i0);
@@ -269,7 +264,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 pre_ok = false;
                 for (int j = 0; j < n; ++j, ++t) {
                     const int page = __shfl_sync(0xffffffffu, my_page, j);
-                    if (i0 - pb + j == rope_at) load_rope();
                     if (lane == 0) {
                         const bool bad = page < 0 || page >= p.num_pages;
                         if (bad && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
@@ -290,7 +284,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (rope_at == pe - pb) load_rope();
             ++k;
         }
         if (lane == 0) {
@@ -299,7 +292,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
             for (uint32_t u = (t > (uint32_t)kRing ? t - kRing : 0); u < t; ++u)
                 mbar_wait(&ring_full[u % kRing], (u / kRing) & 1, no_abort);
-            if (k) mbar_wait(q_full, (k - 1) & 1, no_abort);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- score MMA issuer
@@ -403,12 +395,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&p_full[0], SM::kPRemote);
             mbar_arrive_expect_tx(&p_full[1], SM::kPRemote);
         }
+        // the RoPE columns of a piece's q~, by TMA: the first piece's at once, each next
+        // piece's as soon as this piece's last scores are complete (one thread)
+        auto load_rope = [&](int bq) {
+            if (xw == 0 && lane == 0) {
+                mbar_arrive_expect_tx(q_full, SM::kQRope);
+                tma_load_2d(smem + SM::oQ, &qrope_map, q_full, 512 + 32 * rank, bq * p.rows_total + rb * kRows);
+            }
+        };
+        bool rope_issued = false;
         PieceIter it = it0;
         int b, L, pb, pe;
         bool too_long;
         uint32_t t = 0, k = 0;
         while (next_piece(p, it, b, L, pb, pe, too_long)) {
             if (too_long) continue;
+            if (!rope_issued) load_rope(b);
+            int b_next = 0;
+            const bool more_pieces = another_piece(p, it, b_next);  // its tiles then occupy the ring
+            rope_issued = more_pieces;
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             const uint32_t t0 = t;
             const int nt = pe - pb;
@@ -506,27 +511,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 GQLA_SPAN_BEGIN(t_tile);
                 if (j < nt) {
                     stage_a(j);
-                    // the last scores of the piece are read: the producer may load the next RoPE q~
-                    if (j == nt - 1) {
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(q_empty);
-                    }
+                    // the piece's last scores are complete: the next piece's RoPE q~ may come
+                    if (j == nt - 1 && more_pieces) load_rope(b_next);
                 }
                 if (j >= 1) stage_c(j - 1, page_prev);
                 GQLA_SPAN_END(10, t_tile);
                 page_prev = page_j;
             }
             t = t0 + nt;
-            // is another piece coming (its tiles then occupy the ring)?
-            bool more_pieces;
-            {
-                PieceIter nx = it;
-                int b2, L2, pb2, pe2;
-                bool tl2 = false;
-                do {
-                    more_pieces = next_piece(p, nx, b2, L2, pb2, pe2, tl2);
-                } while (more_pieces && tl2);
-            }
             // ---- epilogue: O / l for this warp's 32 rows x 128 columns through TMA stores of
             // 32 x 32 fp32 boxes (128-byte swizzle) staged in shared memory.  After the last
             // piece the ring is free (every tile is consumed) and holds all of it, one store
