@@ -5,6 +5,9 @@
 One step = one decode step of the batch through the whole hot path: the
 MQA-absorb path (gqla_absorb_query -> gqla_decode_absorb -> gqla_combine with
 W_UV) and the GQA path (gqla_decode_gqa -> gqla_combine) over the same batch.
+The two paths are independent, so the GQA path runs on a second stream beside
+the absorb path's decode and combine (after the query absorption has started):
+CTAs of one path take the SMs the other path's tail leaves idle.
 The one-shot cache expansion (gqla_expand_cache) is a deploy-time conversion,
 not part of a step; it is timed once and reported under "expand".
 
@@ -17,12 +20,13 @@ e2e     = the same through the C ABI with host buffers: each step copies the
           both paths' outputs back into pinned memory, inside the timed region
           (the copies and the five calls replayed as one CUDA graph; the page
           table and lengths are one buffer copied on a second stream beside
-          q and the query absorption, and the absorb path's output is copied
-          back on that stream while the GQA path runs).
+          q and the query absorption; the GQA path and its output copy run on
+          a third stream beside the absorb path).
 Timing  = the step is captured into a CUDA graph; each timed step replays it
           between two CUDA events on the stream (device time, no host launch
-          overhead).  The per-call breakdown comes from a second graph with an
-          event record around every call.  L2 is flushed (a 256 MiB write, then a
+          overhead).  The per-call breakdown comes from a second graph that
+          runs the five calls in order on one stream with an event record
+          around every call.  L2 is flushed (a 256 MiB write, then a
           256 MiB read so no dirty line is left) before every step, outside
           its events; W >= 3 untimed eager and W
           graph warm-up steps come first.
@@ -293,30 +297,47 @@ def run_ours(args, rank, world, local_rank):
         lambda: gqla.gqla_combine(dims, kv, s_q, bg.num_splits, 128, bg.o_part, bg.lse_part,
                                   None, bg.out, bg.lse),
     ]
-    def step(events=None):
+    gqa_stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        # query absorption first, then the GQA path on its own stream beside the
+        # absorb path's decode and combine; the step ends when both are done
+        main = torch.cuda.current_stream()
+        calls[0]()
+        fork = torch.cuda.Event()
+        fork.record(main)
+        gqa_stream.wait_event(fork)
+        with torch.cuda.stream(gqa_stream):
+            calls[3]()
+            calls[4]()
+        calls[1]()
+        calls[2]()
+        join = torch.cuda.Event()
+        join.record(gqa_stream)
+        main.wait_event(join)
+
+    def step_in_order(events):
         for i, c in enumerate(calls):
-            if events is not None:
-                events[i].record()
+            events[i].record()
             c()
-        if events is not None:
-            events[-1].record()
+        events[-1].record()
 
     for _ in range(args.warmup):
         flush_l2()
         step()
     torch.cuda.synchronize()
 
-    # The step is captured into a CUDA graph twice: as is (the five launches
-    # replay without host overhead, each kernel's set-up overlapping the
-    # previous kernel's tail) for the step time, and with an event record
-    # around every call for the per-call breakdown.
+    # The step is captured into a CUDA graph (the launches replay without host
+    # overhead, each kernel's set-up overlapping the previous kernel's tail on
+    # its stream) for the step time; a second graph runs the calls in order with
+    # an event record around every call for the per-call breakdown.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step()
     gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
     graph_ev = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_ev):
-        step(gev)
+        step_in_order(gev)
     for g_ in (graph, graph_ev):
         for _ in range(args.warmup):
             flush_l2()
@@ -355,8 +376,8 @@ def run_ours(args, rank, world, local_rank):
     # ---- e2e: host buffers through the C ABI, copies inside the timed region.
     # Every copy costs ~10 us however small, so the page table and the lengths
     # travel as one int32 buffer, on a second stream while q is copied and the
-    # query absorption runs; the absorb path's output goes back on that stream
-    # while the GQA path computes; the step ends when every copy has landed.
+    # query absorption runs; the GQA path and its output copy run on a third
+    # stream beside the absorb path; the step ends when every copy has landed.
     pt_c, sl_c = case["page_table"].cpu(), case["seqlens"].cpu()
     n_pt = pt_c.numel()
     q_h = case["q"].cpu().pin_memory()
@@ -391,20 +412,21 @@ def run_ours(args, rank, world, local_rank):
         meta_in.record(side)
         q_e.copy_(q_h, non_blocking=True)
         calls_e[0]()  # query absorption: needs q only
+        q_in = torch.cuda.Event()
+        q_in.record(main)
+        gqa_stream.wait_event(q_in)
+        gqa_stream.wait_event(meta_in)
+        with torch.cuda.stream(gqa_stream):
+            calls_e[3]()
+            calls_e[4]()
+            outg_h.copy_(bg.out, non_blocking=True)
         main.wait_event(meta_in)
         calls_e[1]()
         calls_e[2]()
-        absorb_done = torch.cuda.Event()
-        absorb_done.record(main)
-        side.wait_event(absorb_done)
-        with torch.cuda.stream(side):
-            outa_h.copy_(ba.out, non_blocking=True)
-        calls_e[3]()
-        calls_e[4]()
-        outg_h.copy_(bg.out, non_blocking=True)
-        side_done = torch.cuda.Event()
-        side_done.record(side)
-        main.wait_event(side_done)
+        outa_h.copy_(ba.out, non_blocking=True)
+        gqa_done = torch.cuda.Event()
+        gqa_done.record(gqa_stream)
+        main.wait_event(gqa_done)
 
     for _ in range(args.warmup):  # eager warm-up, then the same step as one graph
         e2e_step()
