@@ -275,15 +275,21 @@ def run_ours(args, rank, world, local_rank):
         flush.fill_(1.0)
         torch.sum(flush_rd, dim=0, out=flush_sum)
 
-    # one-shot expansion, timed on its own
-    gqla.gqla_expand_cache(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
+    # one-shot expansion, timed on its own: the tensor-core version, then the
+    # bit-exact sequential-order one (whose output the steps below use)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    flush_l2()
-    e0.record()
-    gqla.gqla_expand_cache(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
-    e1.record()
-    torch.cuda.synchronize()
-    expand_ms = e0.elapsed_time(e1)
+
+    def time_expand(fn):
+        fn(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
+        flush_l2()
+        e0.record()
+        fn(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    expand_tc_ms = time_expand(gqla.gqla_expand_cache_tc)
+    expand_ms = time_expand(gqla.gqla_expand_cache)
 
     names = ["absorb_query", "decode_absorb", "combine_absorb", "decode_gqa", "combine_gqa"]
     calls = [
@@ -515,7 +521,9 @@ def run_ours(args, rank, world, local_rank):
                      "gqa": path_info(["decode_gqa", "combine_gqa"], "decode_gqa")},
         "per_kernel": {n: dict(per_kernel[n], share=share[n]) for n in names},
         "expand": {"ms": expand_ms, "slots": n_slots,
-                   "tflops": acc["expand"]["flops"] / (expand_ms * 1e-3) / 1e12},
+                   "tflops": acc["expand"]["flops"] / (expand_ms * 1e-3) / 1e12,
+                   "tc_ms": expand_tc_ms,
+                   "tc_tflops": acc["expand"]["flops"] / (expand_tc_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": len(calls) * args.steps,

@@ -8,6 +8,9 @@ namespace gqla {
 cudaError_t launch_expand(const void *latent, int64_t num_slots, const void *w_uk,
                           const void *w_uv, void *kv, void *k_rope, int num_groups,
                           cudaStream_t stream);
+cudaError_t launch_expand_tc(const void *latent, int64_t num_slots, const void *w_uk,
+                             const void *w_uv, void *kv, void *k_rope, int num_groups,
+                             cudaStream_t stream);
 cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_groups,
                                 const void *w_uk, void *qa, cudaStream_t stream);
 cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups, const void *kv,
@@ -63,6 +66,20 @@ int cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return GQLA_OK;
     g_last_cuda_error = e;
     return GQLA_ERR_CUDA;
+}
+
+int check_expand_args(const gqla_dims *dims, const void *latent, int64_t num_slots, const void *w_uk,
+                      const void *w_uv, void *kv_expanded, void *k_rope) {
+    int st = check_dims(dims, 1);
+    if (st == GQLA_ERR_UNSUPPORTED && dims && dims_supported(dims)) st = GQLA_OK;  // head split irrelevant here
+    if (st != GQLA_OK) return st;
+    if (num_slots < 0) return GQLA_ERR_INVALID_ARG;
+    if (!latent || !w_uk || !w_uv || !kv_expanded || !k_rope) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(latent) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(kv_expanded) ||
+        !aligned16(k_rope))
+        return GQLA_ERR_INVALID_ARG;
+    if (num_slots > ((int64_t)1 << 31) - 1) return GQLA_ERR_UNSUPPORTED;
+    return GQLA_OK;
 }
 
 }  // namespace
@@ -124,17 +141,19 @@ int gqla_clear_device_error(void *workspace, gqla_stream_t stream) {
 int gqla_expand_cache(const gqla_dims *dims, const void *latent, int64_t num_slots,
                       const void *w_uk, const void *w_uv, void *kv_expanded, void *k_rope,
                       gqla_stream_t stream) {
-    int st = check_dims(dims, 1);
-    if (st == GQLA_ERR_UNSUPPORTED && dims && dims_supported(dims)) st = GQLA_OK;  // head split irrelevant here
+    const int st = check_expand_args(dims, latent, num_slots, w_uk, w_uv, kv_expanded, k_rope);
     if (st != GQLA_OK) return st;
-    if (num_slots < 0) return GQLA_ERR_INVALID_ARG;
-    if (!latent || !w_uk || !w_uv || !kv_expanded || !k_rope) return GQLA_ERR_INVALID_ARG;
-    if (!aligned16(latent) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(kv_expanded) ||
-        !aligned16(k_rope))
-        return GQLA_ERR_INVALID_ARG;
-    if (num_slots > ((int64_t)1 << 31) - 1) return GQLA_ERR_UNSUPPORTED;
     return cuda_status(launch_expand(latent, num_slots, w_uk, w_uv, kv_expanded, k_rope,
                                      dims->num_groups, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_expand_cache_tc(const gqla_dims *dims, const void *latent, int64_t num_slots,
+                         const void *w_uk, const void *w_uv, void *kv_expanded, void *k_rope,
+                         gqla_stream_t stream) {
+    const int st = check_expand_args(dims, latent, num_slots, w_uk, w_uv, kv_expanded, k_rope);
+    if (st != GQLA_OK) return st;
+    return cuda_status(launch_expand_tc(latent, num_slots, w_uk, w_uv, kv_expanded, k_rope,
+                                        dims->num_groups, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int gqla_absorb_query(const gqla_dims *dims, const void *q, int batch, int s_q,

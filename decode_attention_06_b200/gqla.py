@@ -58,6 +58,7 @@ _P, _I, _I64, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size
 _DP, _KP = ctypes.POINTER(gqla_dims), ctypes.POINTER(gqla_kv_index)
 _SIGS = {
     "gqla_expand_cache": [_DP, _P, _I64, _P, _P, _P, _P, _P],
+    "gqla_expand_cache_tc": [_DP, _P, _I64, _P, _P, _P, _P, _P],
     "gqla_absorb_query": [_DP, _P, _I, _I, _P, _P, _P],
     "gqla_decode_absorb": [_DP, _P, _I, _P, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _SZ, _P],
@@ -127,6 +128,17 @@ def gqla_expand_cache(dims, latent, w_uk, w_uv, kv_expanded, k_rope, stream=None
     n = latent.numel() // D_ROW
     g = dims.num_groups
     _check("gqla_expand_cache", _lib.gqla_expand_cache(
+        ctypes.byref(dims), _dev(latent, "latent", torch.bfloat16), n,
+        _dev(w_uk, "w_uk", torch.bfloat16, (g, D_LATENT, D_NOPE)),
+        _dev(w_uv, "w_uv", torch.bfloat16, (g, D_LATENT, D_V)),
+        _dev(kv_expanded, "kv_expanded", torch.bfloat16, (g, n, D_NOPE + D_V)),
+        _dev(k_rope, "k_rope", torch.bfloat16, (n, D_ROPE)), _stream(stream)))
+
+
+def gqla_expand_cache_tc(dims, latent, w_uk, w_uv, kv_expanded, k_rope, stream=None):
+    n = latent.numel() // D_ROW
+    g = dims.num_groups
+    _check("gqla_expand_cache_tc", _lib.gqla_expand_cache_tc(
         ctypes.byref(dims), _dev(latent, "latent", torch.bfloat16), n,
         _dev(w_uk, "w_uk", torch.bfloat16, (g, D_LATENT, D_NOPE)),
         _dev(w_uv, "w_uv", torch.bfloat16, (g, D_LATENT, D_V)),

@@ -104,6 +104,19 @@ int gqla_expand_cache(const gqla_dims *dims, const void *latent, int64_t num_slo
                       gqla_stream_t stream);
 
 /*
+ * The same expansion on the tensor cores (tcgen05): identical arguments,
+ * layouts, ownership and errors as gqla_expand_cache; each output is the
+ * fp32 tensor-core accumulation of the same 512 exact bf16 x bf16 products in
+ * the hardware's own order, rounded once to bf16 (nearest, ties to even).
+ * Not bit-reproducible against gqla_expand_cache: every output x satisfies
+ * |x - exact| <= 2^-8 |exact| + 2^-15 sum_k |c_k w_k| (the bf16 rounding plus
+ * the fp32 accumulation bound for 512 terms); k_rope is copied exactly.
+ */
+int gqla_expand_cache_tc(const gqla_dims *dims, const void *latent, int64_t num_slots,
+                         const void *w_uk, const void *w_uv, void *kv_expanded, void *k_rope,
+                         gqla_stream_t stream);
+
+/*
  * Query absorption: W_UK folded into the query (paperlayer.ai summary, sec. 2).
  *   q           bf16 [batch][s_q][h][192]  (0..127 q^C, 128..191 q^R, RoPE applied)
  *   w_uk        bf16 [g][512][128]

@@ -47,6 +47,48 @@ def test_expand_cache_bit_exact(n_pages, extra):
     assert (got_kr == ref_kr).all()
 
 
+@pytest.mark.parametrize("n_pages,extra,g", [(3, 0, 8), (5, 17, 8), (4, 100, 4)])
+def test_expand_cache_tc_within_rounding_bound(n_pages, extra, g):
+    """Tensor-core expansion: every value within one bf16 rounding of the exact
+    product plus the fp32 accumulation bound for 512 terms (the header's contract);
+    k_rope copied exactly."""
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(128, g, [64 * n_pages], 1, seed=200 + n_pages)
+    lat = case["latent"].reshape(-1, 576)
+    if extra:  # a slot count that is not a multiple of the 128-slot tile
+        lat = torch.cat([lat, lat[:extra] * 0.5]).contiguous()
+    n = lat.shape[0]
+    dims = gqla.make_dims(128, g)
+    kv = torch.empty(g, n, 256, dtype=torch.bfloat16, device="cuda")
+    kr = torch.empty(n, 64, dtype=torch.bfloat16, device="cuda")
+    gqla.gqla_expand_cache_tc(dims, lat.cuda(), case["w_uk"].cuda(), case["w_uv"].cuda(), kv, kr)
+    torch.cuda.synchronize()
+    exact, ref_kr = oracle.expand_f64(lat, case["w_uk"], case["w_uv"])
+    c = lat[:, :512].double().numpy()
+    w = torch.cat([case["w_uk"], case["w_uv"]], dim=2).double().numpy()  # [g][512][256]
+    mag = np.einsum("nk,gkc->gnc", np.abs(c), np.abs(w))
+    # bf16 rounding to nearest: at most half a unit in the last place, 2^-8 |x|
+    bound = 2.0 ** -8 * np.abs(exact) + 2.0 ** -15 * mag
+    got = kv.cpu().double().numpy()
+    err = np.abs(got - exact)
+    excess = err - bound
+    assert excess.max() <= 0, f"{(excess > 0).sum()} values outside the bound, worst by {excess.max():.3g}"
+    assert np.array_equal(kr.cpu().double().numpy(), ref_kr)
+    # and no more than one bf16 step from the sequential-order expansion wherever the
+    # two fp32 sums (each within 2^-15 mag of exact) differ by less than one bf16 step
+    # (|exact| >= 2^-6 mag); below that, cancellation makes the bound above the test
+    seq = torch.empty_like(kv)
+    kr2 = torch.empty_like(kr)
+    gqla.gqla_expand_cache(dims, lat.cuda(), case["w_uk"].cuda(), case["w_uv"].cuda(), seq, kr2)
+    torch.cuda.synchronize()
+    a = kv.cpu().view(torch.int16).numpy().astype(np.int32)
+    b = seq.cpu().view(torch.int16).numpy().astype(np.int32)
+    same_sign = (a ^ b) >= 0
+    checked = same_sign & (np.abs(exact) >= 2.0 ** -6 * mag)
+    assert checked.mean() > 0.5
+    assert np.all(np.abs(a - b)[checked] <= 1), "values more than one bf16 step apart"
+
+
 @pytest.mark.parametrize("h,B,s_q", [(32, 3, 1), (128, 5, 2), (128, 9, 1)])
 def test_absorb_query_matches_oracle(h, B, s_q):
     from decode_attention_06_b200 import gqla
