@@ -133,3 +133,24 @@ def make_workload(name: str, s_q: Optional[int] = None, device: str = "cpu"):
         raise ValueError(f"{name} is defined for s_q in {w.s_q}")
     return make_case(w.num_heads, w.num_groups, w.seqlens(), s, paged=w.paged,
                      seed=w.seed, device=device)
+
+
+def make_topk(seqlens, s_q: int, topk: int, seed: int = 0, unused: int = 0) -> torch.Tensor:
+    """Selected token positions for sparse attention: int32 [B][s_q][topk].
+
+    Query token s of sequence b gets min(topk - unused, visible) distinct
+    positions drawn uniformly from its visible tokens [0, L_b - s_q + s], in
+    random order; the remaining entries are -1 (unused).  The indexer that
+    would choose them from the data is outside this path, so a seeded uniform
+    choice stands in for it.
+    """
+    g = torch.Generator().manual_seed(seed)
+    sl = [int(x) for x in torch.as_tensor(seqlens).tolist()]
+    out = torch.full((len(sl), s_q, topk), -1, dtype=torch.int32)
+    for b, L in enumerate(sl):
+        for s in range(s_q):
+            vis = L - s_q + s + 1
+            n = max(0, min(topk - unused, vis))
+            if n:
+                out[b, s, :n] = torch.randperm(vis, generator=g)[:n].to(torch.int32)
+    return out

@@ -18,7 +18,11 @@ Sources, by page and section:
   * GQLA, gist.science technical summary: sec. 2 Methodik (group-indexed
     W_UK / W_UV, the two paths).
   * GQLA, pwwt.cn article: sec. 3 (4224 B / 1152 B per token, 16 heads per
-    group), sec. 4 (LLaMA-3-8B 2048-element GQA cache, 28.125 %).
+    group), sec. 4 (LLaMA-3-8B 2048-element GQA cache, 28.125 %), sec. 5
+    (sparse attention: each new token attends to a selected subset).
+
+``decode_sparse`` is numpy (fp64, library matmuls), not C: the sparse variant
+is small and its per-query selection makes the C unit loop a poor fit.
 """
 from __future__ import annotations
 
@@ -150,6 +154,45 @@ def decode(q, cache, page_table, seqlens, w_uk, w_uv, num_groups, page_size=64,
                                 u_ptr, n_units, _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("gqla_oracle_decode: bad arguments")
+    return out, lse
+
+
+def decode_sparse(q, cache, page_table, seqlens, w_uk, w_uv, num_groups, topk_idx, page_size=64,
+                  scale=None):
+    """Sparse GQLA (paperlayer.ai summary, sec. 2 "Sparse GQLA"; pwwt.cn article,
+    sec. 5): query token s of sequence b attends only to the token positions in
+    topk_idx[b][s] (the same set for every head; -1 = unused entry), with the
+    un-absorbed definition of ``decode`` otherwise: K = [c W_UK_g | k^R],
+    V = c W_UV_g, softmax of q.K * scale over the set, out = sum p V.
+    Positions must be visible (0 <= t <= L_b - s_q + s).  Returns
+    (out [B][s_q][h][128], lse [B][s_q][h]) in fp64; an empty set gives out = 0
+    and lse = -inf.
+    """
+    q = _f64(q); pages = _f64(cache); pt = _i32(page_table); sl = _i32(seqlens)
+    wk = _f64(w_uk); wv = _f64(w_uv); idx = np.asarray(_to_numpy(topk_idx), dtype=np.int64)
+    B, s_q, h, dqk = q.shape
+    assert dqk == D_QK and pages.shape[1] == page_size and pages.shape[-1] == D_ROW
+    G = h // num_groups
+    sc = default_scale() if scale is None else scale
+    out = np.zeros((B, s_q, h, D_V))
+    lse = np.full((B, s_q, h), -np.inf)
+    for b in range(B):
+        for s in range(s_q):
+            t = idx[b, s][idx[b, s] >= 0]
+            if t.size == 0:
+                continue
+            assert t.max() <= sl[b] - s_q + s, "a selected token is not visible"
+            rows = pages[pt[b, t // page_size], t % page_size]     # [n][576]
+            c, kr = rows[:, :D_LATENT], rows[:, D_LATENT:]
+            for g in range(num_groups):
+                K = np.concatenate([c @ wk[g], kr], axis=1)       # [n][192]
+                V = c @ wv[g]                                      # [n][128]
+                x = (q[b, s, g * G:(g + 1) * G] @ K.T) * sc        # [G][n]
+                m = x.max(axis=1, keepdims=True)
+                e = np.exp(x - m)
+                l = e.sum(axis=1, keepdims=True)
+                out[b, s, g * G:(g + 1) * G] = (e / l) @ V
+                lse[b, s, g * G:(g + 1) * G] = (m + np.log(l))[:, 0]
     return out, lse
 
 

@@ -385,3 +385,92 @@ def test_rising_scores_case_rescales():
         rises.append(np.diff(pm, axis=1).ravel())
     rises = np.concatenate(rises)
     assert (rises > 8.0).mean() > 0.4
+
+
+# ---------------------------------------------------------------- sparse variant
+
+def _sparse_case(h=32, g=8, seqlens=(70, 130), s_q=2, seed=21):
+    return synth.make_case(h, g, list(seqlens), s_q, paged=True, seed=seed)
+
+
+def test_sparse_all_visible_equals_dense():
+    """Selecting every visible token is ordinary decode attention (the C oracle)."""
+    case = _sparse_case()
+    sl, s_q = case["seqlens"].tolist(), case["s_q"]
+    idx = synth.make_topk(sl, s_q, max(sl), seed=3)  # topk >= visible: every token, shuffled
+    got, got_lse = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                        case["w_uk"], case["w_uv"], 8, idx)
+    ref, ref_lse = oracle.decode(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                 case["w_uk"], case["w_uv"], 8)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=1e-11)
+
+
+def test_sparse_single_token_is_its_value_row():
+    """One selected token: the output is that token's V row and the LSE its score."""
+    case = _sparse_case(h=32, g=8, seqlens=(90,), s_q=1, seed=22)
+    t = 37
+    idx = torch.full((1, 1, 5), -1, dtype=torch.int32)
+    idx[0, 0, 3] = t
+    out, lse = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                    case["w_uk"], case["w_uv"], 8, idx)
+    row = case["latent"].reshape(-1, 576)[int(case["page_table"][0, t // 64]) * 64 + t % 64].double().numpy()
+    wk, wv = case["w_uk"].double().numpy(), case["w_uv"].double().numpy()
+    q = case["q"].double().numpy()[0, 0]
+    for hh in range(32):
+        gg = hh // 4
+        np.testing.assert_allclose(out[0, 0, hh], row[:512] @ wv[gg], rtol=0, atol=1e-12)
+        k = np.concatenate([row[:512] @ wk[gg], row[512:]])
+        assert abs(lse[0, 0, hh] - (q[hh] @ k) * SCALE) < 1e-12
+
+
+def test_sparse_brute_force_tiny():
+    """A four-token subset against explicit loops over tokens and dimensions."""
+    case = _sparse_case(h=32, g=8, seqlens=(40,), s_q=1, seed=23)
+    sel = [3, 17, 31, 39]
+    idx = torch.tensor([[sel + [-1, -1]]], dtype=torch.int32)
+    out, lse = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                    case["w_uk"], case["w_uv"], 8, idx)
+    lat = case["latent"].reshape(-1, 576).double().numpy()
+    pt = case["page_table"][0].tolist()
+    wk, wv = case["w_uk"].double().numpy(), case["w_uv"].double().numpy()
+    q = case["q"].double().numpy()[0, 0]
+    for hh in (0, 13, 31):
+        gg = hh // 4
+        scores, values = [], []
+        for t in sel:
+            c = lat[pt[t // 64] * 64 + t % 64]
+            k = [sum(c[i] * wk[gg, i, j] for i in range(512)) for j in range(128)] + list(c[512:])
+            scores.append(sum(q[hh, j] * k[j] for j in range(192)) * SCALE)
+            values.append([sum(c[i] * wv[gg, i, j] for i in range(512)) for j in range(128)])
+        m = max(scores)
+        w = [math.exp(x - m) for x in scores]
+        want = [sum(w[n] * values[n][j] for n in range(4)) / sum(w) for j in range(128)]
+        np.testing.assert_allclose(out[0, 0, hh], want, rtol=0, atol=1e-11)
+        assert abs(lse[0, 0, hh] - (m + math.log(sum(w)))) < 1e-11
+
+
+def test_sparse_order_and_padding_invariant():
+    case = _sparse_case(seed=24)
+    sl, s_q = case["seqlens"].tolist(), case["s_q"]
+    idx = synth.make_topk(sl, s_q, 40, seed=5, unused=9)
+    perm = idx.clone()
+    for b in range(idx.shape[0]):
+        for s in range(s_q):
+            perm[b, s] = idx[b, s][torch.randperm(idx.shape[-1], generator=torch.Generator().manual_seed(b * 7 + s))]
+    a, la = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                 case["w_uk"], case["w_uv"], 8, idx)
+    b_, lb = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                  case["w_uk"], case["w_uv"], 8, perm)
+    np.testing.assert_allclose(a, b_, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(la, lb, rtol=0, atol=1e-12)
+
+
+def test_make_topk_draws_distinct_visible_positions():
+    idx = synth.make_topk([10, 300], 2, 64, seed=1, unused=4)
+    for b, L in enumerate([10, 300]):
+        for s in range(2):
+            t = idx[b, s][idx[b, s] >= 0]
+            assert t.numel() == min(60, L - 2 + s + 1)
+            assert len(set(t.tolist())) == t.numel()
+            assert int(t.max()) <= L - 2 + s
