@@ -11,6 +11,10 @@ cudaError_t launch_expand(const void *latent, int64_t num_slots, const void *w_u
 cudaError_t launch_expand_tc(const void *latent, int64_t num_slots, const void *w_uk,
                              const void *w_uv, void *kv, void *k_rope, int num_groups,
                              cudaStream_t stream);
+cudaError_t launch_sparse_gather(const void *kv, const void *k_rope, int64_t num_slots,
+                                 const gqla_kv_index *idx, int s_q, const int32_t *topk_idx, int topk,
+                                 int num_groups, void *kv_sel, void *k_rope_sel, int32_t *sel_page_table,
+                                 int32_t *sel_seqlens, void *ws, cudaStream_t stream);
 cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_groups,
                                 const void *w_uk, void *qa, cudaStream_t stream);
 cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups, const void *kv,
@@ -205,6 +209,29 @@ int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *k
                                          k_rope, num_slots, kv, num_splits, dims->softmax_scale,
                                          o_part, lse_part, workspace,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_sparse_gather(const gqla_dims *dims, const void *kv_expanded, const void *k_rope,
+                       int64_t num_slots, const gqla_kv_index *kv, int s_q, const int32_t *topk_idx,
+                       int topk, void *kv_sel, void *k_rope_sel, int32_t *sel_page_table,
+                       int32_t *sel_seqlens, void *workspace, size_t workspace_bytes,
+                       gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if ((st = check_index(kv)) != GQLA_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes)) != GQLA_OK) return st;
+    if (topk <= 0 || topk > 65536) return GQLA_ERR_INVALID_ARG;
+    if (!kv_expanded || !k_rope || !topk_idx || !kv_sel || !k_rope_sel || !sel_page_table || !sel_seqlens)
+        return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(kv_expanded) || !aligned16(k_rope) || !aligned16(kv_sel) || !aligned16(k_rope_sel))
+        return GQLA_ERR_INVALID_ARG;
+    if (num_slots != (int64_t)kv->num_pages * kv->page_size) return GQLA_ERR_INVALID_ARG;
+    if (dims->num_groups != 8 && dims->num_groups != 4) return GQLA_ERR_UNSUPPORTED;
+    const int64_t cap = (topk + 63) / 64 * 64;
+    if ((int64_t)kv->batch * s_q * cap > ((int64_t)1 << 31) - 1) return GQLA_ERR_UNSUPPORTED;
+    return cuda_status(launch_sparse_gather(kv_expanded, k_rope, num_slots, kv, s_q, topk_idx, topk,
+                                            dims->num_groups, kv_sel, k_rope_sel, sel_page_table,
+                                            sel_seqlens, workspace, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,

@@ -63,6 +63,7 @@ _SIGS = {
     "gqla_decode_absorb": [_DP, _P, _I, _P, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_combine": [_DP, _KP, _I, _I, _I, _P, _P, _P, _P, _P, _P],
+    "gqla_sparse_gather": [_DP, _P, _P, _I64, _KP, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa_noalloc": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _P],
     "gqla_partial_slots": [_I, _I],
     "gqla_workspace_bytes": [],
@@ -195,6 +196,24 @@ def gqla_combine(dims, kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out, l
         _stream(stream)))
 
 
+def gqla_sparse_gather(dims, kv_expanded, k_rope, kv, s_q, topk_idx, kv_sel, k_rope_sel,
+                       sel_page_table, sel_seqlens, workspace, stream=None):
+    B = kv.batch
+    n = kv.num_pages * kv.page_size
+    topk = topk_idx.shape[-1]
+    cap = (topk + PAGE_SIZE - 1) // PAGE_SIZE * PAGE_SIZE
+    ns = B * s_q * cap
+    _check("gqla_sparse_gather", _lib.gqla_sparse_gather(
+        ctypes.byref(dims), _dev(kv_expanded, "kv_expanded", torch.bfloat16, (dims.num_groups, n, D_NOPE + D_V)),
+        _dev(k_rope, "k_rope", torch.bfloat16, (n, D_ROPE)), n, ctypes.byref(kv), s_q,
+        _dev(topk_idx, "topk_idx", torch.int32, (B, s_q, topk)), topk,
+        _dev(kv_sel, "kv_sel", torch.bfloat16, (dims.num_groups, ns, D_NOPE + D_V)),
+        _dev(k_rope_sel, "k_rope_sel", torch.bfloat16, (ns, D_ROPE)),
+        _dev(sel_page_table, "sel_page_table", torch.int32, (B * s_q, cap // PAGE_SIZE)),
+        _dev(sel_seqlens, "sel_seqlens", torch.int32, (B * s_q,)),
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream)))
+
+
 def gqla_decode_gqa_noalloc(dims, q, kv_expanded, k_rope, kv, num_splits, out, lse_out=None,
                             device_error=None, stream=None):
     """GQA decode step with library-owned static scratch (no o_part/lse_part/workspace)."""
@@ -272,6 +291,39 @@ class DecodeBuffers:
         self.out = torch.empty(batch, s_q, h, D_V, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(batch, s_q, h, dtype=torch.float32, device=device)
         self.workspace = new_workspace(device)
+
+
+class SparseBuffers:
+    """Device buffers of one sparse GQA step: the selected cache, its index and
+    the decode buffers of the batch * s_q selected sequences."""
+
+    def __init__(self, dims, batch: int, s_q: int, topk: int, num_splits: int, device="cuda"):
+        self.s_q, self.topk = s_q, topk
+        self.cap = (topk + PAGE_SIZE - 1) // PAGE_SIZE * PAGE_SIZE
+        v = batch * s_q
+        self.kv_sel = torch.empty(dims.num_groups, v * self.cap, D_NOPE + D_V, dtype=torch.bfloat16,
+                                  device=device)
+        self.k_rope_sel = torch.empty(v * self.cap, D_ROPE, dtype=torch.bfloat16, device=device)
+        self.sel_page_table = torch.empty(v, self.cap // PAGE_SIZE, dtype=torch.int32, device=device)
+        self.sel_seqlens = torch.empty(v, dtype=torch.int32, device=device)
+        self.sel_index = make_kv_index(self.sel_page_table, self.sel_seqlens, v * self.cap // PAGE_SIZE)
+        self.dec = DecodeBuffers(dims, v, 1, num_splits, "gqa", device=device)
+        self.workspace = self.dec.workspace
+
+
+def sparse_gqa_step(dims, bufs: SparseBuffers, q, kv_expanded, k_rope, kv, topk_idx, stream=None):
+    """Sparse GQA step through the C ABI: gather the selected tokens, then the
+    GQA decode and combine over batch * s_q one-token queries.  Returns
+    (out [batch][s_q][h][128] bf16, lse [batch][s_q][h])."""
+    B, s_q, h, _ = q.shape
+    gqla_sparse_gather(dims, kv_expanded, k_rope, kv, s_q, topk_idx, bufs.kv_sel, bufs.k_rope_sel,
+                       bufs.sel_page_table, bufs.sel_seqlens, bufs.workspace, stream)
+    q1 = q.view(B * s_q, 1, h, D_QK)
+    gqla_decode_gqa(dims, q1, bufs.kv_sel, bufs.k_rope_sel, bufs.sel_index, bufs.dec.num_splits,
+                    bufs.dec.o_part, bufs.dec.lse_part, bufs.workspace, stream)
+    gqla_combine(dims, bufs.sel_index, 1, bufs.dec.num_splits, D_V, bufs.dec.o_part, bufs.dec.lse_part,
+                 None, bufs.dec.out, bufs.dec.lse, stream)
+    return bufs.dec.out.view(B, s_q, h, D_V), bufs.dec.lse.view(B, s_q, h)
 
 
 def decode_step(dims, bufs: DecodeBuffers, q, w_uk, w_uv, kv, latent_cache=None,

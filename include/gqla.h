@@ -167,6 +167,35 @@ int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *k
                     size_t workspace_bytes, gqla_stream_t stream);
 
 /*
+ * Sparse GQLA, GQA path (paperlayer.ai summary, sec. 2 "Sparse GQLA";
+ * pwwt.cn article, sec. 5): each query token (b, s) attends only to its own
+ * selected token positions, the same set for all heads.  This call gathers
+ * them into a compact "selected" cache on which gqla_decode_gqa and
+ * gqla_combine then run unchanged, as batch * s_q sequences of one query
+ * token each (q and out keep their [batch][s_q][h][...] layout).
+ *   kv_expanded, k_rope, num_slots, kv   the GQA-path cache, as for gqla_decode_gqa
+ *   s_q          1 or 2
+ *   topk_idx     int32 [batch][s_q][topk] device: token positions, distinct
+ *                within a list; -1 marks an unused entry.  A position outside
+ *                [0, L_b - s_q + s] or on a page outside the pool is reported
+ *                (GQLA_ERR_DEVICE, info = b * s_q + s) and skipped.
+ *   topk         1 .. 65536; cap = topk rounded up to a multiple of 64
+ *   kv_sel       bf16 [g][batch * s_q * cap][256]   out (rows past each list's
+ *   k_rope_sel   bf16 [batch * s_q * cap][64]        out  valid entries untouched)
+ *   sel_page_table int32 [batch * s_q][cap / 64]     out (identity)
+ *   sel_seqlens  int32 [batch * s_q]                 out: valid entries per list
+ *   workspace    as for the decode calls (device error record)
+ * Then: gqla_decode_gqa(dims, q, 1, kv_sel, k_rope_sel, batch * s_q * cap,
+ * {sel_page_table, sel_seqlens, batch * s_q, cap / 64, 64, batch * s_q * cap / 64}, ...)
+ * and gqla_combine with the same index and s_q = 1.
+ */
+int gqla_sparse_gather(const gqla_dims *dims, const void *kv_expanded, const void *k_rope,
+                       int64_t num_slots, const gqla_kv_index *kv, int s_q, const int32_t *topk_idx,
+                       int topk, void *kv_sel, void *k_rope_sel, int32_t *sel_page_table,
+                       int32_t *sel_seqlens, void *workspace, size_t workspace_bytes,
+                       gqla_stream_t stream);
+
+/*
  * Log-sum-exp merge of the partials of each sequence, then (absorb path,
  * d_in == 512) the per-group up-projection out = o~ W_UV_{g(h)}: W_UV folded into
  * the output (paperlayer.ai summary, sec. 2).

@@ -222,3 +222,64 @@ def test_decode_parity_full_size_sampled(path, name, s_q):
     compare_lse(lse[torch.tensor(picks, device="cuda")], ref_lse, mask=mask)
     from decode_attention_06_b200 import gqla
     assert gqla.gqla_read_device_error(ws)[0] == 0
+
+
+# ------------------------------------------------------------------ sparse GQLA (GQA path)
+
+SPARSE = [
+    # id, h, g, seqlens, s_q, topk, unused entries, splits
+    ("h128_topk256_pad", 128, 8, [1000, 70, 3000], 1, 256, 20, None),
+    ("h128_mtp_topk100", 128, 8, [513, 130], 2, 100, 0, 5),
+    ("g4_topk64", 128, 4, [700], 1, 64, 0, 3),
+    ("h32_mtp_topk300_short", 32, 8, [2000, 3], 2, 300, 7, None),
+]
+
+
+def _sparse_run(case, idx, splits):
+    from decode_attention_06_b200 import gqla
+    g = to_gpu(case)
+    h, ng, s_q = case["num_heads"], case["num_groups"], case["s_q"]
+    dims = gqla.make_dims(h, ng)
+    kv = gqla.make_kv_index(g["page_table"], g["seqlens"], g["num_pages"])
+    n = case["num_pages"] * case["page_size"]
+    kvx = torch.empty(ng, n, 256, dtype=torch.bfloat16, device="cuda")
+    kr = torch.empty(n, 64, dtype=torch.bfloat16, device="cuda")
+    gqla.gqla_expand_cache(dims, g["latent"], g["w_uk"], g["w_uv"], kvx, kr)
+    B = case["seqlens"].numel()
+    if splits is None:
+        splits = gqla.gqla_num_splits_hint("gqa", h, 1)
+    bufs = gqla.SparseBuffers(dims, B, s_q, idx.shape[-1], splits)
+    out, lse = gqla.sparse_gqa_step(dims, bufs, g["q"], kvx, kr, kv, idx.cuda())
+    torch.cuda.synchronize()
+    return out.clone(), lse.clone(), bufs
+
+
+@pytest.mark.parametrize("cid,h,g,seqlens,s_q,topk,unused,splits", SPARSE, ids=[c[0] for c in SPARSE])
+def test_sparse_gqa_parity(cid, h, g, seqlens, s_q, topk, unused, splits):
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(h, g, seqlens, s_q, paged=True, seed=300 + len(cid))
+    idx = synth.make_topk(seqlens, s_q, topk, seed=400 + len(cid), unused=unused)
+    out, lse, bufs = _sparse_run(case, idx, splits)
+    st, _ = gqla.gqla_read_device_error(bufs.workspace)
+    assert st == 0
+    ref, ref_lse = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                        case["w_uk"], case["w_uv"], g, idx)
+    compare(out, ref, what=f"sparse/{cid}")
+    compare_lse(lse, ref_lse, what=f"sparse/{cid}")
+    counts = (idx >= 0).sum(-1).flatten()
+    assert torch.equal(bufs.sel_seqlens.cpu(), counts.to(torch.int32))
+
+
+def test_sparse_invalid_position_is_reported_and_skipped():
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(128, 8, [300, 200], 1, paged=True, seed=311)
+    idx = synth.make_topk([300, 200], 1, 64, seed=312, unused=2)
+    idx[1, 0, 62] = 200   # past the last visible token of sequence 1 (199)
+    out, lse, bufs = _sparse_run(case, idx, None)
+    st, info = gqla.gqla_read_device_error(bufs.workspace)
+    assert st == -5 and info == 1
+    idx_ok = idx.clone()
+    idx_ok[1, 0, 62] = -1
+    ref, ref_lse = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
+                                        case["w_uk"], case["w_uv"], 8, idx_ok)
+    compare(out, ref, what="sparse/invalid-skipped")
