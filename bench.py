@@ -529,11 +529,83 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": len(calls) * args.steps,
         "clocks": clocks.summary(),
     }
+    if args.sparse_topk:
+        result["sparse"] = run_sparse(args, dims, case, s_q, kvx, kr, kv, flush_l2, hbm_peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, what = cpu_oracle_rate(case, w, s_q, budget_s=args.cpu_budget)
         result["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
                                   "kind": "oracle", "sample": what}
     return result
+
+
+def run_sparse(args, dims, case, s_q, kvx, kr, kv, flush_l2, hbm_peak):
+    """Sparse GQLA on the GQA path: every query token attends to --sparse-topk
+    seeded positions of its visible context; gather + GQA decode + combine,
+    timed like the step (one graph, L2 flushed before each replay) and per call."""
+    from decode_attention_06_b200 import gqla, synth
+    B = case["seqlens"].numel()
+    topk = args.sparse_topk
+    idx = synth.make_topk(case["seqlens"].cpu(), s_q, topk, seed=77).to(case["q"].device)
+    splits = args.splits or gqla.gqla_num_splits_hint("gqa", dims.num_heads, 1)
+    sb = gqla.SparseBuffers(dims, B, s_q, topk, splits, device=case["q"].device)
+    q1 = case["q"].view(B * s_q, 1, dims.num_heads, 192)
+    calls = [
+        lambda: gqla.gqla_sparse_gather(dims, kvx, kr, kv, s_q, idx, sb.kv_sel, sb.k_rope_sel,
+                                        sb.sel_page_table, sb.sel_seqlens, sb.workspace),
+        lambda: gqla.gqla_decode_gqa(dims, q1, sb.kv_sel, sb.k_rope_sel, sb.sel_index, splits,
+                                     sb.dec.o_part, sb.dec.lse_part, sb.workspace),
+        lambda: gqla.gqla_combine(dims, sb.sel_index, 1, splits, 128, sb.dec.o_part, sb.dec.lse_part,
+                                  None, sb.dec.out, sb.dec.lse),
+    ]
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+
+    def step(events=None):
+        for i, c in enumerate(calls):
+            if events is not None:
+                events[i].record()
+            c()
+        if events is not None:
+            events[-1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    graphs = []
+    for events in (None, ev):
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_):
+            step(events)
+        graphs.append(g_)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_step, t_call = [], [[] for _ in calls]
+    for _ in range(args.steps):
+        flush_l2()
+        e0.record()
+        graphs[0].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        t_step.append(e0.elapsed_time(e1))
+        flush_l2()
+        graphs[1].replay()
+        torch.cuda.synchronize()
+        for i in range(len(calls)):
+            t_call[i].append(ev[i].elapsed_time(ev[i + 1]))
+    st, _ = gqla.gqla_read_device_error(sb.workspace)
+    if st:
+        raise RuntimeError(f"device-side error in the sparse step: {st}")
+    n_sel = int(sb.sel_seqlens.sum())
+    tok_bytes = 2 * (2 * dims.num_groups * 128 + 64)
+    q_bytes = B * s_q * dims.num_heads * 192 * 2
+    ms = sum(t_step) / len(t_step)
+    us = {n: 1e3 * sum(v) / len(v) for n, v in zip(["gather", "decode_gqa", "combine"], t_call)}
+    # one pass over the selected rows, the queries and the output: what a fused kernel would move
+    fused_bytes = n_sel * tok_bytes + q_bytes + B * s_q * dims.num_heads * 128 * 2
+    return {"topk": topk, "selected_tokens": n_sel, "us_per_step": ms * 1e3,
+            "tokens_per_s": B * s_q / (ms * 1e-3), "per_call_us": us,
+            "gather_gbs": 2 * n_sel * tok_bytes / (us["gather"] * 1e-6) / 1e9,
+            "fused_bytes": fused_bytes,
+            "hbm_frac_of_fused": fused_bytes / (ms * 1e-3) / 1e9 / hbm_peak,
+            "selection": "seeded uniform distinct visible positions (synth.make_topk)"}
 
 
 def run_reference(args, rank, world):
@@ -622,6 +694,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--sparse-topk", type=int, default=0,
+                    help="also time sparse GQLA with this many selected positions per query token")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
                     help="print the per-kernel summary of an ncu launch list and exit")
     args = ap.parse_args()

@@ -227,6 +227,7 @@ int gqla_sparse_gather(const gqla_dims *dims, const void *kv_expanded, const voi
         return GQLA_ERR_INVALID_ARG;
     if (num_slots != (int64_t)kv->num_pages * kv->page_size) return GQLA_ERR_INVALID_ARG;
     if (dims->num_groups != 8 && dims->num_groups != 4) return GQLA_ERR_UNSUPPORTED;
+    if ((int64_t)kv->batch * s_q > 65535) return GQLA_ERR_UNSUPPORTED;  // one grid row per query token
     const int64_t cap = (topk + 63) / 64 * 64;
     if ((int64_t)kv->batch * s_q * cap > ((int64_t)1 << 31) - 1) return GQLA_ERR_UNSUPPORTED;
     return cuda_status(launch_sparse_gather(kv_expanded, k_rope, num_slots, kv, s_q, topk_idx, topk,

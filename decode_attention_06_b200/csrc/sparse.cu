@@ -13,11 +13,11 @@
 // (every selected token is visible to its query), and the usual combine
 // merges the splits.
 //
-// One CTA per query token; 256 entries of the list at a time are checked
-// (-1 marks an unused entry; any other position outside [0, L_b - s_q + s] or
-// on a page outside the pool is a device error and is skipped), compacted by
-// a block-wide prefix count, and copied with consecutive threads on
-// consecutive 16-byte chunks of a row.
+// One CTA per 64 entries of a list: it counts the valid entries before its
+// own (-1 marks an unused entry; any other position outside [0, L_b - s_q + s]
+// or on a page outside the pool is a device error and is skipped), compacts
+// its entries with a warp ballot, and copies their rows with consecutive
+// threads on consecutive 16-byte chunks of a row.
 #include "common.cuh"
 
 namespace gqla {
@@ -25,6 +25,7 @@ namespace gqla {
 namespace {
 
 constexpr int kSgThreads = 256;
+constexpr int kSgChunk = 32;   // list entries per CTA (one warp compacts them)
 
 struct SgParams {
     const __nv_bfloat16 *kv;      // [g][num_slots][256]
@@ -41,64 +42,79 @@ struct SgParams {
     int s_q, topk, cap, max_pages, num_pages, num_groups;
 };
 
+// Cache slot of list entry t for a query that sees tokens [0, last], or -1.
+__device__ __forceinline__ int entry_slot(const SgParams &p, const int32_t *prow, int t, int last) {
+    if (t < 0 || t > last || t / kPage >= p.max_pages) return -1;
+    const int page = prow[t / kPage];
+    return page >= 0 && page < p.num_pages ? page * kPage + t % kPage : -1;
+}
+
+// grid (entries / kSgChunk, batch * s_q): CTA (c, v) compacts entries
+// [c * kSgChunk, (c + 1) * kSgChunk) of list v, after counting the valid entries
+// before them.
 __global__ void __launch_bounds__(kSgThreads) sparse_gather_kernel(const SgParams p) {
     __shared__ int s_warp[kSgThreads / 32];
-    __shared__ int s_slot[kSgThreads];
-    __shared__ int s_dst[kSgThreads];
-    const int v = blockIdx.x;
+    __shared__ int s_slot[kSgChunk];
+    __shared__ int s_dst[kSgChunk];
+    const int v = blockIdx.y, j0 = blockIdx.x * kSgChunk;
     const int b = v / p.s_q, s = v % p.s_q;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int L = p.seqlens[b];
     const int last = L - p.s_q + s;  // this query sees t <= last
     const int32_t *idx = p.idx + (int64_t)v * p.topk;
     const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
-    const int chunks16 = p.num_groups * 32 + 8;  // 16-byte chunks per selected token
-    int count = 0;
-    for (int j0 = 0; j0 < p.topk; j0 += kSgThreads) {
+    // valid entries before this chunk
+    int n = 0;
+    for (int j = threadIdx.x; j < j0; j += kSgThreads) n += entry_slot(p, prow, idx[j], last) >= 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    if (lane == 0) s_warp[warp] = n;
+    __syncthreads();
+    int before = 0;
+#pragma unroll
+    for (int w = 0; w < kSgThreads / 32; ++w) before += s_warp[w];
+    __syncthreads();  // s_warp is reused below
+    // this chunk (warp 0): validity (errors reported here only), compaction by a ballot
+    static_assert(kSgChunk == 32, "one warp compacts a chunk");
+    int total = 0;
+    if (warp < kSgChunk / 32) {
         const int j = j0 + threadIdx.x;
         const int t = j < p.topk ? idx[j] : -1;
-        int slot = -1;
-        if (t >= 0 && t <= last && t / kPage < p.max_pages) {
-            const int page = prow[t / kPage];
-            if (page >= 0 && page < p.num_pages) slot = page * kPage + t % kPage;
-        }
-        if (slot < 0 && t != -1 && j < p.topk) report_error(p.ws, GQLA_ERR_DEVICE, v);
-        // block-wide exclusive count of the valid entries before this one
+        const int slot = j < p.topk ? entry_slot(p, prow, t, last) : -1;
+        if (slot < 0 && t != -1) report_error(p.ws, GQLA_ERR_DEVICE, v);
         const unsigned m = __ballot_sync(0xffffffffu, slot >= 0);
         if (lane == 0) s_warp[warp] = __popc(m);
-        __syncthreads();
-        int before = 0, total = 0;
-#pragma unroll
-        for (int w = 0; w < kSgThreads / 32; ++w) {
-            before += w < warp ? s_warp[w] : 0;
-            total += s_warp[w];
-        }
+        const int k = __popc(m & ((1u << lane) - 1u));
         if (slot >= 0) {
-            const int k = before + __popc(m & ((1u << lane) - 1u));
             s_slot[k] = slot;
-            s_dst[k] = v * p.cap + count + k;
+            s_dst[k] = v * p.cap + before + k;
         }
-        __syncthreads();
-        // copy the chunk's `total` rows: every group's 512-byte [K_nope | V] row, then k^R
-        for (int e = threadIdx.x; e < total * chunks16; e += kSgThreads) {
-            const int k = e / chunks16, part = e % chunks16;
-            const int64_t src = s_slot[k], dst = s_dst[k];
-            if (part < p.num_groups * 32) {
-                const int g = part >> 5, c = part & 31;
-                reinterpret_cast<uint4 *>(p.kv_sel + ((int64_t)g * p.sel_slots + dst) * kKv)[c] =
-                    reinterpret_cast<const uint4 *>(p.kv + ((int64_t)g * p.num_slots + src) * kKv)[c];
-            } else {
-                const int c = part - p.num_groups * 32;
-                reinterpret_cast<uint4 *>(p.k_rope_sel + dst * kRope)[c] =
-                    reinterpret_cast<const uint4 *>(p.k_rope + src * kRope)[c];
-            }
-        }
-        count += total;
-        __syncthreads();  // s_slot / s_dst / s_warp are rewritten by the next chunk
     }
-    const int pages = p.cap / kPage;
-    for (int i = threadIdx.x; i < pages; i += kSgThreads) p.sel_page_table[(int64_t)v * pages + i] = v * pages + i;
-    if (threadIdx.x == 0) p.sel_seqlens[v] = count;
+    __syncthreads();
+    total = s_warp[0];
+    // copy the chunk's rows: every group's 512-byte [K_nope | V] row, then k^R;
+    // consecutive threads take consecutive 16-byte chunks of a row
+    const int chunks16 = p.num_groups * 32 + 8;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < total * chunks16; e += kSgThreads) {
+        const int k = e / chunks16, part = e % chunks16;
+        const int64_t src = s_slot[k], dst = s_dst[k];
+        if (part < p.num_groups * 32) {
+            const int g = part >> 5, c = part & 31;
+            reinterpret_cast<uint4 *>(p.kv_sel + ((int64_t)g * p.sel_slots + dst) * kKv)[c] =
+                reinterpret_cast<const uint4 *>(p.kv + ((int64_t)g * p.num_slots + src) * kKv)[c];
+        } else {
+            const int c = part - p.num_groups * 32;
+            reinterpret_cast<uint4 *>(p.k_rope_sel + dst * kRope)[c] =
+                reinterpret_cast<const uint4 *>(p.k_rope + src * kRope)[c];
+        }
+    }
+    if (j0 + kSgChunk >= p.topk && threadIdx.x == 0) p.sel_seqlens[v] = before + total;
+    if (blockIdx.x == 0) {
+        const int pages = p.cap / kPage;
+        for (int i = threadIdx.x; i < pages; i += kSgThreads)
+            p.sel_page_table[(int64_t)v * pages + i] = v * pages + i;
+    }
 }
 
 }  // namespace
@@ -127,7 +143,8 @@ cudaError_t launch_sparse_gather(const void *kv, const void *k_rope, int64_t num
     p.max_pages = idx->max_pages_per_seq;
     p.num_pages = idx->num_pages;
     p.num_groups = num_groups;
-    sparse_gather_kernel<<<virt, kSgThreads, 0, stream>>>(p);
+    sparse_gather_kernel<<<dim3((unsigned)((topk + kSgChunk - 1) / kSgChunk), (unsigned)virt), kSgThreads, 0,
+                           stream>>>(p);
     return cudaGetLastError();
 }
 
