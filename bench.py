@@ -540,71 +540,85 @@ def run_ours(args, rank, world, local_rank):
 
 def run_sparse(args, dims, case, s_q, kvx, kr, kv, flush_l2, hbm_peak):
     """Sparse GQLA on the GQA path: every query token attends to --sparse-topk
-    seeded positions of its visible context; gather + GQA decode + combine,
-    timed like the step (one graph, L2 flushed before each replay) and per call."""
+    seeded positions of its visible context.  Two forms, each timed like the step
+    (one graph, L2 flushed before each replay) and per call: the selected cache
+    (gather the rows, GQA decode over them, combine) and the fused one (slot lists,
+    the GQA decode gathering the rows itself with tile::gather4, combine)."""
     from decode_attention_06_b200 import gqla, synth
     B = case["seqlens"].numel()
     topk = args.sparse_topk
     idx = synth.make_topk(case["seqlens"].cpu(), s_q, topk, seed=77).to(case["q"].device)
     splits = args.splits or gqla.gqla_num_splits_hint("gqa", dims.num_heads, 1)
-    sb = gqla.SparseBuffers(dims, B, s_q, topk, splits, device=case["q"].device)
-    q1 = case["q"].view(B * s_q, 1, dims.num_heads, 192)
-    calls = [
-        lambda: gqla.gqla_sparse_gather(dims, kvx, kr, kv, s_q, idx, sb.kv_sel, sb.k_rope_sel,
-                                        sb.sel_page_table, sb.sel_seqlens, sb.workspace),
-        lambda: gqla.gqla_decode_gqa(dims, q1, sb.kv_sel, sb.k_rope_sel, sb.sel_index, splits,
-                                     sb.dec.o_part, sb.dec.lse_part, sb.workspace),
-        lambda: gqla.gqla_combine(dims, sb.sel_index, 1, splits, 128, sb.dec.o_part, sb.dec.lse_part,
-                                  None, sb.dec.out, sb.dec.lse),
-    ]
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
-
-    def step(events=None):
-        for i, c in enumerate(calls):
-            if events is not None:
-                events[i].record()
-            c()
-        if events is not None:
-            events[-1].record()
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    graphs = []
-    for events in (None, ev):
-        g_ = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_):
-            step(events)
-        graphs.append(g_)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_step, t_call = [], [[] for _ in calls]
-    for _ in range(args.steps):
-        flush_l2()
-        e0.record()
-        graphs[0].replay()
-        e1.record()
-        torch.cuda.synchronize()
-        t_step.append(e0.elapsed_time(e1))
-        flush_l2()
-        graphs[1].replay()
-        torch.cuda.synchronize()
-        for i in range(len(calls)):
-            t_call[i].append(ev[i].elapsed_time(ev[i + 1]))
-    st, _ = gqla.gqla_read_device_error(sb.workspace)
-    if st:
-        raise RuntimeError(f"device-side error in the sparse step: {st}")
-    n_sel = int(sb.sel_seqlens.sum())
+    n_slots = kv.num_pages * kv.page_size
     tok_bytes = 2 * (2 * dims.num_groups * 128 + 64)
     q_bytes = B * s_q * dims.num_heads * 192 * 2
-    ms = sum(t_step) / len(t_step)
-    us = {n: 1e3 * sum(v) / len(v) for n, v in zip(["gather", "decode_gqa", "combine"], t_call)}
-    # one pass over the selected rows, the queries and the output: what a fused kernel would move
-    fused_bytes = n_sel * tok_bytes + q_bytes + B * s_q * dims.num_heads * 128 * 2
-    return {"topk": topk, "selected_tokens": n_sel, "us_per_step": ms * 1e3,
-            "tokens_per_s": B * s_q / (ms * 1e-3), "per_call_us": us,
-            "gather_gbs": 2 * n_sel * tok_bytes / (us["gather"] * 1e-6) / 1e9,
-            "fused_bytes": fused_bytes,
-            "hbm_frac_of_fused": fused_bytes / (ms * 1e-3) / 1e9 / hbm_peak,
+
+    def measure(fused):
+        sb = gqla.SparseBuffers(dims, B, s_q, topk, splits, device=case["q"].device, fused=fused)
+        if fused:
+            names = ["select", "decode_gqa_sparse", "combine"]
+            calls = [
+                lambda: gqla.gqla_sparse_select(dims, kv, s_q, idx, sb.sel_slot, sb.sel_page_table,
+                                                sb.sel_seqlens, sb.workspace),
+                lambda: gqla.gqla_decode_gqa_sparse(dims, case["q"], kvx, kr, n_slots, sb.sel_index, sb.sel_slot,
+                                                    splits, sb.dec.o_part, sb.dec.lse_part, sb.workspace)]
+        else:
+            names = ["gather", "decode_gqa", "combine"]
+            q1 = case["q"].view(B * s_q, 1, dims.num_heads, 192)
+            calls = [
+                lambda: gqla.gqla_sparse_gather(dims, kvx, kr, kv, s_q, idx, sb.kv_sel, sb.k_rope_sel,
+                                                sb.sel_page_table, sb.sel_seqlens, sb.workspace),
+                lambda: gqla.gqla_decode_gqa(dims, q1, sb.kv_sel, sb.k_rope_sel, sb.sel_index, splits,
+                                             sb.dec.o_part, sb.dec.lse_part, sb.workspace)]
+        calls.append(lambda: gqla.gqla_combine(dims, sb.sel_index, 1, splits, 128, sb.dec.o_part,
+                                               sb.dec.lse_part, None, sb.dec.out, sb.dec.lse))
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+
+        def step(events=None):
+            for i, c in enumerate(calls):
+                if events is not None:
+                    events[i].record()
+                c()
+            if events is not None:
+                events[-1].record()
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        graphs = []
+        for events in (None, ev):
+            g_ = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_):
+                step(events)
+            graphs.append(g_)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_step, t_call = [], [[] for _ in calls]
+        for _ in range(args.steps):
+            flush_l2()
+            e0.record()
+            graphs[0].replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t_step.append(e0.elapsed_time(e1))
+            flush_l2()
+            graphs[1].replay()
+            torch.cuda.synchronize()
+            for i in range(len(calls)):
+                t_call[i].append(ev[i].elapsed_time(ev[i + 1]))
+        st, _ = gqla.gqla_read_device_error(sb.workspace)
+        if st:
+            raise RuntimeError(f"device-side error in the sparse step: {st}")
+        n_sel = int(sb.sel_seqlens.sum())
+        ms = sum(t_step) / len(t_step)
+        us = {n: 1e3 * sum(v) / len(v) for n, v in zip(names, t_call)}
+        # one pass over the selected rows, the queries and the output: what a single
+        # kernel would have to move at least
+        fused_bytes = n_sel * tok_bytes + q_bytes + B * s_q * dims.num_heads * 128 * 2
+        return {"us_per_step": ms * 1e3, "tokens_per_s": B * s_q / (ms * 1e-3), "per_call_us": us,
+                "selected_tokens": n_sel, "min_bytes": fused_bytes,
+                "hbm_frac_of_min_bytes": fused_bytes / (ms * 1e-3) / 1e9 / hbm_peak}
+
+    return {"topk": topk, "selected_cache": measure(False), "fused": measure(True),
             "selection": "seeded uniform distinct visible positions (synth.make_topk)"}
 
 

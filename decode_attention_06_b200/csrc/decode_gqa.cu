@@ -86,6 +86,11 @@ struct GqaParams {
     int batch, max_pages, num_pages, num_splits, s_q, heads, G;
     int NG;  // KV groups g: 8, or 4 (the (g, s_q) = (4, 1) configuration's 2176-byte tokens)
     float scale_log2;
+    // sparse mode: the "pages" are those of a selection (identity page table, lengths =
+    // selected rows per query token); row r of selected page P is cache slot sel_slot[64 P + r]
+    // (-1: none), gathered from a cache of real_slots slots
+    const int32_t *sel_slot;
+    int real_slots;
 };
 
 // Iterates the pieces (sequence b, pages [pb, pe)) of chunk `c`; identical in every role.
@@ -257,11 +262,13 @@ __device__ __forceinline__ void write_p(const uint32_t (&sv)[NQ], const float (&
     }
 }
 
-template <int NQ>
+template <int NQ, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap kv_map,
                          const __grid_constant__ CUtensorMap kr_map,
-                         const __grid_constant__ CUtensorMap q_map, const GqaParams p) {
+                         const __grid_constant__ CUtensorMap q_map,
+                         const __grid_constant__ CUtensorMap kv_rows_map,
+                         const __grid_constant__ CUtensorMap kr_rows_map, const GqaParams p) {
     using SM = GqaSmem<NQ>;
     constexpr int KS = SM::kKSlots, VS = SM::kVSlots;
     extern __shared__ uint8_t smem_raw[];
@@ -333,7 +340,130 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sm_kr = smem_u32(smem + SM::oKr);
     const uint32_t sm_p = smem_u32(smem + SM::oP);
 
-    if (warp == 0) {
+    if (warp == 0 && SPARSE) {
+        // ---------------------------------------------------------------- TMA producer, sparse
+        // The same units and rings as below; the rows of a unit are gathered four at a
+        // time (tile::gather4): lane l takes rows 4 (l % 16) .. + 3 of page l / 16 of the
+        // unit's pair, for K_nope_g, V_g and the pair's RoPE keys.  Lane 0 waits for
+        // the slots and sets each barrier's byte count before the warp issues.
+        if (lane == 0) {
+            prefetch_tensormap(&kv_rows_map);
+            prefetch_tensormap(&kr_rows_map);
+            prefetch_tensormap(&q_map);
+        }
+        const uint32_t q_bytes = 3u * 128u * (uint32_t)real_cols;
+        const uint64_t stream_policy = l2_evict_first_policy();
+        const int half = lane >> 4, r0 = 4 * (lane & 15);
+        UnitCursor kc, vc;
+        kc.start(p, it0);
+        vc.start(p, it0);
+        uint32_t kpos = 0, vpos = 0, pc = 0;
+        int4 ksl = make_int4(-1, -1, -1, -1), vsl = ksl;  // this lane's four cache slots
+        auto pair_slots = [&](const UnitCursor &cur) {
+            const int page = half ? cur.pp.page1 : cur.pp.page0;
+            return page < 0 ? make_int4(-1, -1, -1, -1)
+                            : *reinterpret_cast<const int4 *>(p.sel_slot + (int64_t)page * kPage + r0);
+        };
+        auto row_of = [&](int slot, int gi) { return slot < 0 ? -1 : gi * p.real_slots + slot; };
+        long long idle_since = clock64();
+        while (kc.valid || vc.valid) {  // warp-uniform: every decision is lane 0's, broadcast
+            bool progressed = false;
+            const int aborted = __shfl_sync(0xffffffffu, (int)*abort_flag, 0);
+            if (kc.valid && !aborted) {
+                const int ks = kpos % KS, kb = pc & 1;
+                const bool need_kr = kc.gi == 0;
+                int ready = 0;
+                if (lane == 0)
+                    ready = (!need_kr || mbar_test_wait(&kr_empty[kb], ((pc >> 1) & 1) ^ 1)) &&
+                            mbar_test_wait(&k_empty[ks], ((kpos / KS) & 1) ^ 1);
+                if (__shfl_sync(0xffffffffu, ready, 0)) {
+                    if (need_kr) ksl = pair_slots(kc);  // the first unit of a pair
+                    const PagePair &pp = kc.pp;
+                    const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                    const bool mine = half ? pp.page1 >= 0 : pp.page0 >= 0;
+                    if (need_kr) {
+                        uint8_t *dst = smem + SM::oKr + kb * SM::kKrBytes;
+                        if (lane == 0) {
+                            if (np) mbar_arrive_expect_tx(&kr_full[kb], np * kBox);
+                            else mbar_arrive(&kr_full[kb]);
+                        }
+                        __syncwarp();
+                        if (mine)
+                            tma_gather4_hint(dst + half * kBox + r0 * 128, &kr_rows_map, &kr_full[kb], 0,
+                                             ksl.x, ksl.y, ksl.z, ksl.w, stream_policy);
+                        ++pc;
+                    }
+                    uint8_t *dst = smem + SM::oK + ks * SM::kKSlotBytes;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
+#pragma unroll
+                        for (int cb = 0; cb < 3; ++cb)  // q_g rows of this query token
+                            tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
+                                        kc.gi * p.G, kc.b * p.s_q);
+                    }
+                    __syncwarp();
+                    if (mine) {
+#pragma unroll
+                        for (int cb = 0; cb < 2; ++cb)  // K_nope lo / hi
+                            tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &k_full[ks],
+                                             cb * 64, row_of(ksl.x, kc.gi), row_of(ksl.y, kc.gi),
+                                             row_of(ksl.z, kc.gi), row_of(ksl.w, kc.gi), stream_policy);
+                    }
+                    kc.advance(p);
+                    ++kpos;
+                    progressed = true;
+                }
+            }
+            if (vc.valid && vpos < kpos && !aborted) {
+                const int vs = vpos % VS;
+                int ready = 0;
+                if (lane == 0) ready = mbar_test_wait(&v_empty[vs], ((vpos / VS) & 1) ^ 1);
+                if (__shfl_sync(0xffffffffu, ready, 0)) {
+                    if (vc.gi == 0) vsl = pair_slots(vc);
+                    const PagePair &pp = vc.pp;
+                    const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                    const bool mine = half ? pp.page1 >= 0 : pp.page0 >= 0;
+                    uint8_t *dst = smem + SM::oV + vs * SM::kVBytes;
+                    if (lane == 0) {
+                        if (np) mbar_arrive_expect_tx(&v_full[vs], np * 2 * kBox);
+                        else mbar_arrive(&v_full[vs]);
+                    }
+                    __syncwarp();
+                    if (mine) {
+#pragma unroll
+                        for (int cb = 0; cb < 2; ++cb)  // V lo / hi
+                            tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &v_full[vs],
+                                             128 + cb * 64, row_of(vsl.x, vc.gi), row_of(vsl.y, vc.gi),
+                                             row_of(vsl.z, vc.gi), row_of(vsl.w, vc.gi), stream_policy);
+                    }
+                    vc.advance(p);
+                    ++vpos;
+                    progressed = true;
+                }
+            }
+            int give_up = 0;
+            if (lane == 0 && !progressed) give_up = aborted || clock64() - idle_since > kWaitCycles;
+            if (progressed) {
+                idle_since = clock64();
+            } else if (!__shfl_sync(0xffffffffu, give_up, 0)) {
+                __nanosleep(20);
+            } else {
+                if (lane == 0) *abort_flag = 1;  // give up: the consumers stop waiting on us as well
+                break;
+            }
+        }
+        // never leave with copies in flight: wait (bounded) for the last loads issued
+        if (lane == 0) {
+            int dummy = 0;
+            volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
+            for (uint32_t u = (kpos > (uint32_t)KS ? kpos - KS : 0); u < kpos; ++u)
+                mbar_wait(&k_full[u % KS], (u / KS) & 1, no_abort);
+            for (uint32_t u = (vpos > (uint32_t)VS ? vpos - VS : 0); u < vpos; ++u)
+                mbar_wait(&v_full[u % VS], (u / VS) & 1, no_abort);
+            for (uint32_t u = (pc > 2u ? pc - 2 : 0); u < pc; ++u)
+                mbar_wait(&kr_full[u & 1], (u >> 1) & 1, no_abort);
+        }
+    } else if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             prefetch_tensormap(&kv_map);
@@ -773,15 +903,22 @@ bool make_map(CUtensorMap *map, const void *base, int rank, const cuuint64_t *di
     return r == CUDA_SUCCESS;
 }
 
+template <int NQ, bool SPARSE>
+cudaError_t launch_nq_mode(const CUtensorMap &kvm, const CUtensorMap &krm, const CUtensorMap &qm,
+                           const CUtensorMap &kvrm, const CUtensorMap &krrm, const GqaParams &p,
+                           cudaStream_t stream) {
+    const int bytes = GqaSmem<NQ>::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(decode_gqa_tc_kernel<NQ, SPARSE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    return launch_dependent(decode_gqa_tc_kernel<NQ, SPARSE>, dim3(p.num_splits), dim3(kThreads), bytes,
+                            stream, kvm, krm, qm, kvrm, krrm, p);
+}
+
 template <int NQ>
 cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const CUtensorMap &qm,
                       const GqaParams &p, cudaStream_t stream) {
-    const int bytes = GqaSmem<NQ>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(decode_gqa_tc_kernel<NQ>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    return launch_dependent(decode_gqa_tc_kernel<NQ>, dim3(p.num_splits), dim3(kThreads), bytes, stream,
-                            kvm, krm, qm, p);
+    return launch_nq_mode<NQ, false>(kvm, krm, qm, kvm, krm, p, stream);  // no row maps in dense mode
 }
 
 }  // namespace
@@ -826,8 +963,59 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
     p.G = G;
     p.NG = num_groups;
     p.scale_log2 = scale * kLog2e;
+    p.sel_slot = nullptr;
+    p.real_slots = 0;
     return G * s_q <= 16 ? launch_nq<16>(kvm, krm, qm, p, stream)
                          : launch_nq<32>(kvm, krm, qm, p, stream);
+}
+
+// Sparse GQLA: the decode over a selection (sel: batch * s_q one-token sequences over
+// an identity page table), gathering each selected row straight from the cache.
+cudaError_t launch_decode_gqa_sparse(const void *q, int heads, int num_groups, const void *kv,
+                                     const void *k_rope, int64_t real_slots, const gqla_kv_index *sel,
+                                     const int32_t *sel_slot, int num_splits, float scale, float *o_part,
+                                     float *lse_part, void *ws, cudaStream_t stream) {
+    if (num_groups != 8 && num_groups != 4) return cudaErrorInvalidValue;
+    const int G = heads / num_groups;
+    CUtensorMap kvr, krr, qm;
+    {  // [g * real_slots][256]: one-row boxes for tile::gather4
+        cuuint64_t dims[2] = {256, (cuuint64_t)num_groups * real_slots};
+        cuuint64_t strides[1] = {256 * 2};
+        cuuint32_t box[2] = {64, 1};
+        if (!make_map(&kvr, kv, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[2] = {64, (cuuint64_t)real_slots};
+        cuuint64_t strides[1] = {64 * 2};
+        cuuint32_t box[2] = {64, 1};
+        if (!make_map(&krr, k_rope, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {  // q [batch * s_q][heads][192]: one query token per selected sequence
+        cuuint64_t dims[3] = {(cuuint64_t)kQk, (cuuint64_t)heads, (cuuint64_t)sel->batch};
+        cuuint64_t strides[2] = {(cuuint64_t)kQk * 2, (cuuint64_t)heads * kQk * 2};
+        cuuint32_t box[3] = {64, (cuuint32_t)G, 1};
+        if (!make_map(&qm, q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    GqaParams p;
+    p.page_table = sel->page_table;
+    p.seqlens = sel->seqlens;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.ws = ws;
+    p.batch = sel->batch;
+    p.max_pages = sel->max_pages_per_seq;
+    p.num_pages = sel->num_pages;
+    p.num_splits = num_splits;
+    p.s_q = 1;
+    p.heads = heads;
+    p.G = G;
+    p.NG = num_groups;
+    p.scale_log2 = scale * kLog2e;
+    p.sel_slot = sel_slot;
+    p.real_slots = (int)real_slots;
+    // the dense tile maps are not used in sparse mode: the row maps stand in for them
+    return G <= 16 ? launch_nq_mode<16, true>(kvr, krr, qm, kvr, krr, p, stream)
+                   : launch_nq_mode<32, true>(kvr, krr, qm, kvr, krr, p, stream);
 }
 
 }  // namespace gqla

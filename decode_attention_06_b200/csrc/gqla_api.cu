@@ -14,7 +14,11 @@ cudaError_t launch_expand_tc(const void *latent, int64_t num_slots, const void *
 cudaError_t launch_sparse_gather(const void *kv, const void *k_rope, int64_t num_slots,
                                  const gqla_kv_index *idx, int s_q, const int32_t *topk_idx, int topk,
                                  int num_groups, void *kv_sel, void *k_rope_sel, int32_t *sel_page_table,
-                                 int32_t *sel_seqlens, void *ws, cudaStream_t stream);
+                                 int32_t *sel_seqlens, int32_t *sel_slot, void *ws, cudaStream_t stream);
+cudaError_t launch_decode_gqa_sparse(const void *q, int heads, int num_groups, const void *kv,
+                                     const void *k_rope, int64_t real_slots, const gqla_kv_index *sel,
+                                     const int32_t *sel_slot, int num_splits, float scale, float *o_part,
+                                     float *lse_part, void *ws, cudaStream_t stream);
 cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_groups,
                                 const void *w_uk, void *qa, cudaStream_t stream);
 cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups, const void *kv,
@@ -232,7 +236,48 @@ int gqla_sparse_gather(const gqla_dims *dims, const void *kv_expanded, const voi
     if ((int64_t)kv->batch * s_q * cap > ((int64_t)1 << 31) - 1) return GQLA_ERR_UNSUPPORTED;
     return cuda_status(launch_sparse_gather(kv_expanded, k_rope, num_slots, kv, s_q, topk_idx, topk,
                                             dims->num_groups, kv_sel, k_rope_sel, sel_page_table,
-                                            sel_seqlens, workspace, reinterpret_cast<cudaStream_t>(stream)));
+                                            sel_seqlens, nullptr, workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_sparse_select(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, const int32_t *topk_idx,
+                       int topk, int32_t *sel_slot, int32_t *sel_page_table, int32_t *sel_seqlens,
+                       void *workspace, size_t workspace_bytes, gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if ((st = check_index(kv)) != GQLA_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes)) != GQLA_OK) return st;
+    if (topk <= 0 || topk > 65536) return GQLA_ERR_INVALID_ARG;
+    if (!topk_idx || !sel_slot || !sel_page_table || !sel_seqlens || !aligned16(sel_slot))
+        return GQLA_ERR_INVALID_ARG;
+    if ((int64_t)kv->batch * s_q > 65535) return GQLA_ERR_UNSUPPORTED;
+    const int64_t cap = (topk + 63) / 64 * 64;
+    if ((int64_t)kv->batch * s_q * cap > ((int64_t)1 << 31) - 1) return GQLA_ERR_UNSUPPORTED;
+    return cuda_status(launch_sparse_gather(nullptr, nullptr, 0, kv, s_q, topk_idx, topk, dims->num_groups,
+                                            nullptr, nullptr, sel_page_table, sel_seqlens, sel_slot, workspace,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_decode_gqa_sparse(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
+                           const void *k_rope, int64_t num_slots, const gqla_kv_index *sel,
+                           const int32_t *sel_slot, int num_splits, float *o_part, float *lse_part,
+                           void *workspace, size_t workspace_bytes, gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if ((st = check_index(sel)) != GQLA_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes)) != GQLA_OK) return st;
+    if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
+    if (!q || !kv_expanded || !k_rope || !sel_slot || !o_part || !lse_part) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv_expanded) || !aligned16(k_rope) || !aligned16(o_part) ||
+        !aligned16(sel_slot))
+        return GQLA_ERR_INVALID_ARG;
+    if (sel->page_size != 64 || sel->batch % s_q != 0) return GQLA_ERR_INVALID_ARG;
+    if (num_slots <= 0 || (int64_t)dims->num_groups * num_slots > ((int64_t)1 << 31) - 1)
+        return GQLA_ERR_UNSUPPORTED;
+    if (dims->num_groups != 8 && dims->num_groups != 4) return GQLA_ERR_UNSUPPORTED;
+    return cuda_status(launch_decode_gqa_sparse(q, dims->num_heads, dims->num_groups, kv_expanded, k_rope,
+                                                num_slots, sel, sel_slot, num_splits, dims->softmax_scale,
+                                                o_part, lse_part, workspace,
+                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,

@@ -161,6 +161,20 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Four rows (y0..y3) of a 2D tensor, `x` the first column of a one-row box,
+// into four consecutive box rows at `dst` (the map's swizzle applies as for a
+// four-row box); completes their bytes on `bar`.  Rows outside the tensor
+// read as zeros.
+__device__ __forceinline__ void tma_gather4_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int x,
+                                                 int y0, int y1, int y2, int y3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
+        "r"(y3), "l"(policy)
+        : "memory");
+}
+
 // L2 policy for data read once per launch (a KV cache stream): its lines are the
 // first to go, so that what is reused (queries, partials, weights) stays in L2.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {

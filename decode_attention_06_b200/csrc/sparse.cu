@@ -13,7 +13,11 @@
 // (every selected token is visible to its query), and the usual combine
 // merges the splits.
 //
-// One CTA per 64 entries of a list: it counts the valid entries before its
+// With a slot list instead of a selected cache (the fused path), only each
+// selected row's cache slot is written, and the GQA decode gathers the rows
+// itself.
+//
+// One CTA per 32 entries of a list: it counts the valid entries before its
 // own (-1 marks an unused entry; any other position outside [0, L_b - s_q + s]
 // or on a page outside the pool is a device error and is skipped), compacts
 // its entries with a warp ballot, and copies their rows with consecutive
@@ -37,6 +41,7 @@ struct SgParams {
     __nv_bfloat16 *k_rope_sel;    // [sel_slots][64]
     int32_t *sel_page_table;      // [batch * s_q][cap / 64]
     int32_t *sel_seqlens;         // [batch * s_q]
+    int32_t *sel_slot;            // [batch * s_q * cap]: the cache slot of each selected row, or null
     void *ws;
     int64_t num_slots, sel_slots;
     int s_q, topk, cap, max_pages, num_pages, num_groups;
@@ -52,6 +57,9 @@ __device__ __forceinline__ int entry_slot(const SgParams &p, const int32_t *prow
 // grid (entries / kSgChunk, batch * s_q): CTA (c, v) compacts entries
 // [c * kSgChunk, (c + 1) * kSgChunk) of list v, after counting the valid entries
 // before them.
+// With COPY the rows themselves go to the selected cache; without, only their
+// cache slots go to sel_slot (the rows past a list's valid entries get -1).
+template <bool COPY>
 __global__ void __launch_bounds__(kSgThreads) sparse_gather_kernel(const SgParams p) {
     __shared__ int s_warp[kSgThreads / 32];
     __shared__ int s_slot[kSgChunk];
@@ -92,11 +100,16 @@ __global__ void __launch_bounds__(kSgThreads) sparse_gather_kernel(const SgParam
     }
     __syncthreads();
     total = s_warp[0];
+    if constexpr (!COPY) {
+        if (threadIdx.x < total) p.sel_slot[s_dst[threadIdx.x]] = s_slot[threadIdx.x];
+        if (j0 + kSgChunk >= p.topk)  // the list's last chunk: rows past its valid entries
+            for (int i = before + total + threadIdx.x; i < p.cap; i += kSgThreads) p.sel_slot[(int64_t)v * p.cap + i] = -1;
+    }
     // copy the chunk's rows: every group's 512-byte [K_nope | V] row, then k^R;
     // consecutive threads take consecutive 16-byte chunks of a row
     const int chunks16 = p.num_groups * 32 + 8;
 #pragma unroll 4
-    for (int e = threadIdx.x; e < total * chunks16; e += kSgThreads) {
+    for (int e = threadIdx.x; e < (COPY ? total * chunks16 : 0); e += kSgThreads) {
         const int k = e / chunks16, part = e % chunks16;
         const int64_t src = s_slot[k], dst = s_dst[k];
         if (part < p.num_groups * 32) {
@@ -122,7 +135,7 @@ __global__ void __launch_bounds__(kSgThreads) sparse_gather_kernel(const SgParam
 cudaError_t launch_sparse_gather(const void *kv, const void *k_rope, int64_t num_slots,
                                  const gqla_kv_index *idx, int s_q, const int32_t *topk_idx, int topk,
                                  int num_groups, void *kv_sel, void *k_rope_sel, int32_t *sel_page_table,
-                                 int32_t *sel_seqlens, void *ws, cudaStream_t stream) {
+                                 int32_t *sel_seqlens, int32_t *sel_slot, void *ws, cudaStream_t stream) {
     const int virt = idx->batch * s_q;
     SgParams p;
     p.kv = static_cast<const __nv_bfloat16 *>(kv);
@@ -134,6 +147,7 @@ cudaError_t launch_sparse_gather(const void *kv, const void *k_rope, int64_t num
     p.k_rope_sel = static_cast<__nv_bfloat16 *>(k_rope_sel);
     p.sel_page_table = sel_page_table;
     p.sel_seqlens = sel_seqlens;
+    p.sel_slot = sel_slot;
     p.ws = ws;
     p.num_slots = num_slots;
     p.s_q = s_q;
@@ -143,8 +157,11 @@ cudaError_t launch_sparse_gather(const void *kv, const void *k_rope, int64_t num
     p.max_pages = idx->max_pages_per_seq;
     p.num_pages = idx->num_pages;
     p.num_groups = num_groups;
-    sparse_gather_kernel<<<dim3((unsigned)((topk + kSgChunk - 1) / kSgChunk), (unsigned)virt), kSgThreads, 0,
-                           stream>>>(p);
+    const dim3 grid((unsigned)((topk + kSgChunk - 1) / kSgChunk), (unsigned)virt);
+    if (sel_slot)
+        sparse_gather_kernel<false><<<grid, kSgThreads, 0, stream>>>(p);
+    else
+        sparse_gather_kernel<true><<<grid, kSgThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -64,6 +64,8 @@ _SIGS = {
     "gqla_decode_gqa": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_combine": [_DP, _KP, _I, _I, _I, _P, _P, _P, _P, _P, _P],
     "gqla_sparse_gather": [_DP, _P, _P, _I64, _KP, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
+    "gqla_sparse_select": [_DP, _KP, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
+    "gqla_decode_gqa_sparse": [_DP, _P, _I, _P, _P, _I64, _KP, _P, _I, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa_noalloc": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _P],
     "gqla_partial_slots": [_I, _I],
     "gqla_workspace_bytes": [],
@@ -214,6 +216,33 @@ def gqla_sparse_gather(dims, kv_expanded, k_rope, kv, s_q, topk_idx, kv_sel, k_r
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream)))
 
 
+def gqla_sparse_select(dims, kv, s_q, topk_idx, sel_slot, sel_page_table, sel_seqlens, workspace,
+                       stream=None):
+    B = kv.batch
+    topk = topk_idx.shape[-1]
+    cap = (topk + PAGE_SIZE - 1) // PAGE_SIZE * PAGE_SIZE
+    _check("gqla_sparse_select", _lib.gqla_sparse_select(
+        ctypes.byref(dims), ctypes.byref(kv), s_q, _dev(topk_idx, "topk_idx", torch.int32, (B, s_q, topk)), topk,
+        _dev(sel_slot, "sel_slot", torch.int32, (B * s_q * cap,)),
+        _dev(sel_page_table, "sel_page_table", torch.int32, (B * s_q, cap // PAGE_SIZE)),
+        _dev(sel_seqlens, "sel_seqlens", torch.int32, (B * s_q,)),
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream)))
+
+
+def gqla_decode_gqa_sparse(dims, q, kv_expanded, k_rope, num_slots, sel, sel_slot, num_splits, o_part,
+                           lse_part, workspace, stream=None):
+    B, s_q, h, _ = q.shape
+    slots = gqla_partial_slots(sel.batch, num_splits)
+    _check("gqla_decode_gqa_sparse", _lib.gqla_decode_gqa_sparse(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16, (sel.batch // s_q, s_q, dims.num_heads, D_QK)), s_q,
+        _dev(kv_expanded, "kv_expanded", torch.bfloat16, (dims.num_groups, num_slots, D_NOPE + D_V)),
+        _dev(k_rope, "k_rope", torch.bfloat16, (num_slots, D_ROPE)), num_slots, ctypes.byref(sel),
+        _dev(sel_slot, "sel_slot", torch.int32), num_splits,
+        _dev(o_part, "o_part", torch.float32, (slots, 1, h, D_V)),
+        _dev(lse_part, "lse_part", torch.float32, (slots, 1, h)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def gqla_decode_gqa_noalloc(dims, q, kv_expanded, k_rope, kv, num_splits, out, lse_out=None,
                             device_error=None, stream=None):
     """GQA decode step with library-owned static scratch (no o_part/lse_part/workspace)."""
@@ -294,16 +323,23 @@ class DecodeBuffers:
 
 
 class SparseBuffers:
-    """Device buffers of one sparse GQA step: the selected cache, its index and
-    the decode buffers of the batch * s_q selected sequences."""
+    """Device buffers of one sparse GQA step: the selection (its slot list for the
+    fused path, or a selected cache), its index, and the decode buffers of the
+    batch * s_q selected sequences."""
 
-    def __init__(self, dims, batch: int, s_q: int, topk: int, num_splits: int, device="cuda"):
-        self.s_q, self.topk = s_q, topk
+    def __init__(self, dims, batch: int, s_q: int, topk: int, num_splits: int, device="cuda",
+                 fused: bool = False):
+        self.s_q, self.topk, self.fused = s_q, topk, fused
         self.cap = (topk + PAGE_SIZE - 1) // PAGE_SIZE * PAGE_SIZE
         v = batch * s_q
-        self.kv_sel = torch.empty(dims.num_groups, v * self.cap, D_NOPE + D_V, dtype=torch.bfloat16,
-                                  device=device)
-        self.k_rope_sel = torch.empty(v * self.cap, D_ROPE, dtype=torch.bfloat16, device=device)
+        if fused:
+            self.sel_slot = torch.empty(v * self.cap, dtype=torch.int32, device=device)
+            self.kv_sel = self.k_rope_sel = None
+        else:
+            self.sel_slot = None
+            self.kv_sel = torch.empty(dims.num_groups, v * self.cap, D_NOPE + D_V, dtype=torch.bfloat16,
+                                      device=device)
+            self.k_rope_sel = torch.empty(v * self.cap, D_ROPE, dtype=torch.bfloat16, device=device)
         self.sel_page_table = torch.empty(v, self.cap // PAGE_SIZE, dtype=torch.int32, device=device)
         self.sel_seqlens = torch.empty(v, dtype=torch.int32, device=device)
         self.sel_index = make_kv_index(self.sel_page_table, self.sel_seqlens, v * self.cap // PAGE_SIZE)
@@ -312,15 +348,23 @@ class SparseBuffers:
 
 
 def sparse_gqa_step(dims, bufs: SparseBuffers, q, kv_expanded, k_rope, kv, topk_idx, stream=None):
-    """Sparse GQA step through the C ABI: gather the selected tokens, then the
-    GQA decode and combine over batch * s_q one-token queries.  Returns
+    """Sparse GQA step through the C ABI: the selection, then the GQA decode (the
+    fused one gathering the selected rows itself, or the plain one over a selected
+    cache) and the combine over batch * s_q one-token queries.  Returns
     (out [batch][s_q][h][128] bf16, lse [batch][s_q][h])."""
     B, s_q, h, _ = q.shape
-    gqla_sparse_gather(dims, kv_expanded, k_rope, kv, s_q, topk_idx, bufs.kv_sel, bufs.k_rope_sel,
-                       bufs.sel_page_table, bufs.sel_seqlens, bufs.workspace, stream)
-    q1 = q.view(B * s_q, 1, h, D_QK)
-    gqla_decode_gqa(dims, q1, bufs.kv_sel, bufs.k_rope_sel, bufs.sel_index, bufs.dec.num_splits,
-                    bufs.dec.o_part, bufs.dec.lse_part, bufs.workspace, stream)
+    if bufs.fused:
+        gqla_sparse_select(dims, kv, s_q, topk_idx, bufs.sel_slot, bufs.sel_page_table, bufs.sel_seqlens,
+                           bufs.workspace, stream)
+        gqla_decode_gqa_sparse(dims, q, kv_expanded, k_rope, kv.num_pages * kv.page_size, bufs.sel_index,
+                               bufs.sel_slot, bufs.dec.num_splits, bufs.dec.o_part, bufs.dec.lse_part,
+                               bufs.workspace, stream)
+    else:
+        gqla_sparse_gather(dims, kv_expanded, k_rope, kv, s_q, topk_idx, bufs.kv_sel, bufs.k_rope_sel,
+                           bufs.sel_page_table, bufs.sel_seqlens, bufs.workspace, stream)
+        q1 = q.view(B * s_q, 1, h, D_QK)
+        gqla_decode_gqa(dims, q1, bufs.kv_sel, bufs.k_rope_sel, bufs.sel_index, bufs.dec.num_splits,
+                        bufs.dec.o_part, bufs.dec.lse_part, bufs.workspace, stream)
     gqla_combine(dims, bufs.sel_index, 1, bufs.dec.num_splits, D_V, bufs.dec.o_part, bufs.dec.lse_part,
                  None, bufs.dec.out, bufs.dec.lse, stream)
     return bufs.dec.out.view(B, s_q, h, D_V), bufs.dec.lse.view(B, s_q, h)

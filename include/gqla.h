@@ -196,6 +196,37 @@ int gqla_sparse_gather(const gqla_dims *dims, const void *kv_expanded, const voi
                        gqla_stream_t stream);
 
 /*
+ * Sparse GQLA without the selected cache (the fused path): the same selection
+ * as gqla_sparse_gather, but only each selected row's cache slot is written,
+ *   sel_slot      int32 [batch * s_q * cap]  out: cache slot of selected row
+ *                 r of query token v at [v * cap + r]; -1 past the list's
+ *                 valid entries
+ * with sel_page_table / sel_seqlens as there (kv_expanded and k_rope are not
+ * read: pass NULL).  gqla_decode_gqa_sparse then gathers the rows itself.
+ */
+int gqla_sparse_select(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, const int32_t *topk_idx,
+                       int topk, int32_t *sel_slot, int32_t *sel_page_table, int32_t *sel_seqlens,
+                       void *workspace, size_t workspace_bytes, gqla_stream_t stream);
+
+/*
+ * GQA-path decode over a selection written by gqla_sparse_select: the split
+ * partials of batch * s_q one-token queries, each over its own selected rows,
+ * which the kernel gathers from the cache four at a time (TMA tile::gather4)
+ * instead of reading page tiles.
+ *   q            bf16 [batch][s_q][h][192] (as for gqla_decode_gqa)
+ *   kv_expanded, k_rope, num_slots   the cache, as for gqla_decode_gqa
+ *   sel          {sel_page_table, sel_seqlens, batch * s_q, cap / 64, 64,
+ *                 batch * s_q * cap / 64}
+ *   sel_slot     as written by gqla_sparse_select
+ *   o_part, lse_part, workspace   as for gqla_decode_gqa with sel's batch
+ * Then gqla_combine(dims, sel, 1, num_splits, 128, ...).
+ */
+int gqla_decode_gqa_sparse(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
+                           const void *k_rope, int64_t num_slots, const gqla_kv_index *sel,
+                           const int32_t *sel_slot, int num_splits, float *o_part, float *lse_part,
+                           void *workspace, size_t workspace_bytes, gqla_stream_t stream);
+
+/*
  * Log-sum-exp merge of the partials of each sequence, then (absorb path,
  * d_in == 512) the per-group up-projection out = o~ W_UV_{g(h)}: W_UV folded into
  * the output (paperlayer.ai summary, sec. 2).

@@ -235,7 +235,7 @@ SPARSE = [
 ]
 
 
-def _sparse_run(case, idx, splits):
+def _sparse_run(case, idx, splits, fused=True):
     from decode_attention_06_b200 import gqla
     g = to_gpu(case)
     h, ng, s_q = case["num_heads"], case["num_groups"], case["s_q"]
@@ -248,18 +248,19 @@ def _sparse_run(case, idx, splits):
     B = case["seqlens"].numel()
     if splits is None:
         splits = gqla.gqla_num_splits_hint("gqa", h, 1)
-    bufs = gqla.SparseBuffers(dims, B, s_q, idx.shape[-1], splits)
+    bufs = gqla.SparseBuffers(dims, B, s_q, idx.shape[-1], splits, fused=fused)
     out, lse = gqla.sparse_gqa_step(dims, bufs, g["q"], kvx, kr, kv, idx.cuda())
     torch.cuda.synchronize()
     return out.clone(), lse.clone(), bufs
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "selected_cache"])
 @pytest.mark.parametrize("cid,h,g,seqlens,s_q,topk,unused,splits", SPARSE, ids=[c[0] for c in SPARSE])
-def test_sparse_gqa_parity(cid, h, g, seqlens, s_q, topk, unused, splits):
+def test_sparse_gqa_parity(cid, h, g, seqlens, s_q, topk, unused, splits, fused):
     from decode_attention_06_b200 import gqla
     case = synth.make_case(h, g, seqlens, s_q, paged=True, seed=300 + len(cid))
     idx = synth.make_topk(seqlens, s_q, topk, seed=400 + len(cid), unused=unused)
-    out, lse, bufs = _sparse_run(case, idx, splits)
+    out, lse, bufs = _sparse_run(case, idx, splits, fused)
     st, _ = gqla.gqla_read_device_error(bufs.workspace)
     assert st == 0
     ref, ref_lse = oracle.decode_sparse(case["q"], case["latent"], case["page_table"], case["seqlens"],
@@ -270,12 +271,13 @@ def test_sparse_gqa_parity(cid, h, g, seqlens, s_q, topk, unused, splits):
     assert torch.equal(bufs.sel_seqlens.cpu(), counts.to(torch.int32))
 
 
-def test_sparse_invalid_position_is_reported_and_skipped():
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "selected_cache"])
+def test_sparse_invalid_position_is_reported_and_skipped(fused):
     from decode_attention_06_b200 import gqla
     case = synth.make_case(128, 8, [300, 200], 1, paged=True, seed=311)
     idx = synth.make_topk([300, 200], 1, 64, seed=312, unused=2)
     idx[1, 0, 62] = 200   # past the last visible token of sequence 1 (199)
-    out, lse, bufs = _sparse_run(case, idx, None)
+    out, lse, bufs = _sparse_run(case, idx, None, fused)
     st, info = gqla.gqla_read_device_error(bufs.workspace)
     assert st == -5 and info == 1
     idx_ok = idx.clone()
