@@ -124,3 +124,37 @@ def test_other_calls_reject_bad_arguments(lib):
     assert lib.gqla_read_device_error(None, None, None) == -1
     assert lib.gqla_num_splits_hint(7, 128, 1) == -1
     assert lib.gqla_num_splits_hint(0, 0, 1) == -1
+
+
+def test_expand_tc_and_sparse_calls_reject_bad_arguments(lib):
+    """The tensor-core expansion and the sparse entry points validate before any launch."""
+    d, kv = _dims(), _kv()
+    I64 = ctypes.c_int64
+    assert lib.gqla_expand_cache_tc(ctypes.byref(d), None, I64(64), FAKE, FAKE, FAKE, FAKE, None) == -1
+    assert lib.gqla_expand_cache_tc(ctypes.byref(d), FAKE, I64(-1), FAKE, FAKE, FAKE, FAKE, None) == -1
+    assert lib.gqla_expand_cache_tc(ctypes.byref(d), ctypes.c_void_p((1 << 20) + 8), I64(64), FAKE, FAKE,
+                                    FAKE, FAKE, None) == -1
+    slots = I64(16 * 64)
+    ws, wsb = FAKE, ctypes.c_size_t(256)
+    # gather: topk out of range, null output, workspace too small, 2 groups unsupported
+    assert lib.gqla_sparse_gather(ctypes.byref(d), FAKE, FAKE, slots, ctypes.byref(kv), 1, FAKE, 0,
+                                  FAKE, FAKE, FAKE, FAKE, ws, wsb, None) == -1
+    assert lib.gqla_sparse_gather(ctypes.byref(d), FAKE, FAKE, slots, ctypes.byref(kv), 1, FAKE, 64,
+                                  None, FAKE, FAKE, FAKE, ws, wsb, None) == -1
+    assert lib.gqla_sparse_gather(ctypes.byref(d), FAKE, FAKE, slots, ctypes.byref(kv), 1, FAKE, 64,
+                                  FAKE, FAKE, FAKE, FAKE, ws, ctypes.c_size_t(4), None) == -3
+    d2 = _dims(h=128, g=2)
+    assert lib.gqla_sparse_gather(ctypes.byref(d2), FAKE, FAKE, slots, ctypes.byref(kv), 1, FAKE, 64,
+                                  FAKE, FAKE, FAKE, FAKE, ws, wsb, None) == -2
+    # select: s_q 3, misaligned slot list
+    assert lib.gqla_sparse_select(ctypes.byref(d), ctypes.byref(kv), 3, FAKE, 64, FAKE, FAKE, FAKE,
+                                  ws, wsb, None) == -2
+    assert lib.gqla_sparse_select(ctypes.byref(d), ctypes.byref(kv), 1, FAKE, 64,
+                                  ctypes.c_void_p((1 << 20) + 4), FAKE, FAKE, ws, wsb, None) == -1
+    # fused decode: a selection whose batch is not a multiple of s_q, zero splits, no slot list
+    assert lib.gqla_decode_gqa_sparse(ctypes.byref(d), FAKE, 2, FAKE, FAKE, slots, ctypes.byref(_kv(batch=3)),
+                                      FAKE, 4, FAKE, FAKE, ws, wsb, None) == -1
+    assert lib.gqla_decode_gqa_sparse(ctypes.byref(d), FAKE, 1, FAKE, FAKE, slots, ctypes.byref(kv),
+                                      FAKE, 0, FAKE, FAKE, ws, wsb, None) == -1
+    assert lib.gqla_decode_gqa_sparse(ctypes.byref(d), FAKE, 1, FAKE, FAKE, slots, ctypes.byref(kv),
+                                      None, 4, FAKE, FAKE, ws, wsb, None) == -1
