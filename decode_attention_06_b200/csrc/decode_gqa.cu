@@ -91,6 +91,9 @@ struct GqaParams {
     // (-1: none), gathered from a cache of real_slots slots
     const int32_t *sel_slot;
     int real_slots;
+    // diagnostic: the V load of this unit is never issued, so a bounded wait runs out
+    // (-1: none)
+    int drop_v_unit;
 };
 
 // Iterates the pieces (sequence b, pages [pb, pe)) of chunk `c`; identical in every role.
@@ -529,7 +532,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         progressed = true;
                     }
                 }
-                if (vc.valid && vpos < kpos && !*abort_flag) {
+                if (vc.valid && vpos < kpos && !*abort_flag && (int)vpos == p.drop_v_unit) {
+                    vc.advance(p);  // diagnostic: no load and no arrival for this unit
+                    ++vpos;
+                    progressed = true;
+                } else if (vc.valid && vpos < kpos && !*abort_flag) {
                     const int vs = vpos % VS;
                     if (mbar_test_wait(&v_empty[vs], ((vpos / VS) & 1) ^ 1)) {
                         const PagePair &pp = vc.pp;
@@ -923,6 +930,9 @@ cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const CUte
 
 }  // namespace
 
+// Set by gqla_debug_drop_v_load, consumed by the next GQA decode launch of the thread.
+thread_local int g_drop_v_unit = -1;
+
 cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups, const void *kv,
                               const void *k_rope, int64_t num_slots, const gqla_kv_index *idx,
                               int num_splits, float scale, float *o_part, float *lse_part,
@@ -965,6 +975,8 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
     p.scale_log2 = scale * kLog2e;
     p.sel_slot = nullptr;
     p.real_slots = 0;
+    p.drop_v_unit = g_drop_v_unit;
+    g_drop_v_unit = -1;
     return G * s_q <= 16 ? launch_nq<16>(kvm, krm, qm, p, stream)
                          : launch_nq<32>(kvm, krm, qm, p, stream);
 }
@@ -1013,6 +1025,7 @@ cudaError_t launch_decode_gqa_sparse(const void *q, int heads, int num_groups, c
     p.scale_log2 = scale * kLog2e;
     p.sel_slot = sel_slot;
     p.real_slots = (int)real_slots;
+    p.drop_v_unit = -1;
     // the dense tile maps are not used in sparse mode: the row maps stand in for them
     return G <= 16 ? launch_nq_mode<16, true>(kvr, krr, qm, kvr, krr, p, stream)
                    : launch_nq_mode<32, true>(kvr, krr, qm, kvr, krr, p, stream);

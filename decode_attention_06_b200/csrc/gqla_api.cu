@@ -32,6 +32,7 @@ cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int
                            const float *o_part, const float *lse_part, const void *w_uv,
                            void *out, float *lse_out, int heads, int num_groups,
                            cudaStream_t stream);
+extern thread_local int g_drop_v_unit;
 }  // namespace gqla
 
 using namespace gqla;
@@ -95,6 +96,12 @@ int check_expand_args(const gqla_dims *dims, const void *latent, int64_t num_slo
 extern "C" {
 
 int gqla_version(void) { return 1; }
+
+int gqla_debug_drop_v_load(int unit) {
+    if (unit < -1) return GQLA_ERR_INVALID_ARG;
+    g_drop_v_unit = unit;
+    return GQLA_OK;
+}
 
 const char *gqla_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 

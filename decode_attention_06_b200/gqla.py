@@ -75,6 +75,7 @@ _SIGS = {
     "gqla_status_string": [_I],
     "gqla_last_cuda_error": [],
     "gqla_version": [],
+    "gqla_debug_drop_v_load": [_I],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -298,6 +299,12 @@ def gqla_last_cuda_error() -> str:
 
 def gqla_version() -> int:
     return _lib.gqla_version()
+
+
+def gqla_debug_drop_v_load(unit: int):
+    """Diagnostic: the next GQA decode of this thread leaves out one V load, so its
+    bounded wait runs out and the call records GQLA_ERR_TIMEOUT (-1 cancels)."""
+    _check("gqla_debug_drop_v_load", _lib.gqla_debug_drop_v_load(unit))
 
 
 def new_workspace(device=None) -> torch.Tensor:

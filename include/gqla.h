@@ -299,6 +299,15 @@ int gqla_read_device_error(const void *workspace, int *info, gqla_stream_t strea
 /* Clears the device error record (asynchronously, on `stream`). */
 int gqla_clear_device_error(void *workspace, gqla_stream_t stream);
 
+/* Diagnostic for testing the failure path: the next gqla_decode_gqa (or
+ * gqla_decode_gqa_noalloc) call made by this host thread leaves out the V load
+ * of work unit `unit` (units count (page pair, group) in issue order within a
+ * CTA), so the wait for it runs out after about two seconds: that call then
+ * records GQLA_ERR_TIMEOUT in its workspace, its outputs are unspecified, and
+ * the context stays usable.  -1 cancels.  Returns GQLA_OK, or
+ * GQLA_ERR_INVALID_ARG for unit < -1. */
+int gqla_debug_drop_v_load(int unit);
+
 /* Static description of a status code. */
 const char *gqla_status_string(int status);
 

@@ -185,6 +185,24 @@ def test_bad_page_index_is_reported_not_faulted():
         assert gqla.gqla_read_device_error(ws)[0] == 0
 
 
+def test_wait_that_runs_out_is_reported_and_context_survives():
+    """A V load that never comes: the bounded wait runs out (about two seconds),
+    the call records GQLA_ERR_TIMEOUT instead of hanging, and the next call on the
+    same context is correct."""
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(128, 8, [700, 300], 1, paged=True, seed=321)
+    g = to_gpu(case)
+    gqla.gqla_debug_drop_v_load(3)
+    out_bad, _, ws, _ = run_decode(g, "gqa", 2)
+    st, _ = gqla.gqla_read_device_error(ws)
+    assert st == -6
+    out, lse, ws2, _ = run_decode(g, "gqa", 2)
+    st2, _ = gqla.gqla_read_device_error(ws2)
+    assert st2 == 0
+    ref, ref_lse = oracle_ref(case)
+    compare(out, ref, what="gqa/after-timeout")
+
+
 def test_sequence_longer_than_page_row_is_reported():
     from decode_attention_06_b200 import gqla
     case = synth.make_case(32, 8, [128, 64], 1, seed=122)
