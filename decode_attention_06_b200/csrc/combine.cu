@@ -12,9 +12,9 @@
 // Both kernels are bound by the read of the fp32 partials; they keep many
 // independent 16-byte loads in flight per thread.  The absorb path's
 // 512 -> 128 product runs on the tcgen05 tensor cores: in a pair of CTAs each
-// merges half of the latent columns of a 64-row tile into bf16, one bulk copy
-// gathers both halves in the first CTA, and that CTA runs the whole K = 512
-// product.
+// merges half of the latent columns of a 64-row tile into bf16, the second CTA
+// stores its half straight into the first CTA's shared memory, and that CTA
+// runs the whole K = 512 product.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -47,12 +47,22 @@ struct CombineParams {
 // sequences, so one warp-wide scan gives every pair its first page.
 __device__ void plan_pairs(const CombineParams &p, int bs_lo, int n, int *c0, int *c1) {
     const int lane = threadIdx.x & 31;
-    const int total = warp_total_pages(p.seqlens, p.batch);
-    const int k = chunk_pages(total, p.num_splits);
     const int b_first = min(bs_lo / p.s_q, p.batch);
-    const int start = warp_sequence_start(p.seqlens, b_first);
     const int bl = b_first + lane;
     const int np = bl < p.batch ? pages_of(p.seqlens[bl]) : 0;
+    // one pass over the lengths: the batch's pages and the pages before b_first
+    int total = 0, start = 0;
+    for (int b = lane; b < p.batch; b += 32) {
+        const int nb = pages_of(p.seqlens[b]);
+        total += nb;
+        start += b < b_first ? nb : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        total += __shfl_xor_sync(0xffffffffu, total, o);
+        start += __shfl_xor_sync(0xffffffffu, start, o);
+    }
+    const int k = chunk_pages(total, p.num_splits);
     const int excl = warp_incl_scan(np) - np;
     const int bs = bs_lo + lane;
     const int d = min(max(bs / p.s_q - b_first, 0), 31);
@@ -206,24 +216,23 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
 // MQA-absorb path (d_in = 512).  A cluster of 2 CTAs per tile of up to 64 rows
 // of one group (bst pairs x G heads).  CTA kq merges latent columns
 // [256 kq, 256 kq + 256) of the tile's rows into bf16 (the MMA's A operand,
-// K-major, 128-byte swizzle); CTA 1 sends its half into CTA 0's shared memory
-// with one bulk copy, and CTA 0 runs the whole product
+// K-major, 128-byte swizzle); CTA 1 stores its half into CTA 0's shared memory
+// with asynchronous remote stores, and CTA 0 runs the whole product
 //   out[64 x 128] = A[64 x 512] * W_UV_g[512 x 128]   (tcgen05 M = 64, fp32 in TMEM)
 // and writes the bf16 rows.
 // ---------------------------------------------------------------------------
 constexpr int kClThreads = 512;
 constexpr int kClRows = 64;      // rows of a tile (MMA M)
 constexpr int kClMaxPairs = 32;  // bst <= 64 / 4 = 16
-constexpr int kClChunk = 16;     // partials whose weights are staged at a time
 
 struct ClSmem {
     static constexpr int kAHalf = kClRows * 256 * 2;       // one CTA's 4 K blocks of A
     static constexpr int oA = 0;                           // 8 K blocks x [64 rows][64] bf16
     static constexpr int oB = 2 * kAHalf;                  // W_UV_g: 2 N blocks x [512 k][64 n] bf16
     static constexpr int oStage = 0;                       // epilogue [64 rows][128] bf16, over A
-    static constexpr int oW = oB + 512 * 128 * 2;          // [32 partials][64 rows] fp32 weights
-    static constexpr int oRowInv = oW + kClChunk * kClRows * 4;
-    static constexpr int oPlan = oRowInv + kClRows * 4;    // c0[32], c1[32], max partials
+    static constexpr int oRowM = oB + 512 * 128 * 2;       // [64 rows] max LSE
+    static constexpr int oRowInv = oRowM + kClRows * 4;    // [64 rows] 1 / sum of weights
+    static constexpr int oPlan = oRowInv + kClRows * 4;    // c0[32], c1[32]
     static constexpr int oBar = oPlan + 2 * kClMaxPairs * 4 + 16;
     static constexpr int kBytes = oBar + 40;
     static constexpr int kAlloc = kBytes + 1024;
@@ -235,11 +244,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    float *sW = reinterpret_cast<float *>(smem + ClSmem::oW);
+    float *sM = reinterpret_cast<float *>(smem + ClSmem::oRowM);
     float *sInv = reinterpret_cast<float *>(smem + ClSmem::oRowInv);
     int *s_c0 = reinterpret_cast<int *>(smem + ClSmem::oPlan);
     int *s_c1 = s_c0 + kClMaxPairs;
-    int *s_maxp = s_c1 + kClMaxPairs;
     uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + ClSmem::oBar);
     uint64_t *b_full = a_full + 1;
     uint64_t *done = a_full + 2;
@@ -279,104 +287,115 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     }
     if (warp == 2) {
         plan_pairs(p, bs0, bst, s_c0, s_c1);
-        if (lane == 0) {
-            int m = 0;
-            for (int j = 0; j < bst; ++j) m = max(m, s_c1[j] - s_c0[j]);
-            *s_maxp = m;
-        }
     }
     tc_fence_before();
     cluster_sync();  // barriers of both CTAs initialised before any remote transfer
     tc_fence_after();
 
-    // ---- merge: warp w owns rows 4w .. 4w+3; lane j covers columns 4j and 128 + 4j of
-    // this CTA's 256 latent columns; two partials are read per step
+    // ---- merge: warp w owns rows 4w .. 4w+3, four heads of one (sequence, token) pair
+    // (the heads per group are a multiple of 4), and computes their weights itself (lane c
+    // holds partial c of a 32-partial block); lane j covers columns 4j and 128 + 4j of
+    // this CTA's 256 latent columns; two partials are read per step, the first two
+    // right behind the LSEs (they do not depend on the weights)
     constexpr int kRw = kClRows / (kClThreads / 32);  // rows per warp
+    static_assert(kRw == 4, "a warp's rows are one pair's heads");
     float4 acc[kRw][2];
 #pragma unroll
     for (int i = 0; i < kRw; ++i) acc[i][0] = acc[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float *src[kRw];
-    int npr[kRw];
-#pragma unroll
-    for (int i = 0; i < kRw; ++i) {
-        const int r = kRw * warp + i;
-        const int j = r / p.G;
-        const bool live = r < rows_in_tile && bs0 + j < p.bs_total;
-        npr[i] = live ? s_c1[j] - s_c0[j] : 0;
+    const int r0 = kRw * warp, j = r0 / p.G;
+    const bool live = r0 < rows_in_tile && bs0 + j < p.bs_total;
+    const int np_max = live ? s_c1[j] - s_c0[j] : 0;  // partials of the warp's rows
+    // partial row of row r0's first partial: < (batch + splits) * s_q * heads < 2^27
+    const int row0 = [&] {
         const int bs = bs0 + j, b = bs / p.s_q, s = bs % p.s_q;
-        src[i] = p.o_part +
-                 (((int64_t)(b + (live ? s_c0[j] : 0)) * p.s_q + s) * p.heads + grp * p.G + r % p.G) *
-                     kLatent +
-                 kq * 256 + lane * 4;
-    }
+        return ((b + (live ? s_c0[j] : 0)) * p.s_q + s) * p.heads + grp * p.G + r0 % p.G;
+    }();
+    const float *src = p.o_part + (int64_t)row0 * kLatent + kq * 256 + lane * 4;
+    const float *lse0 = p.lse_part + row0;
     float4 v[2][kRw][2];
     auto load2 = [&](int c) {
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
             for (int i = 0; i < kRw; ++i) {
-                const bool on = c + u < npr[i];
-                const float *q = src[i] + (int64_t)(c + u) * part_stride * kLatent;
+                const bool on = c + u < np_max;
+                const float *q = src + ((int64_t)(c + u) * part_stride + i) * kLatent;
                 v[u][i][0] = on ? ldg4(q) : make_float4(0.f, 0.f, 0.f, 0.f);
                 v[u][i][1] = on ? ldg4(q + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
     };
-
-    // ---- threads 0..63: one row each -- max LSE and the weights of its partials
-    // (one pass while a row has at most kClChunk partials)
-    float den = 0.0f, Mr = -INFINITY;
-    const float *lse_row = p.lse_part;
-    int np_r = 0;
-    bool live_r = false;
-    const int maxp = *s_maxp;
-    if (tid < kClRows) {
-        const int j = tid / p.G;
-        live_r = tid < rows_in_tile && bs0 + j < p.bs_total;
-        if (live_r) {
-            const int bs = bs0 + j, b = bs / p.s_q, s = bs % p.s_q;
-            np_r = s_c1[j] - s_c0[j];
-            lse_row = p.lse_part + ((int64_t)(b + s_c0[j]) * p.s_q + s) * p.heads + grp * p.G +
-                      tid % p.G;
+    // per row: M = max lse_i, d = sum exp(lse_i - M); the weights below are already
+    // divided by d, and rows with more than 32 partials find M and 1/d in shared memory
+    float l0[kRw];
+#pragma unroll
+    for (int i = 0; i < kRw; ++i) l0[i] = lane < np_max ? __ldg(lse0 + lane * part_stride + i) : -INFINITY;
+    load2(0);
+    float w[kRw];  // weight of partial cb + lane of the current 32-partial block
+    float m[kRw], d[kRw];
+    if (np_max <= 32) {
+        // one block: the four rows' reductions interleave
+#pragma unroll
+        for (int i = 0; i < kRw; ++i) m[i] = l0[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int i = 0; i < kRw; ++i) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
+#pragma unroll
+        for (int i = 0; i < kRw; ++i) d[i] = w[i] = l0[i] == -INFINITY ? 0.0f : __expf(l0[i] - m[i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int i = 0; i < kRw; ++i) d[i] += __shfl_xor_sync(0xffffffffu, d[i], o);
+    } else {
+#pragma unroll
+        for (int i = 0; i < kRw; ++i) {
+            float mi = l0[i];
+            for (int c = lane + 32; c < np_max; c += 32) mi = fmaxf(mi, __ldg(lse0 + c * part_stride + i));
+            m[i] = warp_max(mi);
         }
-        if (maxp > kClChunk) {
-            for (int c = 0; c < np_r; c += 8) {
-                float l[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    l[k] = c + k < np_r ? __ldg(lse_row + (c + k) * part_stride) : -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) Mr = fmaxf(Mr, l[k]);
+        for (int i = 0; i < kRw; ++i) {
+            w[i] = l0[i] == -INFINITY ? 0.0f : __expf(l0[i] - m[i]);
+            float di = w[i];
+            for (int c = lane + 32; c < np_max; c += 32) {
+                const float l = __ldg(lse0 + c * part_stride + i);
+                di += l == -INFINITY ? 0.0f : __expf(l - m[i]);
             }
+            d[i] = warp_sum(di);
         }
     }
-    for (int cb = 0; cb < maxp; cb += kClChunk) {
-        if (cb > 0) __syncthreads();  // the previous chunk's weights are consumed
-        if (tid < kClRows) {
-            float l[kClChunk];
 #pragma unroll
-            for (int k = 0; k < kClChunk; ++k)
-                l[k] = cb + k < np_r ? __ldg(lse_row + (cb + k) * part_stride) : -INFINITY;
-            if (maxp <= kClChunk) {
+    for (int i = 0; i < kRw; ++i) {
+        const float inv = d[i] > 0.0f ? 1.0f / d[i] : 0.0f;
+        w[i] *= inv;
+        if (lane == 0) {
+            sM[r0 + i] = m[i];
+            sInv[r0 + i] = inv;
+            if (leader && p.lse_out && live)
+                p.lse_out[(int64_t)(bs0 + j) * p.heads + grp * p.G + (r0 + i) % p.G] =
+                    d[i] > 0.0f ? m[i] + __logf(d[i]) : -INFINITY;
+        }
+    }
+    __syncwarp();
+    for (int cb = 0; cb < np_max; cb += 32) {
+        if (cb > 0) {
 #pragma unroll
-                for (int k = 0; k < kClChunk; ++k) Mr = fmaxf(Mr, l[k]);
-            }
-#pragma unroll
-            for (int k = 0; k < kClChunk; ++k) {
-                const float w = l[k] == -INFINITY ? 0.0f : __expf(l[k] - Mr);
-                den += w;
-                sW[k * kClRows + tid] = w;  // [partial][row]: conflict-free
+            for (int i = 0; i < kRw; ++i) {
+                const int c = cb + lane;
+                const float l = c < np_max ? __ldg(lse0 + c * part_stride + i) : -INFINITY;
+                w[i] = l == -INFINITY ? 0.0f : __expf(l - sM[r0 + i]) * sInv[r0 + i];
             }
         }
-        __syncthreads();
-        const int n = min(kClChunk, maxp - cb);
+        const int n = min(32, np_max - cb);
 #pragma unroll 1
         for (int j0 = 0; j0 < n; j0 += 2) {
-            load2(cb + j0);
+            if (cb + j0 > 0) load2(cb + j0);
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int i = 0; i < kRw; ++i) {
-                    const float wj = j0 + u < n ? sW[(j0 + u) * kClRows + kRw * warp + i] : 0.0f;
+                    // zero past the row's partials: its LSE there is -inf
+                    const float wj = __shfl_sync(0xffffffffu, w[i], (j0 + u) & 31);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         acc[i][h].x = fmaf(wj, v[u][i][h].x, acc[i][h].x);
@@ -387,44 +406,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
                 }
         }
     }
-    if (tid < kClRows) {
-        sInv[tid] = den > 0.0f ? 1.0f / den : 0.0f;
-        if (leader && p.lse_out && live_r)
-            p.lse_out[(int64_t)(bs0 + tid / p.G) * p.heads + grp * p.G + tid % p.G] =
-                den > 0.0f ? Mr + __logf(den) : -INFINITY;
-    }
-    __syncthreads();
 
     // ---- merged rows -> this CTA's four K blocks of A (bf16, K-major, 128-byte swizzle),
-    // at the same place they take in the leader's A
+    // at the place they take in the leader's A: the leader stores its own, the peer
+    // sends its half straight into the leader's shared memory (8-byte asynchronous
+    // stores counted on the leader's a_full)
     {
         const int chunk = (lane & 15) >> 1, half8 = (lane & 1) * 8;
+        const uint32_t a_remote = leader ? 0u : map_peer(smem_u32(smem + ClSmem::oA), 0);
+        const uint32_t bar_remote = leader ? 0u : map_peer(smem_u32(a_full), 0);
 #pragma unroll
         for (int i = 0; i < kRw; ++i) {
             const int r = kRw * warp + i;
-            const float inv = sInv[r];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int kb = kq * 4 + 2 * h + (lane >> 4);
-                *reinterpret_cast<uint2 *>(smem + ClSmem::oA + kb * (kClRows * 128) + r * 128 +
-                                           ((chunk ^ (r & 7)) << 4) + half8) =
-                    pack_bf16x4(acc[i][h].x * inv, acc[i][h].y * inv, acc[i][h].z * inv,
-                                acc[i][h].w * inv);
+                const uint32_t off = kb * (kClRows * 128) + r * 128 + ((chunk ^ (r & 7)) << 4) + half8;
+                const uint2 val = pack_bf16x4(acc[i][h].x, acc[i][h].y, acc[i][h].z, acc[i][h].w);
+                if (leader)
+                    *reinterpret_cast<uint2 *>(smem + ClSmem::oA + off) = val;
+                else
+                    st_async_v2(a_remote + off, val, bar_remote);
             }
         }
     }
-    fence_proxy_async_smem();
-    __syncthreads();
-
     if (!leader) {
-        // ---- send this half of A to the leader; its mbarrier counts the bytes
-        if (tid == 0)
-            bulk_copy_to_peer(map_peer(smem_u32(smem + ClSmem::oA + ClSmem::kAHalf), 0),
-                              smem + ClSmem::oA + ClSmem::kAHalf, ClSmem::kAHalf,
-                              map_peer(smem_u32(a_full), 0));
-        cluster_sync();  // the leader has received the half: this CTA's memory may go
+        cluster_sync();  // pairs with the leader's arrive once its MMAs have read the half
         return;
     }
+    fence_proxy_async_smem();
+    __syncthreads();
 
     // ---- leader: the other half of A and W_UV_g in place -> 32 MMAs (M = 64, K = 512)
     const uint32_t tmem = *tmem_slot;
@@ -456,6 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     }
     const bool ok = mbar_wait(done, 0, abort_flag);
     tc_fence_after();
+    cluster_arrive_relaxed();  // the MMAs have read the peer's half: the sender may exit
     // ---- epilogue: TMEM (M = 64: row m in lane (m % 16) + 32 (m / 16)) -> bf16 rows in
     // shared memory (over A: the MMAs are done) -> coalesced 256-byte row stores
     if (ok) {
@@ -480,7 +492,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
             }
         }
     }
+    tc_fence_before();
     __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
     if (ok && !*abort_flag) {
         for (int i = tid; i < kClRows * 16; i += kClThreads) {
             const int r = i >> 4, part16 = i & 15;
@@ -490,12 +507,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
             reinterpret_cast<uint4 *>(p.out + orow * kDv)[part16] =
                 reinterpret_cast<const uint4 *>(smem + ClSmem::oStage + r * 256)[part16];
         }
-    }
-    tc_fence_before();
-    cluster_sync();  // pairs with the sender's: its copy has landed
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 128);
     }
 }
 

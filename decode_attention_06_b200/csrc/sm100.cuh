@@ -435,6 +435,15 @@ __device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, uint4 v, uint3
         : "memory");
 }
 
+// Asynchronous 8-byte store into a peer CTA's shared memory; completes 8 bytes
+// of the transaction count of the peer's mbarrier.
+__device__ __forceinline__ void st_async_v2(uint32_t dst_cluster, uint2 v, uint32_t mbar_cluster) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(
+                     dst_cluster),
+                 "r"(v.x), "r"(v.y), "r"(mbar_cluster)
+                 : "memory");
+}
+
 // Asynchronous 4-byte store into a peer CTA's shared memory; completes 4 bytes
 // of the transaction count of the peer's mbarrier.
 __device__ __forceinline__ void st_async_b32(uint32_t dst_cluster, uint32_t v, uint32_t mbar_cluster) {
@@ -454,6 +463,12 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
+}
+
+// The arrive half of cluster_sync without its release ordering, for a CTA that
+// only lets the others go on (it may exit without the matching wait).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {

@@ -117,6 +117,9 @@ SMALL = [
     ("one_split", 128, [300, 200], 2, True, 1),
     ("zero_length_sequence", 32, [0, 65, 0], 1, False, 4),
     ("mtp_single_token", 32, [1, 2], 2, False, 2),
+    # a sequence over more than 32 splits: the combines take the weights in blocks of 32
+    ("many_partials", 128, [5000, 300], 1, True, 70),
+    ("many_partials_mtp", 32, [4000, 9], 2, False, 60),
 ]
 
 
