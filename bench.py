@@ -256,8 +256,11 @@ def run_ours(args, rank, world, local_rank):
     dims = gqla.make_dims(h, g)
     kv = gqla.make_kv_index(case["page_table"], case["seqlens"], case["num_pages"])
     n_slots = case["num_pages"] * case["page_size"]
-    splits = {"absorb": args.splits or gqla.gqla_num_splits_hint("absorb", h, s_q),
-              "gqa": args.splits or gqla.gqla_num_splits_hint("gqa", h, s_q)}
+    # split counts planned on the host from the lengths (one wave at most, chunks
+    # that hold two sequences' pieces counted at their cost)
+    lens_host = case["seqlens"].cpu()
+    splits = {"absorb": args.splits or gqla.plan_splits("absorb", h, s_q, lens_host),
+              "gqa": args.splits or gqla.plan_splits("gqa", h, s_q, lens_host)}
     kvx = torch.empty(g, n_slots, 256, dtype=torch.bfloat16, device=dev)
     kr = torch.empty(n_slots, 64, dtype=torch.bfloat16, device=dev)
     ba = gqla.DecodeBuffers(dims, B, s_q, splits["absorb"], "absorb", device=dev)

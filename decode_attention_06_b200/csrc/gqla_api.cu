@@ -2,6 +2,9 @@
 // include/gqla.h): argument validation, then launches on the caller's stream.
 #include <math.h>
 
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 
 namespace gqla {
@@ -134,6 +137,41 @@ int gqla_num_splits_hint(int path, int num_heads, int s_q) {
     if (path == 1) return sms;
     const int row_blocks = (s_q * num_heads + 127) / 128;
     return sms / (2 * row_blocks) > 0 ? sms / (2 * row_blocks) : 1;
+}
+
+int gqla_plan_splits(const int32_t *seqlens, int batch, int max_splits, int piece_cost_pages) {
+    if (!seqlens || batch <= 0 || batch > 65535 || max_splits <= 0 || max_splits > 65535 ||
+        piece_cost_pages < 0)
+        return GQLA_ERR_INVALID_ARG;
+    // first global page of every non-empty sequence after the first one
+    std::vector<int64_t> starts;
+    int64_t total = 0;
+    for (int b = 0; b < batch; ++b) {
+        if (seqlens[b] < 0) return GQLA_ERR_INVALID_ARG;
+        const int64_t np = (seqlens[b] + kPage - 1) / kPage;
+        if (np > 0 && total > 0) starts.push_back(total);
+        total += np;
+    }
+    if (total == 0) return 1;
+    int best = 1;
+    int64_t best_cost = -1, prev_k = -1;
+    std::vector<int64_t> cost;
+    for (int n = 1; n <= max_splits; ++n) {
+        const int64_t k = (total + n - 1) / n;
+        if (k == prev_k) continue;  // the same chunks as a smaller count
+        prev_k = k;
+        const int64_t chunks = (total + k - 1) / k;
+        cost.assign((size_t)chunks, 0);
+        for (int64_t c = 0; c < chunks; ++c) cost[c] = std::min(k, total - c * k);
+        for (const int64_t st : starts)
+            if (st % k) cost[st / k] += piece_cost_pages;  // a sequence starts inside the chunk
+        const int64_t worst = *std::max_element(cost.begin(), cost.end());
+        if (best_cost < 0 || worst < best_cost) {
+            best_cost = worst;
+            best = n;
+        }
+    }
+    return best;
 }
 
 int gqla_read_device_error(const void *workspace, int *info, gqla_stream_t stream) {

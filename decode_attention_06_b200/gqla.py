@@ -70,6 +70,7 @@ _SIGS = {
     "gqla_partial_slots": [_I, _I],
     "gqla_workspace_bytes": [],
     "gqla_num_splits_hint": [_I, _I, _I],
+    "gqla_plan_splits": [_P, _I, _I, _I],
     "gqla_read_device_error": [_P, ctypes.POINTER(ctypes.c_int), _P],
     "gqla_clear_device_error": [_P, _P],
     "gqla_status_string": [_I],
@@ -277,6 +278,28 @@ def gqla_num_splits_hint(path: str, num_heads: int, s_q: int) -> int:
     if n < 0:
         raise GqlaError("gqla_num_splits_hint", n)
     return n
+
+
+def gqla_plan_splits(seqlens, max_splits: int, piece_cost_pages: int) -> int:
+    """Split count for known lengths (host int32 values: a CPU tensor or a list)."""
+    lens = torch.as_tensor(seqlens, dtype=torch.int32, device="cpu").contiguous()
+    n = _lib.gqla_plan_splits(ctypes.c_void_p(lens.data_ptr()), lens.numel(), max_splits, piece_cost_pages)
+    if n < 0:
+        raise GqlaError("gqla_plan_splits", n)
+    return n
+
+
+# What a chunk's second piece costs, in pages of the chunk, for the two decode
+# kernels on B200 (a sweep of split counts over 32 sequences of 4096 tokens:
+# the absorb decode's time grows by ~0.9 us per page of its longest chunk and by
+# ~6 us when that chunk holds two pieces; the GQA decode, bound by the HBM
+# stream, loses about two pages' worth).
+PIECE_COST_PAGES = {"absorb": 6, "gqa": 2}
+
+
+def plan_splits(path: str, num_heads: int, s_q: int, seqlens) -> int:
+    """gqla_plan_splits up to one wave of the device, with the path's piece cost."""
+    return gqla_plan_splits(seqlens, gqla_num_splits_hint(path, num_heads, s_q), PIECE_COST_PAGES[path])
 
 
 def gqla_read_device_error(workspace: torch.Tensor, stream=None):

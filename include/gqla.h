@@ -291,6 +291,22 @@ size_t gqla_workspace_bytes(void);
  * 1 = GQA.  Returns < 0 on error. */
 int gqla_num_splits_hint(int path, int num_heads, int s_q);
 
+/* Host-side choice of a split count for known sequence lengths.  Both decode
+ * calls cut the batch's pages, concatenated sequence after sequence (T pages
+ * in all), into chunks of k = ceil(T / num_splits) pages, one chunk per split;
+ * a chunk that holds the end of one sequence and the start of the next runs a
+ * second "piece" (its own partial output, epilogue and query), which costs a
+ * split more than a page.  Among num_splits = 1 .. max_splits this returns the
+ * one whose heaviest chunk, counted as its pages plus `piece_cost_pages` for
+ * every sequence that starts inside it after its first page, is lightest (the
+ * smallest such count on a tie).  Host-only: touches no device.
+ *   seqlens           host int32[batch], each >= 0
+ *   batch             1 .. 65535
+ *   max_splits        1 .. 65535 (e.g. gqla_num_splits_hint's value)
+ *   piece_cost_pages  >= 0
+ * Returns the split count, or GQLA_ERR_INVALID_ARG. */
+int gqla_plan_splits(const int32_t *seqlens, int batch, int max_splits, int piece_cost_pages);
+
 /* Reads (synchronising `stream`) and returns the first device-side error
  * recorded in `workspace` (GQLA_OK if none); `info`, if not NULL, receives
  * a code-specific detail (e.g. the sequence index).  Does not clear it. */

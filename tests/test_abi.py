@@ -158,3 +158,68 @@ def test_expand_tc_and_sparse_calls_reject_bad_arguments(lib):
                                       FAKE, 0, FAKE, FAKE, ws, wsb, None) == -1
     assert lib.gqla_decode_gqa_sparse(ctypes.byref(d), FAKE, 1, FAKE, FAKE, slots, ctypes.byref(kv),
                                       None, 4, FAKE, FAKE, ws, wsb, None) == -1
+
+
+# ------------------------------------------------------------------ host-side split planning
+
+def _plan_by_hand(lens, max_splits, piece_cost):
+    """Every split count tried in turn: chunk loads = pages + piece_cost per sequence
+    that starts inside a chunk after its first page; the lightest heaviest chunk wins,
+    the smallest count on a tie."""
+    pages = [(x + 63) // 64 for x in lens]
+    T = sum(pages)
+    if T == 0:
+        return 1
+    starts, acc = [], 0
+    for n in pages:
+        if n > 0 and acc > 0:
+            starts.append(acc)
+        acc += n
+    best, best_load = None, None
+    for n in range(1, max_splits + 1):
+        k = -(-T // n)
+        load = [min(k, T - c * k) for c in range(-(-T // k))]
+        for st in starts:
+            if st % k:
+                load[st // k] += piece_cost
+        if best_load is None or max(load) < best_load:
+            best, best_load = n, max(load)
+    return best
+
+
+def _plan(lib, lens, max_splits, piece_cost):
+    arr = (ctypes.c_int32 * len(lens))(*lens)
+    return lib.gqla_plan_splits(arr, len(lens), max_splits, piece_cost)
+
+
+def test_plan_splits_uniform_batch(lib):
+    lens = [4096] * 32  # 32 sequences of 64 pages
+    # without a piece cost: the most splits that shorten the longest chunk (28 pages)
+    assert _plan(lib, lens, 74, 0) == 74
+    # with one: 64 splits give 32-page chunks inside single sequences, against 28 pages
+    # plus a second piece for 74
+    assert _plan(lib, lens, 74, 6) == 64
+    assert _plan(lib, lens, 148, 2) == 128
+    assert _plan(lib, lens, 1, 6) == 1
+
+
+def test_plan_splits_matches_exhaustive_search(lib):
+    import random
+    rng = random.Random(11)
+    for _ in range(60):
+        B = rng.randint(1, 40)
+        lens = [rng.choice([0, rng.randint(1, 200), rng.randint(1, 9000)]) for _ in range(B)]
+        m, pc = rng.randint(1, 160), rng.randint(0, 9)
+        assert _plan(lib, lens, m, pc) == _plan_by_hand(lens, m, pc), (lens, m, pc)
+
+
+def test_plan_splits_edges(lib):
+    assert _plan(lib, [0, 0, 0], 74, 6) == 1          # no pages: one split
+    assert _plan(lib, [0, 640, 0], 8, 6) == 5         # 2-page chunks from 5 splits on; empty sequences start no piece
+    assert _plan(lib, [64] * 4, 4, 6) == 4            # one page each: one per split
+    assert _plan(lib, [-1, 64], 4, 6) == -1
+    assert _plan(lib, [64], 0, 6) == -1
+    assert _plan(lib, [64], 4, -1) == -1
+    assert lib.gqla_plan_splits(None, 1, 4, 6) == -1
+    arr = (ctypes.c_int32 * 1)(64)
+    assert lib.gqla_plan_splits(arr, 0, 4, 6) == -1
