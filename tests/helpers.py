@@ -25,8 +25,8 @@ def run_decode(gcase, path, num_splits=None, stream=None):
     dims = gqla.make_dims(h, g)
     kv = gqla.make_kv_index(gcase["page_table"], gcase["seqlens"], gcase["num_pages"])
     B = gcase["seqlens"].numel()
-    if num_splits is None:
-        num_splits = gqla.gqla_num_splits_hint(path, h, s_q)
+    if num_splits is None:  # as bench.py plans them: from the host copy of the lengths
+        num_splits = gqla.plan_splits(path, h, s_q, gcase["seqlens"].cpu())
     bufs = gqla.DecodeBuffers(dims, B, s_q, num_splits, path)
     extras = {}
     if path == "gqa":

@@ -216,15 +216,20 @@ def test_sequence_longer_than_page_row_is_reported():
 
 # ------------------------------------------------------------------ full-size workloads, sampled
 
-FULL = [(name, s) for name, w in synth.WORKLOADS.items() for s in w.s_q]
+FULL = [(name, s, None) for name, w in synth.WORKLOADS.items() for s in w.s_q]
+# the bench workload also at the one-wave split counts (chunks holding two sequences' pieces)
+FULL += [("dsv3_h128_b32_l4096", 1, "one_wave")]
 
 
 @pytest.mark.parametrize("path", ["gqa", "absorb"])
-@pytest.mark.parametrize("name,s_q", FULL, ids=[f"{n}-sq{s}" for n, s in FULL])
-def test_decode_parity_full_size_sampled(path, name, s_q):
+@pytest.mark.parametrize("name,s_q,splits", FULL, ids=[f"{n}-sq{s}" + (f"-{m}" if m else "") for n, s, m in FULL])
+def test_decode_parity_full_size_sampled(path, name, s_q, splits):
+    """Full-size workloads at the split counts bench.py plans (or one wave), sampled."""
     w = synth.WORKLOADS[name]
     case = synth.make_workload(name, s_q=s_q, device="cuda")
-    out, lse, ws, _ = run_decode(case, path)
+    from decode_attention_06_b200 import gqla
+    n = gqla.gqla_num_splits_hint(path, w.num_heads, s_q) if splits == "one_wave" else None
+    out, lse, ws, _ = run_decode(case, path, n)
     B = w.batch
     rng = np.random.default_rng(w.seed)
     picks = sorted(set([0, B - 1] + rng.integers(0, B, size=2).tolist()))[:3]
