@@ -9,8 +9,10 @@
 // A row whose sequence saw no token (no partial, or every lse_i = -inf)
 // gets out = 0 and lse = -inf.
 //
-// Both kernels are bound by the read of the fp32 partials; they keep many
-// independent 16-byte loads in flight per thread.  The absorb path's
+// Both kernels spend most of their time on the read of the fp32 partials, on
+// its latency more than on HBM bandwidth; they keep many independent 16-byte
+// loads in flight per thread and compute the merge weights while the partials
+// are on their way.  The absorb path's
 // 512 -> 128 product runs on the tcgen05 tensor cores: in a pair of CTAs each
 // merges half of the latent columns of a 64-row tile into bf16, the second CTA
 // stores its half straight into the first CTA's shared memory, and that CTA
