@@ -153,19 +153,23 @@ int gqla_plan_splits(const int32_t *seqlens, int batch, int max_splits, int piec
         total += np;
     }
     if (total == 0) return 1;
+    // Every chunk but the last holds k pages, so the heaviest chunk is k pages (or the
+    // whole batch when it fits one chunk) unless a chunk with sequence starts inside it
+    // weighs more; the starts are ascending, so one pass groups them by chunk.
+    // O(max_splits * batch) at most.
     int best = 1;
     int64_t best_cost = -1, prev_k = -1;
-    std::vector<int64_t> cost;
     for (int n = 1; n <= max_splits; ++n) {
         const int64_t k = (total + n - 1) / n;
         if (k == prev_k) continue;  // the same chunks as a smaller count
         prev_k = k;
-        const int64_t chunks = (total + k - 1) / k;
-        cost.assign((size_t)chunks, 0);
-        for (int64_t c = 0; c < chunks; ++c) cost[c] = std::min(k, total - c * k);
-        for (const int64_t st : starts)
-            if (st % k) cost[st / k] += piece_cost_pages;  // a sequence starts inside the chunk
-        const int64_t worst = *std::max_element(cost.begin(), cost.end());
+        int64_t worst = std::min(k, total);
+        for (size_t i = 0; i < starts.size();) {
+            const int64_t c = starts[i] / k;
+            int64_t inside = 0;
+            for (; i < starts.size() && starts[i] / k == c; ++i) inside += starts[i] % k != 0;
+            worst = std::max(worst, std::min(k, total - c * k) + inside * piece_cost_pages);
+        }
         if (best_cost < 0 || worst < best_cost) {
             best_cost = worst;
             best = n;
