@@ -356,6 +356,43 @@ def test_expand_f32seq_close_to_exact_and_rounded_once():
     assert (exact_rounded == bits.ravel()[:2000]).mean() > 0.97
 
 
+def test_expand_f32seq_pins_the_ascending_fp32_order():
+    """The fixed rounding order itself: fp32 fused multiply-adds in ascending latent
+    index from +0, one bf16 rounding.  The hand-built case gives different bits for
+    a descending order, for fp64 accumulation rounded twice and for the exact sum
+    rounded once, so this fails for any of them."""
+    from tests.helpers import expansion_order_case
+    lat, wk, wv, want = expansion_order_case()
+    bits, kr_bits = oracle.expand_f32seq_bits(lat, wk, wv)
+    assert bits.shape == (1, 1, 256)
+    np.testing.assert_array_equal(bits[0, 0, :3], want)
+    np.testing.assert_array_equal(bits[0, 0, 128:131], want)
+    assert not bits[0, 0, 3:128].any() and not bits[0, 0, 131:].any()
+    assert not kr_bits.any()
+
+    # the alternatives really differ on this case (fp32 and fp64 sums by numpy)
+    def bf16(x):
+        return oracle.bf16_rne_bits(float(np.float32(x)))
+
+    terms = [lat[0, :512].astype(np.float64) * wk[0, :, d].astype(np.float64) for d in range(3)]
+    for t in terms:  # every product is exact in fp32
+        assert np.array_equal(t.astype(np.float32).astype(np.float64), t)
+
+    def f32_sum(t):
+        acc = np.float32(0.0)
+        for x in t:
+            acc = np.float32(acc + np.float32(x))
+        return acc
+
+    ascending = [bf16(f32_sum(t)) for t in terms]
+    descending = [bf16(f32_sum(t[::-1])) for t in terms]
+    fp64_twice = [bf16(np.float32(sum(t))) for t in terms]
+    assert ascending == want.tolist()
+    assert descending == [0x3F81, 0x3F80, 0x3F80]
+    assert fp64_twice == [0x3F81, 0x3F81, 0x3F80]
+    assert len({tuple(ascending), tuple(descending), tuple(fp64_twice)}) == 3
+
+
 @pytest.mark.parametrize("x,bits", [
     (1.0, 0x3F80),
     (1.0 + 2.0 ** -8, 0x3F80),          # halfway, ties to even (down)
