@@ -4,7 +4,8 @@
 
 One step = one decode step of the batch through the whole hot path: the
 MQA-absorb path (gqla_absorb_query -> gqla_decode_absorb -> gqla_combine with
-W_UV) and the GQA path (gqla_decode_gqa -> gqla_combine) over the same batch.
+W_UV) and the GQA path (gqla_decode_gqa_step: the GQA decode, then the
+combine for the sequences that span more than one chunk) over the same batch.
 The two paths are independent, so the GQA path runs on a second stream beside
 the absorb path's decode and combine (after the query absorption has started):
 CTAs of one path take the SMs the other path's tail leaves idle.
@@ -22,14 +23,22 @@ e2e     = the same through the C ABI with host buffers: each step copies the
           table and lengths are one buffer copied on a second stream beside
           q and the query absorption; the GQA path and its output copy run on
           a third stream beside the absorb path).
-Timing  = the step is captured into a CUDA graph; each timed step replays it
-          between two CUDA events on the stream (device time, no host launch
-          overhead).  The per-call breakdown comes from a second graph that
-          runs the five calls in order on one stream with an event record
-          around every call.  L2 is flushed (a 256 MiB write, then a
-          256 MiB read so no dirty line is left) before every step, outside
-          its events; W >= 3 untimed eager and W
-          graph warm-up steps come first.
+Timing  = the step is captured into a CUDA graph; the K timed steps are issued
+          back to back, each replay between two CUDA events on the stream
+          (device time, no host launch overhead), with an L2 flush (a 256 MiB
+          write, then a 256 MiB read so no dirty line is left) before every
+          step, outside its events; one synchronize ends the timed region,
+          while an NVML sampler records SM clocks and throttle reasons.  The
+          per-call breakdown comes from a second graph that runs the five
+          calls in order on one stream with an event record around every
+          call.  W >= 3 untimed eager and W graph warm-up steps come first.
+workload: by default the largest single-GPU configuration of the suite
+          (dsv3_h128_b64_l8192_mtp2: 128 heads, 8 groups, 64 sequences of
+          8192 tokens, s_q = 2); at N = 1 every other workload of the suite
+          follows under "workloads" (step time, per-call times, each path's
+          roofline fractions), unless --headline-only.
+--gpus N  one rank per GPU: under torchrun WORLD_SIZE must equal N; started
+          without torchrun, the script relaunches itself as N ranks.
 roofline: the dominant kernel's algorithmic bytes (or FLOPs) per launch over
           its mean event-timed duration, against MEASURED_PEAKS.json.
 cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload
@@ -53,7 +62,9 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-DEFAULT_WORKLOAD = "dsv3_h128_b32_l4096"
+# the largest single-GPU configuration of the suite: 64 sequences x 8192 tokens,
+# two MTP query tokens (the absorb path is tensor-bound there)
+DEFAULT_WORKLOAD = "dsv3_h128_b64_l8192_mtp2"
 METRIC = "decode-attn tokens/s & µs/step per path; % of B200 HBM / tensor roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
@@ -87,13 +98,15 @@ def _src_hash(files):
     return h.hexdigest()[:16]
 
 
-def _stored_traffic(kernel, workload):
+def _stored_traffic(kernel, workload, s_q):
+    """ncu DRAM bytes per launch stored for (kernel, workload, s_q), or None when
+    there is none or the kernel's source has changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p) or kernel not in KERNEL_SOURCES:
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kernel, {}).get(workload)
+    e = d.get(kernel, {}).get(f"{workload}/sq{s_q}")
     if not e or e.get("source_hash") != _src_hash(KERNEL_SOURCES[kernel]):
         return None
     return e.get("bytes_per_launch")
@@ -108,7 +121,7 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index, period_s=0.01):
+    def __init__(self, device_index, period_s=0.0002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         self._period = period_s
@@ -125,8 +138,10 @@ class ClockSampler:
         except Exception:  # NVML missing: report no samples rather than guessing
             self._nvml = None
             return self
+        self._started = threading.Event()
         self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
+        self._started.wait(0.5)  # the sampler runs before the timed work is issued
         return self
 
     def _run(self):
@@ -140,6 +155,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
+            self._started.set()
             time.sleep(self._period)
 
     def __exit__(self, *a):
@@ -243,301 +259,439 @@ def cpu_oracle_rate(case, w, s_q, budget_s=10.0, unit_groups=None):
 
 # ------------------------------------------------------------------ the GPU arm
 
-def run_ours(args, rank, world, local_rank):
-    from decode_attention_06_b200 import gqla, synth
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = synth.WORKLOADS[args.workload]
-    s_q = args.s_q or w.s_q[0]
-    case = synth.make_case(w.num_heads, w.num_groups, w.seqlens(), s_q, paged=w.paged,
-                           seed=w.seed + 1000 * rank, device=str(dev))
-    h, g = w.num_heads, w.num_groups
-    B = case["seqlens"].numel()
-    dims = gqla.make_dims(h, g)
-    kv = gqla.make_kv_index(case["page_table"], case["seqlens"], case["num_pages"])
-    n_slots = case["num_pages"] * case["page_size"]
-    # split counts planned on the host from the lengths (one wave at most, chunks
-    # that hold two sequences' pieces counted at their cost)
-    lens_host = case["seqlens"].cpu()
-    splits = {"absorb": args.splits or gqla.plan_splits("absorb", h, s_q, lens_host),
-              "gqa": args.splits or gqla.plan_splits("gqa", h, s_q, lens_host)}
-    kvx = torch.empty(g, n_slots, 256, dtype=torch.bfloat16, device=dev)
-    kr = torch.empty(n_slots, 64, dtype=torch.bfloat16, device=dev)
-    ba = gqla.DecodeBuffers(dims, B, s_q, splits["absorb"], "absorb", device=dev)
-    bg = gqla.DecodeBuffers(dims, B, s_q, splits["gqa"], "gqa", device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_sum = torch.empty((), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
+_FLUSH = {}
 
-    def flush_l2():
-        # Write a buffer larger than L2, then read another one: the write
-        # evicts every line of the step's data, and the read makes L2 write
-        # the dirty lines of the first buffer back before the step starts,
-        # so their write-back does not land in the next timed kernel.
-        flush.fill_(1.0)
-        torch.sum(flush_rd, dim=0, out=flush_sum)
 
-    # one-shot expansion, timed on its own: the tensor-core version, then the
-    # bit-exact sequential-order one (whose output the steps below use)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+def flush_l2(dev):
+    """Write a buffer larger than L2, then read another one: the write evicts every
+    line of the step's data, and the read makes L2 write the dirty lines of the first
+    buffer back before the step starts, so their write-back does not land in the
+    next timed kernel."""
+    if dev not in _FLUSH:
+        _FLUSH[dev] = (torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
+                       torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
+                       torch.empty((), dtype=torch.float32, device=dev))
+    buf, rd, out = _FLUSH[dev]
+    buf.fill_(1.0)
+    torch.sum(rd, dim=0, out=out)
 
-    def time_expand(fn):
-        fn(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
-        flush_l2()
-        e0.record()
-        fn(dims, case["latent"], case["w_uk"], case["w_uv"], kvx, kr)
-        e1.record()
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1)
 
-    expand_tc_ms = time_expand(gqla.gqla_expand_cache_tc)
-    expand_ms = time_expand(gqla.gqla_expand_cache)
+CALL_NAMES = ["absorb_query", "decode_absorb", "combine_absorb", "decode_gqa", "combine_gqa"]
 
-    names = ["absorb_query", "decode_absorb", "combine_absorb", "decode_gqa", "combine_gqa"]
-    calls = [
-        lambda: gqla.gqla_absorb_query(dims, case["q"], case["w_uk"], ba.q_absorbed),
-        lambda: gqla.gqla_decode_absorb(dims, ba.q_absorbed, case["latent"], kv, ba.num_splits,
-                                        ba.o_part, ba.lse_part, ba.workspace),
-        lambda: gqla.gqla_combine(dims, kv, s_q, ba.num_splits, 512, ba.o_part, ba.lse_part,
-                                  case["w_uv"], ba.out, ba.lse),
-        lambda: gqla.gqla_decode_gqa(dims, case["q"], kvx, kr, kv, bg.num_splits, bg.o_part,
-                                     bg.lse_part, bg.workspace),
-        lambda: gqla.gqla_combine(dims, kv, s_q, bg.num_splits, 128, bg.o_part, bg.lse_part,
-                                  None, bg.out, bg.lse),
-    ]
-    gqa_stream = torch.cuda.Stream(device=dev)
 
-    def step():
-        # query absorption first, then the GQA path on its own stream beside the
-        # absorb path's decode and combine; the step ends when both are done
+class Workbench:
+    """One workload (and s_q) on this rank's GPU: its seeded inputs, the expanded
+    cache, both paths' buffers, and the five calls of a step through the C ABI."""
+
+    def __init__(self, name, s_q, rank, dev, splits=None):
+        from decode_attention_06_b200 import gqla, synth
+        self.gqla = gqla
+        self.name, self.dev = name, dev
+        self.w = w = synth.WORKLOADS[name]
+        self.s_q = s_q = s_q or w.s_q[0]
+        self.case = case = synth.make_case(w.num_heads, w.num_groups, w.seqlens(), s_q, paged=w.paged,
+                                           seed=w.seed + 1000 * rank, device=str(dev))
+        h, g = w.num_heads, w.num_groups
+        self.B = case["seqlens"].numel()
+        self.dims = dims = gqla.make_dims(h, g)
+        self.kv = gqla.make_kv_index(case["page_table"], case["seqlens"], case["num_pages"])
+        self.n_slots = case["num_pages"] * case["page_size"]
+        # split counts planned on the host from the lengths (one wave at most, chunks
+        # that hold two sequences' pieces counted at their cost)
+        lens_host = case["seqlens"].cpu()
+        self.splits = {"absorb": splits or gqla.plan_splits("absorb", h, s_q, lens_host),
+                       "gqa": splits or gqla.plan_splits("gqa", h, s_q, lens_host)}
+        self.kvx = torch.empty(g, self.n_slots, 256, dtype=torch.bfloat16, device=dev)
+        self.kr = torch.empty(self.n_slots, 64, dtype=torch.bfloat16, device=dev)
+        self.ba = gqla.DecodeBuffers(dims, self.B, s_q, self.splits["absorb"], "absorb", device=dev)
+        self.bg = gqla.DecodeBuffers(dims, self.B, s_q, self.splits["gqa"], "gqa", device=dev)
+        self.gqa_stream = torch.cuda.Stream(device=dev)
+        self.calls = self.make_calls(case["q"], self.kv)
+
+    def gqa_step_call(self, q, kv):
+        """The GQA path as one call (gqla_decode_gqa_step: the decode, and the combine for
+        the sequences that span more than one chunk)."""
+        gqla, bg = self.gqla, self.bg
+        return lambda: gqla.gqla_decode_gqa_step(self.dims, q, self.kvx, self.kr, kv, bg.num_splits,
+                                                 bg.o_part, bg.lse_part, bg.out, bg.lse, bg.workspace)
+
+    def launches_per_step(self):
+        """Kernels one step launches: query absorption, absorb decode and combine; the GQA
+        decode, and its combine unless every sequence lies in one chunk (one split)."""
+        return 3 + 1 + (1 if self.splits["gqa"] > 1 else 0)
+
+    def make_calls(self, q, kv):
+        gqla, dims, case, ba, bg, s_q = self.gqla, self.dims, self.case, self.ba, self.bg, self.s_q
+        return [
+            lambda: gqla.gqla_absorb_query(dims, q, case["w_uk"], ba.q_absorbed),
+            lambda: gqla.gqla_decode_absorb(dims, ba.q_absorbed, case["latent"], kv, ba.num_splits,
+                                            ba.o_part, ba.lse_part, ba.workspace),
+            lambda: gqla.gqla_combine(dims, kv, s_q, ba.num_splits, 512, ba.o_part, ba.lse_part,
+                                      case["w_uv"], ba.out, ba.lse),
+            lambda: gqla.gqla_decode_gqa(dims, q, self.kvx, self.kr, kv, bg.num_splits, bg.o_part,
+                                         bg.lse_part, bg.workspace),
+            lambda: gqla.gqla_combine(dims, kv, s_q, bg.num_splits, 128, bg.o_part, bg.lse_part,
+                                      None, bg.out, bg.lse),
+        ]
+
+    def time_expand(self):
+        """The one-shot expansion, timed on its own: the tensor-core version, then the
+        bit-exact sequential-order one (whose output the steps use).  Returns ms."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c = self.case
+        res = []
+        for fn in (self.gqla.gqla_expand_cache_tc, self.gqla.gqla_expand_cache):
+            fn(self.dims, c["latent"], c["w_uk"], c["w_uv"], self.kvx, self.kr)
+            flush_l2(self.dev)
+            e0.record()
+            fn(self.dims, c["latent"], c["w_uk"], c["w_uv"], self.kvx, self.kr)
+            e1.record()
+            torch.cuda.synchronize()
+            res.append(e0.elapsed_time(e1))
+        return res[1], res[0]
+
+    def step(self):
+        # query absorption first, then the GQA path (one call) on its own stream beside
+        # the absorb path's decode and combine; the step ends when both are done
+        calls = self.calls
+        gqa_step = self.gqa_step_call(self.case["q"], self.kv)
         main = torch.cuda.current_stream()
         calls[0]()
         fork = torch.cuda.Event()
         fork.record(main)
-        gqa_stream.wait_event(fork)
-        with torch.cuda.stream(gqa_stream):
-            calls[3]()
-            calls[4]()
+        self.gqa_stream.wait_event(fork)
+        with torch.cuda.stream(self.gqa_stream):
+            gqa_step()
         calls[1]()
         calls[2]()
         join = torch.cuda.Event()
-        join.record(gqa_stream)
+        join.record(self.gqa_stream)
         main.wait_event(join)
 
-    def step_in_order(events):
-        for i, c in enumerate(calls):
-            events[i].record()
-            c()
-        events[-1].record()
+    def capture(self, warmup):
+        """The step as one CUDA graph (the launches replay without host overhead, each
+        kernel's set-up overlapping the previous kernel's tail on its stream), and a
+        second graph running the calls in order with an event record around each."""
+        for _ in range(warmup):
+            flush_l2(self.dev)
+            self.step()
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        self.gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(self.calls) + 1)]
+        self.graph_ev = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_ev):
+            for i, c in enumerate(self.calls):
+                self.gev[i].record()
+                c()
+            self.gev[-1].record()
+        for g_ in (self.graph, self.graph_ev):
+            for _ in range(warmup):
+                flush_l2(self.dev)
+                g_.replay()
+        torch.cuda.synchronize()
 
+    def time_steps(self, steps, graph=None):
+        """Per-step device times (ms) of `steps` replays, issued back to back (an L2
+        flush outside each step's event pair), one synchronize at the end."""
+        graph = graph or self.graph
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for e0, e1 in ev:
+            flush_l2(self.dev)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    def time_calls(self, steps):
+        per_call = [[] for _ in self.calls]
+        for _ in range(steps):
+            flush_l2(self.dev)
+            self.graph_ev.replay()
+            torch.cuda.synchronize()
+            for i in range(len(self.calls)):
+                per_call[i].append(self.gev[i].elapsed_time(self.gev[i + 1]))
+        return {n: sum(v) / len(v) for n, v in zip(CALL_NAMES, per_call)}
+
+    def check_device_errors(self):
+        st_a, _ = self.gqla.gqla_read_device_error(self.ba.workspace)
+        st_g, _ = self.gqla.gqla_read_device_error(self.bg.workspace)
+        if st_a or st_g:
+            raise RuntimeError(f"device-side error during the bench ({self.name}): {st_a} {st_g}")
+
+    def e2e(self, steps, warmup):
+        """Host buffers through the C ABI, copies inside the timed region.  Every copy
+        costs ~10 us however small, so the page table and the lengths travel as one
+        int32 buffer, on a second stream while q is copied and the query absorption
+        runs; the GQA path and its output copy run on a third stream beside the absorb
+        path; the step ends when every copy has landed.  Returns (ms, h2d, d2h)."""
+        dev, case, ba, bg = self.dev, self.case, self.ba, self.bg
+        pt_c, sl_c = case["page_table"].cpu(), case["seqlens"].cpu()
+        n_pt = pt_c.numel()
+        q_h = case["q"].cpu().pin_memory()
+        meta_h = torch.cat([pt_c.flatten(), sl_c.flatten()]).pin_memory()
+        outa_h = torch.empty(ba.out.shape, dtype=torch.bfloat16).pin_memory()
+        outg_h = torch.empty(bg.out.shape, dtype=torch.bfloat16).pin_memory()
+        q_e = torch.empty_like(case["q"])
+        meta_d = torch.empty(meta_h.shape, dtype=torch.int32, device=dev)
+        kv_e = self.gqla.make_kv_index(meta_d[:n_pt].view(pt_c.shape), meta_d[n_pt:], case["num_pages"])
+        h2d = q_h.numel() * 2 + meta_h.numel() * 4
+        d2h = outa_h.numel() * 2 + outg_h.numel() * 2
+        calls_e = self.make_calls(q_e, kv_e)
+        gqa_step_e = self.gqa_step_call(q_e, kv_e)
+        side = torch.cuda.Stream(device=dev)
+
+        def e2e_step():
+            main = torch.cuda.current_stream()
+            begin = torch.cuda.Event()
+            begin.record(main)
+            side.wait_event(begin)
+            with torch.cuda.stream(side):
+                meta_d.copy_(meta_h, non_blocking=True)
+            meta_in = torch.cuda.Event()
+            meta_in.record(side)
+            q_e.copy_(q_h, non_blocking=True)
+            calls_e[0]()  # query absorption: needs q only
+            q_in = torch.cuda.Event()
+            q_in.record(main)
+            self.gqa_stream.wait_event(q_in)
+            self.gqa_stream.wait_event(meta_in)
+            with torch.cuda.stream(self.gqa_stream):
+                gqa_step_e()
+                outg_h.copy_(bg.out, non_blocking=True)
+            main.wait_event(meta_in)
+            calls_e[1]()
+            calls_e[2]()
+            outa_h.copy_(ba.out, non_blocking=True)
+            gqa_done = torch.cuda.Event()
+            gqa_done.record(self.gqa_stream)
+            main.wait_event(gqa_done)
+
+        for _ in range(warmup):  # eager warm-up, then the same step as one graph
+            e2e_step()
+        torch.cuda.synchronize()
+        graph_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_e2e):
+            e2e_step()
+        for _ in range(warmup):
+            graph_e2e.replay()
+        torch.cuda.synchronize()
+        times = self.time_steps(steps, graph_e2e)
+        if not torch.equal(outa_h, ba.out.cpu()) or not torch.equal(outg_h, bg.out.cpu()):
+            raise RuntimeError("end-to-end outputs differ from the device results")
+        return sum(times) / len(times), h2d, d2h
+
+    def report(self, mean, world, ms_step=None):
+        """Per-kernel and per-path roofline fractions from the per-call means (ms)."""
+        acc, counts = accounting(self.w, self.case, self.s_q, self.splits["gqa"])
+        acc_a, _ = accounting(self.w, self.case, self.s_q, self.splits["absorb"])
+        acc["decode_absorb"] = acc_a["decode_absorb"]
+        acc["combine_absorb"] = acc_a["combine_absorb"]
+        peaks, peak_kind = _peaks()
+        hbm_peak = float(peaks["hbm_gbs"])
+        tc_peak = float(peaks["bf16_tflops"])
+        tokens_step = self.B * self.s_q
+
+        def roof(name):
+            sec = mean[name] * 1e-3
+            gbs = acc[name]["bytes"] / sec / 1e9
+            tfs = acc[name]["flops"] / sec / 1e12
+            return {"us": mean[name] * 1e3, "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak,
+                    "tflops": tfs, "tensor_frac": tfs / tc_peak}
+
+        per_kernel = {n: roof(n) for n in CALL_NAMES}
+        total = sum(mean.values())
+        for n in CALL_NAMES:
+            per_kernel[n]["share"] = mean[n] / total
+        dominant = max(CALL_NAMES, key=lambda n: mean[n])
+        dk = per_kernel[dominant]
+        t_mem = acc[dominant]["bytes"] / (hbm_peak * 1e9)
+        t_cmp = acc[dominant]["flops"] / (tc_peak * 1e12)
+        if t_cmp > t_mem:
+            roofline = {"bound": "tensor", "achieved": dk["tflops"], "peak": tc_peak,
+                        "unit": "TFLOP/s", "frac": dk["tensor_frac"]}
+        else:
+            roofline = {"bound": "hbm", "achieved": dk["hbm_gbs"], "peak": hbm_peak,
+                        "unit": "GB/s", "frac": dk["hbm_frac"]}
+        roofline.update({"kernel": dominant,
+                         "peak_source": (f"{peak_kind} (MEASURED_PEAKS.json burst)"
+                                         if peak_kind == "measured" else "fallback"),
+                         "algorithmic_bytes_per_launch": acc[dominant]["bytes"],
+                         "algorithmic_flops_per_launch": acc[dominant]["flops"],
+                         "traffic": _stored_traffic(dominant, self.name, self.s_q)})
+
+        def path_info(kernels, dec):
+            us = sum(mean[k] for k in kernels) * 1e3
+            t_m = acc[dec]["bytes"] / (hbm_peak * 1e9)
+            t_c = acc[dec]["flops"] / (tc_peak * 1e12)
+            bound = "tensor" if t_c > t_m else "hbm"
+            frac = (t_c if bound == "tensor" else t_m) / (mean[dec] * 1e-3)
+            return {"us_per_step": us, "tokens_per_s": world * tokens_step / (us * 1e-6),
+                    "decode_kernel": dec, "decode_us": mean[dec] * 1e3, "binding": bound,
+                    "binding_roofline_frac": frac, "hbm_frac": per_kernel[dec]["hbm_frac"],
+                    "tensor_frac": per_kernel[dec]["tensor_frac"]}
+
+        per_path = {"absorb": path_info(["absorb_query", "decode_absorb", "combine_absorb"], "decode_absorb"),
+                    "gqa": path_info(["decode_gqa", "combine_gqa"], "decode_gqa")}
+        return roofline, per_path, per_kernel, acc
+
+    def config(self, world):
+        w = self.w
+        return {"workload": self.name, "num_heads": w.num_heads, "num_groups": w.num_groups,
+                "batch": self.B,
+                "context": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths[1:]),
+                "s_q": self.s_q, "paged": w.paged, "paths": ["absorb", "gqa"],
+                "tokens_per_step": self.B * self.s_q, "num_splits": self.splits,
+                "l2": "flushed (256 MiB write + 256 MiB read) before every timed step",
+                "parallelism": f"replicas x{world} (independent batches per GPU)"}
+
+
+def measure_other_workloads(args, headline, dev):
+    """Every other workload (and s_q) of the suite on this GPU: step time, per-call
+    times and each path's roofline fractions (no end-to-end leg, no CPU baseline)."""
+    from decode_attention_06_b200 import synth
+    out = {}
+    for name, w in synth.WORKLOADS.items():
+        for s in w.s_q:
+            if (name, s) == headline:
+                continue
+            wb = Workbench(name, s, 0, dev, args.splits)
+            wb.time_expand()
+            wb.capture(args.warmup)
+            ms = wb.time_steps(args.steps)
+            mean = wb.time_calls(args.steps)
+            wb.check_device_errors()
+            _, per_path, per_kernel, _ = wb.report(mean, 1)
+            out[f"{name}/sq{s}"] = {
+                "ms_per_step": sum(ms) / len(ms),
+                "tokens_per_s": wb.B * s / (sum(ms) / len(ms) * 1e-3),
+                "num_splits": wb.splits, "per_path": per_path,
+                "per_kernel_us": {n: per_kernel[n]["us"] for n in CALL_NAMES}}
+            del wb
+            torch.cuda.empty_cache()
+    return out
+
+
+def run_tp(args, rank, world, dev):
+    """Group-axis tensor parallelism of the GQA path over the `world` ranks (strong
+    scaling: every rank holds g / world groups of the same batch's expanded cache and
+    decodes its h / world heads; an in-place NCCL all-gather assembles the heads).
+    Each step = the rank's decode + combine + the gather, timed on the device, max
+    over ranks."""
+    from decode_attention_06_b200 import gqla, synth
+    from decode_attention_06_b200.tp import GqaTensorParallel, GroupShard
+    w = synth.WORKLOADS[args.workload]
+    s_q = args.s_q or w.s_q[0]
+    if w.num_groups % world:
+        return {"skipped": f"{w.num_groups} groups do not split over {world} ranks"}
+    case = synth.make_case(w.num_heads, w.num_groups, w.seqlens(), s_q, paged=w.paged,
+                           seed=w.seed, device=str(dev))  # the same batch on every rank
+    shard = GroupShard(w.num_heads, w.num_groups, rank, world)
+    B = case["seqlens"].numel()
+    n_slots = case["num_pages"] * case["page_size"]
+    kv = gqla.make_kv_index(case["page_table"], case["seqlens"], case["num_pages"])
+    splits = args.splits or gqla.plan_splits("gqa", shard.heads, s_q, case["seqlens"].cpu())
+    tp = GqaTensorParallel(shard, B, s_q, splits, dev)
+    kvx = torch.empty(shard.groups, n_slots, 256, dtype=torch.bfloat16, device=dev)
+    kr = torch.empty(n_slots, 64, dtype=torch.bfloat16, device=dev)
+    gqla.gqla_expand_cache(tp.dims, case["latent"], shard.slice_groups(case["w_uk"]),
+                           shard.slice_groups(case["w_uv"]), kvx, kr)
+    q_local = shard.slice_heads(case["q"])
+    del case
+    stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
-        flush_l2()
-        step()
+        flush_l2(dev)
+        tp.step(q_local, kvx, kr, kv)
     torch.cuda.synchronize()
+    torch.distributed.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1, e2 in ev:
+        flush_l2(dev)
+        e0.record(stream)
+        tp.local_step(q_local, kvx, kr, kv)
+        e1.record(stream)
+        tp.gather()
+        e2.record(stream)
+    torch.cuda.synchronize()
+    st, _ = gqla.gqla_read_device_error(tp.bufs.workspace)
+    if st:
+        raise RuntimeError(f"device-side error in the tensor-parallel step: {st}")
+    t = torch.tensor([sum(e0.elapsed_time(e2) for e0, _, e2 in ev) / args.steps,
+                      sum(e0.elapsed_time(e1) for e0, e1, _ in ev) / args.steps],
+                     dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms, local_ms = float(t[0]), float(t[1])
+    return {"scaling": "strong", "ranks": world, "groups_per_rank": shard.groups,
+            "heads_per_rank": shard.heads, "num_splits": splits, "ms_per_step": ms,
+            "local_decode_combine_ms": local_ms, "tokens_per_s": B * s_q / (ms * 1e-3),
+            "gather_bytes_per_rank": tp.out_all.numel() * 2 + tp.lse_all.numel() * 4,
+            "note": "each rank: gqla_decode_gqa + gqla_combine on its groups, then an in-place "
+                    "NCCL all-gather of the heads; device time, max over ranks"}
 
-    # The step is captured into a CUDA graph (the launches replay without host
-    # overhead, each kernel's set-up overlapping the previous kernel's tail on
-    # its stream) for the step time; a second graph runs the calls in order with
-    # an event record around every call for the per-call breakdown.
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step()
-    gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
-    graph_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_ev):
-        step_in_order(gev)
-    for g_ in (graph, graph_ev):
-        for _ in range(args.warmup):
-            flush_l2()
-            g_.replay()
-    torch.cuda.synchronize()
+
+def run_ours(args, rank, world, local_rank):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wb = Workbench(args.workload, args.s_q, rank, dev, args.splits)
+    expand_ms, expand_tc_ms = wb.time_expand()
+    wb.capture(args.warmup)
 
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ms = []
     with ClockSampler(local_rank) as clocks:
-        for k in range(args.steps):
-            flush_l2()  # evict the step's data from L2 (outside the step's events)
-            e0.record(stream)
-            graph.replay()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            step_ms.append(e0.elapsed_time(e1))
+        step_ms = wb.time_steps(args.steps)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     ms_step = sum(step_ms) / args.steps
-    per_call = [[] for _ in calls]
-    for k in range(args.steps):
-        flush_l2()
-        graph_ev.replay()
-        torch.cuda.synchronize()
-        for i in range(len(calls)):
-            per_call[i].append(gev[i].elapsed_time(gev[i + 1]))
-    st_a, _ = gqla.gqla_read_device_error(ba.workspace)
-    st_g, _ = gqla.gqla_read_device_error(bg.workspace)
-    if st_a or st_g:
-        raise RuntimeError(f"device-side error during the bench: {st_a} {st_g}")
-
-    # ---- e2e: host buffers through the C ABI, copies inside the timed region.
-    # Every copy costs ~10 us however small, so the page table and the lengths
-    # travel as one int32 buffer, on a second stream while q is copied and the
-    # query absorption runs; the GQA path and its output copy run on a third
-    # stream beside the absorb path; the step ends when every copy has landed.
-    pt_c, sl_c = case["page_table"].cpu(), case["seqlens"].cpu()
-    n_pt = pt_c.numel()
-    q_h = case["q"].cpu().pin_memory()
-    meta_h = torch.cat([pt_c.flatten(), sl_c.flatten()]).pin_memory()
-    outa_h = torch.empty(ba.out.shape, dtype=torch.bfloat16).pin_memory()
-    outg_h = torch.empty(bg.out.shape, dtype=torch.bfloat16).pin_memory()
-    q_e = torch.empty_like(case["q"])
-    meta_d = torch.empty(meta_h.shape, dtype=torch.int32, device=dev)
-    kv_e = gqla.make_kv_index(meta_d[:n_pt].view(pt_c.shape), meta_d[n_pt:], case["num_pages"])
-    h2d = q_h.numel() * 2 + meta_h.numel() * 4
-    d2h = outa_h.numel() * 2 + outg_h.numel() * 2
-    calls_e = [
-        lambda: gqla.gqla_absorb_query(dims, q_e, case["w_uk"], ba.q_absorbed),
-        lambda: gqla.gqla_decode_absorb(dims, ba.q_absorbed, case["latent"], kv_e, ba.num_splits,
-                                        ba.o_part, ba.lse_part, ba.workspace),
-        lambda: gqla.gqla_combine(dims, kv_e, s_q, ba.num_splits, 512, ba.o_part, ba.lse_part,
-                                  case["w_uv"], ba.out, ba.lse),
-        lambda: gqla.gqla_decode_gqa(dims, q_e, kvx, kr, kv_e, bg.num_splits, bg.o_part,
-                                     bg.lse_part, bg.workspace),
-        lambda: gqla.gqla_combine(dims, kv_e, s_q, bg.num_splits, 128, bg.o_part, bg.lse_part,
-                                  None, bg.out, bg.lse),
-    ]
-    side = torch.cuda.Stream(device=dev)
-    def e2e_step():
-        main = torch.cuda.current_stream()
-        begin = torch.cuda.Event()
-        begin.record(main)
-        side.wait_event(begin)
-        with torch.cuda.stream(side):
-            meta_d.copy_(meta_h, non_blocking=True)
-        meta_in = torch.cuda.Event()
-        meta_in.record(side)
-        q_e.copy_(q_h, non_blocking=True)
-        calls_e[0]()  # query absorption: needs q only
-        q_in = torch.cuda.Event()
-        q_in.record(main)
-        gqa_stream.wait_event(q_in)
-        gqa_stream.wait_event(meta_in)
-        with torch.cuda.stream(gqa_stream):
-            calls_e[3]()
-            calls_e[4]()
-            outg_h.copy_(bg.out, non_blocking=True)
-        main.wait_event(meta_in)
-        calls_e[1]()
-        calls_e[2]()
-        outa_h.copy_(ba.out, non_blocking=True)
-        gqa_done = torch.cuda.Event()
-        gqa_done.record(gqa_stream)
-        main.wait_event(gqa_done)
-
-    for _ in range(args.warmup):  # eager warm-up, then the same step as one graph
-        e2e_step()
-    torch.cuda.synchronize()
-    graph_e2e = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_e2e):
-        e2e_step()
-    for _ in range(args.warmup):
-        graph_e2e.replay()
-    torch.cuda.synchronize()
-    e2e_times = []
-    for k in range(args.steps):
-        flush_l2()
-        e0.record(stream)
-        graph_e2e.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_times.append(e0.elapsed_time(e1))
-    e2e_ms = sum(e2e_times) / args.steps
-    if not torch.equal(outa_h, ba.out.cpu()) or not torch.equal(outg_h, bg.out.cpu()):
-        raise RuntimeError("end-to-end outputs differ from the device results")
+    mean = wb.time_calls(args.steps)
+    wb.check_device_errors()
+    e2e_ms, h2d, d2h = wb.e2e(args.steps, args.warmup)
 
     # ---- max over ranks
-    tokens_step = B * s_q
+    tokens_step = wb.B * wb.s_q
     ms_step, e2e_ms, value, e2e_value = aggregate_over_ranks(ms_step, e2e_ms, world, tokens_step, dev)
-
-    acc, counts = accounting(w, case, s_q, splits["gqa"])
-    acc_a, _ = accounting(w, case, s_q, splits["absorb"])
-    acc["decode_absorb"] = acc_a["decode_absorb"]
-    acc["combine_absorb"] = acc_a["combine_absorb"]
-    mean = {n: sum(v) / len(v) for n, v in zip(names, per_call)}
-    peaks, peak_kind = _peaks()
-    hbm_peak = float(peaks["hbm_gbs"])
-    tc_peak = float(peaks["bf16_tflops"])
-
-    def roof(name):
-        sec = mean[name] * 1e-3
-        gbs = acc[name]["bytes"] / sec / 1e9
-        tfs = acc[name]["flops"] / sec / 1e12
-        return {"us": mean[name] * 1e3, "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak,
-                "tflops": tfs, "tensor_frac": tfs / tc_peak}
-
-    per_kernel = {n: roof(n) for n in names}
-    share = {n: mean[n] / sum(mean.values()) for n in names}
-    dominant = max(names, key=lambda n: mean[n])
-    dk = per_kernel[dominant]
-    t_mem = acc[dominant]["bytes"] / (hbm_peak * 1e9)
-    t_cmp = acc[dominant]["flops"] / (tc_peak * 1e12)
-    if t_cmp > t_mem:
-        roofline = {"bound": "tensor", "achieved": dk["tflops"], "peak": tc_peak,
-                    "unit": "TFLOP/s", "frac": dk["tensor_frac"]}
-    else:
-        roofline = {"bound": "hbm", "achieved": dk["hbm_gbs"], "peak": hbm_peak,
-                    "unit": "GB/s", "frac": dk["hbm_frac"]}
-    roofline.update({"kernel": dominant, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)"
-                     if peak_kind == "measured" else "fallback",
-                     "algorithmic_bytes_per_launch": acc[dominant]["bytes"],
-                     "algorithmic_flops_per_launch": acc[dominant]["flops"],
-                     "traffic": _stored_traffic(dominant, args.workload)})
-
-    def path_info(kernels, dec):
-        us = sum(mean[k] for k in kernels) * 1e3
-        t_m = acc[dec]["bytes"] / (hbm_peak * 1e9)
-        t_c = acc[dec]["flops"] / (tc_peak * 1e12)
-        bound = "tensor" if t_c > t_m else "hbm"
-        frac = (t_c if bound == "tensor" else t_m) / (mean[dec] * 1e-3)
-        return {"us_per_step": us, "tokens_per_s": world * tokens_step / (us * 1e-6),
-                "decode_kernel": dec, "decode_us": mean[dec] * 1e3, "binding": bound,
-                "binding_roofline_frac": frac, "hbm_frac": per_kernel[dec]["hbm_frac"],
-                "tensor_frac": per_kernel[dec]["tensor_frac"]}
-
+    roofline, per_path, per_kernel, acc = wb.report(mean, world)
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 cache/queries, N(0,1/512) bf16 W_UK/W_UV)",
-        "config": {"workload": args.workload, "num_heads": h, "num_groups": g, "batch": B,
-                   "context": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths[1:]),
-                   "s_q": s_q, "paged": w.paged, "paths": ["absorb", "gqa"],
-                   "tokens_per_step": tokens_step, "num_splits": splits,
-                   "l2": "flushed (256 MiB write + 256 MiB read) before every timed step",
-                   "parallelism": f"replicas x{world} (independent batches per GPU)"},
+        "config": wb.config(world),
         "roofline": roofline,
-        "per_path": {"absorb": path_info(["absorb_query", "decode_absorb", "combine_absorb"],
-                                         "decode_absorb"),
-                     "gqa": path_info(["decode_gqa", "combine_gqa"], "decode_gqa")},
-        "per_kernel": {n: dict(per_kernel[n], share=share[n]) for n in names},
-        "expand": {"ms": expand_ms, "slots": n_slots,
+        "per_path": per_path,
+        "per_kernel": per_kernel,
+        "expand": {"ms": expand_ms, "slots": wb.n_slots,
                    "tflops": acc["expand"]["flops"] / (expand_ms * 1e-3) / 1e12,
                    "tc_ms": expand_tc_ms,
                    "tc_tflops": acc["expand"]["flops"] / (expand_tc_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": len(calls) * args.steps,
+        "gpu_launches": wb.launches_per_step() * args.steps,
         "clocks": clocks.summary(),
     }
     if args.sparse_topk:
-        result["sparse"] = run_sparse(args, dims, case, s_q, kvx, kr, kv, flush_l2, hbm_peak)
+        result["sparse"] = run_sparse(args, wb.dims, wb.case, wb.s_q, wb.kvx, wb.kr, wb.kv,
+                                      lambda: flush_l2(dev), float(_peaks()[0]["hbm_gbs"]))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, cores, what = cpu_oracle_rate(case, w, s_q, budget_s=args.cpu_budget)
+        rate, cores, what = cpu_oracle_rate(wb.case, wb.w, wb.s_q, budget_s=args.cpu_budget)
         result["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
                                   "kind": "oracle", "sample": what}
+    if world == 1 and not args.headline_only:
+        headline = (wb.name, wb.s_q)
+        del wb
+        torch.cuda.empty_cache()
+        result["workloads"] = measure_other_workloads(args, headline, dev)
+    if world > 1:
+        del wb
+        torch.cuda.empty_cache()
+        result["tp"] = run_tp(args, rank, world, dev)
     return result
 
 
@@ -700,6 +854,20 @@ def aggregate_over_ranks(ms_step, e2e_ms, world, tokens_per_rank, device):
     return ms_step, e2e_ms, value, e2e_value
 
 
+def _relaunch_under_torchrun(n):
+    """`bench.py --gpus N` (N > 1) started outside torchrun: run the same command as
+    N ranks, one process per GPU, and pass on their exit status."""
+    import socket
+    import subprocess
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -711,6 +879,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="measure the headline workload only (not the rest of the suite)")
     ap.add_argument("--sparse-topk", type=int, default=0,
                     help="also time sparse GQLA with this many selected positions per query token")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
@@ -721,8 +891,15 @@ def main():
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1 and args.impl == "ours":
+        sys.exit(_relaunch_under_torchrun(args.gpus))
+    world = int(env_world or "1")
+    if args.impl == "ours" and world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {world}: launch one rank per GPU")
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 

@@ -41,6 +41,9 @@ struct CombineParams {
     int heads;
     int G;         // heads per group
     int bs_total;  // batch * s_q
+    // leave alone the sequences with exactly one partial: the decode wrote their final
+    // output itself
+    int skip_single;
 };
 
 // One full warp: chunk range [c0, c1) of the sequences of the (sequence,
@@ -112,9 +115,11 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
     const int q_first = blockIdx.x * kQuadsPerBlock;
     const int bs_lo = q_first / quads_per_pair;
     const int n_pairs = (q_first + kQuadsPerBlock - 1) / quads_per_pair - bs_lo + 1;
-    griddep_wait();  // the previous kernel's results are visible from here on
-    griddep_launch_dependents();
+    // The split plan reads only the lengths, which the decode before this kernel read
+    // itself after its own wait for its predecessor: it runs while the decode finishes.
     if (warp == 0) plan_pairs(p, bs_lo, n_pairs, s_c0, s_c1);
+    griddep_wait();  // the decode's partials are visible from here on
+    griddep_launch_dependents();
     __syncthreads();
 
     const int quad = q_first + warp;
@@ -123,6 +128,7 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
     const int h0 = (quad % quads_per_pair) * 4;
     const int b = bs / p.s_q, s = bs % p.s_q;
     const int c0 = s_c0[bs - bs_lo], nparts = s_c1[bs - bs_lo] - c0;
+    if (p.skip_single && nparts == 1) return;
     // partial (b, c) row of head h: ((b + c) * s_q + s) * heads + h
     const int64_t row0 = ((int64_t)(b + c0) * p.s_q + s) * p.heads + h0;
     const int64_t part_stride = (int64_t)p.s_q * p.heads;
@@ -271,8 +277,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    griddep_wait();  // the previous kernel's results are visible from here on
-    griddep_launch_dependents();
+    // W_UV_g and the split plan (from the lengths) do not depend on the decode before
+    // this kernel, which read the same lengths after its own wait: both start while the
+    // decode finishes (the barrier init above is ordered before the TMA by fence and sync)
+    __syncthreads();
     if (tid == 0) {
         if (leader) {
             prefetch_tensormap(&wmap);
@@ -290,6 +298,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     if (warp == 2) {
         plan_pairs(p, bs0, bst, s_c0, s_c1);
     }
+    griddep_wait();  // the decode's partials are visible from here on
+    griddep_launch_dependents();
     tc_fence_before();
     cluster_sync();  // barriers of both CTAs initialised before any remote transfer
     tc_fence_after();
@@ -516,10 +526,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
 
 cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int d_in,
                            const float *o_part, const float *lse_part, const void *w_uv,
-                           void *out, float *lse_out, int heads, int num_groups,
+                           void *out, float *lse_out, int heads, int num_groups, bool skip_single,
                            cudaStream_t stream) {
     CombineParams p{o_part, lse_part, kv->seqlens, static_cast<__nv_bfloat16 *>(out), lse_out,
-                    kv->batch, num_splits, s_q, heads, heads / num_groups, kv->batch * s_q};
+                    kv->batch, num_splits, s_q, heads, heads / num_groups, kv->batch * s_q,
+                    skip_single ? 1 : 0};
     if (d_in == kDv) {
         const int64_t quads = (int64_t)p.bs_total * (heads / 4);
         return launch_dependent(combine_v_kernel,

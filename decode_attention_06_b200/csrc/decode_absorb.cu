@@ -12,7 +12,7 @@
 // CTA streams only its 288 columns of every cache row (the pair reads each
 // byte of the cache exactly once) and computes a partial score tile over
 // them.  The softmax rows are split too: row i of the block belongs to rank
-// (i / 16) % 2.  Each CTA sends the peer the fp16 partials of the peer's rows,
+// (i / 16) % 2.  Each CTA sends the peer the fp32 partials of the peer's rows,
 // adds the two partials of its own 64 rows, computes their P (bf16) and sends
 // those P rows, with each row's O rescale factor, back; both CTAs then hold P
 // for all 128 rows and each accumulates its own 256 columns of O.
@@ -21,27 +21,30 @@
 //    N up to 64).  Tensor memory holds O (256 columns), a double-buffered S
 //    (2 x 64) and the latent half of q~ (128 columns of bf16 pairs: the score
 //    MMA reads q~ from TMEM); P goes through shared memory, beside a 4-slot
-//    ring of cache tiles.
+//    ring of latent tiles and a 2-slot ring of RoPE tiles (the RoPE columns
+//    are read by the score MMAs only, so their slot frees a whole PV earlier).
 //  * Roles, 19 warps:
-//      warp 0      TMA producer of the ring (4 latent boxes 128B-swizzled + 1 RoPE
-//                  box 64B-swizzled, 36 KB per tile), cache tiles read with an L2
-//                  evict-first policy;
+//      warp 0      TMA producer of the rings (4 latent boxes 128B-swizzled, 32 KB,
+//                  and 1 RoPE box 64B-swizzled, 4 KB, per tile), cache tiles read
+//                  with an L2 evict-first policy;
 //      warp 1      TMEM owner, issues S = q~ C^T;
 //      warps 2-9   score warps, two per TMEM lane quadrant, 32 tokens each.  Stage A
-//                  of tile j: scores -> fp16; the block of the CTA's own rows goes
-//                  into its receive buffer, the block of the peer's rows leaves as
-//                  one 1 KB bulk copy.  Stage C of tile j - 1: once P of all rows is
-//                  in, O rows whose maximum rose are rescaled and PV is released.
-//                  Also each piece's RoPE q~ (by TMA, as soon as the previous
-//                  piece's scores are complete) and the epilogue;
+//                  of tile j: the fp32 partial scores of the CTA's own rows go to its
+//                  local buffer, those of the peer's rows to a staging block that
+//                  leaves as one 2 KB bulk copy per warp into the peer's receive buffer.
+//                  Stage C of tile j - 1: once P of all rows is in, O rows whose
+//                  maximum rose are rescaled and PV is released.  Also each piece's
+//                  RoPE q~ (by TMA, as soon as the previous piece's scores are
+//                  complete) and the epilogue;
 //      warps 10-17 softmax warps of the CTA's 64 rows (stage B), four lanes per
-//                  row: partials added, row maxima (lazy rescaling: a maximum has
-//                  to rise by more than 2^8), P = 2^(s - m) written to both CTAs'
-//                  P buffers (bulk copy of each warp's 8 rows); also the q~ copies
-//                  into TMEM, each piece's next q~ prefetched into L2;
+//                  row: the two fp32 partials added, row maxima (lazy rescaling: a
+//                  maximum has to rise by more than 2^8), P = 2^(s - m) written to
+//                  both CTAs' P buffers (bulk copy of each warp's 8 rows); also the
+//                  q~ copies into TMEM, each piece's next q~ prefetched into L2;
 //      warp 18     issues O += P C in tile order.
 //    The stages of consecutive tiles overlap: the score warps run A(j) while the
-//    softmax warps run B(j - 1).
+//    softmax warps run B(j - 1).  Every score is the fp32 sum of two fp32
+//    partials: no precision is given up in the exchange.
 //  * The epilogue writes O / l with TMA stores of 32 x 32 fp32 boxes staged in
 //    shared memory: in the idle ring after the last piece, in the P buffers
 //    between pieces.
@@ -49,13 +52,14 @@
 //    both CTAs of a cluster always execute the same sequence of steps.
 #include <cudaTypedefs.h>
 
-#include <cuda_fp16.h>
-
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tensor_map.cuh"
 
 namespace gqla {
+
+// Set by gqla_debug_drop_v_load, consumed by the next decode launch of the thread.
+extern thread_local int g_drop_v_unit;
 
 namespace {
 
@@ -79,33 +83,51 @@ struct AbsorbSmem {
     static constexpr int kQRope = kRows * 64;             // q~ RoPE columns [128 rows][32]
     static constexpr int kLatBox = kT * 128;              // [64 tokens][64 cols]
     static constexpr int kRopeBox = kT * 64;              // [64 tokens][32 cols]
-    static constexpr int kSlot = 4 * kLatBox + kRopeBox;  // 36 KB
-    // partial scores of this CTA's 64 rows, fp16, in 1 KB blocks
-    // [2 sources][2 token halves][4 lane quadrants][16 rows][32 tokens]: one block is what
-    // one score warp computes for the rows of one owner, so the peer's blocks arrive as
-    // whole bulk copies; 16-byte chunks of a block row XOR-swizzled by (row / 2) % 4
-    static constexpr int kXBlock = 16 * 64;
-    static constexpr int kX = 2 * kOwn * kT * 2;
-    static constexpr int kXRemote = kOwn * kT * 2;
+    static constexpr int kSlot = 4 * kLatBox;             // latent ring slot, 32 KB
+    static constexpr int kRopeRing = 2;
+    // fp32 partial scores of this CTA's 64 rows in two token halves, [2][64 rows][32
+    // tokens]: a half row is 128 bytes, eight 16-byte chunks stored at xoff(); the 16 rows
+    // of one lane quadrant in one half are what one score warp computes, 2 KB in one piece,
+    // so the peer's blocks arrive as whole bulk copies.  Read 16 tokens per lane (four
+    // lanes per row).  One buffer for this CTA's partials and one for the peer's: the
+    // softmax warps of both CTAs read tile j at the start of their stage B, before either
+    // CTA's score warps write tile j + 1 (which waits for that).
+    static constexpr int kX = kOwn * kT * 4;
+    static constexpr int kXBlock = 16 * 32 * 4;           // one score warp's block, 2 KB
     static constexpr int kP = kRows * kT * 2;             // P, [128 rows][64 tokens] bf16, 128B-swizzled
     // the peer's 64 rows of P (bulk copies) and their O rescale factors (st.async)
     static constexpr int kPRemote = kOwn * kT * 2 + kOwn * 4;
     static constexpr int oQ = 0;
     static constexpr int oP = oQ + kQRope;                // 2 buffers
     static constexpr int oRing = oP + 2 * kP;
-    static constexpr int oX = oRing + kRing * kSlot;      // 2 buffers
-    static constexpr int oXStage = oX + 2 * kX;           // [8 score warps] outgoing blocks
+    static constexpr int oRope = oRing + kRing * kSlot;   // kRopeRing RoPE tiles
+    static constexpr int oXR = oRope + kRopeRing * kRopeBox;  // the peer's partials
+    static constexpr int oXL = oXR + kX;                      // this CTA's partials
+    static constexpr int oXStage = oXL + kX;              // [8 score warps] outgoing blocks
     static constexpr int oAlpha = oXStage + kXWarps * kXBlock;  // float [2 buffers][128 rows]
     static constexpr int oL = oAlpha + 2 * kRows * 4;     // float [128 rows]: row sums of a piece
     static constexpr int oBar = oL + kRows * 4;
-    // ring_full/empty[kRing], q_full, s_full/s_free[2], x_full/x_empty[2],
-    // p_full/p_empty[2], o_ready[2], pv_done[2], l_full, o_done, drain[2]
-    static constexpr int kNumBars = 2 * kRing + 1 + 4 + 4 + 4 + 2 + 2 + 1 + 1 + 2;
+    // ring_full/empty[kRing], rope_full/empty[kRopeRing], q_full, s_full/s_free[2],
+    // x_full, x_empty, p_full/p_empty[2], o_ready[2], pv_done[2], l_full, o_done, drain[2]
+    static constexpr int kNumBars = 2 * kRing + 2 * kRopeRing + 1 + 4 + 2 + 4 + 2 + 2 + 1 + 1 + 2;
     static constexpr int oMisc = oBar + kNumBars * 8;     // tmem base, abort, plan[4]
     static constexpr int kBytes = oMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;
 };
 static_assert(AbsorbSmem::kAlloc <= 227 * 1024, "shared memory");
+static_assert(AbsorbSmem::oRing % 1024 == 0 && AbsorbSmem::oRope % 512 == 0 && AbsorbSmem::oP % 1024 == 0,
+              "swizzle atoms of the MMA operands");
+// the last piece's epilogue stages every score warp's 32 x 128 fp32 block in the idle ring
+static_assert(kXWarps * 32 * kXCols * 4 <= kRing * AbsorbSmem::kSlot, "epilogue staging");
+
+// Byte offset of logical chunk c (tokens 4c .. 4c + 3, c < 16) of partial-score row r in a
+// partial buffer: token half c / 8, then the row, then the chunk, XOR-swizzled so that both
+// a lane writing the eight chunks of its half row (8 rows a phase, one chunk each) and four
+// lanes reading four chunks of one row (two rows a phase) meet no bank conflict.
+__device__ __forceinline__ int xoff(int r, int c) {
+    const int x = c >> 3;
+    return x * (kOwn * 128) + r * 128 + (((c & 7) ^ (r & 7) ^ (x << 1)) << 4);
+}
 
 struct AbsorbParams {
     const int32_t *page_table;
@@ -118,6 +140,9 @@ struct AbsorbParams {
     int rows_total;   // s_q * heads: query rows of one sequence
     int row_blocks;   // ceil(rows_total / 128)
     float scale_log2;
+    // diagnostic: the latent load of this tile (issue order within a CTA) is never issued,
+    // so a bounded wait runs out (-1: none)
+    int drop_tile;
 };
 
 struct PieceIter {
@@ -161,10 +186,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::oBar);
     uint64_t *ring_full = bars, *ring_empty = bars + kRing;
-    uint64_t *q_full = bars + 2 * kRing;
+    uint64_t *rope_full = bars + 2 * kRing, *rope_empty = rope_full + SM::kRopeRing;
+    uint64_t *q_full = rope_empty + SM::kRopeRing;
     uint64_t *s_full = q_full + 1, *s_free = s_full + 2;
-    uint64_t *x_full = s_free + 2, *x_empty = x_full + 2;
-    uint64_t *p_full = x_empty + 2, *p_empty = p_full + 2;
+    uint64_t *x_full = s_free + 2, *x_empty = x_full + 1;
+    uint64_t *p_full = x_empty + 1, *p_empty = p_full + 2;
     uint64_t *o_ready = p_empty + 2, *pv_done = o_ready + 2;
     uint64_t *l_full = pv_done + 2, *o_done = l_full + 1, *drain = o_done + 1;
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(smem + SM::oMisc);
@@ -182,11 +208,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i) { mbar_init(&ring_full[i], 1); mbar_init(&ring_empty[i], 1); }
+        for (int i = 0; i < SM::kRopeRing; ++i) { mbar_init(&rope_full[i], 1); mbar_init(&rope_empty[i], 1); }
         mbar_init(q_full, 1 + kYWarps);  // RoPE TMA + the softmax warps' TMEM copies
+        mbar_init(x_full, 1 + kXWarps);  // expect_tx of the peer's partials + local score warps
+        mbar_init(x_empty, 2 * kYWarps); // every softmax warp of both CTAs has read both buffers
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1); mbar_init(&s_free[i], kXThreads);
-            mbar_init(&x_full[i], 1 + kXWarps);      // expect_tx of the peer's half + local score warps
-            mbar_init(&x_empty[i], 2 * kYWarps);     // every softmax warp of both CTAs has read it
             mbar_init(&p_full[i], 1 + kYWarps);      // expect_tx of the peer's rows + local softmax warps
             mbar_init(&p_empty[i], 2);               // PV of both CTAs done with the buffer
             mbar_init(&o_ready[i], kXWarps);
@@ -267,19 +294,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (lane == 0) {
                         const bool bad = page < 0 || page >= p.num_pages;
                         if (bad && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
-                        const int slot = t % kRing;
+                        const int slot = t % kRing, rs = t % SM::kRopeRing;
                         if (!GQLA_WAIT(0, &ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                         uint8_t *dst = smem + SM::oRing + slot * SM::kSlot;
-                        if (!bad && !*abort_flag) {
+                        if ((int)t == p.drop_tile) {
+                            // diagnostic: neither the load nor an arrival for this tile
+                        } else if (!bad && !*abort_flag) {
                             mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
 #pragma unroll
                             for (int bx = 0; bx < 4; ++bx)
                                 tma_load_2d_hint(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
                                                  256 * rank + 64 * bx, page * kPage, stream_policy);
-                            tma_load_2d_hint(dst + 4 * SM::kLatBox, &rope_map, &ring_full[slot], 512 + 32 * rank,
-                                             page * kPage, stream_policy);
                         } else {
                             mbar_arrive(&ring_full[slot]);
+                        }
+                        // the RoPE slot frees once the score MMAs of tile t - kRopeRing are done
+                        if (!GQLA_WAIT(1, &rope_empty[rs], ((t / SM::kRopeRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                        if (!bad && !*abort_flag) {
+                            mbar_arrive_expect_tx(&rope_full[rs], SM::kRopeBox);
+                            tma_load_2d_hint(smem + SM::oRope + rs * SM::kRopeBox, &rope_map, &rope_full[rs],
+                                             512 + 32 * rank, page * kPage, stream_policy);
+                        } else {
+                            mbar_arrive(&rope_full[rs]);
                         }
                     }
                 }
@@ -292,6 +328,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
             for (uint32_t u = (t > (uint32_t)kRing ? t - kRing : 0); u < t; ++u)
                 mbar_wait(&ring_full[u % kRing], (u / kRing) & 1, no_abort);
+            for (uint32_t u = (t > (uint32_t)SM::kRopeRing ? t - SM::kRopeRing : 0); u < t; ++u)
+                mbar_wait(&rope_full[u % SM::kRopeRing], (u / SM::kRopeRing) & 1, no_abort);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- score MMA issuer
@@ -300,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // descriptors of ring slot 0 and of the RoPE q~; a single issuing thread pays
             // for every instruction of a descriptor, so each MMA only adds an offset
             const uint64_t lat_d0 = smem_desc(sm_ring, 16, 1024, kSw128);
-            const uint64_t rope_d0 = smem_desc(sm_ring + 4 * SM::kLatBox, 16, 512, kSw64);
+            const uint64_t rope_d0 = smem_desc(smem_u32(smem + SM::oRope), 16, 512, kSw64);
             const uint64_t q_d0 = smem_desc(sm_q, 16, 512, kSw64);
             PieceIter it = it0;
             int b, L, pb, pe;
@@ -310,12 +348,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (too_long) continue;
                 if (!GQLA_WAIT(2, q_full, k & 1, abort_flag)) *abort_flag = 1;
                 for (int i = 0; i < pe - pb; ++i, ++t) {
-                    const int slot = t % kRing, sb = t & 1;
+                    const int slot = t % kRing, sb = t & 1, rs = t % SM::kRopeRing;
                     if (!GQLA_WAIT(3, &ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(3, &rope_full[rs], (t / SM::kRopeRing) & 1, abort_flag)) *abort_flag = 1;
                     if (!GQLA_WAIT(4, &s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
                     const uint64_t lat_d = desc_advance(lat_d0, slot * SM::kSlot);
-                    const uint64_t rope_d = desc_advance(rope_d0, slot * SM::kSlot);
+                    const uint64_t rope_d = desc_advance(rope_d0, rs * SM::kRopeBox);
                     const uint32_t t_sb = t_s + sb * kT;
                     if (!*abort_flag) {
 #pragma unroll
@@ -327,6 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             mma_bf16(t_sb, desc_advance(q_d0, ks * 32), desc_advance(rope_d, ks * 32), idesc_s, 1u);
                     }
                     mma_commit(&s_full[sb]);
+                    mma_commit(&rope_empty[rs]);
                 }
                 ++k;
             }
@@ -372,8 +412,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp < 2 + kXWarps) {
         // ---------------------------------------------------------------- score warps
-        // Stage A of tile j: scores -> fp16 -> the owner of each row (row r of the block
-        // belongs to rank (r / 16) % 2, so both CTAs use all four TMEM lane quadrants);
+        // Stage A of tile j: fp32 partial scores -> the owner of each row (row r of the
+        // block belongs to rank (r / 16) % 2, so both CTAs use all four TMEM lane quadrants);
         // stage C of tile j - 1: once P and the rescale factors of all 128 rows are in,
         // O rows are rescaled where a row maximum rose and PV is released.  Also the q~
         // copies into TMEM and the epilogue.  Two warps per lane quadrant: warp half
@@ -387,8 +427,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t a_owner = (lane >> 4) & 1;   // the owner of this row (stage A)
         const float *alph = reinterpret_cast<const float *>(smem + SM::oAlpha);
         const float *lsm = reinterpret_cast<const float *>(smem + SM::oL);
-        const uint32_t x_remote = map_peer(smem_u32(smem + SM::oX), peer);
+        const uint32_t x_remote = map_peer(smem_u32(smem + SM::oXR), peer);
         const uint32_t xfull_remote = map_peer(smem_u32(x_full), peer);
+        // this lane's row among the owner's 64 rows, and its eight chunks (32 tokens)
+        const int xrow = 16 * quad + (lane & 15);
         const bool quad_live = 32 * quad < rows_here;  // rows_here is a multiple of 32
         // the first two tiles' P buffers expect the peer's rows
         if (xw == 0 && lane == 0) {
@@ -429,37 +471,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&s_free[sb]);
-                uint32_t h2[kXTok / 2];
-#pragma unroll
-                for (int j = 0; j < kXTok / 2; ++j) {
-                    __half2 v = __floats2half2_rn(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
-                    h2[j] = *reinterpret_cast<uint32_t *>(&v);
-                }
-                // receive buffers sb of both CTAs are free once tile tt - 2 has been read
-                if (!GQLA_WAITC(7, &x_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                if (xw == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[sb], SM::kXRemote);
-                // this warp's block for each owner: rows 16 quad .. 16 quad + 15 of the owner,
-                // tokens 32 xpart .. 32 xpart + 31; the peer's block goes out by bulk copy
-                const uint32_t blk = (((rank * 2 + xpart) * 4 + quad) * SM::kXBlock);
-                uint8_t *dst = a_owner == rank ? smem + SM::oX + sb * SM::kX + blk : smem + SM::oXStage + xw * SM::kXBlock;
-                const int r16 = lane & 15;
+                // both buffers (this CTA's, and the peer's receive buffer) are free once the
+                // softmax warps of both CTAs have read tile tt - 1
+                if (!GQLA_WAITC(7, x_empty, (tt & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                if (xw == 0 && lane == 0) mbar_arrive_expect_tx(x_full, SM::kX);
+                // this lane's row, tokens 32 xpart .. 32 xpart + 31: the CTA's own rows into the
+                // local buffer, the peer's rows into this warp's staging block (the peer's half
+                // rows 16 quad .. 16 quad + 15), which leaves as one bulk copy
                 if (tt > 0) {
                     // the previous tile's outgoing block has been read by its bulk copy
                     if (lane == 0) bulk_wait_group_read<0>();
                     __syncwarp();
                 }
+                // (the staging block holds the same 16 half rows as their place in the peer's
+                // buffer, at the offset of row 16 quad of half xpart there)
+                const int base = a_owner == rank ? SM::oXL
+                                                 : SM::oXStage + xw * SM::kXBlock - xpart * (kOwn * 128) - 16 * quad * 128;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(dst + r16 * 64 + ((q ^ ((r16 >> 1) & 3)) << 4)) =
-                        make_uint4(h2[4 * q], h2[4 * q + 1], h2[4 * q + 2], h2[4 * q + 3]);
-                fence_proxy_async_smem();  // the outgoing block -> the bulk copy (async proxy)
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4 *>(smem + base + xoff(xrow, 8 * xpart + j)) =
+                        make_uint4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+                fence_proxy_async_smem();  // the staging block -> the bulk copy (async proxy)
                 __syncwarp();
                 if (lane == 0) {
-                    bulk_copy_to_peer(x_remote + sb * SM::kX + blk, smem + SM::oXStage + xw * SM::kXBlock,
-                                      SM::kXBlock, xfull_remote + sb * 8);
+                    bulk_copy_to_peer(x_remote + xpart * (kOwn * 128) + 16 * quad * 128,
+                                      smem + SM::oXStage + xw * SM::kXBlock, SM::kXBlock, xfull_remote);
                     bulk_commit_group();
+                    mbar_arrive(x_full);  // this warp's local partials are in
                 }
-                if (lane == 0) mbar_arrive(&x_full[sb]);  // this warp's local partials are in
                 GQLA_SPAN_END(13, t_a);
             };
             auto stage_c = [&](int i, int page) {
@@ -658,38 +697,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const bool bad = page < 0 || page >= p.num_pages;
                 const int n_valid = bad ? 0 : max(0, min(kT, L - tok0));
                 GQLA_SPAN_BEGIN(t_b0);
-                if (!GQLA_WAITC(8, &x_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
+                if (!GQLA_WAITC(8, x_full, tt & 1, abort_flag)) *abort_flag = 1;
                 GQLA_SPAN_BEGIN(t_b);
-                // this row's block from each source (token half bq4 / 2), chunks 2 (bq4 % 2), +1
-                const int bxp = bq4 >> 1, bq = ob >> 4, br = ob & 15;
-                uint4 u[2][2];
-#pragma unroll
-                for (int src2 = 0; src2 < 2; ++src2) {
-                    const uint8_t *blkp = smem + SM::oX + sb * SM::kX + (((src2 * 2 + bxp) * 4 + bq) * SM::kXBlock) + br * 64;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        u[src2][h] = *reinterpret_cast<const uint4 *>(blkp + (((2 * (bq4 & 1) + h) ^ ((br >> 1) & 3)) << 4));
-                }
-                // full scores = the two fp16 partials added in fp32 (one fp16 rounding per
-                // partial; an fp16 sum would add a third)
+                // this row's tokens 16 bq4 .. 16 bq4 + 15 from both partials (fp32), added in fp32
                 float x[16];
+                {
+                    const uint8_t *xl = smem + SM::oXL;
+                    const uint8_t *xr = smem + SM::oXR;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t a4[4] = {u[0][h].x, u[0][h].y, u[0][h].z, u[0][h].w};
-                    const uint32_t b4[4] = {u[1][h].x, u[1][h].y, u[1][h].z, u[1][h].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 fa = __half22float2(*reinterpret_cast<const __half2 *>(&a4[e]));
-                        const float2 fb = __half22float2(*reinterpret_cast<const __half2 *>(&b4[e]));
-                        x[8 * h + 2 * e] = fa.x + fb.x;
-                        x[8 * h + 2 * e + 1] = fa.y + fb.y;
+                    for (int h = 0; h < 4; ++h) {
+                        const int off = xoff(ob, 4 * bq4 + h);
+                        const float4 a = *reinterpret_cast<const float4 *>(xl + off);
+                        const float4 r = *reinterpret_cast<const float4 *>(xr + off);
+                        x[4 * h] = a.x + r.x;
+                        x[4 * h + 1] = a.y + r.y;
+                        x[4 * h + 2] = a.z + r.z;
+                        x[4 * h + 3] = a.w + r.w;
                     }
                 }
                 __syncwarp();
-                // both CTAs' buffers sb may be refilled once every softmax warp has read them
+                // both CTAs' buffers may be refilled once every softmax warp of the pair has
+                // read them
                 if (lane == 0) {
-                    mbar_arrive(&x_empty[sb]);
-                    mbar_arrive_remote_relaxed(xempty_remote + sb * 8);
+                    mbar_arrive(x_empty);
+                    mbar_arrive_remote(xempty_remote);
                 }
                 // mask tokens past the sequence or past this query's causal limit
                 const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + 16 * bq4);
@@ -771,10 +802,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     GQLA_PROF_FLUSH;
     __syncthreads();
-    if (*abort_flag && threadIdx.x == 0) report_error(p.ws, GQLA_ERR_TIMEOUT, c);
+    if (*abort_flag && threadIdx.x == 0) {
+        report_error(p.ws, GQLA_ERR_TIMEOUT, c);
+        st_cluster_b32(map_peer(smem_u32(const_cast<int *>(abort_flag)), peer), 1u);  // tell the peer
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+    // Every step of the pair ran in both CTAs: if neither gave up, every byte either one
+    // sent (partial scores, P rows, rescale factors, row sums) was waited for by the
+    // other, so nothing is in flight here.  A CTA that gave up ran on without waiting and
+    // may have left asynchronous stores and bulk copies to its peer in flight; once the
+    // first barrier has told both CTAs, both wait about 100 us (those copies take
+    // microseconds) before the second barrier lets either exit.
+    cluster_sync();
+    if (*abort_flag) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < 200000) __nanosleep(1000);
     }
     cluster_sync();  // no remote access may target a CTA that has exited
 }
@@ -826,6 +871,8 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
     p.rows_total = s_q * heads;
     p.row_blocks = (p.rows_total + kRows - 1) / kRows;
     p.scale_log2 = scale * kLog2e;
+    p.drop_tile = g_drop_v_unit;
+    g_drop_v_unit = -1;
     cudaError_t e = cudaFuncSetAttribute(decode_absorb_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, AbsorbSmem::kAlloc);
     if (e != cudaSuccess) return e;

@@ -45,7 +45,25 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 352;        // warp 0 TMA, warp 1 score MMA, warps 2-9 softmax, warp 10 PV MMA
+// warp 0 TMA, warp 1 score MMA, warp 2 PV MMA, warp 3 idle (warpgroup 0); warps 4-11 softmax
+// (warpgroups 1 and 2)
+constexpr int kThreads = 384;
+// Register split by setmaxnreg: warpgroup 0 only issues copies and MMAs, the softmax
+// warpgroups hold a unit's scores, probabilities and running maxima (3 x NQ values per
+// thread).  The launch gives every thread kLaunchRegs (the count ptxas reports under
+// these launch bounds, checked on the host before every launch); the split must not
+// ask for more in all than the launch gave, or the increase would wait forever.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsIssue = 56;
+constexpr int kRegsSoftmax = 224;
+static_assert(128 * kRegsIssue + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
+
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIssue));
+}
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+}
 constexpr int kTok = 128;            // tokens per unit (two pages)
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kBox = 64 * 64 * 2;    // one 64-row x 64-column bf16 TMA box (8 KB)
@@ -84,7 +102,16 @@ struct GqaParams {
     float *lse_part;
     void *ws;
     int batch, max_pages, num_pages, num_splits, s_q, heads, G;
-    int NG;  // KV groups g: 8, or 4 (the (g, s_q) = (4, 1) configuration's 2176-byte tokens)
+    // KV groups of one CTA: the cache's g (8, 4 at the (g, s_q) = (4, 1) configuration's
+    // 2176-byte tokens, 2 or 1 for a rank's share of 8 groups under group-axis tensor
+    // parallelism), or g / gridDim.y when the groups are split over gridDim.y CTAs per
+    // chunk (small batches); CTA (c, y) takes groups [y NG, y NG + NG)
+    int NG;
+    // final outputs for the sequences whose pages all fall in one chunk (their partial is
+    // the result): out bf16 [batch][s_q][heads][128], lse_out fp32 (may be null); null out:
+    // partials only
+    __nv_bfloat16 *out;
+    float *lse_out;
     float scale_log2;
     // sparse mode: the "pages" are those of a selection (identity page table, lengths =
     // selected rows per query token); row r of selected page P is cache slot sel_slot[64 P + r]
@@ -117,6 +144,14 @@ __device__ __forceinline__ bool next_piece(const GqaParams &p, PieceIter &it, in
     return false;
 }
 
+// Warpgroup w takes the units of the groups gi = w, w + 2, ...: with an even group count
+// unit u (u = pair * NG + gi) belongs to warpgroup u % 2 and is its (u / 2)-th unit; with
+// one group every unit is warpgroup 0's.
+__device__ __forceinline__ uint32_t wg_unit(uint32_t u, int ng) { return ng == 1 ? u : u >> 1; }
+
+// Groups of warpgroup wg: ceil(NG / 2) for warpgroup 0, floor(NG / 2) for warpgroup 1.
+__device__ __forceinline__ int wg_groups(int ng, int wg) { return (ng + 1 - wg) >> 1; }
+
 // The two pages of a unit and how many of their rows are real tokens.
 struct PagePair {
     int page0, page1;  // -1: missing (past the piece) or outside the pool
@@ -147,7 +182,7 @@ __device__ __forceinline__ PagePair load_pair(const GqaParams &p, int b, int L, 
 struct UnitCursor {
     PieceIter it;
     int b, L, pg, pe, gi;
-    int n0, n1;  // page indices of the pair after this one (valid from gi == NG / 2)
+    int n0, n1;  // page indices of the pair after this one (valid from gi == (NG + 1) / 2)
     PagePair pp;
     bool valid;
     __device__ __forceinline__ bool next_valid_piece(const GqaParams &p) {
@@ -168,7 +203,7 @@ struct UnitCursor {
     }
     __device__ __forceinline__ void advance(const GqaParams &p) {
         ++gi;
-        if (gi == p.NG / 2 && pg + 2 < pe) {
+        if (gi == (p.NG + 1) / 2 && pg + 2 < pe) {
             const int32_t *row = p.page_table + (int64_t)b * p.max_pages;
             n0 = row[pg + 2];
             n1 = pg + 3 < pe ? row[pg + 3] : 0;
@@ -291,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
+    const int gbase = blockIdx.y * p.NG;  // this CTA's first group
     const int real_cols = p.G * p.s_q;
 
     if (threadIdx.x == 0) {
@@ -343,337 +379,345 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sm_kr = smem_u32(smem + SM::oKr);
     const uint32_t sm_p = smem_u32(smem + SM::oP);
 
-    if (warp == 0 && SPARSE) {
-        // ---------------------------------------------------------------- TMA producer, sparse
-        // The same units and rings as below; the rows of a unit are gathered four at a
-        // time (tile::gather4): lane l takes rows 4 (l % 16) .. + 3 of page l / 16 of the
-        // unit's pair, for K_nope_g, V_g and the pair's RoPE keys.  Lane 0 waits for
-        // the slots and sets each barrier's byte count before the warp issues.
-        if (lane == 0) {
-            prefetch_tensormap(&kv_rows_map);
-            prefetch_tensormap(&kr_rows_map);
-            prefetch_tensormap(&q_map);
-        }
-        const uint32_t q_bytes = 3u * 128u * (uint32_t)real_cols;
-        const uint64_t stream_policy = l2_evict_first_policy();
-        const int half = lane >> 4, r0 = 4 * (lane & 15);
-        UnitCursor kc, vc;
-        kc.start(p, it0);
-        vc.start(p, it0);
-        uint32_t kpos = 0, vpos = 0, pc = 0;
-        int4 ksl = make_int4(-1, -1, -1, -1), vsl = ksl;  // this lane's four cache slots
-        auto pair_slots = [&](const UnitCursor &cur) {
-            const int page = half ? cur.pp.page1 : cur.pp.page0;
-            return page < 0 ? make_int4(-1, -1, -1, -1)
-                            : *reinterpret_cast<const int4 *>(p.sel_slot + (int64_t)page * kPage + r0);
-        };
-        auto row_of = [&](int slot, int gi) { return slot < 0 ? -1 : gi * p.real_slots + slot; };
-        long long idle_since = clock64();
-        while (kc.valid || vc.valid) {  // warp-uniform: every decision is lane 0's, broadcast
-            bool progressed = false;
-            const int aborted = __shfl_sync(0xffffffffu, (int)*abort_flag, 0);
-            if (kc.valid && !aborted) {
-                const int ks = kpos % KS, kb = pc & 1;
-                const bool need_kr = kc.gi == 0;
-                int ready = 0;
-                if (lane == 0)
-                    ready = (!need_kr || mbar_test_wait(&kr_empty[kb], ((pc >> 1) & 1) ^ 1)) &&
-                            mbar_test_wait(&k_empty[ks], ((kpos / KS) & 1) ^ 1);
-                if (__shfl_sync(0xffffffffu, ready, 0)) {
-                    if (need_kr) ksl = pair_slots(kc);  // the first unit of a pair
-                    const PagePair &pp = kc.pp;
-                    const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
-                    const bool mine = half ? pp.page1 >= 0 : pp.page0 >= 0;
-                    if (need_kr) {
-                        uint8_t *dst = smem + SM::oKr + kb * SM::kKrBytes;
-                        if (lane == 0) {
-                            if (np) mbar_arrive_expect_tx(&kr_full[kb], np * kBox);
-                            else mbar_arrive(&kr_full[kb]);
-                        }
-                        __syncwarp();
-                        if (mine)
-                            tma_gather4_hint(dst + half * kBox + r0 * 128, &kr_rows_map, &kr_full[kb], 0,
-                                             ksl.x, ksl.y, ksl.z, ksl.w, stream_policy);
-                        ++pc;
-                    }
-                    uint8_t *dst = smem + SM::oK + ks * SM::kKSlotBytes;
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
-#pragma unroll
-                        for (int cb = 0; cb < 3; ++cb)  // q_g rows of this query token
-                            tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
-                                        kc.gi * p.G, kc.b * p.s_q);
-                    }
-                    __syncwarp();
-                    if (mine) {
-#pragma unroll
-                        for (int cb = 0; cb < 2; ++cb)  // K_nope lo / hi
-                            tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &k_full[ks],
-                                             cb * 64, row_of(ksl.x, kc.gi), row_of(ksl.y, kc.gi),
-                                             row_of(ksl.z, kc.gi), row_of(ksl.w, kc.gi), stream_policy);
-                    }
-                    kc.advance(p);
-                    ++kpos;
-                    progressed = true;
-                }
-            }
-            if (vc.valid && vpos < kpos && !aborted) {
-                const int vs = vpos % VS;
-                int ready = 0;
-                if (lane == 0) ready = mbar_test_wait(&v_empty[vs], ((vpos / VS) & 1) ^ 1);
-                if (__shfl_sync(0xffffffffu, ready, 0)) {
-                    if (vc.gi == 0) vsl = pair_slots(vc);
-                    const PagePair &pp = vc.pp;
-                    const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
-                    const bool mine = half ? pp.page1 >= 0 : pp.page0 >= 0;
-                    uint8_t *dst = smem + SM::oV + vs * SM::kVBytes;
-                    if (lane == 0) {
-                        if (np) mbar_arrive_expect_tx(&v_full[vs], np * 2 * kBox);
-                        else mbar_arrive(&v_full[vs]);
-                    }
-                    __syncwarp();
-                    if (mine) {
-#pragma unroll
-                        for (int cb = 0; cb < 2; ++cb)  // V lo / hi
-                            tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &v_full[vs],
-                                             128 + cb * 64, row_of(vsl.x, vc.gi), row_of(vsl.y, vc.gi),
-                                             row_of(vsl.z, vc.gi), row_of(vsl.w, vc.gi), stream_policy);
-                    }
-                    vc.advance(p);
-                    ++vpos;
-                    progressed = true;
-                }
-            }
-            int give_up = 0;
-            if (lane == 0 && !progressed) give_up = aborted || clock64() - idle_since > kWaitCycles;
-            if (progressed) {
-                idle_since = clock64();
-            } else if (!__shfl_sync(0xffffffffu, give_up, 0)) {
-                __nanosleep(20);
-            } else {
-                if (lane == 0) *abort_flag = 1;  // give up: the consumers stop waiting on us as well
-                break;
-            }
-        }
-        // never leave with copies in flight: wait (bounded) for the last loads issued
-        if (lane == 0) {
-            int dummy = 0;
-            volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
-            for (uint32_t u = (kpos > (uint32_t)KS ? kpos - KS : 0); u < kpos; ++u)
-                mbar_wait(&k_full[u % KS], (u / KS) & 1, no_abort);
-            for (uint32_t u = (vpos > (uint32_t)VS ? vpos - VS : 0); u < vpos; ++u)
-                mbar_wait(&v_full[u % VS], (u / VS) & 1, no_abort);
-            for (uint32_t u = (pc > 2u ? pc - 2 : 0); u < pc; ++u)
-                mbar_wait(&kr_full[u & 1], (u >> 1) & 1, no_abort);
-        }
-    } else if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            prefetch_tensormap(&kv_map);
-            prefetch_tensormap(&kr_map);
-            prefetch_tensormap(&q_map);
-            {
-                PieceIter it = it0;
-                int b, L, pb, pe;
-                bool too_long;
-                while (next_piece(p, it, b, L, pb, pe, too_long))
-                    if (too_long) report_error(p.ws, GQLA_ERR_DEVICE, b);
+    // Register split: each warpgroup changes its register budget once, at the top of its
+    // branch.  Warpgroup 0 gives registers up before it waits on anything, so the softmax
+    // warpgroups' increase never waits on a warp that waits on them.
+    if (warp < 4) {
+        regs_decrease();
+        if (warp == 0 && SPARSE) {
+            // ---------------------------------------------------------------- TMA producer, sparse
+            // The same units and rings as below; the rows of a unit are gathered four at a
+            // time (tile::gather4): lane l takes rows 4 (l % 16) .. + 3 of page l / 16 of the
+            // unit's pair, for K_nope_g, V_g and the pair's RoPE keys.  Lane 0 waits for
+            // the slots and sets each barrier's byte count before the warp issues.
+            if (lane == 0) {
+                prefetch_tensormap(&kv_rows_map);
+                prefetch_tensormap(&kr_rows_map);
+                prefetch_tensormap(&q_map);
             }
             const uint32_t q_bytes = 3u * 128u * (uint32_t)real_cols;
-            const uint64_t stream_policy = l2_evict_first_policy();  // the cache is read once
+            const uint64_t stream_policy = l2_evict_first_policy();
+            const int half = lane >> 4, r0 = 4 * (lane & 15);
             UnitCursor kc, vc;
             kc.start(p, it0);
             vc.start(p, it0);
             uint32_t kpos = 0, vpos = 0, pc = 0;
-            // Issue whichever load has a free slot: q_g + K_g as far ahead as their ring
-            // allows (with the pair's RoPE keys before its first group), V_g never ahead of K_g.
+            int4 ksl = make_int4(-1, -1, -1, -1), vsl = ksl;  // this lane's four cache slots
+            auto pair_slots = [&](const UnitCursor &cur) {
+                const int page = half ? cur.pp.page1 : cur.pp.page0;
+                return page < 0 ? make_int4(-1, -1, -1, -1)
+                                : *reinterpret_cast<const int4 *>(p.sel_slot + (int64_t)page * kPage + r0);
+            };
+            auto row_of = [&](int slot, int gi) { return slot < 0 ? -1 : (gbase + gi) * p.real_slots + slot; };
             long long idle_since = clock64();
-            while (kc.valid || vc.valid) {
+            while (kc.valid || vc.valid) {  // warp-uniform: every decision is lane 0's, broadcast
                 bool progressed = false;
-                if (kc.valid && !*abort_flag) {
+                const int aborted = __shfl_sync(0xffffffffu, (int)*abort_flag, 0);
+                if (kc.valid && !aborted) {
                     const int ks = kpos % KS, kb = pc & 1;
                     const bool need_kr = kc.gi == 0;
-                    if ((!need_kr || mbar_test_wait(&kr_empty[kb], ((pc >> 1) & 1) ^ 1)) &&
-                        mbar_test_wait(&k_empty[ks], ((kpos / KS) & 1) ^ 1)) {
+                    int ready = 0;
+                    if (lane == 0)
+                        ready = (!need_kr || mbar_test_wait(&kr_empty[kb], ((pc >> 1) & 1) ^ 1)) &&
+                                mbar_test_wait(&k_empty[ks], ((kpos / KS) & 1) ^ 1);
+                    if (__shfl_sync(0xffffffffu, ready, 0)) {
+                        if (need_kr) ksl = pair_slots(kc);  // the first unit of a pair
                         const PagePair &pp = kc.pp;
                         const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                        const bool mine = half ? pp.page1 >= 0 : pp.page0 >= 0;
                         if (need_kr) {
-                            if (pp.bad) report_error(p.ws, GQLA_ERR_DEVICE, kc.b);
                             uint8_t *dst = smem + SM::oKr + kb * SM::kKrBytes;
-                            if (np) {
-                                mbar_arrive_expect_tx(&kr_full[kb], np * kBox);
-                                if (pp.page0 >= 0)
-                                    tma_load_2d_hint(dst, &kr_map, &kr_full[kb], 0, pp.page0 * kPage, stream_policy);
-                                if (pp.page1 >= 0)
-                                    tma_load_2d_hint(dst + kBox, &kr_map, &kr_full[kb], 0, pp.page1 * kPage,
-                                                     stream_policy);
-                            } else {
-                                mbar_arrive(&kr_full[kb]);
+                            if (lane == 0) {
+                                if (np) mbar_arrive_expect_tx(&kr_full[kb], np * kBox);
+                                else mbar_arrive(&kr_full[kb]);
                             }
+                            __syncwarp();
+                            if (mine)
+                                tma_gather4_hint(dst + half * kBox + r0 * 128, &kr_rows_map, &kr_full[kb], 0,
+                                                 ksl.x, ksl.y, ksl.z, ksl.w, stream_policy);
                             ++pc;
                         }
                         uint8_t *dst = smem + SM::oK + ks * SM::kKSlotBytes;
-                        mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
-#pragma unroll
-                        for (int cb = 0; cb < 3; ++cb)  // q_g rows (s, hg) of this sequence
-                            tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
-                                        kc.gi * p.G, kc.b * p.s_q);
-#pragma unroll
-                        for (int cb = 0; cb < 2; ++cb) {  // K_nope lo / hi: page 0 rows, then page 1 rows
-                            if (pp.page0 >= 0)
-                                tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &k_full[ks], cb * 64,
-                                                 pp.page0 * kPage, kc.gi, stream_policy);
-                            if (pp.page1 >= 0)
-                                tma_load_3d_hint(dst + cb * 2 * kBox + kBox, &kv_map, &k_full[ks], cb * 64,
-                                                 pp.page1 * kPage, kc.gi, stream_policy);
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
+    #pragma unroll
+                            for (int cb = 0; cb < 3; ++cb)  // q_g rows of this query token
+                                tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
+                                            (gbase + kc.gi) * p.G, kc.b * p.s_q);
+                        }
+                        __syncwarp();
+                        if (mine) {
+    #pragma unroll
+                            for (int cb = 0; cb < 2; ++cb)  // K_nope lo / hi
+                                tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &k_full[ks],
+                                                 cb * 64, row_of(ksl.x, kc.gi), row_of(ksl.y, kc.gi),
+                                                 row_of(ksl.z, kc.gi), row_of(ksl.w, kc.gi), stream_policy);
                         }
                         kc.advance(p);
                         ++kpos;
                         progressed = true;
                     }
                 }
-                if (vc.valid && vpos < kpos && !*abort_flag && (int)vpos == p.drop_v_unit) {
-                    vc.advance(p);  // diagnostic: no load and no arrival for this unit
-                    ++vpos;
-                    progressed = true;
-                } else if (vc.valid && vpos < kpos && !*abort_flag) {
+                if (vc.valid && vpos < kpos && !aborted) {
                     const int vs = vpos % VS;
-                    if (mbar_test_wait(&v_empty[vs], ((vpos / VS) & 1) ^ 1)) {
+                    int ready = 0;
+                    if (lane == 0) ready = mbar_test_wait(&v_empty[vs], ((vpos / VS) & 1) ^ 1);
+                    if (__shfl_sync(0xffffffffu, ready, 0)) {
+                        if (vc.gi == 0) vsl = pair_slots(vc);
                         const PagePair &pp = vc.pp;
                         const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                        const bool mine = half ? pp.page1 >= 0 : pp.page0 >= 0;
                         uint8_t *dst = smem + SM::oV + vs * SM::kVBytes;
-                        if (np) {
-                            mbar_arrive_expect_tx(&v_full[vs], np * 2 * kBox);
-#pragma unroll
-                            for (int cb = 0; cb < 2; ++cb) {
-                                if (pp.page0 >= 0)
-                                    tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &v_full[vs], 128 + cb * 64,
-                                                     pp.page0 * kPage, vc.gi, stream_policy);
-                                if (pp.page1 >= 0)
-                                    tma_load_3d_hint(dst + cb * 2 * kBox + kBox, &kv_map, &v_full[vs],
-                                                     128 + cb * 64, pp.page1 * kPage, vc.gi, stream_policy);
-                            }
-                        } else {
-                            mbar_arrive(&v_full[vs]);
+                        if (lane == 0) {
+                            if (np) mbar_arrive_expect_tx(&v_full[vs], np * 2 * kBox);
+                            else mbar_arrive(&v_full[vs]);
+                        }
+                        __syncwarp();
+                        if (mine) {
+    #pragma unroll
+                            for (int cb = 0; cb < 2; ++cb)  // V lo / hi
+                                tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &v_full[vs],
+                                                 128 + cb * 64, row_of(vsl.x, vc.gi), row_of(vsl.y, vc.gi),
+                                                 row_of(vsl.z, vc.gi), row_of(vsl.w, vc.gi), stream_policy);
                         }
                         vc.advance(p);
                         ++vpos;
                         progressed = true;
                     }
                 }
+                int give_up = 0;
+                if (lane == 0 && !progressed) give_up = aborted || clock64() - idle_since > kWaitCycles;
                 if (progressed) {
                     idle_since = clock64();
-                } else if (!*abort_flag && clock64() - idle_since <= kWaitCycles) {
+                } else if (!__shfl_sync(0xffffffffu, give_up, 0)) {
                     __nanosleep(20);
                 } else {
-                    *abort_flag = 1;  // give up: the consumers stop waiting on us as well
+                    if (lane == 0) *abort_flag = 1;  // give up: the consumers stop waiting on us as well
                     break;
                 }
             }
             // never leave with copies in flight: wait (bounded) for the last loads issued
-            int dummy = 0;
-            volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
-            for (uint32_t u = (kpos > (uint32_t)KS ? kpos - KS : 0); u < kpos; ++u)
-                mbar_wait(&k_full[u % KS], (u / KS) & 1, no_abort);
-            for (uint32_t u = (vpos > (uint32_t)VS ? vpos - VS : 0); u < vpos; ++u)
-                mbar_wait(&v_full[u % VS], (u / VS) & 1, no_abort);
-            for (uint32_t u = (pc > 2u ? pc - 2 : 0); u < pc; ++u)
-                mbar_wait(&kr_full[u & 1], (u >> 1) & 1, no_abort);
-        }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------------- score MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16(kTok, NQ, 0, 0);
-            PieceIter it = it0;
-            int b, L, pb, pe;
-            bool too_long;
-            uint32_t u = 0, pc = 0;
-            while (next_piece(p, it, b, L, pb, pe, too_long)) {
-                if (too_long) continue;
-                for (int pg = pb; pg < pe; pg += 2, ++pc) {
-                    const int kb = pc & 1;
-                    if (!GQLA_WAIT(2, &kr_full[kb], (pc >> 1) & 1, abort_flag)) *abort_flag = 1;
-                    const uint32_t kr = sm_kr + kb * SM::kKrBytes;
-                    for (int gi = 0; gi < p.NG; ++gi, ++u) {
-                        // S^T(u) = [K_nope_g | k^R] q_g^T into S buffer u & 3
-                        const int ks_ = u % KS, sb = u & 3;
-                        if (!GQLA_WAIT(3, &k_full[ks_], (u / KS) & 1, abort_flag)) *abort_flag = 1;
-                        if (!GQLA_WAIT(4, &s_free[sb], ((u >> 2) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                        tc_fence_after();
-                        // descriptors from the slot bases: each MMA only adds an offset
-                        const uint64_t k_d = smem_desc(sm_k + ks_ * SM::kKSlotBytes, 16, 1024, kSw128);
-                        const uint64_t q_d = desc_advance(k_d, SM::kKBytes);
-                        const uint64_t kr_d = smem_desc(kr, 16, 1024, kSw128);
-                        if (!*abort_flag) {
-#pragma unroll
-                            for (int ks = 0; ks < 12; ++ks) {
-                                const uint64_t ad = ks < 8 ? desc_advance(k_d, (ks >> 2) * 2 * kBox + (ks & 3) * 32)
-                                                           : desc_advance(kr_d, (ks - 8) * 32);
-                                const uint64_t bd = desc_advance(q_d, (ks >> 2) * NQ * 128 + (ks & 3) * 32);
-                                mma_bf16(t_s + sb * NQ, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+            if (lane == 0) {
+                int dummy = 0;
+                volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
+                for (uint32_t u = (kpos > (uint32_t)KS ? kpos - KS : 0); u < kpos; ++u)
+                    mbar_wait(&k_full[u % KS], (u / KS) & 1, no_abort);
+                for (uint32_t u = (vpos > (uint32_t)VS ? vpos - VS : 0); u < vpos; ++u)
+                    mbar_wait(&v_full[u % VS], (u / VS) & 1, no_abort);
+                for (uint32_t u = (pc > 2u ? pc - 2 : 0); u < pc; ++u)
+                    mbar_wait(&kr_full[u & 1], (u >> 1) & 1, no_abort);
+            }
+        } else if (warp == 0) {
+            // ---------------------------------------------------------------- TMA producer
+            if (lane == 0) {
+                prefetch_tensormap(&kv_map);
+                prefetch_tensormap(&kr_map);
+                prefetch_tensormap(&q_map);
+                {
+                    PieceIter it = it0;
+                    int b, L, pb, pe;
+                    bool too_long;
+                    while (next_piece(p, it, b, L, pb, pe, too_long))
+                        if (too_long) report_error(p.ws, GQLA_ERR_DEVICE, b);
+                }
+                const uint32_t q_bytes = 3u * 128u * (uint32_t)real_cols;
+                const uint64_t stream_policy = l2_evict_first_policy();  // the cache is read once
+                UnitCursor kc, vc;
+                kc.start(p, it0);
+                vc.start(p, it0);
+                uint32_t kpos = 0, vpos = 0, pc = 0;
+                // Issue whichever load has a free slot: q_g + K_g as far ahead as their ring
+                // allows (with the pair's RoPE keys before its first group), V_g never ahead of K_g.
+                long long idle_since = clock64();
+                while (kc.valid || vc.valid) {
+                    bool progressed = false;
+                    if (kc.valid && !*abort_flag) {
+                        const int ks = kpos % KS, kb = pc & 1;
+                        const bool need_kr = kc.gi == 0;
+                        if ((!need_kr || mbar_test_wait(&kr_empty[kb], ((pc >> 1) & 1) ^ 1)) &&
+                            mbar_test_wait(&k_empty[ks], ((kpos / KS) & 1) ^ 1)) {
+                            const PagePair &pp = kc.pp;
+                            const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                            if (need_kr) {
+                                if (pp.bad) report_error(p.ws, GQLA_ERR_DEVICE, kc.b);
+                                uint8_t *dst = smem + SM::oKr + kb * SM::kKrBytes;
+                                if (np) {
+                                    mbar_arrive_expect_tx(&kr_full[kb], np * kBox);
+                                    if (pp.page0 >= 0)
+                                        tma_load_2d_hint(dst, &kr_map, &kr_full[kb], 0, pp.page0 * kPage, stream_policy);
+                                    if (pp.page1 >= 0)
+                                        tma_load_2d_hint(dst + kBox, &kr_map, &kr_full[kb], 0, pp.page1 * kPage,
+                                                         stream_policy);
+                                } else {
+                                    mbar_arrive(&kr_full[kb]);
+                                }
+                                ++pc;
                             }
+                            uint8_t *dst = smem + SM::oK + ks * SM::kKSlotBytes;
+                            mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
+    #pragma unroll
+                            for (int cb = 0; cb < 3; ++cb)  // q_g rows (s, hg) of this sequence
+                                tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
+                                            (gbase + kc.gi) * p.G, kc.b * p.s_q);
+    #pragma unroll
+                            for (int cb = 0; cb < 2; ++cb) {  // K_nope lo / hi: page 0 rows, then page 1 rows
+                                if (pp.page0 >= 0)
+                                    tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &k_full[ks], cb * 64,
+                                                     pp.page0 * kPage, gbase + kc.gi, stream_policy);
+                                if (pp.page1 >= 0)
+                                    tma_load_3d_hint(dst + cb * 2 * kBox + kBox, &kv_map, &k_full[ks], cb * 64,
+                                                     pp.page1 * kPage, gbase + kc.gi, stream_policy);
+                            }
+                            kc.advance(p);
+                            ++kpos;
+                            progressed = true;
                         }
-                        mma_commit(&s_full[sb]);
-                        mma_commit(&k_empty[ks_]);
-                        if (gi == p.NG - 1) mma_commit(&kr_empty[kb]);
+                    }
+                    if (vc.valid && vpos < kpos && !*abort_flag && (int)vpos == p.drop_v_unit) {
+                        vc.advance(p);  // diagnostic: no load and no arrival for this unit
+                        ++vpos;
+                        progressed = true;
+                    } else if (vc.valid && vpos < kpos && !*abort_flag) {
+                        const int vs = vpos % VS;
+                        if (mbar_test_wait(&v_empty[vs], ((vpos / VS) & 1) ^ 1)) {
+                            const PagePair &pp = vc.pp;
+                            const int np = (pp.page0 >= 0) + (pp.page1 >= 0);
+                            uint8_t *dst = smem + SM::oV + vs * SM::kVBytes;
+                            if (np) {
+                                mbar_arrive_expect_tx(&v_full[vs], np * 2 * kBox);
+    #pragma unroll
+                                for (int cb = 0; cb < 2; ++cb) {
+                                    if (pp.page0 >= 0)
+                                        tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &v_full[vs], 128 + cb * 64,
+                                                         pp.page0 * kPage, gbase + vc.gi, stream_policy);
+                                    if (pp.page1 >= 0)
+                                        tma_load_3d_hint(dst + cb * 2 * kBox + kBox, &kv_map, &v_full[vs],
+                                                         128 + cb * 64, pp.page1 * kPage, gbase + vc.gi, stream_policy);
+                                }
+                            } else {
+                                mbar_arrive(&v_full[vs]);
+                            }
+                            vc.advance(p);
+                            ++vpos;
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        idle_since = clock64();
+                    } else if (!*abort_flag && clock64() - idle_since <= kWaitCycles) {
+                        __nanosleep(20);
+                    } else {
+                        *abort_flag = 1;  // give up: the consumers stop waiting on us as well
+                        break;
                     }
                 }
+                // never leave with copies in flight: wait (bounded) for the last loads issued
+                int dummy = 0;
+                volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
+                for (uint32_t u = (kpos > (uint32_t)KS ? kpos - KS : 0); u < kpos; ++u)
+                    mbar_wait(&k_full[u % KS], (u / KS) & 1, no_abort);
+                for (uint32_t u = (vpos > (uint32_t)VS ? vpos - VS : 0); u < vpos; ++u)
+                    mbar_wait(&v_full[u % VS], (u / VS) & 1, no_abort);
+                for (uint32_t u = (pc > 2u ? pc - 2 : 0); u < pc; ++u)
+                    mbar_wait(&kr_full[u & 1], (u >> 1) & 1, no_abort);
             }
-            // drain: nothing may still be running when TMEM is freed
-            mma_commit(&drain[0]);
-            int dummy = 0;
-            mbar_wait(&drain[0], 0, reinterpret_cast<volatile int *>(&dummy));
-        }
-    } else if (warp == 10) {
-        // ---------------------------------------------------------------- PV MMA issuer
-        // O^T_g(u) (+)= V_g^T P^T(u), in unit order, as soon as the owning warpgroup
-        // has published P^T(u) and V_g(u) has landed; no softmax warp waits for V.
-        if (lane == 0) {
-            constexpr uint32_t idesc_pv = idesc_bf16(128, NQ, 1, 1);
-            constexpr uint32_t p_sw = NQ == 16 ? kSw32 : kSw64;
-            constexpr uint32_t p_sbo = NQ == 16 ? 256 : 512;
-            const uint64_t v_d0 = smem_desc(sm_v, 2 * kBox, 1024, kSw128);
-            const uint64_t p_d0 = smem_desc(sm_p, SM::kPBytes, p_sbo, p_sw);
-            PieceIter it = it0;
-            int b, L, pb, pe;
-            bool too_long;
-            uint32_t u = 0;
-            while (next_piece(p, it, b, L, pb, pe, too_long)) {
-                if (too_long) continue;
-                const int npairs = (pe - pb + 1) >> 1;
-                for (int ip = 0; ip < npairs; ++ip) {
-                    for (int gi = 0; gi < p.NG; ++gi, ++u) {
-                        const int w = gi & 1, vs = u % VS;
-                        if (!GQLA_WAIT(5, &p_full[w], (u >> 1) & 1, abort_flag)) *abort_flag = 1;
-                        if (!GQLA_WAIT(13, &v_full[vs], (u / VS) & 1, abort_flag)) *abort_flag = 1;
-                        tc_fence_after();
-                        const uint64_t v_d = desc_advance(v_d0, vs * SM::kVBytes);
-                        const uint64_t p_d = desc_advance(p_d0, w * SM::kPBytes);
-                        if (!*abort_flag) {
-#pragma unroll
-                            for (int ks = 0; ks < kTok / 16; ++ks)
-                                mma_bf16(t_o + gi * NQ, desc_advance(v_d, ks * 2048), desc_advance(p_d, ks * 16 * NQ * 2),
-                                         idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
+        } else if (warp == 1) {
+            // ---------------------------------------------------------------- score MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = idesc_bf16(kTok, NQ, 0, 0);
+                PieceIter it = it0;
+                int b, L, pb, pe;
+                bool too_long;
+                uint32_t u = 0, pc = 0;
+                while (next_piece(p, it, b, L, pb, pe, too_long)) {
+                    if (too_long) continue;
+                    for (int pg = pb; pg < pe; pg += 2, ++pc) {
+                        const int kb = pc & 1;
+                        if (!GQLA_WAIT(2, &kr_full[kb], (pc >> 1) & 1, abort_flag)) *abort_flag = 1;
+                        const uint32_t kr = sm_kr + kb * SM::kKrBytes;
+                        for (int gi = 0; gi < p.NG; ++gi, ++u) {
+                            // S^T(u) = [K_nope_g | k^R] q_g^T into S buffer u & 3
+                            const int ks_ = u % KS, sb = u & 3;
+                            if (!GQLA_WAIT(3, &k_full[ks_], (u / KS) & 1, abort_flag)) *abort_flag = 1;
+                            if (!GQLA_WAIT(4, &s_free[sb], ((u >> 2) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                            tc_fence_after();
+                            // descriptors from the slot bases: each MMA only adds an offset
+                            const uint64_t k_d = smem_desc(sm_k + ks_ * SM::kKSlotBytes, 16, 1024, kSw128);
+                            const uint64_t q_d = desc_advance(k_d, SM::kKBytes);
+                            const uint64_t kr_d = smem_desc(kr, 16, 1024, kSw128);
+                            if (!*abort_flag) {
+    #pragma unroll
+                                for (int ks = 0; ks < 12; ++ks) {
+                                    const uint64_t ad = ks < 8 ? desc_advance(k_d, (ks >> 2) * 2 * kBox + (ks & 3) * 32)
+                                                               : desc_advance(kr_d, (ks - 8) * 32);
+                                    const uint64_t bd = desc_advance(q_d, (ks >> 2) * NQ * 128 + (ks & 3) * 32);
+                                    mma_bf16(t_s + sb * NQ, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                                }
+                            }
+                            mma_commit(&s_full[sb]);
+                            mma_commit(&k_empty[ks_]);
+                            if (gi == p.NG - 1) mma_commit(&kr_empty[kb]);
                         }
-                        mma_commit(&p_free[w]);
-                        mma_commit(&v_empty[vs]);
                     }
                 }
-                mma_commit(&o_done[0]);
-                mma_commit(&o_done[1]);
+                // drain: nothing may still be running when TMEM is freed
+                mma_commit(&drain[0]);
+                int dummy = 0;
+                mbar_wait(&drain[0], 0, reinterpret_cast<volatile int *>(&dummy));
             }
-            mma_commit(&drain[1]);
-            int dummy = 0;
-            mbar_wait(&drain[1], 0, reinterpret_cast<volatile int *>(&dummy));
+        } else if (warp == 2) {
+            // ---------------------------------------------------------------- PV MMA issuer
+            // O^T_g(u) (+)= V_g^T P^T(u), in unit order, as soon as the owning warpgroup
+            // has published P^T(u) and V_g(u) has landed; no softmax warp waits for V.
+            if (lane == 0) {
+                constexpr uint32_t idesc_pv = idesc_bf16(128, NQ, 1, 1);
+                constexpr uint32_t p_sw = NQ == 16 ? kSw32 : kSw64;
+                constexpr uint32_t p_sbo = NQ == 16 ? 256 : 512;
+                const uint64_t v_d0 = smem_desc(sm_v, 2 * kBox, 1024, kSw128);
+                const uint64_t p_d0 = smem_desc(sm_p, SM::kPBytes, p_sbo, p_sw);
+                PieceIter it = it0;
+                int b, L, pb, pe;
+                bool too_long;
+                uint32_t u = 0;
+                while (next_piece(p, it, b, L, pb, pe, too_long)) {
+                    if (too_long) continue;
+                    const int npairs = (pe - pb + 1) >> 1;
+                    for (int ip = 0; ip < npairs; ++ip) {
+                        for (int gi = 0; gi < p.NG; ++gi, ++u) {
+                            const int w = gi & 1, vs = u % VS;
+                            if (!GQLA_WAIT(5, &p_full[w], wg_unit(u, p.NG) & 1, abort_flag)) *abort_flag = 1;
+                            if (!GQLA_WAIT(13, &v_full[vs], (u / VS) & 1, abort_flag)) *abort_flag = 1;
+                            tc_fence_after();
+                            const uint64_t v_d = desc_advance(v_d0, vs * SM::kVBytes);
+                            const uint64_t p_d = desc_advance(p_d0, w * SM::kPBytes);
+                            if (!*abort_flag) {
+    #pragma unroll
+                                for (int ks = 0; ks < kTok / 16; ++ks)
+                                    mma_bf16(t_o + gi * NQ, desc_advance(v_d, ks * 2048), desc_advance(p_d, ks * 16 * NQ * 2),
+                                             idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
+                            }
+                            mma_commit(&p_free[w]);
+                            mma_commit(&v_empty[vs]);
+                        }
+                    }
+                    mma_commit(&o_done[0]);
+                    mma_commit(&o_done[1]);
+                }
+                mma_commit(&drain[1]);
+                int dummy = 0;
+                mbar_wait(&drain[1], 0, reinterpret_cast<volatile int *>(&dummy));
+            }
         }
+        // warp 3 is idle: it completes warpgroup 0 for the register split
     } else {
+        regs_increase();
         // ---------------------------------------------------------------- softmax, PV, epilogue
         // Warpgroup wg owns the groups gi = wg, wg + 2, ... (units of
         // one parity), so the two warpgroups never share a group.
-        const int wg = (warp - 2) >> 2;        // 0 or 1
-        const int wq = (warp - 2) & 3;         // warp within the warpgroup
+        const int wg = (warp - 4) >> 2;        // 0 or 1
+        const int wq = (warp - 4) & 3;         // warp within the warpgroup
         const int quad = warp & 3;             // TMEM lane quadrant of this warp
-        const int wtid = (threadIdx.x - 64) & 127;
+        const int wtid = (threadIdx.x - 128) & 127;
         const int tok = 32 * quad + lane;      // this thread's token row in a unit (and dv row of O^T)
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         float *red = reinterpret_cast<float *>(smem + SM::oRed) + wg * NQ * 4;
@@ -697,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // s_q <= 2 only the last token can be hidden, and only from columns n < G
                 const bool hide_low = pg * kPage + tok - (L - p.s_q) > 0;
 #pragma unroll 1
-                for (int gl = 0; gl < p.NG / 2; ++gl) {
+                for (int gl = 0; gl < wg_groups(p.NG, wg); ++gl) {
                     const int gi = 2 * gl + wg;
                     const uint32_t jj = j + ip * p.NG + gi;
                     // lane n (< NQ) keeps the column-n sum over this warp's tokens in shared memory
@@ -725,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int n = 0; n < NQ; ++n)
                         exceed |= score_of(sv[n], n, tok_ok, hide_low, p.G, p.scale_log2) > mu[n] + kRescaleLog2;
                     // the P^T buffer (and O^T_g) are free once this warpgroup's previous PV completed
-                    if (!GQLA_WAIT(7, &p_free[wg], ((jj >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(7, &p_free[wg], (wg_unit(jj, p.NG) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
                     float ps[NQ];
                     GQLA_SPAN_BEGIN(t_wp);
@@ -827,10 +871,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             wg_bar(wg);  // all column partials of this warpgroup are in lred
             const int slot = b + c;
             const int dv = tok;
-            // rows of the partial for columns n = s*G + hg: ((slot*s_q + s)*h + gi*G + hg)
-            const int64_t row_s0 = (int64_t)slot * p.s_q * p.heads;
+            // a piece that is its sequence's only one (all its pages in this chunk) is the
+            // result itself: with final outputs given it goes there, in bf16, and no partial
+            // is written (the combine then leaves the sequence alone)
+            const bool final_out = p.out != nullptr && pb == 0 && pe == pages_of(L);
+            // rows of the partial for columns n = s*G + hg: ((slot*s_q + s)*h + g*G + hg);
+            // rows of the final output: ((b*s_q + s)*h + g*G + hg)
+            const int64_t row_s0 = (int64_t)(final_out ? b : slot) * p.s_q * p.heads;
 #pragma unroll 1
-            for (int gl = 0; gl < p.NG / 2; ++gl) {
+            for (int gl = 0; gl < wg_groups(p.NG, wg); ++gl) {
                 const int gi = 2 * gl + wg;
                 if (wtid < NQ) {  // per column: 1 / l and the natural-log LSE
                     const float4 l4 = *reinterpret_cast<const float4 *>(lred + (gi * NQ + wtid) * 4);
@@ -841,24 +890,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     inv_l[NQ + wtid] = ok ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
                     if (wtid < real_cols) {
                         const int s = wtid / p.G, hg = wtid - s * p.G;
-                        p.lse_part[row_s0 + (int64_t)s * p.heads + gi * p.G + hg] = inv_l[NQ + wtid];
+                        float *lse_dst = final_out ? p.lse_out : p.lse_part;
+                        if (lse_dst) lse_dst[row_s0 + (int64_t)s * p.heads + (gbase + gi) * p.G + hg] = inv_l[NQ + wtid];
                     }
                 }
-                uint32_t r[NQ];
-                GQLA_SPAN_BEGIN(t_eld);
-                tmem_ld16(t_o + gi * NQ + lane_off, r);
-                if constexpr (NQ == 32) tmem_ld16(t_o + gi * NQ + lane_off + 16, r + 16);
-                tmem_wait_ld();
-                GQLA_SPAN_END(18, t_eld);
                 wg_bar(wg);  // inv_l ready
                 GQLA_SPAN_BEGIN(t_est);
-                float *dst = p.o_part + (row_s0 + gi * p.G) * kDv + dv;
+                // 16 columns at a time: O^T row dv of columns n = s*G + hg -> row (s*h + g*G + hg)
+                const int64_t row_g = row_s0 + (int64_t)(gbase + gi) * p.G;
+                float *dst_p = p.o_part + row_g * kDv + dv;
+                __nv_bfloat16 *dst_o = final_out ? p.out + row_g * kDv + dv : nullptr;
                 int s = 0, hg = 0;
 #pragma unroll
-                for (int n = 0; n < NQ; ++n) {
-                    if (n < real_cols)
-                        dst[((int64_t)s * p.heads + hg) * kDv] = __uint_as_float(r[n]) * inv_l[n];
-                    if (++hg == p.G) { hg = 0; ++s; }
+                for (int h16 = 0; h16 < NQ; h16 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(t_o + gi * NQ + lane_off + h16, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        if (h16 + e < real_cols) {
+                            const int64_t off = ((int64_t)s * p.heads + hg) * kDv;
+                            const float v = __uint_as_float(r[e]) * inv_l[h16 + e];
+                            if (dst_o) dst_o[off] = __float2bfloat16_rn(v);
+                            else dst_p[off] = v;
+                        }
+                        if (++hg == p.G) { hg = 0; ++s; }
+                    }
                 }
                 GQLA_SPAN_END(19, t_est);
                 wg_bar(wg);  // inv_l is rewritten for the next group
@@ -869,6 +926,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             GQLA_SPAN_END(20, t_ebar);
             GQLA_SPAN_END(21, t_epi);
             ++k;
+        }
+        if (p.out != nullptr && c == 0) {
+            // sequences with no token have no piece: with final outputs given, the CTAs of
+            // chunk 0 write out = 0 and lse = -inf for their groups' heads (one thread per
+            // sequence)
+            const int hcols = p.NG * p.G;  // this CTA's heads
+            for (int b2 = threadIdx.x - 128; b2 < p.batch; b2 += 256) {
+                if (p.seqlens[b2] != 0) continue;
+                for (int s = 0; s < p.s_q; ++s) {
+                    const int64_t row0 = ((int64_t)b2 * p.s_q + s) * p.heads + (int64_t)gbase * p.G;
+                    for (int i = 0; i < hcols * (kDv / 8); ++i)
+                        *reinterpret_cast<uint4 *>(p.out + (row0 + i / (kDv / 8)) * kDv + (i % (kDv / 8)) * 8) =
+                            make_uint4(0, 0, 0, 0);
+                    if (p.lse_out)
+                        for (int i = 0; i < hcols; ++i) p.lse_out[row0 + i] = -INFINITY;
+                }
+            }
         }
     }
 
@@ -913,19 +987,37 @@ bool make_map(CUtensorMap *map, const void *base, int rank, const cuuint64_t *di
 template <int NQ, bool SPARSE>
 cudaError_t launch_nq_mode(const CUtensorMap &kvm, const CUtensorMap &krm, const CUtensorMap &qm,
                            const CUtensorMap &kvrm, const CUtensorMap &krrm, const GqaParams &p,
-                           cudaStream_t stream) {
+                           int group_splits, cudaStream_t stream) {
     const int bytes = GqaSmem<NQ>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(decode_gqa_tc_kernel<NQ, SPARSE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    return launch_dependent(decode_gqa_tc_kernel<NQ, SPARSE>, dim3(p.num_splits), dim3(kThreads), bytes,
-                            stream, kvm, krm, qm, kvrm, krrm, p);
+    // the register split asks for 128 x kRegsIssue + 256 x kRegsSoftmax registers: the
+    // launch must give at least that many, or the kernel's increase would never return
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, decode_gqa_tc_kernel<NQ, SPARSE>);
+    if (e != cudaSuccess) return e;
+    if (128 * kRegsIssue + 256 * kRegsSoftmax > kThreads * fa.numRegs) return cudaErrorInvalidConfiguration;
+    return launch_dependent(decode_gqa_tc_kernel<NQ, SPARSE>, dim3(p.num_splits, group_splits), dim3(kThreads),
+                            bytes, stream, kvm, krm, qm, kvrm, krrm, p);
 }
 
 template <int NQ>
 cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const CUtensorMap &qm,
-                      const GqaParams &p, cudaStream_t stream) {
-    return launch_nq_mode<NQ, false>(kvm, krm, qm, kvm, krm, p, stream);  // no row maps in dense mode
+                      const GqaParams &p, int group_splits, cudaStream_t stream) {
+    return launch_nq_mode<NQ, false>(kvm, krm, qm, kvm, krm, p, group_splits, stream);  // no row maps in dense mode
+}
+
+// CTAs per chunk: a batch too small to fill the GPU with one CTA per chunk has its groups
+// split over up to g CTAs per chunk (each reads the chunk's RoPE keys again: 128 of the
+// 4224 bytes of a token per extra CTA), as long as two such grids still fit in one wave.
+int group_splits_for(int num_splits, int num_groups) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int gs = 1;
+    while (gs < num_groups && (int64_t)num_splits * gs * 4 <= sms) gs *= 2;
+    return gs;
 }
 
 }  // namespace
@@ -936,8 +1028,8 @@ thread_local int g_drop_v_unit = -1;
 cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups, const void *kv,
                               const void *k_rope, int64_t num_slots, const gqla_kv_index *idx,
                               int num_splits, float scale, float *o_part, float *lse_part,
-                              void *ws, cudaStream_t stream) {
-    if (num_groups != 8 && num_groups != 4) return cudaErrorInvalidValue;
+                              void *out, float *lse_out, void *ws, cudaStream_t stream) {
+    if (num_groups != 8 && num_groups != 4 && num_groups != 2 && num_groups != 1) return cudaErrorInvalidValue;
     const int G = heads / num_groups;
     CUtensorMap kvm, krm, qm;
     {
@@ -971,14 +1063,17 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
     p.s_q = s_q;
     p.heads = heads;
     p.G = G;
-    p.NG = num_groups;
+    const int gs = group_splits_for(num_splits, num_groups);
+    p.NG = num_groups / gs;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse_out = lse_out;
     p.scale_log2 = scale * kLog2e;
     p.sel_slot = nullptr;
     p.real_slots = 0;
     p.drop_v_unit = g_drop_v_unit;
     g_drop_v_unit = -1;
-    return G * s_q <= 16 ? launch_nq<16>(kvm, krm, qm, p, stream)
-                         : launch_nq<32>(kvm, krm, qm, p, stream);
+    return G * s_q <= 16 ? launch_nq<16>(kvm, krm, qm, p, gs, stream)
+                         : launch_nq<32>(kvm, krm, qm, p, gs, stream);
 }
 
 // Sparse GQLA: the decode over a selection (sel: batch * s_q one-token sequences over
@@ -1022,13 +1117,15 @@ cudaError_t launch_decode_gqa_sparse(const void *q, int heads, int num_groups, c
     p.heads = heads;
     p.G = G;
     p.NG = num_groups;
+    p.out = nullptr;
+    p.lse_out = nullptr;
     p.scale_log2 = scale * kLog2e;
     p.sel_slot = sel_slot;
     p.real_slots = (int)real_slots;
     p.drop_v_unit = -1;
     // the dense tile maps are not used in sparse mode: the row maps stand in for them
-    return G <= 16 ? launch_nq_mode<16, true>(kvr, krr, qm, kvr, krr, p, stream)
-                   : launch_nq_mode<32, true>(kvr, krr, qm, kvr, krr, p, stream);
+    return G <= 16 ? launch_nq_mode<16, true>(kvr, krr, qm, kvr, krr, p, 1, stream)
+                   : launch_nq_mode<32, true>(kvr, krr, qm, kvr, krr, p, 1, stream);
 }
 
 }  // namespace gqla

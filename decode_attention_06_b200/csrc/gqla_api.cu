@@ -27,13 +27,13 @@ cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_grou
 cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups, const void *kv,
                               const void *k_rope, int64_t num_slots, const gqla_kv_index *idx,
                               int num_splits, float scale, float *o_part, float *lse_part,
-                              void *ws, cudaStream_t stream);
+                              void *out, float *lse_out, void *ws, cudaStream_t stream);
 cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
                                  const gqla_kv_index *idx, int num_splits, float scale,
                                  float *o_part, float *lse_part, void *ws, cudaStream_t stream);
 cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int d_in,
                            const float *o_part, const float *lse_part, const void *w_uv,
-                           void *out, float *lse_out, int heads, int num_groups,
+                           void *out, float *lse_out, int heads, int num_groups, bool skip_single,
                            cudaStream_t stream);
 extern thread_local int g_drop_v_unit;
 }  // namespace gqla
@@ -257,11 +257,38 @@ int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *k
     if (!aligned16(q) || !aligned16(kv_expanded) || !aligned16(k_rope) || !aligned16(o_part))
         return GQLA_ERR_INVALID_ARG;
     if (num_slots != (int64_t)kv->num_pages * kv->page_size) return GQLA_ERR_INVALID_ARG;
-    if (dims->num_groups != 8 && dims->num_groups != 4) return GQLA_ERR_UNSUPPORTED;
+    if (dims->num_groups != 8 && dims->num_groups != 4 && dims->num_groups != 2 && dims->num_groups != 1)
+        return GQLA_ERR_UNSUPPORTED;
     return cuda_status(launch_decode_gqa(q, s_q, dims->num_heads, dims->num_groups, kv_expanded,
                                          k_rope, num_slots, kv, num_splits, dims->softmax_scale,
-                                         o_part, lse_part, workspace,
+                                         o_part, lse_part, nullptr, nullptr, workspace,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gqla_decode_gqa_step(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
+                         const void *k_rope, int64_t num_slots, const gqla_kv_index *kv,
+                         int num_splits, float *o_part, float *lse_part, void *out, float *lse_out,
+                         void *workspace, size_t workspace_bytes, gqla_stream_t stream) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if ((st = check_index(kv)) != GQLA_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes)) != GQLA_OK) return st;
+    if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
+    if (!q || !kv_expanded || !k_rope || !out) return GQLA_ERR_INVALID_ARG;
+    if (num_splits > 1 && (!o_part || !lse_part)) return GQLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv_expanded) || !aligned16(k_rope) || !aligned16(out) ||
+        (o_part && !aligned16(o_part)))
+        return GQLA_ERR_INVALID_ARG;
+    if (num_slots != (int64_t)kv->num_pages * kv->page_size) return GQLA_ERR_INVALID_ARG;
+    if (dims->num_groups != 8 && dims->num_groups != 4 && dims->num_groups != 2 && dims->num_groups != 1)
+        return GQLA_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = cuda_status(launch_decode_gqa(q, s_q, dims->num_heads, dims->num_groups, kv_expanded, k_rope,
+                                       num_slots, kv, num_splits, dims->softmax_scale, o_part, lse_part,
+                                       out, lse_out, workspace, s));
+    if (st != GQLA_OK || num_splits == 1) return st;  // one chunk: every sequence is final already
+    return cuda_status(launch_combine(kv, s_q, num_splits, kDv, o_part, lse_part, nullptr, out, lse_out,
+                                      dims->num_heads, dims->num_groups, true, s));
 }
 
 int gqla_sparse_gather(const gqla_dims *dims, const void *kv_expanded, const void *k_rope,
@@ -347,7 +374,7 @@ int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int nu
         return GQLA_ERR_INVALID_ARG;
     }
     return cuda_status(launch_combine(kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out,
-                                      lse_out, dims->num_heads, dims->num_groups,
+                                      lse_out, dims->num_heads, dims->num_groups, false,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 

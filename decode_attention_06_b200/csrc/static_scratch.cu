@@ -9,7 +9,10 @@
 // plugins handed only their input/output tensors, or hosts whose allocator
 // cannot be called from the decode thread.  This entry point takes the same
 // inputs and the final outputs only; the scratch is the file-scope array
-// below, which every GPU that loads libgqla holds until the process exits.
+// below.  Under CUDA's lazy module loading (the default) a device claims the
+// array when the first call there resolves its address, and holds it until the
+// process exits: that first call belongs at start-up, before serving and
+// before any stream capture.
 #include <mutex>
 
 #include "common.cuh"

@@ -62,6 +62,7 @@ _SIGS = {
     "gqla_absorb_query": [_DP, _P, _I, _I, _P, _P, _P],
     "gqla_decode_absorb": [_DP, _P, _I, _P, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _SZ, _P],
+    "gqla_decode_gqa_step": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "gqla_combine": [_DP, _KP, _I, _I, _I, _P, _P, _P, _P, _P, _P],
     "gqla_sparse_gather": [_DP, _P, _P, _I64, _KP, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "gqla_sparse_select": [_DP, _KP, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
@@ -183,6 +184,24 @@ def gqla_decode_gqa(dims, q, kv_expanded, k_rope, kv, num_splits, o_part, lse_pa
         _dev(k_rope, "k_rope", torch.bfloat16, (n, D_ROPE)), n, ctypes.byref(kv), num_splits,
         _dev(o_part, "o_part", torch.float32, (slots, s_q, h, D_V)),
         _dev(lse_part, "lse_part", torch.float32, (slots, s_q, h)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gqla_decode_gqa_step(dims, q, kv_expanded, k_rope, kv, num_splits, o_part, lse_part, out, lse_out,
+                         workspace, stream=None):
+    """gqla_decode_gqa + gqla_combine in one call; sequences that fall in one chunk get
+    their output from the decode itself (o_part / lse_part may be None for one split)."""
+    B, s_q, h, _ = q.shape
+    n = kv.num_pages * kv.page_size
+    slots = gqla_partial_slots(kv.batch, num_splits)
+    _check("gqla_decode_gqa_step", _lib.gqla_decode_gqa_step(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16, (kv.batch, s_q, dims.num_heads, D_QK)), s_q,
+        _dev(kv_expanded, "kv_expanded", torch.bfloat16, (dims.num_groups, n, D_NOPE + D_V)),
+        _dev(k_rope, "k_rope", torch.bfloat16, (n, D_ROPE)), n, ctypes.byref(kv), num_splits,
+        None if o_part is None else _dev(o_part, "o_part", torch.float32, (slots, s_q, h, D_V)),
+        None if lse_part is None else _dev(lse_part, "lse_part", torch.float32, (slots, s_q, h)),
+        _dev(out, "out", torch.bfloat16, (kv.batch, s_q, h, D_V)),
+        None if lse_out is None else _dev(lse_out, "lse_out", torch.float32, (kv.batch, s_q, h)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
@@ -325,8 +344,9 @@ def gqla_version() -> int:
 
 
 def gqla_debug_drop_v_load(unit: int):
-    """Diagnostic: the next GQA decode of this thread leaves out one V load, so its
-    bounded wait runs out and the call records GQLA_ERR_TIMEOUT (-1 cancels)."""
+    """Diagnostic: the next decode call of this thread leaves out one load (GQA decode:
+    a V load; absorb decode: a latent tile), so its bounded wait runs out and the call
+    records GQLA_ERR_TIMEOUT (-1 cancels)."""
     _check("gqla_debug_drop_v_load", _lib.gqla_debug_drop_v_load(unit))
 
 
@@ -401,9 +421,14 @@ def sparse_gqa_step(dims, bufs: SparseBuffers, q, kv_expanded, k_rope, kv, topk_
 
 
 def decode_step(dims, bufs: DecodeBuffers, q, w_uk, w_uv, kv, latent_cache=None,
-                kv_expanded=None, k_rope=None, stream=None):
+                kv_expanded=None, k_rope=None, stream=None, fused=False):
     """One decode step through the C ABI: absorb path = absorb_query ->
-    decode_absorb -> combine(W_UV); GQA path = decode_gqa -> combine."""
+    decode_absorb -> combine(W_UV); GQA path = decode_gqa -> combine, or with
+    `fused` the one call gqla_decode_gqa_step."""
+    if bufs.path == "gqa" and fused:
+        gqla_decode_gqa_step(dims, q, kv_expanded, k_rope, kv, bufs.num_splits, bufs.o_part,
+                             bufs.lse_part, bufs.out, bufs.lse, bufs.workspace, stream)
+        return bufs.out, bufs.lse
     if bufs.path == "absorb":
         gqla_absorb_query(dims, q, w_uk, bufs.q_absorbed, stream)
         gqla_decode_absorb(dims, bufs.q_absorbed, latent_cache, kv, bufs.num_splits, bufs.o_part,

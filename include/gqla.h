@@ -130,7 +130,10 @@ int gqla_absorb_query(const gqla_dims *dims, const void *q, int batch, int s_q,
 
 /*
  * Split-KV partial attention, MQA-absorb path: every head scores its absorbed
- * query against the latent row and accumulates the 512-d latent.
+ * query against the latent row and accumulates the 512-d latent (paperlayer.ai
+ * summary, sec. 2 "Algebraically equivalent decoding paths" and sec. 4
+ * Roofline Analysis, "MQA-absorb path": one 576-element latent row per token
+ * shared by all heads).
  *   q_absorbed    bf16 [batch][s_q][h][576]
  *   latent_cache  bf16 [num_pages][page_size][576]
  *   kv            page table / lengths (kv->batch is the batch)
@@ -142,10 +145,9 @@ int gqla_absorb_query(const gqla_dims *dims, const void *q, int batch, int s_q,
  *                 scaled scores (-inf for an empty partial); unused slots are not written
  *   workspace  >= gqla_workspace_bytes() bytes of device memory, zeroed once
  *              before first use (holds the device error record)
- * Precision: the two halves of each score (288 latent and RoPE columns each,
- * one per CTA of a pair) are exchanged as fp16 and added in fp32, so very
- * large raw scores (halves beyond a few hundred) lose accuracy; the GQA path
- * forms scores in fp32.
+ * Precision: bf16 operands, every score and the online softmax in fp32 (the
+ * two 288-column halves of a score, computed on the two CTAs of a pair, are
+ * exchanged and added in fp32), P in bf16, O accumulated in fp32.
  */
 int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
                        const void *latent_cache, const gqla_kv_index *kv, int num_splits,
@@ -154,17 +156,38 @@ int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
 
 /*
  * Split-KV partial attention, GQA path: the G*s_q query rows of each group
- * score [K_nope_g | k^R] (192) and accumulate V_g (128).
+ * score [K_nope_g | k^R] (192) and accumulate V_g (128) (paperlayer.ai
+ * summary, sec. 3 "Two equivalent decoding paths" and sec. 4, "GQA path";
+ * pwwt.cn article, sec. 5: h_q/g query heads share a group).
  *   q            bf16 [batch][s_q][h][192]
  *   kv_expanded  bf16 [g][num_slots][256], k_rope bf16 [num_slots][64]
  *                (as written by gqla_expand_cache; num_slots = num_pages * page_size)
  *   o_part  fp32 [gqla_partial_slots(batch, C)][s_q][h][128], lse_part as above.
- * g must be 8 or 4 (GQLA_ERR_UNSUPPORTED otherwise).
+ * g must be 8, 4, 2 or 1 (GQLA_ERR_UNSUPPORTED otherwise; 2 and 1 are a
+ * rank's share of the groups under group-axis tensor parallelism).  Precision:
+ * bf16 operands, scores and softmax in fp32, P in bf16, O in fp32.
  */
 int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
                     const void *k_rope, int64_t num_slots, const gqla_kv_index *kv,
                     int num_splits, float *o_part, float *lse_part, void *workspace,
                     size_t workspace_bytes, gqla_stream_t stream);
+
+/*
+ * The GQA-path step in one call: gqla_decode_gqa, then gqla_combine (d_in =
+ * 128) for the sequences that need it.  A sequence whose pages all fall in one
+ * of the C chunks has a single partial, which is its result: the decode writes
+ * it straight to `out` / `lse_out` in the combine's format, and the combine
+ * leaves it alone.  With C = 1 every sequence is such a sequence and no combine
+ * is launched at all (the single-split fusion: one kernel for the step).
+ *   arguments as for gqla_decode_gqa and gqla_combine; o_part / lse_part may
+ *   be NULL when num_splits == 1 (then nothing is written there); out bf16
+ *   [batch][s_q][h][128] (required), lse_out fp32 [batch][s_q][h] or NULL.
+ * A sequence with no token gets out = 0 and lse = -inf, as from gqla_combine.
+ */
+int gqla_decode_gqa_step(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
+                         const void *k_rope, int64_t num_slots, const gqla_kv_index *kv,
+                         int num_splits, float *o_part, float *lse_part, void *out, float *lse_out,
+                         void *workspace, size_t workspace_bytes, gqla_stream_t stream);
 
 /*
  * Sparse GQLA, GQA path (paperlayer.ai summary, sec. 2 "Sparse GQLA";
@@ -239,6 +262,9 @@ int gqla_decode_gqa_sparse(const gqla_dims *dims, const void *q, int s_q, const 
  * to bf16 (the tensor-core operand type) before the product with W_UV, which
  * accumulates in fp32.  Like gqla_absorb_query this call has no workspace: a
  * bounded device-side wait that runs out leaves `out` unwritten.
+ * Launched right after the decode call that wrote the partials, the combine
+ * reads kv->seqlens (and W_UV) while that decode is still finishing: the
+ * lengths must be the ones the decode call used.
  */
 int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
                  int d_in, const float *o_part, const float *lse_part, const void *w_uv,
@@ -263,11 +289,15 @@ int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int nu
  *   Limit: the partials of (batch + num_splits) * s_q * h rows, 516 bytes
  *   each (rounded up), plus 256 bytes must fit in GQLA_NOALLOC_SCRATCH_BYTES
  *   (32 MiB); larger requests return GQLA_ERR_WORKSPACE before any launch.
- *   Every GPU that loads libgqla reserves this array until the process exits.
- *   Set-up: the first call on each device looks up the array's device address
- *   with cudaGetSymbolAddress (with that device current); make that first
- *   call before any stream capture.  Nothing is allocated or freed, by this
- *   call or by any library it uses.
+ *   When the array is claimed: under CUDA's default lazy module loading the
+ *   32 MiB are taken on a device when the first call there looks up the
+ *   array's device address (cudaGetSymbolAddress, with that device current),
+ *   not when the library is loaded; from then on the device holds them until
+ *   the process exits.  On a device whose memory is nearly all claimed later
+ *   (by a serving allocator), that first call could fail with GQLA_ERR_CUDA:
+ *   make it at start-up, before serving begins and before any stream capture.
+ *   Nothing is allocated or freed by the later calls, nor by any library they
+ *   use.
  *   Sharing: every call on a device uses the same array, which keeps the last
  *   call's contents (the error record is cleared at the start of each call).
  *   Calls that overlap on the GPU -- on different streams, or from different
@@ -315,10 +345,12 @@ int gqla_read_device_error(const void *workspace, int *info, gqla_stream_t strea
 /* Clears the device error record (asynchronously, on `stream`). */
 int gqla_clear_device_error(void *workspace, gqla_stream_t stream);
 
-/* Diagnostic for testing the failure path: the next gqla_decode_gqa (or
- * gqla_decode_gqa_noalloc) call made by this host thread leaves out the V load
- * of work unit `unit` (units count (page pair, group) in issue order within a
- * CTA), so the wait for it runs out after about two seconds: that call then
+/* Diagnostic for testing the failure path: the next decode call made by this
+ * host thread leaves out one load -- gqla_decode_gqa (or
+ * gqla_decode_gqa_noalloc): the V load of work unit `unit` (units count
+ * (page pair, group) in issue order within a CTA); gqla_decode_absorb: the
+ * latent load of tile `unit` (64-token tiles in issue order within a CTA) --
+ * so the wait for it runs out after about two seconds: that call then
  * records GQLA_ERR_TIMEOUT in its workspace, its outputs are unspecified, and
  * the context stays usable.  -1 cancels.  Returns GQLA_OK, or
  * GQLA_ERR_INVALID_ARG for unit < -1. */
