@@ -28,10 +28,12 @@ Timing  = the step is captured into a CUDA graph; the K timed steps are issued
           (device time, no host launch overhead), with an L2 flush (a 256 MiB
           write, then a 256 MiB read so no dirty line is left) before every
           step, outside its events; one synchronize ends the timed region,
-          while an NVML sampler records SM clocks and throttle reasons.  The
-          per-call breakdown comes from a second graph that runs the five
-          calls in order on one stream with an event record around every
-          call.  W >= 3 untimed eager and W graph warm-up steps come first.
+          while an NVML sampler records SM clocks and throttle reasons.  Each
+          path's step ("per_path") is timed the same way from a graph of that
+          path's calls alone; the per-call breakdown ("per_kernel") comes from a
+          graph that runs the five calls in order on one stream with an event
+          record around every call.  W >= 3 untimed eager and W graph warm-up
+          steps come first.
 workload: by default the largest single-GPU configuration of the suite
           (dsv3_h128_b64_l8192_mtp2: 128 heads, 8 groups, 64 sequences of
           8192 tokens, s_q = 2); at N = 1 every other workload of the suite
@@ -300,7 +302,7 @@ class Workbench:
         # that hold two sequences' pieces counted at their cost)
         lens_host = case["seqlens"].cpu()
         self.splits = {"absorb": splits or gqla.plan_splits("absorb", h, s_q, lens_host),
-                       "gqa": splits or gqla.plan_splits("gqa", h, s_q, lens_host)}
+                       "gqa": splits or gqla.plan_splits("gqa", h, s_q, lens_host, fused=True)}
         self.kvx = torch.empty(g, self.n_slots, 256, dtype=torch.bfloat16, device=dev)
         self.kr = torch.empty(self.n_slots, 64, dtype=torch.bfloat16, device=dev)
         self.ba = gqla.DecodeBuffers(dims, self.B, s_q, self.splits["absorb"], "absorb", device=dev)
@@ -386,7 +388,16 @@ class Workbench:
                 self.gev[i].record()
                 c()
             self.gev[-1].record()
-        for g_ in (self.graph, self.graph_ev):
+        # each path's step alone, as a user of that path runs it (its calls back to back on
+        # one stream, each kernel's set-up overlapping its predecessor's tail)
+        self.graph_path = {}
+        for path, cs in (("absorb", self.calls[:3]), ("gqa", [self.gqa_step_call(self.case["q"], self.kv)])):
+            g_ = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_):
+                for c in cs:
+                    c()
+            self.graph_path[path] = g_
+        for g_ in (self.graph, self.graph_ev, *self.graph_path.values()):
             for _ in range(warmup):
                 flush_l2(self.dev)
                 g_.replay()
@@ -406,6 +417,10 @@ class Workbench:
             e1.record(stream)
         torch.cuda.synchronize()
         return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    def time_paths(self, steps):
+        """Mean device time (ms) of each path's step graph."""
+        return {path: sum(self.time_steps(steps, g_)) / steps for path, g_ in self.graph_path.items()}
 
     def time_calls(self, steps):
         per_call = [[] for _ in self.calls]
@@ -485,7 +500,7 @@ class Workbench:
             raise RuntimeError("end-to-end outputs differ from the device results")
         return sum(times) / len(times), h2d, d2h
 
-    def report(self, mean, world, ms_step=None):
+    def report(self, mean, world, path_ms=None):
         """Per-kernel and per-path roofline fractions from the per-call means (ms)."""
         acc, counts = accounting(self.w, self.case, self.s_q, self.splits["gqa"])
         acc_a, _ = accounting(self.w, self.case, self.s_q, self.splits["absorb"])
@@ -524,8 +539,9 @@ class Workbench:
                          "algorithmic_flops_per_launch": acc[dominant]["flops"],
                          "traffic": _stored_traffic(dominant, self.name, self.s_q)})
 
-        def path_info(kernels, dec):
-            us = sum(mean[k] for k in kernels) * 1e3
+        def path_info(kernels, dec, path):
+            # the path's own step graph when timed, else its calls' event-separated times
+            us = (path_ms[path] if path_ms else sum(mean[k] for k in kernels)) * 1e3
             t_m = acc[dec]["bytes"] / (hbm_peak * 1e9)
             t_c = acc[dec]["flops"] / (tc_peak * 1e12)
             bound = "tensor" if t_c > t_m else "hbm"
@@ -535,8 +551,8 @@ class Workbench:
                     "binding_roofline_frac": frac, "hbm_frac": per_kernel[dec]["hbm_frac"],
                     "tensor_frac": per_kernel[dec]["tensor_frac"]}
 
-        per_path = {"absorb": path_info(["absorb_query", "decode_absorb", "combine_absorb"], "decode_absorb"),
-                    "gqa": path_info(["decode_gqa", "combine_gqa"], "decode_gqa")}
+        per_path = {"absorb": path_info(["absorb_query", "decode_absorb", "combine_absorb"], "decode_absorb", "absorb"),
+                    "gqa": path_info(["decode_gqa", "combine_gqa"], "decode_gqa", "gqa")}
         return roofline, per_path, per_kernel, acc
 
     def config(self, world):
@@ -564,8 +580,9 @@ def measure_other_workloads(args, headline, dev):
             wb.capture(args.warmup)
             ms = wb.time_steps(args.steps)
             mean = wb.time_calls(args.steps)
+            path_ms = wb.time_paths(args.steps)
             wb.check_device_errors()
-            _, per_path, per_kernel, _ = wb.report(mean, 1)
+            _, per_path, per_kernel, _ = wb.report(mean, 1, path_ms)
             out[f"{name}/sq{s}"] = {
                 "ms_per_step": sum(ms) / len(ms),
                 "tokens_per_s": wb.B * s / (sum(ms) / len(ms) * 1e-3),
@@ -651,13 +668,14 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ms_step = sum(step_ms) / args.steps
     mean = wb.time_calls(args.steps)
+    path_ms = wb.time_paths(args.steps)
     wb.check_device_errors()
     e2e_ms, h2d, d2h = wb.e2e(args.steps, args.warmup)
 
     # ---- max over ranks
     tokens_step = wb.B * wb.s_q
     ms_step, e2e_ms, value, e2e_value = aggregate_over_ranks(ms_step, e2e_ms, world, tokens_step, dev)
-    roofline, per_path, per_kernel, acc = wb.report(mean, world)
+    roofline, per_path, per_kernel, acc = wb.report(mean, world, path_ms)
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -32,16 +32,19 @@
 //                  of tile j: the fp32 partial scores of the CTA's own rows go to its
 //                  local buffer, those of the peer's rows to a staging block that
 //                  leaves as one 2 KB bulk copy per warp into the peer's receive buffer.
-//                  Stage C of tile j - 1: once P of all rows is in, O rows whose
-//                  maximum rose are rescaled and PV is released.  Also each piece's
-//                  RoPE q~ (by TMA, as soon as the previous piece's scores are
-//                  complete) and the epilogue;
+//                  Stage C of tile j - 1, only when the PV warp asks for it: O rows
+//                  whose maximum rose are rescaled.  Also each piece's RoPE q~ (by
+//                  TMA, as soon as the previous piece's scores are complete) and the
+//                  epilogue;
 //      warps 10-17 softmax warps of the CTA's 64 rows (stage B), four lanes per
 //                  row: the two fp32 partials added, row maxima (lazy rescaling: a
 //                  maximum has to rise by more than 2^8), P = 2^(s - m) written to
-//                  both CTAs' P buffers (bulk copy of each warp's 8 rows); also the
+//                  both CTAs' P buffers (bulk copy of each warp's 8 rows, and one of
+//                  their rescale factors); also the
 //                  q~ copies into TMEM, each piece's next q~ prefetched into L2;
-//      warp 18     issues O += P C in tile order.
+//      warp 18     waits for P of all 128 rows and issues O += P C in tile order; it
+//                  zeroes the latent rows past a ragged sequence end and hands a tile to
+//                  the score warps (stage C) only when some row's maximum rose.
 //    The stages of consecutive tiles overlap: the score warps run A(j) while the
 //    softmax warps run B(j - 1).  Every score is the fp32 sum of two fp32
 //    partials: no precision is given up in the exchange.
@@ -90,12 +93,13 @@ struct AbsorbSmem {
     // of one lane quadrant in one half are what one score warp computes, 2 KB in one piece,
     // so the peer's blocks arrive as whole bulk copies.  Read 16 tokens per lane (four
     // lanes per row).  One buffer for this CTA's partials and one for the peer's: the
-    // softmax warps of both CTAs read tile j at the start of their stage B, before either
-    // CTA's score warps write tile j + 1 (which waits for that).
+    // softmax warps of both CTAs read tile j at the start of their stage B; the score warps
+    // write tile j + 1 into the local buffer once this CTA's softmax warps have read it and
+    // send it into the peer's once the peer's have.
     static constexpr int kX = kOwn * kT * 4;
     static constexpr int kXBlock = 16 * 32 * 4;           // one score warp's block, 2 KB
     static constexpr int kP = kRows * kT * 2;             // P, [128 rows][64 tokens] bf16, 128B-swizzled
-    // the peer's 64 rows of P (bulk copies) and their O rescale factors (st.async)
+    // the peer's 64 rows of P and their O rescale factors (bulk copies)
     static constexpr int kPRemote = kOwn * kT * 2 + kOwn * 4;
     static constexpr int oQ = 0;
     static constexpr int oP = oQ + kQRope;                // 2 buffers
@@ -108,9 +112,10 @@ struct AbsorbSmem {
     static constexpr int oL = oAlpha + 2 * kRows * 4;     // float [128 rows]: row sums of a piece
     static constexpr int oBar = oL + kRows * 4;
     // ring_full/empty[kRing], rope_full/empty[kRopeRing], q_full, s_full/s_free[2],
-    // x_full, x_empty, p_full/p_empty[2], o_ready[2], pv_done[2], l_full, o_done, drain[2]
-    static constexpr int kNumBars = 2 * kRing + 2 * kRopeRing + 1 + 4 + 2 + 4 + 2 + 2 + 1 + 1 + 2;
-    static constexpr int oMisc = oBar + kNumBars * 8;     // tmem base, abort, plan[4]
+    // x_full, x_empty_l, x_empty_r, p_full/p_empty[2], o_ready, c_dec[2], pv_done[2], l_full,
+    // o_done, drain[2]
+    static constexpr int kNumBars = 2 * kRing + 2 * kRopeRing + 1 + 4 + 3 + 4 + 3 + 2 + 1 + 1 + 2;
+    static constexpr int oMisc = oBar + kNumBars * 8;     // tmem base, abort, plan[4], c_flag[2]
     static constexpr int kBytes = oMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;
 };
@@ -189,13 +194,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint64_t *rope_full = bars + 2 * kRing, *rope_empty = rope_full + SM::kRopeRing;
     uint64_t *q_full = rope_empty + SM::kRopeRing;
     uint64_t *s_full = q_full + 1, *s_free = s_full + 2;
-    uint64_t *x_full = s_free + 2, *x_empty = x_full + 1;
-    uint64_t *p_full = x_empty + 1, *p_empty = p_full + 2;
-    uint64_t *o_ready = p_empty + 2, *pv_done = o_ready + 2;
+    uint64_t *x_full = s_free + 2, *x_empty_l = x_full + 1, *x_empty_r = x_empty_l + 1;
+    uint64_t *p_full = x_empty_r + 1, *p_empty = p_full + 2;
+    uint64_t *o_ready = p_empty + 2, *c_dec = o_ready + 1, *pv_done = c_dec + 2;
     uint64_t *l_full = pv_done + 2, *o_done = l_full + 1, *drain = o_done + 1;
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(smem + SM::oMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::oMisc + 4);
     int *plan = reinterpret_cast<int *>(smem + SM::oMisc + 8);
+    // per P buffer: whether the score warps rescale O rows before that tile's PV
+    volatile int *c_flag = reinterpret_cast<volatile int *>(smem + SM::oMisc + 24);
     GQLA_PROF_DECL;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -211,15 +218,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = 0; i < SM::kRopeRing; ++i) { mbar_init(&rope_full[i], 1); mbar_init(&rope_empty[i], 1); }
         mbar_init(q_full, 1 + kYWarps);  // RoPE TMA + the softmax warps' TMEM copies
         mbar_init(x_full, 1 + kXWarps);  // expect_tx of the peer's partials + local score warps
-        mbar_init(x_empty, 2 * kYWarps); // every softmax warp of both CTAs has read both buffers
+        mbar_init(x_empty_l, kYWarps);   // this CTA's softmax warps have read both buffers
+        mbar_init(x_empty_r, kYWarps);   // the peer's softmax warps have read both of theirs
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1); mbar_init(&s_free[i], kXThreads);
             mbar_init(&p_full[i], 1 + kYWarps);      // expect_tx of the peer's rows + local softmax warps
             mbar_init(&p_empty[i], 2);               // PV of both CTAs done with the buffer
-            mbar_init(&o_ready[i], kXWarps);
+            mbar_init(&c_dec[i], 1);
             mbar_init(&pv_done[i], 1);
             mbar_init(&drain[i], 1);
         }
+        mbar_init(o_ready, kXWarps);  // only for tiles whose O rows the score warps rescale
         mbar_init(l_full, 1 + kYWarps);
         mbar_init(o_done, 1);
         *abort_flag = 0;
@@ -268,6 +277,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t sm_q = smem_u32(smem + SM::oQ);
     const uint32_t sm_ring = smem_u32(smem + SM::oRing);
     const uint32_t sm_p = smem_u32(smem + SM::oP);
+    // A thread whose wait runs out stops its CTA and the peer (both abort flags): every
+    // role then leaves its loops at its next wait.  After a failed wait a role neither
+    // arrives on a barrier nor sends anything -- an arrival for tile j + 1 on a barrier
+    // whose phase j still waits for bytes would break the barrier's count -- so the
+    // only traffic left is what was already in flight.
+    const uint32_t abort_remote = map_peer(smem_u32(const_cast<int *>(abort_flag)), peer);
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        st_cluster_b32(abort_remote, 1u);
+    };
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
@@ -276,59 +295,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint64_t stream_policy = l2_evict_first_policy();  // the cache is read once
         PieceIter it = it0;
         int b, L, pb, pe;
-        bool too_long;
-        uint32_t t = 0, k = 0;
-        while (next_piece(p, it, b, L, pb, pe, too_long)) {
+        bool too_long, quit = false;
+        uint32_t t = 0, n_rope = 0;  // tiles whose latent / RoPE slot was armed (or skipped)
+        while (!quit && next_piece(p, it, b, L, pb, pe, too_long)) {
             if (too_long) {
                 if (lane == 0 && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
                 continue;
             }
             const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
-            for (int i0 = pb; i0 < pe; i0 += 32) {
+            for (int i0 = pb; i0 < pe && !quit; i0 += 32) {
                 const int n = min(32, pe - i0);
                 // (the first piece is the one the early load above was for)
                 const int my_page = pre_ok ? pre_page : (lane < n ? prow[i0 + lane] : 0);
                 pre_ok = false;
-                for (int j = 0; j < n; ++j, ++t) {
+                for (int j = 0; j < n; ++j) {
                     const int page = __shfl_sync(0xffffffffu, my_page, j);
+                    int ok = 1;
                     if (lane == 0) {
                         const bool bad = page < 0 || page >= p.num_pages;
                         if (bad && rank == 0 && rb == 0) report_error(p.ws, GQLA_ERR_DEVICE, b);
                         const int slot = t % kRing, rs = t % SM::kRopeRing;
-                        if (!GQLA_WAIT(0, &ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                        uint8_t *dst = smem + SM::oRing + slot * SM::kSlot;
-                        if ((int)t == p.drop_tile) {
-                            // diagnostic: neither the load nor an arrival for this tile
-                        } else if (!bad && !*abort_flag) {
-                            mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
+                        if (!GQLA_WAIT(0, &ring_empty[slot], ((t / kRing) & 1) ^ 1, abort_flag)) {
+                            give_up();
+                            ok = 0;
+                        } else {
+                            uint8_t *dst = smem + SM::oRing + slot * SM::kSlot;
+                            if ((int)t == p.drop_tile) {
+                                // diagnostic: neither the load nor an arrival for this tile
+                            } else if (!bad) {
+                                mbar_arrive_expect_tx(&ring_full[slot], SM::kSlot);
 #pragma unroll
-                            for (int bx = 0; bx < 4; ++bx)
-                                tma_load_2d_hint(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
-                                                 256 * rank + 64 * bx, page * kPage, stream_policy);
-                        } else {
-                            mbar_arrive(&ring_full[slot]);
+                                for (int bx = 0; bx < 4; ++bx)
+                                    tma_load_2d_hint(dst + bx * SM::kLatBox, &lat_map, &ring_full[slot],
+                                                     256 * rank + 64 * bx, page * kPage, stream_policy);
+                            } else {
+                                mbar_arrive(&ring_full[slot]);
+                            }
+                            ++t;
+                            // the RoPE slot frees once the score MMAs of tile t - kRopeRing are done
+                            if (!GQLA_WAIT(1, &rope_empty[rs], ((n_rope / SM::kRopeRing) & 1) ^ 1, abort_flag)) {
+                                give_up();
+                                ok = 0;
+                            } else {
+                                if (!bad) {
+                                    mbar_arrive_expect_tx(&rope_full[rs], SM::kRopeBox);
+                                    tma_load_2d_hint(smem + SM::oRope + rs * SM::kRopeBox, &rope_map, &rope_full[rs],
+                                                     512 + 32 * rank, page * kPage, stream_policy);
+                                } else {
+                                    mbar_arrive(&rope_full[rs]);
+                                }
+                                ++n_rope;
+                            }
                         }
-                        // the RoPE slot frees once the score MMAs of tile t - kRopeRing are done
-                        if (!GQLA_WAIT(1, &rope_empty[rs], ((t / SM::kRopeRing) & 1) ^ 1, abort_flag)) *abort_flag = 1;
-                        if (!bad && !*abort_flag) {
-                            mbar_arrive_expect_tx(&rope_full[rs], SM::kRopeBox);
-                            tma_load_2d_hint(smem + SM::oRope + rs * SM::kRopeBox, &rope_map, &rope_full[rs],
-                                             512 + 32 * rank, page * kPage, stream_policy);
-                        } else {
-                            mbar_arrive(&rope_full[rs]);
-                        }
+                    }
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                        quit = true;
+                        break;
                     }
                 }
             }
-            ++k;
         }
         if (lane == 0) {
-            // no TMA may still be writing when the CTA exits
+            // no TMA may still be writing when the CTA exits: wait (bounded) for the last
+            // loads of both rings (a slot left without its load, on purpose or by giving
+            // up, just lets its wait run out)
             int dummy = 0;
             volatile int *no_abort = reinterpret_cast<volatile int *>(&dummy);
             for (uint32_t u = (t > (uint32_t)kRing ? t - kRing : 0); u < t; ++u)
                 mbar_wait(&ring_full[u % kRing], (u / kRing) & 1, no_abort);
-            for (uint32_t u = (t > (uint32_t)SM::kRopeRing ? t - SM::kRopeRing : 0); u < t; ++u)
+            for (uint32_t u = (n_rope > (uint32_t)SM::kRopeRing ? n_rope - SM::kRopeRing : 0); u < n_rope; ++u)
                 mbar_wait(&rope_full[u % SM::kRopeRing], (u / SM::kRopeRing) & 1, no_abort);
         }
     } else if (warp == 1) {
@@ -344,27 +379,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int b, L, pb, pe;
             bool too_long;
             uint32_t t = 0, k = 0;
-            while (next_piece(p, it, b, L, pb, pe, too_long)) {
+            bool quit = false;
+            while (!quit && next_piece(p, it, b, L, pb, pe, too_long)) {
                 if (too_long) continue;
-                if (!GQLA_WAIT(2, q_full, k & 1, abort_flag)) *abort_flag = 1;
+                if (!GQLA_WAIT(2, q_full, k & 1, abort_flag)) {
+                    give_up();
+                    break;
+                }
                 for (int i = 0; i < pe - pb; ++i, ++t) {
                     const int slot = t % kRing, sb = t & 1, rs = t % SM::kRopeRing;
-                    if (!GQLA_WAIT(3, &ring_full[slot], (t / kRing) & 1, abort_flag)) *abort_flag = 1;
-                    if (!GQLA_WAIT(3, &rope_full[rs], (t / SM::kRopeRing) & 1, abort_flag)) *abort_flag = 1;
-                    if (!GQLA_WAIT(4, &s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                    if (!GQLA_WAIT(3, &ring_full[slot], (t / kRing) & 1, abort_flag) ||
+                        !GQLA_WAIT(3, &rope_full[rs], (t / SM::kRopeRing) & 1, abort_flag) ||
+                        !GQLA_WAIT(4, &s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) {
+                        give_up();
+                        quit = true;
+                        break;
+                    }
                     tc_fence_after();
                     const uint64_t lat_d = desc_advance(lat_d0, slot * SM::kSlot);
                     const uint64_t rope_d = desc_advance(rope_d0, rs * SM::kRopeBox);
                     const uint32_t t_sb = t_s + sb * kT;
-                    if (!*abort_flag) {
 #pragma unroll
-                        for (int ks = 0; ks < 16; ++ks)  // latent: A = q~ in TMEM, 16 dims = 8 columns
-                            mma_bf16_ts(t_sb, t_q + ks * 8, desc_advance(lat_d, (ks >> 2) * SM::kLatBox + (ks & 3) * 32),
-                                        idesc_s, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < 16; ++ks)  // latent: A = q~ in TMEM, 16 dims = 8 columns
+                        mma_bf16_ts(t_sb, t_q + ks * 8, desc_advance(lat_d, (ks >> 2) * SM::kLatBox + (ks & 3) * 32),
+                                    idesc_s, ks > 0 ? 1u : 0u);
 #pragma unroll
-                        for (int ks = 0; ks < 2; ++ks)  // RoPE: 32 columns, 64B-swizzled rows
-                            mma_bf16(t_sb, desc_advance(q_d0, ks * 32), desc_advance(rope_d, ks * 32), idesc_s, 1u);
-                    }
+                    for (int ks = 0; ks < 2; ++ks)  // RoPE: 32 columns, 64B-swizzled rows
+                        mma_bf16(t_sb, desc_advance(q_d0, ks * 32), desc_advance(rope_d, ks * 32), idesc_s, 1u);
                     mma_commit(&s_full[sb]);
                     mma_commit(&rope_empty[rs]);
                 }
@@ -376,36 +417,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kPvWarp) {
         // ---------------------------------------------------------------- PV MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_pv = idesc_bf16(kRows, 256, 0, 1);
-            const uint64_t v_d0 = smem_desc(sm_ring, SM::kLatBox, 1024, kSw128);
-            const uint64_t p_d0 = smem_desc(sm_p, 16, 1024, kSw128);
-            PieceIter it = it0;
-            int b, L, pb, pe;
-            bool too_long;
-            uint32_t t = 0;
-            while (next_piece(p, it, b, L, pb, pe, too_long)) {
-                if (too_long) continue;
-                for (int i = 0; i < pe - pb; ++i, ++t) {
-                    const int slot = t % kRing, sb = t & 1;
-                    if (!GQLA_WAIT(5, &o_ready[sb], (t >> 1) & 1, abort_flag)) *abort_flag = 1;
+        // The whole warp waits for P of all 128 rows, checks their O rescale factors and
+        // zeroes the latent rows of a ragged tile; lane 0 issues.  Only when some factor is
+        // not 1 (a row maximum rose) does it hand the tile to the score warps (c_flag, c_dec)
+        // and wait for their rescaling (o_ready) first; otherwise PV follows P at once.
+        const float *alph = reinterpret_cast<const float *>(smem + SM::oAlpha);
+        constexpr uint32_t idesc_pv = idesc_bf16(kRows, 256, 0, 1);
+        const uint64_t v_d0 = smem_desc(sm_ring, SM::kLatBox, 1024, kSw128);
+        const uint64_t p_d0 = smem_desc(sm_p, 16, 1024, kSw128);
+        PieceIter it = it0;
+        int b, L, pb, pe;
+        bool too_long;
+        uint32_t t = 0, n_c = 0;  // n_c: tiles handed to the score warps so far
+        bool quit = false;
+        while (!quit && next_piece(p, it, b, L, pb, pe, too_long)) {
+            if (too_long) continue;
+            const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
+            for (int i = 0; i < pe - pb; ++i, ++t) {
+                const int slot = t % kRing, sb = t & 1;
+                const int page = prow[pb + i];
+                if (!__all_sync(0xffffffffu, GQLA_WAITC(5, &p_full[sb], (t >> 1) & 1, abort_flag))) {
+                    if (lane == 0) give_up();
+                    quit = true;
+                    break;
+                }
+                // P buffer sb takes tile t + 2's rows from the peer, which the peer sends only
+                // after PV(t) below has freed the buffer in both CTAs
+                if (lane == 0) mbar_arrive_expect_tx(&p_full[sb], SM::kPRemote);
+                const float4 a4 = reinterpret_cast<const float4 *>(alph + sb * kRows)[lane];
+                const bool need_c =
+                    __any_sync(0xffffffffu, a4.x != 1.0f || a4.y != 1.0f || a4.z != 1.0f || a4.w != 1.0f);
+                const bool bad = page < 0 || page >= p.num_pages;
+                const int n_valid = bad ? 0 : max(0, min(kT, L - (pb + i) * kPage));
+                if (n_valid < kT) {
+                    // latent rows that are not tokens (never written, maybe NaN) -> 0, once the
+                    // tile's load has landed
+                    if (!__all_sync(0xffffffffu, mbar_wait(&ring_full[slot], (t / kRing) & 1, abort_flag))) {
+                        if (lane == 0) give_up();
+                        quit = true;
+                        break;
+                    }
+                    uint8_t *tile = smem + SM::oRing + slot * SM::kSlot;
+                    const int nz = kT - n_valid;
+                    for (int z = lane; z < 4 * nz * 8; z += 32) {
+                        const int box = z / (nz * 8), rem = z % (nz * 8);
+                        *reinterpret_cast<uint4 *>(tile + box * SM::kLatBox + (n_valid + rem / 8) * 128 +
+                                                   (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();  // the zeros -> the PV MMAs (async proxy)
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    c_flag[sb] = need_c ? 1 : 0;
+                    mbar_arrive(&c_dec[sb]);
+                }
+                if (need_c) {
+                    if (!__all_sync(0xffffffffu, GQLA_WAIT(10, o_ready, n_c & 1, abort_flag))) {
+                        if (lane == 0) give_up();
+                        quit = true;
+                        break;
+                    }
+                    ++n_c;
+                }
+                if (lane == 0) {
                     tc_fence_after();
                     // B = C_lat[tokens][256 cols of this CTA]: MN-major, 4 atoms of 64 columns;
                     // A = P[128 rows][64 tokens], K-major: 16 tokens = 32 bytes of a row
                     const uint64_t v_d = desc_advance(v_d0, slot * SM::kSlot);
                     const uint64_t p_d = desc_advance(p_d0, sb * SM::kP);
-                    if (!*abort_flag) {
 #pragma unroll
-                        for (int ks = 0; ks < kT / 16; ++ks)
-                            mma_bf16(t_o, desc_advance(p_d, ks * 32), desc_advance(v_d, ks * 2048), idesc_pv,
-                                     (i == 0 && ks == 0) ? 0u : 1u);
-                    }
+                    for (int ks = 0; ks < kT / 16; ++ks)
+                        mma_bf16(t_o, desc_advance(p_d, ks * 32), desc_advance(v_d, ks * 2048), idesc_pv,
+                                 (i == 0 && ks == 0) ? 0u : 1u);
                     mma_commit_multicast(&p_empty[sb], 0x3);  // P buffer sb of both CTAs is free
                     mma_commit(&pv_done[sb]);
                     mma_commit(&ring_empty[slot]);
                 }
-                mma_commit(o_done);
+                __syncwarp();
             }
+            if (!quit && lane == 0) mma_commit(o_done);
+        }
+        if (lane == 0) {
             mma_commit(&drain[1]);
             int dummy = 0;
             mbar_wait(&drain[1], 0, reinterpret_cast<volatile int *>(&dummy));
@@ -414,8 +506,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------------- score warps
         // Stage A of tile j: fp32 partial scores -> the owner of each row (row r of the
         // block belongs to rank (r / 16) % 2, so both CTAs use all four TMEM lane quadrants);
-        // stage C of tile j - 1: once P and the rescale factors of all 128 rows are in,
-        // O rows are rescaled where a row maximum rose and PV is released.  Also the q~
+        // stage C of tile j - 1, when the PV warp found a rescale factor that is not 1: O
+        // rows are rescaled where a row maximum rose and PV is released.  Also the q~
         // copies into TMEM and the epilogue.  Two warps per lane quadrant: warp half
         // `xpart` takes tokens [32 xpart, 32 xpart + 32) of a tile and O columns
         // [128 xpart, 128 xpart + 128).
@@ -456,13 +548,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int b_next = 0;
             const bool more_pieces = another_piece(p, it, b_next);  // its tiles then occupy the ring
             rope_issued = more_pieces;
-            const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
             const uint32_t t0 = t;
             const int nt = pe - pb;
-            auto stage_a = [&](int i) {
+            // Each stage returns false when a wait failed (in any lane): the warp then stops.
+            auto stage_a = [&](int i) -> bool {
                 const uint32_t tt = t0 + i;
                 const int sb = tt & 1;
-                if (!GQLA_WAIT(6, &s_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
+                if (!__all_sync(0xffffffffu, GQLA_WAIT(6, &s_full[sb], (tt >> 1) & 1, abort_flag))) {
+                    if (lane == 0) give_up();
+                    return false;
+                }
                 GQLA_SPAN_BEGIN(t_a);
                 tc_fence_after();
                 uint32_t sv[kXTok];
@@ -471,9 +566,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&s_free[sb]);
-                // both buffers (this CTA's, and the peer's receive buffer) are free once the
-                // softmax warps of both CTAs have read tile tt - 1
-                if (!GQLA_WAITC(7, x_empty, (tt & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                // this CTA's buffer is free once its softmax warps have read tile tt - 1
+                if (!__all_sync(0xffffffffu, GQLA_WAIT(7, x_empty_l, (tt & 1) ^ 1, abort_flag))) {
+                    if (lane == 0) give_up();
+                    return false;
+                }
                 if (xw == 0 && lane == 0) mbar_arrive_expect_tx(x_full, SM::kX);
                 // this lane's row, tokens 32 xpart .. 32 xpart + 31: the CTA's own rows into the
                 // local buffer, the peer's rows into this warp's staging block (the peer's half
@@ -493,27 +590,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         make_uint4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
                 fence_proxy_async_smem();  // the staging block -> the bulk copy (async proxy)
                 __syncwarp();
+                if (lane == 0) mbar_arrive(x_full);  // this warp's local partials are in
+                // the peer's receive buffer is free once the peer's softmax warps have read tile
+                // tt - 1
+                if (!__all_sync(0xffffffffu, GQLA_WAITC(7, x_empty_r, (tt & 1) ^ 1, abort_flag))) {
+                    if (lane == 0) give_up();
+                    return false;
+                }
                 if (lane == 0) {
                     bulk_copy_to_peer(x_remote + xpart * (kOwn * 128) + 16 * quad * 128,
                                       smem + SM::oXStage + xw * SM::kXBlock, SM::kXBlock, xfull_remote);
                     bulk_commit_group();
-                    mbar_arrive(x_full);  // this warp's local partials are in
                 }
                 GQLA_SPAN_END(13, t_a);
+                return true;
             };
-            auto stage_c = [&](int i, int page) {
+            auto stage_c = [&](int i) -> bool {
                 const uint32_t tt = t0 + i;
-                const int sb = tt & 1, slot = tt % kRing;
-                const bool bad = page < 0 || page >= p.num_pages;
-                const int n_valid = bad ? 0 : max(0, min(kT, L - (pb + i) * kPage));
-                if (!GQLA_WAITC(11, &p_full[sb], (tt >> 1) & 1, abort_flag)) *abort_flag = 1;
+                const int sb = tt & 1;
+                if (!__all_sync(0xffffffffu, GQLA_WAIT(11, &c_dec[sb], (tt >> 1) & 1, abort_flag))) {
+                    if (lane == 0) give_up();
+                    return false;
+                }
+                if (!c_flag[sb]) return true;  // no factor is not 1: PV(tt) needs nothing from here
                 GQLA_SPAN_BEGIN(t_c);
-                if (xw == 0 && lane == 0) mbar_arrive_expect_tx(&p_full[sb], SM::kPRemote);  // tile tt + 2
                 const float alpha = alph[sb * kRows + row];
                 if (__any_sync(0xffffffffu, alpha != 1.0f)) {
                     // O rows are rescaled only after PV(tt - 1) has completed
-                    if (i > 0)
-                        if (!mbar_wait(&pv_done[(tt - 1) & 1], ((tt - 1) >> 1) & 1, abort_flag)) *abort_flag = 1;
+                    if (i > 0 && !__all_sync(0xffffffffu, mbar_wait(&pv_done[(tt - 1) & 1], ((tt - 1) >> 1) & 1, abort_flag))) {
+                        if (lane == 0) give_up();
+                        return false;
+                    }
                     tc_fence_after();
 #pragma unroll 1
                     for (int c16 = 0; c16 < kXCols; c16 += 16) {
@@ -527,36 +634,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     tmem_wait_st();
                 }
-                // latent rows that are not tokens (never written, maybe NaN) -> 0
-                if (n_valid < kT) {
-                    if (!mbar_wait(&ring_full[slot], (tt / kRing) & 1, abort_flag)) *abort_flag = 1;
-                    uint8_t *tile = smem + SM::oRing + slot * SM::kSlot;
-                    const int nz = kT - n_valid;
-                    for (int z = xw * 32 + lane; z < 4 * nz * 8; z += kXThreads) {
-                        const int box = z / (nz * 8), rem = z % (nz * 8);
-                        *reinterpret_cast<uint4 *>(tile + box * SM::kLatBox + (n_valid + rem / 8) * 128 +
-                                                   (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&o_ready[sb]);
+                if (lane == 0) mbar_arrive(o_ready);
                 GQLA_SPAN_END(18, t_c);
+                return true;
             };
-            int page_prev = 0;
-            for (int j = 0; j <= nt; ++j) {
-                const int page_j = j < nt ? prow[pb + j] : 0;
-                GQLA_SPAN_BEGIN(t_tile);
-                if (j < nt) {
-                    stage_a(j);
-                    // the piece's last scores are complete: the next piece's RoPE q~ may come
-                    if (j == nt - 1 && more_pieces) load_rope(b_next);
+            // The two stages run in whichever order their inputs arrive: lane 0 probes,
+            // without blocking, the PV warp's decision for the oldest tile still waiting for
+            // stage C (first: when it asks for rescaling, its PV holds up the ring) and then
+            // the scores of the next tile with the peer's receive buffer free (stage A), and
+            // the warp runs the first one that is ready.  Stage A runs at most one tile ahead
+            // of stage C, so the PV warp's decision for tile j + 2 (same flag, same barrier)
+            // cannot come before this warp has read the one for tile j.  With nothing ready
+            // for kWaitCycles (or after an abort) the warp falls back to the stage's own
+            // bounded wait, which then reports.
+            int ia = 0, ic = 0;
+            bool ok = true;
+            long long idle_since = clock64();
+            while (ok && ic < nt) {
+                int act = 0;  // 1: stage A of tile ia, 2: stage C of tile ic
+                if (lane == 0) {
+                    const uint32_t ta = t0 + ia, tc = t0 + ic;
+                    if (ic < ia && mbar_test_wait(&c_dec[tc & 1], (tc >> 1) & 1)) act = 2;
+                    else if (ia < nt && ia <= ic + 1 && mbar_test_wait(&s_full[ta & 1], (ta >> 1) & 1) &&
+                             mbar_test_wait(x_empty_l, (ta & 1) ^ 1)) act = 1;
+                    else if (*abort_flag || clock64() - idle_since > kWaitCycles) act = ic < ia ? 2 : 1;
                 }
-                if (j >= 1) stage_c(j - 1, page_prev);
-                GQLA_SPAN_END(10, t_tile);
-                page_prev = page_j;
+                act = __shfl_sync(0xffffffffu, act, 0);
+                if (act == 1) {
+                    ok = stage_a(ia);
+                    if (ok && ia == nt - 1 && more_pieces) load_rope(b_next);
+                    ++ia;
+                    idle_since = clock64();
+                } else if (act == 2) {
+                    ok = stage_c(ic);
+                    ++ic;
+                    idle_since = clock64();
+                } else {
+                    __nanosleep(32);
+                }
             }
+            if (!ok) break;
             t = t0 + nt;
             // ---- epilogue: O / l for this warp's 32 rows x 128 columns through TMA stores of
             // 32 x 32 fp32 boxes (128-byte swizzle) staged in shared memory.  After the last
@@ -565,8 +684,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // one box at a time in the P buffers (free once the piece's last PV is done; P of
             // the next piece is written only after this warp's next scores).
             GQLA_SPAN_BEGIN(t_epi);
-            if (!GQLA_WAIT(15, o_done, k & 1, abort_flag)) *abort_flag = 1;
-            if (!GQLA_WAIT(12, l_full, k & 1, abort_flag)) *abort_flag = 1;
+            if (!__all_sync(0xffffffffu, GQLA_WAIT(15, o_done, k & 1, abort_flag) &&
+                                             GQLA_WAIT(12, l_full, k & 1, abort_flag))) {
+                if (lane == 0) give_up();
+                break;
+            }
             tc_fence_after();
             const float l = lsm[row];
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
@@ -594,7 +716,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0 && quad_live && !*abort_flag) {
+                if (lane == 0 && quad_live) {
                     tma_store_2d(&o_map, stg, ocol0 + 32 * m, orow0);
                     bulk_commit_group();
                 }
@@ -628,7 +750,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
         float *alph = reinterpret_cast<float *>(smem + SM::oAlpha);
         float *lsm = reinterpret_cast<float *>(smem + SM::oL);
-        const uint32_t xempty_remote = map_peer(smem_u32(x_empty), peer);
+        const uint32_t xempty_remote = map_peer(smem_u32(x_empty_r), peer);
         const uint32_t p_remote = map_peer(sm_p, peer);
         const uint32_t pfull_remote = map_peer(smem_u32(p_full), peer);
         const uint32_t alpha_remote = map_peer(smem_u32(alph), peer);
@@ -667,7 +789,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int b, L, pb, pe;
         bool too_long;
         uint32_t t = 0;
-        while (next_piece(p, it, b, L, pb, pe, too_long)) {
+        bool quit = false;
+        while (!quit && next_piece(p, it, b, L, pb, pe, too_long)) {
             if (too_long) continue;
             if (!q_loaded) copy_q(b);
             q_loaded = false;
@@ -697,7 +820,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const bool bad = page < 0 || page >= p.num_pages;
                 const int n_valid = bad ? 0 : max(0, min(kT, L - tok0));
                 GQLA_SPAN_BEGIN(t_b0);
-                if (!GQLA_WAITC(8, x_full, tt & 1, abort_flag)) *abort_flag = 1;
+                if (!__all_sync(0xffffffffu, GQLA_WAITC(8, x_full, tt & 1, abort_flag))) {
+                    if (lane == 0) give_up();
+                    quit = true;
+                    break;
+                }
                 GQLA_SPAN_BEGIN(t_b);
                 // this row's tokens 16 bq4 .. 16 bq4 + 15 from both partials (fp32), added in fp32
                 float x[16];
@@ -719,8 +846,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // both CTAs' buffers may be refilled once every softmax warp of the pair has
                 // read them
                 if (lane == 0) {
-                    mbar_arrive(x_empty);
-                    mbar_arrive_remote(xempty_remote);
+                    mbar_arrive(x_empty_l);
+                    mbar_arrive_remote_relaxed(xempty_remote);
                 }
                 // mask tokens past the sequence or past this query's causal limit
                 const int lim = min(last_visible, tok0 + n_valid - 1) - (tok0 + 16 * bq4);
@@ -754,32 +881,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 l_run += lsum;
                 GQLA_SPAN_END(14, t_b);
                 // P buffer sb of both CTAs is free once both PV(tt - 2) are done
-                if (!GQLA_WAIT(9, &p_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag)) *abort_flag = 1;
+                if (!__all_sync(0xffffffffu, GQLA_WAIT(9, &p_empty[sb], ((tt >> 1) & 1) ^ 1, abort_flag))) {
+                    if (lane == 0) give_up();
+                    quit = true;
+                    break;
+                }
                 GQLA_SPAN_BEGIN(t_b2);
                 uint8_t *prow_s = smem + SM::oP + sb * SM::kP + brow * 128;
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     *reinterpret_cast<uint4 *>(prow_s + (((2 * bq4 + h) ^ (brow & 7)) << 4)) =
                         make_uint4(pw[4 * h], pw[4 * h + 1], pw[4 * h + 2], pw[4 * h + 3]);
-                if (bq4 == 0) {
-                    alph[sb * kRows + brow] = alpha;
-                    st_async_b32(alpha_remote + (sb * kRows + brow) * 4, __float_as_uint(alpha),
-                                 pfull_remote + sb * 8);
-                }
-                fence_proxy_async_smem();  // P -> the PV MMAs of both CTAs (async proxy)
+                if (bq4 == 0) alph[sb * kRows + brow] = alpha;
+                fence_proxy_async_smem();  // P and the factors -> the PV MMAs and the bulk copies
                 __syncwarp();
                 if (lane == 0) {
-                    // this warp's 8 rows of P are 1 KB of contiguous rows: the same rows of the peer's buffer
+                    // this warp's 8 rows of P are 1 KB of contiguous rows and their factors 32
+                    // contiguous bytes: the same places in the peer's buffers
                     const uint32_t r0 = sb * SM::kP + brow * 128;
                     bulk_copy_to_peer(p_remote + r0, smem + SM::oP + r0, 8 * 128, pfull_remote + sb * 8);
+                    const uint32_t a0 = (sb * kRows + brow) * 4;
+                    bulk_copy_to_peer(alpha_remote + a0, smem + SM::oAlpha + a0, 8 * 4, pfull_remote + sb * 8);
                     mbar_arrive(&p_full[sb]);
                 }
                 GQLA_SPAN_END(17, t_b2);
                 GQLA_SPAN_END(19, t_b0);
                 page = page_next;
             }
+            if (quit) break;
             // ---- the owned rows' sums and LSE; the sums of all 128 rows are gathered in
-            // both CTAs' lsm for the score warps' epilogue
+            // both CTAs' lsm for the score warps' epilogue.  They overwrite the previous
+            // piece's sums: once PV of a tile of this piece is done in both CTAs, both CTAs'
+            // score warps have sent that tile's partials, which they do only after the
+            // previous piece's epilogue (which read the sums and waited for l_full's previous
+            // phase), so the overwrite and the next arrivals on l_full are safe even for a
+            // piece of a tile or two.  The tile is the piece's second-to-last
+            // (its only one if it has one): no later tile on its P buffer has reached stage B,
+            // so that buffer's barrier is at most one phase past it.
+            const uint32_t t_pv = nt >= 2 ? t - 2 : t - 1;  // t is one past the piece's last tile
+            if (!__all_sync(0xffffffffu, mbar_wait(&p_empty[t_pv & 1], (t_pv >> 1) & 1, abort_flag))) {
+                if (lane == 0) give_up();
+                break;
+            }
             float l = l_run;
             l += __shfl_xor_sync(0xffffffffu, l, 1);
             l += __shfl_xor_sync(0xffffffffu, l, 2);
@@ -802,20 +945,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     GQLA_PROF_FLUSH;
     __syncthreads();
-    if (*abort_flag && threadIdx.x == 0) {
-        report_error(p.ws, GQLA_ERR_TIMEOUT, c);
-        st_cluster_b32(map_peer(smem_u32(const_cast<int *>(abort_flag)), peer), 1u);  // tell the peer
-    }
+    if (*abort_flag && threadIdx.x == 0) report_error(p.ws, GQLA_ERR_TIMEOUT, c);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
     // Every step of the pair ran in both CTAs: if neither gave up, every byte either one
     // sent (partial scores, P rows, rescale factors, row sums) was waited for by the
-    // other, so nothing is in flight here.  A CTA that gave up ran on without waiting and
-    // may have left asynchronous stores and bulk copies to its peer in flight; once the
-    // first barrier has told both CTAs, both wait about 100 us (those copies take
-    // microseconds) before the second barrier lets either exit.
+    // other, so nothing is in flight here.  When one gave up (both flags are set then),
+    // the copies sent before the roles stopped may still be in flight: after the first
+    // barrier both CTAs wait about 100 us (those copies take microseconds) before the
+    // second barrier lets either exit.
     cluster_sync();
     if (*abort_flag) {
         const long long t0 = clock64();
