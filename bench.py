@@ -19,10 +19,12 @@ value   = decode tokens per second of the whole job: N ranks x batch x s_q
 e2e     = the same through the C ABI with host buffers: each step copies the
           queries, page table and lengths from pinned host memory and reads
           both paths' outputs back into pinned memory, inside the timed region
-          (the copies and the five calls replayed as one CUDA graph; the page
-          table and lengths are one buffer copied on a second stream beside
-          q and the query absorption; the GQA path and its output copy run on
-          a third stream beside the absorb path).
+          (replayed as one CUDA graph).  The batch is cut into sub-batches of
+          whole sequences ("sub_batches", 2 from 8 sequences up), each a full
+          step of its own with its own split plan, so one sub-batch's copies
+          overlap another's kernels: inputs on a copy-in stream, the absorb
+          path on the main stream, the GQA path on a second stream, outputs
+          on a copy-out stream as soon as each path of a sub-batch is done.
 Timing  = the step is captured into a CUDA graph; the K timed steps are issued
           back to back, each replay between two CUDA events on the stream
           (device time, no host launch overhead), with an L2 flush (a 256 MiB
@@ -438,53 +440,88 @@ class Workbench:
         if st_a or st_g:
             raise RuntimeError(f"device-side error during the bench ({self.name}): {st_a} {st_g}")
 
-    def e2e(self, steps, warmup):
-        """Host buffers through the C ABI, copies inside the timed region.  Every copy
-        costs ~10 us however small, so the page table and the lengths travel as one
-        int32 buffer, on a second stream while q is copied and the query absorption
-        runs; the GQA path and its output copy run on a third stream beside the absorb
-        path; the step ends when every copy has landed.  Returns (ms, h2d, d2h)."""
-        dev, case, ba, bg = self.dev, self.case, self.ba, self.bg
+    def e2e(self, steps, warmup, parts=None):
+        """Host buffers through the C ABI, copies inside the timed region.  The batch is
+        cut into `parts` sub-batches of whole sequences, each a complete step of its own
+        (its own split plan and buffers), so that one part's host copies overlap another
+        part's kernels: every input copy runs on a copy-in stream (q, then the page table
+        and lengths as one int32 buffer, part by part), each part's query absorption and
+        absorb path run on the main stream, its GQA path on a second stream, and each
+        output goes back on a copy-out stream as soon as its path is done.  The step ends
+        when every copy has landed.  Returns (ms, h2d, d2h, parts)."""
+        gqla, dev, case = self.gqla, self.dev, self.case
+        if parts is None:
+            parts = 2 if self.B >= 8 else 1
         pt_c, sl_c = case["page_table"].cpu(), case["seqlens"].cpu()
-        n_pt = pt_c.numel()
         q_h = case["q"].cpu().pin_memory()
-        meta_h = torch.cat([pt_c.flatten(), sl_c.flatten()]).pin_memory()
-        outa_h = torch.empty(ba.out.shape, dtype=torch.bfloat16).pin_memory()
-        outg_h = torch.empty(bg.out.shape, dtype=torch.bfloat16).pin_memory()
         q_e = torch.empty_like(case["q"])
-        meta_d = torch.empty(meta_h.shape, dtype=torch.int32, device=dev)
-        kv_e = self.gqla.make_kv_index(meta_d[:n_pt].view(pt_c.shape), meta_d[n_pt:], case["num_pages"])
-        h2d = q_h.numel() * 2 + meta_h.numel() * 4
+        outa_h = torch.empty(self.ba.out.shape, dtype=torch.bfloat16).pin_memory()
+        outg_h = torch.empty(self.bg.out.shape, dtype=torch.bfloat16).pin_memory()
+        h, s_q = self.w.num_heads, self.s_q
+        cuts = [self.B * k // parts for k in range(parts + 1)]
+        lanes = []
+        h2d = q_h.numel() * 2
+        for k in range(parts):
+            b0, b1 = cuts[k], cuts[k + 1]
+            pt_k, sl_k = pt_c[b0:b1].contiguous(), sl_c[b0:b1].contiguous()
+            meta_h = torch.cat([pt_k.flatten(), sl_k]).pin_memory()
+            meta_d = torch.empty(meta_h.shape, dtype=torch.int32, device=dev)
+            kv = gqla.make_kv_index(meta_d[:pt_k.numel()].view(pt_k.shape), meta_d[pt_k.numel():],
+                                    case["num_pages"])
+            sa = gqla.plan_splits("absorb", h, s_q, sl_k)
+            sg = gqla.plan_splits("gqa", h, s_q, sl_k, fused=True)
+            ba = gqla.DecodeBuffers(self.dims, b1 - b0, s_q, sa, "absorb", device=dev)
+            bg = gqla.DecodeBuffers(self.dims, b1 - b0, s_q, sg, "gqa", device=dev)
+            q_k = q_e[b0:b1]
+            lanes.append(dict(b0=b0, b1=b1, meta_h=meta_h, meta_d=meta_d, kv=kv, ba=ba, bg=bg, q=q_k,
+                              absorb=[lambda q_k=q_k, ba=ba: gqla.gqla_absorb_query(self.dims, q_k, case["w_uk"], ba.q_absorbed),
+                                      lambda kv=kv, ba=ba: gqla.gqla_decode_absorb(self.dims, ba.q_absorbed, case["latent"], kv,
+                                                                                   ba.num_splits, ba.o_part, ba.lse_part, ba.workspace),
+                                      lambda kv=kv, ba=ba: gqla.gqla_combine(self.dims, kv, s_q, ba.num_splits, 512, ba.o_part,
+                                                                             ba.lse_part, case["w_uv"], ba.out, ba.lse)],
+                              gqa=lambda q_k=q_k, kv=kv, bg=bg: gqla.gqla_decode_gqa_step(
+                                  self.dims, q_k, self.kvx, self.kr, kv, bg.num_splits, bg.o_part, bg.lse_part,
+                                  bg.out, bg.lse, bg.workspace)))
+            h2d += meta_h.numel() * 4
         d2h = outa_h.numel() * 2 + outg_h.numel() * 2
-        calls_e = self.make_calls(q_e, kv_e)
-        gqa_step_e = self.gqa_step_call(q_e, kv_e)
-        side = torch.cuda.Stream(device=dev)
+        copy_in, copy_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
         def e2e_step():
             main = torch.cuda.current_stream()
             begin = torch.cuda.Event()
             begin.record(main)
-            side.wait_event(begin)
-            with torch.cuda.stream(side):
-                meta_d.copy_(meta_h, non_blocking=True)
-            meta_in = torch.cuda.Event()
-            meta_in.record(side)
-            q_e.copy_(q_h, non_blocking=True)
-            calls_e[0]()  # query absorption: needs q only
-            q_in = torch.cuda.Event()
-            q_in.record(main)
-            self.gqa_stream.wait_event(q_in)
-            self.gqa_stream.wait_event(meta_in)
-            with torch.cuda.stream(self.gqa_stream):
-                gqa_step_e()
-                outg_h.copy_(bg.out, non_blocking=True)
-            main.wait_event(meta_in)
-            calls_e[1]()
-            calls_e[2]()
-            outa_h.copy_(ba.out, non_blocking=True)
-            gqa_done = torch.cuda.Event()
-            gqa_done.record(self.gqa_stream)
-            main.wait_event(gqa_done)
+            copy_in.wait_event(begin)
+            copy_out.wait_event(begin)
+            arrived = []
+            with torch.cuda.stream(copy_in):
+                for ln in lanes:
+                    ln["q"].copy_(q_h[ln["b0"]:ln["b1"]], non_blocking=True)
+                    ln["meta_d"].copy_(ln["meta_h"], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(copy_in)
+                    arrived.append(ev)
+            for ln, ev in zip(lanes, arrived):
+                main.wait_event(ev)
+                self.gqa_stream.wait_event(ev)
+                with torch.cuda.stream(self.gqa_stream):
+                    ln["gqa"]()
+                gqa_done = torch.cuda.Event()
+                gqa_done.record(self.gqa_stream)
+                for c in ln["absorb"]:
+                    c()
+                absorb_done = torch.cuda.Event()
+                absorb_done.record(main)
+                with torch.cuda.stream(copy_out):
+                    copy_out.wait_event(gqa_done)
+                    outg_h[ln["b0"]:ln["b1"]].copy_(ln["bg"].out, non_blocking=True)
+                    copy_out.wait_event(absorb_done)
+                    outa_h[ln["b0"]:ln["b1"]].copy_(ln["ba"].out, non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(copy_out)
+            main.wait_event(done)
+            gqa_end = torch.cuda.Event()
+            gqa_end.record(self.gqa_stream)
+            main.wait_event(gqa_end)
 
         for _ in range(warmup):  # eager warm-up, then the same step as one graph
             e2e_step()
@@ -496,9 +533,17 @@ class Workbench:
             graph_e2e.replay()
         torch.cuda.synchronize()
         times = self.time_steps(steps, graph_e2e)
-        if not torch.equal(outa_h, ba.out.cpu()) or not torch.equal(outg_h, bg.out.cpu()):
-            raise RuntimeError("end-to-end outputs differ from the device results")
-        return sum(times) / len(times), h2d, d2h
+        for ln in lanes:
+            if (not torch.equal(outa_h[ln["b0"]:ln["b1"]], ln["ba"].out.cpu())
+                    or not torch.equal(outg_h[ln["b0"]:ln["b1"]], ln["bg"].out.cpu())):
+                raise RuntimeError("end-to-end outputs differ from the device results")
+        # the sub-batches' results agree with the whole batch's (other split plans: fp32
+        # merges in another order, so within rounding, not bit for bit)
+        for got, ref in ((outa_h, self.ba.out), (outg_h, self.bg.out)):
+            diff = (got.float() - ref.float().cpu()).abs().max().item()
+            if not diff <= 2e-2:
+                raise RuntimeError(f"sub-batched outputs differ from the whole batch's by {diff}")
+        return sum(times) / len(times), h2d, d2h, parts
 
     def report(self, mean, world, path_ms=None):
         """Per-kernel and per-path roofline fractions from the per-call means (ms)."""
@@ -670,7 +715,7 @@ def run_ours(args, rank, world, local_rank):
     mean = wb.time_calls(args.steps)
     path_ms = wb.time_paths(args.steps)
     wb.check_device_errors()
-    e2e_ms, h2d, d2h = wb.e2e(args.steps, args.warmup)
+    e2e_ms, h2d, d2h, e2e_parts = wb.e2e(args.steps, args.warmup, args.e2e_parts)
 
     # ---- max over ranks
     tokens_step = wb.B * wb.s_q
@@ -690,7 +735,7 @@ def run_ours(args, rank, world, local_rank):
                    "tc_ms": expand_tc_ms,
                    "tc_tflops": acc["expand"]["flops"] / (expand_tc_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "sub_batches": e2e_parts},
         "gpu_launches": wb.launches_per_step() * args.steps,
         "clocks": clocks.summary(),
     }
@@ -901,6 +946,8 @@ def main():
                     help="measure the headline workload only (not the rest of the suite)")
     ap.add_argument("--sparse-topk", type=int, default=0,
                     help="also time sparse GQLA with this many selected positions per query token")
+    ap.add_argument("--e2e-parts", type=int, default=None,
+                    help="sub-batches of the end-to-end step (default 2 from 8 sequences up, else 1)")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
                     help="print the per-kernel summary of an ncu launch list and exit")
     args = ap.parse_args()
