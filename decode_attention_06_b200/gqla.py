@@ -309,11 +309,13 @@ def gqla_plan_splits(seqlens, max_splits: int, piece_cost_pages: int) -> int:
 
 
 # What a chunk's second piece costs, in pages of the chunk, for the two decode
-# kernels on B200 (a sweep of split counts over 32 sequences of 4096 tokens:
-# the absorb decode's time grows by ~0.9 us per page of its longest chunk and by
+# kernels on B200 (sweeps of split counts: over 32 sequences of 4096 tokens the
+# absorb decode's time grows by ~0.9 us per page of its longest chunk and by
 # ~6 us when that chunk holds two pieces; the GQA decode, bound by the HBM
-# stream, loses about two pages' worth).
-PIECE_COST_PAGES = {"absorb": 6, "gqa": 2}
+# stream, gains little from more CTAs and loses 8-10 pages' worth per extra
+# piece: 389 us at 128 splits of 64 pages, each inside one sequence, against
+# 401 us at 147 splits of 56 pages over 64 sequences of 8192 tokens, s_q = 2).
+PIECE_COST_PAGES = {"absorb": 6, "gqa": 8}
 
 
 # Below this many pages in the batch, one split is fastest for gqla_decode_gqa_step: the
