@@ -54,15 +54,24 @@ constexpr int kThreads = 384;
 // these launch bounds, checked on the host before every launch); the split must not
 // ask for more in all than the launch gave, or the increase would wait forever.
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsIssue = 56;
-constexpr int kRegsSoftmax = 224;
-static_assert(128 * kRegsIssue + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
+// The split per query-column count (ptxas -v shows no spill in any instantiation with
+// these): the issuing roles' loops need more than 56 registers, and the softmax fits in
+// 216 once the running column maxima live in shared memory instead of NQ registers.
+template <int NQ>
+struct RegSplit {
+    static constexpr int kIssue = NQ == 16 ? 72 : 64;
+    static constexpr int kSoftmax = 216;
+    static_assert(128 * kIssue + 256 * kSoftmax <= kThreads * kLaunchRegs, "register split");
+    static_assert(kIssue % 8 == 0 && kSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
+};
 
+template <int NQ>
 __device__ __forceinline__ void regs_decrease() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIssue));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<NQ>::kIssue));
 }
+template <int NQ>
 __device__ __forceinline__ void regs_increase() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<NQ>::kSoftmax));
 }
 constexpr int kTok = 128;            // tokens per unit (two pages)
 constexpr float kRescaleLog2 = 8.0f;
@@ -275,7 +284,7 @@ __device__ __forceinline__ float score_of(uint32_t raw, int n, bool tok_ok, bool
 // P = 2^(score - m) in bf16 into this thread's P^T row (MN-major, 32B/64B-swizzled);
 // ps receives the rounded probabilities.
 template <int NQ>
-__device__ __forceinline__ void write_p(const uint32_t (&sv)[NQ], const float (&mu)[NQ],
+__device__ __forceinline__ void write_p(const uint32_t (&sv)[NQ], const float *mrow,
                                         float (&ps)[NQ], bool tok_ok, bool hide_low, int G,
                                         float scale_log2, uint8_t *pbuf, int tok) {
 #pragma unroll
@@ -285,8 +294,10 @@ __device__ __forceinline__ void write_p(const uint32_t (&sv)[NQ], const float (&
         for (int e = 0; e < 8; e += 2) {
             const float x0 = score_of(sv[n + e], n + e, tok_ok, hide_low, G, scale_log2);
             const float x1 = score_of(sv[n + e + 1], n + e + 1, tok_ok, hide_low, G, scale_log2);
-            const float m0 = mu[n + e] == -INFINITY ? 0.0f : mu[n + e];
-            const float m1 = mu[n + e + 1] == -INFINITY ? 0.0f : mu[n + e + 1];
+            // the column maxima are the same for every thread: broadcast shared-memory reads
+            const float2 mm = *reinterpret_cast<const float2 *>(mrow + n + e);
+            const float m0 = mm.x == -INFINITY ? 0.0f : mm.x;
+            const float m1 = mm.y == -INFINITY ? 0.0f : mm.y;
             const float p0 = x0 == -INFINITY ? 0.0f : fast_exp2(x0 - m0);
             const float p1 = x1 == -INFINITY ? 0.0f : fast_exp2(x1 - m1);
             __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
@@ -383,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // branch.  Warpgroup 0 gives registers up before it waits on anything, so the softmax
     // warpgroups' increase never waits on a warp that waits on them.
     if (warp < 4) {
-        regs_decrease();
+        regs_decrease<NQ>();
         if (warp == 0 && SPARSE) {
             // ---------------------------------------------------------------- TMA producer, sparse
             // The same units and rings as below; the rows of a unit are gathered four at a
@@ -710,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // warp 3 is idle: it completes warpgroup 0 for the register split
     } else {
-        regs_increase();
+        regs_increase<NQ>();
         // ---------------------------------------------------------------- softmax, PV, epilogue
         // Warpgroup wg owns the groups gi = wg, wg + 2, ... (units of
         // one parity), so the two warpgroups never share a group.
@@ -754,12 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     GQLA_SPAN_BEGIN(t_ld);
                     tmem_ld16(t_s + lane_off + sb * NQ, sv);
                     if constexpr (NQ == 32) tmem_ld16(t_s + lane_off + sb * NQ + 16, sv + 16);
-                    float mu[NQ];
-#pragma unroll
-                    for (int n = 0; n < NQ; n += 4) {
-                        const float4 m4 = *reinterpret_cast<const float4 *>(mrun + gi * NQ + n);
-                        mu[n] = m4.x; mu[n + 1] = m4.y; mu[n + 2] = m4.z; mu[n + 3] = m4.w;
-                    }
+                    // the group's running column maxima stay in shared memory (read by every
+                    // thread alike), not in NQ registers
+                    const float *mrow = mrun + gi * NQ;
                     tmem_wait_ld();
                     GQLA_SPAN_END(11, t_ld);
                     tc_fence_before();
@@ -767,14 +775,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bool exceed = ip == 0;
 #pragma unroll
                     for (int n = 0; n < NQ; ++n)
-                        exceed |= score_of(sv[n], n, tok_ok, hide_low, p.G, p.scale_log2) > mu[n] + kRescaleLog2;
+                        exceed |= score_of(sv[n], n, tok_ok, hide_low, p.G, p.scale_log2) > mrow[n] + kRescaleLog2;
                     // the P^T buffer (and O^T_g) are free once this warpgroup's previous PV completed
                     if (!GQLA_WAIT(7, &p_free[wg], (wg_unit(jj, p.NG) & 1) ^ 1, abort_flag)) *abort_flag = 1;
                     tc_fence_after();
                     float ps[NQ];
                     GQLA_SPAN_BEGIN(t_wp);
                     if (ip > 0)  // optimistic: P against the running maxima
-                        write_p<NQ>(sv, mu, ps, tok_ok, hide_low, p.G, p.scale_log2, pbuf, tok);
+                        write_p<NQ>(sv, mrow, ps, tok_ok, hide_low, p.G, p.scale_log2, pbuf, tok);
                     GQLA_SPAN_END(12, t_wp);
                     const int vs = jj % VS;
                     if (partial) {  // V rows that are not tokens (never written, maybe NaN) -> 0
@@ -806,15 +814,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (lane < NQ) red[lane * 4 + wq] = m;
                         }
                         wg_bar(wg);
-                        bool need = false;
-#pragma unroll
-                        for (int n = 0; n < NQ; ++n) {
-                            const float4 r4 = *reinterpret_cast<const float4 *>(red + n * 4);
+                        // the new maxima, one column per thread, into mnew (the epilogue's
+                        // scratch, free during the units); the barrier publishes them and
+                        // tells every thread whether any column changed
+                        float *mnew = inv_l;
+                        bool changed = false;
+                        if (wtid < NQ) {
+                            const float4 r4 = *reinterpret_cast<const float4 *>(red + wtid * 4);
                             const float mt = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
-                            const float mn = ip == 0 ? mt : ((mt > mu[n] + kRescaleLog2) ? mt : mu[n]);
-                            need |= ip > 0 && mn != mu[n];
-                            mu[n] = mn;
+                            const float mold = mrow[wtid];
+                            const float mn = ip == 0 ? mt : ((mt > mold + kRescaleLog2) ? mt : mold);
+                            changed = ip > 0 && mn != mold;
+                            mnew[wtid] = mn;
                         }
+                        const bool need = wg_bar_any(wg, changed);
                         tc_fence_after();
                         if (need) {  // O^T_g columns *= 2^(m_old - m_new)
                             const uint32_t to = t_o + gi * NQ + lane_off;
@@ -825,8 +838,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tmem_wait_ld();
 #pragma unroll
                                 for (int e = 0; e < 16; ++e) {
-                                    const float mold = mrun[gi * NQ + h16 + e];
-                                    const float a = mold == mu[h16 + e] ? 1.0f : exp2f(mold - mu[h16 + e]);
+                                    const float mold = mrow[h16 + e], mn = mnew[h16 + e];
+                                    const float a = mold == mn ? 1.0f : exp2f(mold - mn);
                                     r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
                                 }
                                 tmem_st16(to + h16, r);
@@ -834,22 +847,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tmem_wait_st();
                         }
                         if (lane < NQ) {  // this lane's own column partial follows the same rescale
-                            const float4 r4 = *reinterpret_cast<const float4 *>(red + lane * 4);
-                            const float mt = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
-                            const float mold = mrun[gi * NQ + lane];
-                            const float mn = ip == 0 ? mt : ((mt > mold + kRescaleLog2) ? mt : mold);
+                            const float mold = mrow[lane], mn = mnew[lane];
                             *lw = ip == 0 ? 0.0f : (mn == mold ? *lw : *lw * exp2f(mold - mn));
                         }
-                        write_p<NQ>(sv, mu, ps, tok_ok, hide_low, p.G, p.scale_log2, pbuf, tok);
+                        write_p<NQ>(sv, mnew, ps, tok_ok, hide_low, p.G, p.scale_log2, pbuf, tok);
                         fence_proxy_async_smem();
                         tc_fence_before();
-                        wg_bar(wg);  // P^T complete; everyone has read mrun / red
-                        if (wtid == 0) {
-#pragma unroll
-                            for (int n = 0; n < NQ; n += 4)
-                                *reinterpret_cast<float4 *>(mrun + gi * NQ + n) =
-                                    make_float4(mu[n], mu[n + 1], mu[n + 2], mu[n + 3]);
-                        }
+                        wg_bar(wg);  // P^T complete; everyone has read mrun / mnew / red
+                        if (wtid < NQ) mrun[gi * NQ + wtid] = mnew[wtid];
                         GQLA_SPAN_END(17, t_slow);
                     }
                     mbar_arrive(&p_full[wg]);
@@ -992,12 +997,13 @@ cudaError_t launch_nq_mode(const CUtensorMap &kvm, const CUtensorMap &krm, const
     cudaError_t e = cudaFuncSetAttribute(decode_gqa_tc_kernel<NQ, SPARSE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    // the register split asks for 128 x kRegsIssue + 256 x kRegsSoftmax registers: the
+    // the register split asks for 128 x kIssue + 256 x kSoftmax registers: the
     // launch must give at least that many, or the kernel's increase would never return
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, decode_gqa_tc_kernel<NQ, SPARSE>);
     if (e != cudaSuccess) return e;
-    if (128 * kRegsIssue + 256 * kRegsSoftmax > kThreads * fa.numRegs) return cudaErrorInvalidConfiguration;
+    if (128 * RegSplit<NQ>::kIssue + 256 * RegSplit<NQ>::kSoftmax > kThreads * fa.numRegs)
+        return cudaErrorInvalidConfiguration;
     return launch_dependent(decode_gqa_tc_kernel<NQ, SPARSE>, dim3(p.num_splits, group_splits), dim3(kThreads),
                             bytes, stream, kvm, krm, qm, kvrm, krrm, p);
 }
