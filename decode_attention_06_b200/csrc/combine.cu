@@ -96,19 +96,17 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-__device__ __forceinline__ uint2 pack_bf16x4(float a, float b, float c, float d) {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
-    return make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-}
-
 // ---------------------------------------------------------------------------
 // GQA path (d_in = 128): one warp per quad of heads of one (sequence, token)
-// pair, lane j owns columns 4j .. 4j+3; the partials are read eight at a
-// time so that one warp keeps 32 independent 16-byte loads in flight.
+// pair, lane j owns columns 4j .. 4j+3; the first four partials are read with
+// the LSEs (16 independent 16-byte loads in flight per lane), the rest four at a
+// time.  Four rather than eight keeps the register count low enough for three
+// blocks per SM: the common case (a sequence over one to four chunks) is one
+// round trip either way.
 // ---------------------------------------------------------------------------
 constexpr int kQuadsPerBlock = 4;
 
-__global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineParams p) {
+__global__ void __launch_bounds__(32 * kQuadsPerBlock, 3) combine_v_kernel(CombineParams p) {
     __shared__ int s_c0[kQuadsPerBlock + 1], s_c1[kQuadsPerBlock + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quads_per_pair = p.heads / 4;
@@ -133,12 +131,13 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
     const int64_t row0 = ((int64_t)(b + c0) * p.s_q + s) * p.heads + h0;
     const int64_t part_stride = (int64_t)p.s_q * p.heads;
 
-    // the first eight partials do not depend on the weights: their loads go out with
-    // the LSE loads, so the common case (nparts <= 8) makes one round trip to memory
+    // the first partials do not depend on the weights: their loads go out with the LSE
+    // loads, so the common case (nparts <= kPre) makes one round trip to memory
+    constexpr int kPre = 2;
     const float *base0 = p.o_part + row0 * kDv + lane * 4;
-    float4 v0[8][4];
+    float4 v0[kPre][4];
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj)
+    for (int jj = 0; jj < kPre; ++jj)
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             v0[jj][i] = jj < nparts ? ldg4(base0 + ((int64_t)jj * part_stride + i) * kDv)
@@ -175,9 +174,9 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
         const int n = min(32, nparts - cb);
         const float *base = p.o_part + (row0 + (int64_t)cb * part_stride) * kDv + lane * 4;
         int j0 = 0;
-        if (cb == 0) {  // the eight partials already in registers (zeros past nparts)
+        if (cb == 0) {  // the partials already in registers (zeros past nparts)
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
+            for (int jj = 0; jj < kPre; ++jj)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float wj = __shfl_sync(0xffffffffu, w[i], jj);
@@ -186,7 +185,7 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock) combine_v_kernel(CombineP
                     acc[i].z = fmaf(wj, v0[jj][i].z, acc[i].z);
                     acc[i].w = fmaf(wj, v0[jj][i].w, acc[i].w);
                 }
-            j0 = 8;
+            j0 = kPre;
         }
         for (; j0 < n; j0 += 4) {
             float4 v[4][4];

@@ -26,6 +26,12 @@ struct DeviceError {
     int info;
 };
 
+// Four floats rounded to bf16 (round to nearest even), packed for one 8-byte store.
+__device__ __forceinline__ uint2 pack_bf16x4(float a, float b, float c, float d) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    return make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+}
+
 __device__ __forceinline__ void report_error(void *ws, int code, int info) {
     if (!ws) return;
     DeviceError *e = reinterpret_cast<DeviceError *>(ws);

@@ -54,12 +54,12 @@ constexpr int kThreads = 384;
 // these launch bounds, checked on the host before every launch); the split must not
 // ask for more in all than the launch gave, or the increase would wait forever.
 constexpr int kLaunchRegs = 168;
-// The split per query-column count (ptxas -v shows no spill in any instantiation with
-// these): the issuing roles' loops need more than 56 registers, and the softmax fits in
-// 216 once the running column maxima live in shared memory instead of NQ registers.
+// The split (ptxas -v shows no spill in any instantiation with it): the issuing roles'
+// loops need 72 registers, and the softmax fits in 216 once the running column maxima
+// live in shared memory instead of NQ registers.
 template <int NQ>
 struct RegSplit {
-    static constexpr int kIssue = NQ == 16 ? 72 : 64;
+    static constexpr int kIssue = 72;
     static constexpr int kSoftmax = 216;
     static_assert(128 * kIssue + 256 * kSoftmax <= kThreads * kLaunchRegs, "register split");
     static_assert(kIssue % 8 == 0 && kSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
@@ -360,7 +360,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int r0 = c * k, r1 = min(total, r0 + k);
         int b = p.batch, start = 0;
         if (r0 < r1) warp_find_sequence(p.seqlens, p.batch, r0, &b, &start);
-        if (lane == 0) { plan[0] = r0; plan[1] = r1; plan[2] = b; plan[3] = start; }
+        if (lane == 0) {
+            plan[0] = r0; plan[1] = r1; plan[2] = b; plan[3] = start;
+            // the producer's first reads after the CTA's set-up: the descriptors and the
+            // first pages' page-table entries, headed for L2 now
+            prefetch_tensormap(SPARSE ? &kv_rows_map : &kv_map);
+            prefetch_tensormap(SPARSE ? &kr_rows_map : &kr_map);
+            prefetch_tensormap(&q_map);
+            if (b < p.batch) prefetch_l2(p.page_table + (int64_t)b * p.max_pages + (r0 - start));
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_base_smem, 512);
@@ -451,14 +459,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint8_t *dst = smem + SM::oK + ks * SM::kKSlotBytes;
                         if (lane == 0) {
                             mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
-    #pragma unroll
+#pragma unroll
                             for (int cb = 0; cb < 3; ++cb)  // q_g rows of this query token
                                 tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
                                             (gbase + kc.gi) * p.G, kc.b * p.s_q);
                         }
                         __syncwarp();
                         if (mine) {
-    #pragma unroll
+#pragma unroll
                             for (int cb = 0; cb < 2; ++cb)  // K_nope lo / hi
                                 tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &k_full[ks],
                                                  cb * 64, row_of(ksl.x, kc.gi), row_of(ksl.y, kc.gi),
@@ -485,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         __syncwarp();
                         if (mine) {
-    #pragma unroll
+#pragma unroll
                             for (int cb = 0; cb < 2; ++cb)  // V lo / hi
                                 tma_gather4_hint(dst + cb * 2 * kBox + half * kBox + r0 * 128, &kv_rows_map, &v_full[vs],
                                                  128 + cb * 64, row_of(vsl.x, vc.gi), row_of(vsl.y, vc.gi),
@@ -566,11 +574,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             uint8_t *dst = smem + SM::oK + ks * SM::kKSlotBytes;
                             mbar_arrive_expect_tx(&k_full[ks], np * 2 * kBox + q_bytes);
-    #pragma unroll
+#pragma unroll
                             for (int cb = 0; cb < 3; ++cb)  // q_g rows (s, hg) of this sequence
                                 tma_load_3d(dst + SM::kKBytes + cb * NQ * 128, &q_map, &k_full[ks], cb * 64,
                                             (gbase + kc.gi) * p.G, kc.b * p.s_q);
-    #pragma unroll
+#pragma unroll
                             for (int cb = 0; cb < 2; ++cb) {  // K_nope lo / hi: page 0 rows, then page 1 rows
                                 if (pp.page0 >= 0)
                                     tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &k_full[ks], cb * 64,
@@ -596,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             uint8_t *dst = smem + SM::oV + vs * SM::kVBytes;
                             if (np) {
                                 mbar_arrive_expect_tx(&v_full[vs], np * 2 * kBox);
-    #pragma unroll
+#pragma unroll
                                 for (int cb = 0; cb < 2; ++cb) {
                                     if (pp.page0 >= 0)
                                         tma_load_3d_hint(dst + cb * 2 * kBox, &kv_map, &v_full[vs], 128 + cb * 64,
@@ -657,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint64_t q_d = desc_advance(k_d, SM::kKBytes);
                             const uint64_t kr_d = smem_desc(kr, 16, 1024, kSw128);
                             if (!*abort_flag) {
-    #pragma unroll
+#pragma unroll
                                 for (int ks = 0; ks < 12; ++ks) {
                                     const uint64_t ad = ks < 8 ? desc_advance(k_d, (ks >> 2) * 2 * kBox + (ks & 3) * 32)
                                                                : desc_advance(kr_d, (ks - 8) * 32);
@@ -702,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint64_t v_d = desc_advance(v_d0, vs * SM::kVBytes);
                             const uint64_t p_d = desc_advance(p_d0, w * SM::kPBytes);
                             if (!*abort_flag) {
-    #pragma unroll
+#pragma unroll
                                 for (int ks = 0; ks < kTok / 16; ++ks)
                                     mma_bf16(t_o + gi * NQ, desc_advance(v_d, ks * 2048), desc_advance(p_d, ks * 16 * NQ * 2),
                                              idesc_pv, (ip == 0 && ks == 0) ? 0u : 1u);
@@ -901,25 +909,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 wg_bar(wg);  // inv_l ready
                 GQLA_SPAN_BEGIN(t_est);
-                // 16 columns at a time: O^T row dv of columns n = s*G + hg -> row (s*h + g*G + hg)
+                // O^T row dv of column n = s*G + hg goes to row (s*h + g*G + hg)
                 const int64_t row_g = row_s0 + (int64_t)(gbase + gi) * p.G;
-                float *dst_p = p.o_part + row_g * kDv + dv;
-                __nv_bfloat16 *dst_o = final_out ? p.out + row_g * kDv + dv : nullptr;
-                int s = 0, hg = 0;
-#pragma unroll
-                for (int h16 = 0; h16 < NQ; h16 += 16) {
+                if constexpr (NQ == 16) {
+                    // 16 columns: straight from registers, one 4-byte store per column (the
+                    // 32 lanes of a warp write 128 contiguous bytes of a row)
+                    float *dst_p = p.o_part + row_g * kDv + dv;
+                    __nv_bfloat16 *dst_o = final_out ? p.out + row_g * kDv + dv : nullptr;
+                    int s = 0, hg = 0;
                     uint32_t r[16];
-                    tmem_ld16(t_o + gi * NQ + lane_off + h16, r);
+                    tmem_ld16(t_o + gi * NQ + lane_off, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        if (h16 + e < real_cols) {
+                        if (e < real_cols) {
                             const int64_t off = ((int64_t)s * p.heads + hg) * kDv;
-                            const float v = __uint_as_float(r[e]) * inv_l[h16 + e];
+                            const float v = __uint_as_float(r[e]) * inv_l[e];
                             if (dst_o) dst_o[off] = __float2bfloat16_rn(v);
                             else dst_p[off] = v;
                         }
                         if (++hg == p.G) { hg = 0; ++s; }
+                    }
+                } else {
+                    // 32 columns: through the warpgroup's P^T buffer (free: all its PVs are
+                    // done) 16 columns at a time: each thread writes its dv of every column
+                    // there, then the warpgroup stores whole 16-byte pieces of the rows
+                    // (coalesced, a quarter of the store count)
+                    constexpr int kCC = SM::kPBytes / (kDv * 4);  // columns per round: 16
+                    float *stg = reinterpret_cast<float *>(pbuf);  // [kCC][kDv] fp32
+#pragma unroll 1
+                    for (int h16 = 0; h16 < NQ; h16 += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(t_o + gi * NQ + lane_off + h16, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c0 = 0; c0 < 16; c0 += kCC) {
+#pragma unroll
+                            for (int e = 0; e < kCC; ++e)
+                                stg[e * kDv + dv] = __uint_as_float(r[c0 + e]) * inv_l[h16 + c0 + e];
+                            wg_bar(wg);
+#pragma unroll
+                            for (int i = wtid; i < kCC * (kDv / 4); i += 128) {
+                                const int n = h16 + c0 + i / (kDv / 4), q4 = i % (kDv / 4);
+                                if (n < real_cols) {
+                                    const int sn = n / p.G, hn = n - sn * p.G;
+                                    const int64_t row = row_g + (int64_t)sn * p.heads + hn;
+                                    const float4 v = reinterpret_cast<const float4 *>(stg)[i];
+                                    if (final_out)
+                                        reinterpret_cast<uint2 *>(p.out + row * kDv)[q4] = pack_bf16x4(v.x, v.y, v.z, v.w);
+                                    else
+                                        reinterpret_cast<float4 *>(p.o_part + row * kDv)[q4] = v;
+                                }
+                            }
+                            wg_bar(wg);  // the staging is rewritten by the next round
+                        }
                     }
                 }
                 GQLA_SPAN_END(19, t_est);
