@@ -7,13 +7,15 @@
 //
 // Rows of one group share W_UK_g, so a CTA owns a tile of up to 128 rows of
 // one group -- `bst` consecutive (sequence, query token) pairs x the group's
-// G heads -- and one quarter (128 columns) of the latent output:
-//   D[128 x 128] = A[128 x 128] * B[128 x 128],  A = q^C rows (K-major),
-//   B^T = W_UK_g[quarter] as stored ([latent][d_nope], K-major).
+// G heads -- and N = 128 or 256 columns of the latent output:
+//   D[128 x N] = A[128 x 128] * B[128 x N],  A = q^C rows (K-major),
+//   B^T = W_UK_g[columns] as stored ([latent][d_nope], K-major).
 // Both operands arrive by TMA in the 128-byte swizzled layout; one thread
-// issues 8 MMAs of K = 16 into a 128-column TMEM accumulator; the four warps
+// issues 8 MMAs of K = 16 into an N-column TMEM accumulator; the four warps
 // convert their 32 rows to bf16 into shared memory and write the tile out
-// row by row, each row one contiguous 512-byte segment.
+// row by row, each row one contiguous segment.  N = 128 (3 CTAs per SM) splits
+// a tile over four CTAs, for small batches; when that grid needs more than one
+// wave, N = 256 (2 CTAs per SM) fits the work in one.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -28,12 +30,15 @@ using namespace sm100;
 
 constexpr int kAqThreads = 128;
 constexpr int kAqA = 128 * 128;        // one K block of A: 128 rows x 64 dims (bytes)
-constexpr int kAqN = 128;              // latent columns per CTA
-constexpr int kAqB = kAqN * 128;       // one K block of B: 128 latent rows x 64 dims
-constexpr int kAqBar = 2 * kAqA + 2 * kAqB;
-constexpr int kAqStage = 2 * kAqN + 16;  // staging row pitch (bytes): 128 bf16 + bank skew
-static_assert(128 * kAqStage <= kAqBar, "staging tile overlaps the barriers");
-constexpr int kAqSmem = kAqBar + 64 + 1024;  // + alignment slack
+
+template <int N>  // latent columns per CTA
+struct AqLayout {
+    static constexpr int kB = N * 128;        // one K block of B: N latent rows x 64 dims
+    static constexpr int kBar = 2 * kAqA + 2 * kB;
+    static constexpr int kStage = 2 * N + 16;  // staging row pitch (bytes): N bf16 + bank skew
+    static_assert(128 * kStage <= kBar, "staging tile overlaps the barriers");
+    static constexpr int kSmem = kBar + 64 + 1024;  // + alignment slack
+};
 
 struct AqParams {
     const __nv_bfloat16 *q;
@@ -44,9 +49,14 @@ struct AqParams {
     int bst;       // (sequence, token) pairs per tile: G * bst <= 128
 };
 
+template <int N>
 __global__ void __launch_bounds__(kAqThreads, 2)
     absorb_query_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                            const __grid_constant__ CUtensorMap wmap, AqParams p) {
+    constexpr int kAqN = N;
+    constexpr int kAqB = AqLayout<N>::kB;
+    constexpr int kAqBar = AqLayout<N>::kBar;
+    constexpr int kAqStage = AqLayout<N>::kStage;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
@@ -58,7 +68,7 @@ __global__ void __launch_bounds__(kAqThreads, 2)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(full + 3);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x, grp = blockIdx.y, quarter = blockIdx.z;
+    const int tile = blockIdx.x, grp = blockIdx.y, quarter = blockIdx.z;  // column block N * quarter
     const int bs0 = tile * p.bst;
     const int rows_in_tile = p.G * p.bst;
 
@@ -151,14 +161,16 @@ __global__ void __launch_bounds__(kAqThreads, 2)
     }
     __syncthreads();
     if (ok) {
-        // rows_in_tile rows of 256 bytes; a warp writes two rows at a time, 16 bytes a lane
-        for (int r0 = 2 * warp; r0 < rows_in_tile; r0 += 8) {
-            const int r = r0 + (lane >> 4);
+        // rows_in_tile rows of 2N bytes, 16 bytes a lane: a warp writes 32 / (N / 8) rows
+        // at a time
+        constexpr int kLanesPerRow = kAqN / 8, kRowsPerWarp = 32 / kLanesPerRow;
+        for (int r0 = kRowsPerWarp * warp; r0 < rows_in_tile; r0 += 4 * kRowsPerWarp) {
+            const int r = r0 + lane / kLanesPerRow, part = lane % kLanesPerRow;
             const int bs = bs0 + r / p.G;
             if (r < rows_in_tile && bs < p.bs_total) {
                 const int64_t row = (int64_t)bs * p.heads + grp * p.G + r % p.G;
-                reinterpret_cast<uint4 *>(p.qa + row * kRow + quarter * kAqN)[lane & 15] =
-                    *reinterpret_cast<const uint4 *>(stage + r * kAqStage + (lane & 15) * 16);
+                reinterpret_cast<uint4 *>(p.qa + row * kRow + quarter * kAqN)[part] =
+                    *reinterpret_cast<const uint4 *>(stage + r * kAqStage + part * 16);
             }
         }
         if (quarter == 0) {  // RoPE part: q[row][128:192] -> qa[row][512:576]
@@ -197,20 +209,37 @@ cudaError_t launch_absorb_query(const void *q, int rows, int heads, int num_grou
         if (!make_bf16_map(&qmap, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
+    // N = 128 columns per CTA (a tile over four CTAs, 3 CTAs per SM) unless that grid
+    // needs more than one wave; then N = 256 (2 CTAs per SM), which fits in one
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaErrorInvalidValue;
+    const int tiles = (bs_total + bst - 1) / bst;
+    const bool wide = (int64_t)tiles * num_groups * (kLatent / 128) > 3LL * sms;
+    const uint32_t n = wide ? 256 : 128;
     {
         const uint64_t dims[2] = {(uint64_t)kNope, (uint64_t)num_groups * kLatent};
         const uint64_t strides[1] = {(uint64_t)kNope * 2};
-        const uint32_t box[2] = {64, (uint32_t)kAqN};
+        const uint32_t box[2] = {64, n};
         if (!make_bf16_map(&wmap, w_uk, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
     AqParams p{static_cast<const __nv_bfloat16 *>(q), static_cast<__nv_bfloat16 *>(qa), bs_total,
                heads, G, bst};
-    cudaError_t e = cudaFuncSetAttribute(absorb_query_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAqSmem);
+    dim3 grid((unsigned)tiles, (unsigned)num_groups, kLatent / n);
+    if (wide) {
+        cudaError_t e = cudaFuncSetAttribute(absorb_query_tc_kernel<256>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, AqLayout<256>::kSmem);
+        if (e != cudaSuccess) return e;
+        return launch_dependent(absorb_query_tc_kernel<256>, grid, dim3(kAqThreads), AqLayout<256>::kSmem,
+                                stream, qmap, wmap, p);
+    }
+    cudaError_t e = cudaFuncSetAttribute(absorb_query_tc_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, AqLayout<128>::kSmem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((bs_total + bst - 1) / bst), (unsigned)num_groups, kLatent / kAqN);
-    return launch_dependent(absorb_query_tc_kernel, grid, dim3(kAqThreads), kAqSmem, stream, qmap, wmap, p);
+    return launch_dependent(absorb_query_tc_kernel<128>, grid, dim3(kAqThreads), AqLayout<128>::kSmem, stream,
+                            qmap, wmap, p);
 }
 
 }  // namespace gqla
