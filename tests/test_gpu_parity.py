@@ -380,6 +380,10 @@ FUSED = [
     ("mixed_single_and_multi", 128, 8, [64, 3000, 10, 0, 700], 1, True, 9),
     ("g4_mtp", 32, 4, [513, 64, 3], 2, False, 4),
     ("many_partials", 128, 8, [5000, 300], 1, True, 70),
+    # (g, s_q) = (4, 1) at 128 heads: 32 columns of one query token per group, the
+    # 32-column epilogue's final-output and partial writes
+    ("g4_h128_one_split", 128, 4, [300, 65], 1, False, 1),
+    ("g4_h128_splits", 128, 4, [1000, 130, 0], 1, True, 5),
 ]
 
 
