@@ -220,8 +220,9 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock, 3) combine_v_kernel(Combi
 }
 
 // ---------------------------------------------------------------------------
-// MQA-absorb path (d_in = 512).  A cluster of 2 CTAs per tile of up to 64 rows
-// of one group (bst pairs x G heads).  CTA kq merges latent columns
+// MQA-absorb path (d_in = 512).  A cluster of 2 CTAs takes tiles of up to 64 rows
+// of one group (bst pairs x G heads), one after the other (as many per cluster as
+// keep the grid within one wave).  CTA kq merges latent columns
 // [256 kq, 256 kq + 256) of the tile's rows into bf16 (the MMA's A operand,
 // K-major, 128-byte swizzle); CTA 1 stores its half into CTA 0's shared memory
 // with asynchronous remote stores, and CTA 0 runs the whole product
@@ -247,7 +248,8 @@ struct ClSmem {
 static_assert(ClSmem::kAlloc <= 227 * 1024, "shared memory");
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
-    combine_latent_tc_kernel(const __grid_constant__ CUtensorMap wmap, CombineParams p, int bst) {
+    combine_latent_tc_kernel(const __grid_constant__ CUtensorMap wmap, CombineParams p, int bst,
+                             int tiles_per_cluster, int num_tiles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
@@ -258,14 +260,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + ClSmem::oBar);
     uint64_t *b_full = a_full + 1;
     uint64_t *done = a_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(a_full + 3);
+    uint64_t *a_free = a_full + 3;  // second CTA: the leader is done with A (its half may go)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(a_full + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int kq = (int)cluster_rank();
     const bool leader = kq == 0;
-    const int tile = blockIdx.y, grp = blockIdx.z;
-    const int bs0 = tile * bst;
+    const int grp = blockIdx.z;
+    // this cluster's tiles of group grp: [tile0, tile0 + n_tiles), one after the other, so
+    // that W_UV_g, the barriers and the tensor memory are set up once for all of them
+    const int tile0 = blockIdx.y * tiles_per_cluster;
+    const int n_tiles = max(0, min(tiles_per_cluster, num_tiles - tile0));
     const int rows_in_tile = p.G * bst;
     const int64_t part_stride = (int64_t)p.s_q * p.heads;
 
@@ -273,12 +279,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         mbar_init(a_full, 1);
         mbar_init(b_full, 1);
         mbar_init(done, 1);
+        mbar_init(a_free, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    // W_UV_g and the split plan (from the lengths) do not depend on the decode before
-    // this kernel, which read the same lengths after its own wait: both start while the
-    // decode finishes (the barrier init above is ordered before the TMA by fence and sync)
+    // W_UV_g and the first tile's split plan (from the lengths) do not depend on the decode
+    // before this kernel, which read the same lengths after its own wait: both start while
+    // the decode finishes (the barrier init above is ordered before the TMA by fence and sync)
     __syncthreads();
     if (tid == 0) {
         if (leader) {
@@ -294,14 +301,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         tmem_alloc(tmem_slot, 128);
         tmem_relinquish();
     }
-    if (warp == 2) {
-        plan_pairs(p, bs0, bst, s_c0, s_c1);
+    if (warp == 2 && n_tiles > 0) {
+        plan_pairs(p, tile0 * bst, bst, s_c0, s_c1);
     }
     griddep_wait();  // the decode's partials are visible from here on
     griddep_launch_dependents();
     tc_fence_before();
     cluster_sync();  // barriers of both CTAs initialised before any remote transfer
     tc_fence_after();
+    const uint32_t tmem = leader ? *tmem_slot : 0u;
+    bool ok = true;
+
+#pragma unroll 1
+    for (int k = 0; k < n_tiles && ok; ++k) {
+        const int bs0 = (tile0 + k) * bst;
+        if (k > 0) {
+            // every warp is done with the previous tile's plan (and, in the leader, with the
+            // staging over A): the next plan replaces it
+            __syncthreads();
+            if (warp == 2) plan_pairs(p, bs0, bst, s_c0, s_c1);
+            __syncthreads();
+        }
 
     // ---- merge: warp w owns rows 4w .. 4w+3, four heads of one (sequence, token) pair
     // (the heads per group are a multiple of 4), and computes their weights itself (lane c
@@ -422,6 +442,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     // at the place they take in the leader's A: the leader stores its own, the peer
     // sends its half straight into the leader's shared memory (8-byte asynchronous
     // stores counted on the leader's a_full)
+    if (!leader && k > 0 && !__syncthreads_and(mbar_wait(a_free, (k - 1) & 1, abort_flag))) {
+        ok = false;  // the leader stopped (or never freed A): send nothing more
+        break;
+    }
     {
         const int chunk = (lane & 15) >> 1, half8 = (lane & 1) * 8;
         const uint32_t a_remote = leader ? 0u : map_peer(smem_u32(smem + ClSmem::oA), 0);
@@ -441,31 +465,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
             }
         }
     }
-    if (!leader) {
-        cluster_sync();  // pairs with the leader's arrive once its MMAs have read the half
-        return;
-    }
+    if (!leader) continue;  // the second CTA goes on with its next tile's merge
     fence_proxy_async_smem();
     __syncthreads();
 
     // ---- leader: the other half of A and W_UV_g in place -> 32 MMAs (M = 64, K = 512)
-    const uint32_t tmem = *tmem_slot;
     if (tid == 0) {
         // this CTA's half of K first (its A blocks are in place), the peer's half once it lands
         mbar_arrive_expect_tx(a_full, ClSmem::kAHalf);
         constexpr uint32_t idesc = idesc_bf16(kClRows, 128, 0, 1);
         const uint64_t a_d = smem_desc(smem_u32(smem + ClSmem::oA), 16, 1024, kSw128);
         const uint64_t b_d = smem_desc(smem_u32(smem + ClSmem::oB), 65536, 1024, kSw128);
-        bool ok = mbar_wait(b_full, 0, abort_flag);
-        if (ok) {
+        bool got = k > 0 || mbar_wait(b_full, 0, abort_flag);
+        if (got) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kLatent / 32; ++kk)
                 mma_bf16(tmem, desc_advance(a_d, (kk >> 2) * (kClRows * 128) + (kk & 3) * 32),
                          desc_advance(b_d, kk * 2048), idesc, kk > 0 ? 1u : 0u);
-            ok = mbar_wait_cluster(a_full, 0, abort_flag);
+            got = mbar_wait_cluster(a_full, k & 1, abort_flag);
         }
-        if (ok) {
+        if (got) {
             tc_fence_after();
 #pragma unroll
             for (int kk = kLatent / 32; kk < kLatent / 16; ++kk)
@@ -476,9 +496,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         }
         mma_commit(done);
     }
-    const bool ok = mbar_wait(done, 0, abort_flag);
+    ok = __syncthreads_and(mbar_wait(done, k & 1, abort_flag) && !*abort_flag);
     tc_fence_after();
-    cluster_arrive_relaxed();  // the MMAs have read the peer's half: the sender may exit
     // ---- epilogue: TMEM (M = 64: row m in lane (m % 16) + 32 (m / 16)) -> bf16 rows in
     // shared memory (over A: the MMAs are done) -> coalesced 256-byte row stores
     if (ok) {
@@ -505,19 +524,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 128);
-    }
-    if (ok && !*abort_flag) {
+    if (ok) {
         for (int i = tid; i < kClRows * 16; i += kClThreads) {
             const int r = i >> 4, part16 = i & 15;
-            const int j = r / p.G;
-            if (r >= rows_in_tile || bs0 + j >= p.bs_total) continue;
-            const int64_t orow = (int64_t)(bs0 + j) * p.heads + grp * p.G + r % p.G;
+            const int jr = r / p.G;
+            if (r >= rows_in_tile || bs0 + jr >= p.bs_total) continue;
+            const int64_t orow = (int64_t)(bs0 + jr) * p.heads + grp * p.G + r % p.G;
             reinterpret_cast<uint4 *>(p.out + orow * kDv)[part16] =
                 reinterpret_cast<const uint4 *>(smem + ClSmem::oStage + r * 256)[part16];
         }
+    }
+    if (ok && k + 1 < n_tiles) {
+        // the staging over A has been read: the second CTA may send its next half
+        __syncthreads();
+        if (tid == 0) mbar_arrive_remote(map_peer(smem_u32(a_free), 1));
+    }
+    }  // tiles
+
+    // One cluster barrier operation per thread on every path: the second CTA waits until
+    // the leader has consumed the last half it sent (the leader arrives once its MMAs are
+    // done, or once it stopped), then both may exit.
+    if (!leader) {
+        cluster_sync();
+        return;
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_arrive_relaxed();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
     }
 }
 
@@ -537,6 +573,15 @@ cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int
                                 dim3(32 * kQuadsPerBlock), 0, stream, p);
     }
     const int bst = kClRows / p.G;
+    // tiles of one group per cluster: as few as fill one wave of the SMs (a cluster takes
+    // two), so that W_UV_g and the set-up are paid once per cluster, not once per tile
+    const int num_tiles = (p.bs_total + bst - 1) / bst;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaErrorInvalidValue;
+    const int clusters_per_group = (sms / 2) / num_groups > 0 ? (sms / 2) / num_groups : 1;
+    const int tpc = (num_tiles + clusters_per_group - 1) / clusters_per_group;
     CUtensorMap wmap;
     const uint64_t dims[2] = {(uint64_t)kDv, (uint64_t)num_groups * kLatent};
     const uint64_t strides[1] = {(uint64_t)kDv * 2};
@@ -546,9 +591,9 @@ cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int
     cudaError_t e = cudaFuncSetAttribute(combine_latent_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, ClSmem::kAlloc);
     if (e != cudaSuccess) return e;
-    dim3 grid(2, (unsigned)((p.bs_total + bst - 1) / bst), (unsigned)num_groups);
+    dim3 grid(2, (unsigned)((num_tiles + tpc - 1) / tpc), (unsigned)num_groups);
     return launch_dependent(combine_latent_tc_kernel, grid, dim3(kClThreads), ClSmem::kAlloc, stream,
-                            wmap, p, bst);
+                            wmap, p, bst, tpc, num_tiles);
 }
 
 }  // namespace gqla
