@@ -224,8 +224,8 @@ __global__ void __launch_bounds__(32 * kQuadsPerBlock, 3) combine_v_kernel(Combi
 // of one group (bst pairs x G heads), one after the other (as many per cluster as
 // keep the grid within one wave).  CTA kq merges latent columns
 // [256 kq, 256 kq + 256) of the tile's rows into bf16 (the MMA's A operand,
-// K-major, 128-byte swizzle); CTA 1 stores its half into CTA 0's shared memory
-// with asynchronous remote stores, and CTA 0 runs the whole product
+// K-major, 128-byte swizzle); CTA 1 sends its half into CTA 0's shared memory as
+// one bulk copy, and CTA 0 runs the whole product
 //   out[64 x 128] = A[64 x 512] * W_UV_g[512 x 128]   (tcgen05 M = 64, fp32 in TMEM)
 // and writes the bf16 rows.
 // ---------------------------------------------------------------------------
@@ -317,7 +317,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
         const int bs0 = (tile0 + k) * bst;
         if (k > 0) {
             // every warp is done with the previous tile's plan (and, in the leader, with the
-            // staging over A): the next plan replaces it
+            // staging over A; in the second CTA, the previous half has left its A): the next
+            // plan replaces it
+            if (!leader && tid == 0) bulk_wait_group_read<0>();
             __syncthreads();
             if (warp == 2) plan_pairs(p, bs0, bst, s_c0, s_c1);
             __syncthreads();
@@ -439,17 +441,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     }
 
     // ---- merged rows -> this CTA's four K blocks of A (bf16, K-major, 128-byte swizzle),
-    // at the place they take in the leader's A: the leader stores its own, the peer
-    // sends its half straight into the leader's shared memory (8-byte asynchronous
-    // stores counted on the leader's a_full)
-    if (!leader && k > 0 && !__syncthreads_and(mbar_wait(a_free, (k - 1) & 1, abort_flag))) {
-        ok = false;  // the leader stopped (or never freed A): send nothing more
-        break;
-    }
+    // at the place they take in the leader's A: the leader stores its own in place; the
+    // second CTA stores its half at the same place of its own (otherwise unused) A and
+    // sends it into the leader's as one 32 KB bulk copy counted on the leader's a_full
     {
         const int chunk = (lane & 15) >> 1, half8 = (lane & 1) * 8;
-        const uint32_t a_remote = leader ? 0u : map_peer(smem_u32(smem + ClSmem::oA), 0);
-        const uint32_t bar_remote = leader ? 0u : map_peer(smem_u32(a_full), 0);
 #pragma unroll
         for (int i = 0; i < kRw; ++i) {
             const int r = kRw * warp + i;
@@ -457,15 +453,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
             for (int h = 0; h < 2; ++h) {
                 const int kb = kq * 4 + 2 * h + (lane >> 4);
                 const uint32_t off = kb * (kClRows * 128) + r * 128 + ((chunk ^ (r & 7)) << 4) + half8;
-                const uint2 val = pack_bf16x4(acc[i][h].x, acc[i][h].y, acc[i][h].z, acc[i][h].w);
-                if (leader)
-                    *reinterpret_cast<uint2 *>(smem + ClSmem::oA + off) = val;
-                else
-                    st_async_v2(a_remote + off, val, bar_remote);
+                *reinterpret_cast<uint2 *>(smem + ClSmem::oA + off) =
+                    pack_bf16x4(acc[i][h].x, acc[i][h].y, acc[i][h].z, acc[i][h].w);
             }
         }
     }
-    if (!leader) continue;  // the second CTA goes on with its next tile's merge
+    if (!leader) {
+        fence_proxy_async_smem();  // the half -> the bulk copy (async proxy)
+        // the leader is done with the previous tile's A
+        if (!__syncthreads_and(k == 0 || mbar_wait(a_free, (k - 1) & 1, abort_flag))) {
+            ok = false;  // the leader stopped (or never freed A): send nothing more
+            break;
+        }
+        if (tid == 0) {
+            bulk_copy_to_peer(map_peer(smem_u32(smem + ClSmem::oA + ClSmem::kAHalf), 0),
+                              smem + ClSmem::oA + ClSmem::kAHalf, ClSmem::kAHalf,
+                              map_peer(smem_u32(a_full), 0));
+            bulk_commit_group();
+        }
+        continue;  // the second CTA goes on with its next tile's merge
+    }
     fence_proxy_async_smem();
     __syncthreads();
 
@@ -545,6 +552,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
     // the leader has consumed the last half it sent (the leader arrives once its MMAs are
     // done, or once it stopped), then both may exit.
     if (!leader) {
+        if (tid == 0) bulk_wait_group<0>();  // its last half has landed in the leader
         cluster_sync();
         return;
     }
