@@ -20,8 +20,9 @@ e2e     = the same through the C ABI with host buffers: each step copies the
           queries, page table and lengths from pinned host memory and reads
           both paths' outputs back into pinned memory, inside the timed region
           (replayed as one CUDA graph).  The batch is cut into sub-batches of
-          whole sequences ("sub_batches", 2 from 8 sequences up), each a full
-          step of its own with its own split plan, so one sub-batch's copies
+          whole sequences ("sub_batches": their sizes; two equal ones from 8
+          sequences up, or relative sizes from --e2e-parts such as 1,6,1), each
+          a full step of its own with its own split plan, so one sub-batch's copies
           overlap another's kernels: inputs on a copy-in stream, the absorb
           path on the main stream, the GQA path on a second stream, outputs
           on a copy-out stream as soon as each path of a sub-batch is done.
@@ -451,17 +452,24 @@ class Workbench:
         when every copy has landed.  Returns (ms, h2d, d2h, parts)."""
         gqla, dev, case = self.gqla, self.dev, self.case
         if parts is None:
-            parts = 2 if self.B >= 8 else 1
+            parts = [1, 1] if self.B >= 8 else [1]
+        elif isinstance(parts, int):
+            parts = [1] * parts
+        weights = [float(x) for x in parts]
         pt_c, sl_c = case["page_table"].cpu(), case["seqlens"].cpu()
         q_h = case["q"].cpu().pin_memory()
         q_e = torch.empty_like(case["q"])
         outa_h = torch.empty(self.ba.out.shape, dtype=torch.bfloat16).pin_memory()
         outg_h = torch.empty(self.bg.out.shape, dtype=torch.bfloat16).pin_memory()
         h, s_q = self.w.num_heads, self.s_q
-        cuts = [self.B * k // parts for k in range(parts + 1)]
+        # sub-batch boundaries in whole sequences, in proportion to the weights
+        acc = [sum(weights[:k]) for k in range(len(weights) + 1)]
+        cuts = [round(self.B * a / acc[-1]) for a in acc]
+        if any(b1 <= b0 for b0, b1 in zip(cuts, cuts[1:])):
+            raise ValueError(f"sub-batch weights {parts} leave an empty sub-batch of {self.B} sequences")
         lanes = []
         h2d = q_h.numel() * 2
-        for k in range(parts):
+        for k in range(len(weights)):
             b0, b1 = cuts[k], cuts[k + 1]
             pt_k, sl_k = pt_c[b0:b1].contiguous(), sl_c[b0:b1].contiguous()
             meta_h = torch.cat([pt_k.flatten(), sl_k]).pin_memory()
@@ -533,17 +541,23 @@ class Workbench:
             graph_e2e.replay()
         torch.cuda.synchronize()
         times = self.time_steps(steps, graph_e2e)
-        for ln in lanes:
-            if (not torch.equal(outa_h[ln["b0"]:ln["b1"]], ln["ba"].out.cpu())
-                    or not torch.equal(outg_h[ln["b0"]:ln["b1"]], ln["bg"].out.cpu())):
-                raise RuntimeError("end-to-end outputs differ from the device results")
+        for i, ln in enumerate(lanes):
+            for name, host, dev_out in (("absorb", outa_h, ln["ba"].out), ("gqa", outg_h, ln["bg"].out)):
+                got, ref = host[ln["b0"]:ln["b1"]], dev_out.cpu()
+                if not torch.equal(got, ref):
+                    bad = (got != ref)
+                    raise RuntimeError(
+                        f"end-to-end outputs differ from the device results: sub-batch {i} "
+                        f"({ln['b0']}..{ln['b1']}), {name} path, {int(bad.sum())} of {bad.numel()} values, "
+                        f"first at {tuple(int(x) for x in bad.nonzero()[0])}, NaN in copy "
+                        f"{int(torch.isnan(got.float()).sum())} / on device {int(torch.isnan(ref.float()).sum())}")
         # the sub-batches' results agree with the whole batch's (other split plans: fp32
         # merges in another order, so within rounding, not bit for bit)
         for got, ref in ((outa_h, self.ba.out), (outg_h, self.bg.out)):
             diff = (got.float() - ref.float().cpu()).abs().max().item()
             if not diff <= 2e-2:
                 raise RuntimeError(f"sub-batched outputs differ from the whole batch's by {diff}")
-        return sum(times) / len(times), h2d, d2h, parts
+        return sum(times) / len(times), h2d, d2h, [b1 - b0 for b0, b1 in zip(cuts, cuts[1:])]
 
     def report(self, mean, world, path_ms=None):
         """Per-kernel and per-path roofline fractions from the per-call means (ms)."""
@@ -715,7 +729,10 @@ def run_ours(args, rank, world, local_rank):
     mean = wb.time_calls(args.steps)
     path_ms = wb.time_paths(args.steps)
     wb.check_device_errors()
-    e2e_ms, h2d, d2h, e2e_parts = wb.e2e(args.steps, args.warmup, args.e2e_parts)
+    e2e_arg = None
+    if args.e2e_parts:
+        e2e_arg = [float(x) for x in args.e2e_parts.split(",")] if "," in args.e2e_parts else int(args.e2e_parts)
+    e2e_ms, h2d, d2h, e2e_parts = wb.e2e(args.steps, args.warmup, e2e_arg)
 
     # ---- max over ranks
     tokens_step = wb.B * wb.s_q
@@ -946,8 +963,9 @@ def main():
                     help="measure the headline workload only (not the rest of the suite)")
     ap.add_argument("--sparse-topk", type=int, default=0,
                     help="also time sparse GQLA with this many selected positions per query token")
-    ap.add_argument("--e2e-parts", type=int, default=None,
-                    help="sub-batches of the end-to-end step (default 2 from 8 sequences up, else 1)")
+    ap.add_argument("--e2e-parts", default=None,
+                    help="sub-batches of the end-to-end step: a count (equal parts) or relative "
+                         "sizes such as 1,2,1 (default two equal parts from 8 sequences up, else 1)")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
                     help="print the per-kernel summary of an ncu launch list and exit")
     args = ap.parse_args()
