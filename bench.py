@@ -7,8 +7,16 @@ MQA-absorb path (gqla_absorb_query -> gqla_decode_absorb -> gqla_combine with
 W_UV) and the GQA path (gqla_decode_gqa_step: the GQA decode, then the
 combine for the sequences that span more than one chunk) over the same batch.
 The two paths are independent, so the GQA path runs on a second stream beside
-the absorb path's decode and combine (after the query absorption has started):
-CTAs of one path take the SMs the other path's tail leaves idle.
+the absorb path's decode and combine (after the query absorption has started).
+Both decodes fill the device on their own, so beside each other they would run
+one after the other but for a lead in the absorb split plan
+(gqla_decode_absorb_lead, planned by gqla_plan_lead from the calls' own
+times, reported as "absorb_lead"): the absorb decode, launched first, has a few
+chunks about twice as long as the rest on the CTAs that the SMs left idle by
+the GQA decode's CTA count can hold, so the GQA decode starts on the SMs of
+the short chunks while the long ones keep the rest busy.  --no-lead runs the
+step with equal chunks.  The per-call ("per_kernel") and per-path times are
+always taken with equal chunks.
 The one-shot cache expansion (gqla_expand_cache) is a deploy-time conversion,
 not part of a step; it is timed once and reported under "expand".
 
@@ -288,7 +296,7 @@ class Workbench:
     """One workload (and s_q) on this rank's GPU: its seeded inputs, the expanded
     cache, both paths' buffers, and the five calls of a step through the C ABI."""
 
-    def __init__(self, name, s_q, rank, dev, splits=None):
+    def __init__(self, name, s_q, rank, dev, splits=None, lead=True):
         from decode_attention_06_b200 import gqla, synth
         self.gqla = gqla
         self.name, self.dev = name, dev
@@ -312,6 +320,11 @@ class Workbench:
         self.bg = gqla.DecodeBuffers(dims, self.B, s_q, self.splits["gqa"], "gqa", device=dev)
         self.gqa_stream = torch.cuda.Stream(device=dev)
         self.calls = self.make_calls(case["q"], self.kv)
+        # the absorb split plan's lead chunks in the step (gqla_plan_lead, from the calls'
+        # own times): (0, 16) = equal chunks
+        self.lead = (0, 16)
+        self.use_lead = lead
+        self.call_ms = None
 
     def gqa_step_call(self, q, kv):
         """The GQA path as one call (gqla_decode_gqa_step: the decode, and the combine for
@@ -355,9 +368,31 @@ class Workbench:
             res.append(e0.elapsed_time(e1))
         return res[1], res[0]
 
+    def lead_calls(self, q, kv, ba, lead):
+        """The absorb decode and combine on a split plan with lead chunks."""
+        gqla, dims, case = self.gqla, self.dims, self.case
+        return (lambda: gqla.gqla_decode_absorb_lead(dims, ba.q_absorbed, case["latent"], kv, ba.num_splits,
+                                                     lead[0], lead[1], ba.o_part, ba.lse_part, ba.workspace),
+                lambda: gqla.gqla_combine_lead(dims, kv, self.s_q, ba.num_splits, lead[0], lead[1], 512,
+                                               ba.o_part, ba.lse_part, case["w_uv"], ba.out, ba.lse))
+
+    def plan_lead(self, steps=5):
+        """Times the calls alone (equal chunks) and picks the absorb plan's lead for the
+        step: the absorb decode's CTAs on its short chunks leave their SMs to the GQA
+        decode, those on the lead chunks keep the SMs it leaves idle busy."""
+        self.call_ms = self.time_calls(steps)
+        if not self.use_lead:
+            return
+        self.lead = self.gqla.gqla_plan_lead(
+            self.dims, self.s_q, self.splits["absorb"], self.splits["gqa"],
+            self.call_ms["decode_absorb"] * 1e3, self.call_ms["decode_gqa"] * 1e3,
+            self.call_ms["combine_absorb"] * 1e3)
+
     def step(self):
         # query absorption first, then the GQA path (one call) on its own stream beside
-        # the absorb path's decode and combine; the step ends when both are done
+        # the absorb path's decode and combine; the step ends when both are done.  With a
+        # lead in the absorb plan the absorb decode is launched first, so that its CTAs
+        # are placed before the GQA decode's, which then take the SMs of the short chunks
         calls = self.calls
         gqa_step = self.gqa_step_call(self.case["q"], self.kv)
         main = torch.cuda.current_stream()
@@ -365,10 +400,17 @@ class Workbench:
         fork = torch.cuda.Event()
         fork.record(main)
         self.gqa_stream.wait_event(fork)
-        with torch.cuda.stream(self.gqa_stream):
-            gqa_step()
-        calls[1]()
-        calls[2]()
+        if self.lead[0] > 0:
+            dec, comb = self.lead_calls(self.case["q"], self.kv, self.ba, self.lead)
+            dec()
+            with torch.cuda.stream(self.gqa_stream):
+                gqa_step()
+            comb()
+        else:
+            with torch.cuda.stream(self.gqa_stream):
+                gqa_step()
+            calls[1]()
+            calls[2]()
         join = torch.cuda.Event()
         join.record(self.gqa_stream)
         main.wait_event(join)
@@ -376,14 +418,12 @@ class Workbench:
     def capture(self, warmup):
         """The step as one CUDA graph (the launches replay without host overhead, each
         kernel's set-up overlapping the previous kernel's tail on its stream), and a
-        second graph running the calls in order with an event record around each."""
+        second graph running the calls in order with an event record around each; the
+        latter's times plan the step's absorb lead before the step is captured."""
         for _ in range(warmup):
             flush_l2(self.dev)
             self.step()
         torch.cuda.synchronize()
-        self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph):
-            self.step()
         self.gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(self.calls) + 1)]
         self.graph_ev = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph_ev):
@@ -400,10 +440,22 @@ class Workbench:
                 for c in cs:
                     c()
             self.graph_path[path] = g_
-        for g_ in (self.graph, self.graph_ev, *self.graph_path.values()):
+        for g_ in (self.graph_ev, *self.graph_path.values()):
             for _ in range(warmup):
                 flush_l2(self.dev)
                 g_.replay()
+        torch.cuda.synchronize()
+        self.plan_lead()
+        for _ in range(warmup):
+            flush_l2(self.dev)
+            self.step()
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        for _ in range(warmup):
+            flush_l2(self.dev)
+            self.graph.replay()
         torch.cuda.synchronize()
 
     def time_steps(self, steps, graph=None):
@@ -481,12 +533,26 @@ class Workbench:
             ba = gqla.DecodeBuffers(self.dims, b1 - b0, s_q, sa, "absorb", device=dev)
             bg = gqla.DecodeBuffers(self.dims, b1 - b0, s_q, sg, "gqa", device=dev)
             q_k = q_e[b0:b1]
-            lanes.append(dict(b0=b0, b1=b1, meta_h=meta_h, meta_d=meta_d, kv=kv, ba=ba, bg=bg, q=q_k,
+            # the sub-batch's absorb lead, from the whole batch's call times scaled to its
+            # pages per chunk
+            lead = (0, 16)
+            if self.lead[0] > 0 and self.call_ms:
+                pg_all = int(((sl_c + gqla.PAGE_SIZE - 1) // gqla.PAGE_SIZE).sum())
+                pg_k = int(((sl_k + gqla.PAGE_SIZE - 1) // gqla.PAGE_SIZE).sum())
+                ta = self.call_ms["decode_absorb"] * 1e3 * (pg_k / sa) / (pg_all / self.splits["absorb"])
+                tg = self.call_ms["decode_gqa"] * 1e3 * (pg_k / sg) / (pg_all / self.splits["gqa"])
+                tc = self.call_ms["combine_absorb"] * 1e3 * pg_k / pg_all
+                lead = gqla.gqla_plan_lead(self.dims, s_q, sa, sg, ta, tg, tc)
+            if lead[0] > 0:
+                dec_k, comb_k = self.lead_calls(q_k, kv, ba, lead)
+            else:
+                dec_k = lambda kv=kv, ba=ba: gqla.gqla_decode_absorb(self.dims, ba.q_absorbed, case["latent"], kv,
+                                                                      ba.num_splits, ba.o_part, ba.lse_part, ba.workspace)
+                comb_k = lambda kv=kv, ba=ba: gqla.gqla_combine(self.dims, kv, s_q, ba.num_splits, 512, ba.o_part,
+                                                                 ba.lse_part, case["w_uv"], ba.out, ba.lse)
+            lanes.append(dict(b0=b0, b1=b1, meta_h=meta_h, meta_d=meta_d, kv=kv, ba=ba, bg=bg, q=q_k, lead=lead,
                               absorb=[lambda q_k=q_k, ba=ba: gqla.gqla_absorb_query(self.dims, q_k, case["w_uk"], ba.q_absorbed),
-                                      lambda kv=kv, ba=ba: gqla.gqla_decode_absorb(self.dims, ba.q_absorbed, case["latent"], kv,
-                                                                                   ba.num_splits, ba.o_part, ba.lse_part, ba.workspace),
-                                      lambda kv=kv, ba=ba: gqla.gqla_combine(self.dims, kv, s_q, ba.num_splits, 512, ba.o_part,
-                                                                             ba.lse_part, case["w_uv"], ba.out, ba.lse)],
+                                      dec_k, comb_k],
                               gqa=lambda q_k=q_k, kv=kv, bg=bg: gqla.gqla_decode_gqa_step(
                                   self.dims, q_k, self.kvx, self.kr, kv, bg.num_splits, bg.o_part, bg.lse_part,
                                   bg.out, bg.lse, bg.workspace)))
@@ -511,11 +577,14 @@ class Workbench:
             for ln, ev in zip(lanes, arrived):
                 main.wait_event(ev)
                 self.gqa_stream.wait_event(ev)
+                if ln["lead"][0] > 0:  # the absorb decode first (see step())
+                    ln["absorb"][0]()
+                    ln["absorb"][1]()
                 with torch.cuda.stream(self.gqa_stream):
                     ln["gqa"]()
                 gqa_done = torch.cuda.Event()
                 gqa_done.record(self.gqa_stream)
-                for c in ln["absorb"]:
+                for c in (ln["absorb"][2:] if ln["lead"][0] > 0 else ln["absorb"]):
                     c()
                 absorb_done = torch.cuda.Event()
                 absorb_done.record(main)
@@ -557,6 +626,7 @@ class Workbench:
             diff = (got.float() - ref.float().cpu()).abs().max().item()
             if not diff <= 2e-2:
                 raise RuntimeError(f"sub-batched outputs differ from the whole batch's by {diff}")
+        self.e2e_leads = [list(ln["lead"]) for ln in lanes]
         return sum(times) / len(times), h2d, d2h, [b1 - b0 for b0, b1 in zip(cuts, cuts[1:])]
 
     def report(self, mean, world, path_ms=None):
@@ -621,6 +691,7 @@ class Workbench:
                 "context": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths[1:]),
                 "s_q": self.s_q, "paged": w.paged, "paths": ["absorb", "gqa"],
                 "tokens_per_step": self.B * self.s_q, "num_splits": self.splits,
+                "absorb_lead": list(self.lead),
                 "l2": "flushed (256 MiB write + 256 MiB read) before every timed step",
                 "parallelism": f"replicas x{world} (independent batches per GPU)"}
 
@@ -634,7 +705,7 @@ def measure_other_workloads(args, headline, dev):
         for s in w.s_q:
             if (name, s) == headline:
                 continue
-            wb = Workbench(name, s, 0, dev, args.splits)
+            wb = Workbench(name, s, 0, dev, args.splits, lead=not args.no_lead)
             wb.time_expand()
             wb.capture(args.warmup)
             ms = wb.time_steps(args.steps)
@@ -645,7 +716,7 @@ def measure_other_workloads(args, headline, dev):
             out[f"{name}/sq{s}"] = {
                 "ms_per_step": sum(ms) / len(ms),
                 "tokens_per_s": wb.B * s / (sum(ms) / len(ms) * 1e-3),
-                "num_splits": wb.splits, "per_path": per_path,
+                "num_splits": wb.splits, "absorb_lead": list(wb.lead), "per_path": per_path,
                 "per_kernel_us": {n: per_kernel[n]["us"] for n in CALL_NAMES}}
             del wb
             torch.cuda.empty_cache()
@@ -713,7 +784,7 @@ def run_tp(args, rank, world, dev):
 def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wb = Workbench(args.workload, args.s_q, rank, dev, args.splits)
+    wb = Workbench(args.workload, args.s_q, rank, dev, args.splits, lead=not args.no_lead)
     expand_ms, expand_tc_ms = wb.time_expand()
     wb.capture(args.warmup)
 
@@ -752,7 +823,8 @@ def run_ours(args, rank, world, local_rank):
                    "tc_ms": expand_tc_ms,
                    "tc_tflops": acc["expand"]["flops"] / (expand_tc_ms * 1e-3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "sub_batches": e2e_parts},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "sub_batches": e2e_parts,
+                "absorb_leads": wb.e2e_leads},
         "gpu_launches": wb.launches_per_step() * args.steps,
         "clocks": clocks.summary(),
     }
@@ -966,6 +1038,8 @@ def main():
     ap.add_argument("--e2e-parts", default=None,
                     help="sub-batches of the end-to-end step: a count (equal parts) or relative "
                          "sizes such as 1,2,1 (default two equal parts from 8 sequences up, else 1)")
+    ap.add_argument("--no-lead", action="store_true",
+                    help="equal absorb chunks in the step too (no lead planned beside the GQA path)")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
                     help="print the per-kernel summary of an ncu launch list and exit")
     args = ap.parse_args()

@@ -37,6 +37,7 @@ struct CombineParams {
     float *lse_out;
     int batch;
     int num_splits;
+    int lead, lead_w16;  // the decode's split plan: lead chunks and their length (x 1/16)
     int s_q;
     int heads;
     int G;         // heads per group
@@ -67,7 +68,7 @@ __device__ void plan_pairs(const CombineParams &p, int bs_lo, int n, int *c0, in
         total += __shfl_xor_sync(0xffffffffu, total, o);
         start += __shfl_xor_sync(0xffffffffu, start, o);
     }
-    const int k = chunk_pages(total, p.num_splits);
+    const SplitPlan sp{p.num_splits, p.lead, p.lead_w16};
     const int excl = warp_incl_scan(np) - np;
     const int bs = bs_lo + lane;
     const int d = min(max(bs / p.s_q - b_first, 0), 31);
@@ -75,8 +76,8 @@ __device__ void plan_pairs(const CombineParams &p, int bs_lo, int n, int *c0, in
     const int st = start + __shfl_sync(0xffffffffu, excl, d);
     if (lane < n) {
         const bool any = bs < p.bs_total && np_d > 0;
-        c0[lane] = any ? st / k : 0;
-        c1[lane] = any ? (st + np_d - 1) / k + 1 : 0;
+        c0[lane] = any ? plan_chunk_of(total, sp, st) : 0;
+        c1[lane] = any ? plan_chunk_of(total, sp, st + np_d - 1) + 1 : 0;
     }
 }
 
@@ -567,13 +568,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kClThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int d_in,
-                           const float *o_part, const float *lse_part, const void *w_uv,
+cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int lead, int lead_w16,
+                           int d_in, const float *o_part, const float *lse_part, const void *w_uv,
                            void *out, float *lse_out, int heads, int num_groups, bool skip_single,
                            cudaStream_t stream) {
     CombineParams p{o_part, lse_part, kv->seqlens, static_cast<__nv_bfloat16 *>(out), lse_out,
-                    kv->batch, num_splits, s_q, heads, heads / num_groups, kv->batch * s_q,
-                    skip_single ? 1 : 0};
+                    kv->batch, num_splits, lead, lead_w16, s_q, heads, heads / num_groups,
+                    kv->batch * s_q, skip_single ? 1 : 0};
     if (d_in == kDv) {
         const int64_t quads = (int64_t)p.bs_total * (heads / 4);
         return launch_dependent(combine_v_kernel,

@@ -111,6 +111,43 @@ __device__ __forceinline__ int chunk_pages(int total_pages, int num_splits) {
     return (total_pages + num_splits - 1) / num_splits;
 }
 
+// A split plan with a lead: the batch's pages, concatenated sequence after sequence, are
+// cut into num_splits chunks of which the first `lead` are lead_w16 / 16 times as long as
+// the rest (whole pages, rounded up, the last chunks possibly short or empty).  With
+// lead = 0 this is the equal cut of chunk_pages().  The longer chunks exist for a step that
+// runs the GQA decode beside the absorb decode: the absorb decode's CTAs on the short
+// chunks finish early and leave their SMs to the GQA decode, while those on the long
+// chunks keep the SMs the GQA decode does not use busy.
+struct SplitPlan {
+    int num_splits, lead, lead_w16;
+};
+
+__device__ __forceinline__ void plan_chunk_lengths(int total, const SplitPlan &sp, int *k_lead, int *k_rest) {
+    const long long units = (long long)sp.lead * sp.lead_w16 + (long long)(sp.num_splits - sp.lead) * 16;
+    const long long k = ((long long)total * 16 + units - 1) / units;
+    *k_rest = (int)k;
+    *k_lead = (int)((k * sp.lead_w16 + 15) / 16);
+}
+
+// Pages [r0, r1) of chunk c (empty past the end).
+__device__ __forceinline__ void plan_chunk_range(int total, const SplitPlan &sp, int c, int *r0, int *r1) {
+    int kl, kr;
+    plan_chunk_lengths(total, sp, &kl, &kr);
+    const long long a = c < sp.lead ? (long long)c * kl : (long long)sp.lead * kl + (long long)(c - sp.lead) * kr;
+    const long long e = a + (c < sp.lead ? kl : kr);
+    *r0 = (int)(a < total ? a : total);
+    *r1 = (int)(e < total ? e : total);
+}
+
+// The chunk that holds global page `page` (0 <= page < total).
+__device__ __forceinline__ int plan_chunk_of(int total, const SplitPlan &sp, int page) {
+    int kl, kr;
+    plan_chunk_lengths(total, sp, &kl, &kr);
+    const long long head = (long long)sp.lead * kl;
+    const int c = page < head ? page / kl : sp.lead + (int)((page - head) / kr);
+    return c < sp.num_splits - 1 ? c : sp.num_splits - 1;
+}
+
 // Launch with programmatic stream serialization: the kernel may be scheduled
 // while the previous kernel of the stream finishes, and waits for it with
 // griddepcontrol.wait before touching global memory.

@@ -142,6 +142,7 @@ struct AbsorbParams {
     float *lse_part;
     void *ws;
     int batch, max_pages, num_pages, num_splits, s_q, heads;
+    int lead, lead_w16;  // the split plan's lead chunks and their length (x 1/16)
     int rows_total;   // s_q * heads: query rows of one sequence
     int row_blocks;   // ceil(rows_total / 128)
     float scale_log2;
@@ -235,7 +236,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_barrier_init();
     }
     griddep_wait();  // the previous kernel's results are visible from here on
-    griddep_launch_dependents();
+    // The combine may be scheduled as soon as every CTA has started: its set-up (split plan,
+    // W_UV) then overlaps this kernel's tail.  Not with lead chunks: the SMs of the CTAs that
+    // finish first belong to the GQA decode running beside this one, and a combine waiting
+    // there for the last CTA would hold them.
+    if (p.lead == 0) griddep_launch_dependents();
     // first page indices of the first piece, loaded by the producer warp while the
     // CTA and the cluster synchronise (valid when pre_ok)
     int pre_page = 0;
@@ -247,8 +252,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&qrope_map);
         }
         int total = warp_total_pages(p.seqlens, p.batch);
-        int k = chunk_pages(total, p.num_splits);
-        int r0 = c * k, r1 = min(total, r0 + k);
+        int r0, r1;
+        plan_chunk_range(total, SplitPlan{p.num_splits, p.lead, p.lead_w16}, c, &r0, &r1);
         int b = p.batch, start = 0;
         if (r0 < r1) warp_find_sequence(p.seqlens, p.batch, r0, &b, &start);
         if (lane == 0) { plan[0] = r0; plan[1] = r1; plan[2] = b; plan[3] = start; }
@@ -976,7 +981,7 @@ bool make_row_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t bo
 }  // namespace
 
 cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
-                                 const gqla_kv_index *idx, int num_splits, float scale,
+                                 const gqla_kv_index *idx, int num_splits, int lead, int lead_w16, float scale,
                                  float *o_part, float *lse_part, void *ws, cudaStream_t stream) {
     CUtensorMap lat, rope, qrope, omap;
     const uint64_t slots = (uint64_t)idx->num_pages * kPage;
@@ -1006,6 +1011,8 @@ cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void 
     p.max_pages = idx->max_pages_per_seq;
     p.num_pages = idx->num_pages;
     p.num_splits = num_splits;
+    p.lead = lead;
+    p.lead_w16 = lead_w16;
     p.s_q = s_q;
     p.heads = heads;
     p.rows_total = s_q * heads;

@@ -1057,6 +1057,8 @@ cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const CUte
     return launch_nq_mode<NQ, false>(kvm, krm, qm, kvm, krm, p, group_splits, stream);  // no row maps in dense mode
 }
 
+}  // namespace
+
 // CTAs per chunk: a batch too small to fill the GPU with one CTA per chunk has its groups
 // split over up to g CTAs per chunk (each reads the chunk's RoPE keys again: 128 of the
 // 4224 bytes of a token per extra CTA), as long as two such grids still fit in one wave.
@@ -1068,8 +1070,6 @@ int group_splits_for(int num_splits, int num_groups) {
     while (gs < num_groups && (int64_t)num_splits * gs * 4 <= sms) gs *= 2;
     return gs;
 }
-
-}  // namespace
 
 // Set by gqla_debug_drop_v_load, consumed by the next GQA decode launch of the thread.
 thread_local int g_drop_v_unit = -1;

@@ -29,12 +29,14 @@ cudaError_t launch_decode_gqa(const void *q, int s_q, int heads, int num_groups,
                               int num_splits, float scale, float *o_part, float *lse_part,
                               void *out, float *lse_out, void *ws, cudaStream_t stream);
 cudaError_t launch_decode_absorb(const void *qa, int s_q, int heads, const void *cache,
-                                 const gqla_kv_index *idx, int num_splits, float scale,
-                                 float *o_part, float *lse_part, void *ws, cudaStream_t stream);
-cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int d_in,
-                           const float *o_part, const float *lse_part, const void *w_uv,
+                                 const gqla_kv_index *idx, int num_splits, int lead, int lead_w16,
+                                 float scale, float *o_part, float *lse_part, void *ws,
+                                 cudaStream_t stream);
+cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int lead, int lead_w16,
+                           int d_in, const float *o_part, const float *lse_part, const void *w_uv,
                            void *out, float *lse_out, int heads, int num_groups, bool skip_single,
                            cudaStream_t stream);
+int group_splits_for(int num_splits, int num_groups);
 extern thread_local int g_drop_v_unit;
 }  // namespace gqla
 
@@ -45,6 +47,11 @@ namespace {
 constexpr size_t kWorkspaceBytes = 256;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A lead of 0 .. num_splits chunks, each 1 to 64 times as long as the others (in 1/16).
+bool lead_ok(int num_splits, int lead, int w16) {
+    return lead >= 0 && lead <= num_splits && w16 >= 16 && w16 <= 1024;
+}
 
 int check_dims(const gqla_dims *d, int s_q) {
     if (!d) return GQLA_ERR_INVALID_ARG;
@@ -139,6 +146,44 @@ int gqla_num_splits_hint(int path, int num_heads, int s_q) {
     return sms / (2 * row_blocks) > 0 ? sms / (2 * row_blocks) : 1;
 }
 
+int gqla_plan_lead(const gqla_dims *dims, int s_q, int absorb_splits, int gqa_splits,
+                   float absorb_decode_us, float gqa_decode_us, float absorb_combine_us,
+                   int *lead_splits, int *lead_weight16) {
+    int st = check_dims(dims, s_q);
+    if (st != GQLA_OK) return st;
+    if (absorb_splits <= 0 || absorb_splits > 65535 || gqa_splits <= 0 || gqa_splits > 65535 ||
+        !lead_splits || !lead_weight16 || !(absorb_decode_us > 0.0f) || !(gqa_decode_us >= 0.0f) ||
+        !(absorb_combine_us >= 0.0f))
+        return GQLA_ERR_INVALID_ARG;
+    *lead_splits = 0;
+    *lead_weight16 = 16;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQLA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GQLA_ERR_CUDA;
+    // SMs the GQA decode leaves idle, in absorb chunks (2 CTAs per 128 query rows)
+    const int row_blocks = (s_q * dims->num_heads + 127) / 128;
+    const int gqa_ctas = gqa_splits * group_splits_for(gqa_splits, dims->num_groups);
+    const int free_sms = sms - gqa_ctas;
+    const int n = absorb_splits;
+    int e = free_sms > 0 ? free_sms / (2 * row_blocks) : 0;
+    if (e > n - 1) e = n - 1;
+    // The short chunks' CTAs finish at T_s; the GQA decode then runs on their SMs for
+    // gqa_decode_us, and the lead chunks should end the absorb combine's time before it
+    // does: W T_s = T_s + x with x = gqa - combine.  The work is the same as with equal
+    // chunks of time T_a: (e W + n - e) T_s = n T_a.  So W - 1 = (x / T_a) / (1 - x e / (n T_a)).
+    const double x = (double)gqa_decode_us - (double)absorb_combine_us;
+    if (e <= 0 || x <= 0.0) return GQLA_OK;
+    const double ta = absorb_decode_us;
+    double den = 1.0 - x * e / (n * ta);
+    if (den < 0.05) den = 0.05;
+    double w = 1.0 + (x / ta) / den;
+    if (w > 64.0) w = 64.0;
+    *lead_splits = e;
+    *lead_weight16 = (int)lround(16.0 * w);
+    return GQLA_OK;
+}
+
 int gqla_plan_splits(const int32_t *seqlens, int batch, int max_splits, int piece_cost_pages) {
     if (!seqlens || batch <= 0 || batch > 65535 || max_splits <= 0 || max_splits > 65535 ||
         piece_cost_pages < 0)
@@ -228,11 +273,20 @@ int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
                        const void *latent_cache, const gqla_kv_index *kv, int num_splits,
                        float *o_part, float *lse_part, void *workspace, size_t workspace_bytes,
                        gqla_stream_t stream) {
+    return gqla_decode_absorb_lead(dims, q_absorbed, s_q, latent_cache, kv, num_splits, 0, 16, o_part,
+                                   lse_part, workspace, workspace_bytes, stream);
+}
+
+int gqla_decode_absorb_lead(const gqla_dims *dims, const void *q_absorbed, int s_q,
+                            const void *latent_cache, const gqla_kv_index *kv, int num_splits,
+                            int lead_splits, int lead_weight16, float *o_part, float *lse_part,
+                            void *workspace, size_t workspace_bytes, gqla_stream_t stream) {
     int st = check_dims(dims, s_q);
     if (st != GQLA_OK) return st;
     if ((st = check_index(kv)) != GQLA_OK) return st;
     if ((st = check_workspace(workspace, workspace_bytes)) != GQLA_OK) return st;
     if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
+    if (!lead_ok(num_splits, lead_splits, lead_weight16)) return GQLA_ERR_INVALID_ARG;
     if (!q_absorbed || !latent_cache || !o_part || !lse_part) return GQLA_ERR_INVALID_ARG;
     if (!aligned16(q_absorbed) || !aligned16(latent_cache) || !aligned16(o_part))
         return GQLA_ERR_INVALID_ARG;
@@ -240,8 +294,9 @@ int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
     if ((int64_t)num_splits * ((s_q * dims->num_heads + 127) / 128) * 2 > 65535 * 2)
         return GQLA_ERR_UNSUPPORTED;
     return cuda_status(launch_decode_absorb(q_absorbed, s_q, dims->num_heads, latent_cache, kv,
-                                            num_splits, dims->softmax_scale, o_part, lse_part,
-                                            workspace, reinterpret_cast<cudaStream_t>(stream)));
+                                            num_splits, lead_splits, lead_weight16, dims->softmax_scale,
+                                            o_part, lse_part, workspace,
+                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int gqla_decode_gqa(const gqla_dims *dims, const void *q, int s_q, const void *kv_expanded,
@@ -287,8 +342,8 @@ int gqla_decode_gqa_step(const gqla_dims *dims, const void *q, int s_q, const vo
                                        num_slots, kv, num_splits, dims->softmax_scale, o_part, lse_part,
                                        out, lse_out, workspace, s));
     if (st != GQLA_OK || num_splits == 1) return st;  // one chunk: every sequence is final already
-    return cuda_status(launch_combine(kv, s_q, num_splits, kDv, o_part, lse_part, nullptr, out, lse_out,
-                                      dims->num_heads, dims->num_groups, true, s));
+    return cuda_status(launch_combine(kv, s_q, num_splits, 0, 16, kDv, o_part, lse_part, nullptr, out,
+                                      lse_out, dims->num_heads, dims->num_groups, true, s));
 }
 
 int gqla_sparse_gather(const gqla_dims *dims, const void *kv_expanded, const void *k_rope,
@@ -359,10 +414,19 @@ int gqla_decode_gqa_sparse(const gqla_dims *dims, const void *q, int s_q, const 
 int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
                  int d_in, const float *o_part, const float *lse_part, const void *w_uv,
                  void *out, float *lse_out, gqla_stream_t stream) {
+    return gqla_combine_lead(dims, kv, s_q, num_splits, 0, 16, d_in, o_part, lse_part, w_uv, out,
+                             lse_out, stream);
+}
+
+int gqla_combine_lead(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
+                      int lead_splits, int lead_weight16, int d_in, const float *o_part,
+                      const float *lse_part, const void *w_uv, void *out, float *lse_out,
+                      gqla_stream_t stream) {
     int st = check_dims(dims, s_q);
     if (st != GQLA_OK) return st;
     if ((st = check_index(kv)) != GQLA_OK) return st;
     if (num_splits <= 0 || num_splits > 65535) return GQLA_ERR_INVALID_ARG;
+    if (!lead_ok(num_splits, lead_splits, lead_weight16)) return GQLA_ERR_INVALID_ARG;
     if (!o_part || !lse_part || !out) return GQLA_ERR_INVALID_ARG;
     if (!aligned16(o_part) || !aligned16(out) || (w_uv && !aligned16(w_uv)))
         return GQLA_ERR_INVALID_ARG;
@@ -373,9 +437,9 @@ int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int nu
     } else {
         return GQLA_ERR_INVALID_ARG;
     }
-    return cuda_status(launch_combine(kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out,
-                                      lse_out, dims->num_heads, dims->num_groups, false,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_combine(kv, s_q, num_splits, lead_splits, lead_weight16, d_in, o_part,
+                                      lse_part, w_uv, out, lse_out, dims->num_heads, dims->num_groups,
+                                      false, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -61,9 +61,11 @@ _SIGS = {
     "gqla_expand_cache_tc": [_DP, _P, _I64, _P, _P, _P, _P, _P],
     "gqla_absorb_query": [_DP, _P, _I, _I, _P, _P, _P],
     "gqla_decode_absorb": [_DP, _P, _I, _P, _KP, _I, _P, _P, _P, _SZ, _P],
+    "gqla_decode_absorb_lead": [_DP, _P, _I, _P, _KP, _I, _I, _I, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa_step": [_DP, _P, _I, _P, _P, _I64, _KP, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "gqla_combine": [_DP, _KP, _I, _I, _I, _P, _P, _P, _P, _P, _P],
+    "gqla_combine_lead": [_DP, _KP, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P],
     "gqla_sparse_gather": [_DP, _P, _P, _I64, _KP, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "gqla_sparse_select": [_DP, _KP, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
     "gqla_decode_gqa_sparse": [_DP, _P, _I, _P, _P, _I64, _KP, _P, _I, _P, _P, _P, _SZ, _P],
@@ -72,6 +74,8 @@ _SIGS = {
     "gqla_workspace_bytes": [],
     "gqla_num_splits_hint": [_I, _I, _I],
     "gqla_plan_splits": [_P, _I, _I, _I],
+    "gqla_plan_lead": [_DP, _I, _I, _I, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                       ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)],
     "gqla_read_device_error": [_P, ctypes.POINTER(ctypes.c_int), _P],
     "gqla_clear_device_error": [_P, _P],
     "gqla_status_string": [_I],
@@ -161,16 +165,24 @@ def gqla_absorb_query(dims, q, w_uk, q_absorbed, stream=None):
 
 
 def gqla_decode_absorb(dims, q_absorbed, latent_cache, kv, num_splits, o_part, lse_part,
-                       workspace, stream=None):
+                       workspace, stream=None, lead=None):
+    """lead = (lead_splits, lead_weight16) calls gqla_decode_absorb_lead."""
     B, s_q, h, _ = q_absorbed.shape
     slots = gqla_partial_slots(kv.batch, num_splits)
-    _check("gqla_decode_absorb", _lib.gqla_decode_absorb(
+    fn, extra = ("gqla_decode_absorb", ()) if lead is None else ("gqla_decode_absorb_lead", tuple(lead))
+    _check(fn, getattr(_lib, fn)(
         ctypes.byref(dims), _dev(q_absorbed, "q_absorbed", torch.bfloat16, (kv.batch, s_q, dims.num_heads, D_ROW)),
         s_q, _dev(latent_cache, "latent_cache", torch.bfloat16, (kv.num_pages, kv.page_size, D_ROW)),
-        ctypes.byref(kv), num_splits,
+        ctypes.byref(kv), num_splits, *extra,
         _dev(o_part, "o_part", torch.float32, (slots, s_q, h, D_LATENT)),
         _dev(lse_part, "lse_part", torch.float32, (slots, s_q, h)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gqla_decode_absorb_lead(dims, q_absorbed, latent_cache, kv, num_splits, lead_splits, lead_weight16,
+                            o_part, lse_part, workspace, stream=None):
+    gqla_decode_absorb(dims, q_absorbed, latent_cache, kv, num_splits, o_part, lse_part, workspace,
+                       stream, lead=(lead_splits, lead_weight16))
 
 
 def gqla_decode_gqa(dims, q, kv_expanded, k_rope, kv, num_splits, o_part, lse_part, workspace,
@@ -206,11 +218,13 @@ def gqla_decode_gqa_step(dims, q, kv_expanded, k_rope, kv, num_splits, o_part, l
 
 
 def gqla_combine(dims, kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out, lse_out=None,
-                 stream=None):
+                 stream=None, lead=None):
+    """lead = (lead_splits, lead_weight16), as given to the decode, calls gqla_combine_lead."""
     slots = gqla_partial_slots(kv.batch, num_splits)
     h = dims.num_heads
-    _check("gqla_combine", _lib.gqla_combine(
-        ctypes.byref(dims), ctypes.byref(kv), s_q, num_splits, d_in,
+    fn, extra = ("gqla_combine", ()) if lead is None else ("gqla_combine_lead", tuple(lead))
+    _check(fn, getattr(_lib, fn)(
+        ctypes.byref(dims), ctypes.byref(kv), s_q, num_splits, *extra, d_in,
         _dev(o_part, "o_part", torch.float32, (slots, s_q, h, d_in)),
         _dev(lse_part, "lse_part", torch.float32, (slots, s_q, h)),
         None if w_uv is None else _dev(w_uv, "w_uv", torch.bfloat16, (dims.num_groups, D_LATENT, D_V)),
@@ -297,6 +311,22 @@ def gqla_num_splits_hint(path: str, num_heads: int, s_q: int) -> int:
     if n < 0:
         raise GqlaError("gqla_num_splits_hint", n)
     return n
+
+
+def gqla_combine_lead(dims, kv, s_q, num_splits, lead_splits, lead_weight16, d_in, o_part, lse_part, w_uv,
+                      out, lse_out=None, stream=None):
+    gqla_combine(dims, kv, s_q, num_splits, d_in, o_part, lse_part, w_uv, out, lse_out, stream,
+                 lead=(lead_splits, lead_weight16))
+
+
+def gqla_plan_lead(dims, s_q: int, absorb_splits: int, gqa_splits: int, absorb_decode_us: float,
+                   gqa_decode_us: float, absorb_combine_us: float):
+    """(lead_splits, lead_weight16) for the absorb decode beside the GQA path."""
+    e, w = ctypes.c_int(0), ctypes.c_int(16)
+    _check("gqla_plan_lead", _lib.gqla_plan_lead(
+        ctypes.byref(dims), s_q, absorb_splits, gqa_splits, absorb_decode_us, gqa_decode_us,
+        absorb_combine_us, ctypes.byref(e), ctypes.byref(w)))
+    return e.value, w.value
 
 
 def gqla_plan_splits(seqlens, max_splits: int, piece_cost_pages: int) -> int:

@@ -155,6 +155,28 @@ int gqla_decode_absorb(const gqla_dims *dims, const void *q_absorbed, int s_q,
                        gqla_stream_t stream);
 
 /*
+ * gqla_decode_absorb with a lead in the split plan: of the num_splits chunks,
+ * the first `lead_splits` are lead_weight16 / 16 times as long as the others
+ * (k = ceil(16 T / (lead_splits * lead_weight16 + 16 (num_splits - lead_splits)))
+ * pages for the others, ceil(k * lead_weight16 / 16) for the lead ones, cut in
+ * that order; the last chunks may come out short or empty).  The partials go
+ * to the same slots (b + chunk) and must be merged by gqla_combine_lead with the
+ * same three numbers.  lead_splits 0 (or lead_weight16 16) is gqla_decode_absorb.
+ * This is for a step that runs the GQA path beside the absorb path on another
+ * stream (gqla_plan_lead picks the numbers): the CTAs of the short chunks finish
+ * early and leave their SMs to the GQA decode, while the lead chunks keep busy
+ * the SMs that the GQA decode does not use.  Launched before the GQA decode, and
+ * with a lead the decode does not let the combine be scheduled before its last
+ * CTA is done, so nothing waits on the SMs it frees.
+ *   lead_splits    0 .. num_splits;  lead_weight16  16 .. 1024
+ * Otherwise as gqla_decode_absorb (GQLA_ERR_INVALID_ARG for a lead out of range).
+ */
+int gqla_decode_absorb_lead(const gqla_dims *dims, const void *q_absorbed, int s_q,
+                            const void *latent_cache, const gqla_kv_index *kv, int num_splits,
+                            int lead_splits, int lead_weight16, float *o_part, float *lse_part,
+                            void *workspace, size_t workspace_bytes, gqla_stream_t stream);
+
+/*
  * Split-KV partial attention, GQA path: the G*s_q query rows of each group
  * score [K_nope_g | k^R] (192) and accumulate V_g (128) (paperlayer.ai
  * summary, sec. 3 "Two equivalent decoding paths" and sec. 4, "GQA path";
@@ -270,6 +292,13 @@ int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int nu
                  int d_in, const float *o_part, const float *lse_part, const void *w_uv,
                  void *out, float *lse_out, gqla_stream_t stream);
 
+/* gqla_combine for partials written by gqla_decode_absorb_lead: the same
+ * lead_splits and lead_weight16 locate each sequence's partial slots. */
+int gqla_combine_lead(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
+                      int lead_splits, int lead_weight16, int d_in, const float *o_part,
+                      const float *lse_part, const void *w_uv, void *out, float *lse_out,
+                      gqla_stream_t stream);
+
 /*
  * GQA-path decode step that allocates nothing: gqla_decode_gqa followed by
  * gqla_combine, with the split partials, their LSEs and the device error
@@ -336,6 +365,21 @@ int gqla_num_splits_hint(int path, int num_heads, int s_q);
  *   piece_cost_pages  >= 0
  * Returns the split count, or GQLA_ERR_INVALID_ARG. */
 int gqla_plan_splits(const int32_t *seqlens, int batch, int max_splits, int piece_cost_pages);
+
+/* The lead of the absorb path's split plan (gqla_decode_absorb_lead) for a step
+ * that runs both paths over one batch on two streams, the absorb decode
+ * launched first.  From the times each call takes alone with equal chunks
+ * (measured by the caller, µs): lead_splits = the absorb chunks whose CTAs fit
+ * on the SMs of the current device that the GQA decode (gqa_splits chunks, and
+ * its group split) leaves idle; lead_weight16 such that the lead chunks end
+ * the absorb combine's time before the GQA decode does, with the total work
+ * unchanged: W = 1 + (x / T_a) / (1 - x lead / (absorb_splits T_a)), x = gqa -
+ * combine, T_a = absorb_decode_us, capped at 64.  lead 0 (equal chunks) when
+ * the GQA decode fills the device or x <= 0.
+ * Returns GQLA_OK, GQLA_ERR_INVALID_ARG or GQLA_ERR_CUDA (no device). */
+int gqla_plan_lead(const gqla_dims *dims, int s_q, int absorb_splits, int gqa_splits,
+                   float absorb_decode_us, float gqa_decode_us, float absorb_combine_us,
+                   int *lead_splits, int *lead_weight16);
 
 /* Reads (synchronising `stream`) and returns the first device-side error
  * recorded in `workspace` (GQLA_OK if none); `info`, if not NULL, receives

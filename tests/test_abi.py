@@ -223,3 +223,24 @@ def test_plan_splits_edges(lib):
     assert lib.gqla_plan_splits(None, 1, 4, 6) == -1
     arr = (ctypes.c_int32 * 1)(64)
     assert lib.gqla_plan_splits(arr, 0, 4, 6) == -1
+
+
+def test_lead_calls_reject_bad_arguments(lib):
+    """The lead split plan: 0 .. num_splits lead chunks, each 1 to 64 times as long as the
+    others (weight in 1/16); the planner checks its arguments before it asks the device."""
+    d, kv = _dims(), _kv()
+    wsb = ctypes.c_size_t(256)
+    for lead, w16 in ((5, 32), (-1, 32), (1, 15), (1, 1025)):
+        assert lib.gqla_decode_absorb_lead(ctypes.byref(d), FAKE, 1, FAKE, ctypes.byref(kv), 4, lead, w16,
+                                           FAKE, FAKE, FAKE, wsb, None) == -1, (lead, w16)
+        assert lib.gqla_combine_lead(ctypes.byref(d), ctypes.byref(kv), 1, 4, lead, w16, 512, FAKE, FAKE,
+                                     FAKE, FAKE, None, None) == -1, (lead, w16)
+    F = ctypes.c_float
+    e, w = ctypes.c_int(), ctypes.c_int()
+    plan = lambda *a: lib.gqla_plan_lead(*a)
+    assert plan(ctypes.byref(d), 2, 0, 128, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(ctypes.byref(d), 2, 37, 0, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(ctypes.byref(d), 2, 37, 128, F(0), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(ctypes.byref(d), 2, 37, 128, F(400), F(-1), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(ctypes.byref(d), 2, 37, 128, F(400), F(350), F(30), None, ctypes.byref(w)) == -1
+    assert plan(ctypes.byref(d), 3, 37, 128, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -2

@@ -179,6 +179,61 @@ def test_decode_parity_four_groups(path, cid, h, seqlens, s_q, paged, splits):
     assert gqla.gqla_read_device_error(ws)[0] == 0
 
 
+LEAD = [
+    # id, h, seqlens, s_q, paged, num_splits, (lead_splits, lead_weight16)
+    ("ragged_paged_lead2x", 128, [1000, 64, 1, 777], 1, True, 7, (2, 32)),
+    ("mtp_lead3x", 128, [513, 130], 2, True, 5, (1, 48)),
+    ("every_chunk_lead", 32, [2000, 3, 70], 2, False, 6, (6, 40)),
+    # the lead chunks take nearly everything, the last chunks come out empty
+    ("lead_swallows_batch", 128, [300, 200], 2, True, 6, (2, 512)),
+    ("zero_length_lead", 32, [0, 65, 0, 700], 1, False, 4, (1, 24)),
+    ("headline_shape_lead", 128, [4096, 4096, 4096], 2, True, 9, (2, 30)),
+]
+
+
+@pytest.mark.parametrize("cid,h,seqlens,s_q,paged,splits,lead", LEAD, ids=[c[0] for c in LEAD])
+def test_absorb_lead_split_parity(cid, h, seqlens, s_q, paged, splits, lead):
+    """Absorb decode and combine on a split plan with lead chunks (the first lead_splits
+    chunks lead_weight16 / 16 times as long): the same outputs as the oracle, and within
+    fp32 merge rounding of the equal-chunk plan."""
+    from decode_attention_06_b200 import gqla
+    case = synth.make_case(h, 8, seqlens, s_q, paged=paged, seed=zlib.crc32(cid.encode()) % 1000)
+    g = to_gpu(case)
+    dims = gqla.make_dims(h, 8)
+    kv = gqla.make_kv_index(g["page_table"], g["seqlens"], g["num_pages"])
+    B = g["seqlens"].numel()
+    bufs = gqla.DecodeBuffers(dims, B, s_q, splits, "absorb")
+    gqla.gqla_absorb_query(dims, g["q"], g["w_uk"], bufs.q_absorbed)
+    gqla.gqla_decode_absorb(dims, bufs.q_absorbed, g["latent"], kv, splits, bufs.o_part, bufs.lse_part,
+                            bufs.workspace, lead=lead)
+    gqla.gqla_combine(dims, kv, s_q, splits, 512, bufs.o_part, bufs.lse_part, g["w_uv"], bufs.out,
+                      bufs.lse, lead=lead)
+    torch.cuda.synchronize()
+    assert gqla.gqla_read_device_error(bufs.workspace)[0] == 0
+    ref, ref_lse = oracle_ref(case)
+    compare(bufs.out, ref, what=f"absorb-lead/{cid}")
+    compare_lse(bufs.lse, ref_lse, what=f"absorb-lead/{cid}")
+    eq, eq_lse, _, _ = run_decode(g, "absorb", splits)
+    d = (bufs.out.float() - eq.float()).abs().max().item()
+    assert d <= 2e-2, f"lead plan vs equal chunks: {d}"
+
+
+def test_plan_lead_on_device():
+    """gqla_plan_lead at the 64 x 8192 s_q = 2 shape: the absorb chunks whose 2 x 2 CTAs
+    fit on the SMs the GQA decode's 128 CTAs leave idle, each about twice as long."""
+    from decode_attention_06_b200 import gqla
+    dims = gqla.make_dims(128, 8)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    e, w16 = gqla.gqla_plan_lead(dims, 2, 37, 128, 414.0, 359.0, 37.0)
+    assert e == min(max((sms - 128) // 4, 0), 36)
+    if e:
+        # W = 1 + (x / T_a) / (1 - x e / (n T_a)), x = 359 - 37
+        x, ta = 359.0 - 37.0, 414.0
+        assert w16 == round(16 * (1 + (x / ta) / (1 - x * e / (37 * ta))))
+    # the GQA decode fills the device: no lead
+    assert gqla.gqla_plan_lead(dims, 2, 37, sms, 414.0, 359.0, 37.0) == (0, 16)
+
+
 def test_paths_agree():
     case = synth.make_case(128, 8, [700, 129], 2, paged=True, seed=120)
     g = to_gpu(case)
