@@ -324,6 +324,7 @@ class Workbench:
         # own times): (0, 16) = equal chunks
         self.lead = (0, 16)
         self.use_lead = lead
+        self.e2e_lead = False
         self.call_ms = None
 
     def gqa_step_call(self, q, kv):
@@ -534,9 +535,10 @@ class Workbench:
             bg = gqla.DecodeBuffers(self.dims, b1 - b0, s_q, sg, "gqa", device=dev)
             q_k = q_e[b0:b1]
             # the sub-batch's absorb lead, from the whole batch's call times scaled to its
-            # pages per chunk
+            # pages per chunk (only with --e2e-lead: the sub-batches overlap one another's
+            # paths, which the lead's model does not cover)
             lead = (0, 16)
-            if self.lead[0] > 0 and self.call_ms:
+            if self.e2e_lead and self.lead[0] > 0 and self.call_ms:
                 pg_all = int(((sl_c + gqla.PAGE_SIZE - 1) // gqla.PAGE_SIZE).sum())
                 pg_k = int(((sl_k + gqla.PAGE_SIZE - 1) // gqla.PAGE_SIZE).sum())
                 ta = self.call_ms["decode_absorb"] * 1e3 * (pg_k / sa) / (pg_all / self.splits["absorb"])
@@ -785,6 +787,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wb = Workbench(args.workload, args.s_q, rank, dev, args.splits, lead=not args.no_lead)
+    wb.e2e_lead = args.e2e_lead
     expand_ms, expand_tc_ms = wb.time_expand()
     wb.capture(args.warmup)
 
@@ -1038,6 +1041,8 @@ def main():
     ap.add_argument("--e2e-parts", default=None,
                     help="sub-batches of the end-to-end step: a count (equal parts) or relative "
                          "sizes such as 1,2,1 (default two equal parts from 8 sequences up, else 1)")
+    ap.add_argument("--e2e-lead", action="store_true",
+                    help="give the end-to-end sub-batches absorb leads too (scaled from the step's)")
     ap.add_argument("--no-lead", action="store_true",
                     help="equal absorb chunks in the step too (no lead planned beside the GQA path)")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
