@@ -385,7 +385,8 @@ class Workbench:
         if not self.use_lead:
             return
         self.lead = self.gqla.gqla_plan_lead(
-            self.dims, self.s_q, self.splits["absorb"], self.splits["gqa"],
+            self.dims, self.s_q, torch.cuda.get_device_properties(self.dev).multi_processor_count,
+            self.splits["absorb"], self.splits["gqa"],
             self.call_ms["decode_absorb"] * 1e3, self.call_ms["decode_gqa"] * 1e3,
             self.call_ms["combine_absorb"] * 1e3)
 
@@ -544,7 +545,8 @@ class Workbench:
                 ta = self.call_ms["decode_absorb"] * 1e3 * (pg_k / sa) / (pg_all / self.splits["absorb"])
                 tg = self.call_ms["decode_gqa"] * 1e3 * (pg_k / sg) / (pg_all / self.splits["gqa"])
                 tc = self.call_ms["combine_absorb"] * 1e3 * pg_k / pg_all
-                lead = gqla.gqla_plan_lead(self.dims, s_q, sa, sg, ta, tg, tc)
+                sms = torch.cuda.get_device_properties(dev).multi_processor_count
+                lead = gqla.gqla_plan_lead(self.dims, s_q, sms, sa, sg, ta, tg, tc)
             if lead[0] > 0:
                 dec_k, comb_k = self.lead_calls(q_k, kv, ba, lead)
             else:

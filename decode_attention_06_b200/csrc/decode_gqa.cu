@@ -1062,13 +1062,17 @@ cudaError_t launch_nq(const CUtensorMap &kvm, const CUtensorMap &krm, const CUte
 // CTAs per chunk: a batch too small to fill the GPU with one CTA per chunk has its groups
 // split over up to g CTAs per chunk (each reads the chunk's RoPE keys again: 128 of the
 // 4224 bytes of a token per extra CTA), as long as two such grids still fit in one wave.
+int group_splits_rule(int num_splits, int num_groups, int sms) {
+    int gs = 1;
+    while (gs < num_groups && (int64_t)num_splits * gs * 4 <= sms) gs *= 2;
+    return gs;
+}
+
 int group_splits_for(int num_splits, int num_groups) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int gs = 1;
-    while (gs < num_groups && (int64_t)num_splits * gs * 4 <= sms) gs *= 2;
-    return gs;
+    return group_splits_rule(num_splits, num_groups, sms);
 }
 
 // Set by gqla_debug_drop_v_load, consumed by the next GQA decode launch of the thread.

@@ -36,7 +36,7 @@ cudaError_t launch_combine(const gqla_kv_index *kv, int s_q, int num_splits, int
                            int d_in, const float *o_part, const float *lse_part, const void *w_uv,
                            void *out, float *lse_out, int heads, int num_groups, bool skip_single,
                            cudaStream_t stream);
-int group_splits_for(int num_splits, int num_groups);
+int group_splits_rule(int num_splits, int num_groups, int sms);
 extern thread_local int g_drop_v_unit;
 }  // namespace gqla
 
@@ -146,24 +146,21 @@ int gqla_num_splits_hint(int path, int num_heads, int s_q) {
     return sms / (2 * row_blocks) > 0 ? sms / (2 * row_blocks) : 1;
 }
 
-int gqla_plan_lead(const gqla_dims *dims, int s_q, int absorb_splits, int gqa_splits,
+int gqla_plan_lead(const gqla_dims *dims, int s_q, int num_sms, int absorb_splits, int gqa_splits,
                    float absorb_decode_us, float gqa_decode_us, float absorb_combine_us,
                    int *lead_splits, int *lead_weight16) {
     int st = check_dims(dims, s_q);
     if (st != GQLA_OK) return st;
-    if (absorb_splits <= 0 || absorb_splits > 65535 || gqa_splits <= 0 || gqa_splits > 65535 ||
-        !lead_splits || !lead_weight16 || !(absorb_decode_us > 0.0f) || !(gqa_decode_us >= 0.0f) ||
-        !(absorb_combine_us >= 0.0f))
+    if (num_sms <= 0 || absorb_splits <= 0 || absorb_splits > 65535 || gqa_splits <= 0 ||
+        gqa_splits > 65535 || !lead_splits || !lead_weight16 || !(absorb_decode_us > 0.0f) ||
+        !(gqa_decode_us >= 0.0f) || !(absorb_combine_us >= 0.0f))
         return GQLA_ERR_INVALID_ARG;
     *lead_splits = 0;
     *lead_weight16 = 16;
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GQLA_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return GQLA_ERR_CUDA;
+    const int sms = num_sms;
     // SMs the GQA decode leaves idle, in absorb chunks (2 CTAs per 128 query rows)
     const int row_blocks = (s_q * dims->num_heads + 127) / 128;
-    const int gqa_ctas = gqa_splits * group_splits_for(gqa_splits, dims->num_groups);
+    const int gqa_ctas = gqa_splits * group_splits_rule(gqa_splits, dims->num_groups, sms);
     const int free_sms = sms - gqa_ctas;
     const int n = absorb_splits;
     int e = free_sms > 0 ? free_sms / (2 * row_blocks) : 0;

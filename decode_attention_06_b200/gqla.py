@@ -74,7 +74,7 @@ _SIGS = {
     "gqla_workspace_bytes": [],
     "gqla_num_splits_hint": [_I, _I, _I],
     "gqla_plan_splits": [_P, _I, _I, _I],
-    "gqla_plan_lead": [_DP, _I, _I, _I, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+    "gqla_plan_lead": [_DP, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)],
     "gqla_read_device_error": [_P, ctypes.POINTER(ctypes.c_int), _P],
     "gqla_clear_device_error": [_P, _P],
@@ -319,12 +319,13 @@ def gqla_combine_lead(dims, kv, s_q, num_splits, lead_splits, lead_weight16, d_i
                  lead=(lead_splits, lead_weight16))
 
 
-def gqla_plan_lead(dims, s_q: int, absorb_splits: int, gqa_splits: int, absorb_decode_us: float,
-                   gqa_decode_us: float, absorb_combine_us: float):
-    """(lead_splits, lead_weight16) for the absorb decode beside the GQA path."""
+def gqla_plan_lead(dims, s_q: int, num_sms: int, absorb_splits: int, gqa_splits: int,
+                   absorb_decode_us: float, gqa_decode_us: float, absorb_combine_us: float):
+    """(lead_splits, lead_weight16) for the absorb decode beside the GQA path on a device
+    with num_sms SMs."""
     e, w = ctypes.c_int(0), ctypes.c_int(16)
     _check("gqla_plan_lead", _lib.gqla_plan_lead(
-        ctypes.byref(dims), s_q, absorb_splits, gqa_splits, absorb_decode_us, gqa_decode_us,
+        ctypes.byref(dims), s_q, num_sms, absorb_splits, gqa_splits, absorb_decode_us, gqa_decode_us,
         absorb_combine_us, ctypes.byref(e), ctypes.byref(w)))
     return e.value, w.value
 

@@ -369,15 +369,18 @@ int gqla_plan_splits(const int32_t *seqlens, int batch, int max_splits, int piec
 /* The lead of the absorb path's split plan (gqla_decode_absorb_lead) for a step
  * that runs both paths over one batch on two streams, the absorb decode
  * launched first.  From the times each call takes alone with equal chunks
- * (measured by the caller, µs): lead_splits = the absorb chunks whose CTAs fit
- * on the SMs of the current device that the GQA decode (gqa_splits chunks, and
- * its group split) leaves idle; lead_weight16 such that the lead chunks end
- * the absorb combine's time before the GQA decode does, with the total work
- * unchanged: W = 1 + (x / T_a) / (1 - x lead / (absorb_splits T_a)), x = gqa -
- * combine, T_a = absorb_decode_us, capped at 64.  lead 0 (equal chunks) when
- * the GQA decode fills the device or x <= 0.
- * Returns GQLA_OK, GQLA_ERR_INVALID_ARG or GQLA_ERR_CUDA (no device). */
-int gqla_plan_lead(const gqla_dims *dims, int s_q, int absorb_splits, int gqa_splits,
+ * (measured by the caller, µs): lead_splits = the absorb chunks whose CTAs
+ * (2 per 128 query rows) fit on the SMs of a device with num_sms SMs that the
+ * GQA decode (gqa_splits chunks, times its group split, the rule the GQA
+ * decode applies on such a device) leaves idle, at most absorb_splits - 1;
+ * lead_weight16 such that the lead chunks end the absorb combine's time before
+ * the GQA decode does, with the total work unchanged:
+ * W = 1 + (x / T_a) / (1 - x lead / (absorb_splits T_a)), x = gqa - combine,
+ * T_a = absorb_decode_us, the denominator at least 0.05, W at most 64,
+ * lead_weight16 = round(16 W).  lead 0 and weight 16 (equal chunks) when the
+ * GQA decode fills the device or x <= 0.  Host-only: touches no device.
+ * Returns GQLA_OK or GQLA_ERR_INVALID_ARG. */
+int gqla_plan_lead(const gqla_dims *dims, int s_q, int num_sms, int absorb_splits, int gqa_splits,
                    float absorb_decode_us, float gqa_decode_us, float absorb_combine_us,
                    int *lead_splits, int *lead_weight16);
 

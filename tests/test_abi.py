@@ -2,6 +2,7 @@
 entry point include/gqla.h declares, and rejects bad arguments before any
 launch (no CUDA call is reached by these cases)."""
 import ctypes
+import math
 import os
 import re
 
@@ -238,9 +239,63 @@ def test_lead_calls_reject_bad_arguments(lib):
     F = ctypes.c_float
     e, w = ctypes.c_int(), ctypes.c_int()
     plan = lambda *a: lib.gqla_plan_lead(*a)
-    assert plan(ctypes.byref(d), 2, 0, 128, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
-    assert plan(ctypes.byref(d), 2, 37, 0, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
-    assert plan(ctypes.byref(d), 2, 37, 128, F(0), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
-    assert plan(ctypes.byref(d), 2, 37, 128, F(400), F(-1), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
-    assert plan(ctypes.byref(d), 2, 37, 128, F(400), F(350), F(30), None, ctypes.byref(w)) == -1
-    assert plan(ctypes.byref(d), 3, 37, 128, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -2
+    D = ctypes.byref(d)
+    assert plan(D, 2, 148, 0, 128, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(D, 2, 148, 37, 0, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(D, 2, 0, 37, 128, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(D, 2, 148, 37, 128, F(0), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(D, 2, 148, 37, 128, F(400), F(-1), F(30), ctypes.byref(e), ctypes.byref(w)) == -1
+    assert plan(D, 2, 148, 37, 128, F(400), F(350), F(30), None, ctypes.byref(w)) == -1
+    assert plan(D, 3, 148, 37, 128, F(400), F(350), F(30), ctypes.byref(e), ctypes.byref(w)) == -2
+
+
+def _lead(lib, h, g, s_q, sms, ca, cg, ta, tg, tc):
+    d = _dims(h, g)
+    e, w = ctypes.c_int(-7), ctypes.c_int(-7)
+    F = ctypes.c_float
+    st = lib.gqla_plan_lead(ctypes.byref(d), s_q, sms, ca, cg, F(ta), F(tg), F(tc), ctypes.byref(e), ctypes.byref(w))
+    assert st == 0
+    return e.value, w.value
+
+
+def _lead_by_hand(h, g, s_q, sms, ca, cg, ta, tg, tc):
+    """The plan written out: lead chunks = the absorb chunks (2 CTAs per 128 query rows)
+    that fit on the SMs the GQA decode's CTAs (its splits times the group split it takes
+    when splits x 4 x gs <= SMs) leave idle; W from equal total work and the lead chunks
+    ending the combine's time before the GQA decode."""
+    gs = 1
+    while gs < g and cg * gs * 4 <= sms:
+        gs *= 2
+    free = sms - cg * gs
+    rb = -(-(s_q * h) // 128)
+    e = min(free // (2 * rb) if free > 0 else 0, ca - 1)
+    x = float(F32(tg)) - float(F32(tc))
+    if e <= 0 or x <= 0:
+        return 0, 16
+    ta = float(F32(ta))
+    den = max(1.0 - x * e / (ca * ta), 0.05)
+    wgt = min(1.0 + (x / ta) / den, 64.0)
+    return e, int(math.floor(16 * wgt + 0.5))
+
+
+def F32(v):
+    import numpy as np
+    return np.float32(v)
+
+
+def test_plan_lead_matches_the_formula(lib):
+    """gqla_plan_lead against the plan written out by hand (host-only: no device)."""
+    cases = [
+        # (h, g, s_q, sms, absorb splits, gqa splits, T_a, T_g, T_c) in us
+        (128, 8, 2, 148, 37, 128, 414.0, 359.0, 37.0),   # the 64 x 8192 step: 5 chunks, W16 30
+        (128, 8, 1, 148, 64, 128, 77.6, 93.6, 14.4),
+        (32, 8, 1, 148, 4, 1, 16.8, 16.4, 10.0),          # one GQA split, its groups over 8 CTAs
+        (128, 8, 2, 148, 37, 148, 414.0, 359.0, 37.0),    # the GQA decode fills the device
+        (128, 8, 2, 148, 37, 128, 414.0, 30.0, 37.0),     # x <= 0
+        (128, 4, 1, 148, 64, 128, 78.2, 60.2, 14.4),
+        (128, 8, 2, 132, 33, 100, 400.0, 380.0, 20.0),    # another SM count
+        (128, 8, 2, 148, 3, 100, 50.0, 400.0, 1.0),       # lead capped at splits - 1, W capped at 64
+    ]
+    for c in cases:
+        assert _lead(lib, *c) == _lead_by_hand(*c), c
+    assert _lead(lib, *cases[0]) == (5, 30)

@@ -219,19 +219,14 @@ def test_absorb_lead_split_parity(cid, h, seqlens, s_q, paged, splits, lead):
 
 
 def test_plan_lead_on_device():
-    """gqla_plan_lead at the 64 x 8192 s_q = 2 shape: the absorb chunks whose 2 x 2 CTAs
-    fit on the SMs the GQA decode's 128 CTAs leave idle, each about twice as long."""
+    """gqla_plan_lead with this device's SM count at the 64 x 8192 s_q = 2 shape: the absorb
+    chunks whose 2 x 2 CTAs fit on the SMs the GQA decode's 128 CTAs leave idle."""
     from decode_attention_06_b200 import gqla
     dims = gqla.make_dims(128, 8)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    e, w16 = gqla.gqla_plan_lead(dims, 2, 37, 128, 414.0, 359.0, 37.0)
+    e, w16 = gqla.gqla_plan_lead(dims, 2, sms, 37, 128, 414.0, 359.0, 37.0)
     assert e == min(max((sms - 128) // 4, 0), 36)
-    if e:
-        # W = 1 + (x / T_a) / (1 - x e / (n T_a)), x = 359 - 37
-        x, ta = 359.0 - 37.0, 414.0
-        assert w16 == round(16 * (1 + (x / ta) / (1 - x * e / (37 * ta))))
-    # the GQA decode fills the device: no lead
-    assert gqla.gqla_plan_lead(dims, 2, 37, sms, 414.0, 359.0, 37.0) == (0, 16)
+    assert gqla.gqla_plan_lead(dims, 2, sms, 37, sms, 414.0, 359.0, 37.0) == (0, 16)
 
 
 def test_paths_agree():
