@@ -71,9 +71,21 @@ __global__ void __launch_bounds__(kSgThreads) sparse_gather_kernel(const SgParam
     const int last = L - p.s_q + s;  // this query sees t <= last
     const int32_t *idx = p.idx + (int64_t)v * p.topk;
     const int32_t *prow = p.page_table + (int64_t)b * p.max_pages;
-    // valid entries before this chunk
+    // valid entries before this chunk: eight list entries per thread are loaded first and
+    // their page-table entries next, so a CTA late in a long list waits for two rounds of
+    // loads per 2048 entries instead of two per 256
     int n = 0;
-    for (int j = threadIdx.x; j < j0; j += kSgThreads) n += entry_slot(p, prow, idx[j], last) >= 0;
+    constexpr int kU = 8;
+    for (int jb = 0; jb < j0; jb += kSgThreads * kU) {
+        int t[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int j = jb + u * kSgThreads + threadIdx.x;
+            t[u] = j < j0 ? idx[j] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) n += entry_slot(p, prow, t[u], last) >= 0;
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
     if (lane == 0) s_warp[warp] = n;
