@@ -430,7 +430,8 @@ int gqla_combine_lead(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, i
     if (d_in == kLatent) {
         if (!w_uv) return GQLA_ERR_INVALID_ARG;
     } else if (d_in == kDv) {
-        if (w_uv) return GQLA_ERR_INVALID_ARG;
+        // no GQA decode writes partials on a plan with lead chunks
+        if (w_uv || (lead_splits > 0 && lead_weight16 != 16)) return GQLA_ERR_INVALID_ARG;
     } else {
         return GQLA_ERR_INVALID_ARG;
     }

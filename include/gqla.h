@@ -293,7 +293,9 @@ int gqla_combine(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int nu
                  void *out, float *lse_out, gqla_stream_t stream);
 
 /* gqla_combine for partials written by gqla_decode_absorb_lead: the same
- * lead_splits and lead_weight16 locate each sequence's partial slots. */
+ * lead_splits and lead_weight16 locate each sequence's partial slots.  d_in
+ * 512 only when the lead is not empty (no GQA decode writes such partials):
+ * d_in 128 with lead_splits > 0 and lead_weight16 != 16 is GQLA_ERR_INVALID_ARG. */
 int gqla_combine_lead(const gqla_dims *dims, const gqla_kv_index *kv, int s_q, int num_splits,
                       int lead_splits, int lead_weight16, int d_in, const float *o_part,
                       const float *lse_part, const void *w_uv, void *out, float *lse_out,

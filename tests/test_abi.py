@@ -236,6 +236,9 @@ def test_lead_calls_reject_bad_arguments(lib):
                                            FAKE, FAKE, FAKE, wsb, None) == -1, (lead, w16)
         assert lib.gqla_combine_lead(ctypes.byref(d), ctypes.byref(kv), 1, 4, lead, w16, 512, FAKE, FAKE,
                                      FAKE, FAKE, None, None) == -1, (lead, w16)
+    # GQA partials never come from a plan with lead chunks
+    assert lib.gqla_combine_lead(ctypes.byref(d), ctypes.byref(kv), 1, 4, 1, 32, 128, FAKE, FAKE,
+                                 None, FAKE, None, None) == -1
     F = ctypes.c_float
     e, w = ctypes.c_int(), ctypes.c_int()
     plan = lambda *a: lib.gqla_plan_lead(*a)
